@@ -1,0 +1,181 @@
+/*
+ * kca.h -- C ABI of the B200 (sm_100a) states-form KV-cache attention library
+ *          (libkca.so).
+ *
+ * The operation (Karume v0.12.0 release notes, "Performance", items 1-3;
+ * Karume v0.8.0 release notes, "Features", conversation-window item, and
+ * "Breaking Changes", softmax NaN item):
+ *
+ *   For a query row at absolute position pos of one sequence and query head h,
+ *   with KV head g = h / (n_q_heads / n_kv_heads):
+ *     visible keys  J(pos) = [lo, pos],  lo = window > 0 ? max(0, pos-window+1) : 0
+ *     s_j  = scale * <q[h,:], K[j,g,:]>                         (j in J(pos))
+ *     out[h,:] = sum_j exp(s_j - max s) V[j,g,:] / sum_j exp(s_j - max s)
+ *   A NaN score makes the row NaN; a row with no visible key is exactly 0.
+ *
+ * Prefill (attn_prefill): a chunk of chunk_rows <= 768 query rows at positions
+ * chunk_start .. chunk_start+chunk_rows-1 of one sequence; every row sees the
+ * cached rows before the chunk and the chunk's own rows up to itself
+ * ("chunked prefill", 768-row chunks).  Decode (attn_decode): one query row per
+ * sequence of a batch, at position ctx_len[b]-1.
+ *
+ * Fixed geometry: n_q_heads = 8, n_kv_heads = 1, head_dim = 256.  The
+ * arguments are still passed so that a mismatch is an error, not a silent
+ * misread.
+ *
+ * MEMORY LAYOUT (all row-major, no padding, device memory):
+ *   K cache, V cache : [batch][capacity][n_kv_heads][head_dim], kv_dtype.
+ *                      Row p of sequence b starts at element
+ *                      ((b*capacity + p)*n_kv_heads)*head_dim.
+ *                      attn_prefill works on one sequence: pass the pointers
+ *                      of that sequence's row 0.
+ *   q (prefill)      : [chunk_rows][n_q_heads][head_dim], q_dtype
+ *   q (decode)       : [batch][n_q_heads][head_dim], q_dtype
+ *   out              : [rows or batch][n_q_heads][head_dim], float32
+ *   All of q, k_cache, v_cache, out must be 16-byte aligned; workspace
+ *   256-byte aligned.
+ *
+ * PRECONDITIONS: the caller has written the K/V rows of every position the
+ * call reads (for prefill the chunk's own rows too; for decode the row at
+ * ctx_len-1).  Prefill requires ctx_len == chunk_start + chunk_rows.
+ * Rows outside the union of the call's visible ranges are never read.
+ *
+ * DTYPES: decode takes any q_dtype with any kv_dtype.  Prefill with
+ * q_dtype == kv_dtype in {F16, BF16} and chunk_rows >= 16 runs on the
+ * tcgen05 tensor cores (f32 accumulation); every other prefill combination
+ * runs on the CUDA cores in f32.
+ *
+ * OWNERSHIP: every buffer is allocated and owned by the caller.  The library
+ * allocates no device memory, keeps no per-call state and never synchronises
+ * the stream.  Work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) of the current device.
+ *
+ * WORKSPACE: scratch device memory of at least attn_*_workspace_bytes()
+ * bytes for the same arguments on the same device.  Its first 256 bytes hold
+ * a device status word: zero them once after allocation (attn_workspace_init)
+ * and read them with attn_device_status.  Calls that run concurrently must not
+ * share a workspace or an output buffer.
+ *
+ * ERRORS: every entry point validates all of its arguments on the host before
+ * touching the GPU and returns a negative KCA_ERR_* without launching
+ * anything.  KCA_ERR_CUDA reports a failed CUDA runtime call (launch
+ * configuration, driver entry point); device-side faults are not possible by
+ * design, and the only device-side error (a bounded wait inside the tensor-core
+ * kernel that ran out) is recorded in the workspace status word.
+ */
+#ifndef KCA_H
+#define KCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types */
+#define KCA_F32 0
+#define KCA_F16 1
+#define KCA_BF16 2
+
+/* status codes */
+#define KCA_OK 0
+#define KCA_ERR_NULL (-1)       /* a required pointer is NULL                      */
+#define KCA_ERR_GEOMETRY (-2)   /* heads / head_dim other than 8 / 1 / 256         */
+#define KCA_ERR_DTYPE (-3)      /* unknown dtype code                              */
+#define KCA_ERR_RANGE (-4)      /* rows, positions, capacity, batch or window      */
+#define KCA_ERR_WORKSPACE (-5)  /* workspace too small or misaligned               */
+#define KCA_ERR_ALIGN (-6)      /* q / k / v / out not 16-byte aligned             */
+#define KCA_ERR_CUDA (-7)       /* a CUDA runtime call failed                      */
+#define KCA_ERR_DEVICE (-8)     /* the device recorded an error (attn_device_status) */
+
+/* limits (v0.8.0 release notes: maxChunkLength 768, maxPosition 131072) */
+#define KCA_N_Q_HEADS 8
+#define KCA_N_KV_HEADS 1
+#define KCA_HEAD_DIM 256
+#define KCA_MAX_CHUNK_ROWS 768
+#define KCA_MAX_POSITION 131072
+#define KCA_MAX_BATCH 256
+#define KCA_WORKSPACE_HEADER 256
+
+/*
+ * attn_prefill -- chunked causal prefill of one sequence.
+ *   q_chunk      [chunk_rows][8][256] q_dtype, device
+ *   k_cache/v_cache  the sequence's [capacity][1][256] kv_dtype rows, device
+ *   capacity     rows the cache holds, 1..131072
+ *   chunk_start  position of the chunk's first row, >= 0
+ *   chunk_rows   1..768
+ *   ctx_len      must equal chunk_start + chunk_rows, <= capacity
+ *   window       <= 0: none; otherwise keys [pos-window+1, pos]
+ *   scale        finite score scale (1/sqrt(256) for Gemma 4)
+ *   out          [chunk_rows][8][256] float32, device
+ *   workspace    >= attn_prefill_workspace_bytes(...) bytes, device
+ * Returns KCA_OK or a negative KCA_ERR_*.
+ */
+int attn_prefill(const void *q_chunk, int32_t q_dtype,
+                 const void *k_cache, const void *v_cache, int32_t kv_dtype,
+                 int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity,
+                 int64_t chunk_start, int32_t chunk_rows, int64_t ctx_len, int32_t window,
+                 float scale, float *out, void *workspace, size_t workspace_bytes,
+                 void *stream);
+
+/*
+ * attn_decode -- one query row per sequence (split-context decode + merge).
+ *   q            [batch][8][256] q_dtype, device
+ *   k_cache/v_cache  [batch][capacity][1][256] kv_dtype, device
+ *   batch        1..256
+ *   ctx_len      HOST array [batch], 0..capacity; the query sits at ctx_len[b]-1
+ *                and ctx_len[b] == 0 yields an all-zero output row
+ *   out          [batch][8][256] float32, device
+ */
+int attn_decode(const void *q, int32_t q_dtype,
+                const void *k_cache, const void *v_cache, int32_t kv_dtype,
+                int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity,
+                int32_t batch, const int64_t *ctx_len, int32_t window,
+                float scale, float *out, void *workspace, size_t workspace_bytes,
+                void *stream);
+
+/* Workspace bytes the calls above need on the current device (0 on a bad
+ * argument).  Always >= KCA_WORKSPACE_HEADER. */
+size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
+                                    int32_t chunk_rows, int32_t window);
+size_t attn_decode_workspace_bytes(int32_t batch, const int64_t *ctx_len, int32_t window);
+
+/* Zero the workspace's status header (cudaMemsetAsync on `stream`). */
+int attn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Reads and clears the workspace status word (synchronises `stream`).
+ * Returns KCA_OK when no kernel recorded an error since the last read,
+ * KCA_ERR_DEVICE when one did (*detail, if not NULL, receives the record),
+ * or KCA_ERR_CUDA when the copy itself failed.
+ */
+int attn_device_status(void *workspace, void *stream, uint32_t *detail);
+
+/*
+ * Integer plans, for bit-exact tests; host only, no GPU needed.
+ * Each work item is 4 int64: (unit, key_begin, key_end, slot):
+ *   prefill, tensor-core path: unit = 16-row tile index, [key_begin, key_end)
+ *     the absolute key positions the item covers (64-key tiles clipped to the
+ *     call's visible union), slot = partial slot or -1 when the tile is not split;
+ *   rows path (decode, and prefill on the CUDA cores): unit = query row
+ *     (prefill) or sequence (decode), [key_begin, key_end) within J(pos),
+ *     slot = partial slot or -1.
+ * num_sms is the SM count the plan is made for (the calls use the device's).
+ * *path receives 0 for the rows path, 1 for the tensor-core path.
+ * Returns KCA_OK, or KCA_ERR_RANGE when more than max_items items exist
+ * (*n_items still receives the count).
+ */
+int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
+                      int32_t chunk_rows, int32_t window, int32_t num_sms,
+                      int64_t *items, int32_t max_items, int32_t *n_items, int32_t *path);
+int attn_decode_plan(int32_t batch, const int64_t *ctx_len, int32_t window, int32_t num_sms,
+                     int64_t *items, int32_t max_items, int32_t *n_items);
+
+/* Static description of a status code. */
+const char *attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KCA_H */

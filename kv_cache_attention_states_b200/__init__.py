@@ -1,1 +1,235 @@
-"""B200-native states-form KV-cache attention (package placeholder; binding follows)."""
+"""B200-native states-form KV-cache attention (chunked causal prefill and
+split-context decode, 8 query heads sharing one KV head, head_dim 256).
+
+Thin ctypes binding over libkca.so, whose C ABI is declared in
+include/kca.h.  The functions keep the C names and only marshal arguments:
+torch tensors become device pointers, dtypes become codes, the current torch
+stream becomes the cudaStream_t.  Every step of the attention runs in the
+library's CUDA kernels; there is no fallback, and a missing or unloadable
+library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import synth  # noqa: F401  (seeded inputs; no attention arithmetic)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkca.so")
+
+F32, F16, BF16 = 0, 1, 2
+N_Q_HEADS, N_KV_HEADS, HEAD_DIM = 8, 1, 256
+MAX_CHUNK_ROWS, MAX_POSITION, MAX_BATCH = 768, 131072, 256
+WORKSPACE_HEADER = 256
+STATUS = {0: "KCA_OK", -1: "KCA_ERR_NULL", -2: "KCA_ERR_GEOMETRY", -3: "KCA_ERR_DTYPE",
+          -4: "KCA_ERR_RANGE", -5: "KCA_ERR_WORKSPACE", -6: "KCA_ERR_ALIGN", -7: "KCA_ERR_CUDA",
+          -8: "KCA_ERR_DEVICE"}
+
+_lib = None
+
+
+class KcaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libkca.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m kv_cache_attention_states_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                 ctypes.c_size_t)
+        p64 = ctypes.POINTER(ctypes.c_int64)
+        p32 = ctypes.POINTER(ctypes.c_int32)
+        L.attn_prefill.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i64, i32, i64, i32,
+                                   f32, vp, vp, sz, vp]
+        L.attn_prefill.restype = ctypes.c_int
+        L.attn_decode.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp,
+                                  vp, sz, vp]
+        L.attn_decode.restype = ctypes.c_int
+        L.attn_prefill_workspace_bytes.argtypes = [i32, i32, i64, i32, i32]
+        L.attn_prefill_workspace_bytes.restype = sz
+        L.attn_decode_workspace_bytes.argtypes = [i32, p64, i32]
+        L.attn_decode_workspace_bytes.restype = sz
+        L.attn_workspace_init.argtypes = [vp, sz, vp]
+        L.attn_workspace_init.restype = ctypes.c_int
+        L.attn_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.attn_device_status.restype = ctypes.c_int
+        L.attn_prefill_plan.argtypes = [i32, i32, i64, i32, i32, i32, p64, i32, p32, p32]
+        L.attn_prefill_plan.restype = ctypes.c_int
+        L.attn_decode_plan.argtypes = [i32, p64, i32, i32, p64, i32, p32]
+        L.attn_decode_plan.restype = ctypes.c_int
+        L.attn_status_string.argtypes = [ctypes.c_int]
+        L.attn_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def dtype_code(t) -> int:
+    import torch
+    codes = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def _stream_ptr(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _i64_array(vals):
+    arr = np.ascontiguousarray(np.asarray(vals, dtype=np.int64).reshape(-1))
+    return arr, arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise KcaError(status, what)
+
+
+# ----------------------------------------------------------------- workspace
+
+def attn_prefill_workspace_bytes(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows: int,
+                                 window: int = 0) -> int:
+    n = lib().attn_prefill_workspace_bytes(q_dtype, kv_dtype, chunk_start, chunk_rows, window)
+    if n == 0:
+        raise KcaError(-4, "attn_prefill_workspace_bytes")
+    return int(n)
+
+
+def attn_decode_workspace_bytes(ctx_len, window: int = 0) -> int:
+    arr, ptr = _i64_array(ctx_len)
+    n = lib().attn_decode_workspace_bytes(arr.size, ptr, window)
+    if n == 0:
+        raise KcaError(-4, "attn_decode_workspace_bytes")
+    return int(n)
+
+
+def new_workspace(nbytes: int, device="cuda", stream=None):
+    """A zero-status workspace of at least nbytes (torch uint8, 256-aligned)."""
+    import torch
+    ws = torch.empty(max(int(nbytes), WORKSPACE_HEADER), dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    _check(lib().attn_workspace_init(ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream_ptr(stream)),
+           "attn_workspace_init")
+    return ws
+
+
+def attn_device_status(workspace, stream=None) -> tuple[int, int]:
+    """(status, detail) of the workspace's device status word; clears it."""
+    detail = ctypes.c_uint32(0)
+    st = lib().attn_device_status(ctypes.c_void_p(workspace.data_ptr()), _stream_ptr(stream),
+                                  ctypes.byref(detail))
+    return int(st), int(detail.value)
+
+
+# --------------------------------------------------------------------- calls
+
+def attn_prefill(q_chunk, k_cache, v_cache, chunk_start: int, window: int = 0,
+                 scale: float = 1.0 / 16.0, out=None, workspace=None, stream=None):
+    """Chunked causal prefill of one sequence.
+
+    q_chunk: [rows, 8, 256]; k_cache / v_cache: the sequence's [capacity, 256]
+    (or [capacity, 1, 256]) rows with the chunk's own rows already written;
+    returns out [rows, 8, 256] float32.
+    """
+    import torch
+    rows = q_chunk.shape[0]
+    capacity = k_cache.shape[0]
+    for t in (q_chunk, k_cache, v_cache):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if k_cache.dtype != v_cache.dtype:
+        raise TypeError("k_cache and v_cache must share a dtype")
+    if out is None:
+        out = torch.empty((rows, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q_chunk.device)
+    qd, kd = dtype_code(q_chunk), dtype_code(k_cache)
+    if workspace is None:
+        workspace = new_workspace(attn_prefill_workspace_bytes(qd, kd, chunk_start, rows, window),
+                                  q_chunk.device, stream)
+    st = lib().attn_prefill(ctypes.c_void_p(q_chunk.data_ptr()), qd, ctypes.c_void_p(k_cache.data_ptr()),
+                            ctypes.c_void_p(v_cache.data_ptr()), kd, N_Q_HEADS, N_KV_HEADS, HEAD_DIM,
+                            capacity, chunk_start, rows, chunk_start + rows, window, scale,
+                            ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+                            workspace.numel(), _stream_ptr(stream))
+    _check(st, "attn_prefill")
+    return out
+
+
+def attn_decode(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.0 / 16.0,
+                out=None, workspace=None, stream=None):
+    """One query row per sequence at position ctx_len[b]-1.
+
+    q: [batch, 8, 256]; k_cache / v_cache: [batch, capacity, 256] (or with a
+    KV-head axis of 1); ctx_len: host sequence of ints; returns out
+    [batch, 8, 256] float32.
+    """
+    import torch
+    batch = q.shape[0]
+    capacity = k_cache.shape[1]
+    for t in (q, k_cache, v_cache):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if k_cache.shape[0] != batch:
+        raise ValueError("k_cache batch does not match q")
+    arr, ptr = _i64_array(ctx_len)
+    if arr.size != batch:
+        raise ValueError("ctx_len must have one entry per sequence")
+    if out is None:
+        out = torch.empty((batch, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(attn_decode_workspace_bytes(arr, window), q.device, stream)
+    st = lib().attn_decode(ctypes.c_void_p(q.data_ptr()), dtype_code(q), ctypes.c_void_p(k_cache.data_ptr()),
+                           ctypes.c_void_p(v_cache.data_ptr()), dtype_code(k_cache), N_Q_HEADS,
+                           N_KV_HEADS, HEAD_DIM, capacity, batch, ptr, window, scale,
+                           ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+                           workspace.numel(), _stream_ptr(stream))
+    _check(st, "attn_decode")
+    return out
+
+
+# --------------------------------------------------------------------- plans
+
+def attn_prefill_plan(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows: int,
+                      window: int = 0, num_sms: int = 148):
+    """(path, items[n, 4]) -- see include/kca.h; host only."""
+    n = ctypes.c_int32(0)
+    path = ctypes.c_int32(0)
+    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, num_sms, None,
+                                 0, ctypes.byref(n), ctypes.byref(path))
+    if st not in (0, -4) or (st == -4 and n.value == 0):
+        raise KcaError(st, "attn_prefill_plan")
+    items = np.zeros((max(n.value, 1), 4), dtype=np.int64)
+    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, num_sms,
+                                 items.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n.value,
+                                 ctypes.byref(n), ctypes.byref(path))
+    _check(st, "attn_prefill_plan")
+    return int(path.value), items[:n.value]
+
+
+def attn_decode_plan(ctx_len, window: int = 0, num_sms: int = 148):
+    arr, ptr = _i64_array(ctx_len)
+    n = ctypes.c_int32(0)
+    st = lib().attn_decode_plan(arr.size, ptr, window, num_sms, None, 0, ctypes.byref(n))
+    if st not in (0, -4) or (st == -4 and n.value == 0):
+        raise KcaError(st, "attn_decode_plan")
+    items = np.zeros((max(n.value, 1), 4), dtype=np.int64)
+    st = lib().attn_decode_plan(arr.size, ptr, window, num_sms,
+                                items.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n.value,
+                                ctypes.byref(n))
+    _check(st, "attn_decode_plan")
+    return items[:n.value]

@@ -1,0 +1,376 @@
+// kca_abi.cu -- the extern "C" entry points of libkca.so (declared and
+// documented in include/kca.h): argument validation on the host, planning,
+// workspace carving, tensor-map encoding and kernel launches.  Nothing here
+// allocates device memory or synchronises a stream (attn_device_status aside,
+// which exists to read the device status word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "../../include/kca.h"
+#include "kca_plan.h"
+#include "kca_rows.h"
+#include "kca_tc.h"
+
+namespace {
+
+using kca::kDim;
+using kca::kHeads;
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool dtype_ok(int32_t d) { return d == KCA_F32 || d == KCA_F16 || d == KCA_BF16; }
+size_t elem_bytes(int32_t d) { return d == KCA_F32 ? 4 : 2; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int geometry_status(int32_t hq, int32_t hkv, int32_t d) {
+  return (hq == KCA_N_Q_HEADS && hkv == KCA_N_KV_HEADS && d == KCA_HEAD_DIM) ? KCA_OK
+                                                                             : KCA_ERR_GEOMETRY;
+}
+
+// SM count of the current device (cached per device).
+int current_sms(int* out) {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KCA_ERR_CUDA;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) {
+    *out = cache[dev];
+    return KCA_OK;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return KCA_ERR_CUDA;
+  if (dev >= 0 && dev < 64) cache[dev] = sms;
+  *out = sms;
+  return KCA_OK;
+}
+
+// "tc" / "rows" forces the prefill path (tests use it to run both paths on
+// the same inputs); unset or anything else chooses by the rules in kca.h.
+bool use_tc(int32_t q_dtype, int32_t kv_dtype, int32_t rows) {
+  const bool eligible = q_dtype == kv_dtype && (q_dtype == KCA_F16 || q_dtype == KCA_BF16);
+  const char* env = std::getenv("KCA_PREFILL_PATH");
+  if (env != nullptr && std::strcmp(env, "rows") == 0) return false;
+  if (env != nullptr && std::strcmp(env, "tc") == 0) return eligible;
+  return eligible && rows >= kca::kRowTile;
+}
+
+std::vector<int64_t> prefill_unit_keys(int64_t chunk_start, int32_t rows, int32_t window) {
+  std::vector<int64_t> nk(rows);
+  for (int32_t i = 0; i < rows; ++i) nk[i] = kca::n_visible(chunk_start + i, window);
+  return nk;
+}
+std::vector<int64_t> decode_unit_keys(int32_t batch, const int64_t* ctx_len, int32_t window) {
+  std::vector<int64_t> nk(batch);
+  for (int32_t b = 0; b < batch; ++b) nk[b] = kca::n_visible(ctx_len[b] - 1, window);
+  return nk;
+}
+
+size_t rows_ws_bytes(const kca::RowsPlan& p) {
+  if (p.max_splits <= 1) return KCA_WORKSPACE_HEADER;
+  const size_t slots = (size_t)p.n_units * p.max_splits;
+  return KCA_WORKSPACE_HEADER + align_up(slots * kHeads * 2 * 4) + align_up(slots * kHeads * kDim * 4);
+}
+size_t tc_ws_bytes(const kca::TcPlan& p) {
+  if (p.n_slots == 0) return KCA_WORKSPACE_HEADER;
+  const size_t slots = (size_t)p.n_slots;
+  return KCA_WORKSPACE_HEADER + align_up(slots * 128 * 2 * 4) + align_up(slots * 128 * kDim * 4);
+}
+
+int prefill_args_status(int64_t capacity, int64_t chunk_start, int32_t chunk_rows) {
+  if (capacity < 1 || capacity > KCA_MAX_POSITION) return KCA_ERR_RANGE;
+  if (chunk_rows < 1 || chunk_rows > KCA_MAX_CHUNK_ROWS) return KCA_ERR_RANGE;
+  if (chunk_start < 0 || chunk_start + chunk_rows > capacity) return KCA_ERR_RANGE;
+  return KCA_OK;
+}
+
+int decode_args_status(int64_t capacity, int32_t batch, const int64_t* ctx_len) {
+  if (capacity < 1 || capacity > KCA_MAX_POSITION) return KCA_ERR_RANGE;
+  if (batch < 1 || batch > KCA_MAX_BATCH) return KCA_ERR_RANGE;
+  for (int32_t b = 0; b < batch; ++b)
+    if (ctx_len[b] < 0 || ctx_len[b] > capacity) return KCA_ERR_RANGE;
+  return KCA_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Map over rows [kv_lo, ctx_len) of one cache: inner extent 256 elements,
+// 64 x 64 boxes, 128-byte swizzle, zero fill outside.
+bool encode_kv_map(CUtensorMap* m, const void* cache, int32_t dtype, int64_t kv_lo, int64_t ctx_len) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const char* base = static_cast<const char*>(cache) + kv_lo * kDim * 2;
+  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)(ctx_len - kv_lo)};
+  cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kca::kKeyTile};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType t =
+      dtype == KCA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(m, t, 2, const_cast<char*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+void carve(void* ws, size_t ml_bytes, float** ml, float** acc) {
+  char* p = static_cast<char*>(ws) + KCA_WORKSPACE_HEADER;
+  *ml = reinterpret_cast<float*>(p);
+  *acc = reinterpret_cast<float*>(p + align_up(ml_bytes));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case KCA_OK: return "ok";
+    case KCA_ERR_NULL: return "a required pointer is NULL";
+    case KCA_ERR_GEOMETRY: return "unsupported geometry (needs 8 query heads, 1 KV head, head_dim 256)";
+    case KCA_ERR_DTYPE: return "unknown element type";
+    case KCA_ERR_RANGE: return "row count, position, context length, capacity, batch or scale out of range";
+    case KCA_ERR_WORKSPACE: return "workspace too small or not 256-byte aligned";
+    case KCA_ERR_ALIGN: return "q, k, v or out not 16-byte aligned";
+    case KCA_ERR_CUDA: return "a CUDA runtime call failed";
+    case KCA_ERR_DEVICE: return "a kernel recorded a device-side error (bounded wait ran out)";
+    default: return "unknown status";
+  }
+}
+
+int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, int32_t chunk_rows,
+                      int32_t window, int32_t num_sms, int64_t* items, int32_t max_items,
+                      int32_t* n_items, int32_t* path) {
+  if (n_items == nullptr || path == nullptr || (items == nullptr && max_items > 0)) return KCA_ERR_NULL;
+  if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
+  if (chunk_rows < 1 || chunk_rows > KCA_MAX_CHUNK_ROWS || chunk_start < 0 ||
+      chunk_start + chunk_rows > KCA_MAX_POSITION || num_sms < 1)
+    return KCA_ERR_RANGE;
+  int32_t count = 0;
+  if (use_tc(q_dtype, kv_dtype, chunk_rows)) {
+    *path = 1;
+    const kca::TcPlan p = kca::make_tc_plan(chunk_start, chunk_rows, window, num_sms);
+    for (int32_t i = 0; i < p.n_items; ++i, ++count) {
+      if (count >= max_items) continue;
+      const kca::TcItem it = kca::tc_item(p, i);
+      int64_t kb = p.kv_lo + (int64_t)it.kt_begin * kca::kKeyTile;
+      int64_t ke = p.kv_lo + (int64_t)it.kt_end * kca::kKeyTile;
+      if (ke > p.ctx_len) ke = p.ctx_len;
+      items[4 * count + 0] = it.tile;
+      items[4 * count + 1] = kb;
+      items[4 * count + 2] = ke;
+      items[4 * count + 3] = it.slot;
+    }
+  } else {
+    *path = 0;
+    const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
+    const kca::RowsPlan p = kca::make_rows_plan(chunk_rows, nk.data(), num_sms);
+    for (int32_t u = 0; u < chunk_rows; ++u) {
+      const int64_t pos = chunk_start + u;
+      const int64_t lo = kca::lo_of(pos, window);
+      const int32_t ns = kca::rows_n_splits(nk[u], p.split_len);
+      for (int32_t s = 0; s < ns; ++s, ++count) {
+        if (count >= max_items) continue;
+        int64_t kb = lo + (int64_t)s * p.split_len, ke = kb + p.split_len;
+        if (ke > pos + 1) ke = pos + 1;
+        if (nk[u] == 0) kb = ke = lo;
+        items[4 * count + 0] = u;
+        items[4 * count + 1] = kb;
+        items[4 * count + 2] = ke;
+        items[4 * count + 3] = ns > 1 ? (int64_t)u * p.max_splits + s : -1;
+      }
+    }
+  }
+  *n_items = count;
+  return count <= max_items ? KCA_OK : KCA_ERR_RANGE;
+}
+
+int attn_decode_plan(int32_t batch, const int64_t* ctx_len, int32_t window, int32_t num_sms,
+                     int64_t* items, int32_t max_items, int32_t* n_items) {
+  if (ctx_len == nullptr || n_items == nullptr || (items == nullptr && max_items > 0)) return KCA_ERR_NULL;
+  if (batch < 1 || batch > KCA_MAX_BATCH || num_sms < 1) return KCA_ERR_RANGE;
+  for (int32_t b = 0; b < batch; ++b)
+    if (ctx_len[b] < 0 || ctx_len[b] > KCA_MAX_POSITION) return KCA_ERR_RANGE;
+  const std::vector<int64_t> nk = decode_unit_keys(batch, ctx_len, window);
+  const kca::RowsPlan p = kca::make_rows_plan(batch, nk.data(), num_sms);
+  int32_t count = 0;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int64_t pos = ctx_len[b] - 1;
+    const int64_t lo = kca::lo_of(pos, window);
+    const int32_t ns = kca::rows_n_splits(nk[b], p.split_len);
+    for (int32_t s = 0; s < ns; ++s, ++count) {
+      if (count >= max_items) continue;
+      int64_t kb = lo + (int64_t)s * p.split_len, ke = kb + p.split_len;
+      if (ke > pos + 1) ke = pos + 1;
+      if (nk[b] == 0) kb = ke = lo;
+      items[4 * count + 0] = b;
+      items[4 * count + 1] = kb;
+      items[4 * count + 2] = ke;
+      items[4 * count + 3] = ns > 1 ? (int64_t)b * p.max_splits + s : -1;
+    }
+  }
+  *n_items = count;
+  return count <= max_items ? KCA_OK : KCA_ERR_RANGE;
+}
+
+size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
+                                    int32_t chunk_rows, int32_t window) {
+  if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return 0;
+  if (prefill_args_status(KCA_MAX_POSITION, chunk_start, chunk_rows) != KCA_OK) return 0;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return 0;
+  if (use_tc(q_dtype, kv_dtype, chunk_rows))
+    return tc_ws_bytes(kca::make_tc_plan(chunk_start, chunk_rows, window, sms));
+  const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
+  return rows_ws_bytes(kca::make_rows_plan(chunk_rows, nk.data(), sms));
+}
+
+size_t attn_decode_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_t window) {
+  if (ctx_len == nullptr || decode_args_status(KCA_MAX_POSITION, batch, ctx_len) != KCA_OK) return 0;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return 0;
+  const std::vector<int64_t> nk = decode_unit_keys(batch, ctx_len, window);
+  return rows_ws_bytes(kca::make_rows_plan(batch, nk.data(), sms));
+}
+
+int attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (workspace == nullptr) return KCA_ERR_NULL;
+  if (workspace_bytes < KCA_WORKSPACE_HEADER || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return KCA_ERR_WORKSPACE;
+  return cudaMemsetAsync(workspace, 0, KCA_WORKSPACE_HEADER, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? KCA_OK
+             : KCA_ERR_CUDA;
+}
+
+int attn_device_status(void* workspace, void* stream, uint32_t* detail) {
+  if (workspace == nullptr) return KCA_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word[2] = {0, 0};
+  if (cudaMemcpyAsync(word, workspace, sizeof word, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return KCA_ERR_CUDA;
+  if (word[0] == 0) return KCA_OK;
+  if (detail != nullptr) *detail = word[1];
+  if (cudaMemsetAsync(workspace, 0, sizeof word, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+    return KCA_ERR_CUDA;
+  return KCA_ERR_DEVICE;
+}
+
+int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, const void* v_cache,
+                 int32_t kv_dtype, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                 int64_t capacity, int64_t chunk_start, int32_t chunk_rows, int64_t ctx_len,
+                 int32_t window, float scale, float* out, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  if (!q_chunk || !k_cache || !v_cache || !out || !workspace) return KCA_ERR_NULL;
+  int st = geometry_status(n_q_heads, n_kv_heads, head_dim);
+  if (st != KCA_OK) return st;
+  if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
+  st = prefill_args_status(capacity, chunk_start, chunk_rows);
+  if (st != KCA_OK) return st;
+  if (ctx_len != chunk_start + chunk_rows || !std::isfinite(scale)) return KCA_ERR_RANGE;
+  if (!aligned16(q_chunk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return KCA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  if (use_tc(q_dtype, kv_dtype, chunk_rows)) {
+    kca::TcArgs a{};
+    a.plan = kca::make_tc_plan(chunk_start, chunk_rows, window, sms);
+    if (workspace_bytes < tc_ws_bytes(a.plan)) return KCA_ERR_WORKSPACE;
+    a.q = q_chunk;
+    a.out = out;
+    a.status = workspace;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    carve(workspace, (size_t)a.plan.n_slots * 128 * 2 * 4, &a.part_ml, &a.part_acc);
+    CUtensorMap tmk, tmv;
+    if (!encode_kv_map(&tmk, k_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len) ||
+        !encode_kv_map(&tmv, v_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len))
+      return KCA_ERR_CUDA;
+    return kca::launch_prefill_tc(kv_dtype, tmk, tmv, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+  }
+
+  const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
+  const kca::RowsPlan p = kca::make_rows_plan(chunk_rows, nk.data(), sms);
+  if (workspace_bytes < rows_ws_bytes(p)) return KCA_ERR_WORKSPACE;
+  kca::RowsArgs a{};
+  a.q = q_chunk;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.out = out;
+  a.status = workspace;
+  a.seq_rows = 0;
+  a.chunk_start = chunk_start;
+  a.mode = 1;
+  a.n_units = chunk_rows;
+  a.split_len = p.split_len;
+  a.max_splits = p.max_splits;
+  a.window = window;
+  a.scale = scale;
+  carve(workspace, (size_t)p.n_units * p.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
+  return kca::launch_rows(q_dtype, kv_dtype, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+}
+
+int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache,
+                int32_t kv_dtype, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                int64_t capacity, int32_t batch, const int64_t* ctx_len, int32_t window, float scale,
+                float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !out || !workspace || !ctx_len) return KCA_ERR_NULL;
+  int st = geometry_status(n_q_heads, n_kv_heads, head_dim);
+  if (st != KCA_OK) return st;
+  if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
+  st = decode_args_status(capacity, batch, ctx_len);
+  if (st != KCA_OK) return st;
+  if (!std::isfinite(scale)) return KCA_ERR_RANGE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return KCA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+  const std::vector<int64_t> nk = decode_unit_keys(batch, ctx_len, window);
+  const kca::RowsPlan p = kca::make_rows_plan(batch, nk.data(), sms);
+  if (workspace_bytes < rows_ws_bytes(p)) return KCA_ERR_WORKSPACE;
+  kca::RowsArgs a{};
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.out = out;
+  a.status = workspace;
+  a.seq_rows = capacity;
+  a.chunk_start = 0;
+  a.mode = 0;
+  a.n_units = batch;
+  a.split_len = p.split_len;
+  a.max_splits = p.max_splits;
+  a.window = window;
+  a.scale = scale;
+  for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
+  carve(workspace, (size_t)p.n_units * p.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
+  return kca::launch_rows(q_dtype, kv_dtype, a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KCA_OK
+             : KCA_ERR_CUDA;
+}
+
+}  // extern "C"

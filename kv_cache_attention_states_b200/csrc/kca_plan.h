@@ -1,0 +1,208 @@
+// kca_plan.h -- integer bookkeeping of the attention calls, shared verbatim by
+// the host (validation, workspace sizes, plan queries) and the device (each
+// CTA recomputes its own work item from the same formulas, so no plan ever
+// has to be copied to the GPU).
+//
+// Visible keys of a query at position pos: J(pos) = [lo(pos), pos] with
+// lo(pos) = window > 0 ? max(0, pos - window + 1) : 0 (the sliding window of
+// the local layers; without a window every cached row before the query and
+// the query's own row, as chunked prefill requires -- Karume v0.8.0 release
+// notes, "Features", conversation-window item).
+#pragma once
+#include <cstdint>
+
+#if defined(__CUDACC__)
+#define KCA_HD __host__ __device__ __forceinline__
+#else
+#define KCA_HD inline
+#endif
+
+namespace kca {
+
+constexpr int kHeads = 8;        // query heads per KV head
+constexpr int kDim = 256;        // head_dim
+constexpr int kRowTile = 16;     // query positions per tensor-core row tile (16 x 8 heads = 128 M rows)
+constexpr int kKeyTile = 64;     // keys per tensor-core KV tile
+constexpr int kPartFloats = 2 + kDim;  // per (slot, row): m, l, acc[256]
+
+KCA_HD int64_t lo_of(int64_t pos, int32_t window) {
+  if (window > 0) {
+    const int64_t lo = pos - window + 1;
+    return lo > 0 ? lo : 0;
+  }
+  return 0;
+}
+KCA_HD int64_t n_visible(int64_t pos, int32_t window) {
+  const int64_t lo = lo_of(pos, window);
+  return pos >= lo ? pos - lo + 1 : 0;
+}
+KCA_HD int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------ rows path
+// One unit = one query row (prefill) or one sequence (decode).  Its visible
+// keys are cut into splits of split_len keys; a unit with no visible key has
+// one empty split that writes zeros.
+struct RowsPlan {
+  int32_t n_units;
+  int32_t split_len;
+  int32_t max_splits;
+};
+
+KCA_HD int32_t rows_n_splits(int64_t nkeys, int32_t split_len) {
+  return nkeys <= 0 ? 1 : (int32_t)cdiv(nkeys, split_len);
+}
+
+// Rows path tuning: resident CTAs per SM the plan aims to fill (the rows
+// kernel runs one CTA per SM), the smallest split, and the split quantum
+// (the kernel's keys per shared-memory stage).
+constexpr int kRowsCtasPerSm = 1;
+constexpr int kRowsMinSplit = 64;
+constexpr int kRowsSplitQuantum = 16;
+
+// nkeys[u]: visible keys of unit u.  split_len is the smallest multiple of
+// the quantum (>= kRowsMinSplit) whose split count fits one wave; when even
+// one split per unit does not fit, every unit gets a single split.
+inline RowsPlan make_rows_plan(int32_t n_units, const int64_t* nkeys, int32_t num_sms) {
+  RowsPlan p;
+  p.n_units = n_units;
+  int64_t max_keys = 0;
+  for (int32_t u = 0; u < n_units; ++u) max_keys = nkeys[u] > max_keys ? nkeys[u] : max_keys;
+  const int64_t target = (int64_t)(num_sms > 0 ? num_sms : 1) * kRowsCtasPerSm;
+  auto count = [&](int64_t len) {
+    int64_t c = 0;
+    for (int32_t u = 0; u < n_units; ++u) c += rows_n_splits(nkeys[u], (int32_t)len);
+    return c;
+  };
+  int64_t hi = cdiv(max_keys > kRowsMinSplit ? max_keys : kRowsMinSplit, kRowsSplitQuantum);
+  int64_t lo = cdiv(kRowsMinSplit, kRowsSplitQuantum);
+  if (count(lo * kRowsSplitQuantum) <= target) {
+    hi = lo;
+  } else {
+    // smallest quantum multiple in (lo, hi] whose count fits (count(hi) == n_units)
+    while (lo + 1 < hi) {
+      const int64_t mid = (lo + hi) / 2;
+      if (count(mid * kRowsSplitQuantum) <= target) hi = mid; else lo = mid;
+    }
+  }
+  p.split_len = (int32_t)(hi * kRowsSplitQuantum);
+  p.max_splits = rows_n_splits(max_keys, p.split_len);
+  return p;
+}
+
+// ------------------------------------------------------ tensor-core path
+// A chunk of `rows` query rows at chunk_start is cut into row tiles of 16
+// positions (x 8 heads = 128 M rows).  Keys are addressed relative to
+// kv_lo = lo(chunk_start), the first key any row of the chunk sees, in tiles
+// of 64.  Row tile t covers key tiles [kb(t), ke(t)); it is split into
+// ceil(n/c) items of near-equal length, c chosen as the smallest value that
+// keeps the item count within one wave of CTAs.
+struct TcPlan {
+  int64_t chunk_start;
+  int64_t kv_lo;
+  int64_t ctx_len;      // chunk_start + rows: keys at or beyond it are outside the map
+  int32_t rows;
+  int32_t window;
+  int32_t n_tiles;
+  int32_t per_item;     // c: most key tiles one item covers
+  int32_t n_items;
+  int32_t n_slots;      // items that belong to split tiles (write partials)
+};
+
+constexpr int kTcMinItemTiles = 4;
+
+KCA_HD void tc_tile_keys(const TcPlan& p, int32_t t, int32_t* kb, int32_t* ke) {
+  const int64_t first = p.chunk_start + (int64_t)t * kRowTile;
+  int64_t last = p.chunk_start + (int64_t)(t + 1) * kRowTile - 1;
+  const int64_t end = p.chunk_start + p.rows - 1;
+  if (last > end) last = end;
+  *kb = (int32_t)((lo_of(first, p.window) - p.kv_lo) / kKeyTile);
+  *ke = (int32_t)((last - p.kv_lo) / kKeyTile + 1);
+}
+KCA_HD int32_t tc_tile_items(const TcPlan& p, int32_t t) {
+  int32_t kb, ke;
+  tc_tile_keys(p, t, &kb, &ke);
+  return (int32_t)cdiv(ke - kb, p.per_item);
+}
+
+struct TcItem {
+  int32_t tile;
+  int32_t kt_begin;   // key tiles, relative to kv_lo
+  int32_t kt_end;
+  int32_t slot;       // partial slot, -1 when the tile is not split
+  int32_t split;      // index within the tile
+  int32_t n_split;
+};
+
+// Item `idx` of the plan (items ordered by tile, then by split).
+KCA_HD TcItem tc_item(const TcPlan& p, int32_t idx) {
+  TcItem it{};
+  int32_t base = 0, slot_base = 0;
+  for (int32_t t = 0; t < p.n_tiles; ++t) {
+    int32_t kb, ke;
+    tc_tile_keys(p, t, &kb, &ke);
+    const int32_t n = ke - kb;
+    const int32_t s = (int32_t)cdiv(n, p.per_item);
+    if (idx < base + s) {
+      const int32_t k = idx - base;
+      it.tile = t;
+      it.kt_begin = kb + (int32_t)(((int64_t)k * n) / s);
+      it.kt_end = kb + (int32_t)(((int64_t)(k + 1) * n) / s);
+      it.split = k;
+      it.n_split = s;
+      it.slot = s > 1 ? slot_base + k : -1;
+      return it;
+    }
+    base += s;
+    if (s > 1) slot_base += s;
+  }
+  it.tile = -1;
+  return it;
+}
+
+// First partial slot of tile t (meaningful when the tile is split).
+KCA_HD int32_t tc_tile_first_slot(const TcPlan& p, int32_t tile) {
+  int32_t slot_base = 0;
+  for (int32_t t = 0; t < tile; ++t) {
+    const int32_t s = tc_tile_items(p, t);
+    if (s > 1) slot_base += s;
+  }
+  return slot_base;
+}
+
+inline TcPlan make_tc_plan(int64_t chunk_start, int32_t rows, int32_t window, int32_t num_sms) {
+  TcPlan p{};
+  p.chunk_start = chunk_start;
+  p.rows = rows;
+  p.window = window;
+  p.kv_lo = lo_of(chunk_start, window);
+  p.ctx_len = chunk_start + rows;
+  p.n_tiles = (int32_t)cdiv(rows, kRowTile);
+  int64_t total = 0;
+  int32_t longest = 1;
+  for (int32_t t = 0; t < p.n_tiles; ++t) {
+    int32_t kb, ke;
+    tc_tile_keys(p, t, &kb, &ke);
+    total += ke - kb;
+    if (ke - kb > longest) longest = ke - kb;
+  }
+  const int32_t sms = num_sms > 0 ? num_sms : 1;
+  int32_t c = (int32_t)cdiv(total, sms);
+  if (c < kTcMinItemTiles) c = kTcMinItemTiles;
+  for (;; ++c) {
+    p.per_item = c;
+    int64_t items = 0;
+    for (int32_t t = 0; t < p.n_tiles; ++t) items += tc_tile_items(p, t);
+    if (items <= sms || c >= longest) break;
+  }
+  int32_t items = 0, slots = 0;
+  for (int32_t t = 0; t < p.n_tiles; ++t) {
+    const int32_t s = tc_tile_items(p, t);
+    items += s;
+    if (s > 1) slots += s;
+  }
+  p.n_items = items;
+  p.n_slots = slots;
+  return p;
+}
+
+}  // namespace kca

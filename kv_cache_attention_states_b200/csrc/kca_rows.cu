@@ -1,0 +1,351 @@
+// kca_rows.cu -- split-context attention of single query rows on the CUDA
+// cores: decode (one row per sequence) and the prefill rows that do not take
+// the tensor cores (f32 inputs, mixed dtypes, chunks under 16 rows).
+//
+// Prior art on the pages: Karume's "parallel" reductions for one-row plans
+// (v0.12.0 release notes, "Performance", items 2-3: QK split along the head
+// dimension, PV split along the KV axis; v0.8.0 release notes, "Performance",
+// long-context item).  Here the context of each row is cut into splits, one
+// CTA per split; K/V rows stream through a shared-memory ring filled by bulk
+// copies, each warp reduces its QK dots with warp shuffles and keeps an online
+// softmax, and the splits are merged by log-sum-exp in merge_rows_kernel.
+#include <cuda_runtime.h>
+
+#include "kca_common.cuh"
+#include "kca_plan.h"
+#include "kca_rows.h"
+
+namespace kca {
+
+namespace {
+
+constexpr int kComputeWarps = 8;
+constexpr int kRowsThreads = (kComputeWarps + 1) * 32;  // + one producer warp
+constexpr int kKeysPerStage = 16;
+constexpr int kStages = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 5.545177444479562f;  // 8 * ln 2: rescale once p could pass 256
+
+template <int KT>
+struct RowsSmem {
+  static constexpr int kRowBytes = kDim * ElemBytes<KT>::value;
+  static constexpr int kStageBytes = 2 * kKeysPerStage * kRowBytes;   // K rows then V rows
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kCombineBytes = kComputeWarps * kHeads * (kDim + 2) * 4;
+  static constexpr int kDataBytes = kRingBytes > kCombineBytes ? kRingBytes : kCombineBytes;
+  static constexpr int kBarOffset = kDataBytes;
+  static constexpr int kTotal = kBarOffset + 2 * kStages * 8 + 16;
+};
+
+// Sum eight per-lane values over the warp.  Returns, in every lane, the full
+// sum of value number (lane >> 2) & 7: three halving exchanges (16, 8, 4)
+// followed by two full ones (2, 1) -- 9 shuffles instead of 40.
+__device__ __forceinline__ float reduce8_transposed(const float (&v)[8], int lane) {
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  float r4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float keep = b4 ? v[i + 4] : v[i];
+    const float send = b4 ? v[i] : v[i + 4];
+    r4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+  float r2[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float keep = b3 ? r4[i + 2] : r4[i];
+    const float send = b3 ? r4[i] : r4[i + 2];
+    r2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  float r = (b2 ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? r2[0] : r2[1], 4);
+  r += __shfl_xor_sync(0xffffffffu, r, 2);
+  r += __shfl_xor_sync(0xffffffffu, r, 1);
+  return r;
+}
+
+template <int QT, int KT>
+__global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a) {
+  using S = RowsSmem<KT>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
+  uint64_t* empty = full + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.status);
+
+  const int unit = blockIdx.y;
+  const int split = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int64_t pos = a.mode == 0 ? a.ctx[unit] - 1 : a.chunk_start + unit;
+  const int64_t lo = lo_of(pos, a.window);
+  const int64_t nkeys = n_visible(pos, a.window);
+  const int32_t nsplit = rows_n_splits(nkeys, a.split_len);
+  if (split >= nsplit) return;
+  const int64_t kbeg = lo + (int64_t)split * a.split_len;
+  int64_t kend = kbeg + a.split_len;
+  if (kend > pos + 1) kend = pos + 1;
+  const int64_t base_row = a.mode == 0 ? (int64_t)unit * a.seq_rows : 0;
+  float* out = a.out + (int64_t)unit * kHeads * kDim;
+
+  if (nkeys == 0) {  // fully masked row: exactly zero
+    if (warp < kComputeWarps)
+      for (int i = threadIdx.x; i < kHeads * kDim; i += kComputeWarps * 32) out[i] = 0.f;
+    return;
+  }
+  const int n_stage = (int)cdiv(kend - kbeg, kKeysPerStage);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kComputeWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const char* kg = static_cast<const char*>(a.k);
+  const char* vg = static_cast<const char*>(a.v);
+
+  if (warp == kComputeWarps) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n_stage; ++i) {
+        const int slot = i % kStages;
+        if (i >= kStages &&
+            !mbar_wait(&empty[slot], ((i / kStages) - 1) & 1, abort_flag, status, kSiteRowsEmpty))
+          break;
+        const int64_t k0 = kbeg + (int64_t)i * kKeysPerStage;
+        const int cnt = (int)((kend - k0) < kKeysPerStage ? (kend - k0) : kKeysPerStage);
+        const uint32_t bytes = (uint32_t)cnt * S::kRowBytes;
+        unsigned char* dst = smem + slot * S::kStageBytes;
+        mbar_arrive_expect_tx(&full[slot], 2 * bytes);
+        bulk_g2s(dst, kg + (base_row + k0) * S::kRowBytes, bytes, &full[slot]);
+        bulk_g2s(dst + kKeysPerStage * S::kRowBytes, vg + (base_row + k0) * S::kRowBytes, bytes,
+                 &full[slot]);
+        issued = i + 1;
+      }
+      if (issued < n_stage) {
+        // Aborted: let every copy already issued land before the CTA exits.
+        for (int s = 0; s < kStages && s < issued; ++s) {
+          const int last = ((issued - 1 - s) / kStages) * kStages + s;
+          mbar_wait(&full[s], (last / kStages) & 1, nullptr, status, kSiteRowsFull);
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- compute
+    // Query of this row, all 8 heads, dims [8*lane, 8*lane+8), in f32.
+    float2 q2[kHeads][4];
+    {
+      const char* qrow = static_cast<const char*>(a.q) +
+                         (int64_t)unit * kHeads * kDim * ElemBytes<QT>::value;
+#pragma unroll
+      for (int h = 0; h < kHeads; ++h) {
+        float x[8];
+        load8<QT>(qrow + ((int64_t)h * kDim + 8 * lane) * ElemBytes<QT>::value, x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q2[h][i] = make_float2(x[2 * i], x[2 * i + 1]);
+      }
+    }
+    float2 acc[kHeads][4];
+#pragma unroll
+    for (int h = 0; h < kHeads; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[h][i] = make_float2(0.f, 0.f);
+    float m_ref = -INFINITY;  // reference max of head (lane >> 2) & 7
+    float l_sum = 0.f;
+    const float scale = a.scale;
+    bool ok = true;
+
+    for (int i = 0; i < n_stage && ok; ++i) {
+      const int slot = i % kStages;
+      if (!mbar_wait(&full[slot], (i / kStages) & 1, abort_flag, status, kSiteRowsFull)) {
+        ok = false;
+        break;
+      }
+      const int64_t k0 = kbeg + (int64_t)i * kKeysPerStage;
+      const int cnt = (int)((kend - k0) < kKeysPerStage ? (kend - k0) : kKeysPerStage);
+      const unsigned char* st = smem + slot * S::kStageBytes;
+      const int nk = (warp < cnt ? 1 : 0) + (warp + kComputeWarps < cnt ? 1 : 0);
+      if (nk > 0) {
+        float s_own[2];
+        float vx[2][8];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (c < nk) {
+            const int r = warp + c * kComputeWarps;
+            float kx[8];
+            load8<KT>(st + r * S::kRowBytes + 8 * lane * ElemBytes<KT>::value, kx);
+            load8<KT>(st + (kKeysPerStage + r) * S::kRowBytes + 8 * lane * ElemBytes<KT>::value,
+                      vx[c]);
+            float part[8];
+#pragma unroll
+            for (int h = 0; h < kHeads; ++h) {
+              float2 d = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int t = 0; t < 4; ++t) d = ffma2(q2[h][t], make_float2(kx[2 * t], kx[2 * t + 1]), d);
+              part[h] = d.x + d.y;
+            }
+            s_own[c] = reduce8_transposed(part, lane) * scale;
+          } else {
+            s_own[c] = -INFINITY;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) vx[c][t] = 0.f;
+          }
+        }
+        // Lazy rescale: move the reference max only when a score exceeds it
+        // by more than the threshold; exp(s - m_ref) then stays <= 256.
+        const float m_cand = fmaxf(s_own[0], s_own[1]);
+        const bool need = m_cand > m_ref + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? exp2f((m_ref - m_cand) * kLog2e) : 1.f;
+          if (need) m_ref = m_cand;
+          l_sum *= alpha;
+#pragma unroll
+          for (int h = 0; h < kHeads; ++h) {
+            const float ah = __shfl_sync(0xffffffffu, alpha, 4 * h);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) acc[h][t] = __fmul2_rn(acc[h][t], make_float2(ah, ah));
+          }
+        }
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        float p_own[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) p_own[c] = exp2f((s_own[c] - m_use) * kLog2e);
+        l_sum += p_own[0] + p_own[1];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (c < nk) {
+#pragma unroll
+            for (int h = 0; h < kHeads; ++h) {
+              const float ph = __shfl_sync(0xffffffffu, p_own[c], 4 * h);
+#pragma unroll
+              for (int t = 0; t < 4; ++t)
+                acc[h][t] = ffma2(make_float2(vx[c][2 * t], vx[c][2 * t + 1]), make_float2(ph, ph),
+                                  acc[h][t]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+
+    // All compute warps are done with the ring; reuse it to combine warps.
+    asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory");
+    if (!*abort_flag) {
+      float* cm = reinterpret_cast<float*>(smem);                  // [warp][head]
+      float* cl = cm + kComputeWarps * kHeads;                      // [warp][head]
+      float* cacc = cl + kComputeWarps * kHeads;                    // [warp][head][256]
+      if ((lane & 3) == 0) {
+        cm[warp * kHeads + (lane >> 2)] = m_ref;
+        cl[warp * kHeads + (lane >> 2)] = l_sum;
+      }
+#pragma unroll
+      for (int h = 0; h < kHeads; ++h) {
+        float4* dst = reinterpret_cast<float4*>(cacc + ((warp * kHeads + h) * kDim + 8 * lane));
+        dst[0] = make_float4(acc[h][0].x, acc[h][0].y, acc[h][1].x, acc[h][1].y);
+        dst[1] = make_float4(acc[h][2].x, acc[h][2].y, acc[h][3].x, acc[h][3].y);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory");
+      // thread (h = warp, lane) combines head h, dims [8*lane, 8*lane+8)
+      const int h = warp;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kComputeWarps; ++w) M = max_nan(M, cm[w * kHeads + h]);
+      const float M_use = M == -INFINITY ? 0.f : M;
+      float L = 0.f;
+      float A[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) A[t] = 0.f;
+#pragma unroll
+      for (int w = 0; w < kComputeWarps; ++w) {
+        const float f = exp2f((cm[w * kHeads + h] - M_use) * kLog2e);
+        L += f * cl[w * kHeads + h];
+        const float4* src = reinterpret_cast<const float4*>(cacc + ((w * kHeads + h) * kDim + 8 * lane));
+        const float4 x0 = src[0], x1 = src[1];
+        A[0] += f * x0.x; A[1] += f * x0.y; A[2] += f * x0.z; A[3] += f * x0.w;
+        A[4] += f * x1.x; A[5] += f * x1.y; A[6] += f * x1.z; A[7] += f * x1.w;
+      }
+      if (nsplit == 1) {
+        const float inv = 1.f / L;
+        float4* o = reinterpret_cast<float4*>(out + h * kDim + 8 * lane);
+        o[0] = make_float4(A[0] * inv, A[1] * inv, A[2] * inv, A[3] * inv);
+        o[1] = make_float4(A[4] * inv, A[5] * inv, A[6] * inv, A[7] * inv);
+      } else {
+        const int64_t slot = (int64_t)unit * a.max_splits + split;
+        if (lane == 0) {
+          a.part_ml[(slot * kHeads + h) * 2 + 0] = M;
+          a.part_ml[(slot * kHeads + h) * 2 + 1] = L;
+        }
+        float4* o = reinterpret_cast<float4*>(a.part_acc + (slot * kHeads + h) * kDim + 8 * lane);
+        o[0] = make_float4(A[0], A[1], A[2], A[3]);
+        o[1] = make_float4(A[4], A[5], A[6], A[7]);
+      }
+    }
+  }
+}
+
+// Log-sum-exp merge of the splits of each unit: one CTA per unit, thread
+// (head = warp, lane) owns dims [8*lane, 8*lane+8).
+__global__ void __launch_bounds__(256) merge_rows_kernel(const RowsArgs a) {
+  const int unit = blockIdx.x;
+  const int64_t pos = a.mode == 0 ? a.ctx[unit] - 1 : a.chunk_start + unit;
+  const int32_t nsplit = rows_n_splits(n_visible(pos, a.window), a.split_len);
+  if (nsplit <= 1) return;
+  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t slot0 = (int64_t)unit * a.max_splits;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = max_nan(M, a.part_ml[((slot0 + s) * kHeads + h) * 2]);
+  const float M_use = M == -INFINITY ? 0.f : M;
+  float L = 0.f, A[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < nsplit; ++s) {
+    const int64_t row = (slot0 + s) * kHeads + h;
+    const float f = exp2f((a.part_ml[row * 2] - M_use) * kLog2e);
+    L += f * a.part_ml[row * 2 + 1];
+    const float4* src = reinterpret_cast<const float4*>(a.part_acc + row * kDim + 8 * lane);
+    const float4 x0 = src[0], x1 = src[1];
+    A[0] += f * x0.x; A[1] += f * x0.y; A[2] += f * x0.z; A[3] += f * x0.w;
+    A[4] += f * x1.x; A[5] += f * x1.y; A[6] += f * x1.z; A[7] += f * x1.w;
+  }
+  const float inv = 1.f / L;
+  float4* o = reinterpret_cast<float4*>(a.out + ((int64_t)unit * kHeads + h) * kDim + 8 * lane);
+  o[0] = make_float4(A[0] * inv, A[1] * inv, A[2] * inv, A[3] * inv);
+  o[1] = make_float4(A[4] * inv, A[5] * inv, A[6] * inv, A[7] * inv);
+}
+
+template <int QT, int KT>
+cudaError_t launch_rows_t(const RowsArgs& a, cudaStream_t stream) {
+  using S = RowsSmem<KT>;
+  auto kern = rows_kernel<QT, KT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.max_splits, a.n_units);
+  kern<<<grid, kRowsThreads, S::kTotal, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.max_splits <= 1) return e;
+  merge_rows_kernel<<<a.n_units, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_rows(int q_dtype, int kv_dtype, const RowsArgs& a, cudaStream_t stream) {
+#define KCA_ROWS_CASE(QD, KD) \
+  if (q_dtype == QD && kv_dtype == KD) return launch_rows_t<QD, KD>(a, stream);
+  KCA_ROWS_CASE(KCA_F32, KCA_F32)
+  KCA_ROWS_CASE(KCA_F32, KCA_F16)
+  KCA_ROWS_CASE(KCA_F32, KCA_BF16)
+  KCA_ROWS_CASE(KCA_F16, KCA_F32)
+  KCA_ROWS_CASE(KCA_F16, KCA_F16)
+  KCA_ROWS_CASE(KCA_F16, KCA_BF16)
+  KCA_ROWS_CASE(KCA_BF16, KCA_F32)
+  KCA_ROWS_CASE(KCA_BF16, KCA_F16)
+  KCA_ROWS_CASE(KCA_BF16, KCA_BF16)
+#undef KCA_ROWS_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kca

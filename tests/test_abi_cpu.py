@@ -1,0 +1,177 @@
+"""Boundary tests that need no GPU: the library loads, exports every symbol
+include/kca.h declares, rejects bad arguments on the host before any CUDA
+call, and its integer plans cover exactly the visible keys of every row
+(J(pos) compared bit-exact with the oracle's definition)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import kv_cache_attention_states_b200 as kca
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kca.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert "attn_prefill" in names and "attn_decode" in names
+    lib = kca.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_header_constants_match_binding():
+    text = open(HEADER).read()
+    for name, val in [("KCA_MAX_CHUNK_ROWS", 768), ("KCA_MAX_POSITION", 131072),
+                      ("KCA_HEAD_DIM", 256), ("KCA_N_Q_HEADS", 8), ("KCA_N_KV_HEADS", 1),
+                      ("KCA_WORKSPACE_HEADER", 256), ("KCA_MAX_BATCH", 256)]:
+        assert re.search(rf"#define {name} {val}\b", text), name
+
+
+def test_status_strings():
+    for code in range(0, -9, -1):
+        assert kca.status_string(code)
+    assert kca.status_string(-99) == "unknown status"
+
+
+P = 0x10000  # a 16-byte aligned fake device address; validation fails before any use
+
+
+def _prefill(**kw):
+    a = dict(q=P, qd=kca.BF16, k=P, v=P, kd=kca.BF16, hq=8, hkv=1, d=256, cap=4096, cs=0, rows=768,
+             ctx=768, window=0, scale=0.0625, out=P, ws=P * 2, wsb=1 << 30, stream=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return kca.lib().attn_prefill(vp(a["q"]), a["qd"], vp(a["k"]), vp(a["v"]), a["kd"], a["hq"],
+                                  a["hkv"], a["d"], a["cap"], a["cs"], a["rows"], a["ctx"],
+                                  a["window"], a["scale"], vp(a["out"]), vp(a["ws"]), a["wsb"],
+                                  a["stream"])
+
+
+def _decode(ctx=(100, 200), **kw):
+    a = dict(q=P, qd=kca.F32, k=P, v=P, kd=kca.F16, hq=8, hkv=1, d=256, cap=4096, window=0,
+             scale=0.0625, out=P, ws=P * 2, wsb=1 << 30, batch=None)
+    a.update(kw)
+    arr = np.asarray(ctx, dtype=np.int64)
+    batch = len(arr) if a["batch"] is None else a["batch"]
+    vp = ctypes.c_void_p
+    return kca.lib().attn_decode(vp(a["q"]), a["qd"], vp(a["k"]), vp(a["v"]), a["kd"], a["hq"],
+                                 a["hkv"], a["d"], a["cap"], batch,
+                                 arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), a["window"],
+                                 a["scale"], vp(a["out"]), vp(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(k=0), -1), (dict(v=0), -1), (dict(out=0), -1), (dict(ws=0), -1),
+    (dict(hq=16), -2), (dict(hkv=2), -2), (dict(d=128), -2),
+    (dict(qd=7), -3), (dict(kd=-1), -3),
+    (dict(rows=0, ctx=0), -4), (dict(rows=769, ctx=769), -4), (dict(cs=-1, ctx=767), -4),
+    (dict(cap=0), -4), (dict(cap=131073), -4), (dict(cs=4000, ctx=4768), -4),
+    (dict(ctx=767), -4), (dict(scale=float("nan")), -4), (dict(scale=float("inf")), -4),
+    (dict(q=P + 8), -6), (dict(k=P + 4), -6), (dict(v=P + 2), -6), (dict(out=P + 8), -6),
+    (dict(ws=P * 2 + 16), -5),
+])
+def test_prefill_rejects_bad_arguments_on_the_host(kw, code):
+    assert _prefill(**kw) == code
+
+
+@pytest.mark.parametrize("ctx,kw,code", [
+    ((1, 2), dict(q=0), -1), ((1, 2), dict(hq=4), -2), ((1, 2), dict(kd=3), -3),
+    ((1, 2), dict(batch=0), -4), ((1,) * 257, dict(), -4), ((1, 4097), dict(), -4),
+    ((-1, 2), dict(), -4), ((1, 2), dict(cap=131073), -4), ((1, 2), dict(scale=float("nan")), -4),
+    ((1, 2), dict(out=P + 4), -6), ((1, 2), dict(ws=P * 2 + 128), -5),
+])
+def test_decode_rejects_bad_arguments_on_the_host(ctx, kw, code):
+    assert _decode(ctx, **kw) == code
+
+
+def _check_rows_plan(items, units, pos_of, window):
+    """Every unit's items tile its visible range exactly, in order, slots unique."""
+    slots = [int(s) for s in items[:, 3] if s >= 0]
+    assert len(slots) == len(set(slots))
+    for u in range(units):
+        its = items[items[:, 0] == u]
+        assert len(its) >= 1
+        lo, hi = oracle.visible_range(pos_of(u), window)
+        if hi < lo:
+            assert len(its) == 1 and its[0, 1] == its[0, 2]
+            continue
+        assert its[0, 1] == lo and its[-1, 2] == hi + 1
+        assert (its[1:, 1] == its[:-1, 2]).all()
+        assert (its[:, 2] > its[:, 1]).all()
+        if len(its) == 1:
+            assert its[0, 3] == -1
+        else:
+            assert (its[:, 3] >= 0).all()
+
+
+@pytest.mark.parametrize("cs,rows,window", [(0, 48, 0), (256, 48, 0), (1000, 15, 0), (5, 9, 3),
+                                            (4090, 7, 512), (130000, 1, 0), (0, 1, 1)])
+def test_prefill_rows_plan_covers_visible_keys(cs, rows, window):
+    path, items = kca.attn_prefill_plan(kca.F32, kca.F32, cs, rows, window)
+    assert path == 0
+    _check_rows_plan(items, rows, lambda u: cs + u, window)
+
+
+@pytest.mark.parametrize("ctx,window", [([305], 0), ([16384], 0), ([0, 1, 2], 0), ([4097], 512),
+                                        ([131072] * 8, 0), ([1024, 99999, 5, 131072], 300)])
+def test_decode_plan_covers_visible_keys(ctx, window):
+    for sms in (1, 7, 148):
+        items = kca.attn_decode_plan(ctx, window, num_sms=sms)
+        _check_rows_plan(items, len(ctx), lambda u: ctx[u] - 1, window)
+
+
+def test_decode_plan_fills_one_wave():
+    items = kca.attn_decode_plan([16384], 0, num_sms=148)
+    assert 130 <= len(items) <= 148
+    rng = np.random.default_rng(0)
+    ctx = rng.integers(1024, 131041, size=8)
+    items = kca.attn_decode_plan(ctx, 0, num_sms=148)
+    assert len(items) <= 148
+
+
+@pytest.mark.parametrize("cs,rows,window", [(0, 768, 0), (15360, 768, 0), (16128, 256, 0),
+                                            (256, 48, 0), (3840, 256, 512), (130304, 768, 0),
+                                            (1000, 17, 0), (7, 16, 5), (100, 200, 64),
+                                            (2000, 768, 1)])
+def test_prefill_tc_plan_covers_every_visible_key(cs, rows, window):
+    path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, rows, window)
+    assert path == 1
+    assert len(items) <= 148
+    kv_lo = oracle.visible_range(cs, window)[0]
+    ctx = cs + rows
+    n_tiles = (rows + 15) // 16
+    slots = [int(s) for s in items[:, 3] if s >= 0]
+    assert len(slots) == len(set(slots))
+    for t in range(n_tiles):
+        its = items[items[:, 0] == t]
+        assert len(its) >= 1
+        # items of a tile are contiguous, 64-aligned relative to kv_lo, within [kv_lo, ctx)
+        assert (its[1:, 1] == its[:-1, 2]).all()
+        assert ((its[:, 1] - kv_lo) % 64 == 0).all()
+        assert its[0, 1] >= kv_lo and its[-1, 2] <= ctx
+        covered = (int(its[0, 1]), int(its[-1, 2]))
+        for r in range(16 * t, min(16 * t + 16, rows)):
+            lo, hi = oracle.visible_range(cs + r, window)
+            assert covered[0] <= lo and hi < covered[1]
+        # the first item starts in the key tile of the tile's first row's lo
+        lo0 = oracle.visible_range(cs + 16 * t, window)[0]
+        assert covered[0] == kv_lo + (lo0 - kv_lo) // 64 * 64
+        assert (len(its) == 1) == (its[0, 3] == -1)
+
+
+def test_small_chunks_and_f32_take_the_rows_path():
+    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 100, 15)[0] == 0
+    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 100, 16)[0] == 1
+    assert kca.attn_prefill_plan(kca.F32, kca.F32, 100, 768)[0] == 0
+    assert kca.attn_prefill_plan(kca.F16, kca.BF16, 100, 768)[0] == 0

@@ -1,0 +1,197 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the f64 oracle
+on the same seeded inputs (from synth).  Tolerances are the stated bars:
+max |error| <= 2e-6 with f32 inputs, <= 4e-3 with f16/bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_attention_states_b200 as kca
+from kv_cache_attention_states_b200 import synth
+from tests.helpers import dev, max_err, oracle_decode, oracle_prefill, oracle_threads, tol
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup(cuda_ok):
+    oracle_threads()
+    kca.lib()
+
+
+def _cache(seed, capacity, rows, dtype, std=1.0, batch=None):
+    shape = (capacity, 256) if batch is None else (batch, capacity, 256)
+    k = np.zeros(shape, dtype=np.float32)
+    v = np.zeros(shape, dtype=np.float32)
+    if batch is None:
+        k[:rows] = synth.normal(seed, "k", (rows, 256), std)
+        v[:rows] = synth.normal(seed, "v", (rows, 256), std)
+    else:
+        for b in range(batch):
+            r = rows[b]
+            k[b, :r] = synth.normal(seed, f"k{b}", (r, 256), std)
+            v[b, :r] = synth.normal(seed, f"v{b}", (r, 256), std)
+    return synth.to_storage(k, dtype), synth.to_storage(v, dtype)
+
+
+def _check_status(ws):
+    st, detail = kca.attn_device_status(ws)
+    assert st == 0, f"device status {st} detail {detail:#x}"
+
+
+# ------------------------------------------------------------ tiny f32 config
+
+def test_tiny_f32_prefill_and_decode():
+    wl = synth.tiny_f32()
+    seed = 0
+    k, v = _cache(seed, wl.capacity, wl.capacity, "f32")
+    kd, vd = dev(k, "f32"), dev(v, "f32")
+    (cs, rows), = wl.prefill
+    q = synth.draw(seed, "q_prefill", (rows, 8, 256), "f32")
+    out = kca.attn_prefill(dev(q, "f32"), kd, vd, cs)
+    want = oracle_prefill(q, k, v, cs, np.arange(rows), 0, "f32", "f32")
+    assert max_err(out.cpu().numpy(), want) <= 2e-6
+    qdec = synth.draw(seed, "q_decode", (len(wl.decode_ctx), 8, 256), "f32")
+    for t, (ctx,) in enumerate(wl.decode_ctx):
+        o = kca.attn_decode(dev(qdec[t:t + 1], "f32"), kd[None], vd[None], [ctx])
+        w = oracle_decode(qdec[t:t + 1], k[None], v[None], [ctx], 0, "f32", "f32", wl.capacity)
+        assert max_err(o.cpu().numpy(), w) <= 2e-6, t
+
+
+# --------------------------------------------------------------- decode f16
+
+@pytest.mark.parametrize("length", [256, 4096, 16384])
+def test_decode_f16_lengths(length):
+    wl = synth.decode_f16(length)
+    k, v = _cache(1, wl.capacity, wl.capacity, "f16")
+    kd, vd = dev(k, "f16")[None], dev(v, "f16")[None]
+    q = synth.draw(1, "q", (len(wl.decode_ctx), 8, 256), "f32")
+    ws = kca.new_workspace(kca.attn_decode_workspace_bytes([wl.capacity]))
+    for t in (0, 1, 31, 63):
+        ctx = wl.decode_ctx[t]
+        o = kca.attn_decode(dev(q[t:t + 1], "f32"), kd, vd, ctx, workspace=ws)
+        w = oracle_decode(q[t:t + 1], k[None], v[None], ctx, 0, "f32", "f16", wl.capacity)
+        assert max_err(o.cpu().numpy(), w) <= 4e-3, (length, t)
+    _check_status(ws)
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("f32", "f32"), ("bf16", "bf16"), ("f16", "f16"),
+                                              ("f32", "bf16"), ("bf16", "f16"), ("f16", "f32")])
+def test_decode_dtype_combinations(q_dtype, kv_dtype):
+    cap = 3000
+    ctx = [1, 17, 2999, 1500]
+    k, v = _cache(2, cap, [cap] * 4, kv_dtype, batch=4)
+    q = synth.draw(2, "q", (4, 8, 256), q_dtype)
+    o = kca.attn_decode(dev(q, q_dtype), dev(k, kv_dtype), dev(v, kv_dtype), ctx)
+    w = oracle_decode(q, k, v, ctx, 0, q_dtype, kv_dtype, cap)
+    assert max_err(o.cpu().numpy(), w) <= tol(q_dtype, kv_dtype)
+
+
+# -------------------------------------------------------- tensor-core prefill
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("cs,rows,window", [(0, 768, 0), (1000, 200, 0), (3000, 17, 0),
+                                            (77, 16, 0), (2048, 255, 100), (500, 300, 1),
+                                            (4000, 96, 5000)])
+def test_prefill_tc_matches_oracle(dtype, cs, rows, window):
+    cap = cs + rows + 5
+    std = 0.5
+    k, v = _cache(3, cap, cs + rows, dtype, std)
+    q = synth.draw(3, "q", (rows, 8, 256), dtype, std)
+    code = kca.BF16 if dtype == "bf16" else kca.F16
+    path, _ = kca.attn_prefill_plan(code, code, cs, rows, window)
+    assert path == 1
+    ws = kca.new_workspace(kca.attn_prefill_workspace_bytes(code, code, cs, rows, window))
+    out = kca.attn_prefill(dev(q, dtype), dev(k, dtype), dev(v, dtype), cs, window, workspace=ws)
+    want = oracle_prefill(q, k, v, cs, np.arange(rows), window, dtype, dtype)
+    err = max_err(out.cpu().numpy(), want)
+    assert err <= 4e-3, err
+    _check_status(ws)
+
+
+@pytest.mark.parametrize("rows", [1, 2, 15])
+def test_prefill_short_chunks_take_rows_path(rows):
+    cs = 300
+    k, v = _cache(4, cs + rows, cs + rows, "bf16")
+    q = synth.draw(4, "q", (rows, 8, 256), "bf16")
+    out = kca.attn_prefill(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), cs)
+    want = oracle_prefill(q, k, v, cs, np.arange(rows), 0, "bf16", "bf16")
+    assert max_err(out.cpu().numpy(), want) <= 4e-3
+
+
+def test_rows_and_tc_paths_agree(monkeypatch):
+    cs, rows = 640, 128
+    k, v = _cache(5, cs + rows, cs + rows, "bf16")
+    q = synth.draw(5, "q", (rows, 8, 256), "bf16")
+    args = (dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), cs)
+    tc = kca.attn_prefill(*args).cpu().numpy()
+    monkeypatch.setenv("KCA_PREFILL_PATH", "rows")
+    rw = kca.attn_prefill(*args).cpu().numpy()
+    want = oracle_prefill(q, k, v, cs, np.arange(rows), 0, "bf16", "bf16")
+    assert max_err(tc, want) <= 4e-3 and max_err(rw, want) <= 4e-3
+
+
+# ------------------------------------------------------- full-size workloads
+
+def test_prefill_16k_bf16_chunked_sampled_rows():
+    wl = synth.prefill_bf16_16k()
+    k, v = _cache(0, wl.capacity, wl.capacity, "bf16", wl.std)
+    q = synth.draw(0, "q", (wl.capacity, 8, 256), "bf16", wl.std)
+    kd, vd, qd = dev(k, "bf16"), dev(v, "bf16"), dev(q, "bf16")
+    out = torch.empty((wl.capacity, 8, 256), dtype=torch.float32, device="cuda")
+    ws = kca.new_workspace(max(kca.attn_prefill_workspace_bytes(2, 2, cs, r) for cs, r in wl.prefill))
+    for cs, r in wl.prefill:
+        kca.attn_prefill(qd[cs:cs + r], kd, vd, cs, out=out[cs:cs + r], workspace=ws)
+    torch.cuda.synchronize()
+    _check_status(ws)
+    rng = np.random.default_rng(0)
+    sample = np.unique(np.concatenate([
+        np.arange(0, 24), np.arange(768 * 10, 768 * 10 + 20), np.arange(768 * 20 - 3, 768 * 20 + 17),
+        np.arange(16384 - 20, 16384), rng.integers(0, 16384, 48)]))
+    want = oracle_prefill(q, k, v, 0, sample, 0, "bf16", "bf16")
+    assert max_err(out.cpu().numpy()[sample], want) <= 4e-3
+
+
+def test_window_bf16_prefill_and_decode():
+    wl = synth.window_bf16()
+    k, v = _cache(0, wl.capacity, wl.capacity, "bf16")
+    q = synth.draw(0, "q", (4096, 8, 256), "bf16")
+    kd, vd = dev(k, "bf16"), dev(v, "bf16")
+    qd = dev(q, "bf16")
+    out = torch.empty((4096, 8, 256), dtype=torch.float32, device="cuda")
+    for cs, r in wl.prefill:
+        kca.attn_prefill(qd[cs:cs + r], kd, vd, cs, wl.window, out=out[cs:cs + r])
+    rows = np.concatenate([np.arange(0, 600), np.arange(3000, 3300), np.arange(3840, 4096)])
+    want = oracle_prefill(q, k, v, 0, rows, wl.window, "bf16", "bf16")
+    assert max_err(out.cpu().numpy()[rows], want) <= 4e-3
+    qdec = synth.draw(0, "q_decode", (len(wl.decode_ctx), 8, 256), "bf16")
+    for t in (0, 1, 40, 63):
+        ctx = wl.decode_ctx[t]
+        o = kca.attn_decode(dev(qdec[t:t + 1], "bf16"), kd[None], vd[None], ctx, wl.window)
+        w = oracle_decode(qdec[t:t + 1], k[None], v[None], ctx, wl.window, "bf16", "bf16", wl.capacity)
+        assert max_err(o.cpu().numpy(), w) <= 4e-3, t
+
+
+def test_ragged_long_context_decode():
+    wl = synth.ragged_f16(0)
+    ctx0 = np.array(wl.decode_ctx[0])
+    need = ctx0 + len(wl.decode_ctx)
+    k, v = _cache(0, wl.capacity, need, "f16", batch=wl.batch)
+    kd, vd = dev(k, "f16"), dev(v, "f16")
+    q = synth.draw(0, "q", (len(wl.decode_ctx), wl.batch, 8, 256), "f32")
+    ws = kca.new_workspace(max(kca.attn_decode_workspace_bytes(c) for c in wl.decode_ctx))
+    for t in (0, 31):
+        o = kca.attn_decode(dev(q[t], "f32"), kd, vd, wl.decode_ctx[t], workspace=ws)
+        w = oracle_decode(q[t], k, v, wl.decode_ctx[t], 0, "f32", "f16", wl.capacity)
+        assert max_err(o.cpu().numpy(), w) <= 4e-3, t
+    _check_status(ws)
+
+
+def test_long_chunk_at_capacity_end_sampled_rows():
+    wl = synth.long_chunk_bf16()
+    (cs, rows), = wl.prefill
+    k, v = _cache(0, wl.capacity, wl.capacity, "bf16")
+    q = synth.draw(0, "q", (rows, 8, 256), "bf16")
+    out = kca.attn_prefill(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), cs)
+    sample = np.array([0, 1, 15, 16, 17, 300, 511, 700, 766, 767])
+    want = oracle_prefill(q, k, v, cs, sample, 0, "bf16", "bf16")
+    assert max_err(out.cpu().numpy()[sample], want) <= 4e-3
