@@ -135,6 +135,32 @@ int attn_decode(const void *q, int32_t q_dtype,
                 float scale, float *out, void *workspace, size_t workspace_bytes,
                 void *stream);
 
+/*
+ * attn_decode_static -- attn_decode for callers that cannot allocate device
+ * memory: code running where cudaMalloc is unavailable or forbidden (inside a
+ * host callback, a custom allocator's own path, a memory pool that admits no
+ * further allocations, a runtime that only hands out the tensors it owns).
+ * The paper has no counterpart to this entry point.
+ *
+ * Arguments, layouts, semantics and errors are those of attn_decode, minus
+ * the workspace: the per-split partials go to a file-scope device array of
+ * KCA_STATIC_SCRATCH_BYTES (16 MiB) that every GPU loading the library holds
+ * until the process exits.  A call whose plan needs more than that (many
+ * sequences next to a very long one) returns KCA_ERR_WORKSPACE without
+ * launching.  The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress) with that device current; make it before any stream
+ * capture.  No call allocates or frees memory.  All calls on a device share
+ * the array: calls that may overlap on the GPU race on it, so serialise them.
+ * Nothing in the array must start at zero; its first KCA_WORKSPACE_HEADER
+ * bytes hold the device status word described above.
+ */
+#define KCA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int attn_decode_static(const void *q, int32_t q_dtype,
+                       const void *k_cache, const void *v_cache, int32_t kv_dtype,
+                       int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity,
+                       int32_t batch, const int64_t *ctx_len, int32_t window,
+                       float scale, float *out, void *stream);
+
 /* Workspace bytes the calls above need on the current device (0 on a bad
  * argument).  Always >= KCA_WORKSPACE_HEADER. */
 size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,

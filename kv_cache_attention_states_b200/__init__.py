@@ -55,6 +55,9 @@ def lib() -> ctypes.CDLL:
         L.attn_decode.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp,
                                   vp, sz, vp]
         L.attn_decode.restype = ctypes.c_int
+        L.attn_decode_static.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32,
+                                         f32, vp, vp]
+        L.attn_decode_static.restype = ctypes.c_int
         L.attn_prefill_workspace_bytes.argtypes = [i32, i32, i64, i32, i32]
         L.attn_prefill_workspace_bytes.restype = sz
         L.attn_decode_workspace_bytes.argtypes = [i32, p64, i32]
@@ -199,6 +202,27 @@ def attn_decode(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.
                            ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
                            workspace.numel(), _stream_ptr(stream))
     _check(st, "attn_decode")
+    return out
+
+
+def attn_decode_static(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.0 / 16.0,
+                       out=None, stream=None):
+    """attn_decode for callers that cannot allocate device memory: the split
+    partials go to the library's fixed 16 MiB device array instead of a
+    workspace (see include/kca.h for the sharing rules)."""
+    import torch
+    batch = q.shape[0]
+    arr, ptr = _i64_array(ctx_len)
+    if arr.size != batch or k_cache.shape[0] != batch:
+        raise ValueError("ctx_len / k_cache must have one entry per sequence")
+    if out is None:
+        out = torch.empty((batch, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
+    st = lib().attn_decode_static(ctypes.c_void_p(q.data_ptr()), dtype_code(q),
+                                  ctypes.c_void_p(k_cache.data_ptr()), ctypes.c_void_p(v_cache.data_ptr()),
+                                  dtype_code(k_cache), N_Q_HEADS, N_KV_HEADS, HEAD_DIM, k_cache.shape[1],
+                                  batch, ptr, window, scale, ctypes.c_void_p(out.data_ptr()),
+                                  _stream_ptr(stream))
+    _check(st, "attn_decode_static")
     return out
 
 

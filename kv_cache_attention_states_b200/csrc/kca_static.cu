@@ -1,0 +1,66 @@
+// kca_static.cu -- attn_decode_static: attn_decode without a caller-provided
+// workspace, for callers that cannot allocate device memory.
+//
+// Who needs it: code that runs where cudaMalloc is not an option -- inside a
+// host callback or a custom allocator's own path, under a memory pool that
+// forbids further allocations, or in a runtime that hands out only the
+// tensors it owns.  Such a caller still owns q, the caches and out, but cannot
+// obtain the scratch that split-context decode writes its per-split partials
+// to.  This entry point takes that scratch from a fixed array in device
+// memory instead.  The paper has no counterpart to this entry point.
+//
+// The array below is created when the module loads on a device and is held
+// by every GPU that loads the library until the process exits.  Its device
+// address is looked up once per device (cudaGetSymbolAddress) on the first
+// call made with that device current; make that first call before any stream
+// capture.  All calls on a device share the array, so calls whose execution
+// can overlap on the GPU (different streams, or graphs replayed
+// concurrently) race on it and must be serialised by the caller.  Nothing in
+// the array needs to start at zero: every partial is written before it is
+// read within the same call, and the status word at its head (see
+// attn_device_status) only records errors.
+#include <cuda_runtime.h>
+
+#include "../../include/kca.h"
+
+namespace {
+
+static __device__ __align__(256) unsigned char kca_static_scratch[KCA_STATIC_SCRATCH_BYTES];
+
+// Device address of kca_static_scratch per device; the name itself is only a
+// host-side stand-in and must never be handed to a kernel.
+void* scratch_address(int* status) {
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *status = KCA_ERR_CUDA;
+    return nullptr;
+  }
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, kca_static_scratch) != cudaSuccess || p == nullptr) {
+      *status = KCA_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  *status = KCA_OK;
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" int attn_decode_static(const void* q, int32_t q_dtype, const void* k_cache,
+                                  const void* v_cache, int32_t kv_dtype, int32_t n_q_heads,
+                                  int32_t n_kv_heads, int32_t head_dim, int64_t capacity,
+                                  int32_t batch, const int64_t* ctx_len, int32_t window,
+                                  float scale, float* out, void* stream) {
+  int st = KCA_OK;
+  void* ws = scratch_address(&st);
+  if (ws == nullptr) return st;
+  // attn_decode validates every argument and returns KCA_ERR_WORKSPACE when
+  // the plan's partials would not fit the array.
+  return attn_decode(q, q_dtype, k_cache, v_cache, kv_dtype, n_q_heads, n_kv_heads, head_dim,
+                     capacity, batch, ctx_len, window, scale, out, ws, KCA_STATIC_SCRATCH_BYTES,
+                     stream);
+}
