@@ -171,6 +171,28 @@ def run_cuda(args, rank, world, local_rank):
         w.decode()
         w.step_index += 1
     torch.cuda.synchronize()
+    graphs = None
+    if not args.eager:
+        # One graph per prefill input replica and one for the 64 decode steps
+        # (each step visits the 32 cache replicas in the same order).
+        graphs = {"pre": [], "dec": None}
+        saved = w.step_index
+        for r in range(PREFILL_REPLICAS):
+            g = torch.cuda.CUDAGraph()
+            w.step_index = r
+            with torch.cuda.graph(g):
+                w.prefill()
+            graphs["pre"].append(g)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            w.decode()
+        graphs["dec"] = g
+        w.step_index = saved
+        for _ in range(2):
+            graphs["pre"][w.step_index % PREFILL_REPLICAS].replay()
+            graphs["dec"].replay()
+            w.step_index += 1
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -181,9 +203,15 @@ def run_cuda(args, rank, world, local_rank):
     start.record(stream)
     for s in range(args.steps):
         ev[s][0].record(stream)
-        w.prefill()
+        if graphs is None:
+            w.prefill()
+        else:
+            graphs["pre"][w.step_index % PREFILL_REPLICAS].replay()
         ev[s][1].record(stream)
-        w.decode()
+        if graphs is None:
+            w.decode()
+        else:
+            graphs["dec"].replay()
         ev[s][2].record(stream)
         w.step_index += 1
     end.record(stream)
@@ -350,6 +378,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="kca", choices=["kca", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="launch every call from Python instead of "
+                    "replaying a captured CUDA graph of the step")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -395,6 +425,7 @@ def main():
                                "1 KV head, head_dim 256, causal",
                    "seq_len": 16384, "global_batch": world, "parallelism": f"replicas x{world}",
                    "value": "prefill part of each step (CUDA events); decode part in 'decode'",
+                   "launch": "eager" if args.eager else "CUDA graph of the step's C-ABI calls",
                    "l2": "inputs larger than L2: decode rotates 32 cache replicas (16.8 MB each), "
                          "prefill alternates 2 input replicas (80 MB each)"},
         "roofline": {"kernel": "prefill_tc_kernel (+ its merge)", "bound": "tensor",

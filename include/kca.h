@@ -83,7 +83,7 @@ extern "C" {
 #define KCA_ERR_NULL (-1)       /* a required pointer is NULL                      */
 #define KCA_ERR_GEOMETRY (-2)   /* heads / head_dim other than 8 / 1 / 256         */
 #define KCA_ERR_DTYPE (-3)      /* unknown dtype code                              */
-#define KCA_ERR_RANGE (-4)      /* rows, positions, capacity, batch or window      */
+#define KCA_ERR_RANGE (-4)      /* rows, positions, capacity, batch or scale       */
 #define KCA_ERR_WORKSPACE (-5)  /* workspace too small or misaligned               */
 #define KCA_ERR_ALIGN (-6)      /* q / k / v / out not 16-byte aligned             */
 #define KCA_ERR_CUDA (-7)       /* a CUDA runtime call failed                      */
@@ -107,7 +107,7 @@ extern "C" {
  *   chunk_rows   1..768
  *   ctx_len      must equal chunk_start + chunk_rows, <= capacity
  *   window       <= 0: none; otherwise keys [pos-window+1, pos]
- *   scale        finite score scale (1/sqrt(256) for Gemma 4)
+ *   scale        finite score scale > 0 (1/sqrt(256) for Gemma 4)
  *   out          [chunk_rows][8][256] float32, device
  *   workspace    >= attn_prefill_workspace_bytes(...) bytes, device
  * Returns KCA_OK or a negative KCA_ERR_*.

@@ -288,7 +288,8 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
   if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
   st = prefill_args_status(capacity, chunk_start, chunk_rows);
   if (st != KCA_OK) return st;
-  if (ctx_len != chunk_start + chunk_rows || !std::isfinite(scale)) return KCA_ERR_RANGE;
+  if (ctx_len != chunk_start + chunk_rows || !std::isfinite(scale) || !(scale > 0.f))
+    return KCA_ERR_RANGE;
   if (!aligned16(q_chunk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return KCA_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
@@ -305,6 +306,7 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
     a.status = workspace;
     a.scale_log2 = scale * 1.4426950408889634f;
     carve(workspace, (size_t)a.plan.n_slots * 128 * 2 * 4, &a.part_ml, &a.part_acc);
+    kca::fill_tc_tables(a);
     CUtensorMap tmk, tmv;
     if (!encode_kv_map(&tmk, k_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len) ||
         !encode_kv_map(&tmv, v_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len))
@@ -343,7 +345,7 @@ int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void*
   if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
   st = decode_args_status(capacity, batch, ctx_len);
   if (st != KCA_OK) return st;
-  if (!std::isfinite(scale)) return KCA_ERR_RANGE;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return KCA_ERR_RANGE;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return KCA_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;

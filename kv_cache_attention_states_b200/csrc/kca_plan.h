@@ -106,6 +106,7 @@ struct TcPlan {
   int32_t per_item;     // c: most key tiles one item covers
   int32_t n_items;
   int32_t n_slots;      // items that belong to split tiles (write partials)
+  int32_t max_split;    // most items of one tile
 };
 
 constexpr int kTcMinItemTiles = 4;
@@ -185,7 +186,8 @@ inline TcPlan make_tc_plan(int64_t chunk_start, int32_t rows, int32_t window, in
     total += ke - kb;
     if (ke - kb > longest) longest = ke - kb;
   }
-  const int32_t sms = num_sms > 0 ? num_sms : 1;
+  // one wave of CTAs, capped by the launch's item table (160 entries)
+  const int32_t sms = num_sms < 1 ? 1 : (num_sms > 160 ? 160 : num_sms);
   int32_t c = (int32_t)cdiv(total, sms);
   if (c < kTcMinItemTiles) c = kTcMinItemTiles;
   for (;; ++c) {
@@ -194,14 +196,16 @@ inline TcPlan make_tc_plan(int64_t chunk_start, int32_t rows, int32_t window, in
     for (int32_t t = 0; t < p.n_tiles; ++t) items += tc_tile_items(p, t);
     if (items <= sms || c >= longest) break;
   }
-  int32_t items = 0, slots = 0;
+  int32_t items = 0, slots = 0, most = 1;
   for (int32_t t = 0; t < p.n_tiles; ++t) {
     const int32_t s = tc_tile_items(p, t);
     items += s;
     if (s > 1) slots += s;
+    if (s > most) most = s;
   }
   p.n_items = items;
   p.n_slots = slots;
+  p.max_split = most;
   return p;
 }
 

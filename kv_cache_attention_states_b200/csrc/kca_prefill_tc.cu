@@ -25,11 +25,12 @@
 // result is exact up to rounding whatever reference max is used.
 //
 // Work items of a split row tile write (m, l, O) partials that
-// merge_tc_kernel combines by log-sum-exp.
+// merge_tc_kernel combines by log-sum-exp (kca_merge.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "kca_common.cuh"
+#include "kca_merge.cuh"
 #include "kca_plan.h"
 #include "kca_tc.h"
 #include "kca_tc_ptx.cuh"
@@ -85,9 +86,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const TcItem it = tc_item(a.plan, blockIdx.x);
+  const TcItemArg it = a.items[blockIdx.x];
   const int n = it.kt_end - it.kt_begin;
-  if (it.tile < 0 || n <= 0) return;  // the host never launches such a CTA
+  if (n <= 0) return;  // the host never launches such a CTA
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kRing; ++i) {
@@ -227,8 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->q_full);
     }
 
-    float m_ref = -INFINITY;   // log2 domain
+    float m_ref = -INFINITY;   // reference max, log2 units
     float l_sum = 0.f;
+    const float cs = a.scale_log2;
     bool ok = true;
     for (int t = 0; t < n; ++t) {
       const int b = t & 1;
@@ -236,39 +238,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort_flag, status, kSiteTcS));
       if (!ok) break;
       ptx::fence_after_sync();
-      float x[64];
+      float s[64];
       {
-        uint32_t r[32];
-        ptx::tmem_ld32(trow + scol, r);
+        uint32_t r0[32], r1[32];
+        ptx::tmem_ld32(trow + scol, r0);
+        ptx::tmem_ld32(trow + scol + 32, r1);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(r[c]) * a.scale_log2;
-        ptx::tmem_ld32(trow + scol + 32, r);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[32 + c] = __uint_as_float(r[c]) * a.scale_log2;
+        for (int c = 0; c < 32; ++c) {
+          s[c] = __uint_as_float(r0[c]);
+          s[32 + c] = __uint_as_float(r1[c]);
+        }
       }
+      // Raw scores of keys outside [lo, pos] become -inf (the scale is > 0,
+      // so they stay -inf below and their probability is exactly 0).
       const int64_t j0 = a.plan.kv_lo + (int64_t)(it.kt_begin + t) * kKeyTile;
       if (j0 < lo || j0 + kKeyTile - 1 > pos) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int64_t j = j0 + c;
-          if (j < lo || j > pos) x[c] = -INFINITY;
+          if (j < lo || j > pos) s[c] = -INFINITY;
         }
       }
-      float mx = -INFINITY;
+      // NaN-preserving row max over eight independent chains.
+      float m8[8];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) mx = max_nan(mx, x[c]);
+      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < 64; ++c) m8[c & 7] = max_nan(m8[c & 7], s[c]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m8[i] = max_nan(m8[i], m8[i + 4]);
+      const float mraw = max_nan(max_nan(m8[0], m8[2]), max_nan(m8[1], m8[3]));
+      const float mx = mraw == -INFINITY ? -INFINITY : mraw * cs;
       const bool need = mx > m_ref + kRescaleLog2;
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? exp2f(m_ref - mx) : 1.f;
+      const bool any_need = __any_sync(0xffffffffu, need);
+      float alpha = 1.f;
+      if (any_need) {
+        alpha = need ? ptx::ex2(m_ref - mx) : 1.f;
         if (need) m_ref = mx;
         l_sum *= alpha;
-        if (t > 0) {
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, status, kSiteTcO));
-          if (!ok) break;
-          ptx::fence_after_sync();
+      }
+      // p = 2^(s*scale*log2e - m_ref), one FFMA and one MUFU op per score.
+      const float nmu = m_ref == -INFINITY ? 0.f : -m_ref;
+      uint32_t pr[32];
+      float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ptx::ex2(fmaf(s[2 * c], cs, nmu));
+        const float p1 = ptx::ex2(fmaf(s[2 * c + 1], cs, nmu));
+        acc2[c & 3] = __fadd2_rn(acc2[c & 3], make_float2(p0, p1));
+        pr[c] = pack2(p0, p1, DT);
+      }
+      acc2[0] = __fadd2_rn(acc2[0], acc2[1]);
+      acc2[2] = __fadd2_rn(acc2[2], acc2[3]);
+      acc2[0] = __fadd2_rn(acc2[0], acc2[2]);
+      l_sum += acc2[0].x + acc2[0].y;
+      ptx::tmem_st32(trow + scol, pr);
+      // PV of the previous tile must be complete before O is touched and
+      // before this thread lets PV of this tile start; waiting on every tile
+      // keeps this thread within one phase of the barrier, which parity
+      // waits require.
+      if (t > 0) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, status, kSiteTcO));
+        if (!ok) break;
+        ptx::fence_after_sync();
+        if (any_need) {
 #pragma unroll 1
           for (int c = 0; c < kDim / 32; ++c) {
             uint32_t r[32];
@@ -278,21 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
             ptx::tmem_st32(trow + kColO + c * 32, r);
           }
-          ptx::tmem_wait_st();
         }
       }
-      const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-      uint32_t pr[32];
-      float ls = 0.f;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = exp2f(x[2 * c] - mu);
-        const float p1 = exp2f(x[2 * c + 1] - mu);
-        ls += p0 + p1;
-        pr[c] = pack2(p0, p1, DT);
-      }
-      l_sum += ls;
-      ptx::tmem_st32(trow + scol, pr);
       ptx::tmem_wait_st();
       ptx::fence_before_sync();
       mbar_arrive(&bars->p_full[b]);
@@ -335,55 +358,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Log-sum-exp merge of the items of each split row tile; warp w takes the M
-// rows w, w+8, ..., lane the dims [8*lane, 8*lane+8).
+// Log-sum-exp merge of the items of each split row tile: a group of W warps
+// per M row, 8 / W rows per CTA, grid (tiles, 16 W).
+template <int W>
 __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
+  constexpr int kRowsPerCta = 8 / W;
   const int tile = blockIdx.x;
-  const int ns = tc_tile_items(a.plan, tile);
+  const int ns = a.tile_items[tile];
   if (ns <= 1) return;
-  const int slot0 = tc_tile_first_slot(a.plan, tile);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int m = warp; m < 128; m += 8) {
-    const int64_t row = (int64_t)tile * kRowTile + (m >> 3);
-    if (row >= a.plan.rows) break;
-    float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = max_nan(M, a.part_ml[((int64_t)(slot0 + s) * 128 + m) * 2]);
-    const float mu = M == -INFINITY ? 0.f : M;
-    float L = 0.f, A[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < ns; ++s) {
-      const int64_t r = (int64_t)(slot0 + s) * 128 + m;
-      const float f = exp2f(a.part_ml[r * 2] - mu);
-      L += f * a.part_ml[r * 2 + 1];
-      const float4* src = reinterpret_cast<const float4*>(a.part_acc + r * kDim + 8 * lane);
-      const float4 x0 = src[0], x1 = src[1];
-      A[0] += f * x0.x; A[1] += f * x0.y; A[2] += f * x0.z; A[3] += f * x0.w;
-      A[4] += f * x1.x; A[5] += f * x1.y; A[6] += f * x1.z; A[7] += f * x1.w;
-    }
-    const float inv = 1.f / L;
-    float4* o = reinterpret_cast<float4*>(a.out + ((int64_t)tile * 128 + m) * kDim + 8 * lane);
-    o[0] = make_float4(A[0] * inv, A[1] * inv, A[2] * inv, A[3] * inv);
-    o[1] = make_float4(A[4] * inv, A[5] * inv, A[6] * inv, A[7] * inv);
-  }
+  __shared__ float red[8 * 264];
+  const int warp = threadIdx.x >> 5;
+  const int gi = warp / W, g = warp % W;
+  const int m = blockIdx.y * kRowsPerCta + gi;
+  if ((int64_t)tile * kRowTile + (m >> 3) >= a.plan.rows) return;  // whole group leaves together
+  const int64_t r0 = (int64_t)a.tile_first_slot[tile] * 128 + m;
+  merge_row<W>(ns, a.part_ml + r0 * 2, 128 * 2, a.part_acc + r0 * kDim, (int64_t)128 * kDim, 1.f,
+               a.out + ((int64_t)tile * 128 + m) * kDim, red + gi * W * 264, g, threadIdx.x & 31,
+               1 + gi);
 }
 
 template <int DT>
 cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const TcArgs& a,
                      cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<DT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev] = true;
   }
   prefill_tc_kernel<DT><<<a.plan.n_items, kThreads, kSmemBytes, stream>>>(tmk, tmv, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.plan.n_slots == 0) return e;
-  merge_tc_kernel<<<a.plan.n_tiles, 256, 0, stream>>>(a);
+  const int ns = a.plan.max_split;
+  const int w = ns > 8 ? 8 : (ns > 4 ? 4 : (ns > 2 ? 2 : 1));
+  const dim3 grid(a.plan.n_tiles, 16 * w);
+  if (w == 8) merge_tc_kernel<8><<<grid, 256, 0, stream>>>(a);
+  else if (w == 4) merge_tc_kernel<4><<<grid, 256, 0, stream>>>(a);
+  else if (w == 2) merge_tc_kernel<2><<<grid, 256, 0, stream>>>(a);
+  else merge_tc_kernel<1><<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+void fill_tc_tables(TcArgs& a) {
+  // One pass over the tiles: O(tiles + items), no per-item plan walk.
+  int32_t idx = 0, slot = 0;
+  for (int32_t t = 0; t < a.plan.n_tiles && t < kTcMaxTiles; ++t) {
+    int32_t kb, ke;
+    tc_tile_keys(a.plan, t, &kb, &ke);
+    const int32_t n = ke - kb;
+    const int32_t s = (int32_t)cdiv(n, a.plan.per_item);
+    a.tile_items[t] = (int16_t)s;
+    a.tile_first_slot[t] = (int16_t)slot;
+    for (int32_t k = 0; k < s && idx < kTcMaxItems; ++k, ++idx) {
+      a.items[idx].kt_begin = kb + (int32_t)(((int64_t)k * n) / s);
+      a.items[idx].kt_end = kb + (int32_t)(((int64_t)(k + 1) * n) / s);
+      a.items[idx].tile = (int16_t)t;
+      a.items[idx].slot = (int16_t)(s > 1 ? slot + k : -1);
+    }
+    if (s > 1) slot += s;
+  }
+}
 
 cudaError_t launch_prefill_tc(int dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                               const TcArgs& a, cudaStream_t stream) {

@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include "kca_common.cuh"
+#include "kca_merge.cuh"
 #include "kca_plan.h"
 #include "kca_rows.h"
 
@@ -161,10 +162,10 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
 
     for (int i = 0; i < n_stage && ok; ++i) {
       const int slot = i % kStages;
-      if (!mbar_wait(&full[slot], (i / kStages) & 1, abort_flag, status, kSiteRowsFull)) {
-        ok = false;
-        break;
-      }
+      // warp-uniform, so no lane reaches the shuffles below without the others
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&full[slot], (i / kStages) & 1, abort_flag, status, kSiteRowsFull));
+      if (!ok) break;
       const int64_t k0 = kbeg + (int64_t)i * kKeysPerStage;
       const int cnt = (int)((kend - k0) < kKeysPerStage ? (kend - k0) : kKeysPerStage);
       const unsigned char* st = smem + slot * S::kStageBytes;
@@ -288,45 +289,38 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
   }
 }
 
-// Log-sum-exp merge of the splits of each unit: one CTA per unit, thread
-// (head = warp, lane) owns dims [8*lane, 8*lane+8).
+// Log-sum-exp merge of the splits of each unit: one CTA per (unit, head),
+// its eight warps taking interleaved splits.
 __global__ void __launch_bounds__(256) merge_rows_kernel(const RowsArgs a) {
-  const int unit = blockIdx.x;
+  const int unit = blockIdx.x >> 3, h = blockIdx.x & 7;
   const int64_t pos = a.mode == 0 ? a.ctx[unit] - 1 : a.chunk_start + unit;
   const int32_t nsplit = rows_n_splits(n_visible(pos, a.window), a.split_len);
   if (nsplit <= 1) return;
-  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t slot0 = (int64_t)unit * a.max_splits;
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = max_nan(M, a.part_ml[((slot0 + s) * kHeads + h) * 2]);
-  const float M_use = M == -INFINITY ? 0.f : M;
-  float L = 0.f, A[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < nsplit; ++s) {
-    const int64_t row = (slot0 + s) * kHeads + h;
-    const float f = exp2f((a.part_ml[row * 2] - M_use) * kLog2e);
-    L += f * a.part_ml[row * 2 + 1];
-    const float4* src = reinterpret_cast<const float4*>(a.part_acc + row * kDim + 8 * lane);
-    const float4 x0 = src[0], x1 = src[1];
-    A[0] += f * x0.x; A[1] += f * x0.y; A[2] += f * x0.z; A[3] += f * x0.w;
-    A[4] += f * x1.x; A[5] += f * x1.y; A[6] += f * x1.z; A[7] += f * x1.w;
-  }
-  const float inv = 1.f / L;
-  float4* o = reinterpret_cast<float4*>(a.out + ((int64_t)unit * kHeads + h) * kDim + 8 * lane);
-  o[0] = make_float4(A[0] * inv, A[1] * inv, A[2] * inv, A[3] * inv);
-  o[1] = make_float4(A[4] * inv, A[5] * inv, A[6] * inv, A[7] * inv);
+  __shared__ float red[8 * 264];
+  const int64_t row0 = (int64_t)unit * a.max_splits * kHeads + h;
+  merge_row<8>(nsplit, a.part_ml + row0 * 2, kHeads * 2, a.part_acc + row0 * kDim, kHeads * kDim,
+               kLog2e, a.out + ((int64_t)unit * kHeads + h) * kDim, red, threadIdx.x >> 5,
+               threadIdx.x & 31, 1);
 }
 
 template <int QT, int KT>
 cudaError_t launch_rows_t(const RowsArgs& a, cudaStream_t stream) {
   using S = RowsSmem<KT>;
   auto kern = rows_kernel<QT, KT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
-  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaError_t e;
   dim3 grid(a.max_splits, a.n_units);
   kern<<<grid, kRowsThreads, S::kTotal, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.max_splits <= 1) return e;
-  merge_rows_kernel<<<a.n_units, 256, 0, stream>>>(a);
+  merge_rows_kernel<<<a.n_units * kHeads, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

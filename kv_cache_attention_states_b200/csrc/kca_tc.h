@@ -8,6 +8,18 @@
 
 namespace kca {
 
+constexpr int kTcMaxItems = 160;   // work items (CTAs) of one call
+constexpr int kTcMaxTiles = 48;    // 768 rows / 16
+
+// One work item, filled in on the host from the plan so that no CTA has to
+// walk the plan itself.
+struct TcItemArg {
+  int32_t kt_begin;   // key tiles relative to plan.kv_lo
+  int32_t kt_end;
+  int16_t tile;       // row tile
+  int16_t slot;       // partial slot, -1 when the tile is not split
+};
+
 struct TcArgs {
   const void* q;      // [rows][8][256], 16-bit
   float* out;         // [rows][8][256]
@@ -16,7 +28,13 @@ struct TcArgs {
   void* status;       // workspace status header
   TcPlan plan;
   float scale_log2;   // scale * log2(e)
+  TcItemArg items[kTcMaxItems];
+  int16_t tile_first_slot[kTcMaxTiles];
+  int16_t tile_items[kTcMaxTiles];
 };
+
+// Fills the item and tile tables of a from a.plan (host).
+void fill_tc_tables(TcArgs& a);
 
 // tmk / tmv: 2-D tensor maps over the rows [plan.kv_lo, plan.ctx_len) of the
 // K and V caches, inner extent 256, box 64 x 64, 128-byte swizzle, zero fill.

@@ -79,6 +79,13 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 2^x on the MUFU unit (flushes subnormal results to zero).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------------------------- TMA
 // 2-D tiled load (no multicast) of box {x, y} into shared memory, completing
 // on an mbarrier.  x * element size must be a multiple of 16 bytes.

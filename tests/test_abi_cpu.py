@@ -78,6 +78,7 @@ def _decode(ctx=(100, 200), **kw):
     (dict(rows=0, ctx=0), -4), (dict(rows=769, ctx=769), -4), (dict(cs=-1, ctx=767), -4),
     (dict(cap=0), -4), (dict(cap=131073), -4), (dict(cs=4000, ctx=4768), -4),
     (dict(ctx=767), -4), (dict(scale=float("nan")), -4), (dict(scale=float("inf")), -4),
+    (dict(scale=0.0), -4), (dict(scale=-0.0625), -4),
     (dict(q=P + 8), -6), (dict(k=P + 4), -6), (dict(v=P + 2), -6), (dict(out=P + 8), -6),
     (dict(ws=P * 2 + 16), -5),
 ])
@@ -89,6 +90,7 @@ def test_prefill_rejects_bad_arguments_on_the_host(kw, code):
     ((1, 2), dict(q=0), -1), ((1, 2), dict(hq=4), -2), ((1, 2), dict(kd=3), -3),
     ((1, 2), dict(batch=0), -4), ((1,) * 257, dict(), -4), ((1, 4097), dict(), -4),
     ((-1, 2), dict(), -4), ((1, 2), dict(cap=131073), -4), ((1, 2), dict(scale=float("nan")), -4),
+    ((1, 2), dict(scale=0.0), -4),
     ((1, 2), dict(out=P + 4), -6), ((1, 2), dict(ws=P * 2 + 128), -5),
 ])
 def test_decode_rejects_bad_arguments_on_the_host(ctx, kw, code):
