@@ -25,7 +25,6 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool dtype_ok(int32_t d) { return d == KCA_F32 || d == KCA_F16 || d == KCA_BF16; }
-size_t elem_bytes(int32_t d) { return d == KCA_F32 ? 4 : 2; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int geometry_status(int32_t hq, int32_t hkv, int32_t d) {
@@ -117,14 +116,15 @@ EncodeTiledFn encode_fn() {
 }
 
 // Map over rows [kv_lo, ctx_len) of one cache: inner extent 256 elements,
-// 64 x 64 boxes, 128-byte swizzle, zero fill outside.
-bool encode_kv_map(CUtensorMap* m, const void* cache, int32_t dtype, int64_t kv_lo, int64_t ctx_len) {
+// boxes of 64 elements x box_rows rows, 128-byte swizzle, zero fill outside.
+bool encode_kv_map(CUtensorMap* m, const void* cache, int32_t dtype, int64_t kv_lo, int64_t ctx_len,
+                   uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const char* base = static_cast<const char*>(cache) + kv_lo * kDim * 2;
   cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)(ctx_len - kv_lo)};
   cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kca::kKeyTile};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType t =
       dtype == KCA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -308,8 +308,9 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
     carve(workspace, (size_t)a.plan.n_slots * 128 * 2 * 4, &a.part_ml, &a.part_acc);
     kca::fill_tc_tables(a);
     CUtensorMap tmk, tmv;
-    if (!encode_kv_map(&tmk, k_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len) ||
-        !encode_kv_map(&tmv, v_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len))
+    // K: one 64-dim chunk of a 128-key tile per box; V: 64-key halves.
+    if (!encode_kv_map(&tmk, k_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, kca::kKeyTile) ||
+        !encode_kv_map(&tmv, v_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, 64))
       return KCA_ERR_CUDA;
     return kca::launch_prefill_tc(kv_dtype, tmk, tmv, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
   }

@@ -22,7 +22,7 @@ namespace kca {
 constexpr int kHeads = 8;        // query heads per KV head
 constexpr int kDim = 256;        // head_dim
 constexpr int kRowTile = 16;     // query positions per tensor-core row tile (16 x 8 heads = 128 M rows)
-constexpr int kKeyTile = 64;     // keys per tensor-core KV tile
+constexpr int kKeyTile = 128;    // keys per tensor-core KV tile
 constexpr int kPartFloats = 2 + kDim;  // per (slot, row): m, l, acc[256]
 
 KCA_HD int64_t lo_of(int64_t pos, int32_t window) {
@@ -93,7 +93,7 @@ inline RowsPlan make_rows_plan(int32_t n_units, const int64_t* nkeys, int32_t nu
 // A chunk of `rows` query rows at chunk_start is cut into row tiles of 16
 // positions (x 8 heads = 128 M rows).  Keys are addressed relative to
 // kv_lo = lo(chunk_start), the first key any row of the chunk sees, in tiles
-// of 64.  Row tile t covers key tiles [kb(t), ke(t)); it is split into
+// of 128.  Row tile t covers key tiles [kb(t), ke(t)); it is split into
 // ceil(n/c) items of near-equal length, c chosen as the smallest value that
 // keeps the item count within one wave of CTAs.
 struct TcPlan {
@@ -109,7 +109,7 @@ struct TcPlan {
   int32_t max_split;    // most items of one tile
 };
 
-constexpr int kTcMinItemTiles = 4;
+constexpr int kTcMinItemTiles = 2;
 
 KCA_HD void tc_tile_keys(const TcPlan& p, int32_t t, int32_t* kb, int32_t* ke) {
   const int64_t first = p.chunk_start + (int64_t)t * kRowTile;

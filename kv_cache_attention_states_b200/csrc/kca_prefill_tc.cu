@@ -4,28 +4,36 @@
 // for plans of 16 or more chunk rows, QK and PV run on a GEMM tile skeleton
 // so that each K / V row is read once per row tile instead of once per query
 // row.  Here one CTA takes one work item -- a row tile of 16 positions x 8
-// heads (M = 128, the heads share their single KV head) and a run of 64-key
-// tiles -- and fuses the three stages the pages keep apart (QK, softmax
-// statistics, PV) so no score matrix ever reaches memory:
+// heads (M = 128: the 8 heads share their single KV head) and a run of
+// 128-key tiles -- and fuses the three stages the pages keep apart (QK,
+// softmax statistics, PV), so no score matrix ever reaches memory.
 //
-//   warp 0      TMA producer: K and V tiles (64 keys x 256 dims, four
-//               64 x 64 boxes with 128-byte swizzle) into a 6-slot ring
+// Warp roles (12 warps):
+//   warp 0      TMA producer of K: each 128-key tile as four 64-dim chunks
+//               (128 rows x 128 B, 128-byte swizzle), two chunks per slot of
+//               a 2-slot ring
 //   warp 1      TMEM allocator and the single MMA-issuing thread
-//   warps 4-7   softmax warpgroup: thread m owns TMEM lane m (= M row m)
+//   warp 2      TMA producer of V: 64-key halves (four 64 x 64 boxes) into a
+//               2-slot ring
+//   warps 4-7   softmax warpgroup 0: keys 0-63 of every S tile
+//   warps 8-11  softmax warpgroup 1: keys 64-127
+//   Thread m of a softmax warpgroup owns TMEM lane m, i.e. M row m.
 //
 // Tensor memory (512 columns x 128 lanes of 32 bits):
-//   [  0,128)  Q tile, bf16/f16 pairs: the A operand of S = Q K^T
-//   [128,192)  S0 (f32, 64 keys);  P0 (16-bit pairs) over its first 32 columns
-//   [192,256)  S1;                 P1 likewise
-//   [256,512)  O accumulator, 256 f32 columns
-// S is double-buffered so QK^T of tile t+1 runs on the tensor cores while the
-// softmax warpgroup works on tile t.  The softmax keeps a reference max per
-// row and rescales O (in TMEM) only when a score exceeds it by more than
-// 2^8, so probabilities stay <= 256 and the O round trip is rare.  The
-// result is exact up to rounding whatever reference max is used.
+//   [  0,128)  Q tile as 16-bit pairs: the A operand of S = Q K^T
+//   [128,256)  S (f32, 128 keys), released as soon as both warpgroups hold
+//              their half in registers, so QK^T of the next tile overlaps
+//              the softmax of this one
+//   [256,512)  O accumulator (f32, 256 dims)
+// P (16-bit) goes to shared memory, double-buffered, as the A operand of
+// O += P V.  Shapes per instruction: QK^T M128 N128 K16, PV M128 N256 K16;
+// both keep the tensor pipe at full rate from a single issuing thread.
 //
-// Work items of a split row tile write (m, l, O) partials that
-// merge_tc_kernel combines by log-sum-exp (kca_merge.cuh).
+// The softmax keeps a reference max per row and rescales O (in TMEM) only
+// when a score exceeds it by more than 2^8, so probabilities stay <= 256 and
+// the O round trip is rare; the result is exact up to rounding whatever
+// reference is used.  Work items of a split row tile write (m, l, O)
+// partials that merge_tc_kernel combines by log-sum-exp (kca_merge.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -38,29 +46,42 @@
 namespace kca {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kRing = 6;
-constexpr int kBoxBytes = kKeyTile * 64 * 2;         // 64 keys x 64 dims x 2 B = 8 KiB
-constexpr int kSlotBytes = 4 * kBoxBytes;            // one K or V tile: 32 KiB
-constexpr int kRingBytes = kRing * kSlotBytes;
-constexpr int kBarBytes = 512;
-constexpr int kSmemBytes = kRingBytes + kBarBytes + 1024;  // + alignment slack
+constexpr int kThreads = 384;
+constexpr int kKRing = 2;                              // K slots of two 64-dim chunks
+constexpr int kVRing = 2;                              // V half-tile slots
+constexpr int kKChunkBytes = kKeyTile * 64 * 2;        // 128 keys x 64 dims: 16 KiB
+constexpr int kKSlotBytes = 2 * kKChunkBytes;          // two chunks: 32 KiB
+constexpr int kVBoxBytes = 64 * 64 * 2;                // 64 keys x 64 dims: 8 KiB
+constexpr int kVHalfBytes = 4 * kVBoxBytes;            // 64 keys x 256 dims: 32 KiB
+constexpr int kPBytes = 128 * kKeyTile * 2;            // 128 rows x 128 keys: 32 KiB
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kKRing * kKSlotBytes;    // 64 KiB
+constexpr int kOffP = kOffV + kVRing * kVHalfBytes;    // 128 KiB
+constexpr int kOffBar = kOffP + 2 * kPBytes;           // 192 KiB
+constexpr int kBarBytes = 4096;
+constexpr int kSmemBytes = kOffBar + kBarBytes + 1024; // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColQ = 0, kColS0 = 128, kColS1 = 192, kColO = 256;
-constexpr float kRescaleLog2 = 8.f;   // rescale O once a score passes the reference by 2^8
+constexpr uint32_t kColQ = 0, kColS = 128, kColO = 256;
+constexpr float kRescaleLog2 = 8.f;  // rescale O once a score passes the reference by 2^8
+constexpr int kSoftmaxThreads = 256;
 
 struct Bars {
-  uint64_t full[kRing];
-  uint64_t empty[kRing];
-  uint64_t q_full;
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done;
-  uint64_t drain;
+  uint64_t kfull[kKRing], kempty[kKRing];
+  uint64_t vfull[kVRing], vempty[kVRing];
+  uint64_t q_full;     // Q in TMEM (256 softmax threads)
+  uint64_t s_full;     // S of the current tile computed (MMA commit)
+  uint64_t s_free;     // S copied to registers by all 256 softmax threads
+  uint64_t p_full[2];  // P of tile t in buffer t&1 written, O corrected (256 threads)
+  uint64_t o_done[2];  // PV of tile u complete (MMA commit), u&1 selects the barrier
+  uint64_t o_final;    // every PV complete (single use)
+  uint64_t drain;      // every MMA complete (single use, MMA thread)
   uint32_t tmem_base;
   int abort;
+  float red_max[2][2][128];  // [tile parity][warpgroup][row]: partial row maxima
+                             // (partial row sums at the end)
 };
 static_assert(sizeof(Bars) <= kBarBytes, "barrier block too large");
+static_assert(kSmemBytes <= 232448, "shared memory over the per-CTA limit");
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, int dt) {
   if (dt == KCA_BF16) {
@@ -71,6 +92,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, int dt) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -79,8 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
   unsigned char* smem = smem_raw + pad;
-  const uint32_t ring_addr = raw_addr + pad;
-  Bars* bars = reinterpret_cast<Bars*>(smem + kRingBytes);
+  const uint32_t sbase = raw_addr + pad;
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
   volatile int* abort_flag = &bars->abort;
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.status);
 
@@ -91,16 +120,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (n <= 0) return;  // the host never launches such a CTA
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRing; ++i) {
-      mbar_init(&bars->full[i], 1);
-      mbar_init(&bars->empty[i], 1);
+    for (int i = 0; i < kKRing; ++i) {
+      mbar_init(&bars->kfull[i], 1);
+      mbar_init(&bars->kempty[i], 1);
     }
-    mbar_init(&bars->q_full, 128);
+    for (int i = 0; i < kVRing; ++i) {
+      mbar_init(&bars->vfull[i], 1);
+      mbar_init(&bars->vempty[i], 1);
+    }
+    mbar_init(&bars->q_full, kSoftmaxThreads);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, kSoftmaxThreads);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->p_full[i], kSoftmaxThreads);
+      mbar_init(&bars->o_done[i], 1);
     }
-    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->o_final, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_barrier_init();
@@ -114,35 +149,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers
     if (lane == 0) {
-      ptx::prefetch_tmap(&tmk);
-      ptx::prefetch_tmap(&tmv);
+      const bool is_k = warp == 0;
+      const int ring = is_k ? kKRing : kVRing;
+      uint64_t* full = is_k ? bars->kfull : bars->vfull;
+      uint64_t* empty = is_k ? bars->kempty : bars->vempty;
+      ptx::prefetch_tmap(is_k ? &tmk : &tmv);
+      const int per_tile = 2;   // K: two slots of two 64-dim chunks, V: two 64-key halves
       int e = 0;
       bool ok = true;
-      auto issue = [&](const CUtensorMap* map, int kt) -> bool {
-        const int slot = e % kRing;
-        if (e >= kRing &&
-            !mbar_wait(&bars->empty[slot], ((e / kRing) - 1) & 1, abort_flag, status, kSiteTcEmpty))
-          return false;
-        mbar_arrive_expect_tx(&bars->full[slot], kSlotBytes);
-        const uint32_t dst = ring_addr + slot * kSlotBytes;
-        const uint32_t bar = smem_u32(&bars->full[slot]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) ptx::tma_load_2d(dst + i * kBoxBytes, map, 64 * i, kt * kKeyTile, bar);
-        ++e;
-        return true;
-      };
       for (int t = 0; t < n && ok; ++t) {
-        ok = issue(&tmk, it.kt_begin + t);
-        if (ok && t >= 1) ok = issue(&tmv, it.kt_begin + t - 1);
+        for (int c = 0; c < per_tile; ++c) {
+          const int slot = e % ring;
+          if (e >= ring &&
+              !mbar_wait(&empty[slot], ((e / ring) - 1) & 1, abort_flag, status, kSiteTcEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t bar = smem_u32(&full[slot]);
+          const int32_t key0 = (it.kt_begin + t) * kKeyTile;
+          if (is_k) {
+            mbar_arrive_expect_tx(&full[slot], kKSlotBytes);
+            const uint32_t dst = sbase + kOffK + slot * kKSlotBytes;
+            ptx::tma_load_2d(dst, &tmk, 128 * c, key0, bar);
+            ptx::tma_load_2d(dst + kKChunkBytes, &tmk, 128 * c + 64, key0, bar);
+          } else {
+            mbar_arrive_expect_tx(&full[slot], kVHalfBytes);
+            const uint32_t dst = sbase + kOffV + slot * kVHalfBytes;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ptx::tma_load_2d(dst + i * kVBoxBytes, &tmv, 64 * i, key0 + 64 * c, bar);
+          }
+          ++e;
+        }
       }
-      if (ok) ok = issue(&tmv, it.kt_begin + n - 1);
       if (!ok) {  // aborted: let every issued copy land before the CTA exits
-        for (int s = 0; s < kRing && s < e; ++s) {
-          const int last = ((e - 1 - s) / kRing) * kRing + s;
-          mbar_wait(&bars->full[s], (last / kRing) & 1, nullptr, status, kSiteTcDrain);
+        for (int s = 0; s < ring && s < e; ++s) {
+          const int last = ((e - 1 - s) / ring) * ring + s;
+          mbar_wait(&full[s], (last / ring) & 1, nullptr, status, kSiteTcDrain);
         }
       }
     }
@@ -153,48 +198,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t ab = DT == KCA_BF16 ? 1u : 0u;
       constexpr uint32_t id_qk = ptx::idesc_f16(ab, 128, kKeyTile, 0);
       constexpr uint32_t id_pv = ptx::idesc_f16(ab, 128, kDim, 1);
-      int e = 0;
+      // Descriptor bases; an operand at byte offset x from a base is the base
+      // plus x >> 4 in the start-address field (addresses stay below 256 KiB).
+      const uint64_t kd0 = ptx::sdesc_sw128(sbase + kOffK, 16, 1024);
+      const uint64_t pd0 = ptx::sdesc_sw128(sbase + kOffP, 16, 1024);
+      const uint64_t vd0 = ptx::sdesc_sw128(sbase + kOffV, kVBoxBytes, 1024);
+      int ek = 0, ev = 0;
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, status, kSiteTcQ);
       ptx::fence_after_sync();
       auto pv = [&](int u) -> bool {
-        const int b = u & 1;
-        if (!mbar_wait(&bars->p_full[b], (u >> 1) & 1, abort_flag, status, kSiteTcP)) return false;
+        if (!mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, abort_flag, status, kSiteTcP)) return false;
         ptx::fence_after_sync();
-        const int slot = e % kRing;
-        if (!mbar_wait(&bars->full[slot], (e / kRing) & 1, abort_flag, status, kSiteTcFull)) return false;
-        ptx::fence_after_sync();
-        const uint32_t vbase = ring_addr + slot * kSlotBytes;
-        const uint32_t pcol = b ? kColS1 : kColS0;
+        const uint64_t pd = pd0 + (uint64_t)(((u & 1) * kPBytes) >> 4);
+        for (int h = 0; h < 2; ++h) {
+          const int slot = ev % kVRing;
+          if (!mbar_wait(&bars->vfull[slot], (ev / kVRing) & 1, abort_flag, status, kSiteTcFull)) return false;
+          const uint64_t vd = vd0 + (uint64_t)((slot * kVHalfBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kKeyTile / 16; ++kk)
-          ptx::mma_ts(tmem + kColO, tmem + pcol + kk * 8,
-                      ptx::sdesc_sw128(vbase + kk * 16 * 128, kBoxBytes, 1024), id_pv,
-                      (u > 0 || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(smem_u32(&bars->empty[slot]));
-        ptx::mma_commit(smem_u32(&bars->o_done));
-        ++e;
+          for (int j = 0; j < 4; ++j)
+            ptx::mma_ss(tmem + kColO, pd + (uint64_t)((h * (kPBytes / 2) + j * 32) >> 4),
+                        vd + (uint64_t)((j * 16 * 128) >> 4), id_pv, (u > 0 || h > 0 || j > 0) ? 1u : 0u);
+          ptx::mma_commit(smem_u32(&bars->vempty[slot]));
+          ++ev;
+        }
+        ptx::mma_commit(smem_u32(&bars->o_done[u & 1]));
         return true;
       };
       for (int t = 0; t < n && ok; ++t) {
-        const int slot = e % kRing;
-        if (!mbar_wait(&bars->full[slot], (e / kRing) & 1, abort_flag, status, kSiteTcFull)) {
-          ok = false;
-          break;
+        if (t > 0) {
+          ok = mbar_wait(&bars->s_free, (t - 1) & 1, abort_flag, status, kSiteTcS);
+          if (!ok) break;
+          ptx::fence_after_sync();   // S was read by other threads' tcgen05.ld
         }
-        ptx::fence_after_sync();
-        const uint32_t kbase = ring_addr + slot * kSlotBytes;
-        const uint32_t scol = (t & 1) ? kColS1 : kColS0;
+        for (int c = 0; c < 2 && ok; ++c) {
+          const int slot = ek % kKRing;
+          ok = mbar_wait(&bars->kfull[slot], (ek / kKRing) & 1, abort_flag, status, kSiteTcFull);
+          if (!ok) break;
+          const uint64_t kd = kd0 + (uint64_t)((slot * kKSlotBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kDim / 16; ++kk)
-          ptx::mma_ts(tmem + scol, tmem + kColQ + kk * 8,
-                      ptx::sdesc_sw128(kbase + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024),
-                      id_qk, kk > 0 ? 1u : 0u);
-        ptx::mma_commit(smem_u32(&bars->empty[slot]));
-        ptx::mma_commit(smem_u32(&bars->s_full[t & 1]));
-        ++e;
-        if (t >= 1) ok = pv(t - 1);
+          for (int j = 0; j < 8; ++j)   // K-steps 8c .. 8c+7: chunk j/4 of the slot
+            ptx::mma_ts(tmem + kColS, tmem + kColQ + (8 * c + j) * 8,
+                        kd + (uint64_t)(((j >> 2) * kKChunkBytes + (j & 3) * 32) >> 4), id_qk,
+                        (c > 0 || j > 0) ? 1u : 0u);
+          ptx::mma_commit(smem_u32(&bars->kempty[slot]));
+          ++ek;
+        }
+        if (!ok) break;
+        ptx::mma_commit(smem_u32(&bars->s_full));
+        if (t > 0) ok = pv(t - 1);
       }
       if (ok) ok = pv(n - 1);
+      if (ok) ptx::mma_commit(smem_u32(&bars->o_final));
       // every MMA issued above has completed once this barrier flips
       ptx::mma_commit(smem_u32(&bars->drain));
       mbar_wait(&bars->drain, 0, nullptr, status, kSiteTcDrain);
@@ -202,44 +256,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax
-    const int m = threadIdx.x - 128;                 // TMEM lane == M row
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t trow = tmem + lane_base;
+    const int wg = (warp - 4) >> 2;                  // key half of every S tile
+    const int m = (warp & 3) * 32 + lane;            // TMEM lane == M row
+    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int64_t row = (int64_t)it.tile * kRowTile + (m >> 3);
     const bool valid = row < a.plan.rows;
     const int64_t pos = a.plan.chunk_start + row;
     const int64_t lo = lo_of(pos, a.plan.window);
 
-    // Q row (row, head m & 7) into TMEM columns [0, 128), zeros past the chunk.
+    // Q row (row, head m & 7), dims [128 wg, 128 wg + 128), into TMEM; zeros past the chunk.
     {
-      const uint4* qsrc = reinterpret_cast<const uint4*>(a.q) + ((int64_t)it.tile * 128 + m) * 32;
+      const uint4* qsrc = reinterpret_cast<const uint4*>(a.q) + ((int64_t)it.tile * 128 + m) * 32 + wg * 16;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint4 v = valid ? qsrc[c * 8 + i] : make_uint4(0, 0, 0, 0);
           r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
         }
-        ptx::tmem_st32(trow + kColQ + c * 32, r);
+        ptx::tmem_st32(trow + kColQ + 64 * wg + 32 * c, r);
       }
       ptx::tmem_wait_st();
       ptx::fence_before_sync();
       mbar_arrive(&bars->q_full);
     }
 
-    float m_ref = -INFINITY;   // reference max, log2 units
-    float l_sum = 0.f;
     const float cs = a.scale_log2;
+    const uint32_t scol = kColS + 64 * wg;
+    float m_ref = -INFINITY;  // reference max of the row, log2 units
+    float l_sum = 0.f;        // this warpgroup's half of the row sum
     bool ok = true;
     for (int t = 0; t < n; ++t) {
-      const int b = t & 1;
-      const uint32_t scol = b ? kColS1 : kColS0;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort_flag, status, kSiteTcS));
-      if (!ok) break;
-      ptx::fence_after_sync();
+      // Every thread runs every iteration (work is skipped after an abort) so
+      // that both warpgroups always meet at the named barrier below.
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->s_full, t & 1, abort_flag, status, kSiteTcS));
       float s[64];
-      {
+      if (ok) {
+        ptx::fence_after_sync();
         uint32_t r0[32], r1[32];
         ptx::tmem_ld32(trow + scol, r0);
         ptx::tmem_ld32(trow + scol + 32, r1);
@@ -250,35 +304,61 @@ __global__ void __launch_bounds__(kThreads, 1)
           s[32 + c] = __uint_as_float(r1[c]);
         }
       }
-      // Raw scores of keys outside [lo, pos] become -inf (the scale is > 0,
-      // so they stay -inf below and their probability is exactly 0).
-      const int64_t j0 = a.plan.kv_lo + (int64_t)(it.kt_begin + t) * kKeyTile;
-      if (j0 < lo || j0 + kKeyTile - 1 > pos) {
+      ptx::fence_before_sync();
+      mbar_arrive(&bars->s_free);   // S may be overwritten by the next QK^T
+      float mloc = -INFINITY;
+      if (ok) {
+        // keys outside [lo, pos] become -inf (scale > 0 keeps them there)
+        const int64_t j0 = a.plan.kv_lo + (int64_t)(it.kt_begin + t) * kKeyTile + 64 * wg;
+        if (j0 < lo || j0 + 63 > pos) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int64_t j = j0 + c;
-          if (j < lo || j > pos) s[c] = -INFINITY;
+          for (int c = 0; c < 64; ++c) {
+            const int64_t j = j0 + c;
+            if (j < lo || j > pos) s[c] = -INFINITY;
+          }
         }
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) m8[c & 7] = max_nan(m8[c & 7], s[c]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m8[i] = max_nan(m8[i], m8[i + 4]);
+        mloc = max_nan(max_nan(m8[0], m8[2]), max_nan(m8[1], m8[3]));
       }
-      // NaN-preserving row max over eight independent chains.
-      float m8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-      for (int c = 8; c < 64; ++c) m8[c & 7] = max_nan(m8[c & 7], s[c]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) m8[i] = max_nan(m8[i], m8[i + 4]);
-      const float mraw = max_nan(max_nan(m8[0], m8[2]), max_nan(m8[1], m8[3]));
+      // The row max spans both warpgroups: exchange halves (buffer by tile parity).
+      bars->red_max[t & 1][wg][m] = mloc;
+      named_sync(1, kSoftmaxThreads);
+      const float mraw = max_nan(mloc, bars->red_max[t & 1][wg ^ 1][m]);
+      if (!ok) continue;
       const float mx = mraw == -INFINITY ? -INFINITY : mraw * cs;
-      const bool need = mx > m_ref + kRescaleLog2;
+      const bool need = mx > m_ref + kRescaleLog2;   // identical in both warpgroups
       const bool any_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.f;
       if (any_need) {
-        alpha = need ? ptx::ex2(m_ref - mx) : 1.f;
+        const float alpha = need ? ptx::ex2(m_ref - mx) : 1.f;
         if (need) m_ref = mx;
         l_sum *= alpha;
+        if (t > 0) {
+          // PV of the previous tile must finish before O is rescaled; PV of
+          // tile t-2 is known complete here (it preceded this tile's QK^T),
+          // so the parity wait on barrier (t-1)&1 is unambiguous.
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1,
+                                                 abort_flag, status, kSiteTcO));
+          if (!ok) continue;
+          ptx::fence_after_sync();
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(trow + kColO + 128 * wg + 32 * c, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            ptx::tmem_st32(trow + kColO + 128 * wg + 32 * c, r);
+          }
+          ptx::tmem_wait_st();
+        }
       }
-      // p = 2^(s*scale*log2e - m_ref), one FFMA and one MUFU op per score.
+      // p = 2^(s*scale*log2e - m_ref): one FFMA and one MUFU op per score.
       const float nmu = m_ref == -INFINITY ? 0.f : -m_ref;
       uint32_t pr[32];
       float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -294,50 +374,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc2[2] = __fadd2_rn(acc2[2], acc2[3]);
       acc2[0] = __fadd2_rn(acc2[0], acc2[2]);
       l_sum += acc2[0].x + acc2[0].y;
-      ptx::tmem_st32(trow + scol, pr);
-      // PV of the previous tile must be complete before O is touched and
-      // before this thread lets PV of this tile start; waiting on every tile
-      // keeps this thread within one phase of the barrier, which parity
-      // waits require.
-      if (t > 0) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, status, kSiteTcO));
-        if (!ok) break;
-        ptx::fence_after_sync();
-        if (any_need) {
-#pragma unroll 1
-          for (int c = 0; c < kDim / 32; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(trow + kColO + c * 32, r);
-            ptx::tmem_wait_ld();
+      // P row m, keys [64 wg, 64 wg + 64): buffer t&1, K-major with 128-byte
+      // swizzle (16-byte unit j of row m at unit j ^ (m & 7)).
+      unsigned char* prow = smem + kOffP + (t & 1) * kPBytes + wg * (kPBytes / 2) + (m >> 3) * 1024 + (m & 7) * 128;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            ptx::tmem_st32(trow + kColO + c * 32, r);
-          }
-        }
-      }
-      ptx::tmem_wait_st();
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(prow + ((j ^ (m & 7)) << 4)) =
+            make_uint4(pr[4 * j], pr[4 * j + 1], pr[4 * j + 2], pr[4 * j + 3]);
+      fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor cores
       ptx::fence_before_sync();
-      mbar_arrive(&bars->p_full[b]);
+      mbar_arrive(&bars->p_full[t & 1]);
     }
-    if (ok)
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (n - 1) & 1, abort_flag, status, kSiteTcO));
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->o_final, 0, abort_flag, status, kSiteTcO));
+    // Row sum over both halves (the buffer of tile parity n&1 is free again).
+    bars->red_max[n & 1][wg][m] = l_sum;
+    named_sync(1, kSoftmaxThreads);
+    const float l_tot = l_sum + bars->red_max[n & 1][wg ^ 1][m];
     if (ok) {
       ptx::fence_after_sync();
-      const float inv = 1.f / l_sum;
       float* dst;
       if (it.slot < 0) {
-        dst = a.out + ((int64_t)it.tile * 128 + m) * kDim;
+        dst = a.out + ((int64_t)it.tile * 128 + m) * kDim + 128 * wg;
       } else {
-        dst = a.part_acc + ((int64_t)it.slot * 128 + m) * kDim;
-        a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 0] = m_ref;
-        a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 1] = l_sum;
+        dst = a.part_acc + ((int64_t)it.slot * 128 + m) * kDim + 128 * wg;
+        if (wg == 0) {
+          a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 0] = m_ref;
+          a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 1] = l_tot;
+        }
       }
-      const float f = it.slot < 0 ? inv : 1.f;
+      const float f = it.slot < 0 ? 1.f / l_tot : 1.f;
 #pragma unroll 1
-      for (int c = 0; c < kDim / 32; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        ptx::tmem_ld32(trow + kColO + c * 32, r);
+        ptx::tmem_ld32(trow + kColO + 128 * wg + 32 * c, r);
         ptx::tmem_wait_ld();
         if (valid) {
           float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
@@ -357,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
 }
+
 
 // Log-sum-exp merge of the items of each split row tile: a group of W warps
 // per M row, 8 / W rows per CTA, grid (tiles, 16 W).

@@ -37,7 +37,8 @@ struct TcArgs {
 void fill_tc_tables(TcArgs& a);
 
 // tmk / tmv: 2-D tensor maps over the rows [plan.kv_lo, plan.ctx_len) of the
-// K and V caches, inner extent 256, box 64 x 64, 128-byte swizzle, zero fill.
+// K and V caches, inner extent 256, 128-byte swizzle, zero fill; boxes of 64
+// elements x 128 rows (K) and 64 x 64 (V).
 cudaError_t launch_prefill_tc(int dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                               const TcArgs& a, cudaStream_t stream);
 

@@ -45,6 +45,7 @@ def test_status_strings():
 
 
 P = 0x10000  # a 16-byte aligned fake device address; validation fails before any use
+KEY_TILE = 128  # keys per tensor-core KV tile (kca_plan.h)
 
 
 def _prefill(**kw):
@@ -158,9 +159,9 @@ def test_prefill_tc_plan_covers_every_visible_key(cs, rows, window):
     for t in range(n_tiles):
         its = items[items[:, 0] == t]
         assert len(its) >= 1
-        # items of a tile are contiguous, 64-aligned relative to kv_lo, within [kv_lo, ctx)
+        # items of a tile are contiguous, tile-aligned relative to kv_lo, within [kv_lo, ctx)
         assert (its[1:, 1] == its[:-1, 2]).all()
-        assert ((its[:, 1] - kv_lo) % 64 == 0).all()
+        assert ((its[:, 1] - kv_lo) % KEY_TILE == 0).all()
         assert its[0, 1] >= kv_lo and its[-1, 2] <= ctx
         covered = (int(its[0, 1]), int(its[-1, 2]))
         for r in range(16 * t, min(16 * t + 16, rows)):
@@ -168,7 +169,7 @@ def test_prefill_tc_plan_covers_every_visible_key(cs, rows, window):
             assert covered[0] <= lo and hi < covered[1]
         # the first item starts in the key tile of the tile's first row's lo
         lo0 = oracle.visible_range(cs + 16 * t, window)[0]
-        assert covered[0] == kv_lo + (lo0 - kv_lo) // 64 * 64
+        assert covered[0] == kv_lo + (lo0 - kv_lo) // KEY_TILE * KEY_TILE
         assert (len(its) == 1) == (its[0, 3] == -1)
 
 
