@@ -51,10 +51,14 @@
  * default stream) of the current device.
  *
  * WORKSPACE: scratch device memory of at least attn_*_workspace_bytes()
- * bytes for the same arguments on the same device.  Its first 256 bytes hold
- * a device status word: zero them once after allocation (attn_workspace_init)
- * and read them with attn_device_status.  Calls that run concurrently must not
- * share a workspace or an output buffer.
+ * bytes for the same arguments on the same device.  Its first
+ * KCA_WORKSPACE_HEADER bytes are the header: a device status word in bytes
+ * [0, 256) (read it with attn_device_status) and, in the rest, one counter
+ * per (row, head) that the tensor-core rows kernel uses to elect the CTA that
+ * merges a row's partials; every call leaves them at zero again.  Zero the
+ * header once after allocation (attn_workspace_init), and again after a call
+ * that recorded a device error.  Calls that run concurrently must not share a
+ * workspace or an output buffer.
  *
  * ERRORS: every entry point validates all of its arguments on the host before
  * touching the GPU and returns a negative KCA_ERR_* without launching
@@ -96,7 +100,8 @@ extern "C" {
 #define KCA_MAX_CHUNK_ROWS 768
 #define KCA_MAX_POSITION 131072
 #define KCA_MAX_BATCH 256
-#define KCA_WORKSPACE_HEADER 256
+/* status word (256 B) + 768 rows x 8 heads x 4-byte counters */
+#define KCA_WORKSPACE_HEADER 24832
 
 /*
  * attn_prefill -- chunked causal prefill of one sequence.
@@ -167,7 +172,7 @@ size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t c
                                     int32_t chunk_rows, int32_t window);
 size_t attn_decode_workspace_bytes(int32_t batch, const int64_t *ctx_len, int32_t window);
 
-/* Zero the workspace's status header (cudaMemsetAsync on `stream`). */
+/* Zero the workspace header (cudaMemsetAsync on `stream`). */
 int attn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /*

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libkca.so")
 F32, F16, BF16 = 0, 1, 2
 N_Q_HEADS, N_KV_HEADS, HEAD_DIM = 8, 1, 256
 MAX_CHUNK_ROWS, MAX_POSITION, MAX_BATCH = 768, 131072, 256
-WORKSPACE_HEADER = 256
+WORKSPACE_HEADER = 24832  # status word + per-(row, head) merge counters
 STATUS = {0: "KCA_OK", -1: "KCA_ERR_NULL", -2: "KCA_ERR_GEOMETRY", -3: "KCA_ERR_DTYPE",
           -4: "KCA_ERR_RANGE", -5: "KCA_ERR_WORKSPACE", -6: "KCA_ERR_ALIGN", -7: "KCA_ERR_CUDA",
           -8: "KCA_ERR_DEVICE"}

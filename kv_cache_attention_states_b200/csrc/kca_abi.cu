@@ -23,6 +23,9 @@ using kca::kHeads;
 
 constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+constexpr size_t kStatusBytes = 256;   // header: status word, then the merge counters
+static_assert(KCA_WORKSPACE_HEADER >= kStatusBytes + KCA_MAX_CHUNK_ROWS * kHeads * 4, "header");
+static_assert(KCA_MAX_BATCH <= KCA_MAX_CHUNK_ROWS, "header counters cover both paths");
 
 bool dtype_ok(int32_t d) { return d == KCA_F32 || d == KCA_F16 || d == KCA_BF16; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -139,6 +142,113 @@ void carve(void* ws, size_t ml_bytes, float** ml, float** acc) {
   *acc = reinterpret_cast<float*>(p + align_up(ml_bytes));
 }
 
+// 16-bit caches take the tensor-core rows kernel; "simt" in KCA_DECODE_PATH
+// forces the CUDA-core one (tests compare the two on the same inputs).
+bool use_rows_mma(int32_t kv_dtype) {
+  if (kv_dtype != KCA_F16 && kv_dtype != KCA_BF16) return false;
+  const char* env = std::getenv("KCA_DECODE_PATH");
+  return !(env != nullptr && std::strcmp(env, "simt") == 0);
+}
+
+// Plan of the tensor-core rows kernel.  Each cluster size c in {8, 4, 2}
+// (and c = 1 when every unit fits one split, so nothing is merged) gets the
+// plan that fills the clusters resident at once; the one with the lowest
+// estimated time wins.  The estimate, from decode sweeps on B200: the key
+// stream takes the longer of all bytes at 6.5 TB/s and one split at 50 GB/s
+// per SM, times the waves of clusters; a unit with several clusters adds
+// 1.5 us (partials, fence, ticket) and 0.6 us per round of loads of the
+// final merge.
+kca::RowsPlan mma_rows_plan(int32_t n_units, const int64_t* nkeys, int sms, int* cluster) {
+  kca::RowsPlan best{};
+  int best_c = 0;
+  double best_t = 0.0;
+  double total_keys = 0.0;
+  for (int32_t u = 0; u < n_units; ++u) total_keys += (double)nkeys[u];
+  int cmax = 8;   // KCA_DECODE_CLUSTER_MAX caps the cluster size (sweeps compare them)
+  if (const char* env = std::getenv("KCA_DECODE_CLUSTER_MAX")) cmax = std::atoi(env);
+  for (int c = 8; c >= 1; c /= 2) {
+    if (c > cmax && c > 1) continue;
+    int slots = c == 1 ? sms : kca::decode_mma_cluster_capacity(c);
+    if (slots > kca::kRowsMmaMaxClusterParts) slots = kca::kRowsMmaMaxClusterParts;
+    if (slots <= 0) continue;
+    const kca::RowsPlan p = kca::make_cluster_rows_plan(n_units, nkeys, c, slots);
+    const int max_clusters = (p.max_splits + c - 1) / c;
+    if (c == 1 && max_clusters > 1) continue;   // one CTA would merge all eight heads
+    int64_t n_clusters = 0;
+    for (int32_t u = 0; u < n_units; ++u) n_clusters += (kca::rows_n_splits(nkeys[u], p.split_len) + c - 1) / c;
+    const double waves = (double)((n_clusters + slots - 1) / slots);
+    const double t_hbm = total_keys * 1024.0 / 6.5e12;
+    const double t_sm = waves * (double)p.split_len * 1024.0 / 50e9;
+    double t = t_hbm > t_sm ? t_hbm : t_sm;
+    if (max_clusters > 1) t += 1.5e-6 + 0.6e-6 * (1 + (kHeads / c) * ((max_clusters + 31) / 32));
+    if (best_c == 0 || t < best_t) {
+      best = p;
+      best_c = c;
+      best_t = t;
+    }
+  }
+  *cluster = best_c;
+  return best;
+}
+
+size_t mma_ws_bytes(const kca::RowsPlan& p, int cluster) {
+  const int max_clusters = (p.max_splits + cluster - 1) / cluster;
+  if (max_clusters <= 1) return KCA_WORKSPACE_HEADER;
+  const size_t slots = (size_t)p.n_units * max_clusters;
+  return KCA_WORKSPACE_HEADER + align_up(slots * kHeads * 2 * 4) + align_up(slots * kHeads * kDim * 4);
+}
+
+// Workspace of the rows path: enough for either rows kernel, so that the
+// query functions (which do not know the path a call will take) and the
+// check at call time agree.  *mma_plan / *cluster: the tensor-core plan.
+size_t rows_ws_bytes_any(int32_t n_units, const int64_t* nkeys, int sms, kca::RowsPlan* mma_plan,
+                         int* cluster) {
+  const size_t simt = rows_ws_bytes(kca::make_rows_plan(n_units, nkeys, sms));
+  *mma_plan = mma_rows_plan(n_units, nkeys, sms, cluster);
+  if (*cluster < 1) return simt;
+  const size_t mma = mma_ws_bytes(*mma_plan, *cluster);
+  return simt > mma ? simt : mma;
+}
+size_t rows_ws_bytes_any(int32_t n_units, const int64_t* nkeys, int sms) {
+  kca::RowsPlan p;
+  int c = 0;
+  return rows_ws_bytes_any(n_units, nkeys, sms, &p, &c);
+}
+
+// Plan of the rows path for this cache dtype (cluster 0: no usable plan),
+// with the workspace a call needs.
+kca::RowsPlan rows_plan(int32_t kv_dtype, int32_t n_units, const int64_t* nkeys, int sms, int* cluster,
+                        size_t* ws_bytes) {
+  kca::RowsPlan mma;
+  *ws_bytes = rows_ws_bytes_any(n_units, nkeys, sms, &mma, cluster);
+  if (use_rows_mma(kv_dtype)) return mma;
+  *cluster = 1;
+  return kca::make_rows_plan(n_units, nkeys, sms);
+}
+
+// Launches the rows path: tensor cores for 16-bit caches (tensor maps over the
+// cache_rows rows of the cache), CUDA cores otherwise.
+int launch_rows_path(int32_t q_dtype, int32_t kv_dtype, const void* k_cache, const void* v_cache,
+                     int64_t cache_rows, kca::RowsArgs a, int cluster, void* workspace, cudaStream_t s) {
+  if (use_rows_mma(kv_dtype)) {
+    a.cluster = cluster;
+    a.max_clusters = (a.max_splits + cluster - 1) / cluster;
+    if (a.max_clusters > 1) {
+      // Counters live in the header (no other path writes there), cluster
+      // partials where the CUDA-core path keeps its split partials.
+      a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+      carve(workspace, (size_t)a.n_units * a.max_clusters * kHeads * 2 * 4, &a.cpart_ml, &a.cpart_acc);
+    }
+    CUtensorMap tmk, tmv;
+    if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, cache_rows, 64) ||
+        !encode_kv_map(&tmv, v_cache, kv_dtype, 0, cache_rows, 64))
+      return KCA_ERR_CUDA;
+    return kca::launch_decode_mma(q_dtype, kv_dtype, tmk, tmv, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+  }
+  carve(workspace, (size_t)a.n_units * a.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
+  return kca::launch_rows(q_dtype, kv_dtype, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -242,7 +352,7 @@ size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t c
   if (use_tc(q_dtype, kv_dtype, chunk_rows))
     return tc_ws_bytes(kca::make_tc_plan(chunk_start, chunk_rows, window, sms));
   const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
-  return rows_ws_bytes(kca::make_rows_plan(chunk_rows, nk.data(), sms));
+  return rows_ws_bytes_any(chunk_rows, nk.data(), sms);
 }
 
 size_t attn_decode_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_t window) {
@@ -250,7 +360,7 @@ size_t attn_decode_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return 0;
   const std::vector<int64_t> nk = decode_unit_keys(batch, ctx_len, window);
-  return rows_ws_bytes(kca::make_rows_plan(batch, nk.data(), sms));
+  return rows_ws_bytes_any(batch, nk.data(), sms);
 }
 
 int attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
@@ -316,8 +426,11 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
   }
 
   const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
-  const kca::RowsPlan p = kca::make_rows_plan(chunk_rows, nk.data(), sms);
-  if (workspace_bytes < rows_ws_bytes(p)) return KCA_ERR_WORKSPACE;
+  int cluster = 1;
+  size_t need = 0;
+  const kca::RowsPlan p = rows_plan(kv_dtype, chunk_rows, nk.data(), sms, &cluster, &need);
+  if (cluster < 1) return KCA_ERR_CUDA;
+  if (workspace_bytes < need) return KCA_ERR_WORKSPACE;
   kca::RowsArgs a{};
   a.q = q_chunk;
   a.k = k_cache;
@@ -332,8 +445,7 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
   a.max_splits = p.max_splits;
   a.window = window;
   a.scale = scale;
-  carve(workspace, (size_t)p.n_units * p.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
-  return kca::launch_rows(q_dtype, kv_dtype, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+  return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, capacity, a, cluster, workspace, s);
 }
 
 int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache,
@@ -353,8 +465,11 @@ int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void*
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
   const std::vector<int64_t> nk = decode_unit_keys(batch, ctx_len, window);
-  const kca::RowsPlan p = kca::make_rows_plan(batch, nk.data(), sms);
-  if (workspace_bytes < rows_ws_bytes(p)) return KCA_ERR_WORKSPACE;
+  int cluster = 1;
+  size_t need = 0;
+  const kca::RowsPlan p = rows_plan(kv_dtype, batch, nk.data(), sms, &cluster, &need);
+  if (cluster < 1) return KCA_ERR_CUDA;
+  if (workspace_bytes < need) return KCA_ERR_WORKSPACE;
   kca::RowsArgs a{};
   a.q = q;
   a.k = k_cache;
@@ -370,10 +485,8 @@ int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void*
   a.window = window;
   a.scale = scale;
   for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
-  carve(workspace, (size_t)p.n_units * p.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
-  return kca::launch_rows(q_dtype, kv_dtype, a, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? KCA_OK
-             : KCA_ERR_CUDA;
+  return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster,
+                          workspace, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -1,0 +1,596 @@
+// kca_decode_mma.cu -- split-context single-row attention with 16-bit K/V on
+// the tensor cores (mma.sync m16n8k16, f32 accumulation): decode, and the
+// prefill rows that the tcgen05 kernel does not take.
+//
+// With 8 query heads sharing one KV head a decode step is a small GEMM per
+// key block (M = 8 heads), not a GEMV.  On the CUDA cores the eight dot
+// products, their warp-shuffle reductions and the f16 -> f32 conversions
+// cost ~130 instructions per key row per warp; here a 64-key stage costs ~80
+// instructions per warp, so the kernel is left with the HBM stream it is
+// meant to be bound by.  Prior art on the pages: the "parallel" QK and PV
+// reductions of Karume's one-row plans (v0.12.0 release notes,
+// "Performance", items 2-3).
+//
+// Precision: the query (any dtype) is split into a 16-bit high part and a
+// 16-bit remainder, stacked as rows 0-7 and 8-15 of the A operand, so the
+// accumulator rows g and g+8 hold q_hi.k and q_lo.k for head g and their sum
+// carries ~16 (bf16) to ~22 (f16) bits of the query.  P is split the same way
+// for the PV product.  Accumulation is f32.
+//
+// One CTA = one split of one unit; warps 0-7 compute, warp 8 issues the TMA
+// loads.  The splits of a unit run as clusters of 2, 4 or 8 CTAs that merge
+// their partials through distributed shared memory at the end; when a unit
+// has several clusters, the CTA that finishes last (atomic ticket, no
+// waiting) merges the cluster partials, so no separate merge kernel runs.
+// The launch allows programmatic dependent launch: the prologue overlaps the
+// previous kernel of the stream.
+//
+// A stage is 64 keys: K and V each as four 64-dim boxes of 64 rows with
+// 128-byte swizzle (conflict-free ldmatrix), 64 KiB per stage, 3 stages.
+// Stage flow (warp w): S for keys 8w..8w+7 (16 MMAs over d = 256), stage max
+// per head exchanged through shared memory, lazy rescale of O, P written to
+// shared memory as 16 rows (hi, lo) x 64 keys, then O[:, 32w .. 32w+31] +=
+// P V (16 MMAs).  Rows past the split's end are zeroed in shared memory, so
+// whatever the cache holds there never reaches the output.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "kca_common.cuh"
+#include "kca_plan.h"
+#include "kca_rows.h"
+
+namespace kca {
+namespace {
+
+constexpr int kDWarps = 8;
+constexpr int kDThreads = (kDWarps + 1) * 32;
+constexpr int kDStageKeys = 64;
+constexpr int kDStages = 3;
+constexpr int kDBoxBytes = 64 * 64 * 2;              // 64 rows x 64 dims, 8 KiB
+constexpr int kDHalfBytes = 4 * kDBoxBytes;          // K or V of one stage: 32 KiB
+constexpr int kDStageBytes = 2 * kDHalfBytes;        // 64 KiB
+constexpr int kDPRow = 144;                          // P row pitch: 128 B + 16 B pad
+constexpr int kDOffBar = kDStages * kDStageBytes;    // 192 KiB
+constexpr float kDLog2e = 1.4426950408889634f;
+constexpr float kDRescale = 5.545177444479562f;      // 8 ln 2
+constexpr int kDMaxClusterParts = kRowsMmaMaxClusterParts;  // cluster partials a unit may have
+
+struct DBars {
+  uint64_t full[kDStages];
+  uint64_t empty[kDStages];
+  int abort;
+  float red[kDWarps][8];                 // per-warp stage max (then row sums) per head
+  int last;                              // this CTA holds the last ticket of its unit
+  __align__(16) unsigned char p[16 * kDPRow];   // P: rows 0-7 hi, 8-15 lo, 64 keys
+  // Partial of this CTA for the cluster merge: reference max (natural units),
+  // row sum and unnormalised output per head.  Own space, not a stage buffer,
+  // so no copy still landing after an abort can overwrite it.
+  float pm[8];
+  float pl[8];
+  float po[8 * 256];
+  float fsc[kHeads][kDMaxClusterParts];  // merge weight of each cluster partial
+  float mred[kHeads][kDWarps];           // block reductions of the merge
+  float lred[kHeads][kDWarps];
+};
+constexpr int kDSmemBytes = kDOffBar + (int)sizeof(DBars) + 1024;
+
+template <int KT>
+__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
+  if (KT == KCA_BF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+template <int KT>
+__device__ __forceinline__ float2 unpack16(uint32_t u) {
+  if (KT == KCA_BF16) return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+  return __half22float2(*reinterpret_cast<__half2*>(&u));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// D = A(16x16) B(16x8) + D, row.col, f32 accumulation.
+template <int KT>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  if (KT == KCA_BF16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+__device__ __forceinline__ void tma2d(uint32_t dst, const void* map, int32_t x, int32_t y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// Byte offset of (row, dim) inside a stage half: four 64-dim boxes of 64 rows,
+// 128-byte swizzle (16-byte unit u of row r stored at unit u ^ (r & 7)).
+__device__ __forceinline__ uint32_t swz(int row, int dim) {
+  const int unit = (dim & 63) >> 3;
+  return (uint32_t)((dim >> 6) * kDBoxBytes + row * 128 + ((unit ^ (row & 7)) << 4));
+}
+
+
+template <int QT>
+__device__ __forceinline__ float load_elem(const void* base, int64_t idx) {
+  if (QT == KCA_F32) return static_cast<const float*>(base)[idx];
+  if (QT == KCA_F16) return __half2float(static_cast<const __half*>(base)[idx]);
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[idx]);
+}
+
+// Cluster-wide barrier (all threads of every CTA of the cluster).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Generic address of the same shared-memory object in CTA `cta` of the
+// cluster; plain loads through it read that CTA's shared memory.
+template <typename T>
+__device__ __forceinline__ const T* cluster_peer(const T* local, uint32_t cta) {
+  uint64_t remote;
+  asm("mapa.u64 %0, %1, %2;" : "=l"(remote) : "l"(reinterpret_cast<uint64_t>(local)), "r"(cta));
+  return reinterpret_cast<const T*>(remote);
+}
+
+template <int QT, int KT>
+__global__ void __launch_bounds__(kDThreads, 1)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                      const RowsArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  unsigned char* smem = smem_raw + pad;
+  const uint32_t sbase = raw_addr + pad;
+  DBars* bars = reinterpret_cast<DBars*>(smem + kDOffBar);
+  volatile int* abort_flag = &bars->abort;
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.status);
+
+  const int C = a.cluster;                 // CTAs per cluster along the splits (1, 2, 4 or 8)
+  const int unit = blockIdx.y;
+  const int split = blockIdx.x;
+  const int rank = split % C, clus = split / C;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t pos = a.mode == 0 ? a.ctx[unit] - 1 : a.chunk_start + unit;
+  const int64_t lo = lo_of(pos, a.window);
+  const int64_t nkeys = n_visible(pos, a.window);
+  const int32_t nsplit = rows_n_splits(nkeys, a.split_len);
+  const int nclus = (nsplit + C - 1) / C;
+  if (clus >= nclus) return;               // the whole cluster leaves together
+  const bool active = split < nsplit && nkeys > 0;
+  const int64_t kbeg = lo + (int64_t)split * a.split_len;
+  int64_t kend = kbeg + a.split_len;
+  if (kend > pos + 1) kend = pos + 1;
+  const int64_t base_row = a.mode == 0 ? (int64_t)unit * a.seq_rows : 0;
+  const int n_stage = active ? (int)cdiv(kend - kbeg, kDStageKeys) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], kDWarps);
+    }
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Everything above overlaps the previous kernel of the stream (programmatic
+  // dependent launch); inputs, outputs and workspace are touched only below.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  float* pm = bars->pm;
+  float* pl = bars->pl;
+  float* po = bars->po;
+
+  if (warp == kDWarps) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && active) {
+      int issued = 0;
+      for (int i = 0; i < n_stage; ++i) {
+        const int slot = i % kDStages;
+        if (i >= kDStages &&
+            !mbar_wait(&bars->empty[slot], ((i / kDStages) - 1) & 1, abort_flag, status, kSiteRowsEmpty))
+          break;
+        const uint32_t kst = sbase + slot * kDStageBytes;
+        const uint32_t bar = smem_u32(&bars->full[slot]);
+        const int32_t row0 = (int32_t)(base_row + kbeg + (int64_t)i * kDStageKeys);
+        mbar_arrive_expect_tx(&bars->full[slot], kDStageBytes);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tma2d(kst + c * kDBoxBytes, &tmk, 64 * c, row0, bar);
+          tma2d(kst + kDHalfBytes + c * kDBoxBytes, &tmv, 64 * c, row0, bar);
+        }
+        issued = i + 1;
+      }
+      if (issued < n_stage) {  // aborted: let every issued copy land
+        for (int s = 0; s < kDStages && s < issued; ++s) {
+          const int last = ((issued - 1 - s) / kDStages) * kDStages + s;
+          mbar_wait(&bars->full[s], (last / kDStages) & 1, nullptr, status, kSiteRowsFull);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (!active) {
+    // no key in this split (or in the whole row): an empty partial
+    if (threadIdx.x < 8) {
+      pm[threadIdx.x] = -INFINITY;
+      pl[threadIdx.x] = 0.f;
+    }
+    for (int i = threadIdx.x; i < kHeads * kDim; i += kDWarps * 32) po[i] = 0.f;
+  } else {
+    // ------------------------------------------------------------------ compute
+    const int g = lane >> 2, tig = lane & 3;
+    // A operand of S = Q K^T: rows 0-7 the 16-bit high parts of the 8 heads,
+    // rows 8-15 the remainders; per k-step: (g, 2tig), (g+8, 2tig), (g, 2tig+8), (g+8, 2tig+8).
+    uint32_t qa[16][4];
+    {
+      const void* q = static_cast<const char*>(a.q) + (int64_t)unit * kHeads * kDim * ElemBytes<QT>::value;
+  #pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+  #pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int d = 16 * ks + 8 * half + 2 * tig;
+          const float x0 = load_elem<QT>(q, g * kDim + d);
+          const float x1 = load_elem<QT>(q, g * kDim + d + 1);
+          const uint32_t hi = pack16<KT>(x0, x1);
+          const float2 f = unpack16<KT>(hi);
+          qa[ks][2 * half] = hi;
+          qa[ks][2 * half + 1] = pack16<KT>(x0 - f.x, x1 - f.y);
+        }
+      }
+    }
+    float o[4][4];
+  #pragma unroll
+    for (int i = 0; i < 4; ++i)
+  #pragma unroll
+      for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
+    float m_ref = -INFINITY;  // reference max of head g (natural units)
+    float l_part = 0.f;
+    const float scale = a.scale;
+    const uint32_t pbase = smem_u32(bars->p);
+    bool ok = true;
+
+    for (int i = 0; i < n_stage; ++i) {
+      const int slot = i % kDStages;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->full[slot], (i / kDStages) & 1, abort_flag,
+                                                   status, kSiteRowsFull));
+      const int64_t k0 = kbeg + (int64_t)i * kDStageKeys;
+      const int cnt = (int)((kend - k0) < kDStageKeys ? (kend - k0) : kDStageKeys);
+      const uint32_t kst = sbase + slot * kDStageBytes;
+      const uint32_t vst = kst + kDHalfBytes;
+      float sx0 = -INFINITY, sx1 = -INFINITY;
+      if (ok) {
+        if (cnt < kDStageKeys) {  // V rows past the split's end -> 0
+          unsigned char* vrows = smem + slot * kDStageBytes + kDHalfBytes;
+          for (int idx = threadIdx.x; idx < (kDStageKeys - cnt) * 32; idx += kDWarps * 32) {
+            const int row = cnt + (idx >> 5), u = idx & 31;
+            *reinterpret_cast<uint4*>(vrows + (u >> 3) * kDBoxBytes + row * 128 + (u & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+        }
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int kr = 8 * warp + (lane & 7);
+  #pragma unroll
+        for (int ks2 = 0; ks2 < 8; ++ks2) {
+          uint32_t b[4];
+          ldsm_x4(kst + swz(kr, 32 * ks2 + 8 * (lane >> 3)), b);
+          mma16816<KT>(sacc, qa[2 * ks2], b[0], b[1]);
+          mma16816<KT>(sacc, qa[2 * ks2 + 1], b[2], b[3]);
+        }
+        const int kk0 = 8 * warp + 2 * tig;
+        sx0 = kk0 < cnt ? (sacc[0] + sacc[2]) * scale : -INFINITY;
+        sx1 = kk0 + 1 < cnt ? (sacc[1] + sacc[3]) * scale : -INFINITY;
+      }
+      float mw = max_nan(sx0, sx1);
+      mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 1));
+      mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 2));
+      if (tig == 0) bars->red[warp][g] = mw;
+      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+      float ms = bars->red[0][g];
+  #pragma unroll
+      for (int w = 1; w < kDWarps; ++w) ms = max_nan(ms, bars->red[w][g]);
+      if (ok) {
+        if (ms > m_ref + kDRescale) {  // lazy rescale: rows g and g+8 are both head g
+          const float alpha = exp2f((m_ref - ms) * kDLog2e);
+          m_ref = ms;
+          l_part *= alpha;
+  #pragma unroll
+          for (int nt = 0; nt < 4; ++nt)
+  #pragma unroll
+            for (int j = 0; j < 4; ++j) o[nt][j] *= alpha;
+        }
+        const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+        const float p0 = exp2f((sx0 - mu) * kDLog2e);
+        const float p1 = exp2f((sx1 - mu) * kDLog2e);
+        l_part += p0 + p1;
+        const uint32_t hi = pack16<KT>(p0, p1);
+        const float2 f = unpack16<KT>(hi);
+        const uint32_t lo16 = pack16<KT>(p0 - f.x, p1 - f.y);
+        const int key = 8 * warp + 2 * tig;
+        *reinterpret_cast<uint32_t*>(bars->p + g * kDPRow + key * 2) = hi;
+        *reinterpret_cast<uint32_t*>(bars->p + (g + 8) * kDPRow + key * 2) = lo16;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");   // P and zeroed rows visible
+      if (ok) {
+        const int mi = lane >> 3;
+  #pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t af[4];
+          ldsm_x4(pbase + (8 * (mi & 1) + (lane & 7)) * kDPRow + (16 * kk + 8 * (mi >> 1)) * 2, af);
+          const int key = 16 * kk + 8 * (mi & 1) + (lane & 7);
+  #pragma unroll
+          for (int pair = 0; pair < 2; ++pair) {
+            uint32_t vb[4];
+            ldsm_x4_t(vst + swz(key, 32 * warp + 16 * pair + 8 * (mi >> 1)), vb);
+            mma16816<KT>(o[2 * pair], af, vb[0], vb[1]);
+            mma16816<KT>(o[2 * pair + 1], af, vb[2], vb[3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->empty[slot]);
+    }
+
+    // Row sums: lanes of one head, then warps (the stage-max slots are free again).
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
+    if (tig == 0) bars->red[warp][g] = l_part;
+    asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDWarps; ++w) L += bars->red[w][g];
+    if (!ok || *abort_flag) {
+      m_ref = NAN;   // an aborted split poisons its row; the status word says why
+      L = NAN;
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int d = 32 * warp + 8 * nt + 2 * tig;
+      po[g * kDim + d] = o[nt][0] + o[nt][2];
+      po[g * kDim + d + 1] = o[nt][1] + o[nt][3];
+    }
+    if (warp == 0 && tig == 0) {
+      pm[g] = m_ref;
+      pl[g] = L;
+    }
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // ------------------------------------------------------------ merge
+  // CTA rank r owns heads r, r+C, ... (C divides 8).  Step 1 merges the C
+  // partials of its cluster through distributed shared memory; thread d owns
+  // dim d.  With one cluster per unit that is the result.  Otherwise each CTA
+  // publishes its heads' cluster partials and takes a ticket of (unit, rank);
+  // the CTA that draws the last one merges every cluster's partial of those
+  // heads (step 2).  Nothing waits on another CTA, so the order in which the
+  // clusters run does not matter.
+  if (C > 1) cluster_sync_all();
+  else __syncthreads();
+  const int nh = kHeads / C;
+  if (threadIdx.x < kDim) {
+    const int d = threadIdx.x;
+    const DBars* peer[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) peer[c] = c < C ? (C > 1 ? cluster_peer(bars, c) : bars) : nullptr;
+    for (int h = rank; h < kHeads; h += C) {
+      // All loads first (independent, so they overlap), then the arithmetic.
+      float mc[8], lc[8], oc[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c < C) {
+          mc[c] = peer[c]->pm[h];
+          lc[c] = peer[c]->pl[h];
+          oc[c] = peer[c]->po[h * kDim + d];
+        } else {
+          mc[c] = -INFINITY;
+          lc[c] = 0.f;
+          oc[c] = 0.f;
+        }
+      }
+      float M = mc[0];
+#pragma unroll
+      for (int c = 1; c < 8; ++c) M = max_nan(M, mc[c]);
+      const float mu = M == -INFINITY ? 0.f : M;
+      float L = 0.f, O = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float f = exp2f((mc[c] - mu) * kDLog2e);
+        L += f * lc[c];
+        O += f * oc[c];
+      }
+      if (nclus == 1) {
+        a.out[((int64_t)unit * kHeads + h) * kDim + d] = (M == -INFINITY && L == 0.f) ? 0.f : O / L;
+        continue;
+      }
+      const int64_t cslot = ((int64_t)unit * a.max_clusters + clus) * kHeads + h;
+      a.cpart_acc[cslot * kDim + d] = O;
+      if (d == 0) {
+        a.cpart_ml[cslot * 2 + 0] = M;
+        a.cpart_ml[cslot * 2 + 1] = L;
+      }
+    }
+    if (nclus > 1) {
+      __threadfence();
+      asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
+      if (d == 0) bars->last = atomicAdd(&a.tickets[unit * kHeads + rank], 1) == nclus - 1;
+      asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
+      if (bars->last) {
+        __threadfence();
+        // Step 2.  Thread c < nclus takes (m, l) of cluster partial c of each
+        // head (nclus <= 256 by plan); block max and sum per head; then
+        // thread d sums dim d over the partials, 32 loads in flight.
+        // L2-coherent loads: other SMs wrote the partials.
+        const int64_t u0 = (int64_t)unit * a.max_clusters * kHeads;   // cluster 0, head 0
+        float mloc[8], lloc[8];
+#pragma unroll
+        for (int hi = 0; hi < 8; ++hi) {
+          mloc[hi] = -INFINITY;
+          lloc[hi] = 0.f;
+          if (hi < nh && d < nclus) {
+            const int64_t r = u0 + (int64_t)d * kHeads + rank + hi * C;
+            mloc[hi] = __ldcg(&a.cpart_ml[r * 2]);
+            lloc[hi] = __ldcg(&a.cpart_ml[r * 2 + 1]);
+          }
+        }
+#pragma unroll
+        for (int hi = 0; hi < 8; ++hi) {
+          if (hi < nh) {
+            float mw = mloc[hi];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+            if (lane == 0) bars->mred[hi][warp] = mw;
+          }
+        }
+        asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
+        float m2[8];
+#pragma unroll
+        for (int hi = 0; hi < 8; ++hi) {
+          if (hi < nh) {
+            float M2 = bars->mred[hi][0];
+#pragma unroll
+            for (int w = 1; w < kDWarps; ++w) M2 = max_nan(M2, bars->mred[hi][w]);
+            m2[hi] = M2;
+            const float mu2 = M2 == -INFINITY ? 0.f : M2;
+            const float f = d < nclus ? exp2f((mloc[hi] - mu2) * kDLog2e) : 0.f;
+            bars->fsc[hi][d] = f;
+            float lw = f * lloc[hi];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+            if (lane == 0) bars->lred[hi][warp] = lw;
+          }
+        }
+        asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
+        for (int hi = 0; hi < nh; ++hi) {
+          const int h = rank + hi * C;
+          float L2 = 0.f;
+#pragma unroll
+          for (int w = 0; w < kDWarps; ++w) L2 += bars->lred[hi][w];
+          const float* acc = a.cpart_acc + (u0 + h) * kDim + d;
+          float O2 = 0.f;
+          for (int c0 = 0; c0 < nclus; c0 += 32) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              v[j] = c0 + j < nclus ? __ldcg(acc + (int64_t)(c0 + j) * kHeads * kDim) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < nclus) O2 += bars->fsc[hi][c0 + j] * v[j];
+          }
+          float M2 = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (k == hi) M2 = m2[k];
+          a.out[((int64_t)unit * kHeads + h) * kDim + d] = (M2 == -INFINITY && L2 == 0.f) ? 0.f : O2 / L2;
+        }
+        if (d == 0) a.tickets[unit * kHeads + rank] = 0;   // ready for the next call
+      }
+    }
+  }
+  if (C > 1) cluster_sync_all();   // no CTA leaves while others read its shared memory
+}
+
+template <int QT, int KT>
+cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsArgs& a,
+                     cudaStream_t stream) {
+  auto kern = decode_mma_kernel<QT, KT>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.max_clusters * a.cluster, a.n_units, 1);
+  cfg.blockDim = dim3(kDThreads, 1, 1);
+  cfg.dynamicSmemBytes = kDSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  int na = 0;
+  if (a.cluster > 1) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = a.cluster;
+    at[na].val.clusterDim.y = 1;
+    at[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a);
+}
+
+template <int QT, int KT>
+int cluster_capacity_t(int c) {
+  auto kern = decode_mma_kernel<QT, KT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDSmemBytes) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c, 1, 1);
+  cfg.blockDim = dim3(kDThreads, 1, 1);
+  cfg.dynamicSmemBytes = kDSmemBytes;
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeClusterDimension;
+  at.val.clusterDim.x = c;
+  at.val.clusterDim.y = 1;
+  at.val.clusterDim.z = 1;
+  cfg.attrs = &at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+}  // namespace
+
+int decode_mma_cluster_capacity(int c) {
+  // Same launch shape for every dtype instantiation; cached per device and size.
+  static int cache[64][4] = {{0}};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int idx = c == 1 ? 0 : (c == 2 ? 1 : (c == 4 ? 2 : 3));
+  if (cache[dev][idx] == 0) cache[dev][idx] = cluster_capacity_t<KCA_F32, KCA_F16>(c);
+  return cache[dev][idx];
+}
+
+cudaError_t launch_decode_mma(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                              const RowsArgs& a, cudaStream_t stream) {
+  cudaError_t e = cudaErrorInvalidValue;
+#define KCA_DMMA_CASE(QD, KD) \
+  if (q_dtype == QD && kv_dtype == KD) e = launch_t<QD, KD>(tmk, tmv, a, stream);
+  KCA_DMMA_CASE(KCA_F32, KCA_F16)
+  KCA_DMMA_CASE(KCA_F32, KCA_BF16)
+  KCA_DMMA_CASE(KCA_F16, KCA_F16)
+  KCA_DMMA_CASE(KCA_F16, KCA_BF16)
+  KCA_DMMA_CASE(KCA_BF16, KCA_F16)
+  KCA_DMMA_CASE(KCA_BF16, KCA_BF16)
+#undef KCA_DMMA_CASE
+  return e;
+}
+
+}  // namespace kca

@@ -89,6 +89,42 @@ inline RowsPlan make_rows_plan(int32_t n_units, const int64_t* nkeys, int32_t nu
   return p;
 }
 
+// Tensor-core rows kernel: the splits of a unit run as clusters of `cluster`
+// CTAs (one CTA per SM), so a unit with n splits takes ceil(n / cluster)
+// clusters.  split_len is the smallest multiple of the kernel's stage
+// (kRowsMmaStage keys) whose clusters all fit the `slots` clusters that can be
+// resident at once; when one split per unit does not fit, every unit gets one.
+constexpr int kRowsMmaStage = 64;
+constexpr int kRowsMmaMaxClusterParts = 256;   // the kernel merges at most this many cluster partials
+
+inline RowsPlan make_cluster_rows_plan(int32_t n_units, const int64_t* nkeys, int32_t cluster,
+                                       int32_t slots) {
+  RowsPlan p;
+  p.n_units = n_units;
+  int64_t max_keys = 0;
+  for (int32_t u = 0; u < n_units; ++u) max_keys = nkeys[u] > max_keys ? nkeys[u] : max_keys;
+  const int64_t c = cluster > 0 ? cluster : 1;
+  const int64_t target = slots > 0 ? slots : 1;
+  auto count = [&](int64_t len) {
+    int64_t n = 0;
+    for (int32_t u = 0; u < n_units; ++u) n += cdiv(rows_n_splits(nkeys[u], (int32_t)len), c);
+    return n;
+  };
+  int64_t hi = cdiv(max_keys > kRowsMmaStage ? max_keys : kRowsMmaStage, kRowsMmaStage);
+  int64_t lo = 1;
+  if (count(lo * kRowsMmaStage) <= target) {
+    hi = lo;
+  } else {
+    while (lo + 1 < hi) {
+      const int64_t mid = (lo + hi) / 2;
+      if (count(mid * kRowsMmaStage) <= target) hi = mid; else lo = mid;
+    }
+  }
+  p.split_len = (int32_t)(hi * kRowsMmaStage);
+  p.max_splits = rows_n_splits(max_keys, p.split_len);
+  return p;
+}
+
 // ------------------------------------------------------ tensor-core path
 // A chunk of `rows` query rows at chunk_start is cut into row tiles of 16
 // positions (x 8 heads = 128 M rows).  Keys are addressed relative to

@@ -320,11 +320,15 @@ cudaError_t launch_rows_t(const RowsArgs& a, cudaStream_t stream) {
   kern<<<grid, kRowsThreads, S::kTotal, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.max_splits <= 1) return e;
-  merge_rows_kernel<<<a.n_units * kHeads, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_merge_rows(a, stream);
 }
 
 }  // namespace
+
+cudaError_t launch_merge_rows(const RowsArgs& a, cudaStream_t stream) {
+  merge_rows_kernel<<<a.n_units * kHeads, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rows(int q_dtype, int kv_dtype, const RowsArgs& a, cudaStream_t stream) {
 #define KCA_ROWS_CASE(QD, KD) \

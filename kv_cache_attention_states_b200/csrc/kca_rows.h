@@ -1,6 +1,7 @@
 // kca_rows.h -- launch interface of the rows kernels (decode split + merge).
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/kca.h"
@@ -23,9 +24,30 @@ struct RowsArgs {
   int32_t max_splits;
   int32_t window;
   float scale;
+  // tensor-core path only: CTAs per cluster (1, 2, 4, 8), clusters per unit at
+  // most, self-resetting tickets [n_units][8] and cluster partials
+  // [n_units][max_clusters][8] x (m, l) / acc[256].
+  int32_t cluster;
+  int32_t max_clusters;
+  int32_t* tickets;
+  float* cpart_ml;
+  float* cpart_acc;
   int64_t ctx[KCA_MAX_BATCH];  // decode: ctx_len per sequence
 };
 
 cudaError_t launch_rows(int q_dtype, int kv_dtype, const RowsArgs& a, cudaStream_t stream);
+
+// Log-sum-exp merge of the split partials in a (units with more than one split).
+cudaError_t launch_merge_rows(const RowsArgs& a, cudaStream_t stream);
+
+// Tensor-core variant for 16-bit K/V (kca_decode_mma.cu); tmk / tmv map the
+// cache rows [rows][256] with 64 x 64 boxes and 128-byte swizzle.  Merges in
+// the same kernel (clusters + tickets).
+// Clusters of c CTAs of the tensor-core rows kernel that fit on the device at
+// once (0 on failure).
+int decode_mma_cluster_capacity(int c);
+
+cudaError_t launch_decode_mma(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                              const RowsArgs& a, cudaStream_t stream);
 
 }  // namespace kca

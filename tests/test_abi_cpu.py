@@ -34,7 +34,7 @@ def test_header_constants_match_binding():
     text = open(HEADER).read()
     for name, val in [("KCA_MAX_CHUNK_ROWS", 768), ("KCA_MAX_POSITION", 131072),
                       ("KCA_HEAD_DIM", 256), ("KCA_N_Q_HEADS", 8), ("KCA_N_KV_HEADS", 1),
-                      ("KCA_WORKSPACE_HEADER", 256), ("KCA_MAX_BATCH", 256)]:
+                      ("KCA_WORKSPACE_HEADER", 24832), ("KCA_MAX_BATCH", 256)]:
         assert re.search(rf"#define {name} {val}\b", text), name
 
 

@@ -195,3 +195,17 @@ def test_long_chunk_at_capacity_end_sampled_rows():
     sample = np.array([0, 1, 15, 16, 17, 300, 511, 700, 766, 767])
     want = oracle_prefill(q, k, v, cs, sample, 0, "bf16", "bf16")
     assert max_err(out.cpu().numpy()[sample], want) <= 4e-3
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("f32", "f16"), ("bf16", "bf16"), ("f32", "bf16")])
+def test_decode_tensor_core_and_cuda_core_paths_agree(monkeypatch, q_dtype, kv_dtype):
+    cap = 20000
+    ctx = [19999, 1, 63, 64, 65, 777, 12000]
+    k, v = _cache(6, cap, [cap] * len(ctx), kv_dtype, batch=len(ctx))
+    q = synth.draw(6, "q", (len(ctx), 8, 256), q_dtype)
+    args = (dev(q, q_dtype), dev(k, kv_dtype), dev(v, kv_dtype), ctx)
+    mma = kca.attn_decode(*args).cpu().numpy()
+    monkeypatch.setenv("KCA_DECODE_PATH", "simt")
+    simt = kca.attn_decode(*args).cpu().numpy()
+    want = oracle_decode(q, k, v, ctx, 0, q_dtype, kv_dtype, cap)
+    assert max_err(mma, want) <= 4e-3 and max_err(simt, want) <= 4e-3
