@@ -50,10 +50,11 @@ constexpr int kDBoxBytes = 64 * 64 * 2;              // 64 rows x 64 dims, 8 KiB
 constexpr int kDHalfBytes = 4 * kDBoxBytes;          // K or V of one stage: 32 KiB
 constexpr int kDStageBytes = 2 * kDHalfBytes;        // 64 KiB
 constexpr int kDPRow = 144;                          // P row pitch: 128 B + 16 B pad
+constexpr int kDQRow = 528;                          // Q row pitch: 512 B + 16 B pad
 constexpr int kDOffBar = kDStages * kDStageBytes;    // 192 KiB
 constexpr float kDLog2e = 1.4426950408889634f;
 constexpr float kDRescale = 5.545177444479562f;      // 8 ln 2
-constexpr int kDMaxClusterParts = kRowsMmaMaxClusterParts;  // cluster partials a unit may have
+constexpr int kDPrefetchKeys = 512;                  // keys per split prefetched into L2 early
 
 struct DBars {
   uint64_t full[kDStages];
@@ -62,15 +63,15 @@ struct DBars {
   float red[kDWarps][8];                 // per-warp stage max (then row sums) per head
   int last;                              // this CTA holds the last ticket of its unit
   __align__(16) unsigned char p[16 * kDPRow];   // P: rows 0-7 hi, 8-15 lo, 64 keys
-  // Partial of this CTA for the cluster merge: reference max (natural units),
-  // row sum and unnormalised output per head.  Own space, not a stage buffer,
-  // so no copy still landing after an abort can overwrite it.
-  float pm[8];
-  float pl[8];
-  float po[8 * 256];
-  float fsc[kHeads][kDMaxClusterParts];  // merge weight of each cluster partial
-  float mred[kHeads][kDWarps];           // block reductions of the merge
-  float lred[kHeads][kDWarps];
+  __align__(16) unsigned char qs[16 * kDQRow];  // Q: rows 0-7 hi, 8-15 lo, 256 dims
+  // Partials this CTA receives for the heads it owns: slot src * (8 / C) + i
+  // holds CTA src's reference max (natural units), row sum and unnormalised
+  // output of head rank + i * C.  Written by the cluster's CTAs (distributed
+  // shared memory stores); own space, so no copy still landing after an
+  // abort can overwrite it.
+  float rm[8];
+  float rl[8];
+  float ro[8][256];
 };
 constexpr int kDSmemBytes = kDOffBar + (int)sizeof(DBars) + 1024;
 
@@ -135,24 +136,37 @@ __device__ __forceinline__ uint32_t swz(int row, int dim) {
 }
 
 
-template <int QT>
-__device__ __forceinline__ float load_elem(const void* base, int64_t idx) {
-  if (QT == KCA_F32) return static_cast<const float*>(base)[idx];
-  if (QT == KCA_F16) return __half2float(static_cast<const __half*>(base)[idx]);
-  return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[idx]);
-}
-
 // Cluster-wide barrier (all threads of every CTA of the cluster).
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Generic address of the same shared-memory object in CTA `cta` of the
-// cluster; plain loads through it read that CTA's shared memory.
-template <typename T>
-__device__ __forceinline__ const T* cluster_peer(const T* local, uint32_t cta) {
-  uint64_t remote;
-  asm("mapa.u64 %0, %1, %2;" : "=l"(remote) : "l"(reinterpret_cast<uint64_t>(local)), "r"(cta));
-  return reinterpret_cast<const T*>(remote);
+// Split cluster barrier: every thread of every CTA of the cluster arrives,
+// and waits for the others' arrival.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Stores into the shared memory of CTA `cta` of the cluster, at the offset
+// that `local` has in this CTA's (a plain store without a cluster).
+__device__ __forceinline__ void st_peer(float* local, uint32_t cta, float v, int C) {
+  if (C == 1) {
+    *local = v;
+    return;
+  }
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(cta));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_peer2(float* local, uint32_t cta, float v0, float v1, int C) {
+  if (C == 1) {
+    *reinterpret_cast<float2*>(local) = make_float2(v0, v1);
+    return;
+  }
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(cta));
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(v0), "f"(v1) : "memory");
 }
 
 template <int QT, int KT>
@@ -195,14 +209,33 @@ __global__ void __launch_bounds__(kDThreads, 1)
     bars->abort = 0;
     fence_barrier_init();
   }
+  if (threadIdx.x == kDWarps * 32) {
+    // Descriptors are kernel parameters: fetch them early.  The first stages
+    // of the split are prefetched into L2 as well, overlapping the previous
+    // kernel of the stream; a prefetch binds no value, so rows that kernel
+    // still writes are read after the wait below all the same.
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+    if (active) {
+      int64_t n = kend - kbeg;
+      if (n > kDPrefetchKeys) n = kDPrefetchKeys;
+      const int64_t off = (base_row + kbeg) * (kDim * 2);
+      const uint32_t bytes = (uint32_t)(n * kDim * 2);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char*>(a.k) + off),
+                   "r"(bytes) : "memory");
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char*>(a.v) + off),
+                   "r"(bytes) : "memory");
+    }
+  }
   __syncthreads();
+  // Distributed shared memory may be written only once every CTA of the
+  // cluster runs: arrive now, wait just before the first remote store.
+  if (C > 1) cluster_arrive();
   // Everything above overlaps the previous kernel of the stream (programmatic
   // dependent launch); inputs, outputs and workspace are touched only below.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  float* pm = bars->pm;
-  float* pl = bars->pl;
-  float* po = bars->po;
+  const int nh = kHeads / C;               // heads each CTA owns in the merge
 
   if (warp == kDWarps) {
     // ---------------------------------------------------------------- producer
@@ -234,11 +267,16 @@ __global__ void __launch_bounds__(kDThreads, 1)
     __syncwarp();
   } else if (!active) {
     // no key in this split (or in the whole row): an empty partial
-    if (threadIdx.x < 8) {
-      pm[threadIdx.x] = -INFINITY;
-      pl[threadIdx.x] = 0.f;
+    if (C > 1) cluster_wait();
+    if (threadIdx.x < kHeads) {
+      const int h = threadIdx.x;
+      st_peer(&bars->rm[rank * nh + h / C], h % C, -INFINITY, C);
+      st_peer(&bars->rl[rank * nh + h / C], h % C, 0.f, C);
     }
-    for (int i = threadIdx.x; i < kHeads * kDim; i += kDWarps * 32) po[i] = 0.f;
+    for (int i = threadIdx.x; i < kHeads * kDim; i += kDWarps * 32) {
+      const int h = i / kDim;
+      st_peer(&bars->ro[rank * nh + h / C][i % kDim], h % C, 0.f, C);
+    }
   } else {
     // ------------------------------------------------------------------ compute
     const int g = lane >> 2, tig = lane & 3;
@@ -246,20 +284,25 @@ __global__ void __launch_bounds__(kDThreads, 1)
     // rows 8-15 the remainders; per k-step: (g, 2tig), (g+8, 2tig), (g, 2tig+8), (g+8, 2tig+8).
     uint32_t qa[16][4];
     {
-      const void* q = static_cast<const char*>(a.q) + (int64_t)unit * kHeads * kDim * ElemBytes<QT>::value;
+      // Stage the split query once, coalesced (thread t: 8 dims of head
+      // t / 32), then every warp takes its A fragments with ldmatrix.
+      const int h = threadIdx.x >> 5, d0 = 8 * (threadIdx.x & 31);
+      float x[8];
+      load8<QT>(static_cast<const char*>(a.q) + ((int64_t)unit * kHeads * kDim + h * kDim + d0) * ElemBytes<QT>::value, x);
+      uint32_t hi[4], lo[4];
   #pragma unroll
-      for (int ks = 0; ks < 16; ++ks) {
-  #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int d = 16 * ks + 8 * half + 2 * tig;
-          const float x0 = load_elem<QT>(q, g * kDim + d);
-          const float x1 = load_elem<QT>(q, g * kDim + d + 1);
-          const uint32_t hi = pack16<KT>(x0, x1);
-          const float2 f = unpack16<KT>(hi);
-          qa[ks][2 * half] = hi;
-          qa[ks][2 * half + 1] = pack16<KT>(x0 - f.x, x1 - f.y);
-        }
+      for (int j = 0; j < 4; ++j) {
+        hi[j] = pack16<KT>(x[2 * j], x[2 * j + 1]);
+        const float2 f = unpack16<KT>(hi[j]);
+        lo[j] = pack16<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
       }
+      *reinterpret_cast<uint4*>(bars->qs + h * kDQRow + d0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(bars->qs + (h + 8) * kDQRow + d0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+      const int mi = lane >> 3;
+      const uint32_t qrow = smem_u32(bars->qs) + (8 * (mi & 1) + (lane & 7)) * kDQRow + 8 * (mi >> 1) * 2;
+  #pragma unroll
+      for (int ks = 0; ks < 16; ++ks) ldsm_x4(qrow + 32 * ks, qa[ks]);
     }
     float o[4][4];
   #pragma unroll
@@ -290,18 +333,26 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 make_uint4(0, 0, 0, 0);
           }
         }
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+        // Four independent accumulation chains over d (shorter latency).
+        float sacc[4][4];
+  #pragma unroll
+        for (int c = 0; c < 4; ++c)
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) sacc[c][j] = 0.f;
         const int kr = 8 * warp + (lane & 7);
   #pragma unroll
         for (int ks2 = 0; ks2 < 8; ++ks2) {
           uint32_t b[4];
           ldsm_x4(kst + swz(kr, 32 * ks2 + 8 * (lane >> 3)), b);
-          mma16816<KT>(sacc, qa[2 * ks2], b[0], b[1]);
-          mma16816<KT>(sacc, qa[2 * ks2 + 1], b[2], b[3]);
+          mma16816<KT>(sacc[(2 * ks2) & 3], qa[2 * ks2], b[0], b[1]);
+          mma16816<KT>(sacc[(2 * ks2 + 1) & 3], qa[2 * ks2 + 1], b[2], b[3]);
         }
+        float st[4];
+  #pragma unroll
+        for (int j = 0; j < 4; ++j) st[j] = (sacc[0][j] + sacc[1][j]) + (sacc[2][j] + sacc[3][j]);
         const int kk0 = 8 * warp + 2 * tig;
-        sx0 = kk0 < cnt ? (sacc[0] + sacc[2]) * scale : -INFINITY;
-        sx1 = kk0 + 1 < cnt ? (sacc[1] + sacc[3]) * scale : -INFINITY;
+        sx0 = kk0 < cnt ? (st[0] + st[2]) * scale : -INFINITY;
+        sx1 = kk0 + 1 < cnt ? (st[1] + st[3]) * scale : -INFINITY;
       }
       float mw = max_nan(sx0, sx1);
       mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 1));
@@ -365,60 +416,57 @@ __global__ void __launch_bounds__(kDThreads, 1)
       m_ref = NAN;   // an aborted split poisons its row; the status word says why
       L = NAN;
     }
+    // Push the partial of head g to the CTA that owns it (rows g and g+8 of
+    // the accumulator are the high and low parts).
+    if (C > 1) cluster_wait();
+    const int owner = g % C, slot = rank * nh + g / C;
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
       const int d = 32 * warp + 8 * nt + 2 * tig;
-      po[g * kDim + d] = o[nt][0] + o[nt][2];
-      po[g * kDim + d + 1] = o[nt][1] + o[nt][3];
+      st_peer2(&bars->ro[slot][d], owner, o[nt][0] + o[nt][2], o[nt][1] + o[nt][3], C);
     }
     if (warp == 0 && tig == 0) {
-      pm[g] = m_ref;
-      pl[g] = L;
+      st_peer(&bars->rm[slot], owner, m_ref, C);
+      st_peer(&bars->rl[slot], owner, L, C);
     }
   }
+  if (warp == kDWarps && C > 1) cluster_wait();   // the producer keeps the barrier phases in step
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ------------------------------------------------------------ merge
-  // CTA rank r owns heads r, r+C, ... (C divides 8).  Step 1 merges the C
-  // partials of its cluster through distributed shared memory; thread d owns
-  // dim d.  With one cluster per unit that is the result.  Otherwise each CTA
-  // publishes its heads' cluster partials and takes a ticket of (unit, rank);
-  // the CTA that draws the last one merges every cluster's partial of those
-  // heads (step 2).  Nothing waits on another CTA, so the order in which the
-  // clusters run does not matter.
+  // CTA rank r owns heads r, r+C, ... (C divides 8) and has received the C
+  // partials of each through distributed shared memory; once the cluster
+  // barrier completes, they are in its own shared memory and no CTA touches
+  // another's again.  Thread d owns dim d.  With one cluster per unit the
+  // merge of the C partials is the result.  Otherwise each CTA publishes its
+  // heads' cluster partials and takes a ticket of (unit, rank); the CTA that
+  // draws the last one merges every cluster's partials of those heads.
+  // Nothing waits on another CTA, so the order in which clusters run does not
+  // matter.
   if (C > 1) cluster_sync_all();
   else __syncthreads();
-  const int nh = kHeads / C;
   if (threadIdx.x < kDim) {
     const int d = threadIdx.x;
-    const DBars* peer[8];
+    for (int i = 0; i < nh; ++i) {
+      const int h = rank + i * C;
+      float mv[8], lv[8], ov[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) peer[c] = c < C ? (C > 1 ? cluster_peer(bars, c) : bars) : nullptr;
-    for (int h = rank; h < kHeads; h += C) {
-      // All loads first (independent, so they overlap), then the arithmetic.
-      float mc[8], lc[8], oc[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        if (c < C) {
-          mc[c] = peer[c]->pm[h];
-          lc[c] = peer[c]->pl[h];
-          oc[c] = peer[c]->po[h * kDim + d];
-        } else {
-          mc[c] = -INFINITY;
-          lc[c] = 0.f;
-          oc[c] = 0.f;
-        }
+      for (int src = 0; src < 8; ++src) {
+        const bool in = src < C;
+        mv[src] = in ? bars->rm[src * nh + i] : -INFINITY;
+        lv[src] = in ? bars->rl[src * nh + i] : 0.f;
+        ov[src] = in ? bars->ro[src * nh + i][d] : 0.f;
       }
-      float M = mc[0];
+      float M = mv[0];
 #pragma unroll
-      for (int c = 1; c < 8; ++c) M = max_nan(M, mc[c]);
+      for (int src = 1; src < 8; ++src) M = max_nan(M, mv[src]);
       const float mu = M == -INFINITY ? 0.f : M;
       float L = 0.f, O = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float f = exp2f((mc[c] - mu) * kDLog2e);
-        L += f * lc[c];
-        O += f * oc[c];
+      for (int src = 0; src < 8; ++src) {
+        const float f = exp2f((mv[src] - mu) * kDLog2e);
+        L += f * lv[src];
+        O += f * ov[src];
       }
       if (nclus == 1) {
         a.out[((int64_t)unit * kHeads + h) * kDim + d] = (M == -INFINITY && L == 0.f) ? 0.f : O / L;
@@ -432,83 +480,94 @@ __global__ void __launch_bounds__(kDThreads, 1)
       }
     }
     if (nclus > 1) {
-      __threadfence();
+      // Release: the block's partial stores, then one thread's fence and
+      // ticket.  Acquire: the last ticket holder's fence, then the block.
       asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
-      if (d == 0) bars->last = atomicAdd(&a.tickets[unit * kHeads + rank], 1) == nclus - 1;
+      if (d == 0) {
+        __threadfence();
+        const bool last = atomicAdd(&a.tickets[unit * kHeads + rank], 1) == nclus - 1;
+        if (last) __threadfence();
+        bars->last = last;
+      }
       asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
       if (bars->last) {
-        __threadfence();
-        // Step 2.  Thread c < nclus takes (m, l) of cluster partial c of each
-        // head (nclus <= 256 by plan); block max and sum per head; then
-        // thread d sums dim d over the partials, 32 loads in flight.
-        // L2-coherent loads: other SMs wrote the partials.
+        // Merge of the nclus cluster partials of each owned head.  (m, l) of
+        // every partial go to shared memory first (the stage buffers are
+        // free now); thread t then sums dims 4(t % 64) .. +3 over the
+        // partials c = t / 64 (mod 4) with 16-byte loads, eight in flight,
+        // and the four groups are added in shared memory.  L2-coherent
+        // loads: other SMs wrote the partials.
+        float* sm_m = reinterpret_cast<float*>(smem);          // [8][256]
+        float* sm_l = sm_m + kHeads * kDim;                    // [8][256]
+        float* sm_o = sm_l + kHeads * kDim;                    // [4][256]
         const int64_t u0 = (int64_t)unit * a.max_clusters * kHeads;   // cluster 0, head 0
-        float mloc[8], lloc[8];
+        const int grp = d >> 6, q4 = d & 63;
+        // Eight partials c0, c0 + 4, ... of head rank + i * C, dims 4 q4 .. +3.
+        auto load_batch = [&](int i, int c0, float4(&v)[8]) {
+          const float4* acc = reinterpret_cast<const float4*>(a.cpart_acc + (u0 + rank + i * C) * kDim) + q4;
 #pragma unroll
-        for (int hi = 0; hi < 8; ++hi) {
-          mloc[hi] = -INFINITY;
-          lloc[hi] = 0.f;
-          if (hi < nh && d < nclus) {
-            const int64_t r = u0 + (int64_t)d * kHeads + rank + hi * C;
-            mloc[hi] = __ldcg(&a.cpart_ml[r * 2]);
-            lloc[hi] = __ldcg(&a.cpart_ml[r * 2 + 1]);
+          for (int j = 0; j < 8; ++j) {
+            const int c = c0 + 4 * j;
+            v[j] = c < nclus ? __ldcg(acc + (int64_t)c * kHeads * (kDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
-        }
+        };
+        // The first batches of heads 0 and 1 are in flight together with the
+        // (m, l) loads, and each head's successor-but-one is requested as
+        // soon as its registers are free, so the merge waits on about one
+        // round trip.
+        auto merge_head = [&](int i, float4(&v)[8]) {
+          const int h = rank + i * C;
+          // (M, L) of head h: each warp reduces them itself.
+          float mw = -INFINITY;
+          for (int c = lane; c < nclus; c += 32) mw = max_nan(mw, sm_m[i * kDim + c]);
 #pragma unroll
-        for (int hi = 0; hi < 8; ++hi) {
-          if (hi < nh) {
-            float mw = mloc[hi];
+          for (int o = 16; o > 0; o >>= 1) mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+          const float M = mw, mu = M == -INFINITY ? 0.f : M;
+          float lw = 0.f;
+          for (int c = lane; c < nclus; c += 32) lw += exp2f((sm_m[i * kDim + c] - mu) * kDLog2e) * sm_l[i * kDim + c];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, o));
-            if (lane == 0) bars->mred[hi][warp] = mw;
+          for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+          const float L = lw;
+          float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int c0 = grp;; c0 += 32) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int c = c0 + 4 * j;
+              const float f = c < nclus ? exp2f((sm_m[i * kDim + c] - mu) * kDLog2e) : 0.f;
+              O.x += f * v[j].x;
+              O.y += f * v[j].y;
+              O.z += f * v[j].z;
+              O.w += f * v[j].w;
+            }
+            if (c0 + 32 >= nclus) break;
+            load_batch(i, c0 + 32, v);
+          }
+          if (i + 2 < nh) load_batch(i + 2, grp, v);
+          reinterpret_cast<float4*>(sm_o + grp * kDim)[q4] = O;
+          asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
+          const float Od = (sm_o[d] + sm_o[kDim + d]) + (sm_o[2 * kDim + d] + sm_o[3 * kDim + d]);
+          a.out[((int64_t)unit * kHeads + h) * kDim + d] = (M == -INFINITY && L == 0.f) ? 0.f : Od / L;
+          asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");   // sm_o is reused by the next head
+        };
+        float4 va[8], vb[8];
+        load_batch(0, grp, va);
+        if (nh > 1) load_batch(1, grp, vb);
+        for (int c = d; c < nclus; c += kDim) {
+          for (int i = 0; i < nh; ++i) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.cpart_ml) + u0 + (int64_t)c * kHeads + rank + i * C);
+            sm_m[i * kDim + c] = ml.x;
+            sm_l[i * kDim + c] = ml.y;
           }
         }
         asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
-        float m2[8];
-#pragma unroll
-        for (int hi = 0; hi < 8; ++hi) {
-          if (hi < nh) {
-            float M2 = bars->mred[hi][0];
-#pragma unroll
-            for (int w = 1; w < kDWarps; ++w) M2 = max_nan(M2, bars->mred[hi][w]);
-            m2[hi] = M2;
-            const float mu2 = M2 == -INFINITY ? 0.f : M2;
-            const float f = d < nclus ? exp2f((mloc[hi] - mu2) * kDLog2e) : 0.f;
-            bars->fsc[hi][d] = f;
-            float lw = f * lloc[hi];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-            if (lane == 0) bars->lred[hi][warp] = lw;
-          }
-        }
-        asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
-        for (int hi = 0; hi < nh; ++hi) {
-          const int h = rank + hi * C;
-          float L2 = 0.f;
-#pragma unroll
-          for (int w = 0; w < kDWarps; ++w) L2 += bars->lred[hi][w];
-          const float* acc = a.cpart_acc + (u0 + h) * kDim + d;
-          float O2 = 0.f;
-          for (int c0 = 0; c0 < nclus; c0 += 32) {
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              v[j] = c0 + j < nclus ? __ldcg(acc + (int64_t)(c0 + j) * kHeads * kDim) : 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c0 + j < nclus) O2 += bars->fsc[hi][c0 + j] * v[j];
-          }
-          float M2 = 0.f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (k == hi) M2 = m2[k];
-          a.out[((int64_t)unit * kHeads + h) * kDim + d] = (M2 == -INFINITY && L2 == 0.f) ? 0.f : O2 / L2;
+        for (int i = 0; i < nh; i += 2) {
+          merge_head(i, va);
+          if (i + 1 < nh) merge_head(i + 1, vb);
         }
         if (d == 0) a.tickets[unit * kHeads + rank] = 0;   // ready for the next call
       }
     }
   }
-  if (C > 1) cluster_sync_all();   // no CTA leaves while others read its shared memory
 }
 
 template <int QT, int KT>

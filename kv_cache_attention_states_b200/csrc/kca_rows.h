@@ -40,13 +40,13 @@ cudaError_t launch_rows(int q_dtype, int kv_dtype, const RowsArgs& a, cudaStream
 // Log-sum-exp merge of the split partials in a (units with more than one split).
 cudaError_t launch_merge_rows(const RowsArgs& a, cudaStream_t stream);
 
-// Tensor-core variant for 16-bit K/V (kca_decode_mma.cu); tmk / tmv map the
-// cache rows [rows][256] with 64 x 64 boxes and 128-byte swizzle.  Merges in
-// the same kernel (clusters + tickets).
 // Clusters of c CTAs of the tensor-core rows kernel that fit on the device at
 // once (0 on failure).
 int decode_mma_cluster_capacity(int c);
 
+// Tensor-core variant for 16-bit K/V (kca_decode_mma.cu); tmk / tmv map the
+// cache rows [rows][256] with 64 x 64 boxes and 128-byte swizzle.  Merges in
+// the same kernel (clusters + tickets).
 cudaError_t launch_decode_mma(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                               const RowsArgs& a, cudaStream_t stream);
 
