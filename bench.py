@@ -34,6 +34,10 @@ DECODE_LEN = 16384
 DECODE_STEPS = 64
 DECODE_REPLICAS = 32
 PREFILL_REPLICAS = 2
+# DRAM bytes (read + write) per launch from one ncu capture of the current
+# kernels; reset to None whenever a kernel changes after its capture.
+PREFILL_TRAFFIC = 19.74e6 + 27.6e3
+DECODE_TRAFFIC = 16.90e6
 METRIC = "prefill q-rows/s & decode tok/s at 16K ctx (1 B200); % of TC/HBM roofline"
 
 
@@ -141,9 +145,9 @@ class Workload:
         for cs, r in self.chunks:
             path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, r, 0, self.sms)
             n += 1 + int((items[:, 3] >= 0).any())
-        for c in self.dec_ctx:
-            items = kca.attn_decode_plan([c], 0, self.sms)
-            n += 1 + int(len(items) > 1)
+        # f16 caches take the tensor-core rows kernel, which merges its
+        # splits in the same launch: one kernel per decode call.
+        n += len(self.dec_ctx)
         return n
 
     def prefill(self):
@@ -430,13 +434,17 @@ def main():
                          "prefill alternates 2 input replicas (80 MB each)"},
         "roofline": {"kernel": "prefill_tc_kernel (+ its merge)", "bound": "tensor",
                      "achieved": achieved_tf, "peak": tflops, "unit": "TFLOP/s",
-                     "frac": achieved_tf / tflops, "traffic": None,
+                     "frac": achieved_tf / tflops, "traffic": PREFILL_TRAFFIC,
+                     "traffic_source": "ncu dram bytes of the chunk-20 launch (768 rows at 15360); "
+                                       "profiles/prefill_tc_kernel_16k_chunk20.md",
                      "peak_source": f"{src} bf16 dense (burst)",
                      "algorithmic": "4*256*8*sum|J(pos)| = 1.0996e12 flop per step"},
         "decode": {"value": dec_tok_s, "unit": "tok/s", "ms_per_step": res["dec_ms"] / K,
-                   "roofline": {"kernel": "rows_kernel<f32,f16> (+ its merge)", "bound": "hbm",
+                   "roofline": {"kernel": "decode_mma_kernel<f32,f16> (merge in-kernel)", "bound": "hbm",
                                 "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                                "frac": achieved_gbs / hbm, "traffic": None,
+                                "frac": achieved_gbs / hbm, "traffic": DECODE_TRAFFIC,
+                                "traffic_source": "ncu dram bytes of one launch at ctx ~16.4K; "
+                                                  "profiles/decode_mma_kernel_16k.md",
                                 "peak_source": f"{src} HBM copy",
                                 "algorithmic": "ctx*1024 B K/V + 16 KiB q/out per token"}},
         "e2e": {"value": world * PREFILL_ROWS * e2e["steps"] / (e2e["pre_ms"] / 1e3), "unit": "q-rows/s",
