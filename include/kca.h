@@ -141,6 +141,35 @@ int attn_decode(const void *q, int32_t q_dtype,
                 void *stream);
 
 /*
+ * attn_decode_dev -- attn_decode with the context lengths in DEVICE memory,
+ * read by the kernels when they run, so that one captured launch (CUDA graph)
+ * serves every decode step while the caller updates ctx_len_dev in place.
+ * The operation is the one-row (decode) plan of Karume v0.12.0 release notes,
+ * "Performance", items 2-3; the pages have no device-side context length:
+ * it serves decode loops replayed from a CUDA graph, step after step.
+ *   ctx_len_dev  DEVICE int64 [batch], 8-byte aligned; each value 0..ctx_bound,
+ *                written before the call's kernels run (stream order)
+ *   ctx_bound    HOST upper bound of every ctx_len_dev[b], 0..capacity.  The
+ *                launch (grid, clusters, workspace) is planned for `batch`
+ *                sequences at ctx_bound; each sequence then cuts its actual
+ *                keys into the planned number of splits on the device.
+ *   workspace    >= attn_decode_workspace_bytes(batch, {ctx_bound, ...}, window)
+ * Everything else is as in attn_decode.  The host work of a call depends only
+ * on the pointers, dtypes, capacity, batch, ctx_bound, window and scale, never
+ * on the device values.  A device value outside 0..ctx_bound is never used to
+ * address memory: that sequence's row is computed as an empty context (zeros)
+ * and the status word records it (attn_device_status returns KCA_ERR_DEVICE,
+ * detail = (10 << 24) | sequence).  ctx_len_dev must not be written while
+ * the call runs.
+ */
+int attn_decode_dev(const void *q, int32_t q_dtype,
+                    const void *k_cache, const void *v_cache, int32_t kv_dtype,
+                    int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity,
+                    int32_t batch, const int64_t *ctx_len_dev, int64_t ctx_bound, int32_t window,
+                    float scale, float *out, void *workspace, size_t workspace_bytes,
+                    void *stream);
+
+/*
  * attn_decode_static -- attn_decode for callers that cannot allocate device
  * memory: code running where cudaMalloc is unavailable or forbidden (inside a
  * host callback, a custom allocator's own path, a memory pool that admits no
@@ -177,6 +206,8 @@ int attn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Reads and clears the workspace status word (synchronises `stream`).
+ * Error bits: 1 = a bounded wait ran out (detail: (site << 24) | block),
+ * 2 = a device context length was out of range (detail: (10 << 24) | sequence).
  * Returns KCA_OK when no kernel recorded an error since the last read,
  * KCA_ERR_DEVICE when one did (*detail, if not NULL, receives the record),
  * or KCA_ERR_CUDA when the copy itself failed.

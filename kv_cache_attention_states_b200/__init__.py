@@ -55,6 +55,9 @@ def lib() -> ctypes.CDLL:
         L.attn_decode.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp,
                                   vp, sz, vp]
         L.attn_decode.restype = ctypes.c_int
+        L.attn_decode_dev.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, vp, i64, i32, f32,
+                                      vp, vp, sz, vp]
+        L.attn_decode_dev.restype = ctypes.c_int
         L.attn_decode_static.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32,
                                          f32, vp, vp]
         L.attn_decode_static.restype = ctypes.c_int
@@ -202,6 +205,36 @@ def attn_decode(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.
                            ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
                            workspace.numel(), _stream_ptr(stream))
     _check(st, "attn_decode")
+    return out
+
+
+def attn_decode_dev(q, k_cache, v_cache, ctx_len_dev, ctx_bound: int, window: int = 0,
+                    scale: float = 1.0 / 16.0, out=None, workspace=None, stream=None):
+    """attn_decode with the context lengths in device memory.
+
+    ctx_len_dev: int64 CUDA tensor [batch], each value in 0..ctx_bound, read
+    by the kernels when they run (so a captured CUDA graph of this call can be
+    replayed after updating it in place); ctx_bound: host upper bound that
+    the launch is planned for.
+    """
+    import torch
+    batch = q.shape[0]
+    capacity = k_cache.shape[1]
+    for t in (q, k_cache, v_cache, ctx_len_dev):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if ctx_len_dev.dtype != torch.int64 or ctx_len_dev.numel() != batch or k_cache.shape[0] != batch:
+        raise ValueError("ctx_len_dev must be int64 with one entry per sequence")
+    if out is None:
+        out = torch.empty((batch, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(attn_decode_workspace_bytes([ctx_bound] * batch, window), q.device, stream)
+    st = lib().attn_decode_dev(ctypes.c_void_p(q.data_ptr()), dtype_code(q), ctypes.c_void_p(k_cache.data_ptr()),
+                               ctypes.c_void_p(v_cache.data_ptr()), dtype_code(k_cache), N_Q_HEADS,
+                               N_KV_HEADS, HEAD_DIM, capacity, batch, ctypes.c_void_p(ctx_len_dev.data_ptr()),
+                               int(ctx_bound), window, scale, ctypes.c_void_p(out.data_ptr()),
+                               ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
+    _check(st, "attn_decode_dev")
     return out
 
 

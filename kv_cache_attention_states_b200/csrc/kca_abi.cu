@@ -489,4 +489,51 @@ int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void*
                           workspace, static_cast<cudaStream_t>(stream));
 }
 
+int attn_decode_dev(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache,
+                    int32_t kv_dtype, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                    int64_t capacity, int32_t batch, const int64_t* ctx_len_dev, int64_t ctx_bound,
+                    int32_t window, float scale, float* out, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  if (!q || !k_cache || !v_cache || !out || !workspace || !ctx_len_dev) return KCA_ERR_NULL;
+  int st = geometry_status(n_q_heads, n_kv_heads, head_dim);
+  if (st != KCA_OK) return st;
+  if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
+  if (batch < 1 || batch > KCA_MAX_BATCH) return KCA_ERR_RANGE;
+  // The plan is the host-array plan of `batch` sequences at the bound.
+  const std::vector<int64_t> bound(batch, ctx_bound);
+  st = decode_args_status(capacity, batch, bound.data());
+  if (st != KCA_OK) return st;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return KCA_ERR_RANGE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(ctx_len_dev) % 8) != 0)
+    return KCA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+  const std::vector<int64_t> nk = decode_unit_keys(batch, bound.data(), window);
+  int cluster = 1;
+  size_t need = 0;
+  const kca::RowsPlan p = rows_plan(kv_dtype, batch, nk.data(), sms, &cluster, &need);
+  if (cluster < 1) return KCA_ERR_CUDA;
+  if (workspace_bytes < need) return KCA_ERR_WORKSPACE;
+  kca::RowsArgs a{};
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.out = out;
+  a.status = workspace;
+  a.seq_rows = capacity;
+  a.chunk_start = 0;
+  a.mode = 0;
+  a.n_units = batch;
+  a.split_len = p.split_len;
+  a.max_splits = p.max_splits;
+  a.window = window;
+  a.scale = scale;
+  a.ctx_dev = ctx_len_dev;
+  a.ctx_bound = ctx_bound;
+  return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster,
+                          workspace, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -19,19 +19,23 @@ namespace kca {
 
 // Status word layout (first 256 bytes of the workspace).
 struct DeviceStatus {
-  unsigned int error;   // bit 0: a bounded wait ran out
-  unsigned int detail;  // (site << 24) | (blockIdx.x & 0xffffff) of the first failure
+  unsigned int error;   // bit 0: a bounded wait ran out; bit 1: a device ctx_len out of range
+  unsigned int detail;  // (site << 24) | (block & 0xffffff) of the first failure
 };
-enum : unsigned int { kErrWaitTimeout = 1u };
+enum : unsigned int { kErrWaitTimeout = 1u, kErrBadCtx = 2u };
 enum : unsigned int {
   kSiteRowsFull = 1, kSiteRowsEmpty = 2, kSiteTcFull = 3, kSiteTcEmpty = 4, kSiteTcS = 5,
-  kSiteTcP = 6, kSiteTcO = 7, kSiteTcQ = 8, kSiteTcDrain = 9
+  kSiteTcP = 6, kSiteTcO = 7, kSiteTcQ = 8, kSiteTcDrain = 9, kSiteCtx = 10
 };
 
-__device__ __forceinline__ void record_error(DeviceStatus* st, unsigned int site) {
+// Records the first failure (detail: site and the block's x index, or the
+// sequence for kSiteCtx) and ORs `bit` into the error word.
+__device__ __forceinline__ void record_error(DeviceStatus* st, unsigned int site,
+                                             unsigned int bit = kErrWaitTimeout,
+                                             unsigned int where = 0xffffffffu) {
   if (st == nullptr) return;
-  unsigned int prev = atomicOr(&st->error, kErrWaitTimeout);
-  if ((prev & kErrWaitTimeout) == 0) st->detail = (site << 24) | (blockIdx.x & 0xffffffu);
+  const unsigned int prev = atomicOr(&st->error, bit);
+  if (prev == 0) st->detail = (site << 24) | ((where == 0xffffffffu ? blockIdx.x : where) & 0xffffffu);
 }
 
 __device__ __forceinline__ uint64_t global_ns() {

@@ -188,15 +188,19 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const int rank = split % C, clus = split / C;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t pos = a.mode == 0 ? a.ctx[unit] - 1 : a.chunk_start + unit;
+  // Device context lengths may come from the previous kernel of the stream:
+  // with them, the dependency wait comes before they are read.
+  if (a.ctx_dev != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, split == 0 && threadIdx.x == 0) - 1 : a.chunk_start + unit;
   const int64_t lo = lo_of(pos, a.window);
   const int64_t nkeys = n_visible(pos, a.window);
-  const int32_t nsplit = rows_n_splits(nkeys, a.split_len);
+  const int32_t split_len = rows_split_len(a, nkeys, kDStageKeys);
+  const int32_t nsplit = rows_n_splits(nkeys, split_len);
   const int nclus = (nsplit + C - 1) / C;
   if (clus >= nclus) return;               // the whole cluster leaves together
   const bool active = split < nsplit && nkeys > 0;
-  const int64_t kbeg = lo + (int64_t)split * a.split_len;
-  int64_t kend = kbeg + a.split_len;
+  const int64_t kbeg = lo + (int64_t)split * split_len;
+  int64_t kend = kbeg + split_len;
   if (kend > pos + 1) kend = pos + 1;
   const int64_t base_row = a.mode == 0 ? (int64_t)unit * a.seq_rows : 0;
   const int n_stage = active ? (int)cdiv(kend - kbeg, kDStageKeys) : 0;

@@ -77,13 +77,14 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int64_t pos = a.mode == 0 ? a.ctx[unit] - 1 : a.chunk_start + unit;
+  const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, split == 0 && threadIdx.x == 0) - 1 : a.chunk_start + unit;
   const int64_t lo = lo_of(pos, a.window);
   const int64_t nkeys = n_visible(pos, a.window);
-  const int32_t nsplit = rows_n_splits(nkeys, a.split_len);
+  const int32_t split_len = rows_split_len(a, nkeys, kRowsSplitQuantum);
+  const int32_t nsplit = rows_n_splits(nkeys, split_len);
   if (split >= nsplit) return;
-  const int64_t kbeg = lo + (int64_t)split * a.split_len;
-  int64_t kend = kbeg + a.split_len;
+  const int64_t kbeg = lo + (int64_t)split * split_len;
+  int64_t kend = kbeg + split_len;
   if (kend > pos + 1) kend = pos + 1;
   const int64_t base_row = a.mode == 0 ? (int64_t)unit * a.seq_rows : 0;
   float* out = a.out + (int64_t)unit * kHeads * kDim;
@@ -293,8 +294,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
 // its eight warps taking interleaved splits.
 __global__ void __launch_bounds__(256) merge_rows_kernel(const RowsArgs a) {
   const int unit = blockIdx.x >> 3, h = blockIdx.x & 7;
-  const int64_t pos = a.mode == 0 ? a.ctx[unit] - 1 : a.chunk_start + unit;
-  const int32_t nsplit = rows_n_splits(n_visible(pos, a.window), a.split_len);
+  const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, false) - 1 : a.chunk_start + unit;
+  const int64_t nkeys = n_visible(pos, a.window);
+  const int32_t nsplit = rows_n_splits(nkeys, rows_split_len(a, nkeys, kRowsSplitQuantum));
   if (nsplit <= 1) return;
   __shared__ float red[8 * 264];
   const int64_t row0 = (int64_t)unit * a.max_splits * kHeads + h;

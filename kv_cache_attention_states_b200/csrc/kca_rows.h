@@ -32,8 +32,38 @@ struct RowsArgs {
   int32_t* tickets;
   float* cpart_ml;
   float* cpart_acc;
+  // decode with device context lengths: ctx_dev[unit] (each in 0..ctx_bound)
+  // replaces ctx[unit], and each unit cuts its keys into max_splits splits
+  // itself (rows_split_len); null for the host-array form.
+  const int64_t* ctx_dev;
+  int64_t ctx_bound;
   int64_t ctx[KCA_MAX_BATCH];  // decode: ctx_len per sequence
 };
+
+#if defined(__CUDACC__)
+}  // namespace kca
+#include "kca_common.cuh"
+namespace kca {
+// Context length of decode unit `unit`.  A device value outside
+// 0..ctx_bound is recorded in the status word (when `record`) and read as an
+// empty context, so no row past the bound is ever touched.
+__device__ __forceinline__ int64_t rows_ctx(const RowsArgs& a, int unit, bool record) {
+  if (a.ctx_dev == nullptr) return a.ctx[unit];
+  const int64_t c = a.ctx_dev[unit];
+  if (c >= 0 && c <= a.ctx_bound) return c;
+  if (record) record_error(static_cast<DeviceStatus*>(a.status), kSiteCtx, kErrBadCtx, (unsigned)unit);
+  return 0;
+}
+// Keys per split of a unit with nkeys visible keys: the host plan's length,
+// or with device context lengths the smallest multiple of `quantum` (>= 64)
+// that cuts nkeys into at most max_splits splits.
+__device__ __forceinline__ int32_t rows_split_len(const RowsArgs& a, int64_t nkeys, int quantum) {
+  if (a.ctx_dev == nullptr) return a.split_len;
+  int64_t s = (nkeys + a.max_splits - 1) / a.max_splits;
+  s = (s + quantum - 1) / quantum * quantum;
+  return (int32_t)(s < 64 ? 64 : s);
+}
+#endif
 
 cudaError_t launch_rows(int q_dtype, int kv_dtype, const RowsArgs& a, cudaStream_t stream);
 

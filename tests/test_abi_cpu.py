@@ -98,6 +98,26 @@ def test_decode_rejects_bad_arguments_on_the_host(ctx, kw, code):
     assert _decode(ctx, **kw) == code
 
 
+def _decode_dev(**kw):
+    a = dict(q=P, qd=kca.F32, k=P, v=P, kd=kca.F16, hq=8, hkv=1, d=256, cap=4096, batch=2, ctx=P * 3,
+             bound=4096, window=0, scale=0.0625, out=P, ws=P * 2, wsb=1 << 30)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return kca.lib().attn_decode_dev(vp(a["q"]), a["qd"], vp(a["k"]), vp(a["v"]), a["kd"], a["hq"],
+                                     a["hkv"], a["d"], a["cap"], a["batch"], vp(a["ctx"]), a["bound"],
+                                     a["window"], a["scale"], vp(a["out"]), vp(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ctx=0), -1), (dict(q=0), -1), (dict(hkv=2), -2), (dict(kd=5), -3),
+    (dict(batch=0), -4), (dict(batch=257), -4), (dict(bound=4097), -4), (dict(bound=-1), -4),
+    (dict(cap=131073, bound=1), -4), (dict(scale=0.0), -4),
+    (dict(ctx=P * 3 + 4), -6), (dict(out=P + 4), -6), (dict(ws=P * 2 + 128), -5),
+])
+def test_decode_dev_rejects_bad_arguments_on_the_host(kw, code):
+    assert _decode_dev(**kw) == code
+
+
 def _check_rows_plan(items, units, pos_of, window):
     """Every unit's items tile its visible range exactly, in order, slots unique."""
     slots = [int(s) for s in items[:, 3] if s >= 0]
