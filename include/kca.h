@@ -195,6 +195,36 @@ int attn_decode_static(const void *q, int32_t q_dtype,
                        int32_t batch, const int64_t *ctx_len, int32_t window,
                        float scale, float *out, void *stream);
 
+/*
+ * attn_append_kv -- the step before the attention calls: writes n_rows new
+ * K/V rows into the cache, K rotated by rotary position embedding with
+ * host-generated cos/sin rows (Karume v0.8.0 release notes, "Features",
+ * conversation-window item: the host generates the cos/sin rows per chunk),
+ * V converted only.  Rotate-half pairing of dim i with dim i + 128:
+ *   k'[i]       = k[i] cos[i] - k[i+128] sin[i]
+ *   k'[i + 128] = k[i+128] cos[i+128] + k[i] sin[i+128]        (i < 128)
+ * each product and sum rounded to f32 (no fused multiply-add), then to the
+ * cache type with round-to-nearest-even: the bytes written depend on the
+ * inputs only.
+ *   k_new/v_new  [n_rows][256] in_dtype, device, 16-byte aligned
+ *   rope_cos/rope_sin  [n_rows][256] f32, device, 16-byte aligned; both NULL
+ *                = no rotation (one NULL alone is KCA_ERR_NULL)
+ *   k_cache/v_cache  [cache_rows][256] kv_dtype, device (a batched cache is
+ *                addressed by absolute row b * capacity + position)
+ *   dst_rows_dev DEVICE int64 [n_rows] destination rows, 8-byte aligned, or
+ *                NULL: rows dst_row0 .. dst_row0 + n_rows - 1 (checked on the
+ *                host against cache_rows)
+ *   workspace    optional status word (a workspace, or NULL): a device
+ *                destination outside 0..cache_rows-1 is skipped and recorded
+ *                there (error bit 3 = value 4, detail (11 << 24) | row)
+ * Rows must not share a destination.  Returns KCA_OK or a KCA_ERR_* before
+ * launching anything.
+ */
+int attn_append_kv(const void *k_new, const void *v_new, int32_t in_dtype, int32_t n_rows,
+                   const float *rope_cos, const float *rope_sin,
+                   void *k_cache, void *v_cache, int32_t kv_dtype, int64_t cache_rows,
+                   const int64_t *dst_rows_dev, int64_t dst_row0, void *workspace, void *stream);
+
 /* Workspace bytes the calls above need on the current device (0 on a bad
  * argument).  Always >= KCA_WORKSPACE_HEADER. */
 size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
@@ -207,7 +237,8 @@ int attn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 /*
  * Reads and clears the workspace status word (synchronises `stream`).
  * Error bits: 1 = a bounded wait ran out (detail: (site << 24) | block),
- * 2 = a device context length was out of range (detail: (10 << 24) | sequence).
+ * 2 = a device context length was out of range (detail: (10 << 24) | sequence),
+ * 4 = an append destination was out of range (detail: (11 << 24) | row).
  * Returns KCA_OK when no kernel recorded an error since the last read,
  * KCA_ERR_DEVICE when one did (*detail, if not NULL, receives the record),
  * or KCA_ERR_CUDA when the copy itself failed.

@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
         L.attn_decode_dev.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, vp, i64, i32, f32,
                                       vp, vp, sz, vp]
         L.attn_decode_dev.restype = ctypes.c_int
+        L.attn_append_kv.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp, i32, i64, vp, i64, vp, vp]
+        L.attn_append_kv.restype = ctypes.c_int
         L.attn_decode_static.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32,
                                          f32, vp, vp]
         L.attn_decode_static.restype = ctypes.c_int
@@ -236,6 +238,45 @@ def attn_decode_dev(q, k_cache, v_cache, ctx_len_dev, ctx_bound: int, window: in
                                ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
     _check(st, "attn_decode_dev")
     return out
+
+
+def attn_append_kv(k_new, v_new, k_cache, v_cache, dst, rope_cos=None, rope_sin=None, workspace=None,
+                   stream=None):
+    """Write new K/V rows into the cache, K rotated by RoPE when cos/sin are given.
+
+    k_new / v_new: [n, 256] (or [n, 1, 256]); k_cache / v_cache: contiguous with
+    a last axis of 256, addressed as rows; dst: an int (rows dst .. dst+n-1) or
+    an int64 CUDA tensor [n] of destination rows; rope_cos / rope_sin: float32
+    CUDA tensors [n, 256] or None.
+    """
+    import torch
+    n = k_new.numel() // HEAD_DIM
+    for t in (k_new, v_new, k_cache, v_cache):
+        if not t.is_cuda or not t.is_contiguous() or t.shape[-1] != HEAD_DIM:
+            raise ValueError("tensors must be contiguous CUDA tensors with a last axis of 256")
+    if v_new.numel() != k_new.numel() or v_cache.numel() != k_cache.numel():
+        raise ValueError("k and v shapes differ")
+    if (rope_cos is None) != (rope_sin is None):
+        raise ValueError("give both rope_cos and rope_sin, or neither")
+    vp = ctypes.c_void_p
+    cos_p = vp(rope_cos.data_ptr()) if rope_cos is not None else None
+    sin_p = vp(rope_sin.data_ptr()) if rope_sin is not None else None
+    if rope_cos is not None:
+        for t in (rope_cos, rope_sin):
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.numel() != n * HEAD_DIM:
+                raise ValueError("rope_cos / rope_sin must be float32 CUDA tensors [n, 256]")
+    if isinstance(dst, int):
+        dst_p, dst0 = None, dst
+    else:
+        if dst.dtype != torch.int64 or not dst.is_cuda or dst.numel() != n:
+            raise ValueError("dst must be an int or an int64 CUDA tensor [n]")
+        dst_p, dst0 = vp(dst.data_ptr()), 0
+    st = lib().attn_append_kv(vp(k_new.data_ptr()), vp(v_new.data_ptr()), dtype_code(k_new), n, cos_p, sin_p,
+                              vp(k_cache.data_ptr()), vp(v_cache.data_ptr()), dtype_code(k_cache),
+                              k_cache.numel() // HEAD_DIM, dst_p, dst0,
+                              vp(workspace.data_ptr()) if workspace is not None else None,
+                              _stream_ptr(stream))
+    _check(st, "attn_append_kv")
 
 
 def attn_decode_static(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.0 / 16.0,

@@ -19,13 +19,15 @@ namespace kca {
 
 // Status word layout (first 256 bytes of the workspace).
 struct DeviceStatus {
-  unsigned int error;   // bit 0: a bounded wait ran out; bit 1: a device ctx_len out of range
+  unsigned int error;   // bit 0: a bounded wait ran out; bit 1: a device ctx_len out of range;
+                        // bit 2: a device destination row out of range (append)
   unsigned int detail;  // (site << 24) | (block & 0xffffff) of the first failure
 };
-enum : unsigned int { kErrWaitTimeout = 1u, kErrBadCtx = 2u };
+enum : unsigned int { kErrWaitTimeout = 1u, kErrBadCtx = 2u, kErrBadRow = 4u };
 enum : unsigned int {
   kSiteRowsFull = 1, kSiteRowsEmpty = 2, kSiteTcFull = 3, kSiteTcEmpty = 4, kSiteTcS = 5,
-  kSiteTcP = 6, kSiteTcO = 7, kSiteTcQ = 8, kSiteTcDrain = 9, kSiteCtx = 10
+  kSiteTcP = 6, kSiteTcO = 7, kSiteTcQ = 8, kSiteTcDrain = 9, kSiteCtx = 10,
+  kSiteAppend = 11
 };
 
 // Records the first failure (detail: site and the block's x index, or the

@@ -118,6 +118,26 @@ def test_decode_dev_rejects_bad_arguments_on_the_host(kw, code):
     assert _decode_dev(**kw) == code
 
 
+def _append(**kw):
+    a = dict(k=P, v=P, it=kca.F32, n=4, cos=P * 3, sin=P * 4, kc=P * 5, vc=P * 6, kt=kca.F16, rows=100,
+             dst=None, dst0=0, ws=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return kca.lib().attn_append_kv(vp(a["k"]), vp(a["v"]), a["it"], a["n"], vp(a["cos"]), vp(a["sin"]),
+                                    vp(a["kc"]), vp(a["vc"]), a["kt"], a["rows"], vp(a["dst"]),
+                                    a["dst0"], vp(a["ws"]), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), -1), (dict(vc=0), -1), (dict(cos=0), -1), (dict(sin=0), -1),
+    (dict(it=3), -3), (dict(kt=-1), -3),
+    (dict(n=0), -4), (dict(rows=0), -4), (dict(dst0=-1), -4), (dict(dst0=97), -4),
+    (dict(k=P + 8), -6), (dict(kc=P * 5 + 2), -6), (dict(cos=P * 3 + 4), -6), (dict(dst=P * 7 + 4), -6),
+])
+def test_append_rejects_bad_arguments_on_the_host(kw, code):
+    assert _append(**kw) == code
+
+
 def _check_rows_plan(items, units, pos_of, window):
     """Every unit's items tile its visible range exactly, in order, slots unique."""
     slots = [int(s) for s in items[:, 3] if s >= 0]
