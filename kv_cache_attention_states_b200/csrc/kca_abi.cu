@@ -136,6 +136,24 @@ bool encode_kv_map(CUtensorMap* m, const void* cache, int32_t dtype, int64_t kv_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over `rows` rows of 256 elements (f32 or 16-bit), box {box_x, 128},
+// 128-byte swizzle; reads past the extent return zeros, stores are clipped.
+bool encode_rows_map(CUtensorMap* m, const void* base, int32_t dtype, int64_t rows, uint32_t box_x) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr || rows < 1) return false;
+  const int esz = dtype == KCA_F32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kDim * esz};
+  cuuint32_t box[2] = {box_x, 128};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType t = dtype == KCA_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : dtype == KCA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(m, t, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 void carve(void* ws, size_t ml_bytes, float** ml, float** acc) {
   char* p = static_cast<char*>(ws) + KCA_WORKSPACE_HEADER;
   *ml = reinterpret_cast<float*>(p);
@@ -417,12 +435,21 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
     a.scale_log2 = scale * 1.4426950408889634f;
     carve(workspace, (size_t)a.plan.n_slots * 128 * 2 * 4, &a.part_ml, &a.part_acc);
     kca::fill_tc_tables(a);
-    CUtensorMap tmk, tmv;
-    // K: one 64-dim chunk of a 128-key tile per box; V: 64-key halves.
+    CUtensorMap tmk, tmv, tmq, tmo, tmpart;
+    // K: one 64-dim chunk of a 128-key tile per box; V: 64-key halves; Q in
+    // 64-dim boxes of a 128-row tile; out / partials in 32-column boxes.
     if (!encode_kv_map(&tmk, k_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, kca::kKeyTile) ||
-        !encode_kv_map(&tmv, v_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, 64))
+        !encode_kv_map(&tmv, v_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, 64) ||
+        !encode_rows_map(&tmq, q_chunk, q_dtype, (int64_t)chunk_rows * kHeads, 64) ||
+        !encode_rows_map(&tmo, out, KCA_F32, (int64_t)chunk_rows * kHeads, 32))
       return KCA_ERR_CUDA;
-    return kca::launch_prefill_tc(kv_dtype, tmk, tmv, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+    if (a.plan.n_slots > 0) {
+      if (!encode_rows_map(&tmpart, a.part_acc, KCA_F32, (int64_t)a.plan.n_slots * 128, 32)) return KCA_ERR_CUDA;
+    } else {
+      tmpart = tmo;   // no split tile: never used
+    }
+    return kca::launch_prefill_tc(kv_dtype, tmk, tmv, tmq, tmo, tmpart, a, s) == cudaSuccess ? KCA_OK
+                                                                                           : KCA_ERR_CUDA;
   }
 
   const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);

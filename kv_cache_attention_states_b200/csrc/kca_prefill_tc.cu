@@ -58,6 +58,11 @@ constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKRing * kKSlotBytes;    // 64 KiB
 constexpr int kOffP = kOffV + kVRing * kVHalfBytes;    // 128 KiB
 constexpr int kOffBar = kOffP + 2 * kPBytes;           // 192 KiB
+constexpr int kQBoxBytes = 128 * 64 * 2;               // Q: 128 M rows x 64 dims, 16 KiB
+constexpr int kQBytes = 4 * kQBoxBytes;                // the whole Q tile over the P buffers
+constexpr int kOBoxBytes = 128 * 32 * 4;               // O: 128 M rows x 32 f32, 16 KiB
+static_assert(kQBytes == 2 * kPBytes, "Q tile fills the P buffers");
+static_assert(8 * kOBoxBytes <= kOffP, "O tile fits the K/V rings");
 constexpr int kBarBytes = 4096;
 constexpr int kSmemBytes = kOffBar + kBarBytes + 1024; // + alignment slack
 constexpr uint32_t kTmemCols = 512;
@@ -68,6 +73,7 @@ constexpr int kSoftmaxThreads = 256;
 struct Bars {
   uint64_t kfull[kKRing], kempty[kKRing];
   uint64_t vfull[kVRing], vempty[kVRing];
+  uint64_t q_tma;      // Q tile landed in shared memory (TMA, over the P buffers)
   uint64_t q_full;     // Q in TMEM (256 softmax threads)
   uint64_t s_full;     // S of the current tile computed (MMA commit)
   uint64_t s_free;     // S copied to registers by all 256 softmax threads
@@ -103,7 +109,8 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                      const TcArgs a) {
+                      const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
+                      const __grid_constant__ CUtensorMap tmpart, const TcArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -128,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->vfull[i], 1);
       mbar_init(&bars->vempty[i], 1);
     }
+    mbar_init(&bars->q_tma, 1);
     mbar_init(&bars->q_full, kSoftmaxThreads);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, kSoftmaxThreads);
@@ -157,6 +165,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* full = is_k ? bars->kfull : bars->vfull;
       uint64_t* empty = is_k ? bars->kempty : bars->vempty;
       ptx::prefetch_tmap(is_k ? &tmk : &tmv);
+      if (is_k) {
+        // Q tile: 128 M rows x 256 dims as four 64-dim boxes (128-byte
+        // swizzle) into the P buffers, which are unused until the first P.
+        ptx::prefetch_tmap(&tmq);
+        mbar_arrive_expect_tx(&bars->q_tma, kQBytes);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          ptx::tma_load_2d(sbase + kOffP + i * kQBoxBytes, &tmq, 64 * i, it.tile * 128, smem_u32(&bars->q_tma));
+      } else {
+        ptx::prefetch_tmap(&tmo);
+        ptx::prefetch_tmap(&tmpart);
+      }
       const int per_tile = 2;   // K: two slots of two 64-dim chunks, V: two 64-key halves
       int e = 0;
       bool ok = true;
@@ -264,15 +284,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t pos = a.plan.chunk_start + row;
     const int64_t lo = lo_of(pos, a.plan.window);
 
-    // Q row (row, head m & 7), dims [128 wg, 128 wg + 128), into TMEM; zeros past the chunk.
+    // Q row (row, head m & 7), dims [128 wg, 128 wg + 128), from the TMA
+    // boxes in shared memory into TMEM (rows past the chunk arrive as zeros).
     {
-      const uint4* qsrc = reinterpret_cast<const uint4*>(a.q) + ((int64_t)it.tile * 128 + m) * 32 + wg * 16;
+      const bool qok = mbar_wait(&bars->q_tma, 0, abort_flag, status, kSiteTcQ);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
+        const unsigned char* box = smem + kOffP + (2 * wg + c) * kQBoxBytes + m * 128;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint4 v = valid ? qsrc[c * 8 + i] : make_uint4(0, 0, 0, 0);
+          const uint4 v = qok ? *reinterpret_cast<const uint4*>(box + ((i ^ (m & 7)) << 4)) : make_uint4(0, 0, 0, 0);
           r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
         }
         ptx::tmem_st32(trow + kColQ + 64 * wg + 32 * c, r);
@@ -390,34 +412,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->red_max[n & 1][wg][m] = l_sum;
     named_sync(1, kSoftmaxThreads);
     const float l_tot = l_sum + bars->red_max[n & 1][wg ^ 1][m];
+    // Epilogue: O (scaled by 1/l, or raw for a partial) goes from TMEM to
+    // shared memory as eight 32-column boxes with 128-byte swizzle (the K/V
+    // rings are free once every PV is done), then out by TMA stores: the
+    // tile's 128 rows are one contiguous block of out or of the partials,
+    // and rows past the chunk fall outside the map and are not written.
     if (ok) {
       ptx::fence_after_sync();
-      float* dst;
-      if (it.slot < 0) {
-        dst = a.out + ((int64_t)it.tile * 128 + m) * kDim + 128 * wg;
-      } else {
-        dst = a.part_acc + ((int64_t)it.slot * 128 + m) * kDim + 128 * wg;
-        if (wg == 0) {
-          a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 0] = m_ref;
-          a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 1] = l_tot;
-        }
+      if (it.slot >= 0 && wg == 0 && valid) {
+        a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 0] = m_ref;
+        a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 1] = l_tot;
       }
       const float f = it.slot < 0 ? 1.f / l_tot : 1.f;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         ptx::tmem_ld32(trow + kColO + 128 * wg + 32 * c, r);
         ptx::tmem_wait_ld();
-        if (valid) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+        unsigned char* box = smem + (4 * wg + c) * kOBoxBytes + m * 128;
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(__uint_as_float(r[4 * i]) * f, __uint_as_float(r[4 * i + 1]) * f,
-                                __uint_as_float(r[4 * i + 2]) * f, __uint_as_float(r[4 * i + 3]) * f);
-        }
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<float4*>(box + ((i ^ (m & 7)) << 4)) =
+              make_float4(__uint_as_float(r[4 * i]) * f, __uint_as_float(r[4 * i + 1]) * f,
+                          __uint_as_float(r[4 * i + 2]) * f, __uint_as_float(r[4 * i + 3]) * f);
       }
+      fence_proxy_async_smem();   // generic-proxy stores -> visible to the TMA unit
     }
     ptx::fence_before_sync();
+    named_sync(1, kSoftmaxThreads);
+    if (ok && threadIdx.x == 4 * 32) {
+      const void* map = it.slot < 0 ? static_cast<const void*>(&tmo) : static_cast<const void*>(&tmpart);
+      const int32_t y = (it.slot < 0 ? (int32_t)it.tile : (int32_t)it.slot) * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ptx::tma_store_2d(map, 32 * j, y, sbase + j * kOBoxBytes);
+      ptx::bulk_commit();
+      ptx::bulk_wait_all();   // shared memory stays allocated until the stores are done
+    }
   }
 
   __syncthreads();
@@ -448,8 +478,8 @@ __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
 }
 
 template <int DT>
-cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const TcArgs& a,
-                     cudaStream_t stream) {
+cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmq,
+                     const CUtensorMap& tmo, const CUtensorMap& tmpart, const TcArgs& a, cudaStream_t stream) {
   static bool attr_set[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -459,7 +489,7 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const TcArg
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  prefill_tc_kernel<DT><<<a.plan.n_items, kThreads, kSmemBytes, stream>>>(tmk, tmv, a);
+  prefill_tc_kernel<DT><<<a.plan.n_items, kThreads, kSmemBytes, stream>>>(tmk, tmv, tmq, tmo, tmpart, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.plan.n_slots == 0) return e;
   const int ns = a.plan.max_split;
@@ -495,9 +525,10 @@ void fill_tc_tables(TcArgs& a) {
 }
 
 cudaError_t launch_prefill_tc(int dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                              const CUtensorMap& tmq, const CUtensorMap& tmo, const CUtensorMap& tmpart,
                               const TcArgs& a, cudaStream_t stream) {
-  if (dtype == KCA_BF16) return launch_t<KCA_BF16>(tmk, tmv, a, stream);
-  if (dtype == KCA_F16) return launch_t<KCA_F16>(tmk, tmv, a, stream);
+  if (dtype == KCA_BF16) return launch_t<KCA_BF16>(tmk, tmv, tmq, tmo, tmpart, a, stream);
+  if (dtype == KCA_F16) return launch_t<KCA_F16>(tmk, tmv, tmq, tmo, tmpart, a, stream);
   return cudaErrorInvalidValue;
 }
 

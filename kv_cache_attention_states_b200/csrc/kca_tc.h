@@ -38,8 +38,11 @@ void fill_tc_tables(TcArgs& a);
 
 // tmk / tmv: 2-D tensor maps over the rows [plan.kv_lo, plan.ctx_len) of the
 // K and V caches, inner extent 256, 128-byte swizzle, zero fill; boxes of 64
-// elements x 128 rows (K) and 64 x 64 (V).
+// elements x 128 rows (K) and 64 x 64 (V).  tmq: the Q chunk as [rows * 8][256]
+// 16-bit, boxes 64 x 128.  tmo / tmpart: out as [rows * 8][256] f32 and the
+// partials as [n_slots * 128][256] f32, boxes 32 x 128; all 128-byte swizzle.
 cudaError_t launch_prefill_tc(int dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                              const CUtensorMap& tmq, const CUtensorMap& tmo, const CUtensorMap& tmpart,
                               const TcArgs& a, cudaStream_t stream);
 
 }  // namespace kca
