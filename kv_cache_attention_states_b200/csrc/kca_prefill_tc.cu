@@ -156,6 +156,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
+  // Programmatic dependent launch: the set-up above overlaps the previous
+  // kernel of the stream; global memory is touched only after this wait.
+  // The next kernel may be scheduled as soon as SMs free up.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0 || warp == 2) {
     // ------------------------------------------------------------ producers
@@ -463,6 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int W>
 __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
   constexpr int kRowsPerCta = 8 / W;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tile = blockIdx.x;
   const int ns = a.tile_items[tile];
   if (ns <= 1) return;
@@ -489,17 +496,28 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  prefill_tc_kernel<DT><<<a.plan.n_items, kThreads, kSmemBytes, stream>>>(tmk, tmv, tmq, tmo, tmpart, a);
-  cudaError_t e = cudaGetLastError();
+  // Both kernels allow programmatic dependent launch (see griddepcontrol).
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.plan.n_items);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<DT>, tmk, tmv, tmq, tmo, tmpart, a);
   if (e != cudaSuccess || a.plan.n_slots == 0) return e;
   const int ns = a.plan.max_split;
   const int w = ns > 8 ? 8 : (ns > 4 ? 4 : (ns > 2 ? 2 : 1));
-  const dim3 grid(a.plan.n_tiles, 16 * w);
-  if (w == 8) merge_tc_kernel<8><<<grid, 256, 0, stream>>>(a);
-  else if (w == 4) merge_tc_kernel<4><<<grid, 256, 0, stream>>>(a);
-  else if (w == 2) merge_tc_kernel<2><<<grid, 256, 0, stream>>>(a);
-  else merge_tc_kernel<1><<<grid, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  cfg.gridDim = dim3(a.plan.n_tiles, 16 * w);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  if (w == 8) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<8>, a);
+  if (w == 4) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<4>, a);
+  if (w == 2) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<2>, a);
+  return cudaLaunchKernelEx(&cfg, merge_tc_kernel<1>, a);
 }
 
 }  // namespace
