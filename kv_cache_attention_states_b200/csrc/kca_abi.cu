@@ -297,17 +297,19 @@ int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, in
   int32_t count = 0;
   if (use_tc(q_dtype, kv_dtype, chunk_rows)) {
     *path = 1;
-    const kca::TcPlan p = kca::make_tc_plan(chunk_start, chunk_rows, window, num_sms);
-    for (int32_t i = 0; i < p.n_items; ++i, ++count) {
-      if (count >= max_items) continue;
+    const kca::TcPlan p = kca::make_tc_plan(chunk_start, chunk_rows, window, num_sms / 2);
+    for (int32_t i = 0; i < p.n_items; ++i) {
       const kca::TcItem it = kca::tc_item(p, i);
       int64_t kb = p.kv_lo + (int64_t)it.kt_begin * kca::kKeyTile;
       int64_t ke = p.kv_lo + (int64_t)it.kt_end * kca::kKeyTile;
       if (ke > p.ctx_len) ke = p.ctx_len;
-      items[4 * count + 0] = it.tile;
-      items[4 * count + 1] = kb;
-      items[4 * count + 2] = ke;
-      items[4 * count + 3] = it.slot;
+      for (int32_t r = 0; r < kca::tc_pair_tiles(p, it.pair); ++r, ++count) {   // one entry per tile of the pair
+        if (count >= max_items) continue;
+        items[4 * count + 0] = 2 * it.pair + r;
+        items[4 * count + 1] = kb;
+        items[4 * count + 2] = ke;
+        items[4 * count + 3] = r == 0 ? it.slot0 : it.slot1;
+      }
     }
   } else {
     *path = 0;
@@ -368,7 +370,7 @@ size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t c
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return 0;
   if (use_tc(q_dtype, kv_dtype, chunk_rows))
-    return tc_ws_bytes(kca::make_tc_plan(chunk_start, chunk_rows, window, sms));
+    return tc_ws_bytes(kca::make_tc_plan(chunk_start, chunk_rows, window, sms / 2));
   const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
   return rows_ws_bytes_any(chunk_rows, nk.data(), sms);
 }
@@ -427,7 +429,7 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
 
   if (use_tc(q_dtype, kv_dtype, chunk_rows)) {
     kca::TcArgs a{};
-    a.plan = kca::make_tc_plan(chunk_start, chunk_rows, window, sms);
+    a.plan = kca::make_tc_plan(chunk_start, chunk_rows, window, sms / 2);
     if (workspace_bytes < tc_ws_bytes(a.plan)) return KCA_ERR_WORKSPACE;
     a.q = q_chunk;
     a.out = out;
@@ -436,9 +438,9 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
     carve(workspace, (size_t)a.plan.n_slots * 128 * 2 * 4, &a.part_ml, &a.part_acc);
     kca::fill_tc_tables(a);
     CUtensorMap tmk, tmv, tmq, tmo, tmpart;
-    // K: one 64-dim chunk of a 128-key tile per box; V: 64-key halves; Q in
-    // 64-dim boxes of a 128-row tile; out / partials in 32-column boxes.
-    if (!encode_kv_map(&tmk, k_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, kca::kKeyTile) ||
+    // K and V: 64 x 64 boxes (each CTA of a pair loads its half of a tile);
+    // Q in 64-dim boxes of a 128-row tile; out / partials in 32-column boxes.
+    if (!encode_kv_map(&tmk, k_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, 64) ||
         !encode_kv_map(&tmv, v_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, 64) ||
         !encode_rows_map(&tmq, q_chunk, q_dtype, (int64_t)chunk_rows * kHeads, 64) ||
         !encode_rows_map(&tmo, out, KCA_F32, (int64_t)chunk_rows * kHeads, 32))

@@ -27,7 +27,7 @@ enum : unsigned int { kErrWaitTimeout = 1u, kErrBadCtx = 2u, kErrBadRow = 4u };
 enum : unsigned int {
   kSiteRowsFull = 1, kSiteRowsEmpty = 2, kSiteTcFull = 3, kSiteTcEmpty = 4, kSiteTcS = 5,
   kSiteTcP = 6, kSiteTcO = 7, kSiteTcQ = 8, kSiteTcDrain = 9, kSiteCtx = 10,
-  kSiteAppend = 11
+  kSiteAppend = 11, kSiteTcAlign = 12
 };
 
 // Records the first failure (detail: site and the block's x index, or the

@@ -129,9 +129,12 @@ inline RowsPlan make_cluster_rows_plan(int32_t n_units, const int64_t* nkeys, in
 // A chunk of `rows` query rows at chunk_start is cut into row tiles of 16
 // positions (x 8 heads = 128 M rows).  Keys are addressed relative to
 // kv_lo = lo(chunk_start), the first key any row of the chunk sees, in tiles
-// of 128.  Row tile t covers key tiles [kb(t), ke(t)); it is split into
-// ceil(n/c) items of near-equal length, c chosen as the smallest value that
-// keeps the item count within one wave of CTAs.
+// of 128.  Row tiles go in pairs (2q, 2q+1) to the two SMs of a CTA pair,
+// which share every K/V tile (each SM loads half of it); a pair covers the
+// union of its tiles' key ranges [kb(2q), ke(2q+1)), each row masking the
+// keys it does not see.  A pair's range is split into ceil(n/c) items of
+// near-equal length, c chosen as the smallest value that keeps the pair
+// items within one wave of CTA pairs.
 struct TcPlan {
   int64_t chunk_start;
   int64_t kv_lo;
@@ -139,10 +142,11 @@ struct TcPlan {
   int32_t rows;
   int32_t window;
   int32_t n_tiles;
+  int32_t n_pairs;
   int32_t per_item;     // c: most key tiles one item covers
-  int32_t n_items;
-  int32_t n_slots;      // items that belong to split tiles (write partials)
-  int32_t max_split;    // most items of one tile
+  int32_t n_items;      // pair items (each runs on a CTA pair)
+  int32_t n_slots;      // partial slots: one per (tile, item) of split pairs
+  int32_t max_split;    // most items of one pair
 };
 
 constexpr int kTcMinItemTiles = 2;
@@ -155,58 +159,63 @@ KCA_HD void tc_tile_keys(const TcPlan& p, int32_t t, int32_t* kb, int32_t* ke) {
   *kb = (int32_t)((lo_of(first, p.window) - p.kv_lo) / kKeyTile);
   *ke = (int32_t)((last - p.kv_lo) / kKeyTile + 1);
 }
-KCA_HD int32_t tc_tile_items(const TcPlan& p, int32_t t) {
+KCA_HD int32_t tc_pair_tiles(const TcPlan& p, int32_t q) { return 2 * q + 1 < p.n_tiles ? 2 : 1; }
+// Key tiles [kb, ke) of pair q: the union of its tiles' ranges (lo and the
+// last position both grow with the tile index).
+KCA_HD void tc_pair_keys(const TcPlan& p, int32_t q, int32_t* kb, int32_t* ke) {
+  int32_t kb1, ke1;
+  tc_tile_keys(p, 2 * q, kb, ke);
+  if (tc_pair_tiles(p, q) == 2) {
+    tc_tile_keys(p, 2 * q + 1, &kb1, &ke1);
+    *ke = ke1;
+  }
+}
+KCA_HD int32_t tc_pair_items(const TcPlan& p, int32_t q) {
   int32_t kb, ke;
-  tc_tile_keys(p, t, &kb, &ke);
+  tc_pair_keys(p, q, &kb, &ke);
   return (int32_t)cdiv(ke - kb, p.per_item);
 }
 
 struct TcItem {
-  int32_t tile;
+  int32_t pair;
   int32_t kt_begin;   // key tiles, relative to kv_lo
   int32_t kt_end;
-  int32_t slot;       // partial slot, -1 when the tile is not split
-  int32_t split;      // index within the tile
+  int32_t slot0;      // partial slot of tile 2 pair, -1 when the pair is not split
+  int32_t slot1;      // partial slot of tile 2 pair + 1 (-1 also when that tile does not exist)
+  int32_t split;      // index within the pair
   int32_t n_split;
 };
 
-// Item `idx` of the plan (items ordered by tile, then by split).
+// Item `idx` of the plan (items ordered by pair, then by split).
 KCA_HD TcItem tc_item(const TcPlan& p, int32_t idx) {
   TcItem it{};
   int32_t base = 0, slot_base = 0;
-  for (int32_t t = 0; t < p.n_tiles; ++t) {
+  for (int32_t q = 0; q < p.n_pairs; ++q) {
     int32_t kb, ke;
-    tc_tile_keys(p, t, &kb, &ke);
+    tc_pair_keys(p, q, &kb, &ke);
     const int32_t n = ke - kb;
     const int32_t s = (int32_t)cdiv(n, p.per_item);
+    const int32_t nt = tc_pair_tiles(p, q);
     if (idx < base + s) {
       const int32_t k = idx - base;
-      it.tile = t;
+      it.pair = q;
       it.kt_begin = kb + (int32_t)(((int64_t)k * n) / s);
       it.kt_end = kb + (int32_t)(((int64_t)(k + 1) * n) / s);
       it.split = k;
       it.n_split = s;
-      it.slot = s > 1 ? slot_base + k : -1;
+      it.slot0 = s > 1 ? slot_base + k : -1;
+      it.slot1 = (s > 1 && nt == 2) ? slot_base + s + k : -1;
       return it;
     }
     base += s;
-    if (s > 1) slot_base += s;
+    if (s > 1) slot_base += s * nt;
   }
-  it.tile = -1;
+  it.pair = -1;
   return it;
 }
 
-// First partial slot of tile t (meaningful when the tile is split).
-KCA_HD int32_t tc_tile_first_slot(const TcPlan& p, int32_t tile) {
-  int32_t slot_base = 0;
-  for (int32_t t = 0; t < tile; ++t) {
-    const int32_t s = tc_tile_items(p, t);
-    if (s > 1) slot_base += s;
-  }
-  return slot_base;
-}
-
-inline TcPlan make_tc_plan(int64_t chunk_start, int32_t rows, int32_t window, int32_t num_sms) {
+// pair_budget: CTA pairs that run at once (one wave).
+inline TcPlan make_tc_plan(int64_t chunk_start, int32_t rows, int32_t window, int32_t pair_budget) {
   TcPlan p{};
   p.chunk_start = chunk_start;
   p.rows = rows;
@@ -214,29 +223,30 @@ inline TcPlan make_tc_plan(int64_t chunk_start, int32_t rows, int32_t window, in
   p.kv_lo = lo_of(chunk_start, window);
   p.ctx_len = chunk_start + rows;
   p.n_tiles = (int32_t)cdiv(rows, kRowTile);
+  p.n_pairs = (int32_t)cdiv(p.n_tiles, 2);
   int64_t total = 0;
   int32_t longest = 1;
-  for (int32_t t = 0; t < p.n_tiles; ++t) {
+  for (int32_t q = 0; q < p.n_pairs; ++q) {
     int32_t kb, ke;
-    tc_tile_keys(p, t, &kb, &ke);
+    tc_pair_keys(p, q, &kb, &ke);
     total += ke - kb;
     if (ke - kb > longest) longest = ke - kb;
   }
-  // one wave of CTAs, capped by the launch's item table (160 entries)
-  const int32_t sms = num_sms < 1 ? 1 : (num_sms > 160 ? 160 : num_sms);
-  int32_t c = (int32_t)cdiv(total, sms);
+  // one wave of CTA pairs, capped by the launch's item table (80 entries)
+  const int32_t budget = pair_budget < 1 ? 1 : (pair_budget > 80 ? 80 : pair_budget);
+  int32_t c = (int32_t)cdiv(total, budget);
   if (c < kTcMinItemTiles) c = kTcMinItemTiles;
   for (;; ++c) {
     p.per_item = c;
     int64_t items = 0;
-    for (int32_t t = 0; t < p.n_tiles; ++t) items += tc_tile_items(p, t);
-    if (items <= sms || c >= longest) break;
+    for (int32_t q = 0; q < p.n_pairs; ++q) items += tc_pair_items(p, q);
+    if (items <= budget || c >= longest) break;
   }
   int32_t items = 0, slots = 0, most = 1;
-  for (int32_t t = 0; t < p.n_tiles; ++t) {
-    const int32_t s = tc_tile_items(p, t);
+  for (int32_t q = 0; q < p.n_pairs; ++q) {
+    const int32_t s = tc_pair_items(p, q);
     items += s;
-    if (s > 1) slots += s;
+    if (s > 1) slots += s * tc_pair_tiles(p, q);
     if (s > most) most = s;
   }
   p.n_items = items;

@@ -3,31 +3,37 @@
 // The pages' design (Karume v0.12.0 release notes, "Performance", item 1):
 // for plans of 16 or more chunk rows, QK and PV run on a GEMM tile skeleton
 // so that each K / V row is read once per row tile instead of once per query
-// row.  Here one CTA takes one work item -- a row tile of 16 positions x 8
-// heads (M = 128: the 8 heads share their single KV head) and a run of
-// 128-key tiles -- and fuses the three stages the pages keep apart (QK,
-// softmax statistics, PV), so no score matrix ever reaches memory.
+// row.  Here a CTA pair (a cluster of two CTAs on two SMs) takes one work
+// item -- two row tiles of 16 positions x 8 heads (M = 128 each: the 8 heads
+// share their single KV head) and a run of 128-key tiles -- and fuses the
+// three stages the pages keep apart (QK, softmax statistics, PV), so no
+// score matrix ever reaches memory.
 //
-// Warp roles (12 warps):
-//   warp 0      TMA producer of K: each 128-key tile as four 64-dim chunks
-//               (128 rows x 128 B, 128-byte swizzle), two chunks per slot of
-//               a 2-slot ring
-//   warp 1      TMEM allocator and the single MMA-issuing thread
-//   warp 2      TMA producer of V: 64-key halves (four 64 x 64 boxes) into a
-//               2-slot ring
+// Why pairs: one SM pulls at most ~53 bytes per clock from L2 by TMA, while
+// a 128-key K + V tile (128 KiB) feeds 2048 clocks of MMA -- 64 B/clk.  With
+// tcgen05 MMAs of M = 256 over the pair (cta_group::2) each SM loads only its
+// half of every K and V tile (B is split along N), so the tensor pipe, not
+// the L2 stream, sets the pace.
+//
+// Warp roles (12 warps per CTA):
+//   warp 0      TMA producer: the CTA's Q tile once, then its half of every
+//               K tile (64 keys x 256 dims as four 64 x 64 boxes)
+//   warp 1      TMEM allocator (both CTAs); in the even CTA the single thread
+//               that issues every MMA of the pair
+//   warp 2      TMA producer of its half of every V tile (128 keys x 128 dims)
 //   warps 4-7   softmax warpgroup 0: keys 0-63 of every S tile
 //   warps 8-11  softmax warpgroup 1: keys 64-127
-//   Thread m of a softmax warpgroup owns TMEM lane m, i.e. M row m.
+//   Thread m of a softmax warpgroup owns TMEM lane m, i.e. M row m of its CTA.
 //
-// Tensor memory (512 columns x 128 lanes of 32 bits):
-//   [  0,128)  Q tile as 16-bit pairs: the A operand of S = Q K^T
+// Operands: S = Q K^T with Q (A) and K (B) in shared memory; O += P V with P
+// (A) in tensor memory and V (B) in shared memory.  Tensor memory per CTA
+// (512 columns x 128 lanes of 32 bits):
+//   [  0,128)  P of tiles t (even / odd) as 16-bit pairs, 64 columns each
 //   [128,256)  S (f32, 128 keys), released as soon as both warpgroups hold
 //              their half in registers, so QK^T of the next tile overlaps
 //              the softmax of this one
 //   [256,512)  O accumulator (f32, 256 dims)
-// P (16-bit) goes to shared memory, double-buffered, as the A operand of
-// O += P V.  Shapes per instruction: QK^T M128 N128 K16, PV M128 N256 K16;
-// both keep the tensor pipe at full rate from a single issuing thread.
+// Shapes per instruction: QK^T M256 N128 K16, PV M256 N256 K16 over the pair.
 //
 // The softmax keeps a reference max per row and rescales O (in TMEM) only
 // when a score exceeds it by more than 2^8, so probabilities stay <= 256 and
@@ -47,40 +53,48 @@ namespace kca {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kKRing = 2;                              // K slots of two 64-dim chunks
-constexpr int kVRing = 2;                              // V half-tile slots
-constexpr int kKChunkBytes = kKeyTile * 64 * 2;        // 128 keys x 64 dims: 16 KiB
-constexpr int kKSlotBytes = 2 * kKChunkBytes;          // two chunks: 32 KiB
+// Per CTA of a pair: its half of every K tile (64 of the 128 keys, all 256
+// dims) and of every V tile (128 of the 256 dims, all 128 keys).
+constexpr int kKRing = 2;                              // K tile halves
+constexpr int kVRing = 2;                              // V tile halves
+constexpr int kKChunkBytes = 64 * 64 * 2;              // 64 keys x 64 dims: 8 KiB
+constexpr int kKSlotBytes = 4 * kKChunkBytes;          // 64 keys x 256 dims: 32 KiB
 constexpr int kVBoxBytes = 64 * 64 * 2;                // 64 keys x 64 dims: 8 KiB
-constexpr int kVHalfBytes = 4 * kVBoxBytes;            // 64 keys x 256 dims: 32 KiB
-constexpr int kPBytes = 128 * kKeyTile * 2;            // 128 rows x 128 keys: 32 KiB
+constexpr int kVSlotBytes = 4 * kVBoxBytes;            // 128 keys x 128 dims: 32 KiB
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKRing * kKSlotBytes;    // 64 KiB
-constexpr int kOffP = kOffV + kVRing * kVHalfBytes;    // 128 KiB
-constexpr int kOffBar = kOffP + 2 * kPBytes;           // 192 KiB
+constexpr int kOffQ = kOffV + kVRing * kVSlotBytes;    // 128 KiB
 constexpr int kQBoxBytes = 128 * 64 * 2;               // Q: 128 M rows x 64 dims, 16 KiB
-constexpr int kQBytes = 4 * kQBoxBytes;                // the whole Q tile over the P buffers
+constexpr int kQBytes = 4 * kQBoxBytes;                // the CTA's Q tile, resident for the whole item
+constexpr int kOffBar = kOffQ + kQBytes;               // 192 KiB
 constexpr int kOBoxBytes = 128 * 32 * 4;               // O: 128 M rows x 32 f32, 16 KiB
-static_assert(kQBytes == 2 * kPBytes, "Q tile fills the P buffers");
-static_assert(8 * kOBoxBytes <= kOffP, "O tile fits the K/V rings");
+static_assert(8 * kOBoxBytes <= kOffQ, "O tile fits the K/V rings");
 constexpr int kBarBytes = 4096;
 constexpr int kSmemBytes = kOffBar + kBarBytes + 1024; // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColQ = 0, kColS = 128, kColO = 256;
+// TMEM: P of tile t (16-bit pairs, the A operand of P V) in buffer t&1 at
+// columns [64 (t&1), +64), S at [128, 256), O at [256, 512).
+constexpr uint32_t kColP = 0, kColS = 128, kColO = 256;
 constexpr float kRescaleLog2 = 8.f;  // rescale O once a score passes the reference by 2^8
 constexpr int kSoftmaxThreads = 256;
+constexpr uint32_t kPairArrivals = 2 * kSoftmaxThreads / 32;  // one per softmax warp of both CTAs
+constexpr uint16_t kPairMask = 3;    // both CTAs of the cluster
 
+// Barriers.  The even CTA ("leader") issues every MMA of the pair, so the
+// barriers it waits on (kfull, vfull, q_full, s_free, p_full) live in its
+// shared memory and collect arrivals / bytes from both CTAs; the ones the
+// MMAs signal (kempty, vempty, s_full, o_done, o_final, drain) are
+// multicast to the same offset in both CTAs.
 struct Bars {
   uint64_t kfull[kKRing], kempty[kKRing];
   uint64_t vfull[kVRing], vempty[kVRing];
-  uint64_t q_tma;      // Q tile landed in shared memory (TMA, over the P buffers)
-  uint64_t q_full;     // Q in TMEM (256 softmax threads)
+  uint64_t q_full;     // both CTAs' Q tiles landed in shared memory (TMA bytes)
   uint64_t s_full;     // S of the current tile computed (MMA commit)
-  uint64_t s_free;     // S copied to registers by all 256 softmax threads
-  uint64_t p_full[2];  // P of tile t in buffer t&1 written, O corrected (256 threads)
+  uint64_t s_free;     // S copied to registers by all 16 softmax warps
+  uint64_t p_full[2];  // P of tile t in TMEM buffer t&1 written, O corrected (16 warps)
   uint64_t o_done[2];  // PV of tile u complete (MMA commit), u&1 selects the barrier
   uint64_t o_final;    // every PV complete (single use)
-  uint64_t drain;      // every MMA complete (single use, MMA thread)
+  uint64_t drain;      // every MMA complete (single use)
   uint32_t tmem_base;
   int abort;
   float red_max[2][2][128];  // [tile parity][warpgroup][row]: partial row maxima
@@ -88,6 +102,30 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= kBarBytes, "barrier block too large");
 static_assert(kSmemBytes <= 232448, "shared memory over the per-CTA limit");
+
+// ---- CTA-pair helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void pair_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The leader's copy of a barrier (shared-memory address with the pair bit
+// cleared, as the 2-SM TMA and arrive forms expect).
+__device__ __forceinline__ uint32_t leader_bar(const uint64_t* bar) { return smem_u32(bar) & 0xFEFFFFFFu; }
+// One arrival per warp on a barrier of the leader CTA, once the warp's lanes
+// have synchronised.  The softmax warps signal only tensor-memory accesses
+// that every lane has already waited for (tcgen05.wait::ld / ::st, then
+// tcgen05.fence::before_thread_sync), so the arrival needs no release
+// semantics -- a release at cluster scope would cost ~700 cycles on the
+// critical path of every tile.
+__device__ __forceinline__ void arrive_leader(const uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0)
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(leader_bar(bar)) : "memory");
+}
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, int dt) {
   if (dt == KCA_BF16) {
@@ -122,9 +160,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const TcItemArg it = a.items[blockIdx.x];
-  const int n = it.kt_end - it.kt_begin;
-  if (n <= 0) return;  // the host never launches such a CTA
+  const uint32_t rank = cluster_rank();           // 0: leader (issues the MMAs), 1: its peer
+  const bool leader = rank == 0;
+  const TcItemArg it = a.items[blockIdx.x >> 1];
+  const int tile = 2 * it.pair + (int)rank;
+  const bool ghost = tile >= a.plan.n_tiles;     // odd tile count: the peer of the last pair has no rows
+  const int slot = it.slot[rank];
+  const int n = it.kt_end - it.kt_begin;         // the same in both CTAs
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kKRing; ++i) {
@@ -135,12 +177,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->vfull[i], 1);
       mbar_init(&bars->vempty[i], 1);
     }
-    mbar_init(&bars->q_tma, 1);
-    mbar_init(&bars->q_full, kSoftmaxThreads);
+    mbar_init(&bars->q_full, 1);
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_free, kSoftmaxThreads);
+    mbar_init(&bars->s_free, kPairArrivals);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->p_full[i], kSoftmaxThreads);
+      mbar_init(&bars->p_full[i], kPairArrivals);
       mbar_init(&bars->o_done[i], 1);
     }
     mbar_init(&bars->o_final, 1);
@@ -149,133 +190,122 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc_pair(smem_u32(&bars->tmem_base), kTmemCols);
+    ptx::tmem_relinquish_pair();
   }
+  // Both CTAs' barriers and TMEM exist before either touches the other's.
   ptx::fence_before_sync();
-  __syncthreads();
+  pair_sync();
   ptx::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
   // Programmatic dependent launch: the set-up above overlaps the previous
   // kernel of the stream; global memory is touched only after this wait.
-  // The next kernel may be scheduled as soon as SMs free up.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0 || warp == 2) {
     // ------------------------------------------------------------ producers
+    // Each CTA loads its half of every K / V tile; the bytes complete on the
+    // leader's full barrier, which the leader arms for both halves.
     if (lane == 0) {
       const bool is_k = warp == 0;
-      const int ring = is_k ? kKRing : kVRing;
       uint64_t* full = is_k ? bars->kfull : bars->vfull;
       uint64_t* empty = is_k ? bars->kempty : bars->vempty;
       ptx::prefetch_tmap(is_k ? &tmk : &tmv);
       if (is_k) {
         // Q tile: 128 M rows x 256 dims as four 64-dim boxes (128-byte
-        // swizzle) into the P buffers, which are unused until the first P.
+        // swizzle), the A operand of Q K^T in this CTA's shared memory;
+        // both CTAs' bytes complete on the leader's q_full.
         ptx::prefetch_tmap(&tmq);
-        mbar_arrive_expect_tx(&bars->q_tma, kQBytes);
+        if (leader) mbar_arrive_expect_tx(&bars->q_full, 2 * kQBytes);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          ptx::tma_load_2d(sbase + kOffP + i * kQBoxBytes, &tmq, 64 * i, it.tile * 128, smem_u32(&bars->q_tma));
+          ptx::tma_load_2d_pair(sbase + kOffQ + i * kQBoxBytes, &tmq, 64 * i, tile * 128, leader_bar(&bars->q_full));
       } else {
         ptx::prefetch_tmap(&tmo);
         ptx::prefetch_tmap(&tmpart);
       }
-      const int per_tile = 2;   // K: two slots of two 64-dim chunks, V: two 64-key halves
-      int e = 0;
       bool ok = true;
       for (int t = 0; t < n && ok; ++t) {
-        for (int c = 0; c < per_tile; ++c) {
-          const int slot = e % ring;
-          if (e >= ring &&
-              !mbar_wait(&empty[slot], ((e / ring) - 1) & 1, abort_flag, status, kSiteTcEmpty)) {
-            ok = false;
-            break;
-          }
-          const uint32_t bar = smem_u32(&full[slot]);
-          const int32_t key0 = (it.kt_begin + t) * kKeyTile;
-          if (is_k) {
-            mbar_arrive_expect_tx(&full[slot], kKSlotBytes);
-            const uint32_t dst = sbase + kOffK + slot * kKSlotBytes;
-            ptx::tma_load_2d(dst, &tmk, 128 * c, key0, bar);
-            ptx::tma_load_2d(dst + kKChunkBytes, &tmk, 128 * c + 64, key0, bar);
-          } else {
-            mbar_arrive_expect_tx(&full[slot], kVHalfBytes);
-            const uint32_t dst = sbase + kOffV + slot * kVHalfBytes;
+        const int s = t % 2;
+        if (t >= 2 && !mbar_wait(&empty[s], ((t / 2) - 1) & 1, abort_flag, status, kSiteTcEmpty)) {
+          ok = false;
+          break;
+        }
+        const int32_t key0 = (it.kt_begin + t) * kKeyTile;
+        if (leader) mbar_arrive_expect_tx(&full[s], 2 * (is_k ? kKSlotBytes : kVSlotBytes));
+        const uint32_t bar = leader_bar(&full[s]);
+        if (is_k) {
+          // keys [key0 + 64 rank, +64), all dims: four 64-dim chunks
+          const uint32_t dst = sbase + kOffK + s * kKSlotBytes;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) ptx::tma_load_2d(dst + i * kVBoxBytes, &tmv, 64 * i, key0 + 64 * c, bar);
-          }
-          ++e;
+          for (int c = 0; c < 4; ++c)
+            ptx::tma_load_2d_pair(dst + c * kKChunkBytes, &tmk, 64 * c, key0 + 64 * (int)rank, bar);
+        } else {
+          // dims [128 rank, +128), all 128 keys: box (key half h, dim block b) at (2h + b)
+          const uint32_t dst = sbase + kOffV + s * kVSlotBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+              ptx::tma_load_2d_pair(dst + (2 * h + b) * kVBoxBytes, &tmv, 128 * (int)rank + 64 * b, key0 + 64 * h, bar);
         }
       }
-      if (!ok) {  // aborted: let every issued copy land before the CTA exits
-        for (int s = 0; s < ring && s < e; ++s) {
-          const int last = ((e - 1 - s) / ring) * ring + s;
-          mbar_wait(&full[s], (last / ring) & 1, nullptr, status, kSiteTcDrain);
-        }
-      }
+      if (!ok) *abort_flag = 1;
     }
     __syncwarp();
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       constexpr uint32_t ab = DT == KCA_BF16 ? 1u : 0u;
-      constexpr uint32_t id_qk = ptx::idesc_f16(ab, 128, kKeyTile, 0);
-      constexpr uint32_t id_pv = ptx::idesc_f16(ab, 128, kDim, 1);
+      constexpr uint32_t id_qk = ptx::idesc_f16(ab, 256, kKeyTile, 0);
+      constexpr uint32_t id_pv = ptx::idesc_f16(ab, 256, kDim, 1);
       // Descriptor bases; an operand at byte offset x from a base is the base
       // plus x >> 4 in the start-address field (addresses stay below 256 KiB).
       const uint64_t kd0 = ptx::sdesc_sw128(sbase + kOffK, 16, 1024);
-      const uint64_t pd0 = ptx::sdesc_sw128(sbase + kOffP, 16, 1024);
+      const uint64_t qd0 = ptx::sdesc_sw128(sbase + kOffQ, 16, 1024);
       const uint64_t vd0 = ptx::sdesc_sw128(sbase + kOffV, kVBoxBytes, 1024);
-      int ek = 0, ev = 0;
+      const uint32_t s_full = smem_u32(&bars->s_full);
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, status, kSiteTcQ);
       ptx::fence_after_sync();
       auto pv = [&](int u) -> bool {
         if (!mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, abort_flag, status, kSiteTcP)) return false;
+        const int s = u % 2;
+        if (!mbar_wait(&bars->vfull[s], (u / 2) & 1, abort_flag, status, kSiteTcFull)) return false;
         ptx::fence_after_sync();
-        const uint64_t pd = pd0 + (uint64_t)(((u & 1) * kPBytes) >> 4);
-        for (int h = 0; h < 2; ++h) {
-          const int slot = ev % kVRing;
-          if (!mbar_wait(&bars->vfull[slot], (ev / kVRing) & 1, abort_flag, status, kSiteTcFull)) return false;
-          const uint64_t vd = vd0 + (uint64_t)((slot * kVHalfBytes) >> 4);
+        const uint32_t pcol = tmem + kColP + 64 * (u & 1);
+        const uint64_t vd = vd0 + (uint64_t)((s * kVSlotBytes) >> 4);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            ptx::mma_ss(tmem + kColO, pd + (uint64_t)((h * (kPBytes / 2) + j * 32) >> 4),
-                        vd + (uint64_t)((j * 16 * 128) >> 4), id_pv, (u > 0 || h > 0 || j > 0) ? 1u : 0u);
-          ptx::mma_commit(smem_u32(&bars->vempty[slot]));
-          ++ev;
-        }
-        ptx::mma_commit(smem_u32(&bars->o_done[u & 1]));
+        for (int j = 0; j < 8; ++j)   // 16 keys per step: 8 TMEM columns of P; V key half j/4, rows 16 (j%4)
+          ptx::mma_ts_pair(tmem + kColO, pcol + 8 * j,
+                           vd + (uint64_t)(((j >> 2) * 2 * kVBoxBytes + (j & 3) * 16 * 128) >> 4), id_pv,
+                           (u > 0 || j > 0) ? 1u : 0u);
+        ptx::mma_commit_pair(smem_u32(&bars->vempty[s]), kPairMask);
+        ptx::mma_commit_pair(smem_u32(&bars->o_done[u & 1]), kPairMask);
         return true;
       };
       for (int t = 0; t < n && ok; ++t) {
         if (t > 0) {
           ok = mbar_wait(&bars->s_free, (t - 1) & 1, abort_flag, status, kSiteTcS);
           if (!ok) break;
-          ptx::fence_after_sync();   // S was read by other threads' tcgen05.ld
         }
-        for (int c = 0; c < 2 && ok; ++c) {
-          const int slot = ek % kKRing;
-          ok = mbar_wait(&bars->kfull[slot], (ek / kKRing) & 1, abort_flag, status, kSiteTcFull);
-          if (!ok) break;
-          const uint64_t kd = kd0 + (uint64_t)((slot * kKSlotBytes) >> 4);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)   // K-steps 8c .. 8c+7: chunk j/4 of the slot
-            ptx::mma_ts(tmem + kColS, tmem + kColQ + (8 * c + j) * 8,
-                        kd + (uint64_t)(((j >> 2) * kKChunkBytes + (j & 3) * 32) >> 4), id_qk,
-                        (c > 0 || j > 0) ? 1u : 0u);
-          ptx::mma_commit(smem_u32(&bars->kempty[slot]));
-          ++ek;
-        }
+        const int s = t % 2;
+        ok = mbar_wait(&bars->kfull[s], (t / 2) & 1, abort_flag, status, kSiteTcFull);
         if (!ok) break;
-        ptx::mma_commit(smem_u32(&bars->s_full));
+        ptx::fence_after_sync();   // S was read by other threads' tcgen05.ld; K landed
+        const uint64_t kd = kd0 + (uint64_t)((s * kKSlotBytes) >> 4);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)   // 16 dims per step: chunk k/4, column group k%4
+          ptx::mma_ss_pair(tmem + kColS, qd0 + (uint64_t)(((k >> 2) * kQBoxBytes + (k & 3) * 32) >> 4),
+                           kd + (uint64_t)(((k >> 2) * kKChunkBytes + (k & 3) * 32) >> 4), id_qk, k > 0 ? 1u : 0u);
+        ptx::mma_commit_pair(smem_u32(&bars->kempty[s]), kPairMask);
+        ptx::mma_commit_pair(s_full, kPairMask);
         if (t > 0) ok = pv(t - 1);
       }
       if (ok) ok = pv(n - 1);
-      if (ok) ptx::mma_commit(smem_u32(&bars->o_final));
+      if (ok) ptx::mma_commit_pair(smem_u32(&bars->o_final), kPairMask);
       // every MMA issued above has completed once this barrier flips
-      ptx::mma_commit(smem_u32(&bars->drain));
+      ptx::mma_commit_pair(smem_u32(&bars->drain), kPairMask);
       mbar_wait(&bars->drain, 0, nullptr, status, kSiteTcDrain);
     }
     __syncwarp();
@@ -284,30 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = (warp - 4) >> 2;                  // key half of every S tile
     const int m = (warp & 3) * 32 + lane;            // TMEM lane == M row
     const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const int64_t row = (int64_t)it.tile * kRowTile + (m >> 3);
+    const int64_t row = (int64_t)tile * kRowTile + (m >> 3);
     const bool valid = row < a.plan.rows;
     const int64_t pos = a.plan.chunk_start + row;
     const int64_t lo = lo_of(pos, a.plan.window);
-
-    // Q row (row, head m & 7), dims [128 wg, 128 wg + 128), from the TMA
-    // boxes in shared memory into TMEM (rows past the chunk arrive as zeros).
-    {
-      const bool qok = mbar_wait(&bars->q_tma, 0, abort_flag, status, kSiteTcQ);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        const unsigned char* box = smem + kOffP + (2 * wg + c) * kQBoxBytes + m * 128;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = qok ? *reinterpret_cast<const uint4*>(box + ((i ^ (m & 7)) << 4)) : make_uint4(0, 0, 0, 0);
-          r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
-        }
-        ptx::tmem_st32(trow + kColQ + 64 * wg + 32 * c, r);
-      }
-      ptx::tmem_wait_st();
-      ptx::fence_before_sync();
-      mbar_arrive(&bars->q_full);
-    }
 
     const float cs = a.scale_log2;
     const uint32_t scol = kColS + 64 * wg;
@@ -332,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ptx::fence_before_sync();
-      mbar_arrive(&bars->s_free);   // S may be overwritten by the next QK^T
+      arrive_leader(&bars->s_free);   // S may be overwritten by the next QK^T
       float mloc = -INFINITY;
       if (ok) {
         // keys outside [lo, pos] become -inf (scale > 0 keeps them there)
@@ -401,16 +411,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc2[2] = __fadd2_rn(acc2[2], acc2[3]);
       acc2[0] = __fadd2_rn(acc2[0], acc2[2]);
       l_sum += acc2[0].x + acc2[0].y;
-      // P row m, keys [64 wg, 64 wg + 64): buffer t&1, K-major with 128-byte
-      // swizzle (16-byte unit j of row m at unit j ^ (m & 7)).
-      unsigned char* prow = smem + kOffP + (t & 1) * kPBytes + wg * (kPBytes / 2) + (m >> 3) * 1024 + (m & 7) * 128;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(prow + ((j ^ (m & 7)) << 4)) =
-            make_uint4(pr[4 * j], pr[4 * j + 1], pr[4 * j + 2], pr[4 * j + 3]);
-      fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor cores
+      // P row m, keys [64 wg, 64 wg + 64): 32 TMEM columns of 16-bit pairs in
+      // buffer t&1.  PV of tile t-2, the last reader of that buffer, has
+      // completed: it preceded QK^T of this tile, whose completion s_full signalled.
+      ptx::tmem_st32(trow + kColP + 64 * (t & 1) + 32 * wg, pr);
+      ptx::tmem_wait_st();
       ptx::fence_before_sync();
-      mbar_arrive(&bars->p_full[t & 1]);
+      arrive_leader(&bars->p_full[t & 1]);
     }
     ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->o_final, 0, abort_flag, status, kSiteTcO));
     // Row sum over both halves (the buffer of tile parity n&1 is free again).
@@ -424,11 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // and rows past the chunk fall outside the map and are not written.
     if (ok) {
       ptx::fence_after_sync();
-      if (it.slot >= 0 && wg == 0 && valid) {
-        a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 0] = m_ref;
-        a.part_ml[((int64_t)it.slot * 128 + m) * 2 + 1] = l_tot;
+      if (slot >= 0 && wg == 0 && valid) {
+        a.part_ml[((int64_t)slot * 128 + m) * 2 + 0] = m_ref;
+        a.part_ml[((int64_t)slot * 128 + m) * 2 + 1] = l_tot;
       }
-      const float f = it.slot < 0 ? 1.f / l_tot : 1.f;
+      const float f = slot < 0 ? 1.f / l_tot : 1.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
@@ -445,9 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::fence_before_sync();
     named_sync(1, kSoftmaxThreads);
-    if (ok && threadIdx.x == 4 * 32) {
-      const void* map = it.slot < 0 ? static_cast<const void*>(&tmo) : static_cast<const void*>(&tmpart);
-      const int32_t y = (it.slot < 0 ? (int32_t)it.tile : (int32_t)it.slot) * 128;
+    if (ok && !ghost && threadIdx.x == 4 * 32) {
+      const void* map = slot < 0 ? static_cast<const void*>(&tmo) : static_cast<const void*>(&tmpart);
+      const int32_t y = (slot < 0 ? tile : slot) * 128;
 #pragma unroll
       for (int j = 0; j < 8; ++j) ptx::tma_store_2d(map, 32 * j, y, sbase + j * kOBoxBytes);
       ptx::bulk_commit();
@@ -455,10 +462,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  __syncthreads();
+  // No CTA of the pair leaves while MMAs may still read its shared memory
+  // or its peer may still arrive on its barriers.
+  ptx::fence_before_sync();
+  pair_sync();
   if (warp == 1) {
     ptx::fence_after_sync();
-    ptx::tmem_dealloc(tmem, kTmemCols);
+    ptx::tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -496,17 +506,22 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  // Both kernels allow programmatic dependent launch (see griddepcontrol).
-  cudaLaunchAttribute pdl;
-  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl.val.programmaticStreamSerializationAllowed = 1;
+  // Both kernels allow programmatic dependent launch (see griddepcontrol);
+  // the attention kernel runs as clusters of two CTAs (one per item).
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.plan.n_items);
+  cfg.gridDim = dim3(2 * a.plan.n_items);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
-  cfg.attrs = &pdl;
-  cfg.numAttrs = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<DT>, tmk, tmv, tmq, tmo, tmpart, a);
   if (e != cudaSuccess || a.plan.n_slots == 0) return e;
   const int ns = a.plan.max_split;
@@ -514,6 +529,7 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
   cfg.gridDim = dim3(a.plan.n_tiles, 16 * w);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
+  cfg.numAttrs = 1;   // no cluster
   if (w == 8) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<8>, a);
   if (w == 4) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<4>, a);
   if (w == 2) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<2>, a);
@@ -523,22 +539,26 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
 }  // namespace
 
 void fill_tc_tables(TcArgs& a) {
-  // One pass over the tiles: O(tiles + items), no per-item plan walk.
+  // One pass over the pairs: O(pairs + items), no per-item plan walk.
   int32_t idx = 0, slot = 0;
-  for (int32_t t = 0; t < a.plan.n_tiles && t < kTcMaxTiles; ++t) {
+  for (int32_t q = 0; q < a.plan.n_pairs && 2 * q < kTcMaxTiles; ++q) {
     int32_t kb, ke;
-    tc_tile_keys(a.plan, t, &kb, &ke);
+    tc_pair_keys(a.plan, q, &kb, &ke);
     const int32_t n = ke - kb;
     const int32_t s = (int32_t)cdiv(n, a.plan.per_item);
-    a.tile_items[t] = (int16_t)s;
-    a.tile_first_slot[t] = (int16_t)slot;
+    const int32_t nt = tc_pair_tiles(a.plan, q);
+    for (int32_t r = 0; r < nt; ++r) {
+      a.tile_items[2 * q + r] = (int16_t)s;
+      a.tile_first_slot[2 * q + r] = (int16_t)(slot + r * s);
+    }
     for (int32_t k = 0; k < s && idx < kTcMaxItems; ++k, ++idx) {
       a.items[idx].kt_begin = kb + (int32_t)(((int64_t)k * n) / s);
       a.items[idx].kt_end = kb + (int32_t)(((int64_t)(k + 1) * n) / s);
-      a.items[idx].tile = (int16_t)t;
-      a.items[idx].slot = (int16_t)(s > 1 ? slot + k : -1);
+      a.items[idx].pair = (int16_t)q;
+      a.items[idx].slot[0] = (int16_t)(s > 1 ? slot + k : -1);
+      a.items[idx].slot[1] = (int16_t)(s > 1 && nt == 2 ? slot + s + k : -1);
     }
-    if (s > 1) slot += s;
+    if (s > 1) slot += s * nt;
   }
 }
 

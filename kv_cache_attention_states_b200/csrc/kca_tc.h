@@ -8,16 +8,16 @@
 
 namespace kca {
 
-constexpr int kTcMaxItems = 160;   // work items (CTAs) of one call
+constexpr int kTcMaxItems = 80;    // work items (CTA pairs) of one call
 constexpr int kTcMaxTiles = 48;    // 768 rows / 16
 
-// One work item, filled in on the host from the plan so that no CTA has to
-// walk the plan itself.
+// One work item of a CTA pair, filled in on the host from the plan so that
+// no CTA has to walk the plan itself.
 struct TcItemArg {
   int32_t kt_begin;   // key tiles relative to plan.kv_lo
   int32_t kt_end;
-  int16_t tile;       // row tile
-  int16_t slot;       // partial slot, -1 when the tile is not split
+  int16_t pair;       // row tiles 2 pair (even CTA) and 2 pair + 1 (odd CTA)
+  int16_t slot[2];    // partial slot of each tile, -1 when the pair is not split
 };
 
 struct TcArgs {
@@ -38,7 +38,7 @@ void fill_tc_tables(TcArgs& a);
 
 // tmk / tmv: 2-D tensor maps over the rows [plan.kv_lo, plan.ctx_len) of the
 // K and V caches, inner extent 256, 128-byte swizzle, zero fill; boxes of 64
-// elements x 128 rows (K) and 64 x 64 (V).  tmq: the Q chunk as [rows * 8][256]
+// elements x 64 rows (K and V).  tmq: the Q chunk as [rows * 8][256]
 // 16-bit, boxes 64 x 128.  tmo / tmpart: out as [rows * 8][256] f32 and the
 // partials as [n_slots * 128][256] f32, boxes 32 x 128; all 128-byte swizzle.
 cudaError_t launch_prefill_tc(int dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,

@@ -207,9 +207,12 @@ def test_prefill_tc_plan_covers_every_visible_key(cs, rows, window):
         for r in range(16 * t, min(16 * t + 16, rows)):
             lo, hi = oracle.visible_range(cs + r, window)
             assert covered[0] <= lo and hi < covered[1]
-        # the first item starts in the key tile of the tile's first row's lo
-        lo0 = oracle.visible_range(cs + 16 * t, window)[0]
+        # tiles go in pairs (2q, 2q+1) that share their items: the first item
+        # starts in the key tile of the pair's first row's lo
+        lo0 = oracle.visible_range(cs + 16 * (t - t % 2), window)[0]
         assert covered[0] == kv_lo + (lo0 - kv_lo) // KEY_TILE * KEY_TILE
+        if t % 2 == 1:
+            assert np.array_equal(its[:, 1:3], items[items[:, 0] == t - 1][:, 1:3])
         assert (len(its) == 1) == (its[0, 3] == -1)
 
 
