@@ -36,7 +36,7 @@ DECODE_REPLICAS = 32
 PREFILL_REPLICAS = 2
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels; reset to None whenever a kernel changes after its capture.
-PREFILL_TRAFFIC = 19.74e6 + 27.6e3
+PREFILL_TRAFFIC = 18.93e6 + 2.3e3
 DECODE_TRAFFIC = 16.90e6
 METRIC = "prefill q-rows/s & decode tok/s at 16K ctx (1 B200); % of TC/HBM roofline"
 
@@ -73,7 +73,7 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
 
@@ -378,7 +378,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="kca", choices=["kca", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -435,8 +435,8 @@ def main():
         "roofline": {"kernel": "prefill_tc_kernel (+ its merge)", "bound": "tensor",
                      "achieved": achieved_tf, "peak": tflops, "unit": "TFLOP/s",
                      "frac": achieved_tf / tflops, "traffic": PREFILL_TRAFFIC,
-                     "traffic_source": "ncu dram bytes of the chunk-20 launch (768 rows at 15360); "
-                                       "profiles/prefill_tc_kernel_16k_chunk20.md",
+                     "traffic_source": "ncu dram bytes of the chunk-19 launch (768 rows at 14592); "
+                                       "profiles/prefill_tc_kernel_16k_late_chunks.md",
                      "peak_source": f"{src} bf16 dense (burst)",
                      "algorithmic": "4*256*8*sum|J(pos)| = 1.0996e12 flop per step"},
         "decode": {"value": dec_tok_s, "unit": "tok/s", "ms_per_step": res["dec_ms"] / K,
