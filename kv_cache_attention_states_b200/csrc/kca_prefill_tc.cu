@@ -39,12 +39,11 @@
 // when a score exceeds it by more than 2^8, so probabilities stay <= 256 and
 // the O round trip is rare; the result is exact up to rounding whatever
 // reference is used.  Work items of a split row tile write (m, l, O)
-// partials that merge_tc_kernel combines by log-sum-exp (kca_merge.cuh).
+// partials that merge_tc_kernel (below) combines by log-sum-exp.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "kca_common.cuh"
-#include "kca_merge.cuh"
 #include "kca_plan.h"
 #include "kca_tc.h"
 #include "kca_tc_ptx.cuh"
@@ -473,25 +472,57 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
-// Log-sum-exp merge of the items of each split row tile: a group of W warps
-// per M row, 8 / W rows per CTA, grid (tiles, 16 W).
-template <int W>
+// Log-sum-exp merge of the items of each split row tile: one warp per M row
+// (lane k owns dims [8k, 8k+8)), the (m, l) and acc of up to eight items in
+// flight at once, an online rescale across groups of eight; 8 rows per CTA,
+// grid (tiles, 16).  Items are combined in slot order, so the result is the
+// same bits on every call.
 __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
-  constexpr int kRowsPerCta = 8 / W;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tile = blockIdx.x;
   const int ns = a.tile_items[tile];
   if (ns <= 1) return;
-  __shared__ float red[8 * 264];
-  const int warp = threadIdx.x >> 5;
-  const int gi = warp / W, g = warp % W;
-  const int m = blockIdx.y * kRowsPerCta + gi;
-  if ((int64_t)tile * kRowTile + (m >> 3) >= a.plan.rows) return;  // whole group leaves together
-  const int64_t r0 = (int64_t)a.tile_first_slot[tile] * 128 + m;
-  merge_row<W>(ns, a.part_ml + r0 * 2, 128 * 2, a.part_acc + r0 * kDim, (int64_t)128 * kDim, 1.f,
-               a.out + ((int64_t)tile * 128 + m) * kDim, red + gi * W * 264, g, threadIdx.x & 31,
-               1 + gi);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.y * 8 + warp;
+  if ((int64_t)tile * kRowTile + (m >> 3) >= a.plan.rows) return;   // the whole warp leaves together
+  const int64_t r0 = (int64_t)a.tile_first_slot[tile] * 128 + m;    // item s: row r0 + 128 s
+  float M = -INFINITY, L = 0.f;
+  float4 A0 = make_float4(0.f, 0.f, 0.f, 0.f), A1 = A0;
+  for (int s0 = 0; s0 < ns; s0 += 8) {
+    float mv[8], lv[8];
+    float4 v0[8], v1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t r = r0 + (int64_t)(s0 + j) * 128;
+      const bool in = s0 + j < ns;
+      mv[j] = in ? a.part_ml[r * 2] : -INFINITY;
+      lv[j] = in ? a.part_ml[r * 2 + 1] : 0.f;
+      const float4* src = reinterpret_cast<const float4*>(a.part_acc + r * kDim + 8 * lane);
+      v0[j] = in ? src[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+      v1[j] = in ? src[1] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float Mn = M;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) Mn = max_nan(Mn, mv[j]);
+    const float mu = Mn == -INFINITY ? 0.f : Mn;
+    const float alpha = exp2f(M - mu);   // m is in log2 units
+    L *= alpha;
+    A0.x *= alpha; A0.y *= alpha; A0.z *= alpha; A0.w *= alpha;
+    A1.x *= alpha; A1.y *= alpha; A1.z *= alpha; A1.w *= alpha;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float f = exp2f(mv[j] - mu);
+      L += f * lv[j];
+      A0.x += f * v0[j].x; A0.y += f * v0[j].y; A0.z += f * v0[j].z; A0.w += f * v0[j].w;
+      A1.x += f * v1[j].x; A1.y += f * v1[j].y; A1.z += f * v1[j].z; A1.w += f * v1[j].w;
+    }
+    M = Mn;
+  }
+  const float inv = 1.f / L;
+  float4* dst = reinterpret_cast<float4*>(a.out + ((int64_t)tile * 128 + m) * kDim + 8 * lane);
+  dst[0] = make_float4(A0.x * inv, A0.y * inv, A0.z * inv, A0.w * inv);
+  dst[1] = make_float4(A1.x * inv, A1.y * inv, A1.z * inv, A1.w * inv);
 }
 
 template <int DT>
@@ -524,16 +555,11 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
   cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<DT>, tmk, tmv, tmq, tmo, tmpart, a);
   if (e != cudaSuccess || a.plan.n_slots == 0) return e;
-  const int ns = a.plan.max_split;
-  const int w = ns > 8 ? 8 : (ns > 4 ? 4 : (ns > 2 ? 2 : 1));
-  cfg.gridDim = dim3(a.plan.n_tiles, 16 * w);
+  cfg.gridDim = dim3(a.plan.n_tiles, 16);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.numAttrs = 1;   // no cluster
-  if (w == 8) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<8>, a);
-  if (w == 4) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<4>, a);
-  if (w == 2) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<2>, a);
-  return cudaLaunchKernelEx(&cfg, merge_tc_kernel<1>, a);
+  return cudaLaunchKernelEx(&cfg, merge_tc_kernel, a);
 }
 
 }  // namespace
