@@ -59,6 +59,7 @@ constexpr int kDPrefetchKeys = 512;                  // keys per split prefetche
 struct DBars {
   uint64_t full[kDStages];
   uint64_t empty[kDStages];
+  uint64_t rx;                           // the partials this CTA owns have arrived (st.async bytes)
   int abort;
   float red[kDWarps][8];                 // per-warp stage max (then row sums) per head
   int last;                              // this CTA holds the last ticket of its unit
@@ -136,10 +137,6 @@ __device__ __forceinline__ uint32_t swz(int row, int dim) {
 }
 
 
-// Cluster-wide barrier (all threads of every CTA of the cluster).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 // Split cluster barrier: every thread of every CTA of the cluster arrives,
 // and waits for the others' arrival.
 __device__ __forceinline__ void cluster_arrive() {
@@ -148,25 +145,32 @@ __device__ __forceinline__ void cluster_arrive() {
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Stores into the shared memory of CTA `cta` of the cluster, at the offset
-// that `local` has in this CTA's (a plain store without a cluster).
-__device__ __forceinline__ void st_peer(float* local, uint32_t cta, float v, int C) {
+// Asynchronous store into the shared memory of CTA `cta` of the cluster, at
+// the offset that `local` has in this CTA's; its bytes complete on that
+// CTA's barrier `rx` (a plain store without a cluster).
+__device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t cta) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(cta));
+  return remote;
+}
+__device__ __forceinline__ void st_peer(float* local, uint32_t cta, float v, int C, uint64_t* rx) {
   if (C == 1) {
     *local = v;
     return;
   }
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(cta));
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(peer_addr(local, cta)),
+               "f"(v), "r"(peer_addr(rx, cta))
+               : "memory");
 }
-__device__ __forceinline__ void st_peer2(float* local, uint32_t cta, float v0, float v1, int C) {
+__device__ __forceinline__ void st_peer2(float* local, uint32_t cta, float v0, float v1, int C, uint64_t* rx) {
   if (C == 1) {
     *reinterpret_cast<float2*>(local) = make_float2(v0, v1);
     return;
   }
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(cta));
-  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(v0), "f"(v1) : "memory");
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+                   peer_addr(local, cta)),
+               "f"(v0), "f"(v1), "r"(peer_addr(rx, cta))
+               : "memory");
 }
 
 template <int QT, int KT>
@@ -210,6 +214,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], kDWarps);
     }
+    // The partials of the heads this CTA owns arrive as st.async bytes from
+    // every CTA of the cluster: C x (8 / C) x (256 + 2) floats.
+    mbar_init(&bars->rx, 1);
+    if (C > 1) mbar_arrive_expect_tx(&bars->rx, kHeads * (kDim + 2) * 4);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -274,12 +282,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
     if (C > 1) cluster_wait();
     if (threadIdx.x < kHeads) {
       const int h = threadIdx.x;
-      st_peer(&bars->rm[rank * nh + h / C], h % C, -INFINITY, C);
-      st_peer(&bars->rl[rank * nh + h / C], h % C, 0.f, C);
+      st_peer(&bars->rm[rank * nh + h / C], h % C, -INFINITY, C, &bars->rx);
+      st_peer(&bars->rl[rank * nh + h / C], h % C, 0.f, C, &bars->rx);
     }
     for (int i = threadIdx.x; i < kHeads * kDim; i += kDWarps * 32) {
       const int h = i / kDim;
-      st_peer(&bars->ro[rank * nh + h / C][i % kDim], h % C, 0.f, C);
+      st_peer(&bars->ro[rank * nh + h / C][i % kDim], h % C, 0.f, C, &bars->rx);
     }
   } else {
     // ------------------------------------------------------------------ compute
@@ -427,28 +435,33 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
       const int d = 32 * warp + 8 * nt + 2 * tig;
-      st_peer2(&bars->ro[slot][d], owner, o[nt][0] + o[nt][2], o[nt][1] + o[nt][3], C);
+      st_peer2(&bars->ro[slot][d], owner, o[nt][0] + o[nt][2], o[nt][1] + o[nt][3], C, &bars->rx);
     }
     if (warp == 0 && tig == 0) {
-      st_peer(&bars->rm[slot], owner, m_ref, C);
-      st_peer(&bars->rl[slot], owner, L, C);
+      st_peer(&bars->rm[slot], owner, m_ref, C, &bars->rx);
+      st_peer(&bars->rl[slot], owner, L, C, &bars->rx);
     }
   }
   if (warp == kDWarps && C > 1) cluster_wait();   // the producer keeps the barrier phases in step
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ------------------------------------------------------------ merge
-  // CTA rank r owns heads r, r+C, ... (C divides 8) and has received the C
-  // partials of each through distributed shared memory; once the cluster
-  // barrier completes, they are in its own shared memory and no CTA touches
-  // another's again.  Thread d owns dim d.  With one cluster per unit the
+  // CTA rank r owns heads r, r+C, ... (C divides 8) and receives the C
+  // partials of each by st.async into its own shared memory; once their
+  // bytes have completed on its barrier rx, no CTA touches another's shared
+  // memory again, so no cluster barrier is needed before any CTA leaves.  Thread d owns dim d.  With one cluster per unit the
   // merge of the C partials is the result.  Otherwise each CTA publishes its
   // heads' cluster partials and takes a ticket of (unit, rank); the CTA that
   // draws the last one merges every cluster's partials of those heads.
   // Nothing waits on another CTA, so the order in which clusters run does not
   // matter.
-  if (C > 1) cluster_sync_all();
-  else __syncthreads();
+  if (C > 1) {
+    // every partial of the owned heads has landed: C sources x 8 / C heads x
+    // (256 + 2) floats
+    if (threadIdx.x < kDim) mbar_wait(&bars->rx, 0, nullptr, status, kSiteRowsFull);
+  } else {
+    __syncthreads();
+  }
   if (threadIdx.x < kDim) {
     const int d = threadIdx.x;
     for (int i = 0; i < nh; ++i) {
@@ -488,9 +501,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
       // ticket.  Acquire: the last ticket holder's fence, then the block.
       asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
       if (d == 0) {
-        __threadfence();
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");
         const bool last = atomicAdd(&a.tickets[unit * kHeads + rank], 1) == nclus - 1;
-        if (last) __threadfence();
+        if (last) asm volatile("fence.acq_rel.gpu;" ::: "memory");
         bars->last = last;
       }
       asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
