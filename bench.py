@@ -50,6 +50,17 @@ def _peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+def max_over_ranks(values, world: int, device):
+    """Element-wise maximum over ranks of this rank's device-timed values
+    (every rank calls it; the job is as slow as its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def prefill_flops() -> float:
     # 2 GEMMs (QK^T and PV) x 2 flop x head_dim x 8 heads per visible (query, key) pair
     pairs = PREFILL_ROWS * (PREFILL_ROWS + 1) // 2
@@ -227,17 +238,16 @@ def run_cuda(args, rank, world, local_rank):
     total_ms = start.elapsed_time(end)
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
     dec_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
-    times = torch.tensor([total_ms, pre_ms, dec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, pre_ms, dec_ms = times.tolist()
+    total_ms, pre_ms, dec_ms = max_over_ranks([total_ms, pre_ms, dec_ms], world, dev)
     st, detail = w.kca.attn_device_status(w.pre_ws)
     st2, _ = w.kca.attn_device_status(w.dec_ws)
     if st != 0 or st2 != 0:
         raise RuntimeError(f"device status {st}/{st2} detail {detail:#x}")
     res = dict(total_ms=total_ms, pre_ms=pre_ms, dec_ms=dec_ms, clocks=clk,
                launches=w.launches_per_step() * args.steps)
-    res["e2e"] = run_e2e(w, args, stream) if rank == 0 or world > 1 else None
+    e2e = run_e2e(w, args, stream)
+    e2e["pre_ms"], e2e["dec_ms"] = max_over_ranks([e2e["pre_ms"], e2e["dec_ms"]], world, dev)
+    res["e2e"] = e2e
     return res
 
 
