@@ -173,6 +173,94 @@ __device__ __forceinline__ void st_peer2(float* local, uint32_t cta, float v0, f
                : "memory");
 }
 
+// Final merge of one owned head (slot hi: head rank + hi C) over the nclus
+// cluster partials, W consecutive dims per thread (dims [W jd, W jd + W)).
+// The first batch of partial accumulators is requested before (m, l) of all
+// partials go to shared memory, so the two round trips overlap; each warp
+// then reduces (M, L) of its head itself and each thread sums its dims over
+// the partials in slot order.  L2-coherent loads: other SMs wrote the
+// partials.  NB partials per batch of loads (the smallest batch that holds
+// all of them, up to 32 / W; loads past nclus repeat partial 0 and are
+// weighted 0).  Every thread of the block calls this (it holds a bar.sync).
+template <int W, int NB>
+__device__ __forceinline__ void merge_cluster_partials(const RowsArgs& a, float* sm_m, float* sm_l, int64_t u0,
+                                                       int unit, int rank, int C, int nh, int d, int nclus,
+                                                       int lane) {
+  const int per = kDim / W;              // threads per head
+  const int hi = d / per, jd = d % per;
+  const int h = rank + hi * C;
+  const float* base = a.cpart_acc + (u0 + h) * kDim + W * jd;   // partial c at + c * kHeads * kDim
+  float v[NB][W];
+  auto load_batch = [&](int c0) {
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const int c = c0 + t;
+      const float* src = base + (int64_t)(c < nclus ? c : 0) * kHeads * kDim;
+      if (W >= 4) {
+#pragma unroll
+        for (int e = 0; e < W; e += 4) {
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(src + e));
+          v[t][e] = x.x; v[t][(e + 1) % W] = x.y; v[t][(e + 2) % W] = x.z; v[t][(e + 3) % W] = x.w;
+        }
+      } else if (W == 2) {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
+        v[t][0] = x.x; v[t][1 % W] = x.y;
+      } else {
+        v[t][0] = __ldcg(src);
+      }
+    }
+  };
+  load_batch(0);
+  for (int c = d; c < nclus; c += kDim) {
+    for (int i = 0; i < nh; ++i) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.cpart_ml) + u0 + (int64_t)c * kHeads + rank + i * C);
+      sm_m[i * kDim + c] = ml.x;
+      sm_l[i * kDim + c] = ml.y;
+    }
+  }
+  asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
+  const float* pm = sm_m + hi * kDim;
+  const float* pl = sm_l + hi * kDim;
+  float mw = -INFINITY;
+  for (int c = lane; c < nclus; c += 32) mw = max_nan(mw, pm[c]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+  const float M = mw, mu = M == -INFINITY ? 0.f : M;
+  float lw = 0.f;
+  for (int c = lane; c < nclus; c += 32) lw += exp2f((pm[c] - mu) * kDLog2e) * pl[c];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+  const float L = lw;
+  float acc[W];
+#pragma unroll
+  for (int e = 0; e < W; ++e) acc[e] = 0.f;
+  for (int c0 = 0;; c0 += NB) {
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const int c = c0 + t;
+      const float f = c < nclus ? exp2f((pm[c < nclus ? c : 0] - mu) * kDLog2e) : 0.f;
+#pragma unroll
+      for (int e = 0; e < W; ++e) acc[e] += f * v[t][e];
+    }
+    if (c0 + NB >= nclus) break;
+    load_batch(c0 + NB);
+  }
+  float* dst = a.out + ((int64_t)unit * kHeads + h) * kDim + W * jd;
+  const bool empty = M == -INFINITY && L == 0.f;
+#pragma unroll
+  for (int e = 0; e < W; ++e) dst[e] = empty ? 0.f : acc[e] / L;
+}
+
+template <int W>
+__device__ __forceinline__ void merge_cluster_partials_nb(const RowsArgs& a, float* sm_m, float* sm_l, int64_t u0,
+                                                          int unit, int rank, int C, int nh, int d, int nclus,
+                                                          int lane) {
+  if (nclus <= 4) merge_cluster_partials<W, 4>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
+  else if (nclus <= 8) merge_cluster_partials<W, 8>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
+  else if (W > 1 || nclus <= 16) merge_cluster_partials<W, 16>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
+  else merge_cluster_partials<W, 32>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
+}
+
 template <int QT, int KT>
 __global__ void __launch_bounds__(kDThreads, 1)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -508,79 +596,18 @@ __global__ void __launch_bounds__(kDThreads, 1)
       }
       asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
       if (bars->last) {
-        // Merge of the nclus cluster partials of each owned head.  (m, l) of
-        // every partial go to shared memory first (the stage buffers are
-        // free now); thread t then sums dims 4(t % 64) .. +3 over the
-        // partials c = t / 64 (mod 4) with 16-byte loads, eight in flight,
-        // and the four groups are added in shared memory.  L2-coherent
-        // loads: other SMs wrote the partials.
+        // Merge of the nclus cluster partials of the nh owned heads, all heads
+        // at once: 256 / nh threads per head, thread jd of head slot hi
+        // owning dims [nh jd, nh jd + nh).  (m, l) of every partial go to
+        // shared memory (the stage buffers are free now) while the first
+        // batch of partial accumulators is in flight.
         float* sm_m = reinterpret_cast<float*>(smem);          // [8][256]
         float* sm_l = sm_m + kHeads * kDim;                    // [8][256]
-        float* sm_o = sm_l + kHeads * kDim;                    // [4][256]
         const int64_t u0 = (int64_t)unit * a.max_clusters * kHeads;   // cluster 0, head 0
-        const int grp = d >> 6, q4 = d & 63;
-        // Eight partials c0, c0 + 4, ... of head rank + i * C, dims 4 q4 .. +3.
-        auto load_batch = [&](int i, int c0, float4(&v)[8]) {
-          const float4* acc = reinterpret_cast<const float4*>(a.cpart_acc + (u0 + rank + i * C) * kDim) + q4;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int c = c0 + 4 * j;
-            v[j] = c < nclus ? __ldcg(acc + (int64_t)c * kHeads * (kDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        };
-        // The first batches of heads 0 and 1 are in flight together with the
-        // (m, l) loads, and each head's successor-but-one is requested as
-        // soon as its registers are free, so the merge waits on about one
-        // round trip.
-        auto merge_head = [&](int i, float4(&v)[8]) {
-          const int h = rank + i * C;
-          // (M, L) of head h: each warp reduces them itself.
-          float mw = -INFINITY;
-          for (int c = lane; c < nclus; c += 32) mw = max_nan(mw, sm_m[i * kDim + c]);
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, o));
-          const float M = mw, mu = M == -INFINITY ? 0.f : M;
-          float lw = 0.f;
-          for (int c = lane; c < nclus; c += 32) lw += exp2f((sm_m[i * kDim + c] - mu) * kDLog2e) * sm_l[i * kDim + c];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-          const float L = lw;
-          float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int c0 = grp;; c0 += 32) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int c = c0 + 4 * j;
-              const float f = c < nclus ? exp2f((sm_m[i * kDim + c] - mu) * kDLog2e) : 0.f;
-              O.x += f * v[j].x;
-              O.y += f * v[j].y;
-              O.z += f * v[j].z;
-              O.w += f * v[j].w;
-            }
-            if (c0 + 32 >= nclus) break;
-            load_batch(i, c0 + 32, v);
-          }
-          if (i + 2 < nh) load_batch(i + 2, grp, v);
-          reinterpret_cast<float4*>(sm_o + grp * kDim)[q4] = O;
-          asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
-          const float Od = (sm_o[d] + sm_o[kDim + d]) + (sm_o[2 * kDim + d] + sm_o[3 * kDim + d]);
-          a.out[((int64_t)unit * kHeads + h) * kDim + d] = (M == -INFINITY && L == 0.f) ? 0.f : Od / L;
-          asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");   // sm_o is reused by the next head
-        };
-        float4 va[8], vb[8];
-        load_batch(0, grp, va);
-        if (nh > 1) load_batch(1, grp, vb);
-        for (int c = d; c < nclus; c += kDim) {
-          for (int i = 0; i < nh; ++i) {
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.cpart_ml) + u0 + (int64_t)c * kHeads + rank + i * C);
-            sm_m[i * kDim + c] = ml.x;
-            sm_l[i * kDim + c] = ml.y;
-          }
-        }
-        asm volatile("bar.sync 2, %0;" ::"n"(kDim) : "memory");
-        for (int i = 0; i < nh; i += 2) {
-          merge_head(i, va);
-          if (i + 1 < nh) merge_head(i + 1, vb);
-        }
+        if (nh == 1) merge_cluster_partials_nb<1>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
+        else if (nh == 2) merge_cluster_partials_nb<2>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
+        else if (nh == 4) merge_cluster_partials_nb<4>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
+        else merge_cluster_partials_nb<8>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
         if (d == 0) a.tickets[unit * kHeads + rank] = 0;   // ready for the next call
       }
     }
