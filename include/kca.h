@@ -42,8 +42,12 @@
  *
  * DTYPES: decode takes any q_dtype with any kv_dtype.  Prefill with
  * q_dtype == kv_dtype in {F16, BF16} and chunk_rows >= 16 runs on the
- * tcgen05 tensor cores (f32 accumulation); every other prefill combination
- * runs on the CUDA cores in f32.
+ * tcgen05 tensor-core path (16-row tiles, f32 accumulation).  Chunks of 3-15
+ * such rows take that path too when their first row sees at least 12,288
+ * keys (one pass over the keys beats one pass per row there), else the rows
+ * path, which also serves every other prefill combination: one unit per
+ * query row, mma.sync with split-precision operands for 16-bit caches,
+ * CUDA-core f32 for f32 caches.
  *
  * OWNERSHIP: every buffer is allocated and owned by the caller.  The library
  * allocates no device memory, keeps no per-call state and never synchronises

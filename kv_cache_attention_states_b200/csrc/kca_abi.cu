@@ -54,12 +54,21 @@ int current_sms(int* out) {
 
 // "tc" / "rows" forces the prefill path (tests use it to run both paths on
 // the same inputs); unset or anything else chooses by the rules in kca.h.
-bool use_tc(int32_t q_dtype, int32_t kv_dtype, int32_t rows) {
+// Chunks of fewer than 16 rows: the rows path streams the visible keys once
+// per row (the first row from HBM, the rest mostly from L2), the tensor-core
+// path once per chunk but with a fixed cost of ~9 us (two launches, the
+// partials of the split tile, the merge).  B200 graph-replay timings of both
+// paths (1-15 rows at 1K-64K keys) put the crossover at about 3 rows once
+// the rows see 12K keys or more; below 12K keys the rows path wins up to 15
+// rows.
+bool use_tc(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, int32_t rows, int32_t window) {
   const bool eligible = q_dtype == kv_dtype && (q_dtype == KCA_F16 || q_dtype == KCA_BF16);
   const char* env = std::getenv("KCA_PREFILL_PATH");
   if (env != nullptr && std::strcmp(env, "rows") == 0) return false;
   if (env != nullptr && std::strcmp(env, "tc") == 0) return eligible;
-  return eligible && rows >= kca::kRowTile;
+  if (!eligible) return false;
+  if (rows >= kca::kRowTile) return true;
+  return rows >= 3 && kca::n_visible(chunk_start, window) >= 12288;
 }
 
 std::vector<int64_t> prefill_unit_keys(int64_t chunk_start, int32_t rows, int32_t window) {
@@ -136,15 +145,17 @@ bool encode_kv_map(CUtensorMap* m, const void* cache, int32_t dtype, int64_t kv_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D map over `rows` rows of 256 elements (f32 or 16-bit), box {box_x, 128},
-// 128-byte swizzle; reads past the extent return zeros, stores are clipped.
-bool encode_rows_map(CUtensorMap* m, const void* base, int32_t dtype, int64_t rows, uint32_t box_x) {
+// 2-D map over `rows` rows of 256 elements (f32 or 16-bit), box {box_x,
+// box_rows}, 128-byte swizzle; reads past the extent return zeros, stores are
+// clipped.
+bool encode_rows_map(CUtensorMap* m, const void* base, int32_t dtype, int64_t rows, uint32_t box_x,
+                     uint32_t box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr || rows < 1) return false;
   const int esz = dtype == KCA_F32 ? 4 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kDim * esz};
-  cuuint32_t box[2] = {box_x, 128};
+  cuuint32_t box[2] = {box_x, box_rows};
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType t = dtype == KCA_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                 : dtype == KCA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -295,7 +306,7 @@ int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, in
       chunk_start + chunk_rows > KCA_MAX_POSITION || num_sms < 1)
     return KCA_ERR_RANGE;
   int32_t count = 0;
-  if (use_tc(q_dtype, kv_dtype, chunk_rows)) {
+  if (use_tc(q_dtype, kv_dtype, chunk_start, chunk_rows, window)) {
     *path = 1;
     const kca::TcPlan p = kca::make_tc_plan(chunk_start, chunk_rows, window, num_sms / 2);
     for (int32_t i = 0; i < p.n_items; ++i) {
@@ -369,7 +380,7 @@ size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t c
   if (prefill_args_status(KCA_MAX_POSITION, chunk_start, chunk_rows) != KCA_OK) return 0;
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return 0;
-  if (use_tc(q_dtype, kv_dtype, chunk_rows))
+  if (use_tc(q_dtype, kv_dtype, chunk_start, chunk_rows, window))
     return tc_ws_bytes(kca::make_tc_plan(chunk_start, chunk_rows, window, sms / 2));
   const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
   return rows_ws_bytes_any(chunk_rows, nk.data(), sms);
@@ -427,7 +438,7 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
   if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  if (use_tc(q_dtype, kv_dtype, chunk_rows)) {
+  if (use_tc(q_dtype, kv_dtype, chunk_start, chunk_rows, window)) {
     kca::TcArgs a{};
     a.plan = kca::make_tc_plan(chunk_start, chunk_rows, window, sms / 2);
     if (workspace_bytes < tc_ws_bytes(a.plan)) return KCA_ERR_WORKSPACE;
@@ -437,7 +448,7 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
     a.scale_log2 = scale * 1.4426950408889634f;
     carve(workspace, (size_t)a.plan.n_slots * 128 * 2 * 4, &a.part_ml, &a.part_acc);
     kca::fill_tc_tables(a);
-    CUtensorMap tmk, tmv, tmq, tmo, tmpart;
+    CUtensorMap tmk, tmv, tmq, tmo, tmpart, tmpart_rag;
     // K and V: 64 x 64 boxes (each CTA of a pair loads its half of a tile);
     // Q in 64-dim boxes of a 128-row tile; out / partials in 32-column boxes.
     if (!encode_kv_map(&tmk, k_cache, kv_dtype, a.plan.kv_lo, a.plan.ctx_len, 64) ||
@@ -450,8 +461,20 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
     } else {
       tmpart = tmo;   // no split tile: never used
     }
-    return kca::launch_prefill_tc(kv_dtype, tmk, tmv, tmq, tmo, tmpart, a, s) == cudaSuccess ? KCA_OK
-                                                                                           : KCA_ERR_CUDA;
+    // A ragged last tile (chunk_rows not a multiple of 16) stores only its
+    // 8 (chunk_rows mod 16) valid M rows of each partial.
+    const int32_t rag = chunk_rows % kca::kRowTile;
+    a.rag_tile = a.plan.n_slots > 0 && rag != 0 ? a.plan.n_tiles - 1 : -1;
+    if (a.rag_tile >= 0) {
+      if (!encode_rows_map(&tmpart_rag, a.part_acc, KCA_F32, (int64_t)a.plan.n_slots * 128, 32,
+                           (uint32_t)(rag * kHeads)))
+        return KCA_ERR_CUDA;
+    } else {
+      tmpart_rag = tmpart;
+    }
+    return kca::launch_prefill_tc(kv_dtype, tmk, tmv, tmq, tmo, tmpart, tmpart_rag, a, s) == cudaSuccess
+               ? KCA_OK
+               : KCA_ERR_CUDA;
   }
 
   const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);

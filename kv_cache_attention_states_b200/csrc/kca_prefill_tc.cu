@@ -147,7 +147,8 @@ template <int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                       const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
-                      const __grid_constant__ CUtensorMap tmpart, const TcArgs a) {
+                      const __grid_constant__ CUtensorMap tmpart,
+                      const __grid_constant__ CUtensorMap tmpart_rag, const TcArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -223,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         ptx::prefetch_tmap(&tmo);
         ptx::prefetch_tmap(&tmpart);
+        ptx::prefetch_tmap(&tmpart_rag);
       }
       bool ok = true;
       for (int t = 0; t < n && ok; ++t) {
@@ -452,7 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_before_sync();
     named_sync(1, kSoftmaxThreads);
     if (ok && !ghost && threadIdx.x == 4 * 32) {
-      const void* map = slot < 0 ? static_cast<const void*>(&tmo) : static_cast<const void*>(&tmpart);
+      // A ragged tile's partial keeps only its valid rows: the first rows of
+      // every box (the swizzle pattern repeats every 8 rows).
+      const void* map = slot < 0             ? static_cast<const void*>(&tmo)
+                        : tile == a.rag_tile ? static_cast<const void*>(&tmpart_rag)
+                                             : static_cast<const void*>(&tmpart);
       const int32_t y = (slot < 0 ? tile : slot) * 128;
 #pragma unroll
       for (int j = 0; j < 8; ++j) ptx::tma_store_2d(map, 32 * j, y, sbase + j * kOBoxBytes);
@@ -472,30 +478,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
-// Log-sum-exp merge of the items of each split row tile: one warp per M row
-// (lane k owns dims [8k, 8k+8)), the (m, l) and acc of up to eight items in
-// flight at once, an online rescale across groups of eight; 8 rows per CTA,
-// grid (tiles, 16).  Items are combined in slot order, so the result is the
-// same bits on every call.
+// Log-sum-exp merge of the items of each split row tile.  WPR warps per M
+// row (8 / WPR rows per CTA, grid (tiles, 16 WPR)); warp sub of a row takes
+// the contiguous items [sub n, sub n + n) of the tile's ns, lane k owning
+// dims [8k, 8k+8), with the (m, l) and acc of eight items in flight at once
+// and an online rescale across groups of eight.  With WPR > 1 the warps'
+// partials of a row are combined in shared memory in sub order.  Items and
+// sub-ranges are combined in slot order, so the result is the same bits on
+// every call.  Many items per tile (few tiles in the chunk) take more warps
+// per row, so that no warp waits on more than a few load round trips.
+template <int WPR>
 __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  constexpr int RPC = 8 / WPR;   // rows per CTA
   const int tile = blockIdx.x;
   const int ns = a.tile_items[tile];
   if (ns <= 1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m = blockIdx.y * 8 + warp;
-  if ((int64_t)tile * kRowTile + (m >> 3) >= a.plan.rows) return;   // the whole warp leaves together
+  const int m = blockIdx.y * RPC + warp / WPR, sub = warp % WPR;
+  const bool row_ok = (int64_t)tile * kRowTile + (m >> 3) < a.plan.rows;
+  if (WPR == 1 && !row_ok) return;   // the whole warp leaves together
+  const int per = (ns + WPR - 1) / WPR;
+  const int sb = sub * per, se = min(ns, sb + per);
   const int64_t r0 = (int64_t)a.tile_first_slot[tile] * 128 + m;    // item s: row r0 + 128 s
   float M = -INFINITY, L = 0.f;
   float4 A0 = make_float4(0.f, 0.f, 0.f, 0.f), A1 = A0;
-  for (int s0 = 0; s0 < ns; s0 += 8) {
+  for (int s0 = sb; row_ok && s0 < se; s0 += 8) {
     float mv[8], lv[8];
     float4 v0[8], v1[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int64_t r = r0 + (int64_t)(s0 + j) * 128;
-      const bool in = s0 + j < ns;
+      const bool in = s0 + j < se;
       mv[j] = in ? a.part_ml[r * 2] : -INFINITY;
       lv[j] = in ? a.part_ml[r * 2 + 1] : 0.f;
       const float4* src = reinterpret_cast<const float4*>(a.part_acc + r * kDim + 8 * lane);
@@ -519,6 +534,32 @@ __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
     }
     M = Mn;
   }
+  if (WPR > 1) {
+    __shared__ float4 sa[8][2][32];
+    __shared__ float sml[8][2];
+    sa[warp][0][lane] = A0;
+    sa[warp][1][lane] = A1;
+    if (lane == 0) {
+      sml[warp][0] = M;
+      sml[warp][1] = L;
+    }
+    __syncthreads();
+    if (sub != 0 || !row_ok) return;
+#pragma unroll
+    for (int j = 1; j < WPR; ++j) {
+      const float mj = sml[warp + j][0], lj = sml[warp + j][1];
+      const float4 b0 = sa[warp + j][0][lane], b1 = sa[warp + j][1][lane];
+      const float Mn = max_nan(M, mj);
+      const float mu = Mn == -INFINITY ? 0.f : Mn;
+      const float fa = exp2f(M - mu), fb = exp2f(mj - mu);
+      L = fa * L + fb * lj;
+      A0.x = fa * A0.x + fb * b0.x; A0.y = fa * A0.y + fb * b0.y;
+      A0.z = fa * A0.z + fb * b0.z; A0.w = fa * A0.w + fb * b0.w;
+      A1.x = fa * A1.x + fb * b1.x; A1.y = fa * A1.y + fb * b1.y;
+      A1.z = fa * A1.z + fb * b1.z; A1.w = fa * A1.w + fb * b1.w;
+      M = Mn;
+    }
+  }
   const float inv = 1.f / L;
   float4* dst = reinterpret_cast<float4*>(a.out + ((int64_t)tile * 128 + m) * kDim + 8 * lane);
   dst[0] = make_float4(A0.x * inv, A0.y * inv, A0.z * inv, A0.w * inv);
@@ -527,7 +568,8 @@ __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
 
 template <int DT>
 cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmq,
-                     const CUtensorMap& tmo, const CUtensorMap& tmpart, const TcArgs& a, cudaStream_t stream) {
+                     const CUtensorMap& tmo, const CUtensorMap& tmpart, const CUtensorMap& tmpart_rag,
+                     const TcArgs& a, cudaStream_t stream) {
   static bool attr_set[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -553,13 +595,19 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<DT>, tmk, tmv, tmq, tmo, tmpart, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<DT>, tmk, tmv, tmq, tmo, tmpart, tmpart_rag, a);
   if (e != cudaSuccess || a.plan.n_slots == 0) return e;
-  cfg.gridDim = dim3(a.plan.n_tiles, 16);
+  int ns_max = 0;
+  for (int32_t t = 0; t < a.plan.n_tiles && t < kTcMaxTiles; ++t) ns_max = a.tile_items[t] > ns_max ? a.tile_items[t] : ns_max;
+  const int wpr = ns_max <= 8 ? 1 : ns_max <= 16 ? 2 : ns_max <= 32 ? 4 : 8;
+  cfg.gridDim = dim3(a.plan.n_tiles, 16 * wpr);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.numAttrs = 1;   // no cluster
-  return cudaLaunchKernelEx(&cfg, merge_tc_kernel, a);
+  if (wpr == 1) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<1>, a);
+  if (wpr == 2) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<2>, a);
+  if (wpr == 4) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<4>, a);
+  return cudaLaunchKernelEx(&cfg, merge_tc_kernel<8>, a);
 }
 
 }  // namespace
@@ -590,9 +638,10 @@ void fill_tc_tables(TcArgs& a) {
 
 cudaError_t launch_prefill_tc(int dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                               const CUtensorMap& tmq, const CUtensorMap& tmo, const CUtensorMap& tmpart,
+                              const CUtensorMap& tmpart_rag,
                               const TcArgs& a, cudaStream_t stream) {
-  if (dtype == KCA_BF16) return launch_t<KCA_BF16>(tmk, tmv, tmq, tmo, tmpart, a, stream);
-  if (dtype == KCA_F16) return launch_t<KCA_F16>(tmk, tmv, tmq, tmo, tmpart, a, stream);
+  if (dtype == KCA_BF16) return launch_t<KCA_BF16>(tmk, tmv, tmq, tmo, tmpart, tmpart_rag, a, stream);
+  if (dtype == KCA_F16) return launch_t<KCA_F16>(tmk, tmv, tmq, tmo, tmpart, tmpart_rag, a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -28,6 +28,7 @@ struct TcArgs {
   void* status;       // workspace status header
   TcPlan plan;
   float scale_log2;   // scale * log2(e)
+  int32_t rag_tile;   // split tile whose partials store only their valid rows (tmpart_rag), or -1
   TcItemArg items[kTcMaxItems];
   int16_t tile_first_slot[kTcMaxTiles];
   int16_t tile_items[kTcMaxTiles];
@@ -40,9 +41,11 @@ void fill_tc_tables(TcArgs& a);
 // K and V caches, inner extent 256, 128-byte swizzle, zero fill; boxes of 64
 // elements x 64 rows (K and V).  tmq: the Q chunk as [rows * 8][256]
 // 16-bit, boxes 64 x 128.  tmo / tmpart: out as [rows * 8][256] f32 and the
-// partials as [n_slots * 128][256] f32, boxes 32 x 128; all 128-byte swizzle.
+// partials as [n_slots * 128][256] f32, boxes 32 x 128; tmpart_rag: the
+// same partials with boxes of 32 x (8 x the valid rows of tile a.rag_tile);
+// all 128-byte swizzle.
 cudaError_t launch_prefill_tc(int dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                               const CUtensorMap& tmq, const CUtensorMap& tmo, const CUtensorMap& tmpart,
-                              const TcArgs& a, cudaStream_t stream);
+                              const CUtensorMap& tmpart_rag, const TcArgs& a, cudaStream_t stream);
 
 }  // namespace kca

@@ -118,6 +118,21 @@ def test_prefill_short_chunks_take_rows_path(rows):
     assert max_err(out.cpu().numpy(), want) <= 4e-3
 
 
+@pytest.mark.parametrize("rows", [3, 9, 15])
+def test_few_row_chunk_on_long_context_takes_tc_path(rows):
+    # one ragged split tile: its partials keep only the chunk's rows
+    cs = 16384 - rows
+    k, v = _cache(6, cs + rows, cs + rows, "bf16", 0.5)
+    q = synth.draw(6, "q", (rows, 8, 256), "bf16", 0.5)
+    path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, rows)
+    assert path == 1 and len(items) > 8
+    ws = kca.new_workspace(kca.attn_prefill_workspace_bytes(kca.BF16, kca.BF16, cs, rows))
+    out = kca.attn_prefill(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), cs, workspace=ws)
+    want = oracle_prefill(q, k, v, cs, np.arange(rows), 0, "bf16", "bf16")
+    assert max_err(out.cpu().numpy(), want) <= 4e-3
+    _check_status(ws)
+
+
 def test_rows_and_tc_paths_agree(monkeypatch):
     cs, rows = 640, 128
     k, v = _cache(5, cs + rows, cs + rows, "bf16")
