@@ -229,11 +229,55 @@ int attn_append_kv(const void *k_new, const void *v_new, int32_t in_dtype, int32
                    void *k_cache, void *v_cache, int32_t kv_dtype, int64_t cache_rows,
                    const int64_t *dst_rows_dev, int64_t dst_row0, void *workspace, void *stream);
 
+/*
+ * attn_decode_partial / attn_merge_partials -- decode with the context split
+ * into shards (one per GPU, say): each shard yields the partial-softmax state
+ * of every (sequence, head) over the keys it holds, and the states of all
+ * shards merge into the output by the log-sum-exp identity.  The operation is
+ * the decode of Karume v0.12.0 release notes, "Performance", items 2-3 (the
+ * same softmax-weighted sum of V, reduced in a different order), restricted
+ * to a key range; the pages have no multi-device form.
+ *
+ * attn_decode_partial: the cache holds, for each sequence b, the rows of
+ * positions [key_begin, key_begin + capacity) at rows b * capacity +
+ * (position - key_begin).  The query of sequence b sits at ctx_len[b] - 1 as
+ * in attn_decode (ctx_len[b] in 0..KCA_MAX_POSITION, and may lie past the
+ * shard); it sees the keys of its causal / window range that the shard
+ * holds, possibly none.  Output: the partial record `part`, f32, device,
+ * 16-byte aligned, KCA_PARTIAL_FLOATS(batch) floats:
+ *   part[(b * 8 + h) * 2 + 0]  m: reference score (the largest scaled score
+ *                              q.k*scale of the range, or up to 8 ln 2 below it)
+ *   part[(b * 8 + h) * 2 + 1]  l = sum_j exp(s_j - m)
+ *   part[batch * 16 + (b * 8 + h) * 256 + d]  acc = sum_j exp(s_j - m) v_j[d]
+ * An empty range gives (m, l, acc) = (-inf, 0, 0).  A NaN score makes m NaN.
+ * Everything else (q, dtypes, window, scale, workspace >=
+ * attn_decode_partial_workspace_bytes, errors) is as in attn_decode.
+ *
+ * attn_merge_partials: n_parts records (part p at parts + p * part_stride
+ * floats, part_stride >= KCA_PARTIAL_FLOATS(batch) and a multiple of 4;
+ * device, 16-byte aligned) -> out [batch][8][256] f32 with
+ *   M = max_p m_p,  out = sum_p e^(m_p - M) acc_p / sum_p e^(m_p - M) l_p,
+ * combined in part order (the same bits on every call); a row whose parts
+ * are all empty is exactly 0, as in attn_decode.  The merge of the shards'
+ * records equals attn_decode over the whole context up to rounding.
+ */
+#define KCA_PARTIAL_FLOATS(batch) ((size_t)(batch) * 8u * 258u)
+int attn_decode_partial(const void *q, int32_t q_dtype,
+                        const void *k_cache, const void *v_cache, int32_t kv_dtype,
+                        int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity,
+                        int32_t batch, const int64_t *ctx_len, int64_t key_begin, int32_t window,
+                        float scale, float *part, void *workspace, size_t workspace_bytes,
+                        void *stream);
+int attn_merge_partials(int32_t n_parts, int32_t batch, const float *parts, int64_t part_stride,
+                        float *out, void *stream);
+
 /* Workspace bytes the calls above need on the current device (0 on a bad
  * argument).  Always >= KCA_WORKSPACE_HEADER. */
 size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
                                     int32_t chunk_rows, int32_t window);
 size_t attn_decode_workspace_bytes(int32_t batch, const int64_t *ctx_len, int32_t window);
+size_t attn_decode_partial_workspace_bytes(int32_t batch, const int64_t *ctx_len, int64_t key_begin,
+                                           int64_t capacity, int32_t window);
 
 /* Zero the workspace header (cudaMemsetAsync on `stream`). */
 int attn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);

@@ -63,6 +63,13 @@ def lib() -> ctypes.CDLL:
         L.attn_decode_static.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32,
                                          f32, vp, vp]
         L.attn_decode_static.restype = ctypes.c_int
+        L.attn_decode_partial.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i64, i32,
+                                          f32, vp, vp, sz, vp]
+        L.attn_decode_partial.restype = ctypes.c_int
+        L.attn_merge_partials.argtypes = [i32, i32, vp, i64, vp, vp]
+        L.attn_merge_partials.restype = ctypes.c_int
+        L.attn_decode_partial_workspace_bytes.argtypes = [i32, p64, i64, i64, i32]
+        L.attn_decode_partial_workspace_bytes.restype = sz
         L.attn_prefill_workspace_bytes.argtypes = [i32, i32, i64, i32, i32]
         L.attn_prefill_workspace_bytes.restype = sz
         L.attn_decode_workspace_bytes.argtypes = [i32, p64, i32]
@@ -237,6 +244,77 @@ def attn_decode_dev(q, k_cache, v_cache, ctx_len_dev, ctx_bound: int, window: in
                                int(ctx_bound), window, scale, ctypes.c_void_p(out.data_ptr()),
                                ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
     _check(st, "attn_decode_dev")
+    return out
+
+
+def partial_floats(batch: int) -> int:
+    """Floats of one partial record of `batch` sequences: (m, l) pairs
+    [batch][8][2], then acc [batch][8][256]."""
+    return batch * N_Q_HEADS * (2 + HEAD_DIM)
+
+
+def split_partial(part, batch: int):
+    """Views (ml [batch, 8, 2], acc [batch, 8, 256]) of a partial record."""
+    n = batch * N_Q_HEADS * 2
+    return (part[..., :n].reshape(*part.shape[:-1], batch, N_Q_HEADS, 2),
+            part[..., n:n + batch * N_Q_HEADS * HEAD_DIM].reshape(*part.shape[:-1], batch, N_Q_HEADS, HEAD_DIM))
+
+
+def attn_decode_partial_workspace_bytes(ctx_len, key_begin: int, capacity: int, window: int = 0) -> int:
+    arr, ptr = _i64_array(ctx_len)
+    n = lib().attn_decode_partial_workspace_bytes(arr.size, ptr, key_begin, capacity, window)
+    if n == 0:
+        raise KcaError(-4, "attn_decode_partial_workspace_bytes")
+    return int(n)
+
+
+def attn_decode_partial(q, k_shard, v_shard, ctx_len, key_begin: int, window: int = 0,
+                        scale: float = 1.0 / 16.0, part=None, workspace=None, stream=None):
+    """Decode over one context shard, as a partial-softmax record.
+
+    k_shard / v_shard: [batch, capacity, 256] holding positions
+    [key_begin, key_begin + capacity) of each sequence; q: [batch, 8, 256];
+    ctx_len: host ints (the whole context, which may extend past the shard).
+    Returns part, float32 [partial_floats(batch)] (see split_partial).
+    """
+    import torch
+    batch = q.shape[0]
+    capacity = k_shard.shape[1]
+    for t in (q, k_shard, v_shard):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if k_shard.shape[0] != batch:
+        raise ValueError("k_shard batch does not match q")
+    arr, ptr = _i64_array(ctx_len)
+    if arr.size != batch:
+        raise ValueError("ctx_len must have one entry per sequence")
+    if part is None:
+        part = torch.empty(partial_floats(batch), dtype=torch.float32, device=q.device)
+    if part.dtype != torch.float32 or not part.is_contiguous() or part.numel() < partial_floats(batch):
+        raise ValueError("part must be a contiguous float32 tensor of partial_floats(batch) elements")
+    if workspace is None:
+        workspace = new_workspace(attn_decode_partial_workspace_bytes(arr, key_begin, capacity, window),
+                                  q.device, stream)
+    vp = ctypes.c_void_p
+    st = lib().attn_decode_partial(vp(q.data_ptr()), dtype_code(q), vp(k_shard.data_ptr()),
+                                   vp(v_shard.data_ptr()), dtype_code(k_shard), N_Q_HEADS, N_KV_HEADS, HEAD_DIM,
+                                   capacity, batch, ptr, int(key_begin), window, scale, vp(part.data_ptr()),
+                                   vp(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
+    _check(st, "attn_decode_partial")
+    return part
+
+
+def attn_merge_partials(parts, batch: int, out=None, stream=None):
+    """Merge partial records parts [n_parts, stride] (float32, stride >=
+    partial_floats(batch), a multiple of 4) into out [batch, 8, 256]."""
+    import torch
+    if parts.dim() != 2 or parts.dtype != torch.float32 or not parts.is_cuda or parts.stride(1) != 1:
+        raise ValueError("parts must be a float32 CUDA tensor [n_parts, stride] with unit inner stride")
+    if out is None:
+        out = torch.empty((batch, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=parts.device)
+    st = lib().attn_merge_partials(parts.shape[0], batch, ctypes.c_void_p(parts.data_ptr()), parts.stride(0),
+                                   ctypes.c_void_p(out.data_ptr()), _stream_ptr(stream))
+    _check(st, "attn_merge_partials")
     return out
 
 

@@ -81,6 +81,14 @@ std::vector<int64_t> decode_unit_keys(int32_t batch, const int64_t* ctx_len, int
   for (int32_t b = 0; b < batch; ++b) nk[b] = kca::n_visible(ctx_len[b] - 1, window);
   return nk;
 }
+// Keys of each decode query that a context shard [key_begin, key_end) holds.
+std::vector<int64_t> shard_unit_keys(int32_t batch, const int64_t* ctx_len, int32_t window, int64_t key_begin,
+                                     int64_t key_end) {
+  std::vector<int64_t> nk(batch);
+  int64_t lo = 0;
+  for (int32_t b = 0; b < batch; ++b) nk[b] = kca::shard_visible(ctx_len[b] - 1, window, key_begin, key_end, &lo);
+  return nk;
+}
 
 size_t rows_ws_bytes(const kca::RowsPlan& p) {
   if (p.max_splits <= 1) return KCA_WORKSPACE_HEADER;
@@ -97,6 +105,14 @@ int prefill_args_status(int64_t capacity, int64_t chunk_start, int32_t chunk_row
   if (capacity < 1 || capacity > KCA_MAX_POSITION) return KCA_ERR_RANGE;
   if (chunk_rows < 1 || chunk_rows > KCA_MAX_CHUNK_ROWS) return KCA_ERR_RANGE;
   if (chunk_start < 0 || chunk_start + chunk_rows > capacity) return KCA_ERR_RANGE;
+  return KCA_OK;
+}
+
+int shard_args_status(int64_t capacity, int32_t batch, const int64_t* ctx_len, int64_t key_begin) {
+  if (capacity < 1 || key_begin < 0 || key_begin > KCA_MAX_POSITION - capacity) return KCA_ERR_RANGE;
+  if (batch < 1 || batch > KCA_MAX_BATCH) return KCA_ERR_RANGE;
+  for (int32_t b = 0; b < batch; ++b)
+    if (ctx_len[b] < 0 || ctx_len[b] > KCA_MAX_POSITION) return KCA_ERR_RANGE;
   return KCA_OK;
 }
 
@@ -386,6 +402,15 @@ size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t c
   return rows_ws_bytes_any(chunk_rows, nk.data(), sms);
 }
 
+size_t attn_decode_partial_workspace_bytes(int32_t batch, const int64_t* ctx_len, int64_t key_begin,
+                                           int64_t capacity, int32_t window) {
+  if (ctx_len == nullptr || shard_args_status(capacity, batch, ctx_len, key_begin) != KCA_OK) return 0;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return 0;
+  const std::vector<int64_t> nk = shard_unit_keys(batch, ctx_len, window, key_begin, key_begin + capacity);
+  return rows_ws_bytes_any(batch, nk.data(), sms);
+}
+
 size_t attn_decode_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_t window) {
   if (ctx_len == nullptr || decode_args_status(KCA_MAX_POSITION, batch, ctx_len) != KCA_OK) return 0;
   int sms = 0;
@@ -586,6 +611,62 @@ int attn_decode_dev(const void* q, int32_t q_dtype, const void* k_cache, const v
   a.ctx_bound = ctx_bound;
   return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster,
                           workspace, static_cast<cudaStream_t>(stream));
+}
+
+int attn_decode_partial(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache,
+                        int32_t kv_dtype, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                        int64_t capacity, int32_t batch, const int64_t* ctx_len, int64_t key_begin,
+                        int32_t window, float scale, float* part, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (!q || !k_cache || !v_cache || !part || !workspace || !ctx_len) return KCA_ERR_NULL;
+  int st = geometry_status(n_q_heads, n_kv_heads, head_dim);
+  if (st != KCA_OK) return st;
+  if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
+  st = shard_args_status(capacity, batch, ctx_len, key_begin);
+  if (st != KCA_OK) return st;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return KCA_ERR_RANGE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(part)) return KCA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+  const int64_t key_end = key_begin + capacity;
+  const std::vector<int64_t> nk = shard_unit_keys(batch, ctx_len, window, key_begin, key_end);
+  int cluster = 1;
+  size_t need = 0;
+  const kca::RowsPlan p = rows_plan(kv_dtype, batch, nk.data(), sms, &cluster, &need);
+  if (cluster < 1) return KCA_ERR_CUDA;
+  if (workspace_bytes < need) return KCA_ERR_WORKSPACE;
+  kca::RowsArgs a{};
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.out = part + (size_t)batch * kHeads * 2;   // acc follows the (m, l) pairs
+  a.out_ml = part;
+  a.status = workspace;
+  a.seq_rows = capacity;
+  a.mode = 0;
+  a.n_units = batch;
+  a.split_len = p.split_len;
+  a.max_splits = p.max_splits;
+  a.window = window;
+  a.scale = scale;
+  a.key_begin = key_begin;
+  a.key_end = key_end;
+  for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
+  return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster,
+                          workspace, static_cast<cudaStream_t>(stream));
+}
+
+int attn_merge_partials(int32_t n_parts, int32_t batch, const float* parts, int64_t part_stride, float* out,
+                        void* stream) {
+  if (!parts || !out) return KCA_ERR_NULL;
+  if (n_parts < 1 || batch < 1 || batch > KCA_MAX_BATCH) return KCA_ERR_RANGE;
+  if (part_stride < (int64_t)KCA_PARTIAL_FLOATS(batch) || part_stride % 4 != 0) return KCA_ERR_RANGE;
+  if (!aligned16(parts) || !aligned16(out)) return KCA_ERR_ALIGN;
+  return kca::launch_merge_partials(n_parts, batch, parts, part_stride, out, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? KCA_OK
+             : KCA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -246,9 +246,9 @@ __device__ __forceinline__ void merge_cluster_partials(const RowsArgs& a, float*
     load_batch(c0 + NB);
   }
   float* dst = a.out + ((int64_t)unit * kHeads + h) * kDim + W * jd;
-  const bool empty = M == -INFINITY && L == 0.f;
 #pragma unroll
-  for (int e = 0; e < W; ++e) dst[e] = empty ? 0.f : acc[e] / L;
+  for (int e = 0; e < W; ++e) dst[e] = rows_final(a, acc[e], M, L);
+  if (jd == 0) rows_write_ml(a, unit, h, M, L);
 }
 
 template <int W>
@@ -284,8 +284,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
   // with them, the dependency wait comes before they are read.
   if (a.ctx_dev != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, split == 0 && threadIdx.x == 0) - 1 : a.chunk_start + unit;
-  const int64_t lo = lo_of(pos, a.window);
-  const int64_t nkeys = n_visible(pos, a.window);
+  int64_t lo;
+  const int64_t nkeys = rows_keys(a, pos, &lo);
   const int32_t split_len = rows_split_len(a, nkeys, kDStageKeys);
   const int32_t nsplit = rows_n_splits(nkeys, split_len);
   const int nclus = (nsplit + C - 1) / C;
@@ -293,8 +293,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const bool active = split < nsplit && nkeys > 0;
   const int64_t kbeg = lo + (int64_t)split * split_len;
   int64_t kend = kbeg + split_len;
-  if (kend > pos + 1) kend = pos + 1;
-  const int64_t base_row = a.mode == 0 ? (int64_t)unit * a.seq_rows : 0;
+  if (kend > lo + nkeys) kend = lo + nkeys;
+  // cache row of key p: base_row + p (a shard's row 0 is position key_begin)
+  const int64_t base_row = (a.mode == 0 ? (int64_t)unit * a.seq_rows : 0) - a.key_begin;
   const int n_stage = active ? (int)cdiv(kend - kbeg, kDStageKeys) : 0;
 
   if (threadIdx.x == 0) {
@@ -574,7 +575,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
         O += f * ov[src];
       }
       if (nclus == 1) {
-        a.out[((int64_t)unit * kHeads + h) * kDim + d] = (M == -INFINITY && L == 0.f) ? 0.f : O / L;
+        a.out[((int64_t)unit * kHeads + h) * kDim + d] = rows_final(a, O, M, L);
+        if (d == 0) rows_write_ml(a, unit, h, M, L);
         continue;
       }
       const int64_t cslot = ((int64_t)unit * a.max_clusters + clus) * kHeads + h;

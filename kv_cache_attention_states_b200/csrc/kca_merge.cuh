@@ -26,7 +26,8 @@ namespace kca {
 template <int W>
 __device__ __forceinline__ void merge_row(int ns, const float* ml, int64_t ml_stride,
                                           const float* acc, int64_t acc_stride, float mscale,
-                                          float* out, float* red, int g, int lane, int bar_id) {
+                                          float* out, float* red, int g, int lane, int bar_id,
+                                          float* out_ml = nullptr) {
   float M = -INFINITY;
   for (int s = g * 32 + lane; s < ns; s += W * 32) M = max_nan(M, ml[s * ml_stride]);
 #pragma unroll
@@ -63,7 +64,13 @@ __device__ __forceinline__ void merge_row(int ns, const float* ml, int64_t ml_st
       for (int i = 0; i < 8; ++i) A[i] += o[8 + 8 * lane + i];
     }
   }
-  const float inv = 1.f / L;
+  // out_ml set: the merged partial (M, L) and unnormalised acc instead; a
+  // row of empty partials only (M = -inf, L = 0) is exactly zero
+  const float inv = out_ml != nullptr ? 1.f : (M == -INFINITY && L == 0.f) ? 0.f : 1.f / L;
+  if (out_ml != nullptr && lane == 0) {
+    out_ml[0] = M;
+    out_ml[1] = L;
+  }
   float4* o4 = reinterpret_cast<float4*>(out + 8 * lane);
   o4[0] = make_float4(A[0] * inv, A[1] * inv, A[2] * inv, A[3] * inv);
   o4[1] = make_float4(A[4] * inv, A[5] * inv, A[6] * inv, A[7] * inv);

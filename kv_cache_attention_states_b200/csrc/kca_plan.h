@@ -37,6 +37,16 @@ KCA_HD int64_t n_visible(int64_t pos, int32_t window) {
   return pos >= lo ? pos - lo + 1 : 0;
 }
 KCA_HD int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+// Visible keys of the query at pos that a context shard holding positions
+// [key_begin, key_end) sees: [*lo, *lo + n), n returned (key_end <= 0: no
+// upper end, i.e. the whole context from key_begin on).
+KCA_HD int64_t shard_visible(int64_t pos, int32_t window, int64_t key_begin, int64_t key_end, int64_t* lo) {
+  int64_t l = lo_of(pos, window), h = pos + 1;
+  if (l < key_begin) l = key_begin;
+  if (key_end > 0 && h > key_end) h = key_end;
+  *lo = l;
+  return h > l ? h - l : 0;
+}
 
 // ------------------------------------------------------------ rows path
 // One unit = one query row (prefill) or one sequence (decode).  Its visible

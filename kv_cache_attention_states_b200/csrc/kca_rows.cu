@@ -78,20 +78,22 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
   const int lane = threadIdx.x & 31;
 
   const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, split == 0 && threadIdx.x == 0) - 1 : a.chunk_start + unit;
-  const int64_t lo = lo_of(pos, a.window);
-  const int64_t nkeys = n_visible(pos, a.window);
+  int64_t lo;
+  const int64_t nkeys = rows_keys(a, pos, &lo);
   const int32_t split_len = rows_split_len(a, nkeys, kRowsSplitQuantum);
   const int32_t nsplit = rows_n_splits(nkeys, split_len);
   if (split >= nsplit) return;
   const int64_t kbeg = lo + (int64_t)split * split_len;
   int64_t kend = kbeg + split_len;
-  if (kend > pos + 1) kend = pos + 1;
-  const int64_t base_row = a.mode == 0 ? (int64_t)unit * a.seq_rows : 0;
+  if (kend > lo + nkeys) kend = lo + nkeys;
+  // cache row of key p: base_row + p (a shard's row 0 is position key_begin)
+  const int64_t base_row = (a.mode == 0 ? (int64_t)unit * a.seq_rows : 0) - a.key_begin;
   float* out = a.out + (int64_t)unit * kHeads * kDim;
 
-  if (nkeys == 0) {  // fully masked row: exactly zero
+  if (nkeys == 0) {  // fully masked row: exactly zero (as a partial: (-inf, 0, 0))
     if (warp < kComputeWarps)
       for (int i = threadIdx.x; i < kHeads * kDim; i += kComputeWarps * 32) out[i] = 0.f;
+    if (threadIdx.x < kHeads) rows_write_ml(a, unit, threadIdx.x, -INFINITY, 0.f);
     return;
   }
   const int n_stage = (int)cdiv(kend - kbeg, kKeysPerStage);
@@ -272,10 +274,11 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
         A[4] += f * x1.x; A[5] += f * x1.y; A[6] += f * x1.z; A[7] += f * x1.w;
       }
       if (nsplit == 1) {
-        const float inv = 1.f / L;
+        const float inv = a.out_ml != nullptr ? 1.f : 1.f / L;
         float4* o = reinterpret_cast<float4*>(out + h * kDim + 8 * lane);
         o[0] = make_float4(A[0] * inv, A[1] * inv, A[2] * inv, A[3] * inv);
         o[1] = make_float4(A[4] * inv, A[5] * inv, A[6] * inv, A[7] * inv);
+        if (lane == 0) rows_write_ml(a, unit, h, M, L);
       } else {
         const int64_t slot = (int64_t)unit * a.max_splits + split;
         if (lane == 0) {
@@ -295,14 +298,15 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
 __global__ void __launch_bounds__(256) merge_rows_kernel(const RowsArgs a) {
   const int unit = blockIdx.x >> 3, h = blockIdx.x & 7;
   const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, false) - 1 : a.chunk_start + unit;
-  const int64_t nkeys = n_visible(pos, a.window);
+  int64_t lo;
+  const int64_t nkeys = rows_keys(a, pos, &lo);
   const int32_t nsplit = rows_n_splits(nkeys, rows_split_len(a, nkeys, kRowsSplitQuantum));
   if (nsplit <= 1) return;
   __shared__ float red[8 * 264];
   const int64_t row0 = (int64_t)unit * a.max_splits * kHeads + h;
   merge_row<8>(nsplit, a.part_ml + row0 * 2, kHeads * 2, a.part_acc + row0 * kDim, kHeads * kDim,
                kLog2e, a.out + ((int64_t)unit * kHeads + h) * kDim, red, threadIdx.x >> 5,
-               threadIdx.x & 31, 1);
+               threadIdx.x & 31, 1, a.out_ml != nullptr ? a.out_ml + ((int64_t)unit * kHeads + h) * 2 : nullptr);
 }
 
 template <int QT, int KT>

@@ -37,6 +37,15 @@ struct RowsArgs {
   // itself (rows_split_len); null for the host-array form.
   const int64_t* ctx_dev;
   int64_t ctx_bound;
+  // Context shard (decode): cache row r of a sequence holds position
+  // key_begin + r, and only positions [key_begin, key_end) are seen
+  // (key_end <= 0: no upper end).  Zero for a whole cache.
+  int64_t key_begin;
+  int64_t key_end;
+  // Partial-softmax output (decode): non-null, each (unit, head) gets
+  // (m, l) here -- m the max scaled score, l the sum of exp(s - m) -- and
+  // its unnormalised sum of exp(s - m) v in out; null: out = that sum / l.
+  float* out_ml;
   int64_t ctx[KCA_MAX_BATCH];  // decode: ctx_len per sequence
 };
 
@@ -54,6 +63,24 @@ __device__ __forceinline__ int64_t rows_ctx(const RowsArgs& a, int unit, bool re
   if (record) record_error(static_cast<DeviceStatus*>(a.status), kSiteCtx, kErrBadCtx, (unsigned)unit);
   return 0;
 }
+// Visible keys [*lo, *lo + n) of the query at pos within the cache's shard.
+__device__ __forceinline__ int64_t rows_keys(const RowsArgs& a, int64_t pos, int64_t* lo) {
+  return shard_visible(pos, a.window, a.key_begin, a.key_end, lo);
+}
+// Final writes of (unit, head) h: rows_write_ml stores its (M, L) when the
+// output is a partial-softmax record (a.out_ml set); rows_final gives the
+// value of one output dim, acc / L normalised or acc itself in a record.  An
+// empty row (M = -inf, L = 0) is exactly zero, or (-inf, 0, 0) in a record.
+__device__ __forceinline__ void rows_write_ml(const RowsArgs& a, int unit, int h, float M, float L) {
+  if (a.out_ml != nullptr) {
+    a.out_ml[((int64_t)unit * kHeads + h) * 2 + 0] = M;
+    a.out_ml[((int64_t)unit * kHeads + h) * 2 + 1] = L;
+  }
+}
+__device__ __forceinline__ float rows_final(const RowsArgs& a, float acc, float M, float L) {
+  if (a.out_ml != nullptr) return acc;
+  return (M == -INFINITY && L == 0.f) ? 0.f : acc / L;
+}
 // Keys per split of a unit with nkeys visible keys: the host plan's length,
 // or with device context lengths the smallest multiple of `quantum` (>= 64)
 // that cuts nkeys into at most max_splits splits.
@@ -69,6 +96,11 @@ cudaError_t launch_rows(int q_dtype, int kv_dtype, const RowsArgs& a, cudaStream
 
 // Log-sum-exp merge of the split partials in a (units with more than one split).
 cudaError_t launch_merge_rows(const RowsArgs& a, cudaStream_t stream);
+
+// Merge of n_parts partial records (layout of attn_decode_partial; record p
+// at parts + p * part_stride floats) into out [batch][8][256] (kca_context.cu).
+cudaError_t launch_merge_partials(int n_parts, int batch, const float* parts, int64_t part_stride, float* out,
+                                  cudaStream_t stream);
 
 // Clusters of c CTAs of the tensor-core rows kernel that fit on the device at
 // once (0 on failure).

@@ -118,6 +118,47 @@ def test_decode_dev_rejects_bad_arguments_on_the_host(kw, code):
     assert _decode_dev(**kw) == code
 
 
+def _decode_partial(ctx=(100, 5000), **kw):
+    a = dict(q=P, qd=kca.F32, k=P, v=P, kd=kca.F16, hq=8, hkv=1, d=256, cap=4096, kb=4096, window=0,
+             scale=0.0625, part=P, ws=P * 2, wsb=1 << 30, batch=None)
+    a.update(kw)
+    arr = np.asarray(ctx, dtype=np.int64)
+    batch = len(arr) if a["batch"] is None else a["batch"]
+    vp = ctypes.c_void_p
+    return kca.lib().attn_decode_partial(vp(a["q"]), a["qd"], vp(a["k"]), vp(a["v"]), a["kd"], a["hq"],
+                                         a["hkv"], a["d"], a["cap"], batch,
+                                         arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), a["kb"],
+                                         a["window"], a["scale"], vp(a["part"]), vp(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("ctx,kw,code", [
+    ((1, 2), dict(part=0), -1), ((1, 2), dict(q=0), -1), ((1, 2), dict(d=64), -2), ((1, 2), dict(qd=9), -3),
+    ((1, 2), dict(batch=0), -4), ((1,) * 257, dict(), -4), ((1, 131073), dict(), -4), ((-1, 2), dict(), -4),
+    ((1, 2), dict(kb=-1), -4), ((1, 2), dict(cap=0), -4), ((1, 2), dict(kb=131072 - 4095), -4),
+    ((1, 2), dict(scale=float("nan")), -4),
+    ((1, 2), dict(part=P + 4), -6), ((1, 2), dict(k=P + 8), -6), ((1, 2), dict(ws=P * 2 + 128), -5),
+])
+def test_decode_partial_rejects_bad_arguments_on_the_host(ctx, kw, code):
+    # ctx may lie past the shard (the rest of the context is on other ranks)
+    assert _decode_partial(ctx, **kw) == code
+
+
+@pytest.mark.parametrize("n,batch,stride,parts,out,code", [
+    (2, 1, 2064, 0, P, -1), (2, 1, 2064, P, 0, -1), (0, 1, 2064, P, P, -4), (2, 0, 2064, P, P, -4),
+    (2, 257, 1 << 20, P, P, -4), (2, 1, 2060, P, P, -4), (2, 1, 2066, P, P, -4), (2, 2, 2064, P, P, -4),
+    (2, 1, 2064, P + 4, P, -6), (2, 1, 2064, P, P + 8, -6),
+])
+def test_merge_partials_rejects_bad_arguments_on_the_host(n, batch, stride, parts, out, code):
+    vp = ctypes.c_void_p
+    assert kca.lib().attn_merge_partials(n, batch, vp(parts), stride, vp(out), None) == code
+
+
+def test_partial_record_layout():
+    assert kca.partial_floats(3) == 3 * 8 * 258
+    text = open(HEADER).read()
+    assert re.search(r"#define KCA_PARTIAL_FLOATS\(batch\) \(\(size_t\)\(batch\) \* 8u \* 258u\)", text)
+
+
 def _append(**kw):
     a = dict(k=P, v=P, it=kca.F32, n=4, cos=P * 3, sin=P * 4, kc=P * 5, vc=P * 6, kt=kca.F16, rows=100,
              dst=None, dst0=0, ws=None)
