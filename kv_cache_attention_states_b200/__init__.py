@@ -92,23 +92,48 @@ def status_string(status: int) -> str:
     return lib().attn_status_string(int(status)).decode()
 
 
+_CODES = None
+
+
 def dtype_code(t) -> int:
-    import torch
-    codes = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
-    if t.dtype not in codes:
+    global _CODES
+    if _CODES is None:
+        import torch
+        _CODES = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+    code = _CODES.get(t.dtype)
+    if code is None:
         raise TypeError(f"unsupported dtype {t.dtype}")
-    return codes[t.dtype]
+    return code
 
 
-def _stream_ptr(stream):
+def _stream_ptr(stream, device=None):
+    """cudaStream_t of `stream`, else of torch's current stream on `device`
+    (a torch.device, an index, or None for the current device).  The current
+    stream is read through torch's raw-stream query, which costs a fraction
+    of building a torch.cuda.Stream object per call."""
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
     import torch
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    idx = device.index if isinstance(device, torch.device) else device
+    if idx is None:
+        idx = torch.cuda.current_device()
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return ctypes.c_void_p(raw(idx))
+    return ctypes.c_void_p(torch.cuda.current_stream(idx).cuda_stream)
+
+
+_I64P = ctypes.POINTER(ctypes.c_int64)
 
 
 def _i64_array(vals):
+    """(n, pointer) of host int64 values; the pointer object keeps them alive.
+    Short lists and tuples become a ctypes array directly (no numpy round
+    trip), anything else goes through numpy."""
+    if isinstance(vals, (list, tuple)) and len(vals) <= 64:
+        return len(vals), (ctypes.c_int64 * len(vals))(*vals)
     arr = np.ascontiguousarray(np.asarray(vals, dtype=np.int64).reshape(-1))
-    return arr, arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+    return arr.size, arr.ctypes.data_as(_I64P)
 
 
 def _check(status: int, what: str):
@@ -127,8 +152,8 @@ def attn_prefill_workspace_bytes(q_dtype: int, kv_dtype: int, chunk_start: int, 
 
 
 def attn_decode_workspace_bytes(ctx_len, window: int = 0) -> int:
-    arr, ptr = _i64_array(ctx_len)
-    n = lib().attn_decode_workspace_bytes(arr.size, ptr, window)
+    nctx, ptr = _i64_array(ctx_len)
+    n = lib().attn_decode_workspace_bytes(nctx, ptr, window)
     if n == 0:
         raise KcaError(-4, "attn_decode_workspace_bytes")
     return int(n)
@@ -201,13 +226,13 @@ def attn_decode(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.
             raise ValueError("tensors must be contiguous CUDA tensors")
     if k_cache.shape[0] != batch:
         raise ValueError("k_cache batch does not match q")
-    arr, ptr = _i64_array(ctx_len)
-    if arr.size != batch:
+    nctx, ptr = _i64_array(ctx_len)
+    if nctx != batch:
         raise ValueError("ctx_len must have one entry per sequence")
     if out is None:
         out = torch.empty((batch, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = new_workspace(attn_decode_workspace_bytes(arr, window), q.device, stream)
+        workspace = new_workspace(attn_decode_workspace_bytes(ctx_len, window), q.device, stream)
     st = lib().attn_decode(ctypes.c_void_p(q.data_ptr()), dtype_code(q), ctypes.c_void_p(k_cache.data_ptr()),
                            ctypes.c_void_p(v_cache.data_ptr()), dtype_code(k_cache), N_Q_HEADS,
                            N_KV_HEADS, HEAD_DIM, capacity, batch, ptr, window, scale,
@@ -261,8 +286,8 @@ def split_partial(part, batch: int):
 
 
 def attn_decode_partial_workspace_bytes(ctx_len, key_begin: int, capacity: int, window: int = 0) -> int:
-    arr, ptr = _i64_array(ctx_len)
-    n = lib().attn_decode_partial_workspace_bytes(arr.size, ptr, key_begin, capacity, window)
+    nctx, ptr = _i64_array(ctx_len)
+    n = lib().attn_decode_partial_workspace_bytes(nctx, ptr, key_begin, capacity, window)
     if n == 0:
         raise KcaError(-4, "attn_decode_partial_workspace_bytes")
     return int(n)
@@ -285,15 +310,15 @@ def attn_decode_partial(q, k_shard, v_shard, ctx_len, key_begin: int, window: in
             raise ValueError("tensors must be contiguous CUDA tensors")
     if k_shard.shape[0] != batch:
         raise ValueError("k_shard batch does not match q")
-    arr, ptr = _i64_array(ctx_len)
-    if arr.size != batch:
+    nctx, ptr = _i64_array(ctx_len)
+    if nctx != batch:
         raise ValueError("ctx_len must have one entry per sequence")
     if part is None:
         part = torch.empty(partial_floats(batch), dtype=torch.float32, device=q.device)
     if part.dtype != torch.float32 or not part.is_contiguous() or part.numel() < partial_floats(batch):
         raise ValueError("part must be a contiguous float32 tensor of partial_floats(batch) elements")
     if workspace is None:
-        workspace = new_workspace(attn_decode_partial_workspace_bytes(arr, key_begin, capacity, window),
+        workspace = new_workspace(attn_decode_partial_workspace_bytes(ctx_len, key_begin, capacity, window),
                                   q.device, stream)
     vp = ctypes.c_void_p
     st = lib().attn_decode_partial(vp(q.data_ptr()), dtype_code(q), vp(k_shard.data_ptr()),
@@ -364,8 +389,8 @@ def attn_decode_static(q, k_cache, v_cache, ctx_len, window: int = 0, scale: flo
     workspace (see include/kca.h for the sharing rules)."""
     import torch
     batch = q.shape[0]
-    arr, ptr = _i64_array(ctx_len)
-    if arr.size != batch or k_cache.shape[0] != batch:
+    nctx, ptr = _i64_array(ctx_len)
+    if nctx != batch or k_cache.shape[0] != batch:
         raise ValueError("ctx_len / k_cache must have one entry per sequence")
     if out is None:
         out = torch.empty((batch, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
@@ -398,13 +423,13 @@ def attn_prefill_plan(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows:
 
 
 def attn_decode_plan(ctx_len, window: int = 0, num_sms: int = 148):
-    arr, ptr = _i64_array(ctx_len)
+    nctx, ptr = _i64_array(ctx_len)
     n = ctypes.c_int32(0)
-    st = lib().attn_decode_plan(arr.size, ptr, window, num_sms, None, 0, ctypes.byref(n))
+    st = lib().attn_decode_plan(nctx, ptr, window, num_sms, None, 0, ctypes.byref(n))
     if st not in (0, -4) or (st == -4 and n.value == 0):
         raise KcaError(st, "attn_decode_plan")
     items = np.zeros((max(n.value, 1), 4), dtype=np.int64)
-    st = lib().attn_decode_plan(arr.size, ptr, window, num_sms,
+    st = lib().attn_decode_plan(nctx, ptr, window, num_sms,
                                 items.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n.value,
                                 ctypes.byref(n))
     _check(st, "attn_decode_plan")

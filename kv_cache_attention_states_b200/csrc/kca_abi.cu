@@ -143,22 +143,64 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// A tensor map is a pure function of its encode arguments, so the last few
+// encodings of each host thread are kept and a repeated argument set (the
+// same cache or chunk buffer call after call) is copied instead of
+// re-encoded.  All maps here are 2-D, 128-byte swizzled, zero-filled.
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType t, const void* base, const cuuint64_t (&dims)[2],
+               cuuint64_t stride, const cuuint32_t (&box)[2]) {
+  struct Entry {
+    const void* base;
+    cuuint64_t dims[2];
+    cuuint64_t stride;
+    cuuint32_t box[2];
+    int t;
+    bool valid;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 16;
+  thread_local Entry cache[kEntries] = {};
+  thread_local int next = 0;
+  for (int i = 0; i < kEntries; ++i) {
+    const Entry& e = cache[i];
+    if (e.valid && e.base == base && e.t == (int)t && e.dims[0] == dims[0] && e.dims[1] == dims[1] &&
+        e.stride == stride && e.box[0] == box[0] && e.box[1] == box[1]) {
+      *m = e.map;
+      return true;
+    }
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(m, t, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  Entry& e = cache[next];
+  next = (next + 1) % kEntries;
+  e.base = base;
+  e.dims[0] = dims[0];
+  e.dims[1] = dims[1];
+  e.stride = stride;
+  e.box[0] = box[0];
+  e.box[1] = box[1];
+  e.t = (int)t;
+  e.map = *m;
+  e.valid = true;
+  return true;
+}
+
 // Map over rows [kv_lo, ctx_len) of one cache: inner extent 256 elements,
 // boxes of 64 elements x box_rows rows, 128-byte swizzle, zero fill outside.
 bool encode_kv_map(CUtensorMap* m, const void* cache, int32_t dtype, int64_t kv_lo, int64_t ctx_len,
                    uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
   const char* base = static_cast<const char*>(cache) + kv_lo * kDim * 2;
-  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)(ctx_len - kv_lo)};
-  cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)(ctx_len - kv_lo)};
+  const cuuint32_t box[2] = {64, box_rows};
   const CUtensorMapDataType t =
       dtype == KCA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  return fn(m, t, 2, const_cast<char*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_2d(m, t, base, dims, (cuuint64_t)kDim * 2, box);
 }
 
 // 2-D map over `rows` rows of 256 elements (f32 or 16-bit), box {box_x,
@@ -166,19 +208,14 @@ bool encode_kv_map(CUtensorMap* m, const void* cache, int32_t dtype, int64_t kv_
 // clipped.
 bool encode_rows_map(CUtensorMap* m, const void* base, int32_t dtype, int64_t rows, uint32_t box_x,
                      uint32_t box_rows = 128) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr || rows < 1) return false;
+  if (rows < 1) return false;
   const int esz = dtype == KCA_F32 ? 4 : 2;
-  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kDim * esz};
-  cuuint32_t box[2] = {box_x, box_rows};
-  cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
+  const cuuint32_t box[2] = {box_x, box_rows};
   const CUtensorMapDataType t = dtype == KCA_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                 : dtype == KCA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  return fn(m, t, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_2d(m, t, base, dims, (cuuint64_t)kDim * esz, box);
 }
 
 void carve(void* ws, size_t ml_bytes, float** ml, float** acc) {
