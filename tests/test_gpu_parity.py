@@ -224,3 +224,26 @@ def test_decode_tensor_core_and_cuda_core_paths_agree(monkeypatch, q_dtype, kv_d
     simt = kca.attn_decode(*args).cpu().numpy()
     want = oracle_decode(q, k, v, ctx, 0, q_dtype, kv_dtype, cap)
     assert max_err(mma, want) <= 4e-3 and max_err(simt, want) <= 4e-3
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("f32", "f16"), ("f32", "f32")])
+def test_decode_at_the_maximum_batch(q_dtype, kv_dtype):
+    # KCA_MAX_BATCH sequences, ragged lengths including an empty context and
+    # one at the capacity: tensor-core (f16) and CUDA-core (f32) kernels
+    batch, cap = kca.MAX_BATCH, 2048
+    ctx = synth.integers(21, "ctx", 0, cap, batch)
+    ctx[0], ctx[1], ctx[2] = 0, cap, 1
+    k, v = _cache(21, cap, ctx, kv_dtype, batch=batch)
+    q = synth.draw(21, "q", (batch, 8, 256), q_dtype)
+    ws = kca.new_workspace(kca.attn_decode_workspace_bytes(ctx))
+    out = kca.attn_decode(dev(q, q_dtype), dev(k, kv_dtype), dev(v, kv_dtype), ctx, workspace=ws)
+    want = oracle_decode(q, k, v, ctx, 0, q_dtype, kv_dtype, cap)
+    assert max_err(out.cpu().numpy(), want) <= tol(q_dtype, kv_dtype)
+    assert torch.all(out[0] == 0)
+    _check_status(ws)
+    one_more = batch + 1                            # past the limit: rejected before any launch
+    qx = torch.zeros((one_more, 8, 256), dtype=torch.float32, device="cuda")
+    kx = torch.zeros((one_more, 16, 256), dtype=torch.float16, device="cuda")
+    with pytest.raises(kca.KcaError):
+        kca.attn_decode(qx, kx, kx.clone(), [1] * one_more)
+
