@@ -481,13 +481,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Log-sum-exp merge of the items of each split row tile.  WPR warps per M
 // row (8 / WPR rows per CTA, grid (tiles, 16 WPR)); warp sub of a row takes
 // the contiguous items [sub n, sub n + n) of the tile's ns, lane k owning
-// dims [8k, 8k+8), with the (m, l) and acc of eight items in flight at once
-// and an online rescale across groups of eight.  With WPR > 1 the warps'
+// dims [8k, 8k+8), with the (m, l) and acc of NB items in flight at once
+// and an online rescale across groups of NB.  NB = 4 when no tile has more
+// than four items: its registers then let the whole grid (6,144 rows of a
+// 768-row chunk) be resident in one wave, where NB = 8 needs two.  With WPR > 1 the warps'
 // partials of a row are combined in shared memory in sub order.  Items and
 // sub-ranges are combined in slot order, so the result is the same bits on
 // every call.  Many items per tile (few tiles in the chunk) take more warps
 // per row, so that no warp waits on more than a few load round trips.
-template <int WPR>
+template <int WPR, int NB>
 __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -504,11 +506,11 @@ __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
   const int64_t r0 = (int64_t)a.tile_first_slot[tile] * 128 + m;    // item s: row r0 + 128 s
   float M = -INFINITY, L = 0.f;
   float4 A0 = make_float4(0.f, 0.f, 0.f, 0.f), A1 = A0;
-  for (int s0 = sb; row_ok && s0 < se; s0 += 8) {
-    float mv[8], lv[8];
-    float4 v0[8], v1[8];
+  for (int s0 = sb; row_ok && s0 < se; s0 += NB) {
+    float mv[NB], lv[NB];
+    float4 v0[NB], v1[NB];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < NB; ++j) {
       const int64_t r = r0 + (int64_t)(s0 + j) * 128;
       const bool in = s0 + j < se;
       mv[j] = in ? a.part_ml[r * 2] : -INFINITY;
@@ -519,14 +521,14 @@ __global__ void __launch_bounds__(256) merge_tc_kernel(const TcArgs a) {
     }
     float Mn = M;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) Mn = max_nan(Mn, mv[j]);
+    for (int j = 0; j < NB; ++j) Mn = max_nan(Mn, mv[j]);
     const float mu = Mn == -INFINITY ? 0.f : Mn;
     const float alpha = exp2f(M - mu);   // m is in log2 units
     L *= alpha;
     A0.x *= alpha; A0.y *= alpha; A0.z *= alpha; A0.w *= alpha;
     A1.x *= alpha; A1.y *= alpha; A1.z *= alpha; A1.w *= alpha;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < NB; ++j) {
       const float f = exp2f(mv[j] - mu);
       L += f * lv[j];
       A0.x += f * v0[j].x; A0.y += f * v0[j].y; A0.z += f * v0[j].z; A0.w += f * v0[j].w;
@@ -604,10 +606,11 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.numAttrs = 1;   // no cluster
-  if (wpr == 1) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<1>, a);
-  if (wpr == 2) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<2>, a);
-  if (wpr == 4) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<4>, a);
-  return cudaLaunchKernelEx(&cfg, merge_tc_kernel<8>, a);
+  if (ns_max <= 4) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<1, 4>, a);
+  if (wpr == 1) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<1, 8>, a);
+  if (wpr == 2) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<2, 8>, a);
+  if (wpr == 4) return cudaLaunchKernelEx(&cfg, merge_tc_kernel<4, 8>, a);
+  return cudaLaunchKernelEx(&cfg, merge_tc_kernel<8, 8>, a);
 }
 
 }  // namespace
