@@ -135,6 +135,37 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, int dt) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// p = 2^(s cs + nmu) for the 64 scores of a half row (one FFMA, over pairs,
+// and one MUFU op per score), packed as 16-bit pairs into pr; returns their sum.
+template <int DT>
+__device__ __forceinline__ float exp_pack(const float (&s)[64], float cs, float nmu, uint32_t (&pr)[32]) {
+  const float2 cs2 = make_float2(cs, cs), nmu2 = make_float2(nmu, nmu);
+  float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), cs2, nmu2);
+    const float p0 = ptx::ex2(x.x), p1 = ptx::ex2(x.y);
+    acc2[c & 3] = __fadd2_rn(acc2[c & 3], make_float2(p0, p1));
+    pr[c] = pack2(p0, p1, DT);
+  }
+  acc2[0] = __fadd2_rn(acc2[0], acc2[1]);
+  acc2[2] = __fadd2_rn(acc2[2], acc2[3]);
+  acc2[0] = __fadd2_rn(acc2[0], acc2[2]);
+  return acc2[0].x + acc2[0].y;
+}
+
+// Named barrier of n threads that also returns whether v held in any of them.
+__device__ __forceinline__ bool bar_red_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pin, pout;\n setp.ne.u32 pin, %1, 0;\n bar.red.or.pred pout, %2, %3, pin;\n"
+      " selp.u32 %0, 1, 0, pout;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -344,7 +375,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::fence_before_sync();
       arrive_leader(&bars->s_free);   // S may be overwritten by the next QK^T
-      float mloc = -INFINITY;
       if (ok) {
         // keys outside [lo, pos] become -inf (scale > 0 keeps them there)
         const int64_t j0 = a.plan.kv_lo + (int64_t)(it.kt_begin + t) * kKeyTile + 64 * wg;
@@ -355,63 +385,72 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j < lo || j > pos) s[c] = -INFINITY;
           }
         }
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-        for (int c = 8; c < 64; ++c) m8[c & 7] = max_nan(m8[c & 7], s[c]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m8[i] = max_nan(m8[i], m8[i + 4]);
-        mloc = max_nan(max_nan(m8[0], m8[2]), max_nan(m8[1], m8[3]));
       }
-      // The row max spans both warpgroups: exchange halves (buffer by tile parity).
-      bars->red_max[t & 1][wg][m] = mloc;
-      named_sync(1, kSoftmaxThreads);
-      const float mraw = max_nan(mloc, bars->red_max[t & 1][wg ^ 1][m]);
-      if (!ok) continue;
-      const float mx = mraw == -INFINITY ? -INFINITY : mraw * cs;
-      const bool need = mx > m_ref + kRescaleLog2;   // identical in both warpgroups
-      const bool any_need = __any_sync(0xffffffffu, need);
-      if (any_need) {
-        const float alpha = need ? ptx::ex2(m_ref - mx) : 1.f;
-        if (need) m_ref = mx;
-        l_sum *= alpha;
-        if (t > 0) {
-          // PV of the previous tile must finish before O is rescaled; PV of
-          // tile t-2 is known complete here (it preceded this tile's QK^T),
-          // so the parity wait on barrier (t-1)&1 is unambiguous.
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1,
-                                                 abort_flag, status, kSiteTcO));
-          if (!ok) continue;
-          ptx::fence_after_sync();
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(trow + kColO + 128 * wg + 32 * c, r);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            ptx::tmem_st32(trow + kColO + 128 * wg + 32 * c, r);
-          }
-          ptx::tmem_wait_st();
-        }
-      }
-      // p = 2^(s*scale*log2e - m_ref): one FFMA and one MUFU op per score.
-      const float nmu = m_ref == -INFINITY ? 0.f : -m_ref;
+      // Probabilities with the current reference first.  When their sum
+      // over this half row is at most 2^8, none of them exceeds 2^8 and the
+      // reference stands: no row max is needed, which is the common case
+      // once a row has seen its first keys.  Otherwise -- the row's first
+      // visible tile, a score past the reference by more than 2^8 in either
+      // half, a NaN score -- every row of the pair of warpgroups takes the
+      // max exchange below, exactly as if no probability had been taken.
       uint32_t pr[32];
-      float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ptx::ex2(fmaf(s[2 * c], cs, nmu));
-        const float p1 = ptx::ex2(fmaf(s[2 * c + 1], cs, nmu));
-        acc2[c & 3] = __fadd2_rn(acc2[c & 3], make_float2(p0, p1));
-        pr[c] = pack2(p0, p1, DT);
+      float lt = 0.f;
+      const bool done = ok && m_ref != -INFINITY;
+      bool redo = ok;
+      if (done) {
+        lt = exp_pack<DT>(s, cs, -m_ref, pr);
+        redo = !(lt <= 256.f);
       }
-      acc2[0] = __fadd2_rn(acc2[0], acc2[1]);
-      acc2[2] = __fadd2_rn(acc2[2], acc2[3]);
-      acc2[0] = __fadd2_rn(acc2[0], acc2[2]);
-      l_sum += acc2[0].x + acc2[0].y;
+      if (bar_red_or(2, kSoftmaxThreads, redo)) {
+        float mloc = -INFINITY;
+        if (ok) {
+          float m8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+          for (int c = 8; c < 64; ++c) m8[c & 7] = max_nan(m8[c & 7], s[c]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) m8[i] = max_nan(m8[i], m8[i + 4]);
+          mloc = max_nan(max_nan(m8[0], m8[2]), max_nan(m8[1], m8[3]));
+        }
+        // The row max spans both warpgroups: exchange halves (buffer by tile parity).
+        bars->red_max[t & 1][wg][m] = mloc;
+        named_sync(1, kSoftmaxThreads);
+        const float mraw = max_nan(mloc, bars->red_max[t & 1][wg ^ 1][m]);
+        if (!ok) continue;
+        const float mx = mraw == -INFINITY ? -INFINITY : mraw * cs;
+        const bool need = mx > m_ref + kRescaleLog2;   // identical in both warpgroups
+        const bool any_need = __any_sync(0xffffffffu, need);
+        if (any_need) {
+          const float alpha = need ? ptx::ex2(m_ref - mx) : 1.f;
+          if (need) m_ref = mx;
+          l_sum *= alpha;
+          if (t > 0) {
+            // PV of the previous tile must finish before O is rescaled; PV of
+            // tile t-2 is known complete here (it preceded this tile's QK^T),
+            // so the parity wait on barrier (t-1)&1 is unambiguous.
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1,
+                                                   abort_flag, status, kSiteTcO));
+            if (!ok) continue;
+            ptx::fence_after_sync();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t r[32];
+              ptx::tmem_ld32(trow + kColO + 128 * wg + 32 * c, r);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              ptx::tmem_st32(trow + kColO + 128 * wg + 32 * c, r);
+            }
+            ptx::tmem_wait_st();
+          }
+        }
+        // A sum past 2^8 whose max stayed within 2^8 of the reference keeps
+        // the probabilities already taken.
+        if (!done || need) lt = exp_pack<DT>(s, cs, m_ref == -INFINITY ? 0.f : -m_ref, pr);
+      }
+      if (!ok) continue;
+      l_sum += lt;
       // P row m, keys [64 wg, 64 wg + 64): 32 TMEM columns of 16-bit pairs in
       // buffer t&1.  PV of tile t-2, the last reader of that buffer, has
       // completed: it preceded QK^T of this tile, whose completion s_full signalled.
