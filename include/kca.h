@@ -189,8 +189,12 @@ int attn_decode_dev(const void *q, int32_t q_dtype,
  * (cudaGetSymbolAddress) with that device current; make it before any stream
  * capture.  No call allocates or frees memory.  All calls on a device share
  * the array: calls that may overlap on the GPU race on it, so serialise them.
- * Nothing in the array must start at zero; its first KCA_WORKSPACE_HEADER
- * bytes hold the device status word described above.
+ * The array keeps the last call's contents.  Its first KCA_WORKSPACE_HEADER
+ * bytes (the device status word and the merge counters described above) must
+ * be zero when a call starts, so each call that passes validation first
+ * clears them with cudaMemsetAsync on `stream` (a memset, no allocation);
+ * the device status of a call is therefore not kept for a later call to
+ * read.
  */
 #define KCA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 int attn_decode_static(const void *q, int32_t q_dtype,

@@ -566,6 +566,18 @@ int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void*
                 int32_t kv_dtype, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                 int64_t capacity, int32_t batch, const int64_t* ctx_len, int32_t window, float scale,
                 float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  return kca::decode_entry(q, q_dtype, k_cache, v_cache, kv_dtype, n_q_heads, n_kv_heads, head_dim, capacity,
+                           batch, ctx_len, window, scale, out, workspace, workspace_bytes, stream, false);
+}
+
+}  // extern "C"
+
+namespace kca {
+
+int decode_entry(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache, int32_t kv_dtype,
+                 int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity, int32_t batch,
+                 const int64_t* ctx_len, int32_t window, float scale, float* out, void* workspace,
+                 size_t workspace_bytes, void* stream, bool clear_header) {
   if (!q || !k_cache || !v_cache || !out || !workspace || !ctx_len) return KCA_ERR_NULL;
   int st = geometry_status(n_q_heads, n_kv_heads, head_dim);
   if (st != KCA_OK) return st;
@@ -599,9 +611,17 @@ int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void*
   a.window = window;
   a.scale = scale;
   for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
+  // Every argument is valid: only now may the header be cleared.
+  if (clear_header &&
+      cudaMemsetAsync(workspace, 0, KCA_WORKSPACE_HEADER, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KCA_ERR_CUDA;
   return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster,
                           workspace, static_cast<cudaStream_t>(stream));
 }
+
+}  // namespace kca
+
+extern "C" {
 
 int attn_decode_dev(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache,
                     int32_t kv_dtype, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,

@@ -15,13 +15,19 @@
 // call made with that device current; make that first call before any stream
 // capture.  All calls on a device share the array, so calls whose execution
 // can overlap on the GPU (different streams, or graphs replayed
-// concurrently) race on it and must be serialised by the caller.  Nothing in
-// the array needs to start at zero: every partial is written before it is
-// read within the same call, and the status word at its head (see
-// attn_device_status) only records errors.
+// concurrently) race on it and must be serialised by the caller.  The array
+// keeps the last call's contents.  Its first KCA_WORKSPACE_HEADER bytes must
+// be zero when a call starts: the status word, and the counters by which the
+// tensor-core decode kernel elects the CTA that merges a row (a call leaves
+// them at zero, but one that recorded a device error may not), so every call
+// clears them first with cudaMemsetAsync on its stream -- a memset, not an
+// allocation.  Everything past the header is written before it is read
+// within the same call.
 #include <cuda_runtime.h>
 
 #include "../../include/kca.h"
+#include "kca_plan.h"
+#include "kca_rows.h"
 
 namespace {
 
@@ -58,9 +64,9 @@ extern "C" int attn_decode_static(const void* q, int32_t q_dtype, const void* k_
   int st = KCA_OK;
   void* ws = scratch_address(&st);
   if (ws == nullptr) return st;
-  // attn_decode validates every argument and returns KCA_ERR_WORKSPACE when
-  // the plan's partials would not fit the array.
-  return attn_decode(q, q_dtype, k_cache, v_cache, kv_dtype, n_q_heads, n_kv_heads, head_dim,
-                     capacity, batch, ctx_len, window, scale, out, ws, KCA_STATIC_SCRATCH_BYTES,
-                     stream);
+  // attn_decode's checks (KCA_ERR_WORKSPACE when the plan's partials would
+  // not fit the array); once they pass, the header is cleared, then the
+  // kernel is launched.  A call that fails validation touches nothing.
+  return kca::decode_entry(q, q_dtype, k_cache, v_cache, kv_dtype, n_q_heads, n_kv_heads, head_dim, capacity,
+                           batch, ctx_len, window, scale, out, ws, KCA_STATIC_SCRATCH_BYTES, stream, true);
 }

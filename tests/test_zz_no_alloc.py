@@ -6,9 +6,9 @@ allocations, a runtime that only hands out the tensors it owns), so they
 cannot provide the workspace that attn_decode writes its per-split partials
 to.  attn_decode_static takes that scratch from a fixed device array inside
 the library instead.  These tests call it through the C ABI (ctypes, raw
-pointers) and check it against attn_decode on the same inputs, twice in a
-row with different shapes so that the array's leftover contents from the
-first call cannot leak into the second.  This file is collected last, and
+pointers) and check it against attn_decode on the same inputs, three times
+in a row with different shapes so that the array's leftover contents from
+one call cannot leak into the next.  This file is collected last, and
 it also passes on its own in a fresh process.
 """
 import ctypes
@@ -45,6 +45,7 @@ def test_static_scratch_decode_matches_attn_decode_twice(cuda_ok):
     cases = [
         (1, 16448, [16384], 0, "f32", "f16"),               # one long sequence: 100+ splits
         (4, 9000, [8999, 1, 4500, 7777], 300, "bf16", "bf16"),  # ragged batch with a window
+        (1, 16448, [16384], 0, "f32", "f16"),               # the first case again, after the second
     ]
     for i, (batch, cap, ctx, window, qd, kd) in enumerate(cases):
         q, k, v = _inputs(10 + i, batch, cap, qd, kd)
