@@ -469,15 +469,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rings are free once every PV is done), then out by TMA stores: the
     // tile's 128 rows are one contiguous block of out or of the partials,
     // and rows past the chunk fall outside the map and are not written.
+    // Boxes c and 4 + c (the two warpgroups' halves) leave as soon as both
+    // are written, while the next ones are; the issuing thread then waits
+    // only until shared memory has been read -- the grid's completion makes
+    // the stores visible to the kernels after it.  A ragged tile's partial
+    // keeps only its valid rows: the first rows of every box (the swizzle
+    // pattern repeats every 8 rows).
+    const void* omap = slot < 0             ? static_cast<const void*>(&tmo)
+                       : tile == a.rag_tile ? static_cast<const void*>(&tmpart_rag)
+                                            : static_cast<const void*>(&tmpart);
+    const int32_t oy = (slot < 0 ? tile : slot) * 128;
     if (ok) {
       ptx::fence_after_sync();
       if (slot >= 0 && wg == 0 && valid) {
         a.part_ml[((int64_t)slot * 128 + m) * 2 + 0] = m_ref;
         a.part_ml[((int64_t)slot * 128 + m) * 2 + 1] = l_tot;
       }
-      const float f = slot < 0 ? 1.f / l_tot : 1.f;
+    }
+    const float f = slot < 0 ? 1.f / l_tot : 1.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 4; ++c) {
+      if (ok) {
         uint32_t r[32];
         ptx::tmem_ld32(trow + kColO + 128 * wg + 32 * c, r);
         ptx::tmem_wait_ld();
@@ -487,23 +499,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<float4*>(box + ((i ^ (m & 7)) << 4)) =
               make_float4(__uint_as_float(r[4 * i]) * f, __uint_as_float(r[4 * i + 1]) * f,
                           __uint_as_float(r[4 * i + 2]) * f, __uint_as_float(r[4 * i + 3]) * f);
+        fence_proxy_async_smem();   // generic-proxy stores -> visible to the TMA unit
       }
-      fence_proxy_async_smem();   // generic-proxy stores -> visible to the TMA unit
+      ptx::fence_before_sync();
+      named_sync(1, kSoftmaxThreads);
+      if (ok && !ghost && threadIdx.x == 4 * 32) {
+        ptx::tma_store_2d(omap, 32 * c, oy, sbase + c * kOBoxBytes);
+        ptx::tma_store_2d(omap, 32 * (4 + c), oy, sbase + (4 + c) * kOBoxBytes);
+        ptx::bulk_commit();
+      }
     }
-    ptx::fence_before_sync();
-    named_sync(1, kSoftmaxThreads);
-    if (ok && !ghost && threadIdx.x == 4 * 32) {
-      // A ragged tile's partial keeps only its valid rows: the first rows of
-      // every box (the swizzle pattern repeats every 8 rows).
-      const void* map = slot < 0             ? static_cast<const void*>(&tmo)
-                        : tile == a.rag_tile ? static_cast<const void*>(&tmpart_rag)
-                                             : static_cast<const void*>(&tmpart);
-      const int32_t y = (slot < 0 ? tile : slot) * 128;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) ptx::tma_store_2d(map, 32 * j, y, sbase + j * kOBoxBytes);
-      ptx::bulk_commit();
-      ptx::bulk_wait_all();   // shared memory stays allocated until the stores are done
-    }
+    // shared memory stays allocated until the stores have read it
+    if (ok && !ghost && threadIdx.x == 4 * 32) ptx::bulk_wait_read_all();
   }
 
   // No CTA of the pair leaves while MMAs may still read its shared memory
