@@ -186,6 +186,15 @@ KCA_HD int32_t tc_pair_items(const TcPlan& p, int32_t q) {
   return (int32_t)cdiv(ke - kb, p.per_item);
 }
 
+// Start of split k of a pair's n key tiles cut into s items: ceil(k n / s),
+// so the items differ by at most one tile and any longer ones come first.
+// The last item holds the causal diagonal (its last tile is partly masked
+// and its K / V rows were not read by the previous chunk), so a spare tile
+// is better placed on an earlier one.
+KCA_HD int32_t tc_split_at(int32_t n, int32_t s, int32_t k) {
+  return (int32_t)(((int64_t)k * n + s - 1) / s);
+}
+
 struct TcItem {
   int32_t pair;
   int32_t kt_begin;   // key tiles, relative to kv_lo
@@ -209,8 +218,8 @@ KCA_HD TcItem tc_item(const TcPlan& p, int32_t idx) {
     if (idx < base + s) {
       const int32_t k = idx - base;
       it.pair = q;
-      it.kt_begin = kb + (int32_t)(((int64_t)k * n) / s);
-      it.kt_end = kb + (int32_t)(((int64_t)(k + 1) * n) / s);
+      it.kt_begin = kb + tc_split_at(n, s, k);
+      it.kt_end = kb + tc_split_at(n, s, k + 1);
       it.split = k;
       it.n_split = s;
       it.slot0 = s > 1 ? slot_base + k : -1;

@@ -675,8 +675,8 @@ void fill_tc_tables(TcArgs& a) {
       a.tile_first_slot[2 * q + r] = (int16_t)(slot + r * s);
     }
     for (int32_t k = 0; k < s && idx < kTcMaxItems; ++k, ++idx) {
-      a.items[idx].kt_begin = kb + (int32_t)(((int64_t)k * n) / s);
-      a.items[idx].kt_end = kb + (int32_t)(((int64_t)(k + 1) * n) / s);
+      a.items[idx].kt_begin = kb + tc_split_at(n, s, k);
+      a.items[idx].kt_end = kb + tc_split_at(n, s, k + 1);
       a.items[idx].pair = (int16_t)q;
       a.items[idx].slot[0] = (int16_t)(s > 1 ? slot + k : -1);
       a.items[idx].slot[1] = (int16_t)(s > 1 && nt == 2 ? slot + s + k : -1);
