@@ -47,7 +47,10 @@
  * keys (one pass over the keys beats one pass per row there), else the rows
  * path, which also serves every other prefill combination: one unit per
  * query row, mma.sync with split-precision operands for 16-bit caches,
- * CUDA-core f32 for f32 caches.
+ * CUDA-core f32 for f32 caches.  Two environment variables, read at each
+ * call, force a path so that tests can compare them on the same inputs:
+ * KCA_PREFILL_PATH=rows (or =tc, where eligible) for prefill, and
+ * KCA_DECODE_PATH=simt for the CUDA-core decode kernel on 16-bit caches.
  *
  * OWNERSHIP: every buffer is allocated and owned by the caller.  The library
  * allocates no device memory, keeps no per-call state and never synchronises

@@ -246,10 +246,7 @@ kca::RowsPlan mma_rows_plan(int32_t n_units, const int64_t* nkeys, int sms, int*
   double best_t = 0.0;
   double total_keys = 0.0;
   for (int32_t u = 0; u < n_units; ++u) total_keys += (double)nkeys[u];
-  int cmax = 8;   // KCA_DECODE_CLUSTER_MAX caps the cluster size (sweeps compare them)
-  if (const char* env = std::getenv("KCA_DECODE_CLUSTER_MAX")) cmax = std::atoi(env);
   for (int c = 8; c >= 1; c /= 2) {
-    if (c > cmax && c > 1) continue;
     int slots = c == 1 ? sms : kca::decode_mma_cluster_capacity(c);
     if (slots > kca::kRowsMmaMaxClusterParts) slots = kca::kRowsMmaMaxClusterParts;
     if (slots <= 0) continue;
