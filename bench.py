@@ -267,21 +267,29 @@ def run_cuda(args, rank, world, local_rank):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    # NVTX ranges name the phases on a profiler timeline (no cost otherwise).
+    nvtx = torch.cuda.nvtx
+    nvtx.range_push("timed steps")
     start.record(stream)
     for s in range(args.steps):
         ev[s][0].record(stream)
+        nvtx.range_push("prefill")
         if graphs is None:
             w.prefill()
         else:
             graphs["pre"][w.step_index % PREFILL_REPLICAS].replay()
+        nvtx.range_pop()
         ev[s][1].record(stream)
+        nvtx.range_push("decode")
         if graphs is None:
             w.decode()
         else:
             graphs["dec"].replay()
+        nvtx.range_pop()
         ev[s][2].record(stream)
         w.step_index += 1
     end.record(stream)
+    nvtx.range_pop()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -389,8 +397,10 @@ def run_e2e(w, args, stream):
 
     step(False)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("e2e steps")
     evs = [step(True) for _ in range(steps)]
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
     return dict(steps=steps, pre_ms=pre_ms, dec_ms=dec_ms, h2d=h2d, d2h=d2h, pre_h2d=pre_h2d,
@@ -430,11 +440,13 @@ def run_ragged(device, stream):
     reps = 5
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("ragged decode")
     e0.record(stream)
     for _ in range(reps):
         graph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     st, detail = kca.attn_device_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {st} detail {detail:#x}")
