@@ -301,24 +301,34 @@ int attn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 int attn_device_status(void *workspace, void *stream, uint32_t *detail);
 
 /*
- * Integer plans, for bit-exact tests; host only, no GPU needed.
- * Each work item is 4 int64: (unit, key_begin, key_end, slot):
+ * Integer plans -- the work items a call with the same arguments runs -- for
+ * bit-exact tests.  Each work item is 4 int64: (unit, key_begin, key_end, slot):
  *   prefill, tensor-core path: unit = 16-row tile index, [key_begin, key_end)
- *     the absolute key positions the item covers (64-key tiles clipped to the
- *     call's visible union), slot = partial slot or -1 when the tile is not split;
- *   rows path (decode, and prefill on the CUDA cores): unit = query row
- *     (prefill) or sequence (decode), [key_begin, key_end) within J(pos),
- *     slot = partial slot or -1.
- * num_sms is the SM count the plan is made for (the calls use the device's).
- * *path receives 0 for the rows path, 1 for the tensor-core path.
+ *     the absolute key positions the item covers (128-key tiles clipped to the
+ *     call's visible union), slot = partial slot or -1 when the tile is not
+ *     split;
+ *   rows path (decode, and prefill of short or mixed-dtype chunks): one item
+ *     per split, unit = query row (prefill) or sequence (decode),
+ *     [key_begin, key_end) within J(pos).  With an f32 cache (or
+ *     KCA_DECODE_PATH=simt) this is the CUDA-core kernel's plan for num_sms
+ *     SMs, host only, and slot = the split's partial slot or -1 when the unit
+ *     has one split.  With a 16-bit cache it is the tensor-core kernel's
+ *     plan, whose splits run as clusters that must fit the resident-cluster
+ *     capacity of the CURRENT DEVICE (num_sms is not used; KCA_ERR_CUDA
+ *     without a device), and slot = the cluster partial that the split's
+ *     cluster writes (sequence * clusters-per-sequence + split / cluster
+ *     size), or -1 when the unit is one cluster and merges in shared memory.
+ * *path receives 0 for the rows path, 1 for the tensor-core path; it is set
+ * once the arguments are valid, before any device query, so it also answers
+ * a call that then fails for want of a device.
  * Returns KCA_OK, or KCA_ERR_RANGE when more than max_items items exist
  * (*n_items still receives the count).
  */
 int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
                       int32_t chunk_rows, int32_t window, int32_t num_sms,
                       int64_t *items, int32_t max_items, int32_t *n_items, int32_t *path);
-int attn_decode_plan(int32_t batch, const int64_t *ctx_len, int32_t window, int32_t num_sms,
-                     int64_t *items, int32_t max_items, int32_t *n_items);
+int attn_decode_plan(int32_t batch, const int64_t *ctx_len, int32_t window, int32_t kv_dtype,
+                     int32_t num_sms, int64_t *items, int32_t max_items, int32_t *n_items);
 
 /* Static description of a status code. */
 const char *attn_status_string(int status);

@@ -80,7 +80,7 @@ def lib() -> ctypes.CDLL:
         L.attn_device_status.restype = ctypes.c_int
         L.attn_prefill_plan.argtypes = [i32, i32, i64, i32, i32, i32, p64, i32, p32, p32]
         L.attn_prefill_plan.restype = ctypes.c_int
-        L.attn_decode_plan.argtypes = [i32, p64, i32, i32, p64, i32, p32]
+        L.attn_decode_plan.argtypes = [i32, p64, i32, i32, i32, p64, i32, p32]
         L.attn_decode_plan.restype = ctypes.c_int
         L.attn_status_string.argtypes = [ctypes.c_int]
         L.attn_status_string.restype = ctypes.c_char_p
@@ -405,9 +405,23 @@ def attn_decode_static(q, k_cache, v_cache, ctx_len, window: int = 0, scale: flo
 
 # --------------------------------------------------------------------- plans
 
+def attn_prefill_path(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows: int,
+                      window: int = 0) -> int:
+    """The path a prefill call takes: 1 tensor-core, 0 rows (host only; no device needed)."""
+    n = ctypes.c_int32(0)
+    path = ctypes.c_int32(-1)
+    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, 148, None, 0,
+                                 ctypes.byref(n), ctypes.byref(path))
+    if path.value < 0:
+        raise KcaError(st, "attn_prefill_plan")
+    return int(path.value)
+
+
 def attn_prefill_plan(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows: int,
                       window: int = 0, num_sms: int = 148):
-    """(path, items[n, 4]) -- see include/kca.h; host only."""
+    """(path, items[n, 4]) -- see include/kca.h.  Host only, except the rows
+    plan of 16-bit caches, which is the tensor-core kernel's cluster plan on
+    the current device."""
     n = ctypes.c_int32(0)
     path = ctypes.c_int32(0)
     st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, num_sms, None,
@@ -422,14 +436,17 @@ def attn_prefill_plan(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows:
     return int(path.value), items[:n.value]
 
 
-def attn_decode_plan(ctx_len, window: int = 0, num_sms: int = 148):
+def attn_decode_plan(ctx_len, window: int = 0, num_sms: int = 148, kv_dtype: int = F32):
+    """items[n, 4] of a decode call -- see include/kca.h.  kv_dtype F32: the
+    CUDA-core kernel's plan for num_sms SMs (host only); F16 / BF16: the
+    tensor-core kernel's cluster plan on the current device."""
     nctx, ptr = _i64_array(ctx_len)
     n = ctypes.c_int32(0)
-    st = lib().attn_decode_plan(nctx, ptr, window, num_sms, None, 0, ctypes.byref(n))
+    st = lib().attn_decode_plan(nctx, ptr, window, kv_dtype, num_sms, None, 0, ctypes.byref(n))
     if st not in (0, -4) or (st == -4 and n.value == 0):
         raise KcaError(st, "attn_decode_plan")
     items = np.zeros((max(n.value, 1), 4), dtype=np.int64)
-    st = lib().attn_decode_plan(nctx, ptr, window, num_sms,
+    st = lib().attn_decode_plan(nctx, ptr, window, kv_dtype, num_sms,
                                 items.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n.value,
                                 ctypes.byref(n))
     _check(st, "attn_decode_plan")

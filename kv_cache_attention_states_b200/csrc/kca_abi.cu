@@ -328,6 +328,47 @@ int launch_rows_path(int32_t q_dtype, int32_t kv_dtype, const void* k_cache, con
   return kca::launch_rows(q_dtype, kv_dtype, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
 }
 
+// Work items of the rows path (unit u at position pos[u], nk[u] visible keys
+// from lo(pos[u])), as the calls run them: the CUDA-core kernel's plan for
+// num_sms SMs, or -- for 16-bit caches, unless KCA_DECODE_PATH forces the
+// CUDA-core kernel -- the tensor-core kernel's cluster plan on the current
+// device (its clusters must fit the device's resident capacity, so that form
+// needs a device).  slot: the split's partial slot (CUDA core), or the
+// cluster partial its cluster writes (tensor cores), -1 when nothing of the
+// unit goes through global memory.
+int rows_plan_items(int32_t kv_dtype, int32_t n, const int64_t* pos, const int64_t* nk, int32_t window,
+                    int32_t num_sms, int64_t* items, int32_t max_items, int32_t* count) {
+  const bool mma = use_rows_mma(kv_dtype);
+  kca::RowsPlan p;
+  int cluster = 1;
+  if (mma) {
+    int sms = 0;
+    if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+    p = mma_rows_plan(n, nk, sms, &cluster);
+    if (cluster < 1) return KCA_ERR_CUDA;
+  } else {
+    p = kca::make_rows_plan(n, nk, num_sms);
+  }
+  const int32_t max_clusters = (p.max_splits + cluster - 1) / cluster;
+  for (int32_t u = 0; u < n; ++u) {
+    const int64_t lo = kca::lo_of(pos[u], window);
+    const int32_t ns = kca::rows_n_splits(nk[u], p.split_len);
+    const int32_t nclus = (ns + cluster - 1) / cluster;
+    for (int32_t sp = 0; sp < ns; ++sp, ++*count) {
+      if (*count >= max_items) continue;
+      int64_t kb = lo + (int64_t)sp * p.split_len, ke = kb + p.split_len;
+      if (ke > pos[u] + 1) ke = pos[u] + 1;
+      if (nk[u] == 0) kb = ke = lo;
+      items[4 * *count + 0] = u;
+      items[4 * *count + 1] = kb;
+      items[4 * *count + 2] = ke;
+      items[4 * *count + 3] = mma ? (nclus > 1 ? (int64_t)u * max_clusters + sp / cluster : -1)
+                                  : (ns > 1 ? (int64_t)u * p.max_splits + sp : -1);
+    }
+  }
+  return KCA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -375,51 +416,29 @@ int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, in
   } else {
     *path = 0;
     const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
-    const kca::RowsPlan p = kca::make_rows_plan(chunk_rows, nk.data(), num_sms);
-    for (int32_t u = 0; u < chunk_rows; ++u) {
-      const int64_t pos = chunk_start + u;
-      const int64_t lo = kca::lo_of(pos, window);
-      const int32_t ns = kca::rows_n_splits(nk[u], p.split_len);
-      for (int32_t s = 0; s < ns; ++s, ++count) {
-        if (count >= max_items) continue;
-        int64_t kb = lo + (int64_t)s * p.split_len, ke = kb + p.split_len;
-        if (ke > pos + 1) ke = pos + 1;
-        if (nk[u] == 0) kb = ke = lo;
-        items[4 * count + 0] = u;
-        items[4 * count + 1] = kb;
-        items[4 * count + 2] = ke;
-        items[4 * count + 3] = ns > 1 ? (int64_t)u * p.max_splits + s : -1;
-      }
-    }
+    std::vector<int64_t> pos(chunk_rows);
+    for (int32_t u = 0; u < chunk_rows; ++u) pos[u] = chunk_start + u;
+    const int st = rows_plan_items(kv_dtype, chunk_rows, pos.data(), nk.data(), window, num_sms, items,
+                                   max_items, &count);
+    if (st != KCA_OK) return st;
   }
   *n_items = count;
   return count <= max_items ? KCA_OK : KCA_ERR_RANGE;
 }
 
-int attn_decode_plan(int32_t batch, const int64_t* ctx_len, int32_t window, int32_t num_sms,
+int attn_decode_plan(int32_t batch, const int64_t* ctx_len, int32_t window, int32_t kv_dtype, int32_t num_sms,
                      int64_t* items, int32_t max_items, int32_t* n_items) {
   if (ctx_len == nullptr || n_items == nullptr || (items == nullptr && max_items > 0)) return KCA_ERR_NULL;
+  if (!dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
   if (batch < 1 || batch > KCA_MAX_BATCH || num_sms < 1) return KCA_ERR_RANGE;
   for (int32_t b = 0; b < batch; ++b)
     if (ctx_len[b] < 0 || ctx_len[b] > KCA_MAX_POSITION) return KCA_ERR_RANGE;
   const std::vector<int64_t> nk = decode_unit_keys(batch, ctx_len, window);
-  const kca::RowsPlan p = kca::make_rows_plan(batch, nk.data(), num_sms);
+  std::vector<int64_t> pos(batch);
+  for (int32_t b = 0; b < batch; ++b) pos[b] = ctx_len[b] - 1;
   int32_t count = 0;
-  for (int32_t b = 0; b < batch; ++b) {
-    const int64_t pos = ctx_len[b] - 1;
-    const int64_t lo = kca::lo_of(pos, window);
-    const int32_t ns = kca::rows_n_splits(nk[b], p.split_len);
-    for (int32_t s = 0; s < ns; ++s, ++count) {
-      if (count >= max_items) continue;
-      int64_t kb = lo + (int64_t)s * p.split_len, ke = kb + p.split_len;
-      if (ke > pos + 1) ke = pos + 1;
-      if (nk[b] == 0) kb = ke = lo;
-      items[4 * count + 0] = b;
-      items[4 * count + 1] = kb;
-      items[4 * count + 2] = ke;
-      items[4 * count + 3] = ns > 1 ? (int64_t)b * p.max_splits + s : -1;
-    }
-  }
+  const int st = rows_plan_items(kv_dtype, batch, pos.data(), nk.data(), window, num_sms, items, max_items, &count);
+  if (st != KCA_OK) return st;
   *n_items = count;
   return count <= max_items ? KCA_OK : KCA_ERR_RANGE;
 }

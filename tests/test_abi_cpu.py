@@ -258,18 +258,18 @@ def test_prefill_tc_plan_covers_every_visible_key(cs, rows, window):
 
 
 def test_small_chunks_and_f32_take_the_rows_path():
-    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 100, 15)[0] == 0
-    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 100, 16)[0] == 1
-    assert kca.attn_prefill_plan(kca.F32, kca.F32, 100, 768)[0] == 0
-    assert kca.attn_prefill_plan(kca.F16, kca.BF16, 100, 768)[0] == 0
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 100, 15) == 0
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 100, 16) == 1
+    assert kca.attn_prefill_path(kca.F32, kca.F32, 100, 768) == 0
+    assert kca.attn_prefill_path(kca.F16, kca.BF16, 100, 768) == 0
 
 
 def test_few_row_chunks_on_long_contexts_take_the_tensor_core_path():
     # 3-15 rows whose first row sees >= 12,288 keys: one pass over the keys
-    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 16381, 3)[0] == 1
-    assert kca.attn_prefill_plan(kca.F16, kca.F16, 12287, 15)[0] == 1
-    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 12287, 3)[0] == 1
-    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 12286, 3)[0] == 0
-    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 16382, 2)[0] == 0
-    assert kca.attn_prefill_plan(kca.BF16, kca.BF16, 16381, 3, 4096)[0] == 0   # window: 4096 keys
-    assert kca.attn_prefill_plan(kca.F32, kca.F32, 16381, 3)[0] == 0
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 16381, 3) == 1
+    assert kca.attn_prefill_path(kca.F16, kca.F16, 12287, 15) == 1
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 12287, 3) == 1
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 12286, 3) == 0
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 16382, 2) == 0
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 16381, 3, 4096) == 0   # window: 4096 keys
+    assert kca.attn_prefill_path(kca.F32, kca.F32, 16381, 3) == 0
