@@ -138,7 +138,11 @@ int attn_prefill(const void *q_chunk, int32_t q_dtype,
  *   batch        1..256
  *   ctx_len      HOST array [batch], 0..capacity; the query sits at ctx_len[b]-1
  *                and ctx_len[b] == 0 yields an all-zero output row
+ *   window, scale  as in attn_prefill
  *   out          [batch][8][256] float32, device
+ *   workspace    >= attn_decode_workspace_bytes(batch, ctx_len, window) bytes, device
+ *   stream       cudaStream_t the kernels are enqueued on
+ * Returns KCA_OK or a negative KCA_ERR_* (nothing launched on error).
  */
 int attn_decode(const void *q, int32_t q_dtype,
                 const void *k_cache, const void *v_cache, int32_t kv_dtype,
