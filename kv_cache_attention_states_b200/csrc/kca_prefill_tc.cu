@@ -83,7 +83,8 @@ constexpr uint16_t kPairMask = 3;    // both CTAs of the cluster
 // barriers it waits on (kfull, vfull, q_full, s_free, p_full) live in its
 // shared memory and collect arrivals / bytes from both CTAs; the ones the
 // MMAs signal (kempty, vempty, s_full, o_done, o_final, drain) are
-// multicast to the same offset in both CTAs.
+// multicast to the same offset in both CTAs (as is s_first, which the V
+// producers wait on).
 struct Bars {
   uint64_t kfull[kKRing], kempty[kKRing];
   uint64_t vfull[kVRing], vempty[kVRing];
@@ -94,6 +95,7 @@ struct Bars {
   uint64_t o_done[2];  // PV of tile u complete (MMA commit), u&1 selects the barrier
   uint64_t o_final;    // every PV complete (single use)
   uint64_t drain;      // every MMA complete (single use)
+  uint64_t s_first;    // the first tile's QK^T complete (single use; MMA commit to both CTAs)
   uint32_t tmem_base;
   int abort;
   float red_max[2][2][128];  // [tile parity][warpgroup][row]: partial row maxima
@@ -217,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->o_final, 1);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->s_first, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -257,7 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::prefetch_tmap(&tmpart);
         ptx::prefetch_tmap(&tmpart_rag);
       }
-      bool ok = true;
+      // V is first needed by the first PV, after the first softmax: its
+      // loads wait until the first QK^T is done, so that Q and the first K
+      // tiles have the SM's load bandwidth to themselves when an item
+      // starts.  s_first has a single phase, so the wait cannot alias a
+      // later one.
+      bool ok = is_k || mbar_wait(&bars->s_first, 0, abort_flag, status, kSiteTcS);
       for (int t = 0; t < n && ok; ++t) {
         const int s = t % 2;
         if (t >= 2 && !mbar_wait(&empty[s], ((t / 2) - 1) & 1, abort_flag, status, kSiteTcEmpty)) {
@@ -332,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            kd + (uint64_t)(((k >> 2) * kKChunkBytes + (k & 3) * 32) >> 4), id_qk, k > 0 ? 1u : 0u);
         ptx::mma_commit_pair(smem_u32(&bars->kempty[s]), kPairMask);
         ptx::mma_commit_pair(s_full, kPairMask);
+        if (t == 0) ptx::mma_commit_pair(smem_u32(&bars->s_first), kPairMask);
         if (t > 0) ok = pv(t - 1);
       }
       if (ok) ok = pv(n - 1);
