@@ -36,7 +36,7 @@ DECODE_REPLICAS = 32
 PREFILL_REPLICAS = 2
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels; reset to None whenever a kernel changes after its capture.
-PREFILL_TRAFFIC = 18.931e6 + 3.6e3
+PREFILL_TRAFFIC = 18.931e6 + 25.6e3
 DECODE_TRAFFIC = 16.919e6
 E2E_GROUP = 4            # prefill chunks per host copy in the end-to-end leg
 METRIC = "prefill q-rows/s & decode tok/s at 16K ctx (1 B200); % of TC/HBM roofline"
