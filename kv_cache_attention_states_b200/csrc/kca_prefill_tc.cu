@@ -20,7 +20,8 @@
 //               K tile (64 keys x 256 dims as four 64 x 64 boxes)
 //   warp 1      TMEM allocator (both CTAs); in the even CTA the single thread
 //               that issues every MMA of the pair
-//   warp 2      TMA producer of its half of every V tile (128 keys x 128 dims)
+//   warp 2      TMA producer of its half of every V tile (128 keys x 128 dims),
+//               from the moment the item's first QK^T is done
 //   warps 4-7   softmax warpgroup 0: keys 0-63 of every S tile
 //   warps 8-11  softmax warpgroup 1: keys 64-127
 //   Thread m of a softmax warpgroup owns TMEM lane m, i.e. M row m of its CTA.
@@ -38,8 +39,11 @@
 // The softmax keeps a reference max per row and rescales O (in TMEM) only
 // when a score exceeds it by more than 2^8, so probabilities stay <= 256 and
 // the O round trip is rare; the result is exact up to rounding whatever
-// reference is used.  Work items of a split row tile write (m, l, O)
-// partials that merge_tc_kernel (below) combines by log-sum-exp.
+// reference is used.  It takes each tile's probabilities with the current
+// reference first and needs the row max (and its exchange between the two
+// warpgroups) only when a half row's sum passes 2^8.  Work items of a split
+// row tile write (m, l, O) partials that merge_tc_kernel (below) combines by
+// log-sum-exp.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
