@@ -590,11 +590,10 @@ int attn_decode(const void* q, int32_t q_dtype, const void* k_cache, const void*
 
 namespace kca {
 
-int decode_entry(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache, int32_t kv_dtype,
-                 int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity, int32_t batch,
-                 const int64_t* ctx_len, int32_t window, float scale, float* out, void* workspace,
-                 size_t workspace_bytes, void* stream, bool clear_header) {
-  if (!q || !k_cache || !v_cache || !out || !workspace || !ctx_len) return KCA_ERR_NULL;
+int decode_args_check(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache, int32_t kv_dtype,
+                      int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity, int32_t batch,
+                      const int64_t* ctx_len, float scale, const float* out) {
+  if (!q || !k_cache || !v_cache || !out || !ctx_len) return KCA_ERR_NULL;
   int st = geometry_status(n_q_heads, n_kv_heads, head_dim);
   if (st != KCA_OK) return st;
   if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
@@ -603,6 +602,17 @@ int decode_entry(const void* q, int32_t q_dtype, const void* k_cache, const void
   if (!std::isfinite(scale) || !(scale > 0.f)) return KCA_ERR_RANGE;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return KCA_ERR_ALIGN;
+  return KCA_OK;
+}
+
+int decode_entry(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache, int32_t kv_dtype,
+                 int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity, int32_t batch,
+                 const int64_t* ctx_len, int32_t window, float scale, float* out, void* workspace,
+                 size_t workspace_bytes, void* stream, bool clear_header) {
+  if (!workspace) return KCA_ERR_NULL;
+  int st = decode_args_check(q, q_dtype, k_cache, v_cache, kv_dtype, n_q_heads, n_kv_heads, head_dim, capacity,
+                             batch, ctx_len, scale, out);
+  if (st != KCA_OK) return st;
   if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;

@@ -102,6 +102,12 @@ cudaError_t launch_merge_rows(const RowsArgs& a, cudaStream_t stream);
 cudaError_t launch_merge_partials(int n_parts, int batch, const float* parts, int64_t part_stride, float* out,
                                   cudaStream_t stream);
 
+// attn_decode's host checks that need no device and no workspace: pointers,
+// geometry, dtypes, ranges, scale, alignment (KCA_OK or the KCA_ERR_* code).
+int decode_args_check(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache, int32_t kv_dtype,
+                      int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity, int32_t batch,
+                      const int64_t* ctx_len, float scale, const float* out);
+
 // attn_decode's body: validates every argument, plans, and launches.  With
 // clear_header the workspace's first KCA_WORKSPACE_HEADER bytes are zeroed on
 // `stream` (after validation, before the launch); attn_decode passes false.

@@ -61,7 +61,11 @@ extern "C" int attn_decode_static(const void* q, int32_t q_dtype, const void* k_
                                   int32_t n_kv_heads, int32_t head_dim, int64_t capacity,
                                   int32_t batch, const int64_t* ctx_len, int32_t window,
                                   float scale, float* out, void* stream) {
-  int st = KCA_OK;
+  // The checks that need no device come first, so that a bad argument is
+  // reported as such before the array's address is looked up.
+  int st = kca::decode_args_check(q, q_dtype, k_cache, v_cache, kv_dtype, n_q_heads, n_kv_heads, head_dim,
+                                  capacity, batch, ctx_len, scale, out);
+  if (st != KCA_OK) return st;
   void* ws = scratch_address(&st);
   if (ws == nullptr) return st;
   // attn_decode's checks (KCA_ERR_WORKSPACE when the plan's partials would

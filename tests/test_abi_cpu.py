@@ -98,6 +98,30 @@ def test_decode_rejects_bad_arguments_on_the_host(ctx, kw, code):
     assert _decode(ctx, **kw) == code
 
 
+def _decode_static(ctx=(100, 200), **kw):
+    a = dict(q=P, qd=kca.F32, k=P, v=P, kd=kca.F16, hq=8, hkv=1, d=256, cap=4096, window=0,
+             scale=0.0625, out=P, batch=None)
+    a.update(kw)
+    arr = np.asarray(ctx, dtype=np.int64)
+    batch = len(arr) if a["batch"] is None else a["batch"]
+    vp = ctypes.c_void_p
+    return kca.lib().attn_decode_static(vp(a["q"]), a["qd"], vp(a["k"]), vp(a["v"]), a["kd"], a["hq"],
+                                        a["hkv"], a["d"], a["cap"], batch,
+                                        arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), a["window"],
+                                        a["scale"], vp(a["out"]), None)
+
+
+@pytest.mark.parametrize("ctx,kw,code", [
+    ((1, 2), dict(q=0), -1), ((1, 2), dict(out=0), -1), ((1, 2), dict(hq=4), -2), ((1, 2), dict(kd=3), -3),
+    ((1, 2), dict(batch=0), -4), ((1,) * 257, dict(), -4), ((1, 4097), dict(), -4),
+    ((1, 2), dict(scale=0.0), -4), ((1, 2), dict(out=P + 4), -6),
+])
+def test_decode_static_rejects_bad_arguments_before_any_device_call(ctx, kw, code):
+    # the checks run before the scratch array's address is looked up, so
+    # they answer even on a machine without a GPU
+    assert _decode_static(ctx, **kw) == code
+
+
 def _decode_dev(**kw):
     a = dict(q=P, qd=kca.F32, k=P, v=P, kd=kca.F16, hq=8, hkv=1, d=256, cap=4096, batch=2, ctx=P * 3,
              bound=4096, window=0, scale=0.0625, out=P, ws=P * 2, wsb=1 << 30)
