@@ -122,8 +122,9 @@ class Clocks:
             self._start_smi(device)
 
     def _start_smi(self, device):
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="kca_clocks_", suffix=".csv")
+        os.close(fd)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -157,6 +158,7 @@ class Clocks:
                     if val.lower() == "active":
                         self.reasons.add(n)
             self.sm_max = max(smax) if smax else None
+            os.remove(self.path)
         else:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
         sm = self.samples
