@@ -2,7 +2,7 @@
  * attn_oracle.c -- f64 CPU oracle for states-form KV-cache attention.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or
- * calls this file; only the tests, the graft smoke check and the CPU
+ * calls this file; only the tests, __graft_entry__.smoke() and the CPU
  * baseline leg of bench.py do.  It shares no code, header or constant with
  * the CUDA library.
  *

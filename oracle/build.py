@@ -1,7 +1,7 @@
 """Compile the C oracle into oracle/liboracle.so (gcc, OpenMP, no fast-math).
 
-TEST INFRASTRUCTURE ONLY: the library built here is loaded by the tests, the
-graft smoke check and the CPU-baseline leg of bench.py, never by the product.
+TEST INFRASTRUCTURE ONLY: the library built here is loaded by the tests,
+__graft_entry__.smoke() and the CPU-baseline leg of bench.py, never by the product.
 """
 import os
 import subprocess
