@@ -60,7 +60,8 @@ def _f(x):
     return float(x)
 
 
-def main():
+def cases():
+    """The cases with their expected outputs from the brute force (as strings)."""
     out = []
     for c in CASES:
         import numpy as np
@@ -72,10 +73,14 @@ def main():
         case = dict(c)
         case["expected"] = [[[str(x) for x in row] for row in head] for head in res]
         out.append(case)
+    return out
+
+
+def main():
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "semantics_cases.json")
     with open(path, "w") as f:
         json.dump({"generator": "tests/golden/make_golden.py (oracle.brute, 50 digits)",
-                   "cases": out}, f, indent=1)
+                   "cases": cases()}, f, indent=1)
     print(path)
 
 

@@ -33,3 +33,14 @@ def test_oracle_reproduces_golden_case(case):
             assert math.isnan(g)
         else:
             assert abs(g - w) <= 1e-12
+
+
+def test_stored_cases_are_what_the_committed_script_writes():
+    # the fixture is the brute force's output for the script's inputs, and
+    # nothing else (no value in it came from anywhere but oracle.brute)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "make_golden", os.path.join(os.path.dirname(__file__), "golden", "make_golden.py"))
+    mg = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mg)
+    assert json.loads(json.dumps(mg.cases())) == _cases()
