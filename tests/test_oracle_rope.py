@@ -96,3 +96,9 @@ def test_append_writes_only_the_destination_rows(in_dtype, kv_dtype):
     norm = lambda a: a[:, :128] ** 2 + a[:, 128:] ** 2
     rel = 8e-3 if kv_dtype != "f32" else 1e-5
     assert np.max(np.abs(norm(k32) - norm(src)) / (1 + norm(src))) <= 2 * rel
+    # the stored K rows are the source rows rotated: pair (i, i + 128) as the
+    # complex number x_i + j x_{i+128} times e^{j angle}, angle from the tables
+    ang = np.arctan2(sin[:2, :128].astype(np.float64), cos[:2, :128].astype(np.float64))
+    z = (src[:, :128] + 1j * src[:, 128:]) * np.exp(1j * ang)
+    want_k = np.concatenate([z.real, z.imag], 1)
+    assert np.max(np.abs(k32 - want_k)) <= rel * (1 + np.max(np.abs(want_k)))
