@@ -1,5 +1,8 @@
-// kca_merge.cuh -- log-sum-exp merge of split partials, shared by the decode
-// (rows) path and the tensor-core prefill path.
+// kca_merge.cuh -- log-sum-exp merge of split partials, shared by the
+// CUDA-core rows path (merge_rows_kernel) and the merge of context-shard
+// records (attn_merge_partials).  The tensor-core prefill path has its own
+// merge kernel in kca_prefill_tc.cu, and the tensor-core decode kernel merges
+// in-kernel.
 //
 // A partial row is (m, l, acc[256]): m the reference max of its scores
 // (m * mscale is in log2 units), l = sum 2^(x - m) and acc = sum 2^(x - m) v
