@@ -14,7 +14,6 @@ Arrays are numpy arrays in their stored format: float32, float16, or bf16
 carried as uint16 bit patterns together with dtype="bf16".
 """
 import ctypes
-import os
 
 import numpy as np
 

@@ -4,12 +4,10 @@ give the same bits as the same calls one after the other (the library keeps
 no per-call device state; its host caches are per thread or idempotent)."""
 import threading
 
-import numpy as np
 import pytest
 import torch
 
 import kv_cache_attention_states_b200 as kca
-from kv_cache_attention_states_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
