@@ -3,6 +3,7 @@
 // workspace carving, tensor-map encoding and kernel launches.  Nothing here
 // allocates device memory or synchronises a stream (attn_device_status aside,
 // which exists to read the device status word).
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -37,7 +38,7 @@ int geometry_status(int32_t hq, int32_t hkv, int32_t d) {
 
 // SM count of the current device (cached per device).
 int current_sms(int* out) {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];   // zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KCA_ERR_CUDA;
   if (dev >= 0 && dev < 64 && cache[dev] > 0) {
@@ -130,16 +131,15 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  // Looked up once; a function-local static is initialised thread-safely.
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+  }();
   return fn;
 }
 

@@ -32,6 +32,7 @@
 // shared memory as 16 rows (hi, lo) x 64 keys, then O[:, 32w .. 32w+31] +=
 // P V (16 MMAs).  Rows past the split's end are zeroed in shared memory, so
 // whatever the cache holds there never reaches the output.
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -625,7 +626,7 @@ template <int QT, int KT>
 cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsArgs& a,
                      cudaStream_t stream) {
   auto kern = decode_mma_kernel<QT, KT>;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
@@ -680,7 +681,7 @@ int cluster_capacity_t(int c) {
 
 int decode_mma_cluster_capacity(int c) {
   // Same launch shape for every dtype instantiation; cached per device and size.
-  static int cache[64][4] = {{0}};
+  static std::atomic<int> cache[64][4];   // zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   const int idx = c == 1 ? 0 : (c == 2 ? 1 : (c == 4 ? 2 : 3));

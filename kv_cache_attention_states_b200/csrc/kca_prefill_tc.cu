@@ -44,6 +44,7 @@
 // warpgroups) only when a half row's sum passes 2^8.  Work items of a split
 // row tile write (m, l, O) partials that merge_tc_kernel (below) combines by
 // log-sum-exp.
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -631,7 +632,7 @@ template <int DT>
 cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmq,
                      const CUtensorMap& tmo, const CUtensorMap& tmpart, const CUtensorMap& tmpart_rag,
                      const TcArgs& a, cudaStream_t stream) {
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {

@@ -9,6 +9,7 @@
 // CTA per split; K/V rows stream through a shared-memory ring filled by bulk
 // copies, each warp reduces its QK dots with warp shuffles and keeps an online
 // softmax, and the splits are merged by log-sum-exp in merge_rows_kernel.
+#include <atomic>
 #include <cuda_runtime.h>
 
 #include "kca_common.cuh"
@@ -313,7 +314,7 @@ template <int QT, int KT>
 cudaError_t launch_rows_t(const RowsArgs& a, cudaStream_t stream) {
   using S = RowsSmem<KT>;
   auto kern = rows_kernel<QT, KT>;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {

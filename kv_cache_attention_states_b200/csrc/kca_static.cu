@@ -23,6 +23,7 @@
 // clears them first with cudaMemsetAsync on its stream -- a memset, not an
 // allocation.  Everything past the header is written before it is read
 // within the same call.
+#include <atomic>
 #include <cuda_runtime.h>
 
 #include "../../include/kca.h"
@@ -36,7 +37,7 @@ static __device__ __align__(256) unsigned char kca_static_scratch[KCA_STATIC_SCR
 // Device address of kca_static_scratch per device; the name itself is only a
 // host-side stand-in and must never be handed to a kernel.
 void* scratch_address(int* status) {
-  static void* addr[64] = {nullptr};
+  static std::atomic<void*> addr[64];   // zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     *status = KCA_ERR_CUDA;
