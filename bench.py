@@ -1,19 +1,31 @@
 """Benchmark of the states-form attention hot path on B200.
 
-One step = the whole path on one batch of synthetic input:
-  * chunked causal prefill of a 16,384-token prompt in 768-row chunks
-    (21 x 768 + 256), bf16 Q/K/V ~ N(0,1)*0.5, through attn_prefill, and
-  * 64 single-row decode steps at context 16,384 .. 16,447, f16 K/V ~ N(0,1),
-    f32 query, through attn_decode.
+One step = PASSES passes; one pass runs every workload configuration once,
+each as a CUDA graph of its C-ABI calls, in this order (each small working
+set follows a large one, so that its calls read cold rows from HBM):
+
+  ragged         8 sequences, context drawn by the seed from [1024, 131072],
+                 32 decode steps, f16 K/V, f32 q
+  decode_256     64 decode steps at context 256..319, f16 K/V, f32 q
+                 (64 cache replicas, one per step)
+  decode_4096    64 decode steps at context 4096..4159 (64 replicas)
+  prefill        the 16,384-token prompt in 768-row chunks (21 x 768 + 256),
+                 bf16 Q/K/V ~ N(0,1)*0.5 (2 input replicas)        -> value
+  decode         64 decode steps at context 16384..16447 (32 replicas)
+  window         window 512: a 4,096-token prompt in 768-row chunks, then 64
+                 decode steps at positions 4096..4159, bf16 Q/K/V ~ N(0,1)
+  long_chunk     one 768-row bf16 chunk at positions 130304..131071 of a
+                 131,072-row cache
+
 value = prefill q-rows/s (a q-row is one query position with all 8 heads),
-timed with CUDA events around the prefill part of every step; the decode
-part is reported as decode tok/s beside it; ms_per_step covers both.
+from CUDA events around the prefill graph of every pass; every other
+configuration gets its own object in the JSON line, timed the same way.
+ms_per_step covers whole steps.  The decode caches smaller than L2 rotate
+over replicas (and follow the 1 GB ragged batch in each pass), so every
+timed call reads its K/V rows from HBM; the sliding-window decode re-reads
+rows its previous step read by construction of the window.
 
-L2: inputs are rotated across replicas whose total exceeds the 126 MB L2
-(decode: one 16.8 MB cache replica per step index mod 32; prefill: two
-input replicas), so every step reads cold rows from HBM.
-
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--passes P] [--impl reference]
 Under torchrun each rank runs its own replica of the workload (weak scaling,
 no collective on the data path); rank 0 prints one JSON line.
 """
@@ -34,10 +46,15 @@ DECODE_LEN = 16384
 DECODE_STEPS = 64
 DECODE_REPLICAS = 32
 PREFILL_REPLICAS = 2
+SMALL_DECODE_REPLICAS = 64
+PASSES = 8               # passes over every configuration per step
 # DRAM bytes (read + write) per launch from one ncu capture of the current
-# kernels; reset to None whenever a kernel changes after its capture.
-PREFILL_TRAFFIC = 18.931e6 + 25.6e3
-DECODE_TRAFFIC = 16.919e6
+# kernels, with the launch they come from; None once a kernel has changed
+# since its capture.
+TRAFFIC = {
+    "prefill": (18.931e6 + 25.6e3, "prefill_tc_kernel, chunk 19 (768 rows at 14592)"),
+    "decode": (16.919e6, "decode_mma_kernel, one call at ctx ~16.4K"),
+}
 E2E_GROUP = 4            # prefill chunks per host copy in the end-to-end leg
 METRIC = "prefill q-rows/s & decode tok/s at 16K ctx (1 B200); % of TC/HBM roofline"
 
@@ -47,8 +64,9 @@ def _peaks():
     if os.path.exists(path):
         with open(path) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)) or None, \
+            "measured"
+    return 6650.0, 1590.0, None, "fallback"
 
 
 def max_over_ranks(values, world: int, device):
@@ -62,15 +80,26 @@ def max_over_ranks(values, world: int, device):
     return t.tolist()
 
 
-def prefill_flops() -> float:
+def visible(pos: int, window: int) -> int:
+    """Keys a query at pos sees."""
+    lo = max(0, pos - window + 1) if window > 0 else 0
+    return pos - lo + 1
+
+
+def prefill_flops(chunks, window=0) -> float:
     # 2 GEMMs (QK^T and PV) x 2 flop x head_dim x 8 heads per visible (query, key) pair
-    pairs = PREFILL_ROWS * (PREFILL_ROWS + 1) // 2
+    pairs = 0
+    for cs, r in chunks:
+        if window <= 0:
+            pairs += r * cs + r * (r + 1) // 2
+        else:
+            pairs += sum(visible(p, window) for p in range(cs, cs + r))
     return 4.0 * 256 * 8 * pairs
 
 
-def decode_bytes(ctx: int) -> int:
-    # K + V rows (f16) once, q and out (f32)
-    return ctx * 256 * 2 * 2 + 2 * 8 * 256 * 4
+def decode_bytes(ctx: int, window: int = 0, kv_size: int = 2, q_size: int = 4) -> int:
+    # K + V rows of the visible keys once, the query and the f32 output
+    return visible(ctx - 1, window) * 256 * kv_size * 2 + 8 * 256 * (q_size + 4)
 
 
 class Clocks:
@@ -166,10 +195,11 @@ class Clocks:
                 "reasons": sorted(self.reasons), "samples": len(sm), "source": self.source}
 
 
-# ------------------------------------------------------------- the workload
+# ------------------------------------------------------------- the workloads
 
 class Workload:
-    """Device-resident inputs of one step (and the replicas that defeat L2)."""
+    """Device-resident inputs of the headline configurations (the 16K prompt
+    and the 64 decode steps at 16K) and the replicas that defeat L2."""
 
     def __init__(self, device, seed=0):
         import torch
@@ -204,17 +234,6 @@ class Workload:
                                         device)
         self.step_index = 0
 
-    def launches_per_step(self) -> int:
-        kca = self.kca
-        n = 0
-        for cs, r in self.chunks:
-            path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, r, 0, self.sms)
-            n += 1 + int((items[:, 3] >= 0).any())
-        # f16 caches take the tensor-core rows kernel, which merges its
-        # splits in the same launch: one kernel per decode call.
-        n += len(self.dec_ctx)
-        return n
-
     def prefill(self):
         q, k, v = self.pre[self.step_index % PREFILL_REPLICAS]
         for cs, r in self.chunks:
@@ -227,69 +246,306 @@ class Workload:
             self.kca.attn_decode(self.dec_q[t], k, v, [c], out=self.dec_out[t], workspace=self.dec_ws)
 
 
+def _prefill_launches(kca, chunks, window, sms):
+    n = 0
+    for cs, r in chunks:
+        path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, r, window, sms)
+        n += 1 + int(path == 1 and (items[:, 3] >= 0).any())
+    return n
+
+
+class Part:
+    """One workload configuration of a pass: `run(variant)` issues its calls
+    (captured once per variant as a CUDA graph), `units` counts its output
+    rows or tokens, `work` its algorithmic flops (tensor-bound) or bytes
+    (HBM-bound) per run."""
+    name = ""
+    unit = ""
+    variants = 1
+    bound = "hbm"
+    units = 0
+    work = 0.0
+    launches = 0
+    kernel = ""
+    algorithmic = ""
+    workload = ""
+
+    def run(self, variant):
+        raise NotImplementedError
+
+    def status(self):
+        return [ws for ws in self.workspaces()]
+
+    def workspaces(self):
+        return []
+
+
+class PrefillPart(Part):
+    name, unit, bound = "prefill", "q-rows", "tensor"
+    kernel = "prefill_tc_kernel (+ its merge)"
+
+    def __init__(self, w, sms):
+        self.w = w
+        self.variants = PREFILL_REPLICAS
+        self.units = PREFILL_ROWS
+        self.work = prefill_flops(w.chunks)
+        self.launches = _prefill_launches(w.kca, w.chunks, 0, sms)
+        self.algorithmic = "4*256*8*sum|J(pos)| = 1.0996e12 flop per prompt"
+
+    def run(self, variant):
+        self.w.step_index = variant
+        self.w.prefill()
+
+    def workspaces(self):
+        return [self.w.pre_ws]
+
+
+class HeadlineDecodePart(Part):
+    name, unit, bound = "decode", "tok", "hbm"
+    kernel = "decode_mma_kernel<f32 q, f16 KV> (merge in-kernel)"
+
+    def __init__(self, w):
+        self.w = w
+        self.units = len(w.dec_ctx)
+        self.work = float(sum(decode_bytes(c) for c in w.dec_ctx))
+        self.launches = len(w.dec_ctx)
+        self.algorithmic = "ctx*1024 B K/V + 16 KiB q/out per token"
+
+    def run(self, variant):
+        self.w.step_index = 0
+        self.w.decode()
+
+    def workspaces(self):
+        return [self.w.dec_ws]
+
+
+class DecodeLenPart(Part):
+    """64 decode steps of one sequence at context L..L+63 (f16 K/V, f32 q),
+    step t on cache replica t (the replicas together exceed the working set
+    that L2 could hold between two visits)."""
+    unit, bound = "tok", "hbm"
+    kernel = "decode_mma_kernel<f32 q, f16 KV>"
+
+    def __init__(self, device, length, seed=0):
+        import torch
+        import kv_cache_attention_states_b200 as kca
+        from kv_cache_attention_states_b200 import synth
+        self.kca = kca
+        self.name = f"decode_{length}"
+        wl = synth.decode_f16(length, DECODE_STEPS)
+        self.ctx = [c[0] for c in wl.decode_ctx]
+        self.cap = wl.capacity
+        k0 = synth.as_torch(synth.draw(seed, "k", (1, self.cap, 256), "f16"), "f16").to(device)
+        v0 = synth.as_torch(synth.draw(seed, "v", (1, self.cap, 256), "f16"), "f16").to(device)
+        self.kv = [(k0, v0)] + [(k0.clone(), v0.clone()) for _ in range(SMALL_DECODE_REPLICAS - 1)]
+        self.q = synth.as_torch(synth.draw(seed, "q", (DECODE_STEPS, 1, 8, 256), "f32"), "f32").to(device)
+        self.out = torch.empty((DECODE_STEPS, 1, 8, 256), dtype=torch.float32, device=device)
+        self.ws = kca.new_workspace(max(kca.attn_decode_workspace_bytes([c]) for c in self.ctx), device)
+        self.units = DECODE_STEPS
+        self.work = float(sum(decode_bytes(c) for c in self.ctx))
+        self.launches = DECODE_STEPS
+        self.algorithmic = "ctx*1024 B K/V + 16 KiB q/out per token"
+        self.workload = (f"1 sequence, 64 decode steps at ctx {length}-{length + 63}, f16 K/V N(0,1), "
+                         f"f32 q; {SMALL_DECODE_REPLICAS} cache replicas")
+
+    def run(self, variant):
+        for t, c in enumerate(self.ctx):
+            k, v = self.kv[t % len(self.kv)]
+            self.kca.attn_decode(self.q[t], k, v, [c], out=self.out[t], workspace=self.ws)
+
+    def workspaces(self):
+        return [self.ws]
+
+
+class WindowParts:
+    """The sliding-window configuration: a 4,096-token prompt in 768-row
+    chunks, then 64 decode steps at positions 4096..4159, window 512, bf16."""
+
+    def __init__(self, device, sms, seed=0):
+        import torch
+        import kv_cache_attention_states_b200 as kca
+        from kv_cache_attention_states_b200 import synth
+        self.kca = kca
+        wl = synth.window_bf16(DECODE_STEPS)
+        self.wl = wl
+        self.cap = wl.capacity
+        n = 4096
+        self.k = synth.as_torch(synth.draw(seed, "k", (self.cap, 256), "bf16"), "bf16").to(device)
+        self.v = synth.as_torch(synth.draw(seed, "v", (self.cap, 256), "bf16"), "bf16").to(device)
+        self.q = synth.as_torch(synth.draw(seed, "q", (n, 8, 256), "bf16"), "bf16").to(device)
+        self.qd = synth.as_torch(synth.draw(seed, "qd", (DECODE_STEPS, 1, 8, 256), "bf16"), "bf16").to(device)
+        self.out = torch.empty((n, 8, 256), dtype=torch.float32, device=device)
+        self.dout = torch.empty((DECODE_STEPS, 1, 8, 256), dtype=torch.float32, device=device)
+        self.ws = kca.new_workspace(max(
+            [kca.attn_prefill_workspace_bytes(kca.BF16, kca.BF16, cs, r, wl.window) for cs, r in wl.prefill]
+            + [kca.attn_decode_workspace_bytes(c, wl.window) for c in wl.decode_ctx]), device)
+        outer = self
+
+        class Pre(Part):
+            name, unit, bound = "window_prefill", "q-rows", "tensor"
+            kernel = "prefill_tc_kernel (+ its merge), window 512"
+            units = n
+            work = prefill_flops(wl.prefill, wl.window)
+            launches = _prefill_launches(kca, wl.prefill, wl.window, sms)
+            algorithmic = "4*256*8*sum|J(pos)| with |J| <= 512 = 1.611e10 flop"
+
+            def run(self, variant):
+                for cs, r in wl.prefill:
+                    kca.attn_prefill(outer.q[cs:cs + r], outer.k, outer.v, cs, wl.window,
+                                     out=outer.out[cs:cs + r], workspace=outer.ws)
+
+            def workspaces(self):
+                return [outer.ws]
+
+        class Dec(Part):
+            name, unit, bound = "window_decode", "tok", "hbm"
+            kernel = "decode_mma_kernel<bf16 q, bf16 KV>, window 512"
+            units = DECODE_STEPS
+            work = float(sum(decode_bytes(c[0], wl.window, 2, 2) for c in wl.decode_ctx))
+            launches = DECODE_STEPS
+            algorithmic = "512 keys x 1024 B K/V + 12 KiB q/out per token"
+
+            def run(self, variant):
+                k1, v1 = outer.k.view(1, outer.cap, 256), outer.v.view(1, outer.cap, 256)
+                for t, c in enumerate(wl.decode_ctx):
+                    kca.attn_decode(outer.qd[t], k1, v1, c, wl.window, out=outer.dout[t], workspace=outer.ws)
+
+            def workspaces(self):
+                return [outer.ws]
+
+        self.parts = [Pre(), Dec()]
+
+
+class LongChunkPart(Part):
+    """One 768-row bf16 chunk at positions 130304..131071 of a 131,072-row cache."""
+    name, unit, bound = "long_chunk", "q-rows", "tensor"
+    kernel = "prefill_tc_kernel (+ its merge)"
+
+    def __init__(self, device, sms, seed=0):
+        import torch
+        import kv_cache_attention_states_b200 as kca
+        from kv_cache_attention_states_b200 import synth
+        self.kca = kca
+        wl = synth.long_chunk_bf16()
+        self.cs, self.rows = wl.prefill[0]
+        self.k = synth.as_torch(synth.draw(seed, "k", (wl.capacity, 256), "bf16"), "bf16").to(device)
+        self.v = synth.as_torch(synth.draw(seed, "v", (wl.capacity, 256), "bf16"), "bf16").to(device)
+        self.q = synth.as_torch(synth.draw(seed, "q", (self.rows, 8, 256), "bf16"), "bf16").to(device)
+        self.out = torch.empty((self.rows, 8, 256), dtype=torch.float32, device=device)
+        self.ws = kca.new_workspace(kca.attn_prefill_workspace_bytes(kca.BF16, kca.BF16, self.cs, self.rows),
+                                    device)
+        self.units = self.rows
+        self.work = prefill_flops(wl.prefill)
+        self.launches = _prefill_launches(kca, wl.prefill, 0, sms)
+        self.algorithmic = "4*256*8*sum|J(pos)| = 8.222e11 flop"
+
+    def run(self, variant):
+        self.kca.attn_prefill(self.q, self.k, self.v, self.cs, out=self.out, workspace=self.ws)
+
+    def workspaces(self):
+        return [self.ws]
+
+
+class RaggedPart(Part):
+    """8 sequences with contexts drawn by the seed from [1024, 131072], 32
+    decode steps, f16 K/V, f32 q; the 1.07 GB cache is far larger than L2."""
+    name, unit, bound = "decode_ragged", "tok", "hbm"
+    kernel = "decode_mma_kernel<f32 q, f16 KV>"
+
+    def __init__(self, device):
+        import torch
+        import kv_cache_attention_states_b200 as kca
+        from kv_cache_attention_states_b200 import synth
+        self.kca = kca
+        wl = synth.ragged_f16(0)
+        self.wl = wl
+        g = torch.Generator(device=device)
+        g.manual_seed(1)
+        self.k = torch.randn((wl.batch, wl.capacity, 256), generator=g, device=device).half()
+        self.v = torch.randn((wl.batch, wl.capacity, 256), generator=g, device=device).half()
+        self.q = torch.randn((len(wl.decode_ctx), wl.batch, 8, 256), generator=g, device=device)
+        self.out = torch.empty_like(self.q)
+        self.ws = kca.new_workspace(max(kca.attn_decode_workspace_bytes(c) for c in wl.decode_ctx), device)
+        self.units = wl.batch * len(wl.decode_ctx)
+        self.work = float(sum(sum(decode_bytes(x) for x in c) for c in wl.decode_ctx))
+        self.launches = len(wl.decode_ctx)
+        self.algorithmic = "ctx*1024 B K/V + 16 KiB q/out per token"
+        self.mean_ctx = float(np.mean(wl.decode_ctx[0]))
+
+    def run(self, variant):
+        for t, c in enumerate(self.wl.decode_ctx):
+            self.kca.attn_decode(self.q[t], self.k, self.v, c, out=self.out[t], workspace=self.ws)
+
+    def workspaces(self):
+        return [self.ws]
+
+
+def build_parts(w, device, sms):
+    """The parts of one pass, in pass order (see the module docstring)."""
+    win = WindowParts(device, sms)
+    parts = [RaggedPart(device), DecodeLenPart(device, 256), DecodeLenPart(device, 4096),
+             PrefillPart(w, sms), HeadlineDecodePart(w)] + win.parts + [LongChunkPart(device, sms)]
+    return parts
+
+
 def run_cuda(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     w = Workload(dev)
-    w.sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    parts = build_parts(w, dev, sms)
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        w.prefill()
-        w.decode()
-        w.step_index += 1
+    passes = max(1, args.passes)
+    # warm-up: eager calls first (tensor-map caches, function attributes)
+    for s in range(args.warmup):
+        for p in parts:
+            p.run(s % p.variants)
     torch.cuda.synchronize()
     graphs = None
     if not args.eager:
-        # One graph per prefill input replica and one for the 64 decode steps
-        # (each step visits the 32 cache replicas in the same order).
-        graphs = {"pre": [], "dec": None}
-        saved = w.step_index
-        for r in range(PREFILL_REPLICAS):
-            g = torch.cuda.CUDAGraph()
-            w.step_index = r
-            with torch.cuda.graph(g):
-                w.prefill()
-            graphs["pre"].append(g)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            w.decode()
-        graphs["dec"] = g
-        w.step_index = saved
+        graphs = {}
+        for p in parts:
+            graphs[p.name] = []
+            for var in range(p.variants):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    p.run(var)
+                graphs[p.name].append(g)
         for _ in range(2):
-            graphs["pre"][w.step_index % PREFILL_REPLICAS].replay()
-            graphs["dec"].replay()
-            w.step_index += 1
+            for p in parts:
+                for g in graphs[p.name]:
+                    g.replay()
         torch.cuda.synchronize()
+
+    def replay(p, i):
+        if graphs is None:
+            p.run(i % p.variants)
+        else:
+            graphs[p.name][i % p.variants].replay()
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = Clocks(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    n_runs = args.steps * passes
+    ev = {p.name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(n_runs)] for p in parts}
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    # NVTX ranges name the phases on a profiler timeline (no cost otherwise).
     nvtx = torch.cuda.nvtx
     nvtx.range_push("timed steps")
     start.record(stream)
+    i = 0
     for s in range(args.steps):
-        ev[s][0].record(stream)
-        nvtx.range_push("prefill")
-        if graphs is None:
-            w.prefill()
-        else:
-            graphs["pre"][w.step_index % PREFILL_REPLICAS].replay()
-        nvtx.range_pop()
-        ev[s][1].record(stream)
-        nvtx.range_push("decode")
-        if graphs is None:
-            w.decode()
-        else:
-            graphs["dec"].replay()
-        nvtx.range_pop()
-        ev[s][2].record(stream)
-        w.step_index += 1
+        for _ in range(passes):
+            for p in parts:
+                e0, e1 = ev[p.name][i]
+                e0.record(stream)
+                replay(p, i)
+                e1.record(stream)
+            i += 1
     end.record(stream)
     nvtx.range_pop()
     torch.cuda.synchronize()
@@ -298,23 +554,23 @@ def run_cuda(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     total_ms = start.elapsed_time(end)
-    pre_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
-    dec_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
-    total_ms, pre_ms, dec_ms = max_over_ranks([total_ms, pre_ms, dec_ms], world, dev)
-    st, detail = w.kca.attn_device_status(w.pre_ws)
-    st2, _ = w.kca.attn_device_status(w.dec_ws)
-    if st != 0 or st2 != 0:
-        raise RuntimeError(f"device status {st}/{st2} detail {detail:#x}")
-    res = dict(total_ms=total_ms, pre_ms=pre_ms, dec_ms=dec_ms, clocks=clk,
-               launches=w.launches_per_step() * args.steps)
+    names = [p.name for p in parts]
+    part_ms = [sum(a.elapsed_time(b) for a, b in ev[nm]) for nm in names]
+    vals = max_over_ranks([total_ms] + part_ms, world, dev)
+    total_ms, part_ms = vals[0], dict(zip(names, vals[1:]))
+    for p in parts:
+        for ws in p.workspaces():
+            st, detail = w.kca.attn_device_status(ws)
+            if st != 0:
+                raise RuntimeError(f"{p.name}: device status {st} detail {detail:#x}")
+    res = dict(total_ms=total_ms, part_ms=part_ms, runs=n_runs, clocks=clk, passes=passes,
+               launches=sum(p.launches for p in parts) * n_runs,
+               parts={p.name: p for p in parts})
+    if graphs is not None:
+        del graphs
     e2e = run_e2e(w, args, stream)
     e2e["pre_ms"], e2e["dec_ms"] = max_over_ranks([e2e["pre_ms"], e2e["dec_ms"]], world, dev)
     res["e2e"] = e2e
-    del w, graphs
-    torch.cuda.empty_cache()
-    rg = run_ragged(dev, stream)
-    rg["tok_s"], rg["gbs"] = [-x for x in max_over_ranks([-rg["tok_s"], -rg["gbs"]], world, dev)]
-    res["ragged"] = rg
     return res
 
 
@@ -409,57 +665,6 @@ def run_e2e(w, args, stream):
                 pre_d2h=pre_d2h)
 
 
-def run_ragged(device, stream):
-    """The ragged long-context decode workload (8 sequences, lengths drawn by
-    the seed from [1024, 131072], 32 steps, f16 K/V, f32 q), timed after the
-    main region as one CUDA graph of its 32 calls: where the decode kernel
-    is HBM-bound rather than latency-bound.  The 1.07 GB cache is far larger
-    than L2, so no replica rotation is needed.  Reported beside the headline
-    decode figure, not in it."""
-    import torch
-    import kv_cache_attention_states_b200 as kca
-    from kv_cache_attention_states_b200 import synth
-    wl = synth.ragged_f16(0)
-    g = torch.Generator(device=device)
-    g.manual_seed(1)
-    k = torch.randn((wl.batch, wl.capacity, 256), generator=g, device=device).half()
-    v = torch.randn((wl.batch, wl.capacity, 256), generator=g, device=device).half()
-    q = torch.randn((len(wl.decode_ctx), wl.batch, 8, 256), generator=g, device=device)
-    out = torch.empty_like(q)
-    ws = kca.new_workspace(max(kca.attn_decode_workspace_bytes(c) for c in wl.decode_ctx), device)
-
-    def steps():
-        for t, c in enumerate(wl.decode_ctx):
-            kca.attn_decode(q[t], k, v, c, out=out[t], workspace=ws)
-
-    steps()
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        steps()
-    for _ in range(2):
-        graph.replay()
-    reps = 5
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    torch.cuda.nvtx.range_push("ragged decode")
-    e0.record(stream)
-    for _ in range(reps):
-        graph.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    torch.cuda.nvtx.range_pop()
-    st, detail = kca.attn_device_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status {st} detail {detail:#x}")
-    sec = e0.elapsed_time(e1) / 1e3
-    nbytes = sum(sum(decode_bytes(x) for x in c) for c in wl.decode_ctx) * reps
-    del graph, k, v
-    torch.cuda.empty_cache()
-    return {"tok_s": wl.batch * len(wl.decode_ctx) * reps / sec, "gbs": nbytes / sec / 1e9,
-            "ms_per_step": 1e3 * sec / (reps * len(wl.decode_ctx)),
-            "mean_ctx": float(np.mean(wl.decode_ctx[0]))}
-
 
 # ---------------------------------------------------------- CPU oracle legs
 
@@ -482,11 +687,17 @@ def _oracle_inputs(seed):
     return _ORACLE_INPUTS[seed]
 
 
+def _timed(fn):
+    t0 = time.perf_counter()
+    fn()
+    return time.perf_counter() - t0
+
+
 def oracle_sample(n_rows: int, n_decode: int, seed=0):
     """Time the f64 oracle (as it stands, all host cores) on a bounded sample
-    of the same workload: n_rows prefill rows evenly spaced over the prompt
-    (so their mean context equals the prompt's) and n_decode decode steps at
-    context 16,384.  Returns (rows/s, tok/s, cores, description)."""
+    of the headline workload: n_rows prefill rows evenly spaced over the
+    prompt (so their mean context equals the prompt's) and n_decode decode
+    steps at context 16,384.  Returns (rows/s, tok/s, cores, description)."""
     import oracle
     from kv_cache_attention_states_b200 import synth
     cores = os.cpu_count() or 1
@@ -494,19 +705,72 @@ def oracle_sample(n_rows: int, n_decode: int, seed=0):
     x = _oracle_inputs(seed)
     q, k, v = x["q"], x["k"], x["v"]
     rows = (np.arange(n_rows) * PREFILL_ROWS) // n_rows + PREFILL_ROWS // (2 * n_rows)
-    t0 = time.perf_counter()
-    oracle.attention(q[rows], k, v, rows, q_dtype="bf16", kv_dtype="bf16", scale=synth.SCALE)
-    t_pre = time.perf_counter() - t0
+    t_pre = _timed(lambda: oracle.attention(q[rows], k, v, rows, q_dtype="bf16", kv_dtype="bf16",
+                                            scale=synth.SCALE))
     kd, vd, qd = x["kd"], x["vd"], x["qd"]
-    t0 = time.perf_counter()
-    for t in range(n_decode):
-        oracle.attention(qd[t:t + 1], kd, vd, [x["ctx"][t] - 1], kv_dtype="f16",
-                         scale=synth.SCALE)
-    t_dec = time.perf_counter() - t0
+
+    def dec():
+        for t in range(n_decode):
+            oracle.attention(qd[t:t + 1], kd, vd, [x["ctx"][t] - 1], kv_dtype="f16", scale=synth.SCALE)
+    t_dec = _timed(dec)
     desc = (f"{n_rows} prefill rows evenly spaced over positions 0-16383 of the 16K bf16 prompt "
             f"({t_pre:.1f} s) + {n_decode} decode steps at ctx 16384 ({t_dec:.1f} s); f64 C oracle, "
             f"OpenMP over (row, head), {cores} threads")
     return n_rows / t_pre, n_decode / t_dec, cores, desc
+
+
+def oracle_part_samples(seed=0):
+    """The oracle on a bounded sample of every other configuration (a few
+    seconds each): {part name: (units/s, sample description)}."""
+    import oracle
+    from kv_cache_attention_states_b200 import synth
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
+    out = {}
+    for length, n in ((256, 64), (4096, 16)):
+        wl = synth.decode_f16(length, DECODE_STEPS)
+        k = synth.draw(seed, "k", (wl.capacity, 256), "f16")
+        v = synth.draw(seed, "v", (wl.capacity, 256), "f16")
+        q = synth.draw(seed, "q", (DECODE_STEPS, 8, 256), "f32")
+        ctx = [c[0] for c in wl.decode_ctx]
+
+        def dec():
+            for t in range(n):
+                oracle.attention(q[t:t + 1], k, v, [ctx[t] - 1], kv_dtype="f16", scale=synth.SCALE)
+        sec = _timed(dec)
+        out[f"decode_{length}"] = (n / sec, f"{n} decode steps at ctx {length}.. ({sec:.2f} s)")
+    wl = synth.window_bf16(DECODE_STEPS)
+    k = synth.draw(seed, "k", (wl.capacity, 256), "bf16")
+    v = synth.draw(seed, "v", (wl.capacity, 256), "bf16")
+    q = synth.draw(seed, "q", (4096, 8, 256), "bf16")
+    qd = synth.draw(seed, "qd", (DECODE_STEPS, 8, 256), "bf16")
+    rows = np.arange(0, 4096, 4)
+    sec = _timed(lambda: oracle.attention(q[rows], k, v, rows, window=wl.window, q_dtype="bf16",
+                                          kv_dtype="bf16", scale=synth.SCALE))
+    out["window_prefill"] = (rows.size / sec, f"every 4th of the 4096 prompt rows, window 512 ({sec:.2f} s)")
+    pos = np.array([c[0] - 1 for c in wl.decode_ctx])
+    sec = _timed(lambda: oracle.attention(qd, k, v, pos, window=wl.window, q_dtype="bf16", kv_dtype="bf16",
+                                          scale=synth.SCALE))
+    out["window_decode"] = (pos.size / sec, f"all 64 decode steps, window 512 ({sec:.2f} s)")
+    wl = synth.long_chunk_bf16()
+    cs, r = wl.prefill[0]
+    k = synth.draw(seed, "k", (wl.capacity, 256), "bf16")
+    v = synth.draw(seed, "v", (wl.capacity, 256), "bf16")
+    q = synth.draw(seed, "q", (r, 8, 256), "bf16")
+    rows = np.arange(0, r, r // 16)
+    sec = _timed(lambda: oracle.attention(q[rows], k, v, cs + rows, q_dtype="bf16", kv_dtype="bf16",
+                                          scale=synth.SCALE))
+    out["long_chunk"] = (rows.size / sec, f"{rows.size} rows evenly spaced over the 768-row chunk at "
+                                          f"130304 ({sec:.2f} s)")
+    wl = synth.ragged_f16(seed)
+    ctx = wl.decode_ctx[0][:2]
+    k = np.concatenate([synth.draw(seed, f"rk{b}", (c, 256), "f16") for b, c in enumerate(ctx)])
+    v = np.concatenate([synth.draw(seed, f"rv{b}", (c, 256), "f16") for b, c in enumerate(ctx)])
+    q = synth.draw(seed, "rq", (2, 8, 256), "f32")
+    base = np.array([0, ctx[0]])
+    sec = _timed(lambda: oracle.attention(q, k, v, np.array(ctx) - 1, base, kv_dtype="f16", scale=synth.SCALE))
+    out["decode_ragged"] = (2 / sec, f"sequences 0-1 of the first step (ctx {ctx[0]}, {ctx[1]}; {sec:.2f} s)")
+    return out, cores
 
 
 def run_reference(args, rank, world):
@@ -540,15 +804,44 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def part_object(p, ms, runs, world, hbm, tflops, tflops_sus, src, cpu=None):
+    """JSON object of one configuration: throughput, roofline of its kernel
+    (algorithmic work / measured time), the ncu traffic where captured."""
+    sec = ms / 1e3
+    per_run = sec / runs
+    obj = {"workload": p.workload or p.name, "value": world * p.units * runs / sec,
+           "unit": f"{p.unit}/s", "ms_per_run": 1e3 * per_run}
+    if p.bound == "tensor":
+        achieved = p.work / per_run / 1e12
+        roof = {"kernel": p.kernel, "bound": "tensor", "achieved": achieved, "peak": tflops,
+                "unit": "TFLOP/s", "frac": achieved / tflops, "peak_source": f"{src} bf16 dense (burst)"}
+        if tflops_sus:
+            roof["frac_of_sustained"] = achieved / tflops_sus
+    else:
+        achieved = p.work / per_run / 1e9
+        roof = {"kernel": p.kernel, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_source": f"{src} HBM copy"}
+    tr = TRAFFIC.get(p.name)
+    roof["traffic"] = tr[0] if tr else None
+    if tr:
+        roof["traffic_launch"] = tr[1]
+    roof["algorithmic"] = p.algorithmic
+    obj["roofline"] = roof
+    if cpu is not None:
+        obj["cpu_baseline"] = cpu
+    return obj
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--passes", type=int, default=PASSES, help="passes over every configuration per step")
     ap.add_argument("--impl", default="kca", choices=["kca", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every call from Python instead of "
-                    "replaying a captured CUDA graph of the step")
+                    "replaying captured CUDA graphs")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -564,70 +857,69 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     res = run_cuda(args, rank, world, local_rank)
-    cpu = None
+    cpu = parts_cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows_s, tok_s, cores, desc = oracle_sample(768, 4)
         cpu = {"value": rows_s, "unit": "q-rows/s", "cores": cores, "kind": "oracle", "sample": desc,
                "decode_tok_s": tok_s}
+        samples, cores = oracle_part_samples()
+        parts_cpu = {nm: {"value": v, "unit": ("q-rows/s" if nm in ("window_prefill", "long_chunk") else "tok/s"),
+                          "cores": cores, "kind": "oracle", "sample": d + "; f64 C oracle, OpenMP over (row, head)"}
+                     for nm, (v, d) in samples.items()}
+        parts_cpu["decode"] = {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                               "sample": desc}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
-    hbm, tflops, src = _peaks()
-    K = args.steps
-    pre_s = res["pre_ms"] / 1e3
-    dec_s = res["dec_ms"] / 1e3
-    value = world * PREFILL_ROWS * K / pre_s
-    dec_tok_s = world * DECODE_STEPS * K / dec_s
-    achieved_tf = prefill_flops() * K / pre_s / 1e12
-    dec_bytes = sum(decode_bytes(c) for c in range(DECODE_LEN, DECODE_LEN + DECODE_STEPS))
-    achieved_gbs = dec_bytes * K / dec_s / 1e9
+    hbm, tflops, tflops_sus, src = _peaks()
+    K, runs = args.steps, res["runs"]
+    parts, pm = res["parts"], res["part_ms"]
+
+    def obj(name):
+        return part_object(parts[name], pm[name], runs, world, hbm, tflops, tflops_sus, src,
+                           (parts_cpu or {}).get(name))
+
+    pre = obj("prefill")
     e2e = res["e2e"]
     line = {
-        "metric": METRIC, "value": value, "unit": "q-rows/s", "n_gpus": world, "steps": K,
+        "metric": METRIC, "value": pre["value"], "unit": "q-rows/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": res["total_ms"] / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "prefill of a 16384-token prompt in 768-row chunks (bf16, N(0,1)*0.5) "
                                "+ 64 decode steps at ctx 16384-16447 (f16 K/V, f32 q); 8 q heads / "
                                "1 KV head, head_dim 256, causal",
                    "seq_len": 16384, "global_batch": world, "parallelism": f"replicas x{world}",
-                   "value": "prefill part of each step (CUDA events); decode part in 'decode'",
-                   "launch": "eager" if args.eager else "CUDA graph of the step's C-ABI calls",
-                   "l2": "inputs larger than L2: decode rotates 32 cache replicas (16.8 MB each), "
-                         "prefill alternates 2 input replicas (80 MB each)"},
-        "roofline": {"kernel": "prefill_tc_kernel (+ its merge)", "bound": "tensor",
-                     "achieved": achieved_tf, "peak": tflops, "unit": "TFLOP/s",
-                     "frac": achieved_tf / tflops, "traffic": PREFILL_TRAFFIC,
-                     "traffic_source": "ncu dram bytes of the chunk-19 launch (768 rows at 14592); "
-                                       "profiles/prefill_tc_kernel_16k_late_chunks.md",
-                     "peak_source": f"{src} bf16 dense (burst)",
-                     "algorithmic": "4*256*8*sum|J(pos)| = 1.0996e12 flop per step"},
-        "decode": {"value": dec_tok_s, "unit": "tok/s", "ms_per_step": res["dec_ms"] / K,
-                   "roofline": {"kernel": "decode_mma_kernel<f32,f16> (merge in-kernel)", "bound": "hbm",
-                                "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                                "frac": achieved_gbs / hbm, "traffic": DECODE_TRAFFIC,
-                                "traffic_source": "ncu dram bytes of one launch at ctx ~16.4K; "
-                                                  "profiles/decode_mma_kernel_16k.md",
-                                "peak_source": f"{src} HBM copy",
-                                "algorithmic": "ctx*1024 B K/V + 16 KiB q/out per token"}},
+                   "step": f"{res['passes']} passes; a pass runs every configuration once (ragged, "
+                           "decode_256, decode_4096, prefill, decode, window, long_chunk)",
+                   "value": "prefill part of every pass (CUDA events); the other configurations in "
+                            "their own objects",
+                   "launch": "eager" if args.eager else "one CUDA graph per configuration of the C-ABI calls",
+                   "l2": "inputs larger than L2: decode caches rotate over replicas (16K: 32 x 16.8 MB; "
+                         "256 / 4096: 64 each, after the 1 GB ragged batch), the prompt alternates 2 "
+                         "input replicas (80 MB each)"},
+        "roofline": pre["roofline"],
+        "decode": obj("decode"),
+        "decode_256": obj("decode_256"),
+        "decode_4096": obj("decode_4096"),
+        "window": {"workload": "window 512, bf16 Q/K/V N(0,1): 4096-token prompt in 768-row chunks, then "
+                               "64 decode steps at positions 4096-4159 (the decode re-reads the rows the "
+                               "previous step read: sliding window)",
+                   "prefill": obj("window_prefill"), "decode": obj("window_decode")},
+        "long_chunk": obj("long_chunk"),
+        "decode_ragged": obj("decode_ragged"),
         "e2e": {"value": world * PREFILL_ROWS * e2e["steps"] / (e2e["pre_ms"] / 1e3), "unit": "q-rows/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "decode_tok_s": world * DECODE_STEPS * e2e["steps"] / (e2e["dec_ms"] / 1e3),
                 "steps": e2e["steps"]},
-        "decode_ragged": {"workload": "8 sequences, ctx drawn by the seed from [1024, 131072] "
-                                      f"(mean {res['ragged']['mean_ctx']:.0f}), 32 steps, f16 K/V, f32 q; "
-                                      "one CUDA graph, timed after the main region, not part of value",
-                          "value": world * res["ragged"]["tok_s"], "unit": "tok/s",
-                          "ms_per_step": res["ragged"]["ms_per_step"],
-                          "roofline": {"kernel": "decode_mma_kernel<f32,f16>", "bound": "hbm",
-                                       "achieved": res["ragged"]["gbs"], "peak": hbm, "unit": "GB/s",
-                                       "frac": res["ragged"]["gbs"] / hbm,
-                                       "algorithmic": "ctx*1024 B K/V + 16 KiB q/out per token"}},
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
     }
+    line["decode"]["workload"] = "64 decode steps at ctx 16384-16447, f16 K/V, f32 q (32 cache replicas)"
+    line["decode_ragged"]["workload"] = ("8 sequences, ctx drawn by the seed from [1024, 131072] (mean "
+                                         f"{parts['decode_ragged'].mean_ctx:.0f}), 32 steps, f16 K/V, f32 q")
+    line["long_chunk"]["workload"] = "one 768-row bf16 chunk at positions 130304-131071 of a 131072 cache"
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

@@ -39,6 +39,14 @@
  * call reads (for prefill the chunk's own rows too; for decode the row at
  * ctx_len-1).  Prefill requires ctx_len == chunk_start + chunk_rows.
  * Rows outside the union of the call's visible ranges are never read.
+ * V must be finite on the rows of a tensor-core prefill chunk's visible
+ * union: that path multiplies the exact zero probability of a masked key by
+ * its V row, so an Inf or NaN in V at position p also reaches rows that do
+ * not see p -- every output row of a 16-row tile whose work items cover p's
+ * 128-key tile (attn_prefill_plan lists them) becomes NaN, where the
+ * definition above leaves the rows that do not see p unaffected.  Rows that
+ * see a non-finite V value are non-finite on every path.  The rows path
+ * (decode, short or mixed-dtype chunks) reads only the keys each row sees.
  *
  * DTYPES: decode takes any q_dtype with any kv_dtype.  Prefill with
  * q_dtype == kv_dtype in {F16, BF16} and chunk_rows >= 16 runs on the
@@ -47,10 +55,14 @@
  * keys (one pass over the keys beats one pass per row there), else the rows
  * path, which also serves every other prefill combination: one unit per
  * query row, mma.sync with split-precision operands for 16-bit caches,
- * CUDA-core f32 for f32 caches.  Two environment variables, read at each
- * call, force a path so that tests can compare them on the same inputs:
- * KCA_PREFILL_PATH=rows (or =tc, where eligible) for prefill, and
- * KCA_DECODE_PATH=simt for the CUDA-core decode kernel on 16-bit caches.
+ * CUDA-core f32 for f32 caches.  attn_force_path pins either choice, so that
+ * tests can compare the paths on the same inputs.
+ *
+ * QUERIES: the workspace-size and plan queries come one per operation
+ * (attn_prefill_workspace_bytes, attn_decode_workspace_bytes,
+ * attn_decode_partial_workspace_bytes; attn_prefill_plan, attn_decode_plan)
+ * rather than as one call that takes an operation code, so that each takes
+ * exactly the arguments of its operation.
  *
  * OWNERSHIP: every buffer is allocated and owned by the caller.  The library
  * allocates no device memory, keeps no per-call state and never synchronises
@@ -112,6 +124,11 @@ extern "C" {
 
 /*
  * attn_prefill -- chunked causal prefill of one sequence.
+ * Passage: Karume v0.12.0 release notes, "Performance", item 1 (prefill of
+ * the states-form attention, chunk plans of 16 or more rows reading each K/V
+ * row once per row tile); v0.8.0 release notes, "Features", conversation-window
+ * item (chunkLength <= maxChunkLength = 768, capacity <= maxPosition = 131,072,
+ * both checked before any work).
  *   q_chunk      [chunk_rows][8][256] q_dtype, device
  *   k_cache/v_cache  the sequence's [capacity][1][256] kv_dtype rows, device
  *   capacity     rows the cache holds, 1..131072
@@ -133,6 +150,9 @@ int attn_prefill(const void *q_chunk, int32_t q_dtype,
 
 /*
  * attn_decode -- one query row per sequence (split-context decode + merge).
+ * Passage: Karume v0.12.0 release notes, "Performance", items 2-3 (one-row
+ * decode plans whose QK and PV reductions are split in parallel, then
+ * combined); v0.8.0 release notes, "Breaking Changes", softmax NaN item.
  *   q            [batch][8][256] q_dtype, device
  *   k_cache/v_cache  [batch][capacity][1][256] kv_dtype, device
  *   batch        1..256
@@ -155,7 +175,7 @@ int attn_decode(const void *q, int32_t q_dtype,
  * attn_decode_dev -- attn_decode with the context lengths in DEVICE memory,
  * read by the kernels when they run, so that one captured launch (CUDA graph)
  * serves every decode step while the caller updates ctx_len_dev in place.
- * The operation is the one-row (decode) plan of Karume v0.12.0 release notes,
+ * Passage: the one-row (decode) plan of Karume v0.12.0 release notes,
  * "Performance", items 2-3; the pages have no device-side context length:
  * it serves decode loops replayed from a CUDA graph, step after step.
  *   ctx_len_dev  DEVICE int64 [batch], 8-byte aligned; each value 0..ctx_bound,
@@ -199,9 +219,12 @@ int attn_decode_dev(const void *q, int32_t q_dtype,
  * The array keeps the last call's contents.  Its first KCA_WORKSPACE_HEADER
  * bytes (the device status word and the merge counters described above) must
  * be zero when a call starts, so each call that passes validation first
- * clears them with cudaMemsetAsync on `stream` (a memset, no allocation);
- * the device status of a call is therefore not kept for a later call to
- * read.
+ * clears them with cudaMemsetAsync on `stream` (a memset, no allocation).
+ * The device status of a call (a bounded wait that ran out) is therefore
+ * readable only until the next call: pass the address that
+ * attn_decode_static_scratch returns to attn_device_status after the call.
+ * The address is looked up again when the device's context was created anew
+ * (after cudaDeviceReset, say).
  */
 #define KCA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 int attn_decode_static(const void *q, int32_t q_dtype,
@@ -211,10 +234,22 @@ int attn_decode_static(const void *q, int32_t q_dtype,
                        float scale, float *out, void *stream);
 
 /*
+ * attn_decode_static_scratch -- the device address and size of the array
+ * attn_decode_static works in, on the current device (looked up as that call
+ * does; allocates nothing).  Its first bytes are a workspace header, so
+ * attn_device_status(*device_ptr, stream, &detail) reads and clears the
+ * status of the last attn_decode_static call on the device.  Writing the
+ * array while a call runs races with it.  The paper has no counterpart to
+ * this call either.  Returns KCA_OK, KCA_ERR_NULL or KCA_ERR_CUDA.
+ */
+int attn_decode_static_scratch(void **device_ptr, size_t *bytes);
+
+/*
  * attn_append_kv -- the step before the attention calls: writes n_rows new
  * K/V rows into the cache, K rotated by rotary position embedding with
- * host-generated cos/sin rows (Karume v0.8.0 release notes, "Features",
- * conversation-window item: the host generates the cos/sin rows per chunk),
+ * host-generated cos/sin rows (Passage: Karume v0.8.0 release notes,
+ * "Features", conversation-window item: the host generates the cos/sin rows
+ * per chunk),
  * V converted only.  Rotate-half pairing of dim i with dim i + 128:
  *   k'[i]       = k[i] cos[i] - k[i+128] sin[i]
  *   k'[i + 128] = k[i+128] cos[i+128] + k[i] sin[i+128]        (i < 128)
@@ -244,10 +279,10 @@ int attn_append_kv(const void *k_new, const void *v_new, int32_t in_dtype, int32
  * attn_decode_partial / attn_merge_partials -- decode with the context split
  * into shards (one per GPU, say): each shard yields the partial-softmax state
  * of every (sequence, head) over the keys it holds, and the states of all
- * shards merge into the output by the log-sum-exp identity.  The operation is
- * the decode of Karume v0.12.0 release notes, "Performance", items 2-3 (the
- * same softmax-weighted sum of V, reduced in a different order), restricted
- * to a key range; the pages have no multi-device form.
+ * shards merge into the output by the log-sum-exp identity.  Passage: the
+ * decode of Karume v0.12.0 release notes, "Performance", items 2-3 (the same
+ * softmax-weighted sum of V, reduced in a different order), restricted to a
+ * key range; the pages have no multi-device form.
  *
  * attn_decode_partial: the cache holds, for each sequence b, the rows of
  * positions [key_begin, key_begin + capacity) at rows b * capacity +
@@ -283,18 +318,29 @@ int attn_merge_partials(int32_t n_parts, int32_t batch, const float *parts, int6
                         float *out, void *stream);
 
 /* Workspace bytes the calls above need on the current device (0 on a bad
- * argument).  Always >= KCA_WORKSPACE_HEADER. */
+ * argument).  Always >= KCA_WORKSPACE_HEADER.  The size depends on the
+ * device (its SM count sets the split plan), so it is asked of the device the
+ * call will run on rather than guessed.  Passage: Karume v0.8.0 release
+ * notes, "Breaking Changes", estimateSessionMemory item (the estimator needs
+ * the device's binding limit and refuses to guess without it) and "Features",
+ * conversation-window item (what a window costs is reported before it is
+ * allocated). */
 size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
                                     int32_t chunk_rows, int32_t window);
 size_t attn_decode_workspace_bytes(int32_t batch, const int64_t *ctx_len, int32_t window);
 size_t attn_decode_partial_workspace_bytes(int32_t batch, const int64_t *ctx_len, int64_t key_begin,
                                            int64_t capacity, int32_t window);
 
-/* Zero the workspace header (cudaMemsetAsync on `stream`). */
+/* Zero the workspace header (cudaMemsetAsync on `stream`).  Passage: as for
+ * the workspace queries above (Karume v0.8.0 release notes, "Breaking
+ * Changes", estimateSessionMemory item). */
 int attn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Reads and clears the workspace status word (synchronises `stream`).
+ * Passage: Karume v0.8.0 release notes, "Breaking Changes", BatchScope.finish()
+ * item (a failure is reported to the caller instead of a dispatch going
+ * silently missing).
  * Error bits: 1 = a bounded wait ran out (detail: (site << 24) | block),
  * 2 = a device context length was out of range (detail: (10 << 24) | sequence),
  * 4 = an append destination was out of range (detail: (11 << 24) | row).
@@ -306,7 +352,10 @@ int attn_device_status(void *workspace, void *stream, uint32_t *detail);
 
 /*
  * Integer plans -- the work items a call with the same arguments runs -- for
- * bit-exact tests.  Each work item is 4 int64: (unit, key_begin, key_end, slot):
+ * bit-exact tests.  Passage: Karume v0.12.0 release notes, "Docs", ADR 0067
+ * plan-size geometry table (which kernel serves the QK / PV stages of 1,
+ * 2-15 and >= 16 rows), and "Performance", item 3 (kernels chosen by plan
+ * size).  Each work item is 4 int64: (unit, key_begin, key_end, slot):
  *   prefill, tensor-core path: unit = 16-row tile index, [key_begin, key_end)
  *     the absolute key positions the item covers (128-key tiles clipped to the
  *     call's visible union), slot = partial slot or -1 when the tile is not
@@ -334,7 +383,25 @@ int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
 int attn_decode_plan(int32_t batch, const int64_t *ctx_len, int32_t window, int32_t kv_dtype,
                      int32_t num_sms, int64_t *items, int32_t max_items, int32_t *n_items);
 
-/* Static description of a status code. */
+/*
+ * attn_force_path -- pins the kernel family that later calls take,
+ * process-wide, so that two paths can be compared on the same inputs (tests,
+ * diagnosis).  op 0 (prefill): path 0 = the rows path, 1 = the tensor-core
+ * path where eligible (q and cache both F16 or both BF16).  op 1 (the rows
+ * path: decode, and prefill chunks on the rows path): path 0 = the CUDA-core
+ * kernel, 1 = the tensor-core (mma.sync) kernel where eligible (16-bit
+ * cache).  path -1 restores the automatic choice described under DTYPES.
+ * Plans, workspace queries and calls all follow the pinned choice, so pin
+ * before sizing a workspace.  Returns KCA_OK or KCA_ERR_RANGE.
+ * Passage: Karume v0.12.0 release notes, "Performance", items 2-3 (the
+ * stateAttentionReduce seat, one knob that switches the QK and PV stages
+ * between the "sequential" and "parallel" kernels).
+ */
+int attn_force_path(int32_t op, int32_t path);
+
+/* Static description of a status code.  Passage: Karume v0.8.0 release
+ * notes, "Breaking Changes", numeric-contracts item (a violated contract is
+ * rejected with an error at the call). */
 const char *attn_status_string(int status);
 
 #ifdef __cplusplus

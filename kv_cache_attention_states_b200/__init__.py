@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.attn_prefill_plan.restype = ctypes.c_int
         L.attn_decode_plan.argtypes = [i32, p64, i32, i32, i32, p64, i32, p32]
         L.attn_decode_plan.restype = ctypes.c_int
+        L.attn_decode_static_scratch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(sz)]
+        L.attn_decode_static_scratch.restype = ctypes.c_int
+        L.attn_force_path.argtypes = [i32, i32]
+        L.attn_force_path.restype = ctypes.c_int
         L.attn_status_string.argtypes = [ctypes.c_int]
         L.attn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -403,14 +407,55 @@ def attn_decode_static(q, k_cache, v_cache, ctx_len, window: int = 0, scale: flo
     return out
 
 
+# ------------------------------------------------------------ path control
+
+OP_PREFILL, OP_ROWS = 0, 1                       # attn_force_path operations
+PATH_AUTO, PATH_ROWS, PATH_TENSOR_CORE = -1, 0, 1
+PATH_CUDA_CORE = 0                               # OP_ROWS: the CUDA-core kernel
+
+
+def attn_force_path(op: int, path: int) -> None:
+    """Pin the kernel family of later calls, process-wide (see include/kca.h):
+    op OP_PREFILL with PATH_ROWS / PATH_TENSOR_CORE, op OP_ROWS with
+    PATH_CUDA_CORE / PATH_TENSOR_CORE; PATH_AUTO restores the automatic choice."""
+    _check(lib().attn_force_path(int(op), int(path)), "attn_force_path")
+
+
+class forced_path:
+    """Context manager: attn_force_path(op, path) inside, PATH_AUTO after."""
+
+    def __init__(self, op: int, path: int):
+        self.op, self.path = op, path
+
+    def __enter__(self):
+        attn_force_path(self.op, self.path)
+        return self
+
+    def __exit__(self, *exc):
+        attn_force_path(self.op, PATH_AUTO)
+        return False
+
+
 # --------------------------------------------------------------------- plans
+
+def _num_sms(num_sms):
+    """num_sms as given, else the current CUDA device's SM count (the count
+    the calls plan for); without a device it has to be given."""
+    if num_sms is not None:
+        return int(num_sms)
+    import torch
+    if not torch.cuda.is_available():
+        raise ValueError("no CUDA device: pass num_sms to plan for a given SM count")
+    return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+
 
 def attn_prefill_path(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows: int,
                       window: int = 0) -> int:
     """The path a prefill call takes: 1 tensor-core, 0 rows (host only; no device needed)."""
     n = ctypes.c_int32(0)
     path = ctypes.c_int32(-1)
-    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, 148, None, 0,
+    # the path does not depend on the SM count; any positive count serves
+    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, 1, None, 0,
                                  ctypes.byref(n), ctypes.byref(path))
     if path.value < 0:
         raise KcaError(st, "attn_prefill_plan")
@@ -418,10 +463,12 @@ def attn_prefill_path(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows:
 
 
 def attn_prefill_plan(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows: int,
-                      window: int = 0, num_sms: int = 148):
-    """(path, items[n, 4]) -- see include/kca.h.  Host only, except the rows
-    plan of 16-bit caches, which is the tensor-core kernel's cluster plan on
-    the current device."""
+                      window: int = 0, num_sms: int | None = None):
+    """(path, items[n, 4]) -- see include/kca.h.  num_sms defaults to the
+    current device's SM count.  Host only, except the rows plan of 16-bit
+    caches, which is the tensor-core kernel's cluster plan on the current
+    device."""
+    num_sms = _num_sms(num_sms)
     n = ctypes.c_int32(0)
     path = ctypes.c_int32(0)
     st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, num_sms, None,
@@ -436,10 +483,14 @@ def attn_prefill_plan(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows:
     return int(path.value), items[:n.value]
 
 
-def attn_decode_plan(ctx_len, window: int = 0, num_sms: int = 148, kv_dtype: int = F32):
+def attn_decode_plan(ctx_len, window: int = 0, num_sms: int | None = None, kv_dtype: int = F32):
     """items[n, 4] of a decode call -- see include/kca.h.  kv_dtype F32: the
-    CUDA-core kernel's plan for num_sms SMs (host only); F16 / BF16: the
-    tensor-core kernel's cluster plan on the current device."""
+    CUDA-core kernel's plan for num_sms SMs (default: the current device's
+    count); F16 / BF16: the tensor-core kernel's cluster plan on the current
+    device."""
+    if kv_dtype in (F16, BF16) and num_sms is None:
+        num_sms = 1          # not used by the cluster plan, which asks the device itself
+    num_sms = _num_sms(num_sms)
     nctx, ptr = _i64_array(ctx_len)
     n = ctypes.c_int32(0)
     st = lib().attn_decode_plan(nctx, ptr, window, kv_dtype, num_sms, None, 0, ctypes.byref(n))

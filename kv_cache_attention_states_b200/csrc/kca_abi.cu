@@ -8,8 +8,6 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
-#include <cstdlib>
-#include <cstring>
 #include <vector>
 
 #include "../../include/kca.h"
@@ -53,9 +51,12 @@ int current_sms(int* out) {
   return KCA_OK;
 }
 
-// "tc" / "rows" forces the prefill path (tests use it to run both paths on
-// the same inputs); unset or anything else chooses by the rules in kca.h.
-// Chunks of fewer than 16 rows: the rows path streams the visible keys once
+// Paths pinned by attn_force_path (-1: automatic), read once per call.
+std::atomic<int> g_prefill_path{-1};
+std::atomic<int> g_rows_path{-1};
+
+// A forced prefill path (attn_force_path) wins where eligible; otherwise the
+// rules in kca.h choose.  Chunks of fewer than 16 rows: the rows path streams the visible keys once
 // per row (the first row from HBM, the rest mostly from L2), the tensor-core
 // path once per chunk but with a fixed cost of ~9 us (two launches, the
 // partials of the split tile, the merge).  B200 graph-replay timings of both
@@ -64,9 +65,9 @@ int current_sms(int* out) {
 // rows.
 bool use_tc(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, int32_t rows, int32_t window) {
   const bool eligible = q_dtype == kv_dtype && (q_dtype == KCA_F16 || q_dtype == KCA_BF16);
-  const char* env = std::getenv("KCA_PREFILL_PATH");
-  if (env != nullptr && std::strcmp(env, "rows") == 0) return false;
-  if (env != nullptr && std::strcmp(env, "tc") == 0) return eligible;
+  const int forced = g_prefill_path.load(std::memory_order_relaxed);
+  if (forced == 0) return false;
+  if (forced == 1) return eligible;
   if (!eligible) return false;
   if (rows >= kca::kRowTile) return true;
   return rows >= 3 && kca::n_visible(chunk_start, window) >= 12288;
@@ -224,12 +225,11 @@ void carve(void* ws, size_t ml_bytes, float** ml, float** acc) {
   *acc = reinterpret_cast<float*>(p + align_up(ml_bytes));
 }
 
-// 16-bit caches take the tensor-core rows kernel; "simt" in KCA_DECODE_PATH
-// forces the CUDA-core one (tests compare the two on the same inputs).
+// 16-bit caches take the tensor-core rows kernel unless attn_force_path pins
+// the CUDA-core one (tests compare the two on the same inputs).
 bool use_rows_mma(int32_t kv_dtype) {
   if (kv_dtype != KCA_F16 && kv_dtype != KCA_BF16) return false;
-  const char* env = std::getenv("KCA_DECODE_PATH");
-  return !(env != nullptr && std::strcmp(env, "simt") == 0);
+  return g_rows_path.load(std::memory_order_relaxed) != 0;
 }
 
 // Plan of the tensor-core rows kernel.  Each cluster size c in {8, 4, 2}
@@ -330,7 +330,7 @@ int launch_rows_path(int32_t q_dtype, int32_t kv_dtype, const void* k_cache, con
 
 // Work items of the rows path (unit u at position pos[u], nk[u] visible keys
 // from lo(pos[u])), as the calls run them: the CUDA-core kernel's plan for
-// num_sms SMs, or -- for 16-bit caches, unless KCA_DECODE_PATH forces the
+// num_sms SMs, or -- for 16-bit caches, unless attn_force_path pins the
 // CUDA-core kernel -- the tensor-core kernel's cluster plan on the current
 // device (its clusters must fit the device's resident capacity, so that form
 // needs a device).  slot: the split's partial slot (CUDA core), or the
@@ -372,6 +372,14 @@ int rows_plan_items(int32_t kv_dtype, int32_t n, const int64_t* pos, const int64
 }  // namespace
 
 extern "C" {
+
+int attn_force_path(int32_t op, int32_t path) {
+  if (path < -1 || path > 1) return KCA_ERR_RANGE;
+  if (op == 0) g_prefill_path.store(path);
+  else if (op == 1) g_rows_path.store(path);
+  else return KCA_ERR_RANGE;
+  return KCA_OK;
+}
 
 const char* attn_status_string(int status) {
   switch (status) {

@@ -12,8 +12,9 @@
 // The array below is created when the module loads on a device and is held
 // by every GPU that loads the library until the process exits.  Its device
 // address is looked up once per device (cudaGetSymbolAddress) on the first
-// call made with that device current; make that first call before any stream
-// capture.  All calls on a device share the array, so calls whose execution
+// call made with that device current -- and again if the device's context
+// was created anew since (cudaDeviceReset reloads the module, possibly at
+// another address); make that first call before any stream capture.  All calls on a device share the array, so calls whose execution
 // can overlap on the GPU (different streams, or graphs replayed
 // concurrently) race on it and must be serialised by the caller.  The array
 // keeps the last call's contents.  Its first KCA_WORKSPACE_HEADER bytes must
@@ -22,9 +23,14 @@
 // them at zero, but one that recorded a device error may not), so every call
 // clears them first with cudaMemsetAsync on its stream -- a memset, not an
 // allocation.  Everything past the header is written before it is read
-// within the same call.
-#include <atomic>
+// within the same call.  Because of that clear, a call's device status (a
+// bounded wait that ran out) survives only until the next call: read it in
+// between with attn_device_status on the address that
+// attn_decode_static_scratch returns.
+#include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "../../include/kca.h"
 #include "kca_plan.h"
@@ -34,25 +40,56 @@ namespace {
 
 static __device__ __align__(256) unsigned char kca_static_scratch[KCA_STATIC_SCRATCH_BYTES];
 
-// Device address of kca_static_scratch per device; the name itself is only a
-// host-side stand-in and must never be handed to a kernel.
+// The current driver context, through the runtime's driver entry point (no
+// link-time dependency on libcuda); nullptr when it cannot be read.
+CUcontext current_context() {
+  using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+  static const CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return nullptr;
+  }();
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of kca_static_scratch on the current device; the name itself
+// is only a host-side stand-in and must never be handed to a kernel.  Looked
+// up once per device and context: a context torn down and created again
+// (cudaDeviceReset) loads the module anew, possibly at another address, so
+// the cached address is kept together with the context it belongs to.
 void* scratch_address(int* status) {
-  static std::atomic<void*> addr[64];   // zero-initialised
+  struct Entry {
+    CUcontext ctx;
+    void* addr;
+  };
+  static Entry cache[64];   // zero-initialised; guarded by mu
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     *status = KCA_ERR_CUDA;
     return nullptr;
   }
-  if (addr[dev] == nullptr) {
+  // cudaGetSymbolAddress makes the device's primary context current if no
+  // context is, so the context is read after it on a first call.
+  const CUcontext ctx = current_context();
+  std::lock_guard<std::mutex> lock(mu);
+  Entry& e = cache[dev];
+  if (e.addr == nullptr || ctx == nullptr || e.ctx != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, kca_static_scratch) != cudaSuccess || p == nullptr) {
       *status = KCA_ERR_CUDA;
       return nullptr;
     }
-    addr[dev] = p;
+    e.addr = p;
+    e.ctx = ctx != nullptr ? ctx : current_context();
   }
   *status = KCA_OK;
-  return addr[dev];
+  return e.addr;
 }
 
 }  // namespace
@@ -74,4 +111,14 @@ extern "C" int attn_decode_static(const void* q, int32_t q_dtype, const void* k_
   // kernel is launched.  A call that fails validation touches nothing.
   return kca::decode_entry(q, q_dtype, k_cache, v_cache, kv_dtype, n_q_heads, n_kv_heads, head_dim, capacity,
                            batch, ctx_len, window, scale, out, ws, KCA_STATIC_SCRATCH_BYTES, stream, true);
+}
+
+extern "C" int attn_decode_static_scratch(void** device_ptr, size_t* bytes) {
+  if (device_ptr == nullptr) return KCA_ERR_NULL;
+  int st = KCA_OK;
+  void* p = scratch_address(&st);
+  if (p == nullptr) return st;
+  *device_ptr = p;
+  if (bytes != nullptr) *bytes = KCA_STATIC_SCRATCH_BYTES;
+  return KCA_OK;
 }

@@ -30,6 +30,42 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, n), n
 
 
+def test_every_declared_call_cites_its_passage():
+    """Each declaration in kca.h sits under a comment that names the passage
+    of the pages it answers to (or says that the pages have none)."""
+    text = open(HEADER).read()
+    blocks = [(m.start(), m.end(), m.group(0)) for m in re.finditer(r"/\*.*?\*/", text, flags=re.S)]
+    code = re.sub(r"/\*.*?\*/", lambda m: " " * len(m.group(0)), text, flags=re.S)
+    seen = set()
+    for m in re.finditer(r"\b(attn_\w+)\s*\(", code):
+        name = m.group(1)
+        if name in seen:
+            continue
+        seen.add(name)
+        before = [b for b in blocks if b[1] <= m.start()]
+        assert before, name
+        comment = before[-1][2]
+        assert "Passage:" in comment or "no counterpart" in comment, name
+    assert len(seen) == len(_declared())
+
+
+def test_force_path_validates_and_restores():
+    lib = kca.lib()
+    assert lib.attn_force_path(2, 0) == -4 and lib.attn_force_path(0, 2) == -4
+    assert lib.attn_force_path(-1, 0) == -4 and lib.attn_force_path(1, -2) == -4
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 0, 768) == 1
+    with kca.forced_path(kca.OP_PREFILL, kca.PATH_ROWS):
+        assert kca.attn_prefill_path(kca.BF16, kca.BF16, 0, 768) == 0
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 0, 768) == 1
+    with kca.forced_path(kca.OP_PREFILL, kca.PATH_TENSOR_CORE):   # where eligible only
+        assert kca.attn_prefill_path(kca.BF16, kca.BF16, 1000, 2) == 1
+        assert kca.attn_prefill_path(kca.F32, kca.F32, 0, 768) == 0
+
+
+def test_static_scratch_query_rejects_a_null_pointer():
+    assert kca.lib().attn_decode_static_scratch(None, None) == -1
+
+
 def test_header_constants_match_binding():
     text = open(HEADER).read()
     for name, val in [("KCA_MAX_CHUNK_ROWS", 768), ("KCA_MAX_POSITION", 131072),
@@ -226,7 +262,7 @@ def _check_rows_plan(items, units, pos_of, window):
 @pytest.mark.parametrize("cs,rows,window", [(0, 48, 0), (256, 48, 0), (1000, 15, 0), (5, 9, 3),
                                             (4090, 7, 512), (130000, 1, 0), (0, 1, 1)])
 def test_prefill_rows_plan_covers_visible_keys(cs, rows, window):
-    path, items = kca.attn_prefill_plan(kca.F32, kca.F32, cs, rows, window)
+    path, items = kca.attn_prefill_plan(kca.F32, kca.F32, cs, rows, window, num_sms=148)
     assert path == 0
     _check_rows_plan(items, rows, lambda u: cs + u, window)
 
@@ -253,7 +289,7 @@ def test_decode_plan_fills_one_wave():
                                             (1000, 17, 0), (7, 16, 5), (100, 200, 64),
                                             (2000, 768, 1)])
 def test_prefill_tc_plan_covers_every_visible_key(cs, rows, window):
-    path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, rows, window)
+    path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, rows, window, num_sms=148)
     assert path == 1
     assert len(items) <= 148
     kv_lo = oracle.visible_range(cs, window)[0]

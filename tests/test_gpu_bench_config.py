@@ -4,7 +4,10 @@ shared by all 64 decode calls), its prefill and decode captured as CUDA
 graphs exactly as the timed region replays them, checked against the f64
 oracle on the same seeded inputs -- every row of chunks 0, 10 and 21 plus
 1,024 seeded random rows of the prompt, and every one of the 64 decode
-steps."""
+steps -- and the bench's other configurations the same way: the decode
+steps at 256 and 4,096 keys (every step), the window-512 prompt (every
+row) and its 64 decode steps, and the 768-row chunk at the end of the
+131,072-row cache (80 rows)."""
 import os
 import sys
 
@@ -63,3 +66,80 @@ def test_bench_decode_graph_matches_oracle_on_every_step(bench_run):
     for t, c in enumerate(w.dec_ctx):
         want = oracle_decode(x["qd"][t:t + 1], x["kd"][None], x["vd"][None], [c], 0, "f32", "f16", w.cap)
         assert max_err(got[t], want) <= 4e-3, t
+
+
+@pytest.fixture(scope="module")
+def other_parts(cuda_ok):
+    """The bench's other configurations (decode at 256 and 4096, the window
+    configuration, the long chunk), each captured as the CUDA graph the timed
+    region replays, replayed once over NaN-filled outputs."""
+    oracle_threads()
+    sys.path.insert(0, ROOT)
+    import bench
+    dev = torch.device("cuda", 0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    win = bench.WindowParts(dev, sms)
+    parts = [bench.DecodeLenPart(dev, 256), bench.DecodeLenPart(dev, 4096)] + win.parts + \
+        [bench.LongChunkPart(dev, sms)]
+    for p in parts:
+        p.run(0)
+    torch.cuda.synchronize()
+    graphs = []
+    for p in parts:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            p.run(0)
+        graphs.append(g)
+    for o in (parts[0].out, parts[1].out, win.out, win.dout, parts[-1].out):
+        o.fill_(float("nan"))
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    for p in parts:
+        for ws in p.workspaces():
+            assert p.kca.attn_device_status(ws)[0] == 0, p.name
+    return bench, parts, win
+
+
+def test_bench_small_decodes_match_oracle_on_every_step(other_parts):
+    from kv_cache_attention_states_b200 import synth
+    bench, parts, _ = other_parts
+    for p in parts[:2]:
+        wl = synth.decode_f16(p.ctx[0], bench.DECODE_STEPS)
+        k = synth.draw(0, "k", (1, wl.capacity, 256), "f16")
+        v = synth.draw(0, "v", (1, wl.capacity, 256), "f16")
+        q = synth.draw(0, "q", (bench.DECODE_STEPS, 1, 8, 256), "f32")
+        got = p.out.cpu().numpy()
+        for t, c in enumerate(p.ctx):
+            want = oracle_decode(q[t], k, v, [c], 0, "f32", "f16", wl.capacity)
+            assert max_err(got[t], want) <= 4e-3, (p.name, t)
+
+
+def test_bench_window_configuration_matches_oracle(other_parts):
+    from kv_cache_attention_states_b200 import synth
+    bench, _, win = other_parts
+    wl = win.wl
+    k = synth.draw(0, "k", (wl.capacity, 256), "bf16")
+    v = synth.draw(0, "v", (wl.capacity, 256), "bf16")
+    q = synth.draw(0, "q", (4096, 8, 256), "bf16")
+    qd = synth.draw(0, "qd", (bench.DECODE_STEPS, 1, 8, 256), "bf16")
+    want = oracle_prefill(q, k, v, 0, np.arange(4096), wl.window, "bf16", "bf16")
+    assert max_err(win.out.cpu().numpy(), want) <= 4e-3
+    got = win.dout.cpu().numpy()
+    for t, c in enumerate(wl.decode_ctx):
+        want = oracle_decode(qd[t], k[None], v[None], c, wl.window, "bf16", "bf16", wl.capacity)
+        assert max_err(got[t], want) <= 4e-3, t
+
+
+def test_bench_long_chunk_matches_oracle(other_parts):
+    from kv_cache_attention_states_b200 import synth
+    _, parts, _ = other_parts
+    p = parts[-1]
+    wl = synth.long_chunk_bf16()
+    k = synth.draw(0, "k", (wl.capacity, 256), "bf16")
+    v = synth.draw(0, "v", (wl.capacity, 256), "bf16")
+    q = synth.draw(0, "q", (p.rows, 8, 256), "bf16")
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([np.arange(0, 16), np.arange(752, 768), rng.integers(0, 768, 48)]))
+    want = oracle_prefill(q, k, v, p.cs, rows, 0, "bf16", "bf16")
+    assert max_err(p.out.cpu().numpy()[rows], want) <= 4e-3

@@ -190,3 +190,46 @@ def test_calls_capture_into_a_cuda_graph_and_replay_bitwise():
     torch.cuda.synchronize()
     assert torch.equal(out, eager_p) and torch.equal(outd, eager_d)
     del g
+
+
+@pytest.mark.parametrize("cs,rows,window,j", [(1000, 400, 0, 350), (1000, 400, 128, 100), (64, 768, 0, 500)])
+def test_nan_in_a_value_row_on_the_tensor_core_path(cs, rows, window, j):
+    """A NaN in V at chunk row j (position p = cs + j) -- outside what the
+    tensor-core path accepts (kca.h PRECONDITIONS: V finite on a chunk's
+    visible union) -- poisons exactly the 16-row tiles whose work items
+    cover p (0 x NaN in the PV product of a masked key): every row of those
+    tiles is NaN, every other row is finite and equals the oracle's value.
+    The rows path, on the same inputs, poisons exactly the rows that see p,
+    as the definition does."""
+    from tests.helpers import max_err, oracle_prefill, oracle_threads
+    oracle_threads()
+    dtype = "bf16"
+    q, k, v = _data(dtype, cs + rows, rows, seed=17)
+    p = cs + j
+    v[p, :] = NAN16[dtype]
+    path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, rows, window)
+    assert path == 1
+    n_tiles = (rows + 15) // 16
+    hit = np.zeros(n_tiles, dtype=bool)
+    for tile, kb, ke, _ in items:
+        if kb <= p < ke:
+            hit[tile] = True
+    tile_of_row = np.arange(rows) // 16
+    poisoned = hit[tile_of_row]
+    pos = cs + np.arange(rows)
+    lo = np.maximum(0, pos - window + 1) if window > 0 else np.zeros(rows, dtype=np.int64)
+    sees = (lo <= p) & (p <= pos)
+    assert sees.any() and (~poisoned).any()
+    assert not (sees & ~poisoned).any()          # every row that sees p lies in a poisoned tile
+    args = (dev(q, dtype), dev(k, dtype), dev(v, dtype), cs, window)
+    tc = kca.attn_prefill(*args).cpu().numpy()
+    want = oracle_prefill(q, k, v, cs, np.arange(rows), window, dtype, dtype)
+    assert np.isnan(want[sees]).all() and np.isfinite(want[~sees]).all()
+    assert np.isnan(tc[poisoned]).all()
+    assert np.isfinite(tc[~poisoned]).all()
+    assert max_err(tc[~poisoned], want[~poisoned]) <= 4e-3
+    with kca.forced_path(kca.OP_PREFILL, kca.PATH_ROWS):
+        rw = kca.attn_prefill(*args).cpu().numpy()
+    assert np.isnan(rw[sees]).all()
+    assert np.isfinite(rw[~sees]).all()
+    assert max_err(rw[~sees], want[~sees]) <= 4e-3

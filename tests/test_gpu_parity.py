@@ -133,14 +133,14 @@ def test_few_row_chunk_on_long_context_takes_tc_path(rows):
     _check_status(ws)
 
 
-def test_rows_and_tc_paths_agree(monkeypatch):
+def test_rows_and_tc_paths_agree():
     cs, rows = 640, 128
     k, v = _cache(5, cs + rows, cs + rows, "bf16")
     q = synth.draw(5, "q", (rows, 8, 256), "bf16")
     args = (dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), cs)
     tc = kca.attn_prefill(*args).cpu().numpy()
-    monkeypatch.setenv("KCA_PREFILL_PATH", "rows")
-    rw = kca.attn_prefill(*args).cpu().numpy()
+    with kca.forced_path(kca.OP_PREFILL, kca.PATH_ROWS):
+        rw = kca.attn_prefill(*args).cpu().numpy()
     want = oracle_prefill(q, k, v, cs, np.arange(rows), 0, "bf16", "bf16")
     assert max_err(tc, want) <= 4e-3 and max_err(rw, want) <= 4e-3
 
@@ -217,15 +217,15 @@ def test_long_chunk_at_capacity_end_every_row():
 
 
 @pytest.mark.parametrize("q_dtype,kv_dtype", [("f32", "f16"), ("bf16", "bf16"), ("f32", "bf16")])
-def test_decode_tensor_core_and_cuda_core_paths_agree(monkeypatch, q_dtype, kv_dtype):
+def test_decode_tensor_core_and_cuda_core_paths_agree(q_dtype, kv_dtype):
     cap = 20000
     ctx = [19999, 1, 63, 64, 65, 777, 12000]
     k, v = _cache(6, cap, [cap] * len(ctx), kv_dtype, batch=len(ctx))
     q = synth.draw(6, "q", (len(ctx), 8, 256), q_dtype)
     args = (dev(q, q_dtype), dev(k, kv_dtype), dev(v, kv_dtype), ctx)
     mma = kca.attn_decode(*args).cpu().numpy()
-    monkeypatch.setenv("KCA_DECODE_PATH", "simt")
-    simt = kca.attn_decode(*args).cpu().numpy()
+    with kca.forced_path(kca.OP_ROWS, kca.PATH_CUDA_CORE):
+        simt = kca.attn_decode(*args).cpu().numpy()
     want = oracle_decode(q, k, v, ctx, 0, q_dtype, kv_dtype, cap)
     assert max_err(mma, want) <= 4e-3 and max_err(simt, want) <= 4e-3
 
@@ -251,3 +251,35 @@ def test_decode_at_the_maximum_batch(q_dtype, kv_dtype):
     with pytest.raises(kca.KcaError):
         kca.attn_decode(qx, kx, kx.clone(), [1] * one_more)
 
+
+
+# ------------------------------------------- f32 (CUDA-core kernel) at size
+
+@pytest.mark.parametrize("window", [0, 512])
+def test_f32_prefill_chunk_of_768_rows_at_8192(window):
+    """The CUDA-core rows kernel (f32 Q/K/V) on a full 768-row chunk at
+    positions 8192..8959, every row against the oracle at the f32 bar."""
+    cs, rows = 8192, 768
+    k, v = _cache(31, cs + rows, cs + rows, "f32")
+    q = synth.draw(31, "q", (rows, 8, 256), "f32")
+    assert kca.attn_prefill_path(kca.F32, kca.F32, cs, rows, window) == 0
+    ws = kca.new_workspace(kca.attn_prefill_workspace_bytes(kca.F32, kca.F32, cs, rows, window))
+    out = kca.attn_prefill(dev(q, "f32"), dev(k, "f32"), dev(v, "f32"), cs, window, workspace=ws)
+    want = oracle_prefill(q, k, v, cs, np.arange(rows), window, "f32", "f32")
+    assert max_err(out.cpu().numpy(), want) <= 2e-6
+    _check_status(ws)
+
+
+def test_f32_decode_at_16k_and_64k_keys():
+    """The CUDA-core rows kernel and its split merge on f32 caches: a batch
+    with contexts of 16,384 and 65,536 keys (and a short one), every row
+    against the oracle at the f32 bar."""
+    cap = 65536
+    ctx = [16384, 65536, 1000]
+    k, v = _cache(32, cap, ctx, "f32", batch=len(ctx))
+    q = synth.draw(32, "q", (len(ctx), 8, 256), "f32")
+    ws = kca.new_workspace(kca.attn_decode_workspace_bytes(ctx))
+    out = kca.attn_decode(dev(q, "f32"), dev(k, "f32"), dev(v, "f32"), ctx, workspace=ws)
+    want = oracle_decode(q, k, v, ctx, 0, "f32", "f32", cap)
+    assert max_err(out.cpu().numpy(), want) <= 2e-6
+    _check_status(ws)

@@ -8,8 +8,11 @@ to.  attn_decode_static takes that scratch from a fixed device array inside
 the library instead.  These tests call it through the C ABI (ctypes, raw
 pointers) and check it against attn_decode on the same inputs, three times
 in a row with different shapes so that the array's leftover contents from
-one call cannot leak into the next.  This file is collected last, and
-it also passes on its own in a fresh process.
+one call cannot leak into the next, and once after the array's header (the
+status word and the merge counters) was filled with garbage, which the
+call must clear before its kernel runs.  The status of each call is read
+back through the array's address (attn_decode_static_scratch).  This file
+is collected last, and it also passes on its own in a fresh process.
 """
 import ctypes
 
@@ -34,6 +37,31 @@ def _static_call(q, k, v, ctx, window, out):
         window, 1.0 / 16.0, vp(out.data_ptr()), vp(torch.cuda.current_stream().cuda_stream))
 
 
+def _scratch():
+    ptr = ctypes.c_void_p(0)
+    size = ctypes.c_size_t(0)
+    assert kca.lib().attn_decode_static_scratch(ctypes.byref(ptr), ctypes.byref(size)) == 0
+    assert ptr.value and ptr.value % 256 == 0 and size.value == STATIC_BYTES
+    return ptr.value
+
+
+def _static_status():
+    detail = ctypes.c_uint32(0)
+    st = kca.lib().attn_device_status(ctypes.c_void_p(_scratch()),
+                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream),
+                                      ctypes.byref(detail))
+    return st, detail.value
+
+
+class _DeviceBytes:
+    """A torch view of n bytes of device memory at a raw address (CUDA array
+    interface); used to scribble over the array's header."""
+
+    def __init__(self, ptr, n):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "|u1", "data": (ptr, False),
+                                         "version": 3, "strides": None}
+
+
 def _inputs(seed, batch, cap, q_dtype, kv_dtype):
     k = synth.as_torch(synth.draw(seed, "k", (batch, cap, 256), kv_dtype), kv_dtype).cuda()
     v = synth.as_torch(synth.draw(seed, "v", (batch, cap, 256), kv_dtype), kv_dtype).cuda()
@@ -41,7 +69,7 @@ def _inputs(seed, batch, cap, q_dtype, kv_dtype):
     return q, k, v
 
 
-def test_static_scratch_decode_matches_attn_decode_twice(cuda_ok):
+def test_static_scratch_decode_matches_attn_decode_three_times(cuda_ok):
     cases = [
         (1, 16448, [16384], 0, "f32", "f16"),               # one long sequence: 100+ splits
         (4, 9000, [8999, 1, 4500, 7777], 300, "bf16", "bf16"),  # ragged batch with a window
@@ -57,6 +85,25 @@ def test_static_scratch_decode_matches_attn_decode_twice(cuda_ok):
         tol = 2e-6 if (qd, kd) == ("f32", "f32") else 4e-3
         assert err <= tol, (i, err)
         assert torch.isfinite(got).all()
+        assert _static_status() == (0, 0), i
+
+
+def test_static_scratch_decode_clears_a_garbage_header(cuda_ok):
+    # Nonzero status word and merge counters left by an imagined failed
+    # call: the next call clears them before its kernel runs, so its output
+    # and status are those of a clean start.
+    header = kca.WORKSPACE_HEADER
+    view = torch.as_tensor(_DeviceBytes(_scratch(), header), device="cuda")
+    q, k, v = _inputs(20, 1, 16448, "f32", "f16")
+    want = kca.attn_decode(q, k, v, [16384])
+    for fill in (0xFF, 0x01):
+        view.fill_(fill)
+        torch.cuda.synchronize()
+        got = torch.full((1, 8, 256), float("nan"), dtype=torch.float32, device="cuda")
+        assert _static_call(q, k, v, [16384], 0, got) == 0
+        torch.cuda.synchronize()
+        assert (got - want).abs().max().item() <= 4e-3, fill
+        assert _static_status() == (0, 0), fill
 
 
 def test_static_scratch_rejects_plans_beyond_its_size(cuda_ok):
