@@ -16,6 +16,8 @@ set follows a large one, so that its calls read cold rows from HBM):
                  decode steps at positions 4096..4159, bf16 Q/K/V ~ N(0,1)
   long_chunk     one 768-row bf16 chunk at positions 130304..131071 of a
                  131,072-row cache
+  prefill_batch  32 sequences x 4 query rows (speculative / multi-row decode)
+                 per call through attn_prefill_batch, 16 calls, f16 K/V
 
 value = prefill q-rows/s (a q-row is one query position with all 8 heads),
 from CUDA events around the prefill graph of every pass; every other
@@ -47,7 +49,7 @@ DECODE_STEPS = 64
 DECODE_REPLICAS = 32
 PREFILL_REPLICAS = 2
 SMALL_DECODE_REPLICAS = 64
-PASSES = 8               # passes over every configuration per step
+PASSES = 10              # passes over every configuration per step
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels, with the launch they come from; None once a kernel has changed
 # since its capture.
@@ -480,11 +482,73 @@ class RaggedPart(Part):
         return [self.ws]
 
 
-def build_parts(w, device, sms):
-    """The parts of one pass, in pass order (see the module docstring)."""
-    win = WindowParts(device, sms)
-    parts = [RaggedPart(device), DecodeLenPart(device, 256), DecodeLenPart(device, 4096),
-             PrefillPart(w, sms), HeadlineDecodePart(w)] + win.parts + [LongChunkPart(device, sms)]
+class BatchRowsPart(Part):
+    """Batched short chunks (speculative or multi-row decode): 32 sequences
+    with contexts drawn by the seed from [1024, 16384], 4 query rows each,
+    16 calls (each advancing every sequence by 4 rows), f16 K/V, f32 q,
+    through attn_prefill_batch."""
+    name, unit, bound = "prefill_batch", "q-rows", "hbm"
+    kernel = "decode_mma_kernel<f32 q, f16 KV> (4 rows per sequence)"
+    BATCH, ROWS, CALLS, CAP = 32, 4, 16, 16448
+
+    def __init__(self, device, seed=0):
+        import torch
+        import kv_cache_attention_states_b200 as kca
+        from kv_cache_attention_states_b200 import synth
+        self.kca = kca
+        ctx0 = synth.integers(seed, "batch_ctx", 1024, 16384, self.BATCH)
+        self.ctx = [[int(c) + self.ROWS * t for c in ctx0] for t in range(self.CALLS)]
+        g = torch.Generator(device=device)
+        g.manual_seed(2)
+        self.k = torch.randn((self.BATCH, self.CAP, 256), generator=g, device=device).half()
+        self.v = torch.randn((self.BATCH, self.CAP, 256), generator=g, device=device).half()
+        self.q = torch.randn((self.CALLS, self.BATCH, self.ROWS, 8, 256), generator=g, device=device)
+        self.out = torch.empty_like(self.q)
+        self.ws = kca.new_workspace(max(kca.attn_prefill_batch_workspace_bytes(c, self.ROWS) for c in self.ctx),
+                                    device)
+        self.units = self.BATCH * self.ROWS * self.CALLS
+        # algorithmic bytes: each sequence's visible K/V rows once per call
+        # (its rows share them), q and the f32 output
+        self.work = float(sum(sum(c) * 1024 + self.BATCH * self.ROWS * 8 * 256 * 8 for c in self.ctx))
+        self.launches = self.CALLS
+        self.algorithmic = "ctx*1024 B K/V per sequence (shared by its 4 rows) + 16 KiB q/out per row"
+        self.workload = ("32 sequences x 4 query rows at ctx drawn by the seed from [1024, 16384], 16 calls, "
+                         "f16 K/V, f32 q (attn_prefill_batch)")
+
+    def run(self, variant):
+        for t, c in enumerate(self.ctx):
+            self.kca.attn_prefill_batch(self.q[t], self.k, self.v, c, out=self.out[t], workspace=self.ws)
+
+    def workspaces(self):
+        return [self.ws]
+
+
+PART_NAMES = ["decode_ragged", "decode_256", "decode_4096", "prefill", "decode", "window_prefill",
+              "window_decode", "long_chunk", "prefill_batch"]
+
+
+def build_parts(w, device, sms, only=None):
+    """The parts of one pass, in pass order (see the module docstring); with
+    `only`, just that one (for profiling a single configuration)."""
+    def want(*names):
+        return only is None or only in names
+    parts = []
+    if want("decode_ragged"):
+        parts.append(RaggedPart(device))
+    if want("decode_256"):
+        parts.append(DecodeLenPart(device, 256))
+    if want("decode_4096"):
+        parts.append(DecodeLenPart(device, 4096))
+    if want("prefill"):
+        parts.append(PrefillPart(w, sms))
+    if want("decode"):
+        parts.append(HeadlineDecodePart(w))
+    if want("window_prefill", "window_decode"):
+        parts += [p for p in WindowParts(device, sms).parts if want(p.name)]
+    if want("long_chunk"):
+        parts.append(LongChunkPart(device, sms))
+    if want("prefill_batch"):
+        parts.append(BatchRowsPart(device))
     return parts
 
 
@@ -494,8 +558,8 @@ def run_cuda(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    w = Workload(dev)
-    parts = build_parts(w, dev, sms)
+    w = Workload(dev) if args.only in (None, "prefill", "decode") else None
+    parts = build_parts(w, dev, sms, args.only)
     stream = torch.cuda.current_stream()
     passes = max(1, args.passes)
     # warm-up: eager calls first (tensor-map caches, function attributes)
@@ -558,9 +622,10 @@ def run_cuda(args, rank, world, local_rank):
     part_ms = [sum(a.elapsed_time(b) for a, b in ev[nm]) for nm in names]
     vals = max_over_ranks([total_ms] + part_ms, world, dev)
     total_ms, part_ms = vals[0], dict(zip(names, vals[1:]))
+    import kv_cache_attention_states_b200 as kca
     for p in parts:
         for ws in p.workspaces():
-            st, detail = w.kca.attn_device_status(ws)
+            st, detail = kca.attn_device_status(ws)
             if st != 0:
                 raise RuntimeError(f"{p.name}: device status {st} detail {detail:#x}")
     res = dict(total_ms=total_ms, part_ms=part_ms, runs=n_runs, clocks=clk, passes=passes,
@@ -568,6 +633,8 @@ def run_cuda(args, rank, world, local_rank):
                parts={p.name: p for p in parts})
     if graphs is not None:
         del graphs
+    if args.only is not None:
+        return res
     e2e = run_e2e(w, args, stream)
     e2e["pre_ms"], e2e["dec_ms"] = max_over_ranks([e2e["pre_ms"], e2e["dec_ms"]], world, dev)
     res["e2e"] = e2e
@@ -770,6 +837,16 @@ def oracle_part_samples(seed=0):
     base = np.array([0, ctx[0]])
     sec = _timed(lambda: oracle.attention(q, k, v, np.array(ctx) - 1, base, kv_dtype="f16", scale=synth.SCALE))
     out["decode_ragged"] = (2 / sec, f"sequences 0-1 of the first step (ctx {ctx[0]}, {ctx[1]}; {sec:.2f} s)")
+    ctx0 = synth.integers(seed, "batch_ctx", 1024, 16384, 32)[:4]
+    rows = 4
+    k = np.concatenate([synth.draw(seed, f"bk{b}", (int(c), 256), "f16") for b, c in enumerate(ctx0)])
+    v = np.concatenate([synth.draw(seed, f"bv{b}", (int(c), 256), "f16") for b, c in enumerate(ctx0)])
+    q = synth.draw(seed, "bq", (4 * rows, 8, 256), "f32")
+    starts = np.concatenate([[0], np.cumsum(ctx0)[:-1]])
+    pos = np.array([int(c) - rows + i for c in ctx0 for i in range(rows)])
+    base = np.repeat(starts, rows)
+    sec = _timed(lambda: oracle.attention(q, k, v, pos, base, kv_dtype="f16", scale=synth.SCALE))
+    out["prefill_batch"] = (pos.size / sec, f"sequences 0-3 of the first call, 4 rows each ({sec:.2f} s)")
     return out, cores
 
 
@@ -842,6 +919,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every call from Python instead of "
                     "replaying captured CUDA graphs")
+    ap.add_argument("--only", choices=PART_NAMES, default=None,
+                    help="time one configuration alone (profiling); prints that part's object only")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -857,13 +936,24 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     res = run_cuda(args, rank, world, local_rank)
+    if args.only is not None:
+        if rank == 0:
+            hbm, tflops, tflops_sus, src = _peaks()
+            p = res["parts"][args.only]
+            print(json.dumps({"only": args.only, "steps": args.steps, "passes": res["passes"],
+                              **part_object(p, res["part_ms"][args.only], res["runs"], world, hbm, tflops,
+                                            tflops_sus, src)}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     cpu = parts_cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows_s, tok_s, cores, desc = oracle_sample(768, 4)
         cpu = {"value": rows_s, "unit": "q-rows/s", "cores": cores, "kind": "oracle", "sample": desc,
                "decode_tok_s": tok_s}
         samples, cores = oracle_part_samples()
-        parts_cpu = {nm: {"value": v, "unit": ("q-rows/s" if nm in ("window_prefill", "long_chunk") else "tok/s"),
+        parts_cpu = {nm: {"value": v, "unit": ("q-rows/s" if nm in ("window_prefill", "long_chunk", "prefill_batch")
+                                                   else "tok/s"),
                           "cores": cores, "kind": "oracle", "sample": d + "; f64 C oracle, OpenMP over (row, head)"}
                      for nm, (v, d) in samples.items()}
         parts_cpu["decode"] = {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
@@ -892,7 +982,7 @@ def main():
                                "1 KV head, head_dim 256, causal",
                    "seq_len": 16384, "global_batch": world, "parallelism": f"replicas x{world}",
                    "step": f"{res['passes']} passes; a pass runs every configuration once (ragged, "
-                           "decode_256, decode_4096, prefill, decode, window, long_chunk)",
+                           "decode_256, decode_4096, prefill, decode, window, long_chunk, prefill_batch)",
                    "value": "prefill part of every pass (CUDA events); the other configurations in "
                             "their own objects",
                    "launch": "eager" if args.eager else "one CUDA graph per configuration of the C-ABI calls",
@@ -909,6 +999,7 @@ def main():
                    "prefill": obj("window_prefill"), "decode": obj("window_decode")},
         "long_chunk": obj("long_chunk"),
         "decode_ragged": obj("decode_ragged"),
+        "prefill_batch": obj("prefill_batch"),
         "e2e": {"value": world * PREFILL_ROWS * e2e["steps"] / (e2e["pre_ms"] / 1e3), "unit": "q-rows/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "decode_tok_s": world * DECODE_STEPS * e2e["steps"] / (e2e["dec_ms"] / 1e3),

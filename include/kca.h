@@ -119,6 +119,7 @@ extern "C" {
 #define KCA_MAX_CHUNK_ROWS 768
 #define KCA_MAX_POSITION 131072
 #define KCA_MAX_BATCH 256
+#define KCA_MAX_BATCH_ROWS 15   /* rows per sequence of attn_prefill_batch */
 /* status word (256 B) + 768 rows x 8 heads x 4-byte counters */
 #define KCA_WORKSPACE_HEADER 24832
 
@@ -170,6 +171,35 @@ int attn_decode(const void *q, int32_t q_dtype,
                 int32_t batch, const int64_t *ctx_len, int32_t window,
                 float scale, float *out, void *workspace, size_t workspace_bytes,
                 void *stream);
+
+/*
+ * attn_prefill_batch -- short chunks of several sequences in one call: each
+ * sequence b has `rows` query rows, at positions ctx_len[b] - rows ..
+ * ctx_len[b] - 1 (speculative or multi-row decode steps), every row seeing
+ * its sequence's keys as in attn_prefill.  One launch (plus the split merge
+ * on f32 caches) serves all batch x rows rows: each row is a unit of the
+ * rows path (decode's kernels), its keys cut into splits across the GPU.
+ * Passage: Karume v0.12.0 release notes, "Docs", ADR 0067 plan-size geometry
+ * table (the 2-15-row plans between decode and the >= 16-row tiles), and
+ * "Performance", item 3 (the parallel PV reduction serves plans under 16
+ * rows).
+ *   q            [batch][rows][8][256] q_dtype, device
+ *   k_cache/v_cache  [batch][capacity][1][256] kv_dtype, device; each
+ *                sequence's rows up to ctx_len[b] - 1 written
+ *   batch        1..256;  rows 1..KCA_MAX_BATCH_ROWS
+ *   ctx_len      HOST array [batch], rows..capacity
+ *   window, scale  as in attn_prefill
+ *   out          [batch][rows][8][256] float32, device
+ *   workspace    >= attn_prefill_batch_workspace_bytes(batch, rows, ctx_len, window)
+ * With rows = 1 this is attn_decode (the same plan and the same bits).
+ * Returns KCA_OK or a negative KCA_ERR_* (nothing launched on error).
+ */
+int attn_prefill_batch(const void *q, int32_t q_dtype,
+                       const void *k_cache, const void *v_cache, int32_t kv_dtype,
+                       int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity,
+                       int32_t batch, int32_t rows, const int64_t *ctx_len, int32_t window,
+                       float scale, float *out, void *workspace, size_t workspace_bytes,
+                       void *stream);
 
 /*
  * attn_decode_dev -- attn_decode with the context lengths in DEVICE memory,
@@ -328,6 +358,8 @@ int attn_merge_partials(int32_t n_parts, int32_t batch, const float *parts, int6
 size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
                                     int32_t chunk_rows, int32_t window);
 size_t attn_decode_workspace_bytes(int32_t batch, const int64_t *ctx_len, int32_t window);
+size_t attn_prefill_batch_workspace_bytes(int32_t batch, int32_t rows, const int64_t *ctx_len,
+                                          int32_t window);
 size_t attn_decode_partial_workspace_bytes(int32_t batch, const int64_t *ctx_len, int64_t key_begin,
                                            int64_t capacity, int32_t window);
 
@@ -362,26 +394,51 @@ int attn_device_status(void *workspace, void *stream, uint32_t *detail);
  *     split;
  *   rows path (decode, and prefill of short or mixed-dtype chunks): one item
  *     per split, unit = query row (prefill) or sequence (decode),
- *     [key_begin, key_end) within J(pos).  With an f32 cache (or
- *     KCA_DECODE_PATH=simt) this is the CUDA-core kernel's plan for num_sms
- *     SMs, host only, and slot = the split's partial slot or -1 when the unit
- *     has one split.  With a 16-bit cache it is the tensor-core kernel's
- *     plan, whose splits run as clusters that must fit the resident-cluster
- *     capacity of the CURRENT DEVICE (num_sms is not used; KCA_ERR_CUDA
- *     without a device), and slot = the cluster partial that the split's
- *     cluster writes (sequence * clusters-per-sequence + split / cluster
- *     size), or -1 when the unit is one cluster and merges in shared memory.
+ *     [key_begin, key_end) within J(pos).  With an f32 cache (or the
+ *     CUDA-core kernel pinned by attn_force_path) this is the CUDA-core
+ *     kernel's plan for num_sms SMs, host only, and slot = the split's partial
+ *     slot or -1 when the unit has one split.  With a 16-bit cache it is the
+ *     tensor-core kernel's plan, whose splits run as clusters of 2, 4 or 8
+ *     CTAs (or of one CTA when every unit has one split) that fit the
+ *     clusters resident at once: for a device of num_sms SMs that holds
+ *     cluster_capacity[0], [1], [2] clusters of 2, 4, 8 CTAs (host only), or
+ *     with cluster_capacity NULL for the CURRENT DEVICE (num_sms is then not
+ *     used; KCA_ERR_CUDA without a device).  For each size the split length
+ *     is the smallest multiple of 64 keys whose clusters fit the capacity
+ *     (one split per unit when none does), and the size with the lowest
+ *     estimated time wins: the key stream takes the longer of all K/V bytes
+ *     at 6.5 TB/s and waves x split_len x 1 KiB at 50 GB/s per SM; a unit of
+ *     several clusters adds 1.5 us + 0.6 us x (1 + (8 / size) x
+ *     ceil(clusters / 32)); ties go to the larger size.
+ *     slot = the partial that the split's cluster writes (sequence *
+ *     clusters-per-sequence + split / cluster size), or -1 when the unit is
+ *     one cluster and merges in shared memory.  *cluster, if not NULL,
+ *     receives the cluster size (1 on the CUDA-core kernel).
  * *path receives 0 for the rows path, 1 for the tensor-core path; it is set
  * once the arguments are valid, before any device query, so it also answers
  * a call that then fails for want of a device.
  * Returns KCA_OK, or KCA_ERR_RANGE when more than max_items items exist
- * (*n_items still receives the count).
+ * (*n_items still receives the count) or a capacity is negative.
  */
 int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start,
                       int32_t chunk_rows, int32_t window, int32_t num_sms,
-                      int64_t *items, int32_t max_items, int32_t *n_items, int32_t *path);
+                      const int32_t *cluster_capacity, int64_t *items, int32_t max_items,
+                      int32_t *n_items, int32_t *path);
 int attn_decode_plan(int32_t batch, const int64_t *ctx_len, int32_t window, int32_t kv_dtype,
-                     int32_t num_sms, int64_t *items, int32_t max_items, int32_t *n_items);
+                     int32_t num_sms, const int32_t *cluster_capacity, int64_t *items,
+                     int32_t max_items, int32_t *n_items, int32_t *cluster);
+
+/*
+ * attn_decode_cluster_capacity -- the resident-cluster capacity that the
+ * plans above use on the CURRENT DEVICE: capacity[0], [1], [2] receive how
+ * many clusters of 2, 4, 8 CTAs of the tensor-core rows kernel fit on it at
+ * once (cudaOccupancyMaxActiveClusters, measured once per device).  With
+ * these and the device's SM count, attn_decode_plan computes on the host the
+ * plan a call on the device runs.  Returns KCA_OK, KCA_ERR_NULL, or
+ * KCA_ERR_CUDA without a device.  Passage: as for the plans (Karume v0.12.0
+ * release notes, "Docs", ADR 0067 plan-size geometry table).
+ */
+int attn_decode_cluster_capacity(int32_t *capacity);
 
 /*
  * attn_force_path -- pins the kernel family that later calls take,

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libkca.so")
 
 F32, F16, BF16 = 0, 1, 2
 N_Q_HEADS, N_KV_HEADS, HEAD_DIM = 8, 1, 256
-MAX_CHUNK_ROWS, MAX_POSITION, MAX_BATCH = 768, 131072, 256
+MAX_CHUNK_ROWS, MAX_POSITION, MAX_BATCH, MAX_BATCH_ROWS = 768, 131072, 256, 15
 WORKSPACE_HEADER = 24832  # status word + per-(row, head) merge counters
 STATUS = {0: "KCA_OK", -1: "KCA_ERR_NULL", -2: "KCA_ERR_GEOMETRY", -3: "KCA_ERR_DTYPE",
           -4: "KCA_ERR_RANGE", -5: "KCA_ERR_WORKSPACE", -6: "KCA_ERR_ALIGN", -7: "KCA_ERR_CUDA",
@@ -55,6 +55,11 @@ def lib() -> ctypes.CDLL:
         L.attn_decode.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp,
                                   vp, sz, vp]
         L.attn_decode.restype = ctypes.c_int
+        L.attn_prefill_batch.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, i32, p64, i32, f32,
+                                         vp, vp, sz, vp]
+        L.attn_prefill_batch.restype = ctypes.c_int
+        L.attn_prefill_batch_workspace_bytes.argtypes = [i32, i32, p64, i32]
+        L.attn_prefill_batch_workspace_bytes.restype = sz
         L.attn_decode_dev.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, vp, i64, i32, f32,
                                       vp, vp, sz, vp]
         L.attn_decode_dev.restype = ctypes.c_int
@@ -78,12 +83,14 @@ def lib() -> ctypes.CDLL:
         L.attn_workspace_init.restype = ctypes.c_int
         L.attn_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.attn_device_status.restype = ctypes.c_int
-        L.attn_prefill_plan.argtypes = [i32, i32, i64, i32, i32, i32, p64, i32, p32, p32]
+        L.attn_prefill_plan.argtypes = [i32, i32, i64, i32, i32, i32, p32, p64, i32, p32, p32]
         L.attn_prefill_plan.restype = ctypes.c_int
-        L.attn_decode_plan.argtypes = [i32, p64, i32, i32, i32, p64, i32, p32]
+        L.attn_decode_plan.argtypes = [i32, p64, i32, i32, i32, p32, p64, i32, p32, p32]
         L.attn_decode_plan.restype = ctypes.c_int
         L.attn_decode_static_scratch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(sz)]
         L.attn_decode_static_scratch.restype = ctypes.c_int
+        L.attn_decode_cluster_capacity.argtypes = [p32]
+        L.attn_decode_cluster_capacity.restype = ctypes.c_int
         L.attn_force_path.argtypes = [i32, i32]
         L.attn_force_path.restype = ctypes.c_int
         L.attn_status_string.argtypes = [ctypes.c_int]
@@ -243,6 +250,46 @@ def attn_decode(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.
                            ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
                            workspace.numel(), _stream_ptr(stream))
     _check(st, "attn_decode")
+    return out
+
+
+def attn_prefill_batch_workspace_bytes(ctx_len, rows: int, window: int = 0) -> int:
+    nctx, ptr = _i64_array(ctx_len)
+    n = lib().attn_prefill_batch_workspace_bytes(nctx, rows, ptr, window)
+    if n == 0:
+        raise KcaError(-4, "attn_prefill_batch_workspace_bytes")
+    return int(n)
+
+
+def attn_prefill_batch(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.0 / 16.0,
+                       out=None, workspace=None, stream=None):
+    """Short chunks of several sequences in one call.
+
+    q: [batch, rows, 8, 256] (rows 1..15); k_cache / v_cache: [batch,
+    capacity, 256]; ctx_len: host ints, row i of sequence b sits at position
+    ctx_len[b] - rows + i; returns out [batch, rows, 8, 256] float32.
+    """
+    import torch
+    batch, rows = q.shape[0], q.shape[1]
+    capacity = k_cache.shape[1]
+    for t in (q, k_cache, v_cache):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if k_cache.shape[0] != batch:
+        raise ValueError("k_cache batch does not match q")
+    nctx, ptr = _i64_array(ctx_len)
+    if nctx != batch:
+        raise ValueError("ctx_len must have one entry per sequence")
+    if out is None:
+        out = torch.empty((batch, rows, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(attn_prefill_batch_workspace_bytes(ctx_len, rows, window), q.device, stream)
+    vp = ctypes.c_void_p
+    st = lib().attn_prefill_batch(vp(q.data_ptr()), dtype_code(q), vp(k_cache.data_ptr()), vp(v_cache.data_ptr()),
+                                  dtype_code(k_cache), N_Q_HEADS, N_KV_HEADS, HEAD_DIM, capacity, batch, rows, ptr,
+                                  window, scale, vp(out.data_ptr()), vp(workspace.data_ptr()), workspace.numel(),
+                                  _stream_ptr(stream))
+    _check(st, "attn_prefill_batch")
     return out
 
 
@@ -455,50 +502,73 @@ def attn_prefill_path(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows:
     n = ctypes.c_int32(0)
     path = ctypes.c_int32(-1)
     # the path does not depend on the SM count; any positive count serves
-    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, 1, None, 0,
+    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, 1, None, None, 0,
                                  ctypes.byref(n), ctypes.byref(path))
     if path.value < 0:
         raise KcaError(st, "attn_prefill_plan")
     return int(path.value)
 
 
+def attn_decode_cluster_capacity() -> tuple[int, int, int]:
+    """Resident clusters of 2, 4 and 8 CTAs of the tensor-core rows kernel on
+    the current device (what the device plans use)."""
+    cap = (ctypes.c_int32 * 3)()
+    _check(lib().attn_decode_cluster_capacity(cap), "attn_decode_cluster_capacity")
+    return int(cap[0]), int(cap[1]), int(cap[2])
+
+
+def _capacity(cluster_capacity):
+    """int32[3] of resident clusters of 2, 4, 8 CTAs, or None (the device's)."""
+    if cluster_capacity is None:
+        return None
+    return (ctypes.c_int32 * 3)(*[int(x) for x in cluster_capacity])
+
+
 def attn_prefill_plan(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows: int,
-                      window: int = 0, num_sms: int | None = None):
+                      window: int = 0, num_sms: int | None = None, cluster_capacity=None):
     """(path, items[n, 4]) -- see include/kca.h.  num_sms defaults to the
     current device's SM count.  Host only, except the rows plan of 16-bit
-    caches, which is the tensor-core kernel's cluster plan on the current
-    device."""
-    num_sms = _num_sms(num_sms)
+    caches without cluster_capacity (resident clusters of 2, 4, 8 CTAs),
+    which is the tensor-core kernel's cluster plan on the current device."""
+    if cluster_capacity is None and num_sms is None:
+        num_sms = _num_sms(None)
+    num_sms = int(num_sms)
+    cap = _capacity(cluster_capacity)
     n = ctypes.c_int32(0)
     path = ctypes.c_int32(0)
-    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, num_sms, None,
+    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, num_sms, cap, None,
                                  0, ctypes.byref(n), ctypes.byref(path))
     if st not in (0, -4) or (st == -4 and n.value == 0):
         raise KcaError(st, "attn_prefill_plan")
     items = np.zeros((max(n.value, 1), 4), dtype=np.int64)
-    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, num_sms,
+    st = lib().attn_prefill_plan(q_dtype, kv_dtype, chunk_start, chunk_rows, window, num_sms, cap,
                                  items.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n.value,
                                  ctypes.byref(n), ctypes.byref(path))
     _check(st, "attn_prefill_plan")
     return int(path.value), items[:n.value]
 
 
-def attn_decode_plan(ctx_len, window: int = 0, num_sms: int | None = None, kv_dtype: int = F32):
-    """items[n, 4] of a decode call -- see include/kca.h.  kv_dtype F32: the
+def attn_decode_plan(ctx_len, window: int = 0, num_sms: int | None = None, kv_dtype: int = F32,
+                     cluster_capacity=None, with_cluster: bool = False):
+    """items[n, 4] of a decode call -- see include/kca.h -- and, with
+    with_cluster, the cluster size (items, cluster).  kv_dtype F32: the
     CUDA-core kernel's plan for num_sms SMs (default: the current device's
-    count); F16 / BF16: the tensor-core kernel's cluster plan on the current
-    device."""
-    if kv_dtype in (F16, BF16) and num_sms is None:
-        num_sms = 1          # not used by the cluster plan, which asks the device itself
+    count); F16 / BF16: the tensor-core kernel's cluster plan for num_sms SMs
+    holding cluster_capacity = (clusters of 2, 4, 8 CTAs) at once, host only,
+    or without cluster_capacity for the current device."""
+    if kv_dtype in (F16, BF16) and cluster_capacity is None and num_sms is None:
+        num_sms = 1          # not used: the plan asks the device itself
     num_sms = _num_sms(num_sms)
+    cap = _capacity(cluster_capacity)
     nctx, ptr = _i64_array(ctx_len)
     n = ctypes.c_int32(0)
-    st = lib().attn_decode_plan(nctx, ptr, window, kv_dtype, num_sms, None, 0, ctypes.byref(n))
+    cl = ctypes.c_int32(0)
+    st = lib().attn_decode_plan(nctx, ptr, window, kv_dtype, num_sms, cap, None, 0, ctypes.byref(n), None)
     if st not in (0, -4) or (st == -4 and n.value == 0):
         raise KcaError(st, "attn_decode_plan")
     items = np.zeros((max(n.value, 1), 4), dtype=np.int64)
-    st = lib().attn_decode_plan(nctx, ptr, window, kv_dtype, num_sms,
+    st = lib().attn_decode_plan(nctx, ptr, window, kv_dtype, num_sms, cap,
                                 items.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n.value,
-                                ctypes.byref(n))
+                                ctypes.byref(n), ctypes.byref(cl))
     _check(st, "attn_decode_plan")
-    return items[:n.value]
+    return (items[:n.value], int(cl.value)) if with_cluster else items[:n.value]

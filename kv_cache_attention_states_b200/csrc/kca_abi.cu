@@ -83,6 +83,23 @@ std::vector<int64_t> decode_unit_keys(int32_t batch, const int64_t* ctx_len, int
   for (int32_t b = 0; b < batch; ++b) nk[b] = kca::n_visible(ctx_len[b] - 1, window);
   return nk;
 }
+// Batched short chunks: unit b * rows + i is row i of sequence b, at
+// position ctx_len[b] - rows + i.
+std::vector<int64_t> batch_unit_keys(int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window) {
+  std::vector<int64_t> nk((size_t)batch * rows);
+  for (int32_t b = 0; b < batch; ++b)
+    for (int32_t i = 0; i < rows; ++i) nk[(size_t)b * rows + i] = kca::n_visible(ctx_len[b] - rows + i, window);
+  return nk;
+}
+
+int batch_args_status(int64_t capacity, int32_t batch, int32_t rows, const int64_t* ctx_len) {
+  if (capacity < 1 || capacity > KCA_MAX_POSITION) return KCA_ERR_RANGE;
+  if (batch < 1 || batch > KCA_MAX_BATCH || rows < 1 || rows > KCA_MAX_BATCH_ROWS) return KCA_ERR_RANGE;
+  for (int32_t b = 0; b < batch; ++b)
+    if (ctx_len[b] < rows || ctx_len[b] > capacity) return KCA_ERR_RANGE;
+  return KCA_OK;
+}
+
 // Keys of each decode query that a context shard [key_begin, key_end) holds.
 std::vector<int64_t> shard_unit_keys(int32_t batch, const int64_t* ctx_len, int32_t window, int64_t key_begin,
                                      int64_t key_end) {
@@ -240,14 +257,18 @@ bool use_rows_mma(int32_t kv_dtype) {
 // per SM, times the waves of clusters; a unit with several clusters adds
 // 1.5 us (partials, fence, ticket) and 0.6 us per round of loads of the
 // final merge.
-kca::RowsPlan mma_rows_plan(int32_t n_units, const int64_t* nkeys, int sms, int* cluster) {
+// capacity: resident clusters of 2, 4 and 8 CTAs (nullptr: the current
+// device's, measured once per device).
+kca::RowsPlan mma_rows_plan(int32_t n_units, const int64_t* nkeys, int sms, int* cluster,
+                            const int32_t* capacity = nullptr) {
   kca::RowsPlan best{};
   int best_c = 0;
   double best_t = 0.0;
   double total_keys = 0.0;
   for (int32_t u = 0; u < n_units; ++u) total_keys += (double)nkeys[u];
   for (int c = 8; c >= 1; c /= 2) {
-    int slots = c == 1 ? sms : kca::decode_mma_cluster_capacity(c);
+    const int ci = c == 2 ? 0 : (c == 4 ? 1 : 2);
+    int slots = c == 1 ? sms : (capacity != nullptr ? capacity[ci] : kca::decode_mma_cluster_capacity(c));
     if (slots > kca::kRowsMmaMaxClusterParts) slots = kca::kRowsMmaMaxClusterParts;
     if (slots <= 0) continue;
     const kca::RowsPlan p = kca::make_cluster_rows_plan(n_units, nkeys, c, slots);
@@ -337,15 +358,16 @@ int launch_rows_path(int32_t q_dtype, int32_t kv_dtype, const void* k_cache, con
 // cluster partial its cluster writes (tensor cores), -1 when nothing of the
 // unit goes through global memory.
 int rows_plan_items(int32_t kv_dtype, int32_t n, const int64_t* pos, const int64_t* nk, int32_t window,
-                    int32_t num_sms, int64_t* items, int32_t max_items, int32_t* count) {
+                    int32_t num_sms, const int32_t* capacity, int64_t* items, int32_t max_items, int32_t* count,
+                    int32_t* cluster_out) {
   const bool mma = use_rows_mma(kv_dtype);
   kca::RowsPlan p;
   int cluster = 1;
   if (mma) {
-    int sms = 0;
-    if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
-    p = mma_rows_plan(n, nk, sms, &cluster);
-    if (cluster < 1) return KCA_ERR_CUDA;
+    int sms = num_sms;
+    if (capacity == nullptr && current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+    p = mma_rows_plan(n, nk, sms, &cluster, capacity);
+    if (cluster < 1) return capacity == nullptr ? KCA_ERR_CUDA : KCA_ERR_RANGE;
   } else {
     p = kca::make_rows_plan(n, nk, num_sms);
   }
@@ -366,12 +388,24 @@ int rows_plan_items(int32_t kv_dtype, int32_t n, const int64_t* pos, const int64
                                   : (ns > 1 ? (int64_t)u * p.max_splits + sp : -1);
     }
   }
+  if (cluster_out != nullptr) *cluster_out = cluster;
   return KCA_OK;
 }
 
 }  // namespace
 
 extern "C" {
+
+int attn_decode_cluster_capacity(int32_t* capacity) {
+  if (capacity == nullptr) return KCA_ERR_NULL;
+  const int sizes[3] = {2, 4, 8};
+  for (int i = 0; i < 3; ++i) {
+    const int n = kca::decode_mma_cluster_capacity(sizes[i]);
+    if (n <= 0) return KCA_ERR_CUDA;
+    capacity[i] = n;
+  }
+  return KCA_OK;
+}
 
 int attn_force_path(int32_t op, int32_t path) {
   if (path < -1 || path > 1) return KCA_ERR_RANGE;
@@ -397,12 +431,14 @@ const char* attn_status_string(int status) {
 }
 
 int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, int32_t chunk_rows,
-                      int32_t window, int32_t num_sms, int64_t* items, int32_t max_items,
-                      int32_t* n_items, int32_t* path) {
+                      int32_t window, int32_t num_sms, const int32_t* cluster_capacity, int64_t* items,
+                      int32_t max_items, int32_t* n_items, int32_t* path) {
   if (n_items == nullptr || path == nullptr || (items == nullptr && max_items > 0)) return KCA_ERR_NULL;
   if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
   if (chunk_rows < 1 || chunk_rows > KCA_MAX_CHUNK_ROWS || chunk_start < 0 ||
       chunk_start + chunk_rows > KCA_MAX_POSITION || num_sms < 1)
+    return KCA_ERR_RANGE;
+  if (cluster_capacity != nullptr && (cluster_capacity[0] < 0 || cluster_capacity[1] < 0 || cluster_capacity[2] < 0))
     return KCA_ERR_RANGE;
   int32_t count = 0;
   if (use_tc(q_dtype, kv_dtype, chunk_start, chunk_rows, window)) {
@@ -426,8 +462,8 @@ int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, in
     const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
     std::vector<int64_t> pos(chunk_rows);
     for (int32_t u = 0; u < chunk_rows; ++u) pos[u] = chunk_start + u;
-    const int st = rows_plan_items(kv_dtype, chunk_rows, pos.data(), nk.data(), window, num_sms, items,
-                                   max_items, &count);
+    const int st = rows_plan_items(kv_dtype, chunk_rows, pos.data(), nk.data(), window, num_sms,
+                                   cluster_capacity, items, max_items, &count, nullptr);
     if (st != KCA_OK) return st;
   }
   *n_items = count;
@@ -435,17 +471,21 @@ int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, in
 }
 
 int attn_decode_plan(int32_t batch, const int64_t* ctx_len, int32_t window, int32_t kv_dtype, int32_t num_sms,
-                     int64_t* items, int32_t max_items, int32_t* n_items) {
+                     const int32_t* cluster_capacity, int64_t* items, int32_t max_items, int32_t* n_items,
+                     int32_t* cluster) {
   if (ctx_len == nullptr || n_items == nullptr || (items == nullptr && max_items > 0)) return KCA_ERR_NULL;
   if (!dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
   if (batch < 1 || batch > KCA_MAX_BATCH || num_sms < 1) return KCA_ERR_RANGE;
+  if (cluster_capacity != nullptr && (cluster_capacity[0] < 0 || cluster_capacity[1] < 0 || cluster_capacity[2] < 0))
+    return KCA_ERR_RANGE;
   for (int32_t b = 0; b < batch; ++b)
     if (ctx_len[b] < 0 || ctx_len[b] > KCA_MAX_POSITION) return KCA_ERR_RANGE;
   const std::vector<int64_t> nk = decode_unit_keys(batch, ctx_len, window);
   std::vector<int64_t> pos(batch);
   for (int32_t b = 0; b < batch; ++b) pos[b] = ctx_len[b] - 1;
   int32_t count = 0;
-  const int st = rows_plan_items(kv_dtype, batch, pos.data(), nk.data(), window, num_sms, items, max_items, &count);
+  const int st = rows_plan_items(kv_dtype, batch, pos.data(), nk.data(), window, num_sms, cluster_capacity, items,
+                                 max_items, &count, cluster);
   if (st != KCA_OK) return st;
   *n_items = count;
   return count <= max_items ? KCA_OK : KCA_ERR_RANGE;
@@ -470,6 +510,14 @@ size_t attn_decode_partial_workspace_bytes(int32_t batch, const int64_t* ctx_len
   if (current_sms(&sms) != KCA_OK) return 0;
   const std::vector<int64_t> nk = shard_unit_keys(batch, ctx_len, window, key_begin, key_begin + capacity);
   return rows_ws_bytes_any(batch, nk.data(), sms);
+}
+
+size_t attn_prefill_batch_workspace_bytes(int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window) {
+  if (ctx_len == nullptr || batch_args_status(KCA_MAX_POSITION, batch, rows, ctx_len) != KCA_OK) return 0;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return 0;
+  const std::vector<int64_t> nk = batch_unit_keys(batch, rows, ctx_len, window);
+  return rows_ws_bytes_any(batch * rows, nk.data(), sms);
 }
 
 size_t attn_decode_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_t window) {
@@ -746,6 +794,47 @@ int attn_decode_partial(const void* q, int32_t q_dtype, const void* k_cache, con
   for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
   return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster,
                           workspace, static_cast<cudaStream_t>(stream));
+}
+
+int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache,
+                       int32_t kv_dtype, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                       int64_t capacity, int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window,
+                       float scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !out || !workspace || !ctx_len) return KCA_ERR_NULL;
+  int st = geometry_status(n_q_heads, n_kv_heads, head_dim);
+  if (st != KCA_OK) return st;
+  if (!dtype_ok(q_dtype) || !dtype_ok(kv_dtype)) return KCA_ERR_DTYPE;
+  st = batch_args_status(capacity, batch, rows, ctx_len);
+  if (st != KCA_OK) return st;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return KCA_ERR_RANGE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return KCA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+  const int32_t n_units = batch * rows;
+  const std::vector<int64_t> nk = batch_unit_keys(batch, rows, ctx_len, window);
+  int cluster = 1;
+  size_t need = 0;
+  const kca::RowsPlan p = rows_plan(kv_dtype, n_units, nk.data(), sms, &cluster, &need);
+  if (cluster < 1) return KCA_ERR_CUDA;
+  if (workspace_bytes < need) return KCA_ERR_WORKSPACE;
+  kca::RowsArgs a{};
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.out = out;
+  a.status = workspace;
+  a.seq_rows = capacity;
+  a.mode = 2;
+  a.rows_per_seq = rows;
+  a.n_units = n_units;
+  a.split_len = p.split_len;
+  a.max_splits = p.max_splits;
+  a.window = window;
+  a.scale = scale;
+  for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
+  return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster, workspace,
+                          static_cast<cudaStream_t>(stream));
 }
 
 int attn_merge_partials(int32_t n_parts, int32_t batch, const float* parts, int64_t part_stride, float* out,

@@ -284,7 +284,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
   // Device context lengths may come from the previous kernel of the stream:
   // with them, the dependency wait comes before they are read.
   if (a.ctx_dev != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, split == 0 && threadIdx.x == 0) - 1 : a.chunk_start + unit;
+  int64_t seq_base;
+  const int64_t pos = rows_unit_pos(a, unit, split == 0 && threadIdx.x == 0, &seq_base);
   int64_t lo;
   const int64_t nkeys = rows_keys(a, pos, &lo);
   const int32_t split_len = rows_split_len(a, nkeys, kDStageKeys);
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
   int64_t kend = kbeg + split_len;
   if (kend > lo + nkeys) kend = lo + nkeys;
   // cache row of key p: base_row + p (a shard's row 0 is position key_begin)
-  const int64_t base_row = (a.mode == 0 ? (int64_t)unit * a.seq_rows : 0) - a.key_begin;
+  const int64_t base_row = seq_base - a.key_begin;
   const int n_stage = active ? (int)cdiv(kend - kbeg, kDStageKeys) : 0;
 
   if (threadIdx.x == 0) {
@@ -571,9 +572,11 @@ __global__ void __launch_bounds__(kDThreads, 1)
       float L = 0.f, O = 0.f;
 #pragma unroll
       for (int src = 0; src < 8; ++src) {
-        const float f = exp2f((mv[src] - mu) * kDLog2e);
-        L += f * lv[src];
-        O += f * ov[src];
+        if (src < C) {   // sources past C are empty: weight exactly 0
+          const float f = exp2f((mv[src] - mu) * kDLog2e);
+          L += f * lv[src];
+          O += f * ov[src];
+        }
       }
       if (nclus == 1) {
         a.out[((int64_t)unit * kHeads + h) * kDim + d] = rows_final(a, O, M, L);

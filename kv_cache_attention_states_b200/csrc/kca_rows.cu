@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, split == 0 && threadIdx.x == 0) - 1 : a.chunk_start + unit;
+  int64_t seq_base;
+  const int64_t pos = rows_unit_pos(a, unit, split == 0 && threadIdx.x == 0, &seq_base);
   int64_t lo;
   const int64_t nkeys = rows_keys(a, pos, &lo);
   const int32_t split_len = rows_split_len(a, nkeys, kRowsSplitQuantum);
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
   int64_t kend = kbeg + split_len;
   if (kend > lo + nkeys) kend = lo + nkeys;
   // cache row of key p: base_row + p (a shard's row 0 is position key_begin)
-  const int64_t base_row = (a.mode == 0 ? (int64_t)unit * a.seq_rows : 0) - a.key_begin;
+  const int64_t base_row = seq_base - a.key_begin;
   float* out = a.out + (int64_t)unit * kHeads * kDim;
 
   if (nkeys == 0) {  // fully masked row: exactly zero (as a partial: (-inf, 0, 0))
@@ -298,7 +299,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
 // its eight warps taking interleaved splits.
 __global__ void __launch_bounds__(256) merge_rows_kernel(const RowsArgs a) {
   const int unit = blockIdx.x >> 3, h = blockIdx.x & 7;
-  const int64_t pos = a.mode == 0 ? rows_ctx(a, unit, false) - 1 : a.chunk_start + unit;
+  int64_t seq_base;
+  const int64_t pos = rows_unit_pos(a, unit, false, &seq_base);
   int64_t lo;
   const int64_t nkeys = rows_keys(a, pos, &lo);
   const int32_t nsplit = rows_n_splits(nkeys, rows_split_len(a, nkeys, kRowsSplitQuantum));

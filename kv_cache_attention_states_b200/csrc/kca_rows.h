@@ -16,9 +16,11 @@ struct RowsArgs {
   float* part_ml;        // [n_units * max_splits][8][2]  (m, l), or null
   float* part_acc;       // [n_units * max_splits][8][256], or null
   void* status;          // workspace status header
-  int64_t seq_rows;      // decode: cache rows per sequence (capacity)
+  int64_t seq_rows;      // decode, batched rows: cache rows per sequence (capacity)
   int64_t chunk_start;   // prefill: position of unit 0
-  int32_t mode;          // 0: decode (unit = sequence), 1: prefill (unit = row of sequence 0)
+  int32_t mode;          // 0: decode (unit = sequence), 1: prefill (unit = row of sequence 0),
+                         // 2: batched rows (unit = row i of sequence unit / rows_per_seq)
+  int32_t rows_per_seq;  // mode 2: query rows per sequence, at ctx[b] - rows_per_seq .. ctx[b] - 1
   int32_t n_units;
   int32_t split_len;
   int32_t max_splits;
@@ -62,6 +64,21 @@ __device__ __forceinline__ int64_t rows_ctx(const RowsArgs& a, int unit, bool re
   if (c >= 0 && c <= a.ctx_bound) return c;
   if (record) record_error(static_cast<DeviceStatus*>(a.status), kSiteCtx, kErrBadCtx, (unsigned)unit);
   return 0;
+}
+// Position of the query of `unit`, and the cache row of position 0 of its
+// sequence (*seq_base; before the shard offset).
+__device__ __forceinline__ int64_t rows_unit_pos(const RowsArgs& a, int unit, bool record, int64_t* seq_base) {
+  if (a.mode == 1) {
+    *seq_base = 0;
+    return a.chunk_start + unit;
+  }
+  if (a.mode == 2) {
+    const int b = unit / a.rows_per_seq;
+    *seq_base = (int64_t)b * a.seq_rows;
+    return a.ctx[b] - a.rows_per_seq + unit % a.rows_per_seq;
+  }
+  *seq_base = (int64_t)unit * a.seq_rows;
+  return rows_ctx(a, unit, record) - 1;
 }
 // Visible keys [*lo, *lo + n) of the query at pos within the cache's shard.
 __device__ __forceinline__ int64_t rows_keys(const RowsArgs& a, int64_t pos, int64_t* lo) {

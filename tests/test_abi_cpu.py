@@ -70,7 +70,8 @@ def test_header_constants_match_binding():
     text = open(HEADER).read()
     for name, val in [("KCA_MAX_CHUNK_ROWS", 768), ("KCA_MAX_POSITION", 131072),
                       ("KCA_HEAD_DIM", 256), ("KCA_N_Q_HEADS", 8), ("KCA_N_KV_HEADS", 1),
-                      ("KCA_WORKSPACE_HEADER", 24832), ("KCA_MAX_BATCH", 256)]:
+                      ("KCA_WORKSPACE_HEADER", 24832), ("KCA_MAX_BATCH", 256),
+                      ("KCA_MAX_BATCH_ROWS", 15)]:
         assert re.search(rf"#define {name} {val}\b", text), name
 
 
@@ -132,6 +133,39 @@ def test_prefill_rejects_bad_arguments_on_the_host(kw, code):
 ])
 def test_decode_rejects_bad_arguments_on_the_host(ctx, kw, code):
     assert _decode(ctx, **kw) == code
+
+
+def _prefill_batch(ctx=(100, 200), rows=3, **kw):
+    a = dict(q=P, qd=kca.F32, k=P, v=P, kd=kca.F16, hq=8, hkv=1, d=256, cap=4096, window=0,
+             scale=0.0625, out=P, ws=P * 2, wsb=1 << 30, batch=None)
+    a.update(kw)
+    arr = np.asarray(ctx, dtype=np.int64)
+    batch = len(arr) if a["batch"] is None else a["batch"]
+    vp = ctypes.c_void_p
+    return kca.lib().attn_prefill_batch(vp(a["q"]), a["qd"], vp(a["k"]), vp(a["v"]), a["kd"], a["hq"],
+                                        a["hkv"], a["d"], a["cap"], batch, rows,
+                                        arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), a["window"],
+                                        a["scale"], vp(a["out"]), vp(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("ctx,rows,kw,code", [
+    ((3, 9), 3, dict(q=0), -1), ((3, 9), 3, dict(ws=0), -1), ((3, 9), 3, dict(hkv=2), -2),
+    ((3, 9), 3, dict(qd=9), -3), ((3, 9), 0, dict(), -4), ((16, 20), 16, dict(), -4),
+    ((2, 9), 3, dict(), -4), ((3, 4097), 3, dict(), -4), ((3, 9), 3, dict(batch=0), -4),
+    ((3,) * 257, 3, dict(), -4), ((3, 9), 3, dict(scale=0.0), -4), ((3, 9), 3, dict(cap=131073), -4),
+    ((3, 9), 3, dict(v=P + 8), -6), ((3, 9), 3, dict(ws=P * 2 + 64), -5),
+])
+def test_prefill_batch_rejects_bad_arguments_on_the_host(ctx, rows, kw, code):
+    assert _prefill_batch(ctx, rows, **kw) == code
+
+
+def test_prefill_batch_workspace_query_rejects_bad_arguments():
+    lib = kca.lib()
+    arr = np.asarray([3, 9], dtype=np.int64)
+    ptr = arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+    assert lib.attn_prefill_batch_workspace_bytes(2, 4, ptr, 0) == 0      # ctx 3 < 4 rows
+    assert lib.attn_prefill_batch_workspace_bytes(2, 16, ptr, 0) == 0
+    assert lib.attn_prefill_batch_workspace_bytes(2, 3, None, 0) == 0
 
 
 def _decode_static(ctx=(100, 200), **kw):

@@ -95,9 +95,10 @@ def other_parts(cuda_ok):
     for g in graphs:
         g.replay()
     torch.cuda.synchronize()
+    import kv_cache_attention_states_b200 as kca
     for p in parts:
         for ws in p.workspaces():
-            assert p.kca.attn_device_status(ws)[0] == 0, p.name
+            assert kca.attn_device_status(ws)[0] == 0, p.name
     return bench, parts, win
 
 

@@ -75,3 +75,18 @@ def test_short_chunk_rows_plan_on_tensor_cores_is_the_documented_cut(cuda_ok, cs
     path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, rows, window)
     assert path == 0
     _check(items, [cs + u for u in range(rows)], window)
+
+
+@pytest.mark.parametrize("ctx,window", [([16384], 0), ([16447], 0), ([4096], 0), ([256], 0), ([131072], 0),
+                                        ([4160], 512), ([131072] * 8, 0)])
+def test_device_plan_is_the_host_plan_for_the_device_capacity(cuda_ok, ctx, window):
+    """The plan a call runs on this device equals the host-only plan for the
+    device's SM count and resident-cluster capacity, which the CPU tests pin
+    to the documented cost model."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cap = kca.attn_decode_cluster_capacity()
+    dev_items, dev_c = kca.attn_decode_plan(ctx, window, kv_dtype=kca.F16, with_cluster=True)
+    host_items, host_c = kca.attn_decode_plan(ctx, window, num_sms=sms, kv_dtype=kca.F16, cluster_capacity=cap,
+                                              with_cluster=True)
+    assert dev_c == host_c and np.array_equal(dev_items, host_items), (cap, dev_c, host_c)
