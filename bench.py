@@ -1,31 +1,33 @@
 """Benchmark of the states-form attention hot path on B200.
 
-One step = PASSES passes; one pass runs every workload configuration once,
-each as a CUDA graph of its C-ABI calls, in this order (each small working
-set follows a large one, so that its calls read cold rows from HBM):
+One step = PASSES passes over the headline workload, each pass a CUDA graph
+of its C-ABI calls:
 
-  ragged         8 sequences, context drawn by the seed from [1024, 131072],
+  prefill        the 16,384-token prompt in 768-row chunks (21 x 768 + 256),
+                 bf16 Q/K/V ~ N(0,1)*0.5 (2 input replicas)        -> value
+  decode         64 decode steps at context 16384..16447, f16 K/V, f32 q
+                 (32 cache replicas)
+
+value = prefill q-rows/s (a q-row is one query position with all 8 heads),
+from CUDA events around the prefill graph of every pass; ms_per_step covers
+whole steps.  Every other workload configuration is then timed the same way
+in a region of its own (OTHER_PASSES passes per step, in this order, so
+that each small working set follows a large one and its calls read cold
+rows from HBM) and reported in its own object of the JSON line:
+
+  decode_ragged  8 sequences, context drawn by the seed from [1024, 131072],
                  32 decode steps, f16 K/V, f32 q
   decode_256     64 decode steps at context 256..319, f16 K/V, f32 q
                  (64 cache replicas, one per step)
   decode_4096    64 decode steps at context 4096..4159 (64 replicas)
-  prefill        the 16,384-token prompt in 768-row chunks (21 x 768 + 256),
-                 bf16 Q/K/V ~ N(0,1)*0.5 (2 input replicas)        -> value
-  decode         64 decode steps at context 16384..16447 (32 replicas)
   window         window 512: a 4,096-token prompt in 768-row chunks, then 64
                  decode steps at positions 4096..4159, bf16 Q/K/V ~ N(0,1)
+                 (the decode re-reads rows its previous step read: the window
+                 slides by one row)
   long_chunk     one 768-row bf16 chunk at positions 130304..131071 of a
                  131,072-row cache
   prefill_batch  32 sequences x 4 query rows (speculative / multi-row decode)
                  per call through attn_prefill_batch, 16 calls, f16 K/V
-
-value = prefill q-rows/s (a q-row is one query position with all 8 heads),
-from CUDA events around the prefill graph of every pass; every other
-configuration gets its own object in the JSON line, timed the same way.
-ms_per_step covers whole steps.  The decode caches smaller than L2 rotate
-over replicas (and follow the 1 GB ragged batch in each pass), so every
-timed call reads its K/V rows from HBM; the sliding-window decode re-reads
-rows its previous step read by construction of the window.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--passes P] [--impl reference]
 Under torchrun each rank runs its own replica of the workload (weak scaling,
@@ -49,13 +51,21 @@ DECODE_STEPS = 64
 DECODE_REPLICAS = 32
 PREFILL_REPLICAS = 2
 SMALL_DECODE_REPLICAS = 64
-PASSES = 10              # passes over every configuration per step
+PASSES = 40              # passes over the headline step per timed step
+OTHER_PASSES = 2         # passes over the other configurations per step (own region)
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels, with the launch they come from; None once a kernel has changed
 # since its capture.
 TRAFFIC = {
     "prefill": (18.931e6 + 25.6e3, "prefill_tc_kernel, chunk 19 (768 rows at 14592)"),
     "decode": (16.919e6, "decode_mma_kernel, one call at ctx ~16.4K"),
+    "decode_256": (402432.0, "decode_mma_kernel, one call at ctx ~256 (the whole last 64-row stage is loaded)"),
+    "decode_4096": (4336384.0, "decode_mma_kernel, one call at ctx ~4.1K"),
+    "decode_ragged": (459086080.0 + 3675136.0, "decode_mma_kernel, one call of the 8-sequence batch"),
+    "window_prefill": (4518912.0, "prefill_tc_kernel, one 768-row chunk, window 512"),
+    "window_decode": (595456.0, "decode_mma_kernel<bf16, bf16>, one call, window 512 (cold caches)"),
+    "long_chunk": (138080256.0 + 4125184.0, "prefill_tc_kernel, the 768-row chunk at 130304"),
+    "prefill_batch": (301921280.0 + 4305664.0, "decode_mma_kernel, one call of 32 sequences x 4 rows"),
 }
 E2E_GROUP = 4            # prefill chunks per host copy in the end-to-end leg
 METRIC = "prefill q-rows/s & decode tok/s at 16K ctx (1 B200); % of TC/HBM roofline"
@@ -589,48 +599,69 @@ def run_cuda(args, rank, world, local_rank):
         else:
             graphs[p.name][i % p.variants].replay()
 
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks = Clocks(dev)
-    n_runs = args.steps * passes
-    ev = {p.name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(n_runs)] for p in parts}
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
+    def timed(region, reps):
+        """K steps of `reps` passes over the parts in `region`, each part
+        bracketed by CUDA events on the launching stream; returns (region ms,
+        {part: ms summed over its runs}, clocks during the region)."""
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clocks = Clocks(dev)
+        n = args.steps * reps
+        ev = {p.name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(n)] for p in region}
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        i = 0
+        for s in range(args.steps):
+            for _ in range(reps):
+                for p in region:
+                    e0, e1 = ev[p.name][i]
+                    e0.record(stream)
+                    replay(p, i)
+                    e1.record(stream)
+                i += 1
+        end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        names = [p.name for p in region]
+        vals = max_over_ranks([start.elapsed_time(end)] + [sum(a.elapsed_time(b) for a, b in ev[nm]) for nm in names],
+                              world, dev)
+        return vals[0], dict(zip(names, vals[1:])), clk
+
+    # The timed region proper: the headline step (the 16K prompt and its 64
+    # decode steps), replayed `passes` times per step.  The other
+    # configurations follow in a region of their own.
+    main = [p for p in parts if p.name in ("prefill", "decode")]
+    others = [p for p in parts if p.name not in ("prefill", "decode")]
     nvtx = torch.cuda.nvtx
-    nvtx.range_push("timed steps")
-    start.record(stream)
-    i = 0
-    for s in range(args.steps):
-        for _ in range(passes):
-            for p in parts:
-                e0, e1 = ev[p.name][i]
-                e0.record(stream)
-                replay(p, i)
-                e1.record(stream)
-            i += 1
-    end.record(stream)
-    nvtx.range_pop()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    total_ms = start.elapsed_time(end)
-    names = [p.name for p in parts]
-    part_ms = [sum(a.elapsed_time(b) for a, b in ev[nm]) for nm in names]
-    vals = max_over_ranks([total_ms] + part_ms, world, dev)
-    total_ms, part_ms = vals[0], dict(zip(names, vals[1:]))
+    res = dict(parts={p.name: p for p in parts}, part_ms={}, runs={}, passes=passes)
+    if main:
+        nvtx.range_push("timed steps")
+        total_ms, pm, clk = timed(main, passes)
+        nvtx.range_pop()
+        res.update(total_ms=total_ms, clocks=clk, launches=sum(p.launches for p in main) * args.steps * passes)
+        res["part_ms"].update(pm)
+        res["runs"].update({nm: args.steps * passes for nm in pm})
+    if others:
+        reps = max(1, args.other_passes)
+        nvtx.range_push("other configurations")
+        other_ms, pm, clk = timed(others, reps)
+        nvtx.range_pop()
+        res.update(other_ms=other_ms, other_clocks=clk, other_passes=reps,
+                   other_launches=sum(p.launches for p in others) * args.steps * reps)
+        res["part_ms"].update(pm)
+        res["runs"].update({nm: args.steps * reps for nm in pm})
     import kv_cache_attention_states_b200 as kca
     for p in parts:
         for ws in p.workspaces():
             st, detail = kca.attn_device_status(ws)
             if st != 0:
                 raise RuntimeError(f"{p.name}: device status {st} detail {detail:#x}")
-    res = dict(total_ms=total_ms, part_ms=part_ms, runs=n_runs, clocks=clk, passes=passes,
-               launches=sum(p.launches for p in parts) * n_runs,
-               parts={p.name: p for p in parts})
     if graphs is not None:
         del graphs
     if args.only is not None:
@@ -914,7 +945,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--passes", type=int, default=PASSES, help="passes over every configuration per step")
+    ap.add_argument("--passes", type=int, default=PASSES, help="passes over the headline step per timed step")
+    ap.add_argument("--other-passes", type=int, default=OTHER_PASSES,
+                    help="passes over the other configurations per step, in their own timed region")
     ap.add_argument("--impl", default="kca", choices=["kca", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every call from Python instead of "
@@ -940,9 +973,9 @@ def main():
         if rank == 0:
             hbm, tflops, tflops_sus, src = _peaks()
             p = res["parts"][args.only]
-            print(json.dumps({"only": args.only, "steps": args.steps, "passes": res["passes"],
-                              **part_object(p, res["part_ms"][args.only], res["runs"], world, hbm, tflops,
-                                            tflops_sus, src)}), flush=True)
+            print(json.dumps({"only": args.only, "steps": args.steps, "runs": res["runs"][args.only],
+                              **part_object(p, res["part_ms"][args.only], res["runs"][args.only], world, hbm,
+                                            tflops, tflops_sus, src)}), flush=True)
         if world > 1:
             dist.destroy_process_group()
         return
@@ -964,11 +997,11 @@ def main():
     if rank != 0:
         return
     hbm, tflops, tflops_sus, src = _peaks()
-    K, runs = args.steps, res["runs"]
+    K = args.steps
     parts, pm = res["parts"], res["part_ms"]
 
     def obj(name):
-        return part_object(parts[name], pm[name], runs, world, hbm, tflops, tflops_sus, src,
+        return part_object(parts[name], pm[name], res["runs"][name], world, hbm, tflops, tflops_sus, src,
                            (parts_cpu or {}).get(name))
 
     pre = obj("prefill")
@@ -981,14 +1014,16 @@ def main():
                                "+ 64 decode steps at ctx 16384-16447 (f16 K/V, f32 q); 8 q heads / "
                                "1 KV head, head_dim 256, causal",
                    "seq_len": 16384, "global_batch": world, "parallelism": f"replicas x{world}",
-                   "step": f"{res['passes']} passes; a pass runs every configuration once (ragged, "
-                           "decode_256, decode_4096, prefill, decode, window, long_chunk, prefill_batch)",
-                   "value": "prefill part of every pass (CUDA events); the other configurations in "
-                            "their own objects",
+                   "step": f"{res['passes']} passes over the prompt's prefill and its 64 decode steps",
+                   "value": "prefill part of every pass (CUDA events); the 16K decode in 'decode'",
+                   "other_configurations": f"timed after the main region, {res['other_passes']} passes per step "
+                                           f"over ragged, decode_256, decode_4096, window, long_chunk, "
+                                           f"prefill_batch ({res['other_ms'] / K:.1f} ms per step, "
+                                           f"{res['other_launches']} launches, clocks {res['other_clocks']})",
                    "launch": "eager" if args.eager else "one CUDA graph per configuration of the C-ABI calls",
-                   "l2": "inputs larger than L2: decode caches rotate over replicas (16K: 32 x 16.8 MB; "
-                         "256 / 4096: 64 each, after the 1 GB ragged batch), the prompt alternates 2 "
-                         "input replicas (80 MB each)"},
+                   "l2": "inputs larger than L2: the 16K decode rotates 32 cache replicas (16.8 MB "
+                         "each), the prompt alternates 2 input replicas (80 MB each); in the other region "
+                         "the 256 / 4096 decodes rotate 64 replicas each after the 1 GB ragged batch"},
         "roofline": pre["roofline"],
         "decode": obj("decode"),
         "decode_256": obj("decode_256"),
