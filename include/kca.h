@@ -100,6 +100,10 @@ extern "C" {
 #define KCA_F32 0
 #define KCA_F16 1
 #define KCA_BF16 2
+/* packed int8 K rows of the quantised-dot calls: 256 int8 codes, the row's
+ * f32 scale at byte 256, 12 zero bytes (272 bytes, 16-byte aligned) */
+#define KCA_I8 3
+#define KCA_I8_ROW_BYTES 272
 
 /* status codes */
 #define KCA_OK 0
@@ -346,6 +350,46 @@ int attn_decode_partial(const void *q, int32_t q_dtype,
                         void *stream);
 int attn_merge_partials(int32_t n_parts, int32_t batch, const float *parts, int64_t part_stride,
                         float *out, void *stream);
+
+/*
+ * Quantised-dot attention: K stored as int8 codes with one scale per row,
+ * the query quantised the same way per head inside the kernel, the QK dot
+ * product taken exactly on the codes, softmax and the V sum in f32.
+ * Passage: Karume v0.8.0 release notes, "Fixes": the attention dot product on
+ * packed int8 pairs (dp4a, behind a device canary that falls back to the
+ * emulation or fails loudly), and the activation-quantisation item (per-token
+ * scale amax * f32(1/127)).
+ *
+ * Quantisation of a row x of 256 values: sx = amax(|x|) * f32(1/127) (NaN when
+ * x holds a NaN); code = clamp(round_half_even(x / sx), -127, 127), the
+ * quotient in f32, when sx is finite and > 0, else 0.  Scores:
+ *   s_j = scale * sq_h * sk_j * sum_t q8_h[t] k8_j[t]
+ * (the integer sum exact), then the softmax and V sum of attn_decode.
+ *
+ * attn_quantize_k: k [n_rows][256] k_dtype (device, 16-byte aligned) ->
+ *   k8 [n_rows][KCA_I8_ROW_BYTES] packed rows (device, 16-byte aligned): the
+ *   256 codes, sx as f32 at byte 256, 12 zero bytes.  Writes a batched cache
+ *   row by row (row b * capacity + p of sequence b at position p).
+ * attn_decode_q8: attn_decode with a packed int8 K cache k8_cache
+ *   [batch][capacity][KCA_I8_ROW_BYTES] and v_cache [batch][capacity][256] of
+ *   v_dtype (F32, F16 or BF16); q of any dtype, out f32; the plan, workspace
+ *   (attn_decode_q8_workspace_bytes), errors and semantics of attn_decode
+ *   (CUDA-core kernel).  The first call on a device runs the canary below
+ *   (a synchronising launch): make it, or call attn_dot_canary, before any
+ *   stream capture.
+ * attn_dot_canary: runs, once per device, the dp4a instruction and its
+ *   emulation on known answers; *variant = 1 when the instruction is right
+ *   (the decode uses it), 0 when only the emulation is (the decode uses the
+ *   emulation); KCA_ERR_DEVICE, and attn_decode_q8 refuses to run, when
+ *   neither is.  Synchronises `stream` on its first call per device.
+ */
+int attn_quantize_k(const void *k, int32_t k_dtype, int64_t n_rows, void *k8, void *stream);
+int attn_decode_q8(const void *q, int32_t q_dtype, const void *k8_cache, const void *v_cache,
+                   int32_t v_dtype, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                   int64_t capacity, int32_t batch, const int64_t *ctx_len, int32_t window,
+                   float scale, float *out, void *workspace, size_t workspace_bytes, void *stream);
+size_t attn_decode_q8_workspace_bytes(int32_t batch, const int64_t *ctx_len, int32_t window);
+int attn_dot_canary(void *stream, int32_t *variant);
 
 /* Workspace bytes the calls above need on the current device (0 on a bad
  * argument).  Always >= KCA_WORKSPACE_HEADER.  The size depends on the

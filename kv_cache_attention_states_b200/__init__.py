@@ -20,7 +20,8 @@ from . import synth  # noqa: F401  (seeded inputs; no attention arithmetic)
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkca.so")
 
-F32, F16, BF16 = 0, 1, 2
+F32, F16, BF16, I8 = 0, 1, 2, 3
+I8_ROW_BYTES = 272        # packed int8 K row: 256 codes, f32 scale, 12 zero bytes
 N_Q_HEADS, N_KV_HEADS, HEAD_DIM = 8, 1, 256
 MAX_CHUNK_ROWS, MAX_POSITION, MAX_BATCH, MAX_BATCH_ROWS = 768, 131072, 256, 15
 WORKSPACE_HEADER = 24832  # status word + per-(row, head) merge counters
@@ -89,6 +90,14 @@ def lib() -> ctypes.CDLL:
         L.attn_decode_plan.restype = ctypes.c_int
         L.attn_decode_static_scratch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(sz)]
         L.attn_decode_static_scratch.restype = ctypes.c_int
+        L.attn_quantize_k.argtypes = [vp, i32, i64, vp, vp]
+        L.attn_quantize_k.restype = ctypes.c_int
+        L.attn_decode_q8.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp, vp, sz, vp]
+        L.attn_decode_q8.restype = ctypes.c_int
+        L.attn_decode_q8_workspace_bytes.argtypes = [i32, p64, i32]
+        L.attn_decode_q8_workspace_bytes.restype = sz
+        L.attn_dot_canary.argtypes = [vp, p32]
+        L.attn_dot_canary.restype = ctypes.c_int
         L.attn_decode_cluster_capacity.argtypes = [p32]
         L.attn_decode_cluster_capacity.restype = ctypes.c_int
         L.attn_force_path.argtypes = [i32, i32]
@@ -431,6 +440,73 @@ def attn_append_kv(k_new, v_new, k_cache, v_cache, dst, rope_cos=None, rope_sin=
                               vp(workspace.data_ptr()) if workspace is not None else None,
                               _stream_ptr(stream))
     _check(st, "attn_append_kv")
+
+
+# ------------------------------------------------------- quantised-dot decode
+
+def attn_quantize_k(k, out=None, stream=None):
+    """K rows [..., 256] (f32 / f16 / bf16, contiguous CUDA) -> packed int8
+    rows uint8 [..., 272]: 256 codes, the row's f32 scale, 12 zero bytes."""
+    import torch
+    if not k.is_cuda or not k.is_contiguous() or k.shape[-1] != HEAD_DIM:
+        raise ValueError("k must be a contiguous CUDA tensor with a last axis of 256")
+    n = k.numel() // HEAD_DIM
+    if out is None:
+        out = torch.empty((*k.shape[:-1], I8_ROW_BYTES), dtype=torch.uint8, device=k.device)
+    if out.dtype != torch.uint8 or not out.is_contiguous() or out.numel() != n * I8_ROW_BYTES:
+        raise ValueError("out must be a contiguous uint8 tensor [..., 272]")
+    st = lib().attn_quantize_k(ctypes.c_void_p(k.data_ptr()), dtype_code(k), n, ctypes.c_void_p(out.data_ptr()),
+                               _stream_ptr(stream, k.device))
+    _check(st, "attn_quantize_k")
+    return out
+
+
+def attn_dot_canary(stream=None) -> int:
+    """1 when the dp4a instruction passed the known-answer check on the
+    current device (the quantised decode uses it), 0 when only its emulation
+    did; raises when neither did."""
+    v = ctypes.c_int32(-1)
+    _check(lib().attn_dot_canary(_stream_ptr(stream), ctypes.byref(v)), "attn_dot_canary")
+    return int(v.value)
+
+
+def attn_decode_q8_workspace_bytes(ctx_len, window: int = 0) -> int:
+    nctx, ptr = _i64_array(ctx_len)
+    n = lib().attn_decode_q8_workspace_bytes(nctx, ptr, window)
+    if n == 0:
+        raise KcaError(-4, "attn_decode_q8_workspace_bytes")
+    return int(n)
+
+
+def attn_decode_q8(q, k8_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.0 / 16.0, out=None,
+                   workspace=None, stream=None):
+    """Quantised-dot decode: q [batch, 8, 256]; k8_cache uint8 [batch, capacity,
+    272] packed int8 rows (attn_quantize_k); v_cache [batch, capacity, 256];
+    returns out [batch, 8, 256] float32."""
+    import torch
+    batch = q.shape[0]
+    capacity = k8_cache.shape[1]
+    for t in (q, k8_cache, v_cache):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if k8_cache.dtype != torch.uint8 or k8_cache.shape[-1] != I8_ROW_BYTES or k8_cache.shape[0] != batch:
+        raise ValueError("k8_cache must be uint8 [batch, capacity, 272]")
+    if v_cache.shape[0] != batch or v_cache.shape[1] != capacity:
+        raise ValueError("v_cache must be [batch, capacity, 256]")
+    nctx, ptr = _i64_array(ctx_len)
+    if nctx != batch:
+        raise ValueError("ctx_len must have one entry per sequence")
+    if out is None:
+        out = torch.empty((batch, N_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(attn_decode_q8_workspace_bytes(ctx_len, window), q.device, stream)
+    vp = ctypes.c_void_p
+    st = lib().attn_decode_q8(vp(q.data_ptr()), dtype_code(q), vp(k8_cache.data_ptr()), vp(v_cache.data_ptr()),
+                              dtype_code(v_cache), N_Q_HEADS, N_KV_HEADS, HEAD_DIM, capacity, batch, ptr, window,
+                              scale, vp(out.data_ptr()), vp(workspace.data_ptr()), workspace.numel(),
+                              _stream_ptr(stream))
+    _check(st, "attn_decode_q8")
+    return out
 
 
 def attn_decode_static(q, k_cache, v_cache, ctx_len, window: int = 0, scale: float = 1.0 / 16.0,

@@ -28,10 +28,16 @@ constexpr int kStages = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 5.545177444479562f;  // 8 * ln 2: rescale once p could pass 256
 
+// K rows: 256 elements of KT, or packed int8 rows (KCA_I8: 256 codes, the
+// row's f32 scale, 12 bytes of padding); V rows: 256 elements of VT.
 template <int KT>
+struct KRowBytes { static constexpr int value = KT == KCA_I8 ? KCA_I8_ROW_BYTES : kDim * ElemBytes<KT>::value; };
+
+template <int KT, int VT = KT>
 struct RowsSmem {
-  static constexpr int kRowBytes = kDim * ElemBytes<KT>::value;
-  static constexpr int kStageBytes = 2 * kKeysPerStage * kRowBytes;   // K rows then V rows
+  static constexpr int kKRowBytes = KRowBytes<KT>::value;
+  static constexpr int kVRowBytes = kDim * ElemBytes<VT>::value;
+  static constexpr int kStageBytes = kKeysPerStage * (kKRowBytes + kVRowBytes);   // K rows then V rows
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kCombineBytes = kComputeWarps * kHeads * (kDim + 2) * 4;
   static constexpr int kDataBytes = kRingBytes > kCombineBytes ? kRingBytes : kCombineBytes;
@@ -64,9 +70,32 @@ __device__ __forceinline__ float reduce8_transposed(const float (&v)[8], int lan
   return r;
 }
 
-template <int QT, int KT>
+// Dot product of four packed int8 pairs plus c: the dp4a instruction, or
+// its emulation from the sign-extended bytes (the canary in kca_q8.cu picks
+// one per device).
+template <bool DP4A>
+__device__ __forceinline__ int dot4(uint32_t a, uint32_t b, int c) {
+  if (DP4A) return __dp4a(static_cast<int>(a), static_cast<int>(b), c);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    c += static_cast<int>(static_cast<int8_t>(a >> (8 * i))) * static_cast<int>(static_cast<int8_t>(b >> (8 * i)));
+  return c;
+}
+
+// int8 code of x under the row scale sx (the quantisation of kca_q8.cu):
+// round-half-even of the f32 quotient, clamped to +-127; 0 unless sx is
+// finite and positive.
+__device__ __forceinline__ uint32_t q8_code(float x, float sx) {
+  if (!(sx > 0.f) || !(sx <= 3.402823466e38f)) return 0u;
+  int c = __float2int_rn(__fdiv_rn(x, sx));
+  c = c > 127 ? 127 : (c < -127 ? -127 : c);
+  return static_cast<uint32_t>(c) & 0xffu;
+}
+
+template <int QT, int KT, int VT = KT, bool DP4A = true>
 __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a) {
-  using S = RowsSmem<KT>;
+  using S = RowsSmem<KT, VT>;
+  constexpr bool kQ8 = KT == KCA_I8;
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
   uint64_t* empty = full + kStages;
@@ -124,11 +153,12 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
           break;
         const int64_t k0 = kbeg + (int64_t)i * kKeysPerStage;
         const int cnt = (int)((kend - k0) < kKeysPerStage ? (kend - k0) : kKeysPerStage);
-        const uint32_t bytes = (uint32_t)cnt * S::kRowBytes;
+        const uint32_t kbytes = (uint32_t)cnt * S::kKRowBytes;
+        const uint32_t vbytes = (uint32_t)cnt * S::kVRowBytes;
         unsigned char* dst = smem + slot * S::kStageBytes;
-        mbar_arrive_expect_tx(&full[slot], 2 * bytes);
-        bulk_g2s(dst, kg + (base_row + k0) * S::kRowBytes, bytes, &full[slot]);
-        bulk_g2s(dst + kKeysPerStage * S::kRowBytes, vg + (base_row + k0) * S::kRowBytes, bytes,
+        mbar_arrive_expect_tx(&full[slot], kbytes + vbytes);
+        bulk_g2s(dst, kg + (base_row + k0) * S::kKRowBytes, kbytes, &full[slot]);
+        bulk_g2s(dst + kKeysPerStage * S::kKRowBytes, vg + (base_row + k0) * S::kVRowBytes, vbytes,
                  &full[slot]);
         issued = i + 1;
       }
@@ -143,7 +173,12 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
   } else {
     // ---------------------------------------------------------------- compute
     // Query of this row, all 8 heads, dims [8*lane, 8*lane+8), in f32.
-    float2 q2[kHeads][4];
+    // Quantised-dot variant: the int8 codes of the query (per head: scale
+    // amax * f32(1/127) over the head's 256 values) and this lane's head's
+    // scale; otherwise the query in f32.
+    float2 q2[kQ8 ? 1 : kHeads][4];
+    uint32_t qp[kQ8 ? kHeads : 1][2];
+    float sq_mine = 0.f;
     {
       const char* qrow = static_cast<const char*>(a.q) +
                          (int64_t)unit * kHeads * kDim * ElemBytes<QT>::value;
@@ -151,8 +186,22 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
       for (int h = 0; h < kHeads; ++h) {
         float x[8];
         load8<QT>(qrow + ((int64_t)h * kDim + 8 * lane) * ElemBytes<QT>::value, x);
+        if constexpr (kQ8) {
+          float am = fabsf(x[0]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) q2[h][i] = make_float2(x[2 * i], x[2 * i + 1]);
+          for (int i = 1; i < 8; ++i) am = max_nan(am, fabsf(x[i]));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) am = max_nan(am, __shfl_xor_sync(0xffffffffu, am, o));
+          const float sx = am * (1.0f / 127.0f);
+          if (h == ((lane >> 2) & 7)) sq_mine = sx;
+#pragma unroll
+          for (int w = 0; w < 2; ++w)
+            qp[h][w] = q8_code(x[4 * w], sx) | (q8_code(x[4 * w + 1], sx) << 8) |
+                       (q8_code(x[4 * w + 2], sx) << 16) | (q8_code(x[4 * w + 3], sx) << 24);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) q2[h][i] = make_float2(x[2 * i], x[2 * i + 1]);
+        }
       }
     }
     float2 acc[kHeads][4];
@@ -182,19 +231,31 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
         for (int c = 0; c < 2; ++c) {
           if (c < nk) {
             const int r = warp + c * kComputeWarps;
-            float kx[8];
-            load8<KT>(st + r * S::kRowBytes + 8 * lane * ElemBytes<KT>::value, kx);
-            load8<KT>(st + (kKeysPerStage + r) * S::kRowBytes + 8 * lane * ElemBytes<KT>::value,
+            const unsigned char* krow = st + r * S::kKRowBytes;
+            load8<VT>(st + kKeysPerStage * S::kKRowBytes + r * S::kVRowBytes + 8 * lane * ElemBytes<VT>::value,
                       vx[c]);
             float part[8];
+            if constexpr (kQ8) {
+              // exact integer dot products (|partial| < 2^24, so f32 holds
+              // them and their warp sum exactly), then the two scales
+              const uint2 kw = *reinterpret_cast<const uint2*>(krow + 8 * lane);
+              const float sk = *reinterpret_cast<const float*>(krow + kDim);
 #pragma unroll
-            for (int h = 0; h < kHeads; ++h) {
-              float2 d = make_float2(0.f, 0.f);
+              for (int h = 0; h < kHeads; ++h)
+                part[h] = static_cast<float>(dot4<DP4A>(qp[h][1], kw.y, dot4<DP4A>(qp[h][0], kw.x, 0)));
+              s_own[c] = reduce8_transposed(part, lane) * ((sq_mine * sk) * scale);
+            } else {
+              float kx[8];
+              load8<KT>(krow + 8 * lane * ElemBytes<KT>::value, kx);
 #pragma unroll
-              for (int t = 0; t < 4; ++t) d = ffma2(q2[h][t], make_float2(kx[2 * t], kx[2 * t + 1]), d);
-              part[h] = d.x + d.y;
+              for (int h = 0; h < kHeads; ++h) {
+                float2 d = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) d = ffma2(q2[h][t], make_float2(kx[2 * t], kx[2 * t + 1]), d);
+                part[h] = d.x + d.y;
+              }
+              s_own[c] = reduce8_transposed(part, lane) * scale;
             }
-            s_own[c] = reduce8_transposed(part, lane) * scale;
           } else {
             s_own[c] = -INFINITY;
 #pragma unroll
@@ -312,10 +373,10 @@ __global__ void __launch_bounds__(256) merge_rows_kernel(const RowsArgs a) {
                threadIdx.x & 31, 1, a.out_ml != nullptr ? a.out_ml + ((int64_t)unit * kHeads + h) * 2 : nullptr);
 }
 
-template <int QT, int KT>
+template <int QT, int KT, int VT = KT, bool DP4A = true>
 cudaError_t launch_rows_t(const RowsArgs& a, cudaStream_t stream) {
-  using S = RowsSmem<KT>;
-  auto kern = rows_kernel<QT, KT>;
+  using S = RowsSmem<KT, VT>;
+  auto kern = rows_kernel<QT, KT, VT, DP4A>;
   static std::atomic<bool> attr_set[64];   // per device; zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -352,6 +413,23 @@ cudaError_t launch_rows(int q_dtype, int kv_dtype, const RowsArgs& a, cudaStream
   KCA_ROWS_CASE(KCA_BF16, KCA_F16)
   KCA_ROWS_CASE(KCA_BF16, KCA_BF16)
 #undef KCA_ROWS_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_rows_q8(int q_dtype, int v_dtype, bool dp4a, const RowsArgs& a, cudaStream_t stream) {
+#define KCA_Q8_CASE(QD, VD)                                                              \
+  if (q_dtype == QD && v_dtype == VD)                                                    \
+    return dp4a ? launch_rows_t<QD, KCA_I8, VD, true>(a, stream) : launch_rows_t<QD, KCA_I8, VD, false>(a, stream);
+  KCA_Q8_CASE(KCA_F32, KCA_F32)
+  KCA_Q8_CASE(KCA_F32, KCA_F16)
+  KCA_Q8_CASE(KCA_F32, KCA_BF16)
+  KCA_Q8_CASE(KCA_F16, KCA_F32)
+  KCA_Q8_CASE(KCA_F16, KCA_F16)
+  KCA_Q8_CASE(KCA_F16, KCA_BF16)
+  KCA_Q8_CASE(KCA_BF16, KCA_F32)
+  KCA_Q8_CASE(KCA_BF16, KCA_F16)
+  KCA_Q8_CASE(KCA_BF16, KCA_BF16)
+#undef KCA_Q8_CASE
   return cudaErrorInvalidValue;
 }
 

@@ -111,6 +111,11 @@ __device__ __forceinline__ int32_t rows_split_len(const RowsArgs& a, int64_t nke
 
 cudaError_t launch_rows(int q_dtype, int kv_dtype, const RowsArgs& a, cudaStream_t stream);
 
+// The CUDA-core rows kernel with packed int8 K rows (KCA_I8) and V of
+// v_dtype: the quantised-dot variant; dp4a selects the instruction over its
+// emulation (kca_q8.cu).  Merges its splits like launch_rows.
+cudaError_t launch_rows_q8(int q_dtype, int v_dtype, bool dp4a, const RowsArgs& a, cudaStream_t stream);
+
 // Log-sum-exp merge of the split partials in a (units with more than one split).
 cudaError_t launch_merge_rows(const RowsArgs& a, cudaStream_t stream);
 

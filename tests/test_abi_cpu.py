@@ -71,7 +71,7 @@ def test_header_constants_match_binding():
     for name, val in [("KCA_MAX_CHUNK_ROWS", 768), ("KCA_MAX_POSITION", 131072),
                       ("KCA_HEAD_DIM", 256), ("KCA_N_Q_HEADS", 8), ("KCA_N_KV_HEADS", 1),
                       ("KCA_WORKSPACE_HEADER", 24832), ("KCA_MAX_BATCH", 256),
-                      ("KCA_MAX_BATCH_ROWS", 15)]:
+                      ("KCA_MAX_BATCH_ROWS", 15), ("KCA_I8", 3), ("KCA_I8_ROW_BYTES", 272)]:
         assert re.search(rf"#define {name} {val}\b", text), name
 
 
@@ -157,6 +157,37 @@ def _prefill_batch(ctx=(100, 200), rows=3, **kw):
 ])
 def test_prefill_batch_rejects_bad_arguments_on_the_host(ctx, rows, kw, code):
     assert _prefill_batch(ctx, rows, **kw) == code
+
+
+def _decode_q8(ctx=(100, 200), **kw):
+    a = dict(q=P, qd=kca.F32, k=P, v=P, vd=kca.F16, hq=8, hkv=1, d=256, cap=4096, window=0,
+             scale=0.0625, out=P, ws=P * 2, wsb=1 << 30, batch=None)
+    a.update(kw)
+    arr = np.asarray(ctx, dtype=np.int64)
+    batch = len(arr) if a["batch"] is None else a["batch"]
+    vp = ctypes.c_void_p
+    return kca.lib().attn_decode_q8(vp(a["q"]), a["qd"], vp(a["k"]), vp(a["v"]), a["vd"], a["hq"], a["hkv"],
+                                    a["d"], a["cap"], batch, arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                    a["window"], a["scale"], vp(a["out"]), vp(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("ctx,kw,code", [
+    ((1, 2), dict(k=0), -1), ((1, 2), dict(ws=0), -1), ((1, 2), dict(hq=4), -2),
+    ((1, 2), dict(vd=3), -3), ((1, 2), dict(qd=3), -3), ((1, 4097), dict(), -4), ((1, 2), dict(batch=0), -4),
+    ((1, 2), dict(scale=float("nan")), -4), ((1, 2), dict(k=P + 8), -6), ((1, 2), dict(ws=P * 2 + 32), -5),
+])
+def test_decode_q8_rejects_bad_arguments_on_the_host(ctx, kw, code):
+    assert _decode_q8(ctx, **kw) == code
+
+
+def test_quantize_k_rejects_bad_arguments_on_the_host():
+    lib = kca.lib()
+    vp = ctypes.c_void_p
+    assert lib.attn_quantize_k(None, kca.F32, 4, vp(P), None) == -1
+    assert lib.attn_quantize_k(vp(P), 3, 4, vp(P), None) == -3
+    assert lib.attn_quantize_k(vp(P), kca.F16, 0, vp(P), None) == -4
+    assert lib.attn_quantize_k(vp(P), kca.F16, 4, vp(P + 4), None) == -6
+    assert lib.attn_dot_canary(None, None) == -1
 
 
 def test_prefill_batch_workspace_query_rejects_bad_arguments():
