@@ -28,6 +28,8 @@ rows from HBM) and reported in its own object of the JSON line:
                  131,072-row cache
   prefill_batch  32 sequences x 4 query rows (speculative / multi-row decode)
                  per call through attn_prefill_batch, 16 calls, f16 K/V
+  decode_q8_ragged  the ragged batch with int8 K rows (quantised-dot decode,
+                 attn_decode_q8), f16 V
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--passes P] [--impl reference]
 Under torchrun each rank runs its own replica of the workload (weak scaling,
@@ -533,8 +535,46 @@ class BatchRowsPart(Part):
         return [self.ws]
 
 
+class RaggedQ8Part(Part):
+    """The ragged batch with int8 K (quantised-dot decode): K quantised per
+    row by attn_quantize_k (272-byte packed rows), f16 V, f32 q, 32 steps."""
+    name, unit, bound = "decode_q8_ragged", "tok", "hbm"
+    kernel = "decode_mma_kernel<f32 q, int8 K, f16 V> (QK on int8 MMAs)"
+
+    def __init__(self, device):
+        import torch
+        import kv_cache_attention_states_b200 as kca
+        from kv_cache_attention_states_b200 import synth
+        self.kca = kca
+        wl = synth.ragged_f16(0)
+        self.wl = wl
+        g = torch.Generator(device=device)
+        g.manual_seed(3)
+        k = torch.randn((wl.batch, wl.capacity, 256), generator=g, device=device).half()
+        self.k8 = kca.attn_quantize_k(k)
+        del k
+        self.v = torch.randn((wl.batch, wl.capacity, 256), generator=g, device=device).half()
+        self.q = torch.randn((len(wl.decode_ctx), wl.batch, 8, 256), generator=g, device=device)
+        self.out = torch.empty_like(self.q)
+        self.ws = kca.new_workspace(max(kca.attn_decode_q8_workspace_bytes(c) for c in wl.decode_ctx), device)
+        kca.attn_dot_canary()
+        self.units = wl.batch * len(wl.decode_ctx)
+        self.work = float(sum(sum(x * (272 + 512) + 8 * 256 * 8 for x in c) for c in wl.decode_ctx))
+        self.launches = len(wl.decode_ctx)
+        self.algorithmic = "ctx*(272 B int8 K row + 512 B f16 V row) + 16 KiB q/out per token"
+        self.workload = ("the ragged batch (8 sequences, ctx drawn by the seed from [1024, 131072], 32 steps) "
+                         "with int8 K (per-row scale) and f16 V, f32 q (attn_decode_q8)")
+
+    def run(self, variant):
+        for t, c in enumerate(self.wl.decode_ctx):
+            self.kca.attn_decode_q8(self.q[t], self.k8, self.v, c, out=self.out[t], workspace=self.ws)
+
+    def workspaces(self):
+        return [self.ws]
+
+
 PART_NAMES = ["decode_ragged", "decode_256", "decode_4096", "prefill", "decode", "window_prefill",
-              "window_decode", "long_chunk", "prefill_batch"]
+              "window_decode", "long_chunk", "prefill_batch", "decode_q8_ragged"]
 
 
 def build_parts(w, device, sms, only=None):
@@ -559,6 +599,8 @@ def build_parts(w, device, sms, only=None):
         parts.append(LongChunkPart(device, sms))
     if want("prefill_batch"):
         parts.append(BatchRowsPart(device))
+    if want("decode_q8_ragged"):
+        parts.append(RaggedQ8Part(device))
     return parts
 
 
@@ -878,6 +920,17 @@ def oracle_part_samples(seed=0):
     base = np.repeat(starts, rows)
     sec = _timed(lambda: oracle.attention(q, k, v, pos, base, kv_dtype="f16", scale=synth.SCALE))
     out["prefill_batch"] = (pos.size / sec, f"sequences 0-3 of the first call, 4 rows each ({sec:.2f} s)")
+    from oracle import quant
+    wl = synth.ragged_f16(seed)
+    ctx = wl.decode_ctx[0][:2]
+    kq = np.concatenate([synth.normal(seed, f"qk{b}", (c, 256)) for b, c in enumerate(ctx)])
+    codes, scales = quant.quantize_rows(kq)
+    v = np.concatenate([synth.draw(seed, f"qv{b}", (c, 256), "f16") for b, c in enumerate(ctx)])
+    q = synth.draw(seed, "qq", (2, 8, 256), "f32")
+    sec = _timed(lambda: quant.attention_q8(q, "f32", codes, scales, v, "f16", np.array(ctx) - 1,
+                                            np.array([0, ctx[0]]), scale=synth.SCALE))
+    out["decode_q8_ragged"] = (2 / sec, f"sequences 0-1 of the first step, quantised-dot oracle (numpy f64; "
+                                        f"{sec:.2f} s)")
     return out, cores
 
 
@@ -987,7 +1040,8 @@ def main():
         samples, cores = oracle_part_samples()
         parts_cpu = {nm: {"value": v, "unit": ("q-rows/s" if nm in ("window_prefill", "long_chunk", "prefill_batch")
                                                    else "tok/s"),
-                          "cores": cores, "kind": "oracle", "sample": d + "; f64 C oracle, OpenMP over (row, head)"}
+                          "cores": cores if "numpy" not in d else 1, "kind": "oracle",
+                          "sample": d if "numpy" in d else d + "; f64 C oracle, OpenMP over (row, head)"}
                      for nm, (v, d) in samples.items()}
         parts_cpu["decode"] = {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
                                "sample": desc}
@@ -1018,7 +1072,7 @@ def main():
                    "value": "prefill part of every pass (CUDA events); the 16K decode in 'decode'",
                    "other_configurations": f"timed after the main region, {res['other_passes']} passes per step "
                                            f"over ragged, decode_256, decode_4096, window, long_chunk, "
-                                           f"prefill_batch ({res['other_ms'] / K:.1f} ms per step, "
+                                           f"prefill_batch, decode_q8_ragged ({res['other_ms'] / K:.1f} ms per step, "
                                            f"{res['other_launches']} launches, clocks {res['other_clocks']})",
                    "launch": "eager" if args.eager else "one CUDA graph per configuration of the C-ABI calls",
                    "l2": "inputs larger than L2: the 16K decode rotates 32 cache replicas (16.8 MB "
@@ -1035,6 +1089,7 @@ def main():
         "long_chunk": obj("long_chunk"),
         "decode_ragged": obj("decode_ragged"),
         "prefill_batch": obj("prefill_batch"),
+        "decode_q8_ragged": obj("decode_q8_ragged"),
         "e2e": {"value": world * PREFILL_ROWS * e2e["steps"] / (e2e["pre_ms"] / 1e3), "unit": "q-rows/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "decode_tok_s": world * DECODE_STEPS * e2e["steps"] / (e2e["dec_ms"] / 1e3),

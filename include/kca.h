@@ -372,16 +372,20 @@ int attn_merge_partials(int32_t n_parts, int32_t batch, const float *parts, int6
  *   row by row (row b * capacity + p of sequence b at position p).
  * attn_decode_q8: attn_decode with a packed int8 K cache k8_cache
  *   [batch][capacity][KCA_I8_ROW_BYTES] and v_cache [batch][capacity][256] of
- *   v_dtype (F32, F16 or BF16); q of any dtype, out f32; the plan, workspace
- *   (attn_decode_q8_workspace_bytes), errors and semantics of attn_decode
- *   (CUDA-core kernel).  The first call on a device runs the canary below
- *   (a synchronising launch): make it, or call attn_dot_canary, before any
- *   stream capture.
- * attn_dot_canary: runs, once per device, the dp4a instruction and its
- *   emulation on known answers; *variant = 1 when the instruction is right
- *   (the decode uses it), 0 when only the emulation is (the decode uses the
- *   emulation); KCA_ERR_DEVICE, and attn_decode_q8 refuses to run, when
- *   neither is.  Synchronises `stream` on its first call per device.
+ *   v_dtype (F32, F16 or BF16); q of any dtype, out f32; the workspace
+ *   (attn_decode_q8_workspace_bytes), errors and semantics of attn_decode.
+ *   16-bit V runs the tensor-core decode kernel with the QK product on int8
+ *   MMAs (the plan of attn_decode for that V dtype); f32 V (or the CUDA-core
+ *   kernel pinned by attn_force_path) runs the CUDA-core kernel with dp4a.
+ *   The first call on a device runs the canary below (a synchronising
+ *   launch): make it, or call attn_dot_canary, before any stream capture.
+ * attn_dot_canary: runs, once per device, the dp4a instruction, its
+ *   emulation and the int8 MMA on known answers; *variant receives the mask
+ *   of the sane ones (1 dp4a, 2 its emulation, 4 int8 MMA).  The decode
+ *   takes the int8 MMA only when it is sane (else the CUDA-core kernel), and
+ *   the emulation where dp4a is not; with neither dp4a nor its emulation
+ *   sane the call returns KCA_ERR_DEVICE and attn_decode_q8 refuses to run.
+ *   Synchronises `stream` on its first call per device.
  */
 int attn_quantize_k(const void *k, int32_t k_dtype, int64_t n_rows, void *k8, void *stream);
 int attn_decode_q8(const void *q, int32_t q_dtype, const void *k8_cache, const void *v_cache,

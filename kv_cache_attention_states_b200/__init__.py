@@ -462,9 +462,9 @@ def attn_quantize_k(k, out=None, stream=None):
 
 
 def attn_dot_canary(stream=None) -> int:
-    """1 when the dp4a instruction passed the known-answer check on the
-    current device (the quantised decode uses it), 0 when only its emulation
-    did; raises when neither did."""
+    """Mask of the dot-product variants that passed the known-answer check on
+    the current device: 1 the dp4a instruction, 2 its emulation, 4 the int8
+    tensor-core MMA; raises when neither dp4a nor its emulation did."""
     v = ctypes.c_int32(-1)
     _check(lib().attn_dot_canary(_stream_ptr(stream), ctypes.byref(v)), "attn_dot_canary")
     return int(v.value)

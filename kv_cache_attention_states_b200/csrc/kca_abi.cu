@@ -166,13 +166,15 @@ EncodeTiledFn encode_fn() {
 // same cache or chunk buffer call after call) is copied instead of
 // re-encoded.  All maps here are 2-D, 128-byte swizzled, zero-filled.
 bool encode_2d(CUtensorMap* m, CUtensorMapDataType t, const void* base, const cuuint64_t (&dims)[2],
-               cuuint64_t stride, const cuuint32_t (&box)[2]) {
+               cuuint64_t stride, const cuuint32_t (&box)[2],
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   struct Entry {
     const void* base;
     cuuint64_t dims[2];
     cuuint64_t stride;
     cuuint32_t box[2];
     int t;
+    int swizzle;
     bool valid;
     CUtensorMap map;
   };
@@ -182,7 +184,7 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType t, const void* base, const cu
   for (int i = 0; i < kEntries; ++i) {
     const Entry& e = cache[i];
     if (e.valid && e.base == base && e.t == (int)t && e.dims[0] == dims[0] && e.dims[1] == dims[1] &&
-        e.stride == stride && e.box[0] == box[0] && e.box[1] == box[1]) {
+        e.stride == stride && e.box[0] == box[0] && e.box[1] == box[1] && e.swizzle == (int)swizzle) {
       *m = e.map;
       return true;
     }
@@ -191,9 +193,8 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType t, const void* base, const cu
   if (fn == nullptr) return false;
   cuuint64_t strides[1] = {stride};
   cuuint32_t estr[2] = {1, 1};
-  if (fn(m, t, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  if (fn(m, t, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   Entry& e = cache[next];
   next = (next + 1) % kEntries;
@@ -204,6 +205,7 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType t, const void* base, const cu
   e.box[0] = box[0];
   e.box[1] = box[1];
   e.t = (int)t;
+  e.swizzle = (int)swizzle;
   e.map = *m;
   e.valid = true;
   return true;
@@ -835,6 +837,76 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
   for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
   return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster, workspace,
                           static_cast<cudaStream_t>(stream));
+}
+
+size_t attn_decode_q8_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_t window) {
+  // the same plans as attn_decode: the CUDA-core kernel's for f32 V, the
+  // tensor-core kernel's for 16-bit V, and the larger of the two
+  return attn_decode_workspace_bytes(batch, ctx_len, window);
+}
+
+int attn_decode_q8(const void* q, int32_t q_dtype, const void* k8_cache, const void* v_cache, int32_t v_dtype,
+                   int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity, int32_t batch,
+                   const int64_t* ctx_len, int32_t window, float scale, float* out, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (!workspace) return KCA_ERR_NULL;
+  int st = kca::decode_args_check(q, q_dtype, k8_cache, v_cache, v_dtype, n_q_heads, n_kv_heads, head_dim, capacity,
+                                  batch, ctx_len, scale, out);
+  if (st != KCA_OK) return st;
+  if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
+  int sms = 0;
+  if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+  const std::vector<int64_t> nk = decode_unit_keys(batch, ctx_len, window);
+  int cluster = 1;
+  size_t need = 0;
+  const kca::RowsPlan p = rows_plan(v_dtype, batch, nk.data(), sms, &cluster, &need);
+  if (cluster < 1) return KCA_ERR_CUDA;
+  if (workspace_bytes < need) return KCA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  kca::RowsArgs a{};
+  a.q = q;
+  a.k = k8_cache;
+  a.v = v_cache;
+  a.out = out;
+  a.status = workspace;
+  a.seq_rows = capacity;
+  a.mode = 0;
+  a.n_units = batch;
+  a.split_len = p.split_len;
+  a.max_splits = p.max_splits;
+  a.window = window;
+  a.scale = scale;
+  for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
+  int sane = 0;
+  st = kca::dot_canary(s, &sane);
+  if (st != KCA_OK) return st;
+  if (use_rows_mma(v_dtype) && (sane & 4)) {
+    // 16-bit V: the tensor-core kernel, QK on int8 MMAs (exact integers)
+    a.cluster = cluster;
+    a.max_clusters = (a.max_splits + cluster - 1) / cluster;
+    if (a.max_clusters > 1) {
+      a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+      carve(workspace, (size_t)a.n_units * a.max_clusters * kHeads * 2 * 4, &a.cpart_ml, &a.cpart_acc);
+    }
+    const int64_t rows = (int64_t)batch * capacity;
+    const cuuint64_t kdims[2] = {(cuuint64_t)KCA_I8_ROW_BYTES, (cuuint64_t)rows};
+    const cuuint32_t kbox[2] = {128, 64}, sbox[2] = {16, 64};
+    CUtensorMap tmk, tms, tmv;
+    if (!encode_2d(&tmk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k8_cache, kdims, KCA_I8_ROW_BYTES, kbox) ||
+        !encode_2d(&tms, CU_TENSOR_MAP_DATA_TYPE_UINT8, k8_cache, kdims, KCA_I8_ROW_BYTES, sbox,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_kv_map(&tmv, v_cache, v_dtype, 0, rows, 64))
+      return KCA_ERR_CUDA;
+    return kca::launch_decode_mma_q8(q_dtype, v_dtype, tmk, tms, tmv, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+  }
+  // f32 V, the CUDA-core kernel pinned, or an int8 MMA the canary found
+  // wrong: dp4a on the CUDA cores, or its emulation where the instruction
+  // is the one found wrong.  This kernel's plan is the CUDA-core one.
+  const kca::RowsPlan pc = kca::make_rows_plan(batch, nk.data(), sms);
+  a.split_len = pc.split_len;
+  a.max_splits = pc.max_splits;
+  carve(workspace, (size_t)a.n_units * a.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
+  return kca::launch_rows_q8(q_dtype, v_dtype, (sane & 1) != 0, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
 }
 
 int attn_merge_partials(int32_t n_parts, int32_t batch, const float* parts, int64_t part_stride, float* out,

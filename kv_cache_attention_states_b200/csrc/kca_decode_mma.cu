@@ -65,7 +65,8 @@ struct DBars {
   float red[kDWarps][8];                 // per-warp stage max (then row sums) per head
   int last;                              // this CTA holds the last ticket of its unit
   __align__(16) unsigned char p[16 * kDPRow];   // P: rows 0-7 hi, 8-15 lo, 64 keys
-  __align__(16) unsigned char qs[16 * kDQRow];  // Q: rows 0-7 hi, 8-15 lo, 256 dims
+  __align__(16) unsigned char qs[16 * kDQRow];  // Q: rows 0-7 hi, 8-15 lo, 256 dims (int8 K: 8 rows of codes)
+  float sq[8];                           // int8 K: the query's per-head scales
   // Partials this CTA receives for the heads it owns: slot src * (8 / C) + i
   // holds CTA src's reference max (natural units), row sum and unnormalised
   // output of head rank + i * C.  Written by the cluster's CTAs (distributed
@@ -137,6 +138,34 @@ __device__ __forceinline__ uint32_t swz(int row, int dim) {
   return (uint32_t)((dim >> 6) * kDBoxBytes + row * 128 + ((unit ^ (row & 7)) << 4));
 }
 
+
+// Byte offset of code byte c (0..255) of key row `row` in the packed int8 K
+// half of a stage: two 128-code boxes of 64 rows, 128-byte swizzle.  The
+// rows' f32 scales follow at kDQ8ScaleOff, 16 bytes per row (unswizzled).
+__device__ __forceinline__ uint32_t swz8(int row, int c) {
+  return (uint32_t)((c >> 7) * kDBoxBytes + row * 128 + ((((c & 127) >> 4) ^ (row & 7)) << 4));
+}
+constexpr int kDQ8ScaleOff = 2 * kDBoxBytes;                 // 16 KiB into the K half
+constexpr int kDQ8StageTx = 2 * kDBoxBytes + 64 * 16 + kDHalfBytes;   // codes + scales + V
+
+// D = A(16x32) B(32x8) + D on int8 codes, exact int32 accumulation.
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+// int8 code of x under scale sx (round half to even of the f32 quotient,
+// clamped to +-127; 0 unless sx is finite and > 0) -- the quantisation of
+// attn_quantize_k.
+__device__ __forceinline__ uint32_t dq8_code(float x, float sx) {
+  if (!(sx > 0.f) || !(sx <= 3.402823466e38f)) return 0u;
+  int c = __float2int_rn(__fdiv_rn(x, sx));
+  c = c > 127 ? 127 : (c < -127 ? -127 : c);
+  return static_cast<uint32_t>(c) & 0xffu;
+}
 
 // Split cluster barrier: every thread of every CTA of the cluster arrives,
 // and waits for the others' arrival.
@@ -262,10 +291,15 @@ __device__ __forceinline__ void merge_cluster_partials_nb(const RowsArgs& a, flo
   else merge_cluster_partials<W, 32>(a, sm_m, sm_l, u0, unit, rank, C, nh, d, nclus, lane);
 }
 
-template <int QT, int KT>
+// KT: K element type, or KCA_I8 for packed int8 K rows (the quantised-dot
+// variant: QK on int8 codes with exact int32 MMA, scaled by the query's and
+// the key's scales); VT: V element type (16-bit); tms: the int8 rows' scale
+// column (unused otherwise).
+template <int QT, int KT, int VT = KT>
 __global__ void __launch_bounds__(kDThreads, 1)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                      const RowsArgs a) {
+                      const __grid_constant__ CUtensorMap tms, const RowsArgs a) {
+  constexpr bool kQ8 = KT == KCA_I8;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -319,15 +353,18 @@ __global__ void __launch_bounds__(kDThreads, 1)
     // still writes are read after the wait below all the same.
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+    if (kQ8) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tms)) : "memory");
     if (active) {
       int64_t n = kend - kbeg;
       if (n > kDPrefetchKeys) n = kDPrefetchKeys;
-      const int64_t off = (base_row + kbeg) * (kDim * 2);
-      const uint32_t bytes = (uint32_t)(n * kDim * 2);
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char*>(a.k) + off),
-                   "r"(bytes) : "memory");
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char*>(a.v) + off),
-                   "r"(bytes) : "memory");
+      constexpr int kKRow = kQ8 ? KCA_I8_ROW_BYTES : kDim * 2;
+      const uint32_t kbytes = (uint32_t)(n * kKRow), vbytes = (uint32_t)(n * kDim * 2);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char*>(a.k) +
+                                                                      (base_row + kbeg) * kKRow),
+                   "r"(kbytes) : "memory");
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char*>(a.v) +
+                                                                      (base_row + kbeg) * (kDim * 2)),
+                   "r"(vbytes) : "memory");
     }
   }
   __syncthreads();
@@ -352,11 +389,20 @@ __global__ void __launch_bounds__(kDThreads, 1)
         const uint32_t kst = sbase + slot * kDStageBytes;
         const uint32_t bar = smem_u32(&bars->full[slot]);
         const int32_t row0 = (int32_t)(base_row + kbeg + (int64_t)i * kDStageKeys);
-        mbar_arrive_expect_tx(&bars->full[slot], kDStageBytes);
+        if constexpr (kQ8) {
+          mbar_arrive_expect_tx(&bars->full[slot], kDQ8StageTx);
+          tma2d(kst, &tmk, 0, row0, bar);                  // codes 0..127
+          tma2d(kst + kDBoxBytes, &tmk, 128, row0, bar);   // codes 128..255
+          tma2d(kst + kDQ8ScaleOff, &tms, kDim, row0, bar);   // scale (+ padding)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tma2d(kst + c * kDBoxBytes, &tmk, 64 * c, row0, bar);
-          tma2d(kst + kDHalfBytes + c * kDBoxBytes, &tmv, 64 * c, row0, bar);
+          for (int c = 0; c < 4; ++c) tma2d(kst + kDHalfBytes + c * kDBoxBytes, &tmv, 64 * c, row0, bar);
+        } else {
+          mbar_arrive_expect_tx(&bars->full[slot], kDStageBytes);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            tma2d(kst + c * kDBoxBytes, &tmk, 64 * c, row0, bar);
+            tma2d(kst + kDHalfBytes + c * kDBoxBytes, &tmv, 64 * c, row0, bar);
+          }
         }
         issued = i + 1;
       }
@@ -385,27 +431,55 @@ __global__ void __launch_bounds__(kDThreads, 1)
     const int g = lane >> 2, tig = lane & 3;
     // A operand of S = Q K^T: rows 0-7 the 16-bit high parts of the 8 heads,
     // rows 8-15 the remainders; per k-step: (g, 2tig), (g+8, 2tig), (g, 2tig+8), (g+8, 2tig+8).
-    uint32_t qa[16][4];
+    uint32_t qa[kQ8 ? 1 : 16][4];
+    // int8 K: the A operand of S = Q K^T is the 8 heads' int8 codes (rows
+    // 8-15 zero); per 32-dim k-step thread (g, tig) holds bytes 4 tig .. and
+    // 16 + 4 tig .. of head g.
+    uint32_t qa8[kQ8 ? 8 : 1][2];
+    float sq_g = 0.f;
     {
       // Stage the split query once, coalesced (thread t: 8 dims of head
       // t / 32), then every warp takes its A fragments with ldmatrix.
       const int h = threadIdx.x >> 5, d0 = 8 * (threadIdx.x & 31);
       float x[8];
       load8<QT>(static_cast<const char*>(a.q) + ((int64_t)unit * kHeads * kDim + h * kDim + d0) * ElemBytes<QT>::value, x);
-      uint32_t hi[4], lo[4];
+      if constexpr (kQ8) {
+        // the head's scale amax * f32(1/127) over its 256 dims (warp h holds head h)
+        float am = fabsf(x[0]);
   #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        hi[j] = pack16<KT>(x[2 * j], x[2 * j + 1]);
-        const float2 f = unpack16<KT>(hi[j]);
-        lo[j] = pack16<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
+        for (int j = 1; j < 8; ++j) am = max_nan(am, fabsf(x[j]));
+  #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = max_nan(am, __shfl_xor_sync(0xffffffffu, am, o));
+        const float sx = am * (1.0f / 127.0f);
+        if ((threadIdx.x & 31) == 0) bars->sq[h] = sx;
+        const uint32_t w0 = dq8_code(x[0], sx) | (dq8_code(x[1], sx) << 8) | (dq8_code(x[2], sx) << 16) |
+                            (dq8_code(x[3], sx) << 24);
+        const uint32_t w1 = dq8_code(x[4], sx) | (dq8_code(x[5], sx) << 8) | (dq8_code(x[6], sx) << 16) |
+                            (dq8_code(x[7], sx) << 24);
+        *reinterpret_cast<uint2*>(bars->qs + h * kDim + d0) = make_uint2(w0, w1);
+        asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+  #pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          qa8[ks][0] = *reinterpret_cast<const uint32_t*>(bars->qs + g * kDim + 32 * ks + 4 * tig);
+          qa8[ks][1] = *reinterpret_cast<const uint32_t*>(bars->qs + g * kDim + 32 * ks + 16 + 4 * tig);
+        }
+        sq_g = bars->sq[g];
+      } else {
+        uint32_t hi[4], lo[4];
+  #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          hi[j] = pack16<KT>(x[2 * j], x[2 * j + 1]);
+          const float2 f = unpack16<KT>(hi[j]);
+          lo[j] = pack16<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
+        }
+        *reinterpret_cast<uint4*>(bars->qs + h * kDQRow + d0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(bars->qs + (h + 8) * kDQRow + d0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+        const int mi = lane >> 3;
+        const uint32_t qrow = smem_u32(bars->qs) + (8 * (mi & 1) + (lane & 7)) * kDQRow + 8 * (mi >> 1) * 2;
+  #pragma unroll
+        for (int ks = 0; ks < 16; ++ks) ldsm_x4(qrow + 32 * ks, qa[ks]);
       }
-      *reinterpret_cast<uint4*>(bars->qs + h * kDQRow + d0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(bars->qs + (h + 8) * kDQRow + d0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
-      const int mi = lane >> 3;
-      const uint32_t qrow = smem_u32(bars->qs) + (8 * (mi & 1) + (lane & 7)) * kDQRow + 8 * (mi >> 1) * 2;
-  #pragma unroll
-      for (int ks = 0; ks < 16; ++ks) ldsm_x4(qrow + 32 * ks, qa[ks]);
     }
     float o[4][4];
   #pragma unroll
@@ -436,26 +510,43 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 make_uint4(0, 0, 0, 0);
           }
         }
-        // Four independent accumulation chains over d (shorter latency).
-        float sacc[4][4];
-  #pragma unroll
-        for (int c = 0; c < 4; ++c)
-  #pragma unroll
-          for (int j = 0; j < 4; ++j) sacc[c][j] = 0.f;
         const int kr = 8 * warp + (lane & 7);
-  #pragma unroll
-        for (int ks2 = 0; ks2 < 8; ++ks2) {
-          uint32_t b[4];
-          ldsm_x4(kst + swz(kr, 32 * ks2 + 8 * (lane >> 3)), b);
-          mma16816<KT>(sacc[(2 * ks2) & 3], qa[2 * ks2], b[0], b[1]);
-          mma16816<KT>(sacc[(2 * ks2 + 1) & 3], qa[2 * ks2 + 1], b[2], b[3]);
-        }
-        float st[4];
-  #pragma unroll
-        for (int j = 0; j < 4; ++j) st[j] = (sacc[0][j] + sacc[1][j]) + (sacc[2][j] + sacc[3][j]);
         const int kk0 = 8 * warp + 2 * tig;
-        sx0 = kk0 < cnt ? (st[0] + st[2]) * scale : -INFINITY;
-        sx1 = kk0 + 1 < cnt ? (st[1] + st[3]) * scale : -INFINITY;
+        if constexpr (kQ8) {
+          // exact integer dot products of the codes, two chains
+          int iacc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+  #pragma unroll
+          for (int kc = 0; kc < 4; ++kc) {
+            uint32_t b[4];
+            ldsm_x4(kst + swz8(kr, 64 * kc + 16 * (lane >> 3)), b);
+            mma_s8(iacc[0], qa8[2 * kc][0], qa8[2 * kc][1], b[0], b[1]);
+            mma_s8(iacc[1], qa8[2 * kc + 1][0], qa8[2 * kc + 1][1], b[2], b[3]);
+          }
+          const unsigned char* sc = smem + slot * kDStageBytes + kDQ8ScaleOff;
+          const float sk0 = *reinterpret_cast<const float*>(sc + kk0 * 16);
+          const float sk1 = *reinterpret_cast<const float*>(sc + (kk0 + 1) * 16);
+          sx0 = kk0 < cnt ? static_cast<float>(iacc[0][0] + iacc[1][0]) * ((sq_g * sk0) * scale) : -INFINITY;
+          sx1 = kk0 + 1 < cnt ? static_cast<float>(iacc[0][1] + iacc[1][1]) * ((sq_g * sk1) * scale) : -INFINITY;
+        } else {
+          // Four independent accumulation chains over d (shorter latency).
+          float sacc[4][4];
+  #pragma unroll
+          for (int c = 0; c < 4; ++c)
+  #pragma unroll
+            for (int j = 0; j < 4; ++j) sacc[c][j] = 0.f;
+  #pragma unroll
+          for (int ks2 = 0; ks2 < 8; ++ks2) {
+            uint32_t b[4];
+            ldsm_x4(kst + swz(kr, 32 * ks2 + 8 * (lane >> 3)), b);
+            mma16816<KT>(sacc[(2 * ks2) & 3], qa[2 * ks2], b[0], b[1]);
+            mma16816<KT>(sacc[(2 * ks2 + 1) & 3], qa[2 * ks2 + 1], b[2], b[3]);
+          }
+          float st[4];
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) st[j] = (sacc[0][j] + sacc[1][j]) + (sacc[2][j] + sacc[3][j]);
+          sx0 = kk0 < cnt ? (st[0] + st[2]) * scale : -INFINITY;
+          sx1 = kk0 + 1 < cnt ? (st[1] + st[3]) * scale : -INFINITY;
+        }
       }
       float mw = max_nan(sx0, sx1);
       mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 1));
@@ -479,9 +570,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
         const float p0 = exp2f((sx0 - mu) * kDLog2e);
         const float p1 = exp2f((sx1 - mu) * kDLog2e);
         l_part += p0 + p1;
-        const uint32_t hi = pack16<KT>(p0, p1);
-        const float2 f = unpack16<KT>(hi);
-        const uint32_t lo16 = pack16<KT>(p0 - f.x, p1 - f.y);
+        const uint32_t hi = pack16<VT>(p0, p1);
+        const float2 f = unpack16<VT>(hi);
+        const uint32_t lo16 = pack16<VT>(p0 - f.x, p1 - f.y);
         const int key = 8 * warp + 2 * tig;
         *reinterpret_cast<uint32_t*>(bars->p + g * kDPRow + key * 2) = hi;
         *reinterpret_cast<uint32_t*>(bars->p + (g + 8) * kDPRow + key * 2) = lo16;
@@ -498,8 +589,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
           for (int pair = 0; pair < 2; ++pair) {
             uint32_t vb[4];
             ldsm_x4_t(vst + swz(key, 32 * warp + 16 * pair + 8 * (mi >> 1)), vb);
-            mma16816<KT>(o[2 * pair], af, vb[0], vb[1]);
-            mma16816<KT>(o[2 * pair + 1], af, vb[2], vb[3]);
+            mma16816<VT>(o[2 * pair], af, vb[0], vb[1]);
+            mma16816<VT>(o[2 * pair + 1], af, vb[2], vb[3]);
           }
         }
       }
@@ -625,10 +716,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
   }
 }
 
-template <int QT, int KT>
-cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsArgs& a,
+template <int QT, int KT, int VT = KT>
+cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tms, const RowsArgs& a,
                      cudaStream_t stream) {
-  auto kern = decode_mma_kernel<QT, KT>;
+  auto kern = decode_mma_kernel<QT, KT, VT>;
   static std::atomic<bool> attr_set[64];   // per device; zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -656,7 +747,7 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsA
   ++na;
   cfg.attrs = at;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a);
+  return cudaLaunchKernelEx(&cfg, kern, tmk, tmv, tms, a);
 }
 
 template <int QT, int KT>
@@ -696,7 +787,7 @@ cudaError_t launch_decode_mma(int q_dtype, int kv_dtype, const CUtensorMap& tmk,
                               const RowsArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaErrorInvalidValue;
 #define KCA_DMMA_CASE(QD, KD) \
-  if (q_dtype == QD && kv_dtype == KD) e = launch_t<QD, KD>(tmk, tmv, a, stream);
+  if (q_dtype == QD && kv_dtype == KD) e = launch_t<QD, KD>(tmk, tmv, tmk, a, stream);
   KCA_DMMA_CASE(KCA_F32, KCA_F16)
   KCA_DMMA_CASE(KCA_F32, KCA_BF16)
   KCA_DMMA_CASE(KCA_F16, KCA_F16)
@@ -704,6 +795,21 @@ cudaError_t launch_decode_mma(int q_dtype, int kv_dtype, const CUtensorMap& tmk,
   KCA_DMMA_CASE(KCA_BF16, KCA_F16)
   KCA_DMMA_CASE(KCA_BF16, KCA_BF16)
 #undef KCA_DMMA_CASE
+  return e;
+}
+
+cudaError_t launch_decode_mma_q8(int q_dtype, int v_dtype, const CUtensorMap& tmk, const CUtensorMap& tms,
+                                 const CUtensorMap& tmv, const RowsArgs& a, cudaStream_t stream) {
+  cudaError_t e = cudaErrorInvalidValue;
+#define KCA_DQ8_CASE(QD, VD) \
+  if (q_dtype == QD && v_dtype == VD) e = launch_t<QD, KCA_I8, VD>(tmk, tmv, tms, a, stream);
+  KCA_DQ8_CASE(KCA_F32, KCA_F16)
+  KCA_DQ8_CASE(KCA_F32, KCA_BF16)
+  KCA_DQ8_CASE(KCA_F16, KCA_F16)
+  KCA_DQ8_CASE(KCA_F16, KCA_BF16)
+  KCA_DQ8_CASE(KCA_BF16, KCA_F16)
+  KCA_DQ8_CASE(KCA_BF16, KCA_BF16)
+#undef KCA_DQ8_CASE
   return e;
 }
 

@@ -1,7 +1,9 @@
-// kca_q8.cu -- the quantised-dot attention: K rows stored as int8 codes with
-// a per-row scale, the query quantised the same way per head inside the
-// decode kernel, QK taken exactly on the codes (four int8 pairs per dp4a),
-// softmax and the V sum in f32 (the CUDA-core rows kernel, kca_rows.cu).
+// kca_q8.cu -- the quantised-dot attention's K quantisation and its device
+// canary.  K rows are stored as int8 codes with a per-row scale; the decode
+// kernels quantise the query the same way per head and take QK exactly on
+// the codes -- on int8 tensor-core MMAs in the decode kernel for 16-bit V
+// (kca_decode_mma.cu), four int8 pairs per dp4a on the CUDA cores for f32 V
+// (kca_rows.cu) -- then the softmax and V sum in f32.
 //
 // Prior art on the pages (Karume v0.8.0 release notes, "Fixes"): attention's
 // dot product runs on packed int8 pairs with a dp4a-style instruction where
@@ -63,10 +65,11 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const void* x, int64
 }
 
 // ------------------------------------------------------------------ canary
-// Known answer: kCanary (a, b, c) triples spanning the int8 extremes; each
-// variant writes its results to its half of the array.
+// Known answers: kCanary (a, b, c) triples spanning the int8 extremes for
+// the dp4a instruction and its emulation, and one int8 tensor-core MMA
+// (m16n8k32, the decode kernel's QK instruction) on patterned fragments.
 constexpr int kCanary = 64;
-__device__ int kca_canary_out[2 * kCanary];
+__device__ int kca_canary_out[2 * kCanary + 128];
 
 __host__ __device__ inline void canary_case(int i, uint32_t* a, uint32_t* b, int* c) {
   const int8_t vals[8] = {-128, -127, -1, 0, 1, 63, 126, 127};
@@ -80,34 +83,94 @@ __host__ __device__ inline void canary_case(int i, uint32_t* a, uint32_t* b, int
   *c = (i * 977) % 20011 - 10005;
 }
 
-__global__ void canary_kernel() {
-  const int i = threadIdx.x;
-  if (i >= kCanary) return;
-  uint32_t a, b;
-  int c;
-  canary_case(i, &a, &b, &c);
-  kca_canary_out[i] = __dp4a(static_cast<int>(a), static_cast<int>(b), c);
-  int e = c;
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    e += static_cast<int>(static_cast<int8_t>(a >> (8 * j))) * static_cast<int>(static_cast<int8_t>(b >> (8 * j)));
-  kca_canary_out[kCanary + i] = e;
+// Byte j of fragment register r of lane l (A: r 0..3, B: r 4..5).
+__host__ __device__ inline int8_t mma_byte(int lane, int r, int j) {
+  return static_cast<int8_t>(((lane * 37 + r * 101 + j * 53) % 255) - 127);
+}
+__host__ __device__ inline uint32_t mma_reg(int lane, int r) {
+  uint32_t x = 0;
+  for (int j = 0; j < 4; ++j) x |= static_cast<uint32_t>(static_cast<uint8_t>(mma_byte(lane, r, j))) << (8 * j);
+  return x;
 }
 
-// Per device: 0 not run, 1 dp4a, 2 emulation, 3 neither sane.
+int dot_ref(uint32_t a, uint32_t b, int c) {
+  for (int j = 0; j < 4; ++j)
+    c += static_cast<int>(static_cast<int8_t>(a >> (8 * j))) * static_cast<int>(static_cast<int8_t>(b >> (8 * j)));
+  return c;
+}
+
+__global__ void canary_kernel() {
+  const int i = threadIdx.x;
+  if (i < kCanary) {
+    uint32_t a, b;
+    int c;
+    canary_case(i, &a, &b, &c);
+    kca_canary_out[i] = __dp4a(static_cast<int>(a), static_cast<int>(b), c);
+    int e = c;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      e += static_cast<int>(static_cast<int8_t>(a >> (8 * j))) * static_cast<int>(static_cast<int8_t>(b >> (8 * j)));
+    kca_canary_out[kCanary + i] = e;
+  }
+  if (i < 32) {   // warp 0: one m16n8k32 int8 MMA
+    int d[4] = {0, 0, 0, 0};
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(mma_reg(i, 0)), "r"(mma_reg(i, 1)), "r"(mma_reg(i, 2)), "r"(mma_reg(i, 3)), "r"(mma_reg(i, 4)),
+          "r"(mma_reg(i, 5)));
+#pragma unroll
+    for (int r = 0; r < 4; ++r) kca_canary_out[2 * kCanary + 4 * i + r] = d[r];
+  }
+}
+
+// The MMA's known answer from its operands' documented fragment layout:
+// A (16 x 32, row-major) -- a0 (row g, cols 4t + j), a1 (row g + 8, same
+// cols), a2 (row g, cols 16 + 4t + j), a3 (row g + 8, cols 16 + 4t + j);
+// B (32 x 8, column-major) -- b0 (rows 4t + j, col g), b1 (rows 16 + 4t + j,
+// col g); D -- d0 (g, 2t), d1 (g, 2t + 1), d2 (g + 8, 2t), d3 (g + 8, 2t + 1);
+// g = lane / 4, t = lane % 4.
+bool mma_answer_ok(const int* got) {
+  int A[16][32], B[32][8];
+  for (int lane = 0; lane < 32; ++lane) {
+    const int g = lane / 4, t = lane % 4;
+    for (int j = 0; j < 4; ++j) {
+      A[g][4 * t + j] = mma_byte(lane, 0, j);
+      A[g + 8][4 * t + j] = mma_byte(lane, 1, j);
+      A[g][16 + 4 * t + j] = mma_byte(lane, 2, j);
+      A[g + 8][16 + 4 * t + j] = mma_byte(lane, 3, j);
+      B[4 * t + j][g] = mma_byte(lane, 4, j);
+      B[16 + 4 * t + j][g] = mma_byte(lane, 5, j);
+    }
+  }
+  for (int lane = 0; lane < 32; ++lane) {
+    const int g = lane / 4, t = lane % 4;
+    const int rows[4] = {g, g, g + 8, g + 8}, cols[4] = {2 * t, 2 * t + 1, 2 * t, 2 * t + 1};
+    for (int r = 0; r < 4; ++r) {
+      int want = 0;
+      for (int k = 0; k < 32; ++k) want += A[rows[r]][k] * B[k][cols[r]];
+      if (got[4 * lane + r] != want) return false;
+    }
+  }
+  return true;
+}
+
+// Per device: -1 not run, else the mask of sane variants (1 dp4a, 2 its
+// emulation, 4 int8 MMA).
 std::atomic<int> g_canary[64];
 std::mutex g_canary_mu;
 
-int run_canary(cudaStream_t s, int* variant) {
+int run_canary(cudaStream_t s, int* mask) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KCA_ERR_CUDA;
-  int v = g_canary[dev].load();
-  if (v == 0) {
+  int v = g_canary[dev].load() - 1;
+  if (v < 0) {
     std::lock_guard<std::mutex> lock(g_canary_mu);
-    v = g_canary[dev].load();
-    if (v == 0) {
+    v = g_canary[dev].load() - 1;
+    if (v < 0) {
       canary_kernel<<<1, kCanary, 0, s>>>();
-      int got[2 * kCanary];
+      int got[2 * kCanary + 128];
       if (cudaGetLastError() != cudaSuccess ||
           cudaMemcpyFromSymbolAsync(got, kca_canary_out, sizeof got, 0, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
           cudaStreamSynchronize(s) != cudaSuccess)
@@ -117,55 +180,25 @@ int run_canary(cudaStream_t s, int* variant) {
         uint32_t a, b;
         int c;
         canary_case(i, &a, &b, &c);
-        int want = c;
-        for (int j = 0; j < 4; ++j)
-          want += static_cast<int>(static_cast<int8_t>(a >> (8 * j))) * static_cast<int>(static_cast<int8_t>(b >> (8 * j)));
+        const int want = dot_ref(a, b, c);
         hw = hw && got[i] == want;
         emu = emu && got[kCanary + i] == want;
       }
-      v = hw ? 1 : (emu ? 2 : 3);
-      g_canary[dev].store(v);
+      v = (hw ? 1 : 0) | (emu ? 2 : 0) | (mma_answer_ok(got + 2 * kCanary) ? 4 : 0);
+      g_canary[dev].store(v + 1);
     }
   }
-  if (v == 3) return KCA_ERR_DEVICE;
-  *variant = v == 1 ? 1 : 0;
-  return KCA_OK;
+  *mask = v;
+  return (v & 3) == 0 ? KCA_ERR_DEVICE : KCA_OK;
 }
 
 bool dtype3(int32_t d) { return d == KCA_F32 || d == KCA_F16 || d == KCA_BF16; }
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int device_sms(int* out) {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    return KCA_ERR_CUDA;
-  *out = n;
-  return KCA_OK;
-}
-
-int q8_args_status(int64_t capacity, int32_t batch, const int64_t* ctx_len) {
-  if (capacity < 1 || capacity > KCA_MAX_POSITION) return KCA_ERR_RANGE;
-  if (batch < 1 || batch > KCA_MAX_BATCH) return KCA_ERR_RANGE;
-  for (int32_t b = 0; b < batch; ++b)
-    if (ctx_len[b] < 0 || ctx_len[b] > capacity) return KCA_ERR_RANGE;
-  return KCA_OK;
-}
-
-std::vector<int64_t> q8_unit_keys(int32_t batch, const int64_t* ctx_len, int32_t window) {
-  std::vector<int64_t> nk(batch);
-  for (int32_t b = 0; b < batch; ++b) nk[b] = n_visible(ctx_len[b] - 1, window);
-  return nk;
-}
-
-size_t q8_ws_bytes(const RowsPlan& p) {
-  if (p.max_splits <= 1) return KCA_WORKSPACE_HEADER;
-  const size_t slots = (size_t)p.n_units * p.max_splits;
-  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-  return KCA_WORKSPACE_HEADER + al(slots * kHeads * 2 * 4) + al(slots * kHeads * kDim * 4);
-}
-
 }  // namespace
+
+int dot_canary(cudaStream_t s, int* mask) { return run_canary(s, mask); }
+
 }  // namespace kca
 
 extern "C" {
@@ -188,61 +221,8 @@ int attn_dot_canary(void* stream, int32_t* variant) {
   if (variant == nullptr) return KCA_ERR_NULL;
   int v = 0;
   const int st = kca::run_canary(static_cast<cudaStream_t>(stream), &v);
-  if (st == KCA_OK) *variant = v;
+  if (st == KCA_OK || st == KCA_ERR_DEVICE) *variant = v;
   return st;
-}
-
-size_t attn_decode_q8_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_t window) {
-  if (ctx_len == nullptr || kca::q8_args_status(KCA_MAX_POSITION, batch, ctx_len) != KCA_OK) return 0;
-  int sms = 0;
-  if (kca::device_sms(&sms) != KCA_OK) return 0;
-  const std::vector<int64_t> nk = kca::q8_unit_keys(batch, ctx_len, window);
-  return kca::q8_ws_bytes(kca::make_rows_plan(batch, nk.data(), sms));
-}
-
-int attn_decode_q8(const void* q, int32_t q_dtype, const void* k8_cache, const void* v_cache, int32_t v_dtype,
-                   int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int64_t capacity, int32_t batch,
-                   const int64_t* ctx_len, int32_t window, float scale, float* out, void* workspace,
-                   size_t workspace_bytes, void* stream) {
-  if (!q || !k8_cache || !v_cache || !out || !workspace || !ctx_len) return KCA_ERR_NULL;
-  if (n_q_heads != KCA_N_Q_HEADS || n_kv_heads != KCA_N_KV_HEADS || head_dim != KCA_HEAD_DIM)
-    return KCA_ERR_GEOMETRY;
-  if (!kca::dtype3(q_dtype) || !kca::dtype3(v_dtype)) return KCA_ERR_DTYPE;
-  int st = kca::q8_args_status(capacity, batch, ctx_len);
-  if (st != KCA_OK) return st;
-  if (!std::isfinite(scale) || !(scale > 0.f)) return KCA_ERR_RANGE;
-  if (!kca::al16(q) || !kca::al16(k8_cache) || !kca::al16(v_cache) || !kca::al16(out)) return KCA_ERR_ALIGN;
-  if ((reinterpret_cast<uintptr_t>(workspace) % 256) != 0) return KCA_ERR_WORKSPACE;
-  int sms = 0;
-  if (kca::device_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
-  const std::vector<int64_t> nk = kca::q8_unit_keys(batch, ctx_len, window);
-  const kca::RowsPlan p = kca::make_rows_plan(batch, nk.data(), sms);
-  if (workspace_bytes < kca::q8_ws_bytes(p)) return KCA_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int dp4a = 0;
-  st = kca::run_canary(s, &dp4a);
-  if (st != KCA_OK) return st;
-  kca::RowsArgs a{};
-  a.q = q;
-  a.k = k8_cache;
-  a.v = v_cache;
-  a.out = out;
-  a.status = workspace;
-  a.seq_rows = capacity;
-  a.mode = 0;
-  a.n_units = batch;
-  a.split_len = p.split_len;
-  a.max_splits = p.max_splits;
-  a.window = window;
-  a.scale = scale;
-  if (p.max_splits > 1) {
-    char* base = static_cast<char*>(workspace) + KCA_WORKSPACE_HEADER;
-    const size_t ml = (size_t)batch * p.max_splits * kca::kHeads * 2 * 4;
-    a.part_ml = reinterpret_cast<float*>(base);
-    a.part_acc = reinterpret_cast<float*>(base + (ml + 255) / 256 * 256);
-  }
-  for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
-  return kca::launch_rows_q8(q_dtype, v_dtype, dp4a != 0, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -138,6 +138,19 @@ int decode_entry(const void* q, int32_t q_dtype, const void* k_cache, const void
                  const int64_t* ctx_len, int32_t window, float scale, float* out, void* workspace,
                  size_t workspace_bytes, void* stream, bool clear_header);
 
+// The dot-product canary of the quantised-dot decode (kca_q8.cu): once per
+// device, the dp4a instruction, its emulation and the int8 MMA against known
+// answers; *mask: 1 dp4a sane, 2 emulation sane, 4 int8 MMA sane.
+// KCA_ERR_DEVICE when neither dp4a nor its emulation is, KCA_ERR_CUDA when
+// the check could not run.
+int dot_canary(cudaStream_t s, int* mask);
+
+// Tensor-core rows kernel with packed int8 K rows: tmk maps the codes (uint8
+// [rows][272], 128 x 64 boxes, 128-byte swizzle), tms their scale column
+// (16 x 64 boxes at x = 256, no swizzle), tmv the 16-bit V rows.
+cudaError_t launch_decode_mma_q8(int q_dtype, int v_dtype, const CUtensorMap& tmk, const CUtensorMap& tms,
+                                 const CUtensorMap& tmv, const RowsArgs& a, cudaStream_t stream);
+
 // Clusters of c CTAs of the tensor-core rows kernel that fit on the device at
 // once (0 on failure).
 int decode_mma_cluster_capacity(int c);

@@ -25,8 +25,9 @@ def _setup(cuda_ok):
     kca.lib()
 
 
-def test_canary_finds_the_dp4a_instruction_sane():
-    assert kca.attn_dot_canary() == 1
+def test_canary_finds_every_variant_sane():
+    # dp4a, its emulation and the int8 MMA all give the known answers on B200
+    assert kca.attn_dot_canary() == 7
 
 
 @pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
@@ -42,9 +43,11 @@ def test_quantized_rows_are_the_oracle_bytes(dtype):
         k32 = k
     got = kca.attn_quantize_k(dev(k, dtype)).cpu().numpy()
     codes, scales = quant.quantize_rows(k32)
-    want = quant.pack_rows(codes, scales)
-    assert got.shape == want.shape
-    assert np.array_equal(got, want)
+    assert got.shape == (1000, quant.ROW_BYTES)
+    got_codes, got_scales = quant.unpack_rows(got)
+    assert np.array_equal(got_codes, codes)                       # every integer decision
+    assert np.array_equal(got_scales, scales, equal_nan=True)     # bit for bit, NaN payloads aside
+    assert not got[:, 260:].any()
 
 
 def _case(seed, batch, cap, ctx, q_dtype, v_dtype, std=1.0):
@@ -67,6 +70,7 @@ def _oracle(codes, scales, v, q, ctx, window, q_dtype, v_dtype):
 @pytest.mark.parametrize("q_dtype,v_dtype,window", [("f32", "f32", 0), ("f32", "f16", 0), ("bf16", "bf16", 300),
                                                     ("f16", "f32", 1000), ("f32", "bf16", 0)])
 def test_decode_q8_matches_oracle(q_dtype, v_dtype, window):
+    # 16-bit V: the tensor-core kernel (int8 MMA); f32 V: the CUDA-core one (dp4a)
     batch, cap = 6, 5000
     ctx = [5000, 1, 0, 64, 4097, 2345]
     codes, scales, packed, v, q = _case(71, batch, cap, ctx, q_dtype, v_dtype)
@@ -103,3 +107,14 @@ def test_decode_q8_on_the_library_quantizer_and_nan_rows():
     want = _oracle(codes, scales, v, q, ctx, 0, "f32", "f16")
     assert np.isnan(out[0]).all() and np.isnan(want[0]).all()
     assert max_err(out[1:], want[1:]) <= 4e-3
+
+
+def test_decode_q8_cuda_core_kernel_on_16bit_v():
+    # the dp4a kernel pinned on a 16-bit V cache gives the oracle's values too
+    batch, cap = 3, 4000
+    ctx = [4000, 17, 2500]
+    codes, scales, packed, v, q = _case(74, batch, cap, ctx, "f32", "f16")
+    with kca.forced_path(kca.OP_ROWS, kca.PATH_CUDA_CORE):
+        out = kca.attn_decode_q8(dev(q, "f32"), torch.from_numpy(packed).cuda(), dev(v, "f16"), ctx)
+    want = _oracle(codes, scales, v, q, ctx, 0, "f32", "f16")
+    assert max_err(out.cpu().numpy(), want) <= 4e-3
