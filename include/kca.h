@@ -180,9 +180,13 @@ int attn_decode(const void *q, int32_t q_dtype,
  * attn_prefill_batch -- short chunks of several sequences in one call: each
  * sequence b has `rows` query rows, at positions ctx_len[b] - rows ..
  * ctx_len[b] - 1 (speculative or multi-row decode steps), every row seeing
- * its sequence's keys as in attn_prefill.  One launch (plus the split merge
- * on f32 caches) serves all batch x rows rows: each row is a unit of the
- * rows path (decode's kernels), its keys cut into splits across the GPU.
+ * its sequence's keys as in attn_prefill.  With a 16-bit cache and rows > 1,
+ * one launch of the multi-row tensor-core kernel (units of up to 4
+ * consecutive rows of a sequence, so each K/V row crosses to the SM once per
+ * unit; the union of the unit's keys cut into splits across the GPU) plus a
+ * merge launch; otherwise the rows path of decode (one unit per row).  As in
+ * tensor-core prefill, V must be finite on the rows of a unit's key union:
+ * a masked key's zero probability multiplies its V row.
  * Passage: Karume v0.12.0 release notes, "Docs", ADR 0067 plan-size geometry
  * table (the 2-15-row plans between decode and the >= 16-row tiles), and
  * "Performance", item 3 (the parallel PV reduction serves plans under 16

@@ -92,6 +92,26 @@ std::vector<int64_t> batch_unit_keys(int32_t batch, int32_t rows, const int64_t*
   return nk;
 }
 
+// Multi-row units of the tensor-core batched path: unit b * blocks + k holds
+// rows 4k .. 4k+3 (at most) of sequence b; its keys are the union of theirs.
+std::vector<int64_t> multirow_unit_keys(int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window) {
+  const int32_t blocks = (rows + kca::kMultiRows - 1) / kca::kMultiRows;
+  std::vector<int64_t> nk((size_t)batch * blocks);
+  for (int32_t b = 0; b < batch; ++b)
+    for (int32_t k = 0; k < blocks; ++k) {
+      const int32_t i0 = k * kca::kMultiRows;
+      const int32_t nr = rows - i0 < kca::kMultiRows ? rows - i0 : kca::kMultiRows;
+      const int64_t pos0 = ctx_len[b] - rows + i0;
+      nk[(size_t)b * blocks + k] = pos0 + nr - kca::lo_of(pos0, window);
+    }
+  return nk;
+}
+size_t multirow_ws_bytes(int32_t batch, int32_t rows, const kca::RowsPlan& p) {
+  if (p.max_splits <= 1) return KCA_WORKSPACE_HEADER;
+  const size_t slots = (size_t)batch * rows * p.max_splits;
+  return KCA_WORKSPACE_HEADER + align_up(slots * kHeads * 2 * 4) + align_up(slots * kHeads * kDim * 4);
+}
+
 int batch_args_status(int64_t capacity, int32_t batch, int32_t rows, const int64_t* ctx_len) {
   if (capacity < 1 || capacity > KCA_MAX_POSITION) return KCA_ERR_RANGE;
   if (batch < 1 || batch > KCA_MAX_BATCH || rows < 1 || rows > KCA_MAX_BATCH_ROWS) return KCA_ERR_RANGE;
@@ -250,6 +270,10 @@ bool use_rows_mma(int32_t kv_dtype) {
   if (kv_dtype != KCA_F16 && kv_dtype != KCA_BF16) return false;
   return g_rows_path.load(std::memory_order_relaxed) != 0;
 }
+
+// The batched call takes the multi-row tensor-core kernel for 16-bit caches
+// and more than one row per sequence (one row per sequence is decode).
+bool use_multirow(int32_t kv_dtype, int32_t rows) { return rows > 1 && use_rows_mma(kv_dtype); }
 
 // Plan of the tensor-core rows kernel.  Each cluster size c in {8, 4, 2}
 // (and c = 1 when every unit fits one split, so nothing is merged) gets the
@@ -519,7 +543,13 @@ size_t attn_prefill_batch_workspace_bytes(int32_t batch, int32_t rows, const int
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return 0;
   const std::vector<int64_t> nk = batch_unit_keys(batch, rows, ctx_len, window);
-  return rows_ws_bytes_any(batch * rows, nk.data(), sms);
+  size_t need = rows_ws_bytes_any(batch * rows, nk.data(), sms);
+  if (rows > 1) {   // the multi-row kernel's partials, whichever path a call takes
+    const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window);
+    const size_t mr = multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms));
+    if (mr > need) need = mr;
+  }
+  return need;
 }
 
 size_t attn_decode_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_t window) {
@@ -813,6 +843,33 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
   if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return KCA_ERR_WORKSPACE;
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_multirow(kv_dtype, rows)) {
+    const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window);
+    const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms);
+    if (workspace_bytes < multirow_ws_bytes(batch, rows, mp)) return KCA_ERR_WORKSPACE;
+    kca::RowsArgs a{};
+    a.q = q;
+    a.k = k_cache;
+    a.v = v_cache;
+    a.out = out;
+    a.status = workspace;
+    a.seq_rows = capacity;
+    a.mode = 2;
+    a.rows_per_seq = rows;
+    a.n_units = (int32_t)nku.size();
+    a.split_len = mp.split_len;
+    a.max_splits = mp.max_splits;
+    a.window = window;
+    a.scale = scale;
+    for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
+    if (mp.max_splits > 1) carve(workspace, (size_t)batch * rows * mp.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
+    CUtensorMap tmk, tmv;
+    if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, (int64_t)batch * capacity, 64) ||
+        !encode_kv_map(&tmv, v_cache, kv_dtype, 0, (int64_t)batch * capacity, 64))
+      return KCA_ERR_CUDA;
+    return kca::launch_decode_multirow(q_dtype, kv_dtype, tmk, tmv, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+  }
   const int32_t n_units = batch * rows;
   const std::vector<int64_t> nk = batch_unit_keys(batch, rows, ctx_len, window);
   int cluster = 1;
@@ -835,8 +892,7 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
   a.window = window;
   a.scale = scale;
   for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
-  return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster, workspace,
-                          static_cast<cudaStream_t>(stream));
+  return launch_rows_path(q_dtype, kv_dtype, k_cache, v_cache, (int64_t)batch * capacity, a, cluster, workspace, s);
 }
 
 size_t attn_decode_q8_workspace_bytes(int32_t batch, const int64_t* ctx_len, int32_t window) {

@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 
 #include "kca_common.cuh"
+#include "kca_merge.cuh"
 #include "kca_plan.h"
 #include "kca_rows.h"
 
@@ -771,6 +772,388 @@ int cluster_capacity_t(int c) {
   return n;
 }
 
+// ------------------------------------------------------------ multi-row units
+// Batched short chunks (attn_prefill_batch): one unit = up to kMRows
+// consecutive query rows of one sequence, so each K/V stage crosses from L2
+// to the SM once for all of them.  The unit's keys are the union of its
+// rows' visible ranges, cut into splits of the host plan's length; each row
+// masks the keys it does not see (an empty row of a split writes the empty
+// partial (-inf, 0, 0)).  Per stage and warp: the K fragments of its 8 keys
+// are loaded once and multiplied by every row's query (hi/lo, from shared
+// memory), the stage max, lazy rescale and P of each row as in the decode
+// kernel, then the V fragments of its 32 dims are loaded once for every
+// row's P.  One CTA per split, no cluster: a unit with several splits writes
+// per-row partials that multirow_merge_kernel combines.
+constexpr int kMRows = 4;
+constexpr int kMStages = 2;
+constexpr int kMOffBar = kMStages * kDStageBytes;    // 128 KiB
+
+struct MBars {
+  uint64_t full[kMStages];
+  uint64_t empty[kMStages];
+  int abort;
+  float red[kDWarps][kMRows][8];
+  __align__(16) unsigned char p[kMRows][16 * kDPRow];
+  __align__(16) unsigned char qs[kMRows][16 * kDQRow];
+};
+constexpr int kMSmemBytes = kMOffBar + (int)sizeof(MBars) + 1024;
+
+// Unit u of a batched call: sequence *b, first row *i0 (of the sequence's
+// rows), *nr rows; positions ctx[b] - rows + i0 + r.
+__device__ __forceinline__ void multirow_unit(const RowsArgs& a, int u, int* b, int* i0, int* nr) {
+  const int blocks = (a.rows_per_seq + kMRows - 1) / kMRows;
+  *b = u / blocks;
+  *i0 = (u % blocks) * kMRows;
+  const int left = a.rows_per_seq - *i0;
+  *nr = left < kMRows ? left : kMRows;
+}
+
+template <int QT, int KT>
+__global__ void __launch_bounds__(kDThreads, 1)
+    decode_multirow_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                           const RowsArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  unsigned char* smem = smem_raw + pad;
+  const uint32_t sbase = raw_addr + pad;
+  MBars* bars = reinterpret_cast<MBars*>(smem + kMOffBar);
+  volatile int* abort_flag = &bars->abort;
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.status);
+
+  const int unit = blockIdx.y;
+  const int split = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  int b, i0, nr;
+  multirow_unit(a, unit, &b, &i0, &nr);
+  const int64_t pos0 = a.ctx[b] - a.rows_per_seq + i0;       // first row's position
+  const int64_t lo_u = lo_of(pos0, a.window);
+  const int64_t hi_u = pos0 + nr - 1;
+  const int64_t nk_u = hi_u - lo_u + 1;
+  const int32_t nsplit = rows_n_splits(nk_u, a.split_len);
+  if (split >= nsplit) return;
+  const int64_t kbeg = lo_u + (int64_t)split * a.split_len;
+  int64_t kend = kbeg + a.split_len;
+  if (kend > hi_u + 1) kend = hi_u + 1;
+  const int64_t base_row = (int64_t)b * a.seq_rows;
+  const int n_stage = (int)cdiv(kend - kbeg, kDStageKeys);
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kMStages; ++st) {
+      mbar_init(&bars->full[st], 1);
+      mbar_init(&bars->empty[st], kDWarps);
+    }
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x == kDWarps * 32) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+  }
+  __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  if (warp == kDWarps) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n_stage; ++i) {
+        const int slot = i % kMStages;
+        if (i >= kMStages &&
+            !mbar_wait(&bars->empty[slot], ((i / kMStages) - 1) & 1, abort_flag, status, kSiteRowsEmpty))
+          break;
+        const uint32_t kst = sbase + slot * kDStageBytes;
+        const uint32_t bar = smem_u32(&bars->full[slot]);
+        const int32_t row0 = (int32_t)(base_row + kbeg + (int64_t)i * kDStageKeys);
+        mbar_arrive_expect_tx(&bars->full[slot], kDStageBytes);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tma2d(kst + c * kDBoxBytes, &tmk, 64 * c, row0, bar);
+          tma2d(kst + kDHalfBytes + c * kDBoxBytes, &tmv, 64 * c, row0, bar);
+        }
+        issued = i + 1;
+      }
+      if (issued < n_stage) {  // aborted: let every issued copy land
+        for (int st = 0; st < kMStages && st < issued; ++st) {
+          const int last = ((issued - 1 - st) / kMStages) * kMStages + st;
+          mbar_wait(&bars->full[st], (last / kMStages) & 1, nullptr, status, kSiteRowsFull);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ compute
+    const int g = lane >> 2, tig = lane & 3;
+    {
+      // Stage each row's query (hi / lo 16-bit parts, 16 rows of 256 dims);
+      // rows past nr are zero.  Thread t: 8 dims of head t / 32.
+      const int h = threadIdx.x >> 5, d0 = 8 * (threadIdx.x & 31);
+#pragma unroll
+      for (int r = 0; r < kMRows; ++r) {
+        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (r < nr) {
+          const int64_t orow = (int64_t)b * a.rows_per_seq + i0 + r;
+          load8<QT>(static_cast<const char*>(a.q) + ((orow * kHeads + h) * kDim + d0) * ElemBytes<QT>::value, x);
+        }
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          hi[j] = pack16<KT>(x[2 * j], x[2 * j + 1]);
+          const float2 f = unpack16<KT>(hi[j]);
+          lo[j] = pack16<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
+        }
+        *reinterpret_cast<uint4*>(bars->qs[r] + h * kDQRow + d0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(bars->qs[r] + (h + 8) * kDQRow + d0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+    }
+    const int mi = lane >> 3;
+    const uint32_t qoff = (8 * (mi & 1) + (lane & 7)) * kDQRow + 8 * (mi >> 1) * 2;
+    float o[kMRows][4][4];
+#pragma unroll
+    for (int r = 0; r < kMRows; ++r)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[r][i][j] = 0.f;
+    float m_ref[kMRows], l_part[kMRows];
+    int64_t rlo[kMRows], rpos[kMRows];
+#pragma unroll
+    for (int r = 0; r < kMRows; ++r) {
+      m_ref[r] = -INFINITY;
+      l_part[r] = 0.f;
+      rpos[r] = pos0 + r;
+      rlo[r] = lo_of(rpos[r], a.window);
+    }
+    const float scale = a.scale;
+    bool ok = true;
+
+    for (int i = 0; i < n_stage; ++i) {
+      const int slot = i % kMStages;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->full[slot], (i / kMStages) & 1, abort_flag,
+                                                   status, kSiteRowsFull));
+      const int64_t k0 = kbeg + (int64_t)i * kDStageKeys;
+      const int cnt = (int)((kend - k0) < kDStageKeys ? (kend - k0) : kDStageKeys);
+      const uint32_t kst = sbase + slot * kDStageBytes;
+      const uint32_t vst = kst + kDHalfBytes;
+      float sx[kMRows][2];
+#pragma unroll
+      for (int r = 0; r < kMRows; ++r) sx[r][0] = sx[r][1] = -INFINITY;
+      if (ok) {
+        if (cnt < kDStageKeys) {  // V rows past the split's end -> 0
+          unsigned char* vrows = smem + slot * kDStageBytes + kDHalfBytes;
+          for (int idx = threadIdx.x; idx < (kDStageKeys - cnt) * 32; idx += kDWarps * 32) {
+            const int row = cnt + (idx >> 5), u = idx & 31;
+            *reinterpret_cast<uint4*>(vrows + (u >> 3) * kDBoxBytes + row * 128 + (u & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+        }
+        float sacc[kMRows][2][4];
+#pragma unroll
+        for (int r = 0; r < kMRows; ++r)
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sacc[r][c][j] = 0.f;
+        const int kr = 8 * warp + (lane & 7);
+#pragma unroll
+        for (int ks2 = 0; ks2 < 8; ++ks2) {
+          uint32_t bk[4];
+          ldsm_x4(kst + swz(kr, 32 * ks2 + 8 * (lane >> 3)), bk);
+#pragma unroll
+          for (int r = 0; r < kMRows; ++r) {
+            if (r < nr) {
+              uint32_t qa0[4], qa1[4];
+              const uint32_t qb = smem_u32(bars->qs[r]) + qoff;
+              ldsm_x4(qb + 32 * (2 * ks2), qa0);
+              ldsm_x4(qb + 32 * (2 * ks2 + 1), qa1);
+              mma16816<KT>(sacc[r][0], qa0, bk[0], bk[1]);
+              mma16816<KT>(sacc[r][1], qa1, bk[2], bk[3]);
+            }
+          }
+        }
+        const int kk0 = 8 * warp + 2 * tig;
+        const int64_t key0 = k0 + kk0;
+#pragma unroll
+        for (int r = 0; r < kMRows; ++r) {
+          if (r < nr) {
+            const float s0 = (sacc[r][0][0] + sacc[r][1][0]) + (sacc[r][0][2] + sacc[r][1][2]);
+            const float s1 = (sacc[r][0][1] + sacc[r][1][1]) + (sacc[r][0][3] + sacc[r][1][3]);
+            const bool v0 = kk0 < cnt && key0 >= rlo[r] && key0 <= rpos[r];
+            const bool v1 = kk0 + 1 < cnt && key0 + 1 >= rlo[r] && key0 + 1 <= rpos[r];
+            sx[r][0] = v0 ? s0 * scale : -INFINITY;
+            sx[r][1] = v1 ? s1 * scale : -INFINITY;
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kMRows; ++r) {
+        float mw = max_nan(sx[r][0], sx[r][1]);
+        mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 1));
+        mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 2));
+        if (tig == 0) bars->red[warp][r][g] = mw;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+#pragma unroll
+      for (int r = 0; r < kMRows; ++r) {
+        if (r < nr) {
+          float ms = bars->red[0][r][g];
+#pragma unroll
+          for (int w = 1; w < kDWarps; ++w) ms = max_nan(ms, bars->red[w][r][g]);
+          if (ok) {
+            if (ms > m_ref[r] + kDRescale) {
+              const float alpha = exp2f((m_ref[r] - ms) * kDLog2e);
+              m_ref[r] = ms;
+              l_part[r] *= alpha;
+#pragma unroll
+              for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) o[r][nt][j] *= alpha;
+            }
+            const float mu = m_ref[r] == -INFINITY ? 0.f : m_ref[r];
+            const float p0 = exp2f((sx[r][0] - mu) * kDLog2e);
+            const float p1 = exp2f((sx[r][1] - mu) * kDLog2e);
+            l_part[r] += p0 + p1;
+            const uint32_t hi = pack16<KT>(p0, p1);
+            const float2 f = unpack16<KT>(hi);
+            const uint32_t lo16 = pack16<KT>(p0 - f.x, p1 - f.y);
+            const int key = 8 * warp + 2 * tig;
+            *reinterpret_cast<uint32_t*>(bars->p[r] + g * kDPRow + key * 2) = hi;
+            *reinterpret_cast<uint32_t*>(bars->p[r] + (g + 8) * kDPRow + key * 2) = lo16;
+          }
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");   // P and zeroed rows visible
+      if (ok) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t af[kMRows][4];
+#pragma unroll
+          for (int r = 0; r < kMRows; ++r)
+            if (r < nr)
+              ldsm_x4(smem_u32(bars->p[r]) + (8 * (mi & 1) + (lane & 7)) * kDPRow + (16 * kk + 8 * (mi >> 1)) * 2,
+                      af[r]);
+          const int key = 16 * kk + 8 * (mi & 1) + (lane & 7);
+#pragma unroll
+          for (int pair = 0; pair < 2; ++pair) {
+            uint32_t vb[4];
+            ldsm_x4_t(vst + swz(key, 32 * warp + 16 * pair + 8 * (mi >> 1)), vb);
+#pragma unroll
+            for (int r = 0; r < kMRows; ++r) {
+              if (r < nr) {
+                mma16816<KT>(o[r][2 * pair], af[r], vb[0], vb[1]);
+                mma16816<KT>(o[r][2 * pair + 1], af[r], vb[2], vb[3]);
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->empty[slot]);
+    }
+
+    // Row sums of every row: lanes of one head, then warps.
+#pragma unroll
+    for (int r = 0; r < kMRows; ++r) {
+      float l = l_part[r];
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      if (tig == 0) bars->red[warp][r][g] = l;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+    const bool aborted = !ok || *abort_flag;
+#pragma unroll
+    for (int r = 0; r < kMRows; ++r) {
+      if (r < nr) {
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDWarps; ++w) L += bars->red[w][r][g];
+        float M = m_ref[r];
+        if (aborted) {
+          M = NAN;   // an aborted split poisons its rows; the status word says why
+          L = NAN;
+        }
+        const int64_t orow = (int64_t)b * a.rows_per_seq + i0 + r;
+        if (nsplit == 1) {
+          const float inv = (M == -INFINITY && L == 0.f) ? 0.f : 1.f / L;
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const int d = 32 * warp + 8 * nt + 2 * tig;
+            *reinterpret_cast<float2*>(a.out + (orow * kHeads + g) * kDim + d) =
+                make_float2((o[r][nt][0] + o[r][nt][2]) * inv, (o[r][nt][1] + o[r][nt][3]) * inv);
+          }
+        } else {
+          const int64_t slot = (orow * a.max_splits + split) * kHeads + g;
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const int d = 32 * warp + 8 * nt + 2 * tig;
+            *reinterpret_cast<float2*>(a.part_acc + slot * kDim + d) =
+                make_float2(o[r][nt][0] + o[r][nt][2], o[r][nt][1] + o[r][nt][3]);
+          }
+          if (warp == 0 && tig == 0) *reinterpret_cast<float2*>(a.part_ml + slot * 2) = make_float2(M, L);
+        }
+      }
+    }
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Log-sum-exp merge of the split partials of every row of a multi-row call:
+// one CTA per (row, head), its eight warps taking interleaved splits.
+__global__ void __launch_bounds__(256) multirow_merge_kernel(const RowsArgs a) {
+  const int64_t orow = blockIdx.x >> 3;
+  const int h = blockIdx.x & 7;
+  const int b = (int)(orow / a.rows_per_seq);
+  const int i = (int)(orow % a.rows_per_seq);
+  const int u = b * ((a.rows_per_seq + kMRows - 1) / kMRows) + i / kMRows;
+  int bb, i0, nr;
+  multirow_unit(a, u, &bb, &i0, &nr);
+  const int64_t pos0 = a.ctx[bb] - a.rows_per_seq + i0;
+  const int64_t nk_u = pos0 + nr - 1 - lo_of(pos0, a.window) + 1;
+  const int32_t nsplit = rows_n_splits(nk_u, a.split_len);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (nsplit <= 1) return;
+  __shared__ float red[8 * 264];
+  const int64_t row0 = orow * a.max_splits * kHeads + h;
+  merge_row<8>(nsplit, a.part_ml + row0 * 2, kHeads * 2, a.part_acc + row0 * kDim, kHeads * kDim, kDLog2e,
+               a.out + (orow * kHeads + h) * kDim, red, threadIdx.x >> 5, threadIdx.x & 31, 1);
+}
+
+template <int QT, int KT>
+cudaError_t launch_multirow_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsArgs& a, cudaStream_t stream) {
+  auto kern = decode_multirow_kernel<QT, KT>;
+  static std::atomic<bool> attr_set[64];   // per device; zero-initialised
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.max_splits, a.n_units, 1);
+  cfg.blockDim = dim3(kDThreads, 1, 1);
+  cfg.dynamicSmemBytes = kMSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = &at;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a);
+  if (e != cudaSuccess || a.max_splits <= 1) return e;
+  const int blocks = (a.rows_per_seq + kMRows - 1) / kMRows;
+  const int64_t rows_total = (int64_t)(a.n_units / blocks) * a.rows_per_seq;
+  cudaLaunchConfig_t mcfg = {};
+  mcfg.gridDim = dim3((unsigned)(rows_total * kHeads), 1, 1);
+  mcfg.blockDim = dim3(256, 1, 1);
+  mcfg.stream = stream;
+  mcfg.attrs = &at;
+  mcfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&mcfg, multirow_merge_kernel, a);
+}
+
 }  // namespace
 
 int decode_mma_cluster_capacity(int c) {
@@ -811,6 +1194,20 @@ cudaError_t launch_decode_mma_q8(int q_dtype, int v_dtype, const CUtensorMap& tm
   KCA_DQ8_CASE(KCA_BF16, KCA_BF16)
 #undef KCA_DQ8_CASE
   return e;
+}
+
+cudaError_t launch_decode_multirow(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                                   const RowsArgs& a, cudaStream_t stream) {
+#define KCA_MR_CASE(QD, KD) \
+  if (q_dtype == QD && kv_dtype == KD) return launch_multirow_t<QD, KD>(tmk, tmv, a, stream);
+  KCA_MR_CASE(KCA_F32, KCA_F16)
+  KCA_MR_CASE(KCA_F32, KCA_BF16)
+  KCA_MR_CASE(KCA_F16, KCA_F16)
+  KCA_MR_CASE(KCA_F16, KCA_BF16)
+  KCA_MR_CASE(KCA_BF16, KCA_F16)
+  KCA_MR_CASE(KCA_BF16, KCA_BF16)
+#undef KCA_MR_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kca

@@ -151,6 +151,15 @@ int dot_canary(cudaStream_t s, int* mask);
 cudaError_t launch_decode_mma_q8(int q_dtype, int v_dtype, const CUtensorMap& tmk, const CUtensorMap& tms,
                                  const CUtensorMap& tmv, const RowsArgs& a, cudaStream_t stream);
 
+// Batched short chunks on the tensor cores (mode 2, 16-bit K/V): units of up
+// to 4 consecutive rows of one sequence (n_units = batch x ceil(rows / 4)),
+// the union of their keys cut into splits of split_len; per-row split
+// partials in part_ml / part_acc ([batch * rows][max_splits][8]) merged by a
+// second kernel.
+constexpr int kMultiRows = 4;
+cudaError_t launch_decode_multirow(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                                   const RowsArgs& a, cudaStream_t stream);
+
 // Clusters of c CTAs of the tensor-core rows kernel that fit on the device at
 // once (0 on failure).
 int decode_mma_cluster_capacity(int c);
