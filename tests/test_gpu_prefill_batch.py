@@ -101,3 +101,19 @@ def test_multirow_units_with_a_window_cut_inside_a_unit():
     out = kca.attn_prefill_batch(dev(q, "f32"), dev(k, "f16"), dev(v, "f16"), ctx, 100)
     want = _oracle(q, k, v, ctx, rows, 100, "f32", "f16")
     assert max_err(out.cpu().numpy(), want) <= 4e-3
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("f32", "f16"), ("f32", "f32")])
+def test_batched_short_chunks_at_the_maximum_sizes(q_dtype, kv_dtype):
+    # KCA_MAX_BATCH sequences x KCA_MAX_BATCH_ROWS rows (3,840 rows, 1,024
+    # multi-row units on 16-bit caches), short ragged contexts
+    batch, rows, cap = kca.MAX_BATCH, kca.MAX_BATCH_ROWS, 96
+    ctx, q, k, v = _inputs(63, batch, rows, cap, q_dtype, kv_dtype)
+    ws = kca.new_workspace(kca.attn_prefill_batch_workspace_bytes(ctx, rows))
+    out = kca.attn_prefill_batch(dev(q, q_dtype), dev(k, kv_dtype), dev(v, kv_dtype), ctx, workspace=ws)
+    want = _oracle(q, k, v, ctx, rows, 0, q_dtype, kv_dtype)
+    assert max_err(out.cpu().numpy(), want) <= tol(q_dtype, kv_dtype)
+    assert kca.attn_device_status(ws)[0] == 0
+    with pytest.raises(kca.KcaError):   # one row more than the limit: rejected before any launch
+        kca.attn_prefill_batch(torch.zeros((1, rows + 1, 8, 256), device="cuda"),
+                               dev(k[:1], kv_dtype), dev(v[:1], kv_dtype), [rows + 1])

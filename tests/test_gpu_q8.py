@@ -118,3 +118,16 @@ def test_decode_q8_cuda_core_kernel_on_16bit_v():
         out = kca.attn_decode_q8(dev(q, "f32"), torch.from_numpy(packed).cuda(), dev(v, "f16"), ctx)
     want = _oracle(codes, scales, v, q, ctx, 0, "f32", "f16")
     assert max_err(out.cpu().numpy(), want) <= 4e-3
+
+
+def test_decode_q8_at_the_maximum_batch():
+    batch, cap = kca.MAX_BATCH, 700
+    ctx = list(synth.integers(75, "ctx", 0, cap, batch))
+    ctx[0], ctx[1] = 0, cap
+    codes, scales, packed, v, q = _case(75, batch, cap, ctx, "f32", "f16")
+    ws = kca.new_workspace(kca.attn_decode_q8_workspace_bytes(ctx))
+    out = kca.attn_decode_q8(dev(q, "f32"), torch.from_numpy(packed).cuda(), dev(v, "f16"), ctx, workspace=ws)
+    want = _oracle(codes, scales, v, q, ctx, 0, "f32", "f16")
+    assert max_err(out.cpu().numpy(), want) <= 4e-3
+    assert torch.all(out[0] == 0)
+    assert kca.attn_device_status(ws)[0] == 0
