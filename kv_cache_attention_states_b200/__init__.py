@@ -38,74 +38,83 @@ class KcaError(RuntimeError):
         super().__init__(f"{what}: {STATUS.get(status, status)} ({status_string(status)})")
 
 
+LIB_CHECKED_PATH = os.path.join(_HERE, "libkca_checked.so")
+
+
 def lib() -> ctypes.CDLL:
     """The loaded libkca.so (raises if it was not built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: build it with "
-                              "`python -m kv_cache_attention_states_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
-                                 ctypes.c_size_t)
-        p64 = ctypes.POINTER(ctypes.c_int64)
-        p32 = ctypes.POINTER(ctypes.c_int32)
-        L.attn_prefill.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i64, i32, i64, i32,
-                                   f32, vp, vp, sz, vp]
-        L.attn_prefill.restype = ctypes.c_int
-        L.attn_decode.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp,
-                                  vp, sz, vp]
-        L.attn_decode.restype = ctypes.c_int
-        L.attn_prefill_batch.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, i32, p64, i32, f32,
-                                         vp, vp, sz, vp]
-        L.attn_prefill_batch.restype = ctypes.c_int
-        L.attn_prefill_batch_workspace_bytes.argtypes = [i32, i32, p64, i32]
-        L.attn_prefill_batch_workspace_bytes.restype = sz
-        L.attn_decode_dev.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, vp, i64, i32, f32,
-                                      vp, vp, sz, vp]
-        L.attn_decode_dev.restype = ctypes.c_int
-        L.attn_append_kv.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp, i32, i64, vp, i64, vp, vp]
-        L.attn_append_kv.restype = ctypes.c_int
-        L.attn_decode_static.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32,
-                                         f32, vp, vp]
-        L.attn_decode_static.restype = ctypes.c_int
-        L.attn_decode_partial.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i64, i32,
-                                          f32, vp, vp, sz, vp]
-        L.attn_decode_partial.restype = ctypes.c_int
-        L.attn_merge_partials.argtypes = [i32, i32, vp, i64, vp, vp]
-        L.attn_merge_partials.restype = ctypes.c_int
-        L.attn_decode_partial_workspace_bytes.argtypes = [i32, p64, i64, i64, i32]
-        L.attn_decode_partial_workspace_bytes.restype = sz
-        L.attn_prefill_workspace_bytes.argtypes = [i32, i32, i64, i32, i32]
-        L.attn_prefill_workspace_bytes.restype = sz
-        L.attn_decode_workspace_bytes.argtypes = [i32, p64, i32]
-        L.attn_decode_workspace_bytes.restype = sz
-        L.attn_workspace_init.argtypes = [vp, sz, vp]
-        L.attn_workspace_init.restype = ctypes.c_int
-        L.attn_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
-        L.attn_device_status.restype = ctypes.c_int
-        L.attn_prefill_plan.argtypes = [i32, i32, i64, i32, i32, i32, p32, p64, i32, p32, p32]
-        L.attn_prefill_plan.restype = ctypes.c_int
-        L.attn_decode_plan.argtypes = [i32, p64, i32, i32, i32, p32, p64, i32, p32, p32]
-        L.attn_decode_plan.restype = ctypes.c_int
-        L.attn_decode_static_scratch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(sz)]
-        L.attn_decode_static_scratch.restype = ctypes.c_int
-        L.attn_quantize_k.argtypes = [vp, i32, i64, vp, vp]
-        L.attn_quantize_k.restype = ctypes.c_int
-        L.attn_decode_q8.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp, vp, sz, vp]
-        L.attn_decode_q8.restype = ctypes.c_int
-        L.attn_decode_q8_workspace_bytes.argtypes = [i32, p64, i32]
-        L.attn_decode_q8_workspace_bytes.restype = sz
-        L.attn_dot_canary.argtypes = [vp, p32]
-        L.attn_dot_canary.restype = ctypes.c_int
-        L.attn_decode_cluster_capacity.argtypes = [p32]
-        L.attn_decode_cluster_capacity.restype = ctypes.c_int
-        L.attn_force_path.argtypes = [i32, i32]
-        L.attn_force_path.restype = ctypes.c_int
-        L.attn_status_string.argtypes = [ctypes.c_int]
-        L.attn_status_string.restype = ctypes.c_char_p
-        _lib = L
+        _lib = load_library(LIB_PATH)
     return _lib
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """A libkca build at `path` with its C signatures declared (the binding
+    itself uses lib(); tests load the bounds-checked build with this)."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m kv_cache_attention_states_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                             ctypes.c_size_t)
+    p64 = ctypes.POINTER(ctypes.c_int64)
+    p32 = ctypes.POINTER(ctypes.c_int32)
+    L.attn_prefill.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i64, i32, i64, i32,
+                               f32, vp, vp, sz, vp]
+    L.attn_prefill.restype = ctypes.c_int
+    L.attn_decode.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp,
+                              vp, sz, vp]
+    L.attn_decode.restype = ctypes.c_int
+    L.attn_prefill_batch.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, i32, p64, i32, f32,
+                                     vp, vp, sz, vp]
+    L.attn_prefill_batch.restype = ctypes.c_int
+    L.attn_prefill_batch_workspace_bytes.argtypes = [i32, i32, p64, i32]
+    L.attn_prefill_batch_workspace_bytes.restype = sz
+    L.attn_decode_dev.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, vp, i64, i32, f32,
+                                  vp, vp, sz, vp]
+    L.attn_decode_dev.restype = ctypes.c_int
+    L.attn_append_kv.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp, i32, i64, vp, i64, vp, vp]
+    L.attn_append_kv.restype = ctypes.c_int
+    L.attn_decode_static.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32,
+                                     f32, vp, vp]
+    L.attn_decode_static.restype = ctypes.c_int
+    L.attn_decode_partial.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i64, i32,
+                                      f32, vp, vp, sz, vp]
+    L.attn_decode_partial.restype = ctypes.c_int
+    L.attn_merge_partials.argtypes = [i32, i32, vp, i64, vp, vp]
+    L.attn_merge_partials.restype = ctypes.c_int
+    L.attn_decode_partial_workspace_bytes.argtypes = [i32, p64, i64, i64, i32]
+    L.attn_decode_partial_workspace_bytes.restype = sz
+    L.attn_prefill_workspace_bytes.argtypes = [i32, i32, i64, i32, i32]
+    L.attn_prefill_workspace_bytes.restype = sz
+    L.attn_decode_workspace_bytes.argtypes = [i32, p64, i32]
+    L.attn_decode_workspace_bytes.restype = sz
+    L.attn_workspace_init.argtypes = [vp, sz, vp]
+    L.attn_workspace_init.restype = ctypes.c_int
+    L.attn_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.attn_device_status.restype = ctypes.c_int
+    L.attn_prefill_plan.argtypes = [i32, i32, i64, i32, i32, i32, p32, p64, i32, p32, p32]
+    L.attn_prefill_plan.restype = ctypes.c_int
+    L.attn_decode_plan.argtypes = [i32, p64, i32, i32, i32, p32, p64, i32, p32, p32]
+    L.attn_decode_plan.restype = ctypes.c_int
+    L.attn_decode_static_scratch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(sz)]
+    L.attn_decode_static_scratch.restype = ctypes.c_int
+    L.attn_quantize_k.argtypes = [vp, i32, i64, vp, vp]
+    L.attn_quantize_k.restype = ctypes.c_int
+    L.attn_decode_q8.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, p64, i32, f32, vp, vp, sz, vp]
+    L.attn_decode_q8.restype = ctypes.c_int
+    L.attn_decode_q8_workspace_bytes.argtypes = [i32, p64, i32]
+    L.attn_decode_q8_workspace_bytes.restype = sz
+    L.attn_dot_canary.argtypes = [vp, p32]
+    L.attn_dot_canary.restype = ctypes.c_int
+    L.attn_decode_cluster_capacity.argtypes = [p32]
+    L.attn_decode_cluster_capacity.restype = ctypes.c_int
+    L.attn_force_path.argtypes = [i32, i32]
+    L.attn_force_path.restype = ctypes.c_int
+    L.attn_status_string.argtypes = [ctypes.c_int]
+    L.attn_status_string.restype = ctypes.c_char_p
+    return L
 
 
 def status_string(status: int) -> str:

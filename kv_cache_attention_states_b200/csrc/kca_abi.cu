@@ -356,9 +356,11 @@ kca::RowsPlan rows_plan(int32_t kv_dtype, int32_t n_units, const int64_t* nkeys,
 // cache_rows rows of the cache), CUDA cores otherwise.
 int launch_rows_path(int32_t q_dtype, int32_t kv_dtype, const void* k_cache, const void* v_cache,
                      int64_t cache_rows, kca::RowsArgs a, int cluster, void* workspace, cudaStream_t s) {
+  a.cache_rows = cache_rows;
   if (use_rows_mma(kv_dtype)) {
     a.cluster = cluster;
     a.max_clusters = (a.max_splits + cluster - 1) / cluster;
+    a.part_slots = a.max_clusters > 1 ? (int64_t)a.n_units * a.max_clusters : 0;
     if (a.max_clusters > 1) {
       // Counters live in the header (no other path writes there), cluster
       // partials where the CUDA-core path keeps its split partials.
@@ -371,6 +373,7 @@ int launch_rows_path(int32_t q_dtype, int32_t kv_dtype, const void* k_cache, con
       return KCA_ERR_CUDA;
     return kca::launch_decode_mma(q_dtype, kv_dtype, tmk, tmv, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
   }
+  a.part_slots = a.max_splits > 1 ? (int64_t)a.n_units * a.max_splits : 0;
   carve(workspace, (size_t)a.n_units * a.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
   return kca::launch_rows(q_dtype, kv_dtype, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
 }
@@ -863,6 +866,8 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
     a.window = window;
     a.scale = scale;
     for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
+    a.cache_rows = (int64_t)batch * capacity;
+    a.part_slots = mp.max_splits > 1 ? (int64_t)batch * rows * mp.max_splits : 0;
     if (mp.max_splits > 1) carve(workspace, (size_t)batch * rows * mp.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
     CUtensorMap tmk, tmv;
     if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, (int64_t)batch * capacity, 64) ||
@@ -936,10 +941,12 @@ int attn_decode_q8(const void* q, int32_t q_dtype, const void* k8_cache, const v
   int sane = 0;
   st = kca::dot_canary(s, &sane);
   if (st != KCA_OK) return st;
+  a.cache_rows = (int64_t)batch * capacity;
   if (use_rows_mma(v_dtype) && (sane & 4)) {
     // 16-bit V: the tensor-core kernel, QK on int8 MMAs (exact integers)
     a.cluster = cluster;
     a.max_clusters = (a.max_splits + cluster - 1) / cluster;
+    a.part_slots = a.max_clusters > 1 ? (int64_t)a.n_units * a.max_clusters : 0;
     if (a.max_clusters > 1) {
       a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
       carve(workspace, (size_t)a.n_units * a.max_clusters * kHeads * 2 * 4, &a.cpart_ml, &a.cpart_acc);
@@ -961,6 +968,7 @@ int attn_decode_q8(const void* q, int32_t q_dtype, const void* k8_cache, const v
   const kca::RowsPlan pc = kca::make_rows_plan(batch, nk.data(), sms);
   a.split_len = pc.split_len;
   a.max_splits = pc.max_splits;
+  a.part_slots = a.max_splits > 1 ? (int64_t)a.n_units * a.max_splits : 0;
   carve(workspace, (size_t)a.n_units * a.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
   return kca::launch_rows_q8(q_dtype, v_dtype, (sane & 1) != 0, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
 }

@@ -23,11 +23,12 @@ struct DeviceStatus {
                         // bit 2: a device destination row out of range (append)
   unsigned int detail;  // (site << 24) | (block & 0xffffff) of the first failure
 };
-enum : unsigned int { kErrWaitTimeout = 1u, kErrBadCtx = 2u, kErrBadRow = 4u };
+enum : unsigned int { kErrWaitTimeout = 1u, kErrBadCtx = 2u, kErrBadRow = 4u, kErrBounds = 8u };
 enum : unsigned int {
   kSiteRowsFull = 1, kSiteRowsEmpty = 2, kSiteTcFull = 3, kSiteTcEmpty = 4, kSiteTcS = 5,
   kSiteTcP = 6, kSiteTcO = 7, kSiteTcQ = 8, kSiteTcDrain = 9, kSiteCtx = 10,
-  kSiteAppend = 11, kSiteTcAlign = 12
+  kSiteAppend = 11, kSiteTcAlign = 12, kSiteBoundsRows = 13, kSiteBoundsDecode = 14,
+  kSiteBoundsMulti = 15, kSiteBoundsMerge = 16
 };
 
 // Records the first failure (detail: site and the block's x index, or the
@@ -40,6 +41,17 @@ __device__ __forceinline__ void record_error(DeviceStatus* st, unsigned int site
   if (prev == 0) st->detail = (site << 24) | ((where == 0xffffffffu ? blockIdx.x : where) & 0xffffffu);
 }
 
+// Bounds-checked builds (-DKCA_BOUNDS_CHECK, the library's stand-in for a
+// memory sanitizer): KCA_IN_BOUNDS(cond, status, site, where) records a
+// failed index check in the status word (error bit 8) and yields false, so
+// the caller skips the access instead of faulting; in normal builds it is
+// the constant true and costs nothing.
+#ifdef KCA_BOUNDS_CHECK
+#define KCA_IN_BOUNDS(cond, st, site, where) ::kca::in_bounds((cond), (st), (site), (where))
+#else
+#define KCA_IN_BOUNDS(cond, st, site, where) true
+#endif
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -48,6 +60,11 @@ __device__ __forceinline__ uint64_t global_ns() {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ bool in_bounds(bool ok, DeviceStatus* st, unsigned int site, unsigned int where) {
+  if (!ok) record_error(st, site, kErrBounds, where);
+  return ok;
 }
 
 // ---------------------------------------------------------------- mbarrier

@@ -327,12 +327,24 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const int32_t nsplit = rows_n_splits(nkeys, split_len);
   const int nclus = (nsplit + C - 1) / C;
   if (clus >= nclus) return;               // the whole cluster leaves together
-  const bool active = split < nsplit && nkeys > 0;
+  bool active = split < nsplit && nkeys > 0;
   const int64_t kbeg = lo + (int64_t)split * split_len;
   int64_t kend = kbeg + split_len;
   if (kend > lo + nkeys) kend = lo + nkeys;
   // cache row of key p: base_row + p (a shard's row 0 is position key_begin)
   const int64_t base_row = seq_base - a.key_begin;
+  // bounds-checked builds: the unit's plan fits the host's (cluster-partial
+  // slots and tickets; a failure is the same for every CTA of the unit,
+  // which all leave together), and a split whose rows would leave the cache
+  // counts as empty
+  if (!KCA_IN_BOUNDS(nsplit <= a.max_splits && nclus <= a.max_clusters &&
+                         (nclus == 1 || ((int64_t)(unit + 1) * a.max_clusters <= a.part_slots &&
+                                         unit < KCA_MAX_CHUNK_ROWS)),
+                     status, kSiteBoundsDecode, (unsigned)unit))
+    return;
+  if (active && !KCA_IN_BOUNDS(base_row + kbeg >= 0 && base_row + kend <= a.cache_rows, status,
+                               kSiteBoundsDecode, (unsigned)unit))
+    active = false;
   const int n_stage = active ? (int)cdiv(kend - kbeg, kDStageKeys) : 0;
 
   if (threadIdx.x == 0) {
@@ -838,6 +850,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
   if (kend > hi_u + 1) kend = hi_u + 1;
   const int64_t base_row = (int64_t)b * a.seq_rows;
   const int n_stage = (int)cdiv(kend - kbeg, kDStageKeys);
+  // bounds-checked builds: the split's rows in the cache, its rows' partial
+  // slots in the workspace (no CTA of this kernel waits on another)
+  if (!KCA_IN_BOUNDS(nsplit <= a.max_splits && base_row + kbeg >= 0 && base_row + kend <= a.cache_rows &&
+                         (nsplit == 1 || ((int64_t)b * a.rows_per_seq + i0 + nr) * a.max_splits <= a.part_slots),
+                     status, kSiteBoundsMulti, (unsigned)unit))
+    return;
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kMStages; ++st) {
@@ -1114,6 +1132,9 @@ __global__ void __launch_bounds__(256) multirow_merge_kernel(const RowsArgs a) {
   const int32_t nsplit = rows_n_splits(nk_u, a.split_len);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (nsplit <= 1) return;
+  if (!KCA_IN_BOUNDS(nsplit <= a.max_splits && (orow + 1) * a.max_splits <= a.part_slots,
+                     static_cast<DeviceStatus*>(a.status), kSiteBoundsMerge, (unsigned)orow))
+    return;
   __shared__ float red[8 * 264];
   const int64_t row0 = orow * a.max_splits * kHeads + h;
   merge_row<8>(nsplit, a.part_ml + row0 * 2, kHeads * 2, a.part_acc + row0 * kDim, kHeads * kDim, kDLog2e,

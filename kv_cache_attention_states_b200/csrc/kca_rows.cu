@@ -120,6 +120,12 @@ __global__ void __launch_bounds__(kRowsThreads, 1) rows_kernel(const RowsArgs a)
   // cache row of key p: base_row + p (a shard's row 0 is position key_begin)
   const int64_t base_row = seq_base - a.key_begin;
   float* out = a.out + (int64_t)unit * kHeads * kDim;
+  // bounds-checked builds: the split's rows lie in the cache and its partial
+  // slot in the workspace (no CTA of this kernel waits on another)
+  if (!KCA_IN_BOUNDS(nsplit <= a.max_splits && base_row + kbeg >= 0 && base_row + kend <= a.cache_rows &&
+                         (nsplit == 1 || (int64_t)(unit + 1) * a.max_splits <= a.part_slots),
+                     status, kSiteBoundsRows, (unsigned)unit))
+    return;
 
   if (nkeys == 0) {  // fully masked row: exactly zero (as a partial: (-inf, 0, 0))
     if (warp < kComputeWarps)
@@ -366,6 +372,9 @@ __global__ void __launch_bounds__(256) merge_rows_kernel(const RowsArgs a) {
   const int64_t nkeys = rows_keys(a, pos, &lo);
   const int32_t nsplit = rows_n_splits(nkeys, rows_split_len(a, nkeys, kRowsSplitQuantum));
   if (nsplit <= 1) return;
+  if (!KCA_IN_BOUNDS(nsplit <= a.max_splits && (int64_t)(unit + 1) * a.max_splits <= a.part_slots,
+                     static_cast<DeviceStatus*>(a.status), kSiteBoundsMerge, (unsigned)unit))
+    return;
   __shared__ float red[8 * 264];
   const int64_t row0 = (int64_t)unit * a.max_splits * kHeads + h;
   merge_row<8>(nsplit, a.part_ml + row0 * 2, kHeads * 2, a.part_acc + row0 * kDim, kHeads * kDim,

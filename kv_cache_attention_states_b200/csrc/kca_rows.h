@@ -48,6 +48,11 @@ struct RowsArgs {
   // (m, l) here -- m the max scaled score, l the sum of exp(s - m) -- and
   // its unnormalised sum of exp(s - m) v in out; null: out = that sum / l.
   float* out_ml;
+  // Extents of the buffers the kernels address by computed offsets (checked
+  // in bounds-checked builds): cache rows the K / V pointers and maps cover,
+  // and partial slots (split or cluster partials) the workspace holds.
+  int64_t cache_rows;
+  int64_t part_slots;
   int64_t ctx[KCA_MAX_BATCH];  // decode: ctx_len per sequence
 };
 
