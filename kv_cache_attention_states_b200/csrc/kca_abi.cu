@@ -616,7 +616,7 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
     a.status = workspace;
     a.scale_log2 = scale * 1.4426950408889634f;
     carve(workspace, (size_t)a.plan.n_slots * 128 * 2 * 4, &a.part_ml, &a.part_acc);
-    kca::fill_tc_tables(a);
+    if (!kca::fill_tc_tables(a)) return KCA_ERR_RANGE;
     CUtensorMap tmk, tmv, tmq, tmo, tmpart, tmpart_rag;
     // K and V: 64 x 64 boxes (each CTA of a pair loads its half of a tile);
     // Q in 64-dim boxes of a 128-row tile; out / partials in 32-column boxes.

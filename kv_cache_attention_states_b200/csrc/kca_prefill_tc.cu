@@ -675,8 +675,10 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
 
 }  // namespace
 
-void fill_tc_tables(TcArgs& a) {
+bool fill_tc_tables(TcArgs& a) {
   // One pass over the pairs: O(pairs + items), no per-item plan walk.
+  if (a.plan.n_tiles < 1 || a.plan.n_tiles > kTcMaxTiles || a.plan.n_items < 1 || a.plan.n_items > kTcMaxItems)
+    return false;
   int32_t idx = 0, slot = 0;
   for (int32_t q = 0; q < a.plan.n_pairs && 2 * q < kTcMaxTiles; ++q) {
     int32_t kb, ke;
@@ -697,6 +699,23 @@ void fill_tc_tables(TcArgs& a) {
     }
     if (s > 1) slot += s * nt;
   }
+  // The tables must agree with the plan the workspace was sized for: every
+  // item filled, every partial slot inside the n_slots the workspace holds,
+  // every key tile inside the keys the K / V maps cover.
+  if (idx != a.plan.n_items || slot != a.plan.n_slots) return false;
+  const int64_t key_tiles = cdiv(a.plan.ctx_len - a.plan.kv_lo, (int64_t)kKeyTile);
+  for (int32_t i = 0; i < idx; ++i) {
+    const TcItemArg& it = a.items[i];
+    if (it.kt_begin < 0 || it.kt_end <= it.kt_begin || it.kt_end > key_tiles || it.pair < 0 ||
+        2 * it.pair >= a.plan.n_tiles)
+      return false;
+    for (int r = 0; r < 2; ++r)
+      if (it.slot[r] < -1 || it.slot[r] >= a.plan.n_slots) return false;
+  }
+  for (int32_t t = 0; t < a.plan.n_tiles; ++t)
+    if (a.tile_items[t] > 1 && (a.tile_first_slot[t] < 0 || a.tile_first_slot[t] + a.tile_items[t] > a.plan.n_slots))
+      return false;
+  return true;
 }
 
 cudaError_t launch_prefill_tc(int dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,

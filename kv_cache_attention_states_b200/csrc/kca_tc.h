@@ -34,8 +34,9 @@ struct TcArgs {
   int16_t tile_items[kTcMaxTiles];
 };
 
-// Fills the item and tile tables of a from a.plan (host).
-void fill_tc_tables(TcArgs& a);
+// Fills the item and tile tables from a.plan; false when they would not fit
+// the plan (launch tables, partial slots or the keys the maps cover).
+bool fill_tc_tables(TcArgs& a);
 
 // tmk / tmv: 2-D tensor maps over the rows [plan.kv_lo, plan.ctx_len) of the
 // K and V caches, inner extent 256, 128-byte swizzle, zero fill; boxes of 64
