@@ -499,7 +499,10 @@ int attn_decode_cluster_capacity(int32_t *capacity);
  * path where eligible (q and cache both F16 or both BF16).  op 1 (the rows
  * path: decode, and prefill chunks on the rows path): path 0 = the CUDA-core
  * kernel, 1 = the tensor-core (mma.sync) kernel where eligible (16-bit
- * cache).  path -1 restores the automatic choice described under DTYPES.
+ * cache).  op 2 (attn_prefill_batch with 2 or more rows per sequence on a
+ * 16-bit cache, multi-row units): path 0 = the mma.sync kernel, 1 = the
+ * tcgen05 kernel (the automatic choice).  path -1 restores the automatic
+ * choice described under DTYPES.
  * Plans, workspace queries and calls all follow the pinned choice, so pin
  * before sizing a workspace.  Returns KCA_OK or KCA_ERR_RANGE.
  * Passage: Karume v0.12.0 release notes, "Performance", items 2-3 (the

@@ -541,15 +541,17 @@ def attn_decode_static(q, k_cache, v_cache, ctx_len, window: int = 0, scale: flo
 
 # ------------------------------------------------------------ path control
 
-OP_PREFILL, OP_ROWS = 0, 1                       # attn_force_path operations
+OP_PREFILL, OP_ROWS, OP_BATCH = 0, 1, 2           # attn_force_path operations
 PATH_AUTO, PATH_ROWS, PATH_TENSOR_CORE = -1, 0, 1
 PATH_CUDA_CORE = 0                               # OP_ROWS: the CUDA-core kernel
+PATH_MMA_SYNC, PATH_TCGEN05 = 0, 1               # OP_BATCH: the multi-row kernels
 
 
 def attn_force_path(op: int, path: int) -> None:
     """Pin the kernel family of later calls, process-wide (see include/kca.h):
     op OP_PREFILL with PATH_ROWS / PATH_TENSOR_CORE, op OP_ROWS with
-    PATH_CUDA_CORE / PATH_TENSOR_CORE; PATH_AUTO restores the automatic choice."""
+    PATH_CUDA_CORE / PATH_TENSOR_CORE, op OP_BATCH with PATH_MMA_SYNC /
+    PATH_TCGEN05; PATH_AUTO restores the automatic choice."""
     _check(lib().attn_force_path(int(op), int(path)), "attn_force_path")
 
 

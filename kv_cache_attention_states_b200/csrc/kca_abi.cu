@@ -54,6 +54,7 @@ int current_sms(int* out) {
 // Paths pinned by attn_force_path (-1: automatic), read once per call.
 std::atomic<int> g_prefill_path{-1};
 std::atomic<int> g_rows_path{-1};
+std::atomic<int> g_batch_path{-1};
 
 // A forced prefill path (attn_force_path) wins where eligible; otherwise the
 // rules in kca.h choose.  Chunks of fewer than 16 rows: the rows path streams the visible keys once
@@ -274,6 +275,9 @@ bool use_rows_mma(int32_t kv_dtype) {
 // The batched call takes the multi-row tensor-core kernel for 16-bit caches
 // and more than one row per sequence (one row per sequence is decode).
 bool use_multirow(int32_t kv_dtype, int32_t rows) { return rows > 1 && use_rows_mma(kv_dtype); }
+// Multi-row units take the tcgen05 kernel unless attn_force_path pins the
+// mma.sync one (op 2, path 0).
+bool use_batch_tc() { return g_batch_path.load(std::memory_order_relaxed) != 0; }
 
 // Plan of the tensor-core rows kernel.  Each cluster size c in {8, 4, 2}
 // (and c = 1 when every unit fits one split, so nothing is merged) gets the
@@ -440,6 +444,7 @@ int attn_force_path(int32_t op, int32_t path) {
   if (path < -1 || path > 1) return KCA_ERR_RANGE;
   if (op == 0) g_prefill_path.store(path);
   else if (op == 1) g_rows_path.store(path);
+  else if (op == 2) g_batch_path.store(path);
   else return KCA_ERR_RANGE;
   return KCA_OK;
 }
@@ -873,7 +878,9 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
     if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, (int64_t)batch * capacity, 64) ||
         !encode_kv_map(&tmv, v_cache, kv_dtype, 0, (int64_t)batch * capacity, 64))
       return KCA_ERR_CUDA;
-    return kca::launch_decode_multirow(q_dtype, kv_dtype, tmk, tmv, a, s) == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+    const cudaError_t e = use_batch_tc() ? kca::launch_rows_tc(q_dtype, kv_dtype, tmk, tmv, a, s)
+                                         : kca::launch_decode_multirow(q_dtype, kv_dtype, tmk, tmv, a, s);
+    return e == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
   }
   const int32_t n_units = batch * rows;
   const std::vector<int64_t> nk = batch_unit_keys(batch, rows, ctx_len, window);

@@ -790,13 +790,17 @@ int cluster_capacity_t(int c) {
 // to the SM once for all of them.  The unit's keys are the union of its
 // rows' visible ranges, cut into splits of the host plan's length; each row
 // masks the keys it does not see (an empty row of a split writes the empty
-// partial (-inf, 0, 0)).  Per stage and warp: the K fragments of its 8 keys
-// are loaded once and multiplied by every row's query (hi/lo, from shared
-// memory), the stage max, lazy rescale and P of each row as in the decode
-// kernel, then the V fragments of its 32 dims are loaded once for every
-// row's P.  One CTA per split, no cluster: a unit with several splits writes
-// per-row partials that multirow_merge_kernel combines.
-constexpr int kMRows = 4;
+// partial (-inf, 0, 0)).  Per stage: two warps per row take its Q K^T, each
+// over 32 of the stage's 64 keys with the row's query (hi/lo) held in
+// registers for the whole split (re-reading every row's query from shared
+// memory for every stage made the kernel bound by shared-memory latency);
+// then the stage max of each row (its two warps), lazy rescale and P as in
+// the decode kernel; then each warp loads the V fragments of its 32 dims
+// once for every row's P.  One CTA per split, no cluster: a unit with
+// several splits writes per-row partials that multirow_merge_kernel
+// combines.
+constexpr int kMRows = kMultiRows;
+static_assert(2 * kMRows == kDWarps, "the multi-row kernel gives each row two warps");
 constexpr int kMStages = 2;
 constexpr int kMOffBar = kMStages * kDStageBytes;    // 128 KiB
 
@@ -804,21 +808,11 @@ struct MBars {
   uint64_t full[kMStages];
   uint64_t empty[kMStages];
   int abort;
-  float red[kDWarps][kMRows][8];
+  float red[kDWarps][8];                 // per warp and head: stage max, then row sum
   __align__(16) unsigned char p[kMRows][16 * kDPRow];
-  __align__(16) unsigned char qs[kMRows][16 * kDQRow];
+  __align__(16) unsigned char qs[kMRows * 16 * kDQRow];   // the rows' queries, before they move to registers
 };
 constexpr int kMSmemBytes = kMOffBar + (int)sizeof(MBars) + 1024;
-
-// Unit u of a batched call: sequence *b, first row *i0 (of the sequence's
-// rows), *nr rows; positions ctx[b] - rows + i0 + r.
-__device__ __forceinline__ void multirow_unit(const RowsArgs& a, int u, int* b, int* i0, int* nr) {
-  const int blocks = (a.rows_per_seq + kMRows - 1) / kMRows;
-  *b = u / blocks;
-  *i0 = (u % blocks) * kMRows;
-  const int left = a.rows_per_seq - *i0;
-  *nr = left < kMRows ? left : kMRows;
-}
 
 template <int QT, int KT>
 __global__ void __launch_bounds__(kDThreads, 1)
@@ -830,6 +824,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
   unsigned char* smem = smem_raw + pad;
   const uint32_t sbase = raw_addr + pad;
   MBars* bars = reinterpret_cast<MBars*>(smem + kMOffBar);
+  unsigned char* qs = bars->qs;                         // [kMRows][16][kDQRow]
   volatile int* abort_flag = &bars->abort;
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.status);
 
@@ -921,13 +916,27 @@ __global__ void __launch_bounds__(kDThreads, 1)
           const float2 f = unpack16<KT>(hi[j]);
           lo[j] = pack16<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
         }
-        *reinterpret_cast<uint4*>(bars->qs[r] + h * kDQRow + d0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(bars->qs[r] + (h + 8) * kDQRow + d0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(qs + r * 16 * kDQRow + h * kDQRow + d0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(qs + r * 16 * kDQRow + (h + 8) * kDQRow + d0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
     }
     const int mi = lane >> 3;
-    const uint32_t qoff = (8 * (mi & 1) + (lane & 7)) * kDQRow + 8 * (mi >> 1) * 2;
+    // Q K^T: warp w takes row qr = w / 2 of the unit and keys 32 (w % 2) ..
+    // + 31 of every stage, with that row's query (16-bit high and low parts
+    // as M rows 0-7 / 8-15) held in registers for the whole split, so no
+    // stage reads a query from shared memory.  P V: warp w takes dims
+    // 32 w .. + 31 of every row, as in the single-row kernel.
+    const int qr = warp >> 1, kh = warp & 1;
+    const bool q_live = qr < nr;
+    uint32_t qa[16][4];
+    {
+      const uint32_t qrow = smem_u32(qs + (q_live ? qr : 0) * 16 * kDQRow) + (8 * (mi & 1) + (lane & 7)) * kDQRow +
+                            8 * (mi >> 1) * 2;
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) ldsm_x4(qrow + 32 * ks, qa[ks]);
+    }
+    const int64_t qpos = pos0 + qr, qlo = lo_of(qpos, a.window);
     float o[kMRows][4][4];
 #pragma unroll
     for (int r = 0; r < kMRows; ++r)
@@ -935,15 +944,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) o[r][i][j] = 0.f;
-    float m_ref[kMRows], l_part[kMRows];
-    int64_t rlo[kMRows], rpos[kMRows];
+    float m_ref[kMRows];
 #pragma unroll
-    for (int r = 0; r < kMRows; ++r) {
-      m_ref[r] = -INFINITY;
-      l_part[r] = 0.f;
-      rpos[r] = pos0 + r;
-      rlo[r] = lo_of(rpos[r], a.window);
-    }
+    for (int r = 0; r < kMRows; ++r) m_ref[r] = -INFINITY;
+    float l_own = 0.f;   // row qr, head g, this warp's keys
     const float scale = a.scale;
     bool ok = true;
 
@@ -955,9 +959,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const int cnt = (int)((kend - k0) < kDStageKeys ? (kend - k0) : kDStageKeys);
       const uint32_t kst = sbase + slot * kDStageBytes;
       const uint32_t vst = kst + kDHalfBytes;
-      float sx[kMRows][2];
+      float sx[4][2];
 #pragma unroll
-      for (int r = 0; r < kMRows; ++r) sx[r][0] = sx[r][1] = -INFINITY;
+      for (int nt = 0; nt < 4; ++nt) sx[nt][0] = sx[nt][1] = -INFINITY;
       if (ok) {
         if (cnt < kDStageKeys) {  // V rows past the split's end -> 0
           unsigned char* vrows = smem + slot * kDStageBytes + kDHalfBytes;
@@ -967,78 +971,75 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 make_uint4(0, 0, 0, 0);
           }
         }
-        float sacc[kMRows][2][4];
+        if (q_live) {
+          // one accumulation chain per 8-key tile: four independent chains
+          float sacc[4][4];
 #pragma unroll
-        for (int r = 0; r < kMRows; ++r)
+          for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+            for (int j = 0; j < 4; ++j) sacc[nt][j] = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) sacc[r][c][j] = 0.f;
-        const int kr = 8 * warp + (lane & 7);
+          for (int ks2 = 0; ks2 < 8; ++ks2) {
 #pragma unroll
-        for (int ks2 = 0; ks2 < 8; ++ks2) {
-          uint32_t bk[4];
-          ldsm_x4(kst + swz(kr, 32 * ks2 + 8 * (lane >> 3)), bk);
-#pragma unroll
-          for (int r = 0; r < kMRows; ++r) {
-            if (r < nr) {
-              uint32_t qa0[4], qa1[4];
-              const uint32_t qb = smem_u32(bars->qs[r]) + qoff;
-              ldsm_x4(qb + 32 * (2 * ks2), qa0);
-              ldsm_x4(qb + 32 * (2 * ks2 + 1), qa1);
-              mma16816<KT>(sacc[r][0], qa0, bk[0], bk[1]);
-              mma16816<KT>(sacc[r][1], qa1, bk[2], bk[3]);
+            for (int nt = 0; nt < 4; ++nt) {
+              uint32_t bk[4];
+              ldsm_x4(kst + swz(32 * kh + 8 * nt + (lane & 7), 32 * ks2 + 8 * (lane >> 3)), bk);
+              mma16816<KT>(sacc[nt], qa[2 * ks2], bk[0], bk[1]);
+              mma16816<KT>(sacc[nt], qa[2 * ks2 + 1], bk[2], bk[3]);
             }
           }
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const int kk = 32 * kh + 8 * nt + 2 * tig;
+            const int64_t key = k0 + kk;
+            const float s0 = sacc[nt][0] + sacc[nt][2];   // high + low parts of head g
+            const float s1 = sacc[nt][1] + sacc[nt][3];
+            sx[nt][0] = kk < cnt && key >= qlo && key <= qpos ? s0 * scale : -INFINITY;
+            sx[nt][1] = kk + 1 < cnt && key + 1 >= qlo && key + 1 <= qpos ? s1 * scale : -INFINITY;
+          }
         }
-        const int kk0 = 8 * warp + 2 * tig;
-        const int64_t key0 = k0 + kk0;
+      }
+      // Stage max of every row and head: this warp's 32 keys, then the row's
+      // two warps (every warp needs every row's max for its P V columns).
+      float mw = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) mw = max_nan(mw, max_nan(sx[nt][0], sx[nt][1]));
+      mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 1));
+      mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 2));
+      if (tig == 0) bars->red[warp][g] = mw;
+      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
+      if (ok) {
+        float mq = -INFINITY;
 #pragma unroll
         for (int r = 0; r < kMRows; ++r) {
           if (r < nr) {
-            const float s0 = (sacc[r][0][0] + sacc[r][1][0]) + (sacc[r][0][2] + sacc[r][1][2]);
-            const float s1 = (sacc[r][0][1] + sacc[r][1][1]) + (sacc[r][0][3] + sacc[r][1][3]);
-            const bool v0 = kk0 < cnt && key0 >= rlo[r] && key0 <= rpos[r];
-            const bool v1 = kk0 + 1 < cnt && key0 + 1 >= rlo[r] && key0 + 1 <= rpos[r];
-            sx[r][0] = v0 ? s0 * scale : -INFINITY;
-            sx[r][1] = v1 ? s1 * scale : -INFINITY;
-          }
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < kMRows; ++r) {
-        float mw = max_nan(sx[r][0], sx[r][1]);
-        mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 1));
-        mw = max_nan(mw, __shfl_xor_sync(0xffffffffu, mw, 2));
-        if (tig == 0) bars->red[warp][r][g] = mw;
-      }
-      asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
-#pragma unroll
-      for (int r = 0; r < kMRows; ++r) {
-        if (r < nr) {
-          float ms = bars->red[0][r][g];
-#pragma unroll
-          for (int w = 1; w < kDWarps; ++w) ms = max_nan(ms, bars->red[w][r][g]);
-          if (ok) {
+            const float ms = max_nan(bars->red[2 * r][g], bars->red[2 * r + 1][g]);
             if (ms > m_ref[r] + kDRescale) {
               const float alpha = exp2f((m_ref[r] - ms) * kDLog2e);
               m_ref[r] = ms;
-              l_part[r] *= alpha;
+              if (r == qr) l_own *= alpha;
 #pragma unroll
               for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) o[r][nt][j] *= alpha;
             }
-            const float mu = m_ref[r] == -INFINITY ? 0.f : m_ref[r];
-            const float p0 = exp2f((sx[r][0] - mu) * kDLog2e);
-            const float p1 = exp2f((sx[r][1] - mu) * kDLog2e);
-            l_part[r] += p0 + p1;
+            if (r == qr) mq = m_ref[r];
+          }
+        }
+        if (q_live) {
+          const float mu = mq == -INFINITY ? 0.f : mq;
+          unsigned char* prow = bars->p[qr];
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const float p0 = exp2f((sx[nt][0] - mu) * kDLog2e);
+            const float p1 = exp2f((sx[nt][1] - mu) * kDLog2e);
+            l_own += p0 + p1;
             const uint32_t hi = pack16<KT>(p0, p1);
             const float2 f = unpack16<KT>(hi);
             const uint32_t lo16 = pack16<KT>(p0 - f.x, p1 - f.y);
-            const int key = 8 * warp + 2 * tig;
-            *reinterpret_cast<uint32_t*>(bars->p[r] + g * kDPRow + key * 2) = hi;
-            *reinterpret_cast<uint32_t*>(bars->p[r] + (g + 8) * kDPRow + key * 2) = lo16;
+            const int key = 32 * kh + 8 * nt + 2 * tig;
+            *reinterpret_cast<uint32_t*>(prow + g * kDPRow + key * 2) = hi;
+            *reinterpret_cast<uint32_t*>(prow + (g + 8) * kDPRow + key * 2) = lo16;
           }
         }
       }
@@ -1071,22 +1072,19 @@ __global__ void __launch_bounds__(kDThreads, 1)
       if (lane == 0) mbar_arrive(&bars->empty[slot]);
     }
 
-    // Row sums of every row: lanes of one head, then warps.
-#pragma unroll
-    for (int r = 0; r < kMRows; ++r) {
-      float l = l_part[r];
+    // Row sums: lanes of one head, then the row's two warps.
+    {
+      float l = l_own;
       l += __shfl_xor_sync(0xffffffffu, l, 1);
       l += __shfl_xor_sync(0xffffffffu, l, 2);
-      if (tig == 0) bars->red[warp][r][g] = l;
+      if (tig == 0) bars->red[warp][g] = l;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
     const bool aborted = !ok || *abort_flag;
 #pragma unroll
     for (int r = 0; r < kMRows; ++r) {
       if (r < nr) {
-        float L = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDWarps; ++w) L += bars->red[w][r][g];
+        float L = bars->red[2 * r][g] + bars->red[2 * r + 1][g];
         float M = m_ref[r];
         if (aborted) {
           M = NAN;   // an aborted split poisons its rows; the status word says why
@@ -1164,6 +1162,15 @@ cudaError_t launch_multirow_t(const CUtensorMap& tmk, const CUtensorMap& tmv, co
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a);
   if (e != cudaSuccess || a.max_splits <= 1) return e;
+  return launch_multirow_merge(a, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_multirow_merge(const RowsArgs& a, cudaStream_t stream) {
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = 1;
   const int blocks = (a.rows_per_seq + kMRows - 1) / kMRows;
   const int64_t rows_total = (int64_t)(a.n_units / blocks) * a.rows_per_seq;
   cudaLaunchConfig_t mcfg = {};
@@ -1174,8 +1181,6 @@ cudaError_t launch_multirow_t(const CUtensorMap& tmk, const CUtensorMap& tmv, co
   mcfg.numAttrs = 1;
   return cudaLaunchKernelEx(&mcfg, multirow_merge_kernel, a);
 }
-
-}  // namespace
 
 int decode_mma_cluster_capacity(int c) {
   // Same launch shape for every dtype instantiation; cached per device and size.

@@ -56,6 +56,9 @@ struct RowsArgs {
   int64_t ctx[KCA_MAX_BATCH];  // decode: ctx_len per sequence
 };
 
+// Rows of one unit of the batched multi-row kernels.
+constexpr int kMultiRows = 4;
+
 #if defined(__CUDACC__)
 }  // namespace kca
 #include "kca_common.cuh"
@@ -103,6 +106,10 @@ __device__ __forceinline__ float rows_final(const RowsArgs& a, float acc, float 
   if (a.out_ml != nullptr) return acc;
   return (M == -INFINITY && L == 0.f) ? 0.f : acc / L;
 }
+// Unit u of a batched call in multi-row units (kMultiRows rows each):
+// sequence *b, first row *i0 (of the sequence's rows), *nr rows; positions
+// ctx[b] - rows_per_seq + i0 + r.
+__device__ __forceinline__ void multirow_unit(const RowsArgs& a, int u, int* b, int* i0, int* nr);
 // Keys per split of a unit with nkeys visible keys: the host plan's length,
 // or with device context lengths the smallest multiple of `quantum` (>= 64)
 // that cuts nkeys into at most max_splits splits.
@@ -111,6 +118,13 @@ __device__ __forceinline__ int32_t rows_split_len(const RowsArgs& a, int64_t nke
   int64_t s = (nkeys + a.max_splits - 1) / a.max_splits;
   s = (s + quantum - 1) / quantum * quantum;
   return (int32_t)(s < 64 ? 64 : s);
+}
+__device__ __forceinline__ void multirow_unit(const RowsArgs& a, int u, int* b, int* i0, int* nr) {
+  const int blocks = (a.rows_per_seq + kMultiRows - 1) / kMultiRows;
+  *b = u / blocks;
+  *i0 = (u % blocks) * kMultiRows;
+  const int left = a.rows_per_seq - *i0;
+  *nr = left < kMultiRows ? left : kMultiRows;
 }
 #endif
 
@@ -157,13 +171,18 @@ cudaError_t launch_decode_mma_q8(int q_dtype, int v_dtype, const CUtensorMap& tm
                                  const CUtensorMap& tmv, const RowsArgs& a, cudaStream_t stream);
 
 // Batched short chunks on the tensor cores (mode 2, 16-bit K/V): units of up
-// to 4 consecutive rows of one sequence (n_units = batch x ceil(rows / 4)),
-// the union of their keys cut into splits of split_len; per-row split
-// partials in part_ml / part_acc ([batch * rows][max_splits][8]) merged by a
-// second kernel.
-constexpr int kMultiRows = 4;
+// to kMultiRows consecutive rows of one sequence (n_units = batch x
+// ceil(rows / kMultiRows)), the union of their keys cut into splits of
+// split_len; per-row split partials in part_ml / part_acc
+// ([batch * rows][max_splits][8]) merged by a second kernel
+// (launch_multirow_merge).  launch_decode_multirow: mma.sync fragments
+// (kca_decode_mma.cu); launch_rows_tc: tcgen05 MMAs with TMEM accumulators
+// (kca_rows_tc.cu).  tmk / tmv as for launch_decode_mma.
 cudaError_t launch_decode_multirow(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                    const RowsArgs& a, cudaStream_t stream);
+cudaError_t launch_rows_tc(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                           const RowsArgs& a, cudaStream_t stream);
+cudaError_t launch_multirow_merge(const RowsArgs& a, cudaStream_t stream);
 
 // Clusters of c CTAs of the tensor-core rows kernel that fit on the device at
 // once (0 on failure).

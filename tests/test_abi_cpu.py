@@ -51,7 +51,8 @@ def test_every_declared_call_cites_its_passage():
 
 def test_force_path_validates_and_restores():
     lib = kca.lib()
-    assert lib.attn_force_path(2, 0) == -4 and lib.attn_force_path(0, 2) == -4
+    assert lib.attn_force_path(3, 0) == -4 and lib.attn_force_path(0, 2) == -4
+    assert lib.attn_force_path(2, 0) == 0 and lib.attn_force_path(2, -1) == 0   # op 2: the multi-row kernels
     assert lib.attn_force_path(-1, 0) == -4 and lib.attn_force_path(1, -2) == -4
     assert kca.attn_prefill_path(kca.BF16, kca.BF16, 0, 768) == 1
     with kca.forced_path(kca.OP_PREFILL, kca.PATH_ROWS):

@@ -2,10 +2,11 @@
 one call, every row against the f64 oracle (row i of sequence b at position
 ctx[b] - rows + i, its own sequence's keys), for 1, 8 and 64 sequences of
 ragged contexts (the shortest exactly `rows` long, one at the capacity),
-the multi-row tensor-core kernel (16-bit cache: units of up to 4 rows of a
-sequence) and the CUDA-core kernel (f32 cache), with and without a window,
-against attn_prefill of the same rows; and with one row per sequence it is
-attn_decode, bit for bit."""
+both multi-row tensor-core kernels (16-bit cache: units of up to 4 rows of
+a sequence; the tcgen05 kernel and the mma.sync one, pinned with
+attn_force_path) and the CUDA-core kernel (f32 cache), with and without a
+window, against attn_prefill of the same rows; and with one row per
+sequence it is attn_decode, bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -22,6 +23,16 @@ pytestmark = pytest.mark.gpu
 def _setup(cuda_ok):
     oracle_threads()
     kca.lib()
+
+
+# the multi-row kernel of 16-bit caches: tcgen05 (the automatic choice) or mma.sync
+BATCH_PATHS = [kca.PATH_TCGEN05, kca.PATH_MMA_SYNC]
+
+
+@pytest.fixture(params=BATCH_PATHS, ids=["tcgen05", "mma_sync"])
+def batch_path(request):
+    with kca.forced_path(kca.OP_BATCH, request.param):
+        yield request.param
 
 
 def _inputs(seed, batch, rows, cap, q_dtype, kv_dtype):
@@ -46,7 +57,7 @@ def _oracle(q, k, v, ctx, rows, window, q_dtype, kv_dtype):
 
 @pytest.mark.parametrize("batch", [1, 8, 64])
 @pytest.mark.parametrize("rows", [1, 3, 15])
-def test_batched_short_chunks_match_oracle(batch, rows):
+def test_batched_short_chunks_match_oracle(batch, rows, batch_path):
     cap = 20000 if batch <= 8 else 5000
     ctx, q, k, v = _inputs(40 + rows, batch, rows, cap, "f32", "f16")
     ws = kca.new_workspace(kca.attn_prefill_batch_workspace_bytes(ctx, rows))
@@ -59,7 +70,7 @@ def test_batched_short_chunks_match_oracle(batch, rows):
 
 @pytest.mark.parametrize("q_dtype,kv_dtype,window", [("bf16", "bf16", 300), ("f32", "f32", 0), ("f32", "f32", 700),
                                                      ("f16", "bf16", 0)])
-def test_batched_short_chunks_dtypes_and_window(q_dtype, kv_dtype, window):
+def test_batched_short_chunks_dtypes_and_window(q_dtype, kv_dtype, window, batch_path):
     batch, rows, cap = 8, 5, 9000
     ctx, q, k, v = _inputs(50, batch, rows, cap, q_dtype, kv_dtype)
     out = kca.attn_prefill_batch(dev(q, q_dtype), dev(k, kv_dtype), dev(v, kv_dtype), ctx, window)
@@ -78,7 +89,7 @@ def test_one_row_per_sequence_is_decode_bit_for_bit(kv_dtype):
 
 
 @pytest.mark.parametrize("rows", [2, 4, 5, 7, 15])
-def test_rows_of_one_sequence_match_a_prefill_chunk(rows):
+def test_rows_of_one_sequence_match_a_prefill_chunk(rows, batch_path):
     # one sequence: the batched call (multi-row units of up to 4 rows) and
     # attn_prefill of the same rows agree; both against the oracle
     cap = 3000
@@ -93,7 +104,7 @@ def test_rows_of_one_sequence_match_a_prefill_chunk(rows):
     assert max_err(got.cpu().numpy(), ref) <= 4e-3
 
 
-def test_multirow_units_with_a_window_cut_inside_a_unit():
+def test_multirow_units_with_a_window_cut_inside_a_unit(batch_path):
     # window 100 over 15 rows: the unit's rows see different ranges, and the
     # first rows' keys before the later rows' windows are masked per row
     batch, rows, cap = 5, 15, 6000
@@ -104,7 +115,7 @@ def test_multirow_units_with_a_window_cut_inside_a_unit():
 
 
 @pytest.mark.parametrize("q_dtype,kv_dtype", [("f32", "f16"), ("f32", "f32")])
-def test_batched_short_chunks_at_the_maximum_sizes(q_dtype, kv_dtype):
+def test_batched_short_chunks_at_the_maximum_sizes(q_dtype, kv_dtype, batch_path):
     # KCA_MAX_BATCH sequences x KCA_MAX_BATCH_ROWS rows (3,840 rows, 1,024
     # multi-row units on 16-bit caches), short ragged contexts
     batch, rows, cap = kca.MAX_BATCH, kca.MAX_BATCH_ROWS, 96
@@ -117,3 +128,41 @@ def test_batched_short_chunks_at_the_maximum_sizes(q_dtype, kv_dtype):
     with pytest.raises(kca.KcaError):   # one row more than the limit: rejected before any launch
         kca.attn_prefill_batch(torch.zeros((1, rows + 1, 8, 256), device="cuda"),
                                dev(k[:1], kv_dtype), dev(v[:1], kv_dtype), [rows + 1])
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("f32", "f16"), ("f32", "bf16"), ("bf16", "bf16"), ("f16", "f16")])
+def test_the_two_multirow_kernels_agree(q_dtype, kv_dtype):
+    # long ragged contexts (several splits per unit, a ragged last stage),
+    # rows 6 (units of 4 and 2): tcgen05 and mma.sync within the tolerance of
+    # the inputs' type, both within it of the oracle on sampled sequences
+    batch, rows, cap = 12, 6, 40000
+    ctx, q, k, v = _inputs(64, batch, rows, cap, q_dtype, kv_dtype)
+    qd, kd, vd = dev(q, q_dtype), dev(k, kv_dtype), dev(v, kv_dtype)
+    outs = {}
+    for path in BATCH_PATHS:
+        with kca.forced_path(kca.OP_BATCH, path):
+            ws = kca.new_workspace(kca.attn_prefill_batch_workspace_bytes(ctx, rows))
+            outs[path] = kca.attn_prefill_batch(qd, kd, vd, ctx, workspace=ws).cpu().numpy()
+            assert kca.attn_device_status(ws)[0] == 0
+    assert np.isfinite(outs[kca.PATH_TCGEN05]).all()
+    assert np.max(np.abs(outs[kca.PATH_TCGEN05] - outs[kca.PATH_MMA_SYNC])) <= tol(q_dtype, kv_dtype)
+    seqs = [0, 1, 7]
+    want = _oracle(q[seqs], k[seqs], v[seqs], [ctx[s] for s in seqs], rows, 0, q_dtype, kv_dtype)
+    for path in BATCH_PATHS:
+        assert max_err(outs[path][seqs], want) <= tol(q_dtype, kv_dtype)
+
+
+def test_tcgen05_multirow_nan_score_reaches_exactly_the_rows_that_see_it():
+    # a NaN in key j of sequence 0: rows at positions >= j are NaN, the
+    # others (and other sequences) finite and equal to the oracle
+    batch, rows, cap = 3, 7, 5000
+    ctx, q, k, v = _inputs(65, batch, rows, cap, "f32", "f16")
+    ctx[0] = 4000
+    j = ctx[0] - 4                      # seen by rows 3..6 of sequence 0
+    k[0, j, 17] = np.float16(np.nan)
+    with kca.forced_path(kca.OP_BATCH, kca.PATH_TCGEN05):
+        out = kca.attn_prefill_batch(dev(q, "f32"), dev(k, "f16"), dev(v, "f16"), ctx).cpu().numpy()
+    assert np.isnan(out[0, 3:]).all()
+    assert np.isfinite(out[0, :3]).all() and np.isfinite(out[1:]).all()
+    want = _oracle(q[1:], k[1:], v[1:], ctx[1:], rows, 0, "f32", "f16")
+    assert max_err(out[1:], want) <= 4e-3
