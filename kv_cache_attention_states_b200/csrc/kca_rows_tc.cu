@@ -10,27 +10,36 @@
 // K / V stage crosses from L2 once for all of them.  The mma.sync form of
 // this kernel is bound by instruction issue (two warps per SM sub-partition
 // run the QK^T and PV fragments, the softmax and the shared-memory traffic
-// of every stage); here one thread issues every MMA and one warp runs the
-// softmax, so the tensor pipe and the load stream overlap.
+// of every stage); here one thread issues every MMA and four warps run the
+// softmax, so the tensor pipe and the load stream overlap.  A clock trace of
+// one split showed the MMA issue of Q K^T as the longest step of a stage,
+// which is why its high and low parts share one instruction (as M rows).
 //
-// Rows: M row m = 8 i + h (i the unit's row, h the head), 32 of the MMAs'
-// 128 M rows; rows 32-127 of every operand and accumulator are never read.
-// f32 queries keep f32-grade products: q = q_hi + q_lo (16-bit parts of the
-// cache's type) and S = q_hi K^T + q_lo K^T accumulate into the same
-// tensor-memory columns; P = p_hi + p_lo the same way in O += P V.
+// Rows: M row m = 8 i + h (i the unit's row, h the head) holds the high
+// part of the query, M row 32 + m its low part (f32 queries keep f32-grade
+// products: q = q_hi + q_lo in 16-bit parts of the cache's type), so one
+// Q K^T MMA of M = 128 gives both partial scores, in TMEM lanes m and 32 + m;
+// rows 64-127 of the operands and accumulators are never read.  In O += P V
+// the probabilities are split the same way, p = p_hi + p_lo, and both parts
+// accumulate into the same O columns (two passes over the keys).
 //
-// Warp roles (4 warps):
-//   warp 0   softmax of TMEM lanes 0-31 (the unit's rows), then the epilogue
-//   warp 1   TMEM allocator; lane 0 issues every MMA; the warp zeroes the V
+// Warp roles (16 warps, all of which stage the queries):
+//   warps 0, 4, 8, 12   softmax of TMEM lanes 0-31 (the unit's rows), 16 of
+//                       every stage's 64 key columns each, then the epilogue
+//   warps 1, 5, 9, 13   (f32 or mixed queries) read the low-part scores of
+//                       the same columns from lanes 32-63 and hand them over
+//                       through shared memory (only warps 4 k + 1 reach
+//                       those lanes, only warps 4 k reach lanes 0-31)
+//   warp 2   TMEM allocator; lane 0 issues every MMA; the warp zeroes the V
 //            rows of a ragged last stage
-//   warp 2   TMA producer of K stages (64 keys x 256 dims, ring of 3)
-//   warp 3   TMA producer of V stages (ring of 2)
-// Shared memory: Q high and low parts (32 rows x 256 dims each, four
-// 64-dim chunks of 4 KiB with 128-byte swizzle) and 16 KiB of zeros that
-// rows 32-127 of the last chunks' descriptors read; the K and V rings.
-// Tensor memory (512 columns): S of stage j at [64 (j & 1), +64), P of stage
-// j at [128 + 64 (j & 1), +64) (high parts, then low parts, as 16-bit
-// pairs), O at [256, 512).
+//   warps 3, 7   TMA producers of K stages (64 keys x 256 dims, ring of 3)
+//                and of V stages (ring of 2)
+// Shared memory: Q (64 M rows x 256 dims, four 64-dim chunks of 8 KiB with
+// 128-byte swizzle; the descriptors of the last chunk reach on into the
+// bytes after it, which land only in unused M rows), the K and V rings, the
+// low-part scores in flight.  Tensor memory (512 columns): S of stage j at
+// [64 (j & 1), +64), P of stage j at [128 + 64 (j & 1), +64) (high parts,
+// then low parts, as 16-bit pairs), O at [256, 512).
 // Per stage j the MMA thread issues Q K^T of stage j, then P V of stage
 // j - 1 once the softmax has written its P, so the softmax of a stage runs
 // under the MMAs of its neighbours.  The softmax keeps a reference max per
@@ -48,27 +57,27 @@
 namespace kca {
 namespace {
 
-constexpr int kRThreads = 128;
+constexpr int kRThreads = 512;
+constexpr int kRSoftmaxThreads = 128;                // warps 0, 4, 8, 12
 constexpr int kRKeys = 64;                           // keys per stage
 constexpr int kRBox = 64 * 64 * 2;                   // 64 rows x 64 dims (16-bit): 8 KiB
 constexpr int kRSlot = 4 * kRBox;                    // K or V of one stage: 32 KiB
 constexpr int kRKRing = 3, kRVRing = 2;
-constexpr int kRQRows = 8 * kMultiRows;              // 32 M rows
-constexpr int kRQChunk = kRQRows * 128;              // 32 rows x 64 dims: 4 KiB
-constexpr int kRQBytes = 4 * kRQChunk;               // one part (high or low): 16 KiB
-constexpr int kROffQHi = 0;
-constexpr int kROffQLo = kRQBytes;
-constexpr int kROffPad = 2 * kRQBytes;               // zeros: rows 32-127 of the last chunks
-constexpr int kRPadBytes = 16 * 1024;
-constexpr int kROffK = kROffPad + kRPadBytes;        // 48 KiB
-constexpr int kROffV = kROffK + kRKRing * kRSlot;    // 144 KiB
-constexpr int kROffBar = kROffV + kRVRing * kRSlot;  // 208 KiB
-constexpr int kRBarBytes = 1024;
+constexpr int kRQRows = 8 * kMultiRows;              // 32 query rows x heads, twice (high, low)
+constexpr int kRQChunk = 2 * kRQRows * 128;          // 64 M rows x 64 dims: 8 KiB
+constexpr int kROffQ = 0;
+constexpr int kROffK = 4 * kRQChunk;                 // 32 KiB
+constexpr int kROffV = kROffK + kRKRing * kRSlot;    // 128 KiB
+constexpr int kROffLo = kROffV + kRVRing * kRSlot;   // 192 KiB: float [2][4][16][32]
+constexpr int kRLoBytes = 2 * 4 * 16 * 32 * 4;
+constexpr int kROffBar = kROffLo + kRLoBytes;        // 208 KiB
+constexpr int kRBarBytes = 2048;
 constexpr int kRSmemBytes = kROffBar + kRBarBytes + 1024;   // + alignment slack
 static_assert(kRSmemBytes <= 232448, "shared memory over the per-CTA limit");
-// A descriptor of 128 M rows starting at chunk 3 of the low part reads up
-// to 12 KiB past the part: inside the zero pad.
-static_assert(kROffQLo + 3 * kRQChunk + 16 * 1024 <= kROffK, "Q descriptors stay in the Q area");
+// A descriptor of 128 M rows starting at the last Q chunk reads 8 KiB past
+// the Q area, into the first K slot: those bytes only reach M rows 64-127
+// of S, which nothing reads (an MMA's D row depends on its A row alone).
+static_assert(kROffQ + 3 * kRQChunk + 16 * 1024 <= kROffV, "Q descriptors stay inside shared memory");
 constexpr uint32_t kRColS = 0, kRColP = 128, kRColO = 256, kRTmemCols = 512;
 constexpr float kRRescaleLog2 = 8.f;   // rescale O once a score passes the reference by 2^8
 
@@ -76,11 +85,13 @@ struct RBars {
   uint64_t kfull[kRKRing], kempty[kRKRing];
   uint64_t vfull[kRVRing], vempty[kRVRing];
   uint64_t s_full[2];   // Q K^T of stage j complete in S buffer j & 1 (MMA commit)
-  uint64_t p_full[2];   // P of stage j written and O corrected (softmax warp)
+  uint64_t p_full[2];   // P of stage j written and O corrected (the four softmax warps)
   uint64_t o_done[2];   // P V of stage j complete (MMA commit)
   uint64_t drain;       // every MMA complete (single use)
   uint32_t tmem_base;
   int abort;
+  float red[2][4][32];  // [stage parity][softmax warp][row]: partial row maxima
+  float red_l[4][32];   // [softmax warp][row]: partial row sums at the end
 };
 static_assert(sizeof(RBars) <= kRBarBytes, "barrier block too large");
 
@@ -101,6 +112,9 @@ __device__ __forceinline__ float2 upk2(uint32_t u) {
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 template <int QT, int KT>
@@ -151,19 +165,19 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 1);
+      mbar_init(&bars->p_full[s], kRSoftmaxThreads / 32);
       mbar_init(&bars->o_done[s], 1);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == 2) {
     ptx::tmem_alloc(smem_u32(&bars->tmem_base), kRTmemCols);
     ptx::tmem_relinquish();
   }
-  if (threadIdx.x == 64) ptx::prefetch_tmap(&tmk);
-  if (threadIdx.x == 96) ptx::prefetch_tmap(&tmv);
+  if (threadIdx.x == 3 * 32) ptx::prefetch_tmap(&tmk);
+  if (threadIdx.x == 7 * 32) ptx::prefetch_tmap(&tmv);
   ptx::fence_before_sync();
   __syncthreads();
   ptx::fence_after_sync();
@@ -172,8 +186,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
   // kernel of the stream; global memory is touched only after this wait.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // Stage the queries: M row m = 8 i + h, 16-byte group u of its 256 dims
-  // (chunk u / 8, 128-byte swizzle within the chunk); high and low parts.
+  // Stage the queries: M row m = 8 i + h (high part) and 32 + m (low part),
+  // 16-byte group u of the 256 dims (chunk u / 8, 128-byte swizzle within it).
   for (int it = threadIdx.x; it < kRQRows * 32; it += kRThreads) {
     const int m = it >> 5, u = it & 31;
     const int i = m >> 3, h = m & 7;
@@ -189,19 +203,19 @@ __global__ void __launch_bounds__(kRThreads, 1)
       const float2 f = upk2<KT>(hi[j]);
       lo[j] = pk2<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
     }
-    const int off = (u >> 3) * kRQChunk + m * 128 + (((u & 7) ^ (m & 7)) << 4);
-    *reinterpret_cast<uint4*>(smem + kROffQHi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(smem + kROffQLo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    const int mh = m, ml = kRQRows + m;
+    *reinterpret_cast<uint4*>(smem + kROffQ + (u >> 3) * kRQChunk + mh * 128 + (((u & 7) ^ (mh & 7)) << 4)) =
+        make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(smem + kROffQ + (u >> 3) * kRQChunk + ml * 128 + (((u & 7) ^ (ml & 7)) << 4)) =
+        make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
-  for (int it = threadIdx.x; it < kRPadBytes / 16; it += kRThreads)
-    *reinterpret_cast<uint4*>(smem + kROffPad + 16 * it) = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();   // generic stores -> visible to the tensor core
   __syncthreads();
 
-  if (warp >= 2) {
+  if (warp == 3 || warp == 7) {
     // ------------------------------------------------------------ producers
     if (lane == 0) {
-      const bool is_k = warp == 2;
+      const bool is_k = warp == 3;
       const int ring = is_k ? kRKRing : kRVRing;
       uint64_t* full = is_k ? bars->kfull : bars->vfull;
       uint64_t* empty = is_k ? bars->kempty : bars->vempty;
@@ -227,15 +241,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 2) {
     // ----------------------------------------------------------------- MMA
     constexpr uint32_t ab = KT == KCA_BF16 ? 1u : 0u;
     constexpr uint32_t id_qk = ptx::idesc_f16(ab, 128, kRKeys, 0);
     constexpr uint32_t id_pv = ptx::idesc_f16(ab, 128, kDim, 1);
     // Descriptor bases; an operand at byte offset x from a base is the base
     // plus x >> 4 in the start-address field (addresses stay below 256 KiB).
-    const uint64_t qh0 = ptx::sdesc_sw128(sbase + kROffQHi, 16, 1024);
-    const uint64_t ql0 = ptx::sdesc_sw128(sbase + kROffQLo, 16, 1024);
+    const uint64_t qd0 = ptx::sdesc_sw128(sbase + kROffQ, 16, 1024);
     const uint64_t kd0 = ptx::sdesc_sw128(sbase + kROffK, 16, 1024);
     const uint64_t vd0 = ptx::sdesc_sw128(sbase + kROffV, kRBox, 1024);
     // P V of stage u: after its P is written; V rows past the split's end
@@ -288,14 +301,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
         for (int k = 0; k < 16; ++k) {   // 16 dims per step: chunk k / 4, 32-byte column group k % 4
           const uint32_t qo = (k >> 2) * kRQChunk + (k & 3) * 32, ko = (k >> 2) * kRBox + (k & 3) * 32;
-          ptx::mma_ss(scol, qh0 + (uint64_t)(qo >> 4), kd + (uint64_t)(ko >> 4), id_qk, k > 0 ? 1u : 0u);
-        }
-        if (kLo) {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const uint32_t qo = (k >> 2) * kRQChunk + (k & 3) * 32, ko = (k >> 2) * kRBox + (k & 3) * 32;
-            ptx::mma_ss(scol, ql0 + (uint64_t)(qo >> 4), kd + (uint64_t)(ko >> 4), id_qk, 1u);
-          }
+          ptx::mma_ss(scol, qd0 + (uint64_t)(qo >> 4), kd + (uint64_t)(ko >> 4), id_qk, k > 0 ? 1u : 0u);
         }
         ptx::mma_commit(smem_u32(&bars->kempty[s]));
         ptx::mma_commit(smem_u32(&bars->s_full[j & 1]));
@@ -308,8 +314,36 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (lane == 0) ptx::mma_commit(smem_u32(&bars->drain));
     __syncwarp();
     mbar_wait(&bars->drain, 0, nullptr, status, kSiteTcDrain);
-  } else {
+  } else if ((warp & 3) == 1 && kLo) {
+    // ------------------------------------------------- low-part scores
+    // Warp 4 qw + 1: lanes 32-63 (the low parts) of the columns of softmax
+    // warp 4 qw, into shared memory (by stage parity), then the pair's named
+    // barrier -- taken on every stage, whatever happened, as its partner does.
+    const int qw = warp >> 2;
+    float* lo_buf = reinterpret_cast<float*>(smem + kROffLo);
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, status, kSiteTcS));
+      if (ok) {
+        ptx::fence_after_sync();
+        uint32_t r[16];
+        ptx::tmem_ld16(tmem + (32u << 16) + kRColS + 64 * (j & 1) + 16 * qw, r);
+        ptx::tmem_wait_ld();
+        float* dst = lo_buf + ((j & 1) * 4 + qw) * 16 * 32 + lane;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) dst[32 * c] = __uint_as_float(r[c]);
+      }
+      ptx::fence_before_sync();
+      named_sync(2 + qw, 64);
+    }
+  } else if ((warp & 3) == 0) {
     // ------------------------------------------------------------- softmax
+    // Warps 0, 4, 8, 12 reach TMEM lanes 0-31: warp 4 qw takes key columns
+    // [16 qw, +16) of every stage and O columns [64 qw, +64).  A stage's row
+    // max is exchanged through shared memory: one named barrier per stage,
+    // which every softmax warp takes on every stage (work is skipped after
+    // an abort, so no warp waits there for one that left).
+    const int qw = warp >> 2;
     const int m = lane;                              // TMEM lane == M row
     const int i = m >> 3, h = m & 7;
     const bool valid = i < nr;
@@ -317,117 +351,136 @@ __global__ void __launch_bounds__(kRThreads, 1)
     const int64_t lo = lo_of(pos, a.window);
     const float cs = a.scale * 1.4426950408889634f;  // scores in log2 units
     float m_ref = -INFINITY;                         // reference max of the row, log2 units
-    float l_sum = 0.f;
+    float l_part = 0.f;                              // this warp's columns of the row sum
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, status, kSiteTcS));
-      if (!ok) break;
-      ptx::fence_after_sync();
-      uint32_t r0[32], r1[32];
-      ptx::tmem_ld32(tmem + kRColS + 64 * (j & 1), r0);
-      ptx::tmem_ld32(tmem + kRColS + 64 * (j & 1) + 32, r1);
-      ptx::tmem_wait_ld();
-      float s[64];
+      float s[16];
+      float mloc = -INFINITY;
+      if (ok) {
+        ptx::fence_after_sync();
+        uint32_t r[16];
+        ptx::tmem_ld16(tmem + kRColS + 64 * (j & 1) + 16 * qw, r);
+        ptx::tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        s[c] = __uint_as_float(r0[c]);
-        s[32 + c] = __uint_as_float(r1[c]);
+        for (int c = 0; c < 16; ++c) s[c] = __uint_as_float(r[c]);
       }
-      // keys outside [lo, pos], past the split's end, or of a row the unit
-      // does not have become -inf (scale > 0 keeps them there)
-      const int64_t k0 = kbeg + (int64_t)j * kRKeys;
-      const int cnt = (int)((kend - k0) < kRKeys ? (kend - k0) : kRKeys);
-      if (!(valid && cnt == kRKeys && k0 >= lo && k0 + kRKeys - 1 <= pos)) {
+      if (kLo) {
+        // the low-part scores of the same columns, from warp 4 qw + 1
+        named_sync(2 + qw, 64);
+        const float* src = reinterpret_cast<const float*>(smem + kROffLo) + ((j & 1) * 4 + qw) * 16 * 32 + lane;
+        if (ok) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int64_t key = k0 + c;
-          if (!valid || c >= cnt || key < lo || key > pos) s[c] = -INFINITY;
+          for (int c = 0; c < 16; ++c) s[c] += src[32 * c];
         }
       }
-      float m8[8];
+      if (ok) {
+        // keys outside [lo, pos], past the split's end, or of a row the unit
+        // does not have become -inf (scale > 0 keeps them there)
+        const int64_t k0 = kbeg + (int64_t)j * kRKeys + 16 * qw;
+        const int64_t left = kend - k0;               // keys of the split from this warp's first on
+        if (!(valid && left >= 16 && k0 >= lo && k0 + 15 <= pos)) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) m8[c] = s[c];
-#pragma unroll
-      for (int c = 8; c < 64; ++c) m8[c & 7] = max_nan(m8[c & 7], s[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) m8[c] = max_nan(m8[c], m8[c + 4]);
-      const float mloc = max_nan(max_nan(m8[0], m8[2]), max_nan(m8[1], m8[3]));
-      const float mx = mloc == -INFINITY ? -INFINITY : mloc * cs;
-      const bool need = mx > m_ref + kRRescaleLog2;
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ptx::ex2(m_ref - mx) : 1.f;
-        if (need) m_ref = mx;
-        l_sum *= alpha;
-        if (j > 0) {
-          // P V of stage j - 1 must finish before O is rescaled (that of
-          // stage j - 2 preceded this stage's Q K^T, so it has)
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
-                                                 status, kSiteTcO));
-          if (!ok) break;
-          ptx::fence_after_sync();
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tmem + kRColO + 32 * c, r);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            ptx::tmem_st32(tmem + kRColO + 32 * c, r);
+          for (int c = 0; c < 16; ++c) {
+            const int64_t key = k0 + c;
+            if (!valid || c >= left || key < lo || key > pos) s[c] = -INFINITY;
           }
-          ptx::tmem_wait_st();
+        }
+        float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+        for (int c = 4; c < 16; ++c) m4[c & 3] = max_nan(m4[c & 3], s[c]);
+        mloc = max_nan(max_nan(m4[0], m4[1]), max_nan(m4[2], m4[3]));
+      }
+      bars->red[j & 1][qw][lane] = mloc;
+      named_sync(1, kRSoftmaxThreads);
+      if (ok) {
+        const float* rm = bars->red[j & 1][0];
+        const float mraw = max_nan(max_nan(rm[lane], rm[32 + lane]), max_nan(rm[64 + lane], rm[96 + lane]));
+        const float mx = mraw == -INFINITY ? -INFINITY : mraw * cs;
+        const bool need = mx > m_ref + kRRescaleLog2;   // the same in all four warps
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ptx::ex2(m_ref - mx) : 1.f;
+          if (need) m_ref = mx;
+          l_part *= alpha;
+          if (j > 0) {
+            // P V of stage j - 1 must finish before O is rescaled (that of
+            // stage j - 2 preceded this stage's Q K^T, so it has)
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
+                                                   status, kSiteTcO));
+            if (ok) {
+              ptx::fence_after_sync();
+#pragma unroll 1
+              for (int c = 0; c < 2; ++c) {
+                uint32_t r[32];
+                ptx::tmem_ld32(tmem + kRColO + 64 * qw + 32 * c, r);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                ptx::tmem_st32(tmem + kRColO + 64 * qw + 32 * c, r);
+              }
+              ptx::tmem_wait_st();
+            }
+          }
         }
       }
-      // p = 2^(s cs - m_ref), split into 16-bit high and low parts
-      const float nmu = m_ref == -INFINITY ? 0.f : -m_ref;
-      uint32_t ph[32], pl[32];
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (ok) {
+        // p = 2^(s cs - m_ref), split into 16-bit high and low parts
+        const float nmu = m_ref == -INFINITY ? 0.f : -m_ref;
+        uint32_t ph[8], pl[8];
+        float acc[2] = {0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ptx::ex2(fmaf(s[2 * c], cs, nmu));
-        const float p1 = ptx::ex2(fmaf(s[2 * c + 1], cs, nmu));
-        acc[c & 3] += p0 + p1;
-        ph[c] = pk2<KT>(p0, p1);
-        const float2 f = upk2<KT>(ph[c]);
-        pl[c] = pk2<KT>(p0 - f.x, p1 - f.y);
+        for (int c = 0; c < 8; ++c) {
+          const float p0 = ptx::ex2(fmaf(s[2 * c], cs, nmu));
+          const float p1 = ptx::ex2(fmaf(s[2 * c + 1], cs, nmu));
+          acc[c & 1] += p0 + p1;
+          ph[c] = pk2<KT>(p0, p1);
+          const float2 f = upk2<KT>(ph[c]);
+          pl[c] = pk2<KT>(p0 - f.x, p1 - f.y);
+        }
+        l_part += acc[0] + acc[1];
+        // P buffer j & 1 was last read by P V of stage j - 2, complete before
+        // this stage's Q K^T (whose completion s_full signalled).
+        ptx::tmem_st8(tmem + kRColP + 64 * (j & 1) + 8 * qw, ph);
+        ptx::tmem_st8(tmem + kRColP + 64 * (j & 1) + 32 + 8 * qw, pl);
+        ptx::tmem_wait_st();
+        ptx::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[j & 1]);
       }
-      l_sum += (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      // P buffer j & 1 was last read by P V of stage j - 2, complete before
-      // this stage's Q K^T (whose completion s_full signalled).
-      ptx::tmem_st32(tmem + kRColP + 64 * (j & 1), ph);
-      ptx::tmem_st32(tmem + kRColP + 64 * (j & 1) + 32, pl);
-      ptx::tmem_wait_st();
-      ptx::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[j & 1]);
     }
     if (ok)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, status,
                                              kSiteTcO));
+    bars->red_l[qw][lane] = l_part;
+    named_sync(1, kRSoftmaxThreads);
+    // An aborted split poisons its rows; the status word says why.  The flag
+    // is raised before the failing warp reaches the barrier above.
     const bool aborted = !ok || *abort_flag;
-    // Epilogue: row m's 256 dims, scaled by 1 / l (one split) or raw with
-    // (m, l) in natural units (a split partial for multirow_merge_kernel).
-    // An aborted split poisons its rows; the status word says why.
+    const float L = aborted ? NAN : (bars->red_l[0][lane] + bars->red_l[1][lane]) +
+                                        (bars->red_l[2][lane] + bars->red_l[3][lane]);
+    // Epilogue: the warp's 64 dims of row m, scaled by 1 / l (one split) or
+    // raw with (m, l) in natural units (a split partial for
+    // multirow_merge_kernel).
     const float M = aborted ? NAN : m_ref * 0.6931471805599453f;
-    const float L = aborted ? NAN : l_sum;
     const int64_t orow = (int64_t)b * a.rows_per_seq + i0 + i;
     float* dst = nullptr;
     float f = 1.f;
     if (valid) {
       if (nsplit == 1) {
-        dst = a.out + (orow * kHeads + h) * kDim;
+        dst = a.out + (orow * kHeads + h) * kDim + 64 * qw;
         f = (m_ref == -INFINITY && L == 0.f) ? 0.f : 1.f / L;
       } else {
         const int64_t slot = (orow * a.max_splits + split) * kHeads + h;
-        dst = a.part_acc + slot * kDim;
-        *reinterpret_cast<float2*>(a.part_ml + slot * 2) = make_float2(M, L);
+        dst = a.part_acc + slot * kDim + 64 * qw;
+        if (qw == 0) *reinterpret_cast<float2*>(a.part_ml + slot * 2) = make_float2(M, L);
       }
     }
     if (!aborted) ptx::fence_after_sync();
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 2; ++c) {
       uint32_t r[32];
       if (!aborted) {
-        ptx::tmem_ld32(tmem + kRColO + 32 * c, r);
+        ptx::tmem_ld32(tmem + kRColO + 64 * qw + 32 * c, r);
         ptx::tmem_wait_ld();
       }
       if (valid) {
@@ -444,7 +497,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   // No warp leaves while MMAs may still read shared memory or write TMEM.
   ptx::fence_before_sync();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 2) {
     ptx::fence_after_sync();
     ptx::tmem_dealloc(tmem, kRTmemCols);
   }
