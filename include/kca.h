@@ -45,8 +45,13 @@
  * not see p -- every output row of a 16-row tile whose work items cover p's
  * 128-key tile (attn_prefill_plan lists them) becomes NaN, where the
  * definition above leaves the rows that do not see p unaffected.  Rows that
- * see a non-finite V value are non-finite on every path.  The rows path
- * (decode, short or mixed-dtype chunks) reads only the keys each row sees.
+ * see a non-finite V value are non-finite on every path.  The same holds
+ * for attn_prefill_batch on a 16-bit cache with 2 or more rows per sequence
+ * (multi-row units of up to 4 rows share each key): V must be finite on
+ * the union of a unit's visible ranges, else the unit's rows that do not
+ * see the position may be NaN too.  The rows path (decode, short or
+ * mixed-dtype chunks, one row per sequence) reads only the keys each row
+ * sees.
  *
  * DTYPES: decode takes any q_dtype with any kv_dtype.  Prefill with
  * q_dtype == kv_dtype in {F16, BF16} and chunk_rows >= 16 runs on the
