@@ -68,8 +68,7 @@ TRAFFIC = {
     "window_decode": (595456.0, "decode_mma_kernel<bf16, bf16>, one call, window 512 (cold caches)"),
     "long_chunk": (138080256.0 + 4125184.0, "prefill_tc_kernel, the 768-row chunk at 130304"),
     "decode_q8_ragged": (350935296.0 + 3392512.0, "decode_mma_kernel<f32, int8 K, f16 V>, one call of the 8 sequences"),
-    "prefill_batch": (301517824.0 + 480256.0, "rows_tc_kernel, one call of 32 sequences x 4 rows "
-                                               "(its merge kernel reads 4.8 MB more)"),
+    "prefill_batch": None,
 }
 E2E_GROUP = 4            # prefill chunks per host copy in the end-to-end leg
 METRIC = "prefill q-rows/s & decode tok/s at 16K ctx (1 B200); % of TC/HBM roofline"
@@ -502,7 +501,7 @@ class BatchRowsPart(Part):
     16 calls (each advancing every sequence by 4 rows), f16 K/V, f32 q,
     through attn_prefill_batch."""
     name, unit, bound = "prefill_batch", "q-rows", "hbm"
-    kernel = "rows_tc_kernel<f32 q, f16 KV> (tcgen05, + multirow_merge_kernel): 4 rows per unit"
+    kernel = "rows_tc_kernel<f32 q, f16 KV> (tcgen05, splits merged in-kernel): 4 rows per unit"
     BATCH, ROWS, CALLS, CAP = 32, 4, 16, 16448
 
     def __init__(self, device, seed=0):

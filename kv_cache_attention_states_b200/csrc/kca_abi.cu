@@ -873,7 +873,11 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
     for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
     a.cache_rows = (int64_t)batch * capacity;
     a.part_slots = mp.max_splits > 1 ? (int64_t)batch * rows * mp.max_splits : 0;
-    if (mp.max_splits > 1) carve(workspace, (size_t)batch * rows * mp.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
+    if (mp.max_splits > 1) {
+      carve(workspace, (size_t)batch * rows * mp.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
+      // self-resetting per-unit merge tickets of the tcgen05 kernel
+      a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+    }
     CUtensorMap tmk, tmv;
     if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, (int64_t)batch * capacity, 64) ||
         !encode_kv_map(&tmv, v_cache, kv_dtype, 0, (int64_t)batch * capacity, 64))

@@ -174,10 +174,12 @@ cudaError_t launch_decode_mma_q8(int q_dtype, int v_dtype, const CUtensorMap& tm
 // to kMultiRows consecutive rows of one sequence (n_units = batch x
 // ceil(rows / kMultiRows)), the union of their keys cut into splits of
 // split_len; per-row split partials in part_ml / part_acc
-// ([batch * rows][max_splits][8]) merged by a second kernel
-// (launch_multirow_merge).  launch_decode_multirow: mma.sync fragments
-// (kca_decode_mma.cu); launch_rows_tc: tcgen05 MMAs with TMEM accumulators
-// (kca_rows_tc.cu).  tmk / tmv as for launch_decode_mma.
+// ([batch * rows][max_splits][8]).  launch_decode_multirow: mma.sync
+// fragments (kca_decode_mma.cu), the partials merged by a second kernel
+// (launch_multirow_merge); launch_rows_tc: tcgen05 MMAs with TMEM
+// accumulators (kca_rows_tc.cu), the partials merged in-kernel by the last
+// split of each unit (per-unit tickets in a.tickets).  tmk / tmv as for
+// launch_decode_mma.
 cudaError_t launch_decode_multirow(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                    const RowsArgs& a, cudaStream_t stream);
 cudaError_t launch_rows_tc(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,

@@ -80,6 +80,9 @@ static_assert(kRSmemBytes <= 232448, "shared memory over the per-CTA limit");
 static_assert(kROffQ + 3 * kRQChunk + 16 * 1024 <= kROffV, "Q descriptors stay inside shared memory");
 constexpr uint32_t kRColS = 0, kRColP = 128, kRColO = 256, kRTmemCols = 512;
 constexpr float kRRescaleLog2 = 8.f;   // rescale O once a score passes the reference by 2^8
+// Merge tickets: one per unit, after the workspace's 256-byte status word.
+constexpr int kRTickets = (KCA_WORKSPACE_HEADER - 256) / 4;
+static_assert(KCA_MAX_BATCH * ((KCA_MAX_BATCH_ROWS + kMultiRows - 1) / kMultiRows) <= kRTickets, "tickets");
 
 struct RBars {
   uint64_t kfull[kRKRing], kempty[kRKRing];
@@ -90,6 +93,7 @@ struct RBars {
   uint64_t drain;       // every MMA complete (single use)
   uint32_t tmem_base;
   int abort;
+  int last;             // this CTA drew the unit's last ticket: it merges the splits
   float red[2][4][32];  // [stage parity][softmax warp][row]: partial row maxima
   float red_l[4][32];   // [softmax warp][row]: partial row sums at the end
 };
@@ -150,7 +154,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
   // bounds-checked builds: the split's rows in the cache, its rows' partial
   // slots in the workspace (no CTA of this kernel waits on another)
   if (!KCA_IN_BOUNDS(nsplit <= a.max_splits && base_row + kbeg >= 0 && base_row + kend <= a.cache_rows &&
-                         (nsplit == 1 || ((int64_t)b * a.rows_per_seq + i0 + nr) * a.max_splits <= a.part_slots),
+                         (nsplit == 1 || (((int64_t)b * a.rows_per_seq + i0 + nr) * a.max_splits <= a.part_slots &&
+                                          unit < kRTickets)),
                      status, kSiteBoundsMulti, (unsigned)unit))
     return;
 
@@ -493,7 +498,6 @@ __global__ void __launch_bounds__(kRThreads, 1)
       }
     }
   }
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // No warp leaves while MMAs may still read shared memory or write TMEM.
   ptx::fence_before_sync();
   __syncthreads();
@@ -501,6 +505,52 @@ __global__ void __launch_bounds__(kRThreads, 1)
     ptx::fence_after_sync();
     ptx::tmem_dealloc(tmem, kRTmemCols);
   }
+  if (nsplit > 1) {
+    // The unit's splits meet by ticket: the CTA that draws the last one
+    // merges every split's partials of the unit's rows (log-sum-exp, as in
+    // multirow_merge_kernel), so no second kernel and no CTA waits on
+    // another.  Release: the block's partial stores, ordered by the barrier
+    // above before one thread's acq_rel atomic; acquire: the same atomic in
+    // the last CTA, then the barrier below.
+    if (threadIdx.x == 0) {
+      int prev;
+      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(prev) : "l"(a.tickets + unit) : "memory");
+      bars->last = prev == nsplit - 1;
+    }
+    __syncthreads();
+    if (bars->last) {
+      // warp w: (row, head) pairs p = 8 i + h, w and w + 16; lane l: dims 8 l .. 8 l + 7
+      for (int p = warp; p < 8 * nr; p += kRThreads / 32) {
+        const int i = p >> 3, h = p & 7;
+        const int64_t orow = (int64_t)b * a.rows_per_seq + i0 + i;
+        const int64_t row0 = orow * a.max_splits * kHeads + h;   // split sp: partial row row0 + sp * 8
+        float M = -INFINITY;
+        for (int sp = lane; sp < nsplit; sp += 32)
+          M = max_nan(M, __ldcg(a.part_ml + (row0 + (int64_t)sp * kHeads) * 2));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = max_nan(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float mu = M == -INFINITY ? 0.f : M;
+        float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int sp = 0; sp < nsplit; ++sp) {
+          const int64_t r = row0 + (int64_t)sp * kHeads;
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + r * 2));
+          const float4* src = reinterpret_cast<const float4*>(a.part_acc + r * kDim + 8 * lane);
+          const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
+          const float f = exp2f((ml.x - mu) * 1.4426950408889634f);
+          L += f * ml.y;
+          acc[0] += f * v0.x; acc[1] += f * v0.y; acc[2] += f * v0.z; acc[3] += f * v0.w;
+          acc[4] += f * v1.x; acc[5] += f * v1.y; acc[6] += f * v1.z; acc[7] += f * v1.w;
+        }
+        const float inv = (M == -INFINITY && L == 0.f) ? 0.f : 1.f / L;
+        float4* dst = reinterpret_cast<float4*>(a.out + (orow * kHeads + h) * kDim + 8 * lane);
+        dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+      }
+      if (threadIdx.x == 0) a.tickets[unit] = 0;   // ready for the next call
+    }
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 template <int QT, int KT>
@@ -524,9 +574,7 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsA
   cfg.stream = stream;
   cfg.attrs = &at;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a);
-  if (e != cudaSuccess || a.max_splits <= 1) return e;
-  return launch_multirow_merge(a, stream);
+  return cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a);
 }
 
 }  // namespace
