@@ -10,36 +10,40 @@
 // K / V stage crosses from L2 once for all of them.  The mma.sync form of
 // this kernel is bound by instruction issue (two warps per SM sub-partition
 // run the QK^T and PV fragments, the softmax and the shared-memory traffic
-// of every stage); here one thread issues every MMA and four warps run the
-// softmax, so the tensor pipe and the load stream overlap.  A clock trace of
-// one split showed the MMA issue of Q K^T as the longest step of a stage,
-// which is why its high and low parts share one instruction (as M rows).
+// of every stage); here one thread issues every MMA and eight warps on two
+// SM sub-partitions run the softmax, so the tensor pipe, the softmax and
+// the load stream overlap.  Clock traces of one split chose the layout: the
+// high and low parts of Q and of P share their MMA instructions as M rows
+// (the MMA issue was the longest step), and the rows sit in two TMEM lane
+// quarters with full warps (the softmax chain was the next).
 //
-// Rows: M row m = 8 i + h (i the unit's row, h the head) holds the high
-// part of the query, M row 32 + m its low part (f32 queries keep f32-grade
-// products: q = q_hi + q_lo in 16-bit parts of the cache's type), so one
-// Q K^T MMA of M = 128 gives both partial scores, in TMEM lanes m and 32 + m;
-// rows 64-127 of the operands and accumulators are never read.  In O += P V
-// the probabilities are split the same way, p = p_hi + p_lo, and both parts
-// accumulate into the same O columns (two passes over the keys).
+// Rows.  A warp reaches only the TMEM lane quarter of its SM sub-partition
+// (warp w: lanes 32 (w % 4) .. +31).  Query rows i = 0, 1 of a unit live in
+// quarter 0 and rows 2, 3 in quarter 1: lane 8 (i % 2) + h of the quarter
+// holds the high 16-bit part of head h's query, lane 16 + 8 (i % 2) + h its
+// low part (f32 queries keep f32-grade products: q = q_hi + q_lo in the
+// cache's 16-bit type), so one Q K^T MMA of M = 128 gives both partial
+// scores of every head of every row, in lanes l and l ^ 16 of one warp,
+// which add them with a shuffle; M rows 64-127 are never read.  In O += P V
+// the probabilities are stacked the same way (p = p_hi + p_lo in the same
+// two lanes) and the two O rows are added at the end.
 //
 // Warp roles (16 warps, all of which stage the queries):
-//   warps 0, 4, 8, 12   softmax of TMEM lanes 0-31 (the unit's rows), 16 of
-//                       every stage's 64 key columns each, then the epilogue
-//   warps 1, 5, 9, 13   (f32 or mixed queries) read the low-part scores of
-//                       the same columns from lanes 32-63 and hand them over
-//                       through shared memory (only warps 4 k + 1 reach
-//                       those lanes, only warps 4 k reach lanes 0-31)
+//   warps 0, 4, 8, 12 (quarter 0) and 1, 5, 9, 13 (quarter 1)   softmax:
+//            warp 4 g + q takes key columns [16 g, +16) of every stage for
+//            the rows of quarter q (the high lane of a head columns 16 g ..
+//            + 7, the low lane 16 g + 8 .. + 15) and O columns [64 g, +64),
+//            then the epilogue; a stage's row max is exchanged between the
+//            quarter's four warps through shared memory
 //   warp 2   TMEM allocator; lane 0 issues every MMA; the warp zeroes the V
 //            rows of a ragged last stage
 //   warps 3, 7   TMA producers of K stages (64 keys x 256 dims, ring of 3)
 //                and of V stages (ring of 2)
 // Shared memory: Q (64 M rows x 256 dims, four 64-dim chunks of 8 KiB with
 // 128-byte swizzle; the descriptors of the last chunk reach on into the
-// bytes after it, which land only in unused M rows), the K and V rings, the
-// low-part scores in flight.  Tensor memory (512 columns): S of stage j at
-// [64 (j & 1), +64), P of stage j at [128 + 64 (j & 1), +64) (high parts,
-// then low parts, as 16-bit pairs), O at [256, 512).
+// bytes after it, which land only in unused M rows), the K and V rings.
+// Tensor memory (512 columns): S of stage j at [64 (j & 1), +64), P of stage
+// j at [128 + 32 (j & 1), +32) (16-bit pairs), O at [256, 512).
 // Per stage j the MMA thread issues Q K^T of stage j, then P V of stage
 // j - 1 once the softmax has written its P, so the softmax of a stage runs
 // under the MMAs of its neighbours.  The softmax keeps a reference max per
@@ -58,7 +62,7 @@ namespace kca {
 namespace {
 
 constexpr int kRThreads = 512;
-constexpr int kRSoftmaxThreads = 128;                // warps 0, 4, 8, 12
+constexpr int kRQuarterThreads = 128;                // the softmax warps of one TMEM lane quarter
 constexpr int kRKeys = 64;                           // keys per stage
 constexpr int kRBox = 64 * 64 * 2;                   // 64 rows x 64 dims (16-bit): 8 KiB
 constexpr int kRSlot = 4 * kRBox;                    // K or V of one stage: 32 KiB
@@ -68,10 +72,8 @@ constexpr int kRQChunk = 2 * kRQRows * 128;          // 64 M rows x 64 dims: 8 K
 constexpr int kROffQ = 0;
 constexpr int kROffK = 4 * kRQChunk;                 // 32 KiB
 constexpr int kROffV = kROffK + kRKRing * kRSlot;    // 128 KiB
-constexpr int kROffLo = kROffV + kRVRing * kRSlot;   // 192 KiB: float [2][4][16][32]
-constexpr int kRLoBytes = 2 * 4 * 16 * 32 * 4;
-constexpr int kROffBar = kROffLo + kRLoBytes;        // 208 KiB
-constexpr int kRBarBytes = 2048;
+constexpr int kROffBar = kROffV + kRVRing * kRSlot;  // 192 KiB
+constexpr int kRBarBytes = 4096;
 constexpr int kRSmemBytes = kROffBar + kRBarBytes + 1024;   // + alignment slack
 static_assert(kRSmemBytes <= 232448, "shared memory over the per-CTA limit");
 // A descriptor of 128 M rows starting at the last Q chunk reads 8 KiB past
@@ -88,14 +90,14 @@ struct RBars {
   uint64_t kfull[kRKRing], kempty[kRKRing];
   uint64_t vfull[kRVRing], vempty[kRVRing];
   uint64_t s_full[2];   // Q K^T of stage j complete in S buffer j & 1 (MMA commit)
-  uint64_t p_full[2];   // P of stage j written and O corrected (the four softmax warps)
+  uint64_t p_full[2];   // P of stage j written and O corrected (the eight softmax warps)
   uint64_t o_done[2];   // P V of stage j complete (MMA commit)
   uint64_t drain;       // every MMA complete (single use)
   uint32_t tmem_base;
   int abort;
   int last;             // this CTA drew the unit's last ticket: it merges the splits
-  float red[2][4][32];  // [stage parity][softmax warp][row]: partial row maxima
-  float red_l[4][32];   // [softmax warp][row]: partial row sums at the end
+  float red[2][2][4][32];  // [stage parity][quarter][column group][lane]: partial row maxima
+  float red_l[2][4][32];   // [quarter][column group][lane]: partial row sums at the end
 };
 static_assert(sizeof(RBars) <= kRBarBytes, "barrier block too large");
 
@@ -125,7 +127,6 @@ template <int QT, int KT>
 __global__ void __launch_bounds__(kRThreads, 1)
     rows_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const RowsArgs a) {
-  constexpr bool kLo = QT != KT;   // a query of the cache's own type has no low part
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], kRSoftmaxThreads / 32);
+      mbar_init(&bars->p_full[s], 2 * kRQuarterThreads / 32);
       mbar_init(&bars->o_done[s], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -191,28 +192,26 @@ __global__ void __launch_bounds__(kRThreads, 1)
   // kernel of the stream; global memory is touched only after this wait.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // Stage the queries: M row m = 8 i + h (high part) and 32 + m (low part),
-  // 16-byte group u of the 256 dims (chunk u / 8, 128-byte swizzle within it).
-  for (int it = threadIdx.x; it < kRQRows * 32; it += kRThreads) {
+  // Stage the queries: M row m = 32 q + 16 part + 8 (i % 2) + h for query
+  // row i = 2 q + ..., head h, part 0 (high) or 1 (low); absent rows zero.
+  // 16-byte group u of the 256 dims: chunk u / 8, 128-byte swizzle within it.
+  for (int it = threadIdx.x; it < 64 * 32; it += kRThreads) {
     const int m = it >> 5, u = it & 31;
-    const int i = m >> 3, h = m & 7;
+    const int part = (m >> 4) & 1, i = 2 * (m >> 5) + ((m >> 3) & 1), h = m & 7;
     float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (i < nr) {
       const int64_t orow = (int64_t)b * a.rows_per_seq + i0 + i;
       load8<QT>(static_cast<const char*>(a.q) + ((orow * kHeads + h) * kDim + 8 * u) * ElemBytes<QT>::value, x);
     }
-    uint32_t hi[4], lo[4];
+    uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      hi[j] = pk2<KT>(x[2 * j], x[2 * j + 1]);
-      const float2 f = upk2<KT>(hi[j]);
-      lo[j] = pk2<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
+      const uint32_t hi = pk2<KT>(x[2 * j], x[2 * j + 1]);
+      const float2 f = upk2<KT>(hi);
+      w[j] = part == 0 ? hi : pk2<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
     }
-    const int mh = m, ml = kRQRows + m;
-    *reinterpret_cast<uint4*>(smem + kROffQ + (u >> 3) * kRQChunk + mh * 128 + (((u & 7) ^ (mh & 7)) << 4)) =
-        make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(smem + kROffQ + (u >> 3) * kRQChunk + ml * 128 + (((u & 7) ^ (ml & 7)) << 4)) =
-        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4*>(smem + kROffQ + (u >> 3) * kRQChunk + m * 128 + (((u & 7) ^ (m & 7)) << 4)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
   }
   fence_proxy_async_smem();   // generic stores -> visible to the tensor core
   __syncthreads();
@@ -277,15 +276,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
       }
       ptx::fence_after_sync();
       if (lane == 0) {
-        const uint32_t pcol = tmem + kRColP + 64 * (u & 1);
+        // P's high and low parts in lanes l and l ^ 16 of the same columns:
+        // their O rows get p_hi V and p_lo V
+        const uint32_t pcol = tmem + kRColP + 32 * (u & 1);
         const uint64_t vd = vd0 + (uint64_t)((s * kRSlot) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)   // 16 keys per step: 8 TMEM columns of P, V rows 16 kk
           ptx::mma_ts(tmem + kRColO, pcol + 8 * kk, vd + (uint64_t)((kk * 16 * 128) >> 4), id_pv,
                       (u > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)   // the low parts of P
-          ptx::mma_ts(tmem + kRColO, pcol + 32 + 8 * kk, vd + (uint64_t)((kk * 16 * 128) >> 4), id_pv, 1u);
         ptx::mma_commit(smem_u32(&bars->vempty[s]));
         ptx::mma_commit(smem_u32(&bars->o_done[u & 1]));
       }
@@ -319,97 +317,74 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (lane == 0) ptx::mma_commit(smem_u32(&bars->drain));
     __syncwarp();
     mbar_wait(&bars->drain, 0, nullptr, status, kSiteTcDrain);
-  } else if ((warp & 3) == 1 && kLo) {
-    // ------------------------------------------------- low-part scores
-    // Warp 4 qw + 1: lanes 32-63 (the low parts) of the columns of softmax
-    // warp 4 qw, into shared memory (by stage parity), then the pair's named
-    // barrier -- taken on every stage, whatever happened, as its partner does.
-    const int qw = warp >> 2;
-    float* lo_buf = reinterpret_cast<float*>(smem + kROffLo);
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, status, kSiteTcS));
-      if (ok) {
-        ptx::fence_after_sync();
-        uint32_t r[16];
-        ptx::tmem_ld16(tmem + (32u << 16) + kRColS + 64 * (j & 1) + 16 * qw, r);
-        ptx::tmem_wait_ld();
-        float* dst = lo_buf + ((j & 1) * 4 + qw) * 16 * 32 + lane;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) dst[32 * c] = __uint_as_float(r[c]);
-      }
-      ptx::fence_before_sync();
-      named_sync(2 + qw, 64);
-    }
-  } else if ((warp & 3) == 0) {
+  } else if ((warp & 3) <= 1) {
     // ------------------------------------------------------------- softmax
-    // Warps 0, 4, 8, 12 reach TMEM lanes 0-31: warp 4 qw takes key columns
-    // [16 qw, +16) of every stage and O columns [64 qw, +64).  A stage's row
-    // max is exchanged through shared memory: one named barrier per stage,
-    // which every softmax warp takes on every stage (work is skipped after
-    // an abort, so no warp waits there for one that left).
-    const int qw = warp >> 2;
-    const int m = lane;                              // TMEM lane == M row
-    const int i = m >> 3, h = m & 7;
+    // Warp 4 g + q: quarter q (query rows 2 q, 2 q + 1), key columns
+    // [16 g, +16) of every stage, O columns [64 g, +64).  Lane l: query row
+    // 2 q + ((l >> 3) & 1), head l & 7, high part (l < 16) or low (l >= 16);
+    // lanes l and l ^ 16 pair up: the high lane takes columns 16 g .. + 7, the
+    // low lane 16 g + 8 .. + 15, each first fetching the other part of its
+    // columns' scores from its partner.  The quarter's four warps exchange
+    // their row maxima at a named barrier that each takes on every stage
+    // (work is skipped after an abort, so no warp waits there for one that
+    // left).
+    const int q = warp & 3, g = warp >> 2;
+    const bool low = lane >= 16;
+    const int i = 2 * q + ((lane >> 3) & 1), h = lane & 7;
     const bool valid = i < nr;
+    const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
     const int64_t pos = pos0 + i;
     const int64_t lo = lo_of(pos, a.window);
     const float cs = a.scale * 1.4426950408889634f;  // scores in log2 units
+    const int cofs = 16 * g + (low ? 8 : 0);         // this lane's 8 columns within a stage
     float m_ref = -INFINITY;                         // reference max of the row, log2 units
-    float l_part = 0.f;                              // this warp's columns of the row sum
+    float l_part = 0.f;                              // this lane's columns of the row sum
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, status, kSiteTcS));
-      float s[16];
+      float s[8];
       float mloc = -INFINITY;
       if (ok) {
         ptx::fence_after_sync();
         uint32_t r[16];
-        ptx::tmem_ld16(tmem + kRColS + 64 * (j & 1) + 16 * qw, r);
+        ptx::tmem_ld16(trow + kRColS + 64 * (j & 1) + 16 * g, r);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; ++c) s[c] = __uint_as_float(r[c]);
-      }
-      if (kLo) {
-        // the low-part scores of the same columns, from warp 4 qw + 1
-        named_sync(2 + qw, 64);
-        const float* src = reinterpret_cast<const float*>(smem + kROffLo) + ((j & 1) * 4 + qw) * 16 * 32 + lane;
-        if (ok) {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) s[c] += src[32 * c];
+        for (int c = 0; c < 8; ++c) {
+          const float mine = __uint_as_float(low ? r[8 + c] : r[c]);
+          const float give = __uint_as_float(low ? r[c] : r[8 + c]);
+          s[c] = mine + __shfl_xor_sync(0xffffffffu, give, 16);
         }
-      }
-      if (ok) {
         // keys outside [lo, pos], past the split's end, or of a row the unit
         // does not have become -inf (scale > 0 keeps them there)
-        const int64_t k0 = kbeg + (int64_t)j * kRKeys + 16 * qw;
-        const int64_t left = kend - k0;               // keys of the split from this warp's first on
-        if (!(valid && left >= 16 && k0 >= lo && k0 + 15 <= pos)) {
+        const int64_t k0 = kbeg + (int64_t)j * kRKeys + cofs;
+        const int64_t left = kend - k0;               // keys of the split from this lane's first on
+        if (!(valid && left >= 8 && k0 >= lo && k0 + 7 <= pos)) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < 8; ++c) {
             const int64_t key = k0 + c;
             if (!valid || c >= left || key < lo || key > pos) s[c] = -INFINITY;
           }
         }
-        float m4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-        for (int c = 4; c < 16; ++c) m4[c & 3] = max_nan(m4[c & 3], s[c]);
-        mloc = max_nan(max_nan(m4[0], m4[1]), max_nan(m4[2], m4[3]));
+        mloc = max_nan(max_nan(max_nan(s[0], s[1]), max_nan(s[2], s[3])),
+                       max_nan(max_nan(s[4], s[5]), max_nan(s[6], s[7])));
+        mloc = max_nan(mloc, __shfl_xor_sync(0xffffffffu, mloc, 16));   // the warp's 16 columns
       }
-      bars->red[j & 1][qw][lane] = mloc;
-      named_sync(1, kRSoftmaxThreads);
+      bars->red[j & 1][q][g][lane] = mloc;
+      named_sync(1 + q, kRQuarterThreads);
       if (ok) {
-        const float* rm = bars->red[j & 1][0];
+        const float* rm = bars->red[j & 1][q][0];
         const float mraw = max_nan(max_nan(rm[lane], rm[32 + lane]), max_nan(rm[64 + lane], rm[96 + lane]));
         const float mx = mraw == -INFINITY ? -INFINITY : mraw * cs;
-        const bool need = mx > m_ref + kRRescaleLog2;   // the same in all four warps
+        const bool need = mx > m_ref + kRRescaleLog2;   // the same in all the row's lanes
         if (__any_sync(0xffffffffu, need)) {
           const float alpha = need ? ptx::ex2(m_ref - mx) : 1.f;
           if (need) m_ref = mx;
           l_part *= alpha;
           if (j > 0) {
             // P V of stage j - 1 must finish before O is rescaled (that of
-            // stage j - 2 preceded this stage's Q K^T, so it has)
+            // stage j - 2 preceded this stage's Q K^T, so it has); each lane
+            // scales its own O row (high or low part)
             ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
                                                    status, kSiteTcO));
             if (ok) {
@@ -417,11 +392,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll 1
               for (int c = 0; c < 2; ++c) {
                 uint32_t r[32];
-                ptx::tmem_ld32(tmem + kRColO + 64 * qw + 32 * c, r);
+                ptx::tmem_ld32(trow + kRColO + 64 * g + 32 * c, r);
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                ptx::tmem_st32(tmem + kRColO + 64 * qw + 32 * c, r);
+                ptx::tmem_st32(trow + kRColO + 64 * g + 32 * c, r);
               }
               ptx::tmem_wait_st();
             }
@@ -429,24 +404,30 @@ __global__ void __launch_bounds__(kRThreads, 1)
         }
       }
       if (ok) {
-        // p = 2^(s cs - m_ref), split into 16-bit high and low parts
+        // p = 2^(s cs - m_ref) for this lane's columns, split into 16-bit
+        // high and low parts; the high lane keeps the high parts of the
+        // warp's 16 columns, the low lane the low parts (each gives the
+        // partner the other half)
         const float nmu = m_ref == -INFINITY ? 0.f : -m_ref;
-        uint32_t ph[8], pl[8];
-        float acc[2] = {0.f, 0.f};
+        uint32_t pr[8];
+        float acc = 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           const float p0 = ptx::ex2(fmaf(s[2 * c], cs, nmu));
           const float p1 = ptx::ex2(fmaf(s[2 * c + 1], cs, nmu));
-          acc[c & 1] += p0 + p1;
-          ph[c] = pk2<KT>(p0, p1);
-          const float2 f = upk2<KT>(ph[c]);
-          pl[c] = pk2<KT>(p0 - f.x, p1 - f.y);
+          acc += p0 + p1;
+          const uint32_t ph = pk2<KT>(p0, p1);
+          const float2 f = upk2<KT>(ph);
+          const uint32_t pl = pk2<KT>(p0 - f.x, p1 - f.y);
+          const uint32_t got = __shfl_xor_sync(0xffffffffu, low ? ph : pl, 16);
+          // P row, the warp's 16 columns: 16 g .. + 7 (pairs 0-3), 16 g + 8 .. (pairs 4-7)
+          pr[c] = low ? got : ph;
+          pr[4 + c] = low ? pl : got;
         }
-        l_part += acc[0] + acc[1];
+        l_part += acc;
         // P buffer j & 1 was last read by P V of stage j - 2, complete before
         // this stage's Q K^T (whose completion s_full signalled).
-        ptx::tmem_st8(tmem + kRColP + 64 * (j & 1) + 8 * qw, ph);
-        ptx::tmem_st8(tmem + kRColP + 64 * (j & 1) + 32 + 8 * qw, pl);
+        ptx::tmem_st8(trow + kRColP + 32 * (j & 1) + 8 * g, pr);
         ptx::tmem_wait_st();
         ptx::fence_before_sync();
         __syncwarp();
@@ -456,46 +437,55 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (ok)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, status,
                                              kSiteTcO));
-    bars->red_l[qw][lane] = l_part;
-    named_sync(1, kRSoftmaxThreads);
+    bars->red_l[q][g][lane] = l_part + __shfl_xor_sync(0xffffffffu, l_part, 16);
+    named_sync(1 + q, kRQuarterThreads);
     // An aborted split poisons its rows; the status word says why.  The flag
     // is raised before the failing warp reaches the barrier above.
     const bool aborted = !ok || *abort_flag;
-    const float L = aborted ? NAN : (bars->red_l[0][lane] + bars->red_l[1][lane]) +
-                                        (bars->red_l[2][lane] + bars->red_l[3][lane]);
-    // Epilogue: the warp's 64 dims of row m, scaled by 1 / l (one split) or
-    // raw with (m, l) in natural units (a split partial for
-    // multirow_merge_kernel).
-    const float M = aborted ? NAN : m_ref * 0.6931471805599453f;
+    const float* rl = bars->red_l[q][0];
+    const float L = aborted ? NAN : (rl[lane] + rl[32 + lane]) + (rl[64 + lane] + rl[96 + lane]);
+    const float M = aborted ? NAN : m_ref * 0.6931471805599453f;   // natural units for the merge
+    // Epilogue: O = (high row) + (low row) over the warp's 64 columns; the
+    // high lane writes dims 64 g .. + 31 of its head, the low lane 64 g + 32
+    // .. + 63, scaled by 1 / l (one split) or raw with (m, l) (a split
+    // partial, merged below).
     const int64_t orow = (int64_t)b * a.rows_per_seq + i0 + i;
     float* dst = nullptr;
     float f = 1.f;
     if (valid) {
       if (nsplit == 1) {
-        dst = a.out + (orow * kHeads + h) * kDim + 64 * qw;
+        dst = a.out + (orow * kHeads + h) * kDim + 64 * g + (low ? 32 : 0);
         f = (m_ref == -INFINITY && L == 0.f) ? 0.f : 1.f / L;
       } else {
         const int64_t slot = (orow * a.max_splits + split) * kHeads + h;
-        dst = a.part_acc + slot * kDim + 64 * qw;
-        if (qw == 0) *reinterpret_cast<float2*>(a.part_ml + slot * 2) = make_float2(M, L);
+        dst = a.part_acc + slot * kDim + 64 * g + (low ? 32 : 0);
+        if (!low && g == 0) *reinterpret_cast<float2*>(a.part_ml + slot * 2) = make_float2(M, L);
       }
     }
-    if (!aborted) ptx::fence_after_sync();
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      uint32_t r[32];
-      if (!aborted) {
-        ptx::tmem_ld32(tmem + kRColO + 64 * qw + 32 * c, r);
-        ptx::tmem_wait_ld();
-      }
-      if (valid) {
+    uint32_t ra[32], rb[32];
+    if (!aborted) {
+      ptx::fence_after_sync();
+      ptx::tmem_ld32(trow + kRColO + 64 * g, ra);
+      ptx::tmem_ld32(trow + kRColO + 64 * g + 32, rb);
+      ptx::tmem_wait_ld();
+    } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          *reinterpret_cast<float4*>(dst + 32 * c + 4 * e) =
-              aborted ? make_float4(NAN, NAN, NAN, NAN)
-                      : make_float4(__uint_as_float(r[4 * e]) * f, __uint_as_float(r[4 * e + 1]) * f,
-                                    __uint_as_float(r[4 * e + 2]) * f, __uint_as_float(r[4 * e + 3]) * f);
-      }
+      for (int e = 0; e < 32; ++e) ra[e] = rb[e] = 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      // the high lane adds the low row's dim 64 g + e, the low lane the high row's 64 g + 32 + e
+      const float give = __uint_as_float(low ? ra[e] : rb[e]);
+      const float got = __shfl_xor_sync(0xffffffffu, give, 16);
+      ra[e] = __float_as_uint((__uint_as_float(low ? rb[e] : ra[e]) + got) * f);
+    }
+    if (valid) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        *reinterpret_cast<float4*>(dst + 4 * e) =
+            aborted ? make_float4(NAN, NAN, NAN, NAN)
+                    : make_float4(__uint_as_float(ra[4 * e]), __uint_as_float(ra[4 * e + 1]),
+                                  __uint_as_float(ra[4 * e + 2]), __uint_as_float(ra[4 * e + 3]));
     }
   }
   // No warp leaves while MMAs may still read shared memory or write TMEM.
