@@ -166,3 +166,27 @@ def test_tcgen05_multirow_nan_score_reaches_exactly_the_rows_that_see_it():
     assert np.isfinite(out[0, :3]).all() and np.isfinite(out[1:]).all()
     want = _oracle(q[1:], k[1:], v[1:], ctx[1:], rows, 0, "f32", "f16")
     assert max_err(out[1:], want) <= 4e-3
+
+
+@pytest.mark.parametrize("path", BATCH_PATHS, ids=["tcgen05", "mma_sync"])
+def test_nan_in_a_value_row_reaches_the_whole_multirow_unit(path):
+    # include/kca.h, PRECONDITIONS: V must be finite on the union of a
+    # multi-row unit's visible ranges.  A NaN V row at position ctx - 4 of
+    # sequence 0 (6 rows: units of rows 0-3 and 4-5) is seen by rows 2-5;
+    # rows 0-1 share unit 0 with rows that see it, so the kernels' exact-zero
+    # probabilities meet the NaN there too: the whole of both units is NaN,
+    # every other sequence finite and equal to the oracle.  The f32 rows path
+    # (one unit per row) poisons exactly the rows that see the position.
+    batch, rows, cap = 3, 6, 3000
+    ctx, q, k, v = _inputs(66, batch, rows, cap, "f32", "f16")
+    ctx[0] = 2000
+    v[0, ctx[0] - 4, 100] = np.float16(np.nan)
+    with kca.forced_path(kca.OP_BATCH, path):
+        out = kca.attn_prefill_batch(dev(q, "f32"), dev(k, "f16"), dev(v, "f16"), ctx).cpu().numpy()
+    assert np.isnan(out[0]).any(axis=(1, 2)).all()
+    assert np.isfinite(out[1:]).all()
+    want = _oracle(q[1:], k[1:], v[1:], ctx[1:], rows, 0, "f32", "f16")
+    assert max_err(out[1:], want) <= 4e-3
+    out32 = kca.attn_prefill_batch(dev(q, "f32"), dev(k.astype(np.float32), "f32"), dev(v.astype(np.float32), "f32"),
+                                   ctx).cpu().numpy()
+    assert np.isfinite(out32[0, :2]).all() and np.isnan(out32[0, 2:]).any(axis=(1, 2)).all()
