@@ -77,9 +77,11 @@
  * WORKSPACE: scratch device memory of at least attn_*_workspace_bytes()
  * bytes for the same arguments on the same device.  Its first
  * KCA_WORKSPACE_HEADER bytes are the header: a device status word in bytes
- * [0, 256) (read it with attn_device_status) and, in the rest, one counter
- * per (row, head) that the tensor-core rows kernel uses to elect the CTA that
- * merges a row's partials; every call leaves them at zero again.  Zero the
+ * [0, 256) (read it with attn_device_status) and, in the rest, merge
+ * counters: one per (row, head) with which the tensor-core rows kernel
+ * elects the CTA that merges a row's partials, one per multi-row unit with
+ * which the tcgen05 kernel of attn_prefill_batch elects the split that
+ * merges a unit's; every call leaves them at zero again.  Zero the
  * header once after allocation (attn_workspace_init), and again after a call
  * that recorded a device error.  Calls that run concurrently must not share a
  * workspace or an output buffer.
