@@ -875,8 +875,12 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
     a.part_slots = mp.max_splits > 1 ? (int64_t)batch * rows * mp.max_splits : 0;
     if (mp.max_splits > 1) {
       carve(workspace, (size_t)batch * rows * mp.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
-      // self-resetting per-unit merge tickets of the tcgen05 kernel
-      a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+      // self-resetting per-unit merge tickets of the tcgen05 kernel, which
+      // then merges in-kernel; a unit with many splits is merged by a second
+      // kernel instead (one CTA would read all its partials: at 1 x 131,072
+      // keys, 147 splits, 141 us against 52 us with the merge kernel)
+      if (mp.max_splits <= kca::kRowsTcMergeSplits)
+        a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
     }
     CUtensorMap tmk, tmv;
     if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, (int64_t)batch * capacity, 64) ||

@@ -178,12 +178,15 @@ cudaError_t launch_decode_mma_q8(int q_dtype, int v_dtype, const CUtensorMap& tm
 // fragments (kca_decode_mma.cu), the partials merged by a second kernel
 // (launch_multirow_merge); launch_rows_tc: tcgen05 MMAs with TMEM
 // accumulators (kca_rows_tc.cu), the partials merged in-kernel by the last
-// split of each unit (per-unit tickets in a.tickets).  tmk / tmv as for
-// launch_decode_mma.
+// split of each unit (per-unit tickets in a.tickets) or, without tickets, by
+// the merge kernel.  tmk / tmv as for launch_decode_mma.
 cudaError_t launch_decode_multirow(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                    const RowsArgs& a, cudaStream_t stream);
 cudaError_t launch_rows_tc(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                            const RowsArgs& a, cudaStream_t stream);
+// Most splits per unit that the tcgen05 kernel merges in-kernel (a.tickets
+// set); with more, a.tickets is null and launch_rows_tc adds the merge kernel.
+constexpr int kRowsTcMergeSplits = 16;
 cudaError_t launch_multirow_merge(const RowsArgs& a, cudaStream_t stream);
 
 // Clusters of c CTAs of the tensor-core rows kernel that fit on the device at

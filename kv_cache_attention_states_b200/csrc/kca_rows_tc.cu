@@ -495,11 +495,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
     ptx::fence_after_sync();
     ptx::tmem_dealloc(tmem, kRTmemCols);
   }
-  if (nsplit > 1) {
+  if (nsplit > 1 && a.tickets != nullptr) {
     // The unit's splits meet by ticket: the CTA that draws the last one
     // merges every split's partials of the unit's rows (log-sum-exp, as in
     // multirow_merge_kernel), so no second kernel and no CTA waits on
-    // another.  Release: the block's partial stores, ordered by the barrier
+    // another.  The host gives tickets only while a unit has few splits;
+    // with many, multirow_merge_kernel merges across the whole GPU after
+    // this kernel instead of one CTA reading every partial.  Release: the block's partial stores, ordered by the barrier
     // above before one thread's acq_rel atomic; acquire: the same atomic in
     // the last CTA, then the barrier below.
     if (threadIdx.x == 0) {
@@ -564,7 +566,9 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsA
   cfg.stream = stream;
   cfg.attrs = &at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a);
+  if (e != cudaSuccess || a.max_splits <= 1 || a.tickets != nullptr) return e;
+  return launch_multirow_merge(a, stream);
 }
 
 }  // namespace
