@@ -47,7 +47,8 @@
  * definition above leaves the rows that do not see p unaffected.  Rows that
  * see a non-finite V value are non-finite on every path.  The same holds
  * for attn_prefill_batch on a 16-bit cache with 2 or more rows per sequence
- * (multi-row units of up to 4 rows share each key): V must be finite on
+ * (multi-row units of up to 4 rows, 8 when a call has more than 4 rows per
+ * sequence, share each key): V must be finite on
  * the union of a unit's visible ranges, else the unit's rows that do not
  * see the position are NaN too (in the dims where V is not finite).  The rows path (decode, short or
  * mixed-dtype chunks, one row per sequence) reads only the keys each row

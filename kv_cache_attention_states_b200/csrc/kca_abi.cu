@@ -94,14 +94,16 @@ std::vector<int64_t> batch_unit_keys(int32_t batch, int32_t rows, const int64_t*
 }
 
 // Multi-row units of the tensor-core batched path: unit b * blocks + k holds
-// rows 4k .. 4k+3 (at most) of sequence b; its keys are the union of theirs.
-std::vector<int64_t> multirow_unit_keys(int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window) {
-  const int32_t blocks = (rows + kca::kMultiRows - 1) / kca::kMultiRows;
+// rows ur k .. ur k + ur - 1 (at most) of sequence b; its keys are the union
+// of theirs.
+std::vector<int64_t> multirow_unit_keys(int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window,
+                                        int32_t ur) {
+  const int32_t blocks = (rows + ur - 1) / ur;
   std::vector<int64_t> nk((size_t)batch * blocks);
   for (int32_t b = 0; b < batch; ++b)
     for (int32_t k = 0; k < blocks; ++k) {
-      const int32_t i0 = k * kca::kMultiRows;
-      const int32_t nr = rows - i0 < kca::kMultiRows ? rows - i0 : kca::kMultiRows;
+      const int32_t i0 = k * ur;
+      const int32_t nr = rows - i0 < ur ? rows - i0 : ur;
       const int64_t pos0 = ctx_len[b] - rows + i0;
       nk[(size_t)b * blocks + k] = pos0 + nr - kca::lo_of(pos0, window);
     }
@@ -552,10 +554,12 @@ size_t attn_prefill_batch_workspace_bytes(int32_t batch, int32_t rows, const int
   if (current_sms(&sms) != KCA_OK) return 0;
   const std::vector<int64_t> nk = batch_unit_keys(batch, rows, ctx_len, window);
   size_t need = rows_ws_bytes_any(batch * rows, nk.data(), sms);
-  if (rows > 1) {   // the multi-row kernel's partials, whichever path a call takes
-    const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window);
-    const size_t mr = multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms));
-    if (mr > need) need = mr;
+  if (rows > 1) {   // the multi-row kernels' partials, whichever path and unit size a call takes
+    for (const int32_t ur : {kca::kMultiRows, kca::kMultiRowsWide}) {
+      const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, ur);
+      const size_t mr = multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms));
+      if (mr > need) need = mr;
+    }
   }
   return need;
 }
@@ -853,7 +857,10 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
   if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_multirow(kv_dtype, rows)) {
-    const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window);
+    // the tcgen05 kernel takes units of 8 rows when a sequence has more than 4
+    const bool tc = use_batch_tc();
+    const int32_t ur = tc && rows > kca::kMultiRows ? kca::kMultiRowsWide : kca::kMultiRows;
+    const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, ur);
     const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms);
     if (workspace_bytes < multirow_ws_bytes(batch, rows, mp)) return KCA_ERR_WORKSPACE;
     kca::RowsArgs a{};
@@ -865,6 +872,7 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
     a.seq_rows = capacity;
     a.mode = 2;
     a.rows_per_seq = rows;
+    a.unit_rows = ur;
     a.n_units = (int32_t)nku.size();
     a.split_len = mp.split_len;
     a.max_splits = mp.max_splits;
@@ -886,8 +894,8 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
     if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, (int64_t)batch * capacity, 64) ||
         !encode_kv_map(&tmv, v_cache, kv_dtype, 0, (int64_t)batch * capacity, 64))
       return KCA_ERR_CUDA;
-    const cudaError_t e = use_batch_tc() ? kca::launch_rows_tc(q_dtype, kv_dtype, tmk, tmv, a, s)
-                                         : kca::launch_decode_multirow(q_dtype, kv_dtype, tmk, tmv, a, s);
+    const cudaError_t e = tc ? kca::launch_rows_tc(q_dtype, kv_dtype, tmk, tmv, a, s)
+                             : kca::launch_decode_multirow(q_dtype, kv_dtype, tmk, tmv, a, s);
     return e == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
   }
   const int32_t n_units = batch * rows;

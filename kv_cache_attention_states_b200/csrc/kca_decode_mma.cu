@@ -1122,7 +1122,7 @@ __global__ void __launch_bounds__(256) multirow_merge_kernel(const RowsArgs a) {
   const int h = blockIdx.x & 7;
   const int b = (int)(orow / a.rows_per_seq);
   const int i = (int)(orow % a.rows_per_seq);
-  const int u = b * ((a.rows_per_seq + kMRows - 1) / kMRows) + i / kMRows;
+  const int u = b * ((a.rows_per_seq + a.unit_rows - 1) / a.unit_rows) + i / a.unit_rows;
   int bb, i0, nr;
   multirow_unit(a, u, &bb, &i0, &nr);
   const int64_t pos0 = a.ctx[bb] - a.rows_per_seq + i0;
@@ -1171,7 +1171,7 @@ cudaError_t launch_multirow_merge(const RowsArgs& a, cudaStream_t stream) {
   cudaLaunchAttribute at;
   at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at.val.programmaticStreamSerializationAllowed = 1;
-  const int blocks = (a.rows_per_seq + kMRows - 1) / kMRows;
+  const int blocks = (a.rows_per_seq + a.unit_rows - 1) / a.unit_rows;
   const int64_t rows_total = (int64_t)(a.n_units / blocks) * a.rows_per_seq;
   cudaLaunchConfig_t mcfg = {};
   mcfg.gridDim = dim3((unsigned)(rows_total * kHeads), 1, 1);

@@ -21,6 +21,7 @@ struct RowsArgs {
   int32_t mode;          // 0: decode (unit = sequence), 1: prefill (unit = row of sequence 0),
                          // 2: batched rows (unit = row i of sequence unit / rows_per_seq)
   int32_t rows_per_seq;  // mode 2: query rows per sequence, at ctx[b] - rows_per_seq .. ctx[b] - 1
+  int32_t unit_rows;     // multi-row units: rows per unit (kMultiRows, or kMultiRowsWide for tcgen05)
   int32_t n_units;
   int32_t split_len;
   int32_t max_splits;
@@ -56,8 +57,10 @@ struct RowsArgs {
   int64_t ctx[KCA_MAX_BATCH];  // decode: ctx_len per sequence
 };
 
-// Rows of one unit of the batched multi-row kernels.
+// Rows of one unit of the batched multi-row kernels: 4 (both kernels), or 8
+// (the tcgen05 kernel, when a call has more than 4 rows per sequence).
 constexpr int kMultiRows = 4;
+constexpr int kMultiRowsWide = 8;
 
 #if defined(__CUDACC__)
 }  // namespace kca
@@ -106,7 +109,7 @@ __device__ __forceinline__ float rows_final(const RowsArgs& a, float acc, float 
   if (a.out_ml != nullptr) return acc;
   return (M == -INFINITY && L == 0.f) ? 0.f : acc / L;
 }
-// Unit u of a batched call in multi-row units (kMultiRows rows each):
+// Unit u of a batched call in multi-row units (a.unit_rows rows each):
 // sequence *b, first row *i0 (of the sequence's rows), *nr rows; positions
 // ctx[b] - rows_per_seq + i0 + r.
 __device__ __forceinline__ void multirow_unit(const RowsArgs& a, int u, int* b, int* i0, int* nr);
@@ -120,11 +123,12 @@ __device__ __forceinline__ int32_t rows_split_len(const RowsArgs& a, int64_t nke
   return (int32_t)(s < 64 ? 64 : s);
 }
 __device__ __forceinline__ void multirow_unit(const RowsArgs& a, int u, int* b, int* i0, int* nr) {
-  const int blocks = (a.rows_per_seq + kMultiRows - 1) / kMultiRows;
+  const int ur = a.unit_rows;
+  const int blocks = (a.rows_per_seq + ur - 1) / ur;
   *b = u / blocks;
-  *i0 = (u % blocks) * kMultiRows;
+  *i0 = (u % blocks) * ur;
   const int left = a.rows_per_seq - *i0;
-  *nr = left < kMultiRows ? left : kMultiRows;
+  *nr = left < ur ? left : ur;
 }
 #endif
 
@@ -171,8 +175,9 @@ cudaError_t launch_decode_mma_q8(int q_dtype, int v_dtype, const CUtensorMap& tm
                                  const CUtensorMap& tmv, const RowsArgs& a, cudaStream_t stream);
 
 // Batched short chunks on the tensor cores (mode 2, 16-bit K/V): units of up
-// to kMultiRows consecutive rows of one sequence (n_units = batch x
-// ceil(rows / kMultiRows)), the union of their keys cut into splits of
+// to a.unit_rows consecutive rows of one sequence (n_units = batch x
+// ceil(rows / unit_rows); kMultiRows for the mma.sync kernel, kMultiRows or
+// kMultiRowsWide for tcgen05), the union of their keys cut into splits of
 // split_len; per-row split partials in part_ml / part_acc
 // ([batch * rows][max_splits][8]).  launch_decode_multirow: mma.sync
 // fragments (kca_decode_mma.cu), the partials merged by a second kernel

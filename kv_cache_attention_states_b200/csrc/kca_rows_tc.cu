@@ -5,43 +5,45 @@
 // The pages' geometry (Karume v0.12.0 release notes, "Performance", item 3,
 // and "Docs", ADR 0067): plans of 2-15 query rows sit between single-row
 // decode and the row tiles of prefill.  A unit is up to four consecutive
-// query rows of one sequence (the same units, splits, partials and merge
-// kernel as the mma.sync multi-row kernel in kca_decode_mma.cu), so each
-// K / V stage crosses from L2 once for all of them.  The mma.sync form of
-// this kernel is bound by instruction issue (two warps per SM sub-partition
-// run the QK^T and PV fragments, the softmax and the shared-memory traffic
-// of every stage); here one thread issues every MMA and eight warps on two
-// SM sub-partitions run the softmax, so the tensor pipe, the softmax and
-// the load stream overlap.  Clock traces of one split chose the layout: the
-// high and low parts of Q and of P share their MMA instructions as M rows
-// (the MMA issue was the longest step), and the rows sit in two TMEM lane
-// quarters with full warps (the softmax chain was the next).
+// query rows of one sequence (the units, splits and partials of the mma.sync
+// multi-row kernel in kca_decode_mma.cu), or up to eight when a call has
+// more than four rows per sequence, so each K / V stage crosses from L2 once
+// for all of them.  The mma.sync form of this kernel is bound by instruction
+// issue (two warps per SM sub-partition run the QK^T and PV fragments, the
+// softmax and the shared-memory traffic of every stage); here one thread
+// issues every MMA and four warps per TMEM lane quarter in use run the
+// softmax, so the tensor pipe, the softmax and the load stream overlap.
+// Clock traces of one split chose the layout: the high and low parts of Q
+// and of P share their MMA instructions as M rows (the MMA issue was the
+// longest step), and the rows sit in lane quarters with full warps (the
+// softmax chain was the next).
 //
 // Rows.  A warp reaches only the TMEM lane quarter of its SM sub-partition
-// (warp w: lanes 32 (w % 4) .. +31).  Query rows i = 0, 1 of a unit live in
-// quarter 0 and rows 2, 3 in quarter 1: lane 8 (i % 2) + h of the quarter
-// holds the high 16-bit part of head h's query, lane 16 + 8 (i % 2) + h its
-// low part (f32 queries keep f32-grade products: q = q_hi + q_lo in the
-// cache's 16-bit type), so one Q K^T MMA of M = 128 gives both partial
-// scores of every head of every row, in lanes l and l ^ 16 of one warp,
-// which add them with a shuffle; M rows 64-127 are never read.  In O += P V
-// the probabilities are stacked the same way (p = p_hi + p_lo in the same
-// two lanes) and the two O rows are added at the end.
+// (warp w: lanes 32 (w % 4) .. +31).  Query rows i = 2 q, 2 q + 1 of a unit
+// live in quarter q (quarters 0-1 for 4-row units, 0-3 for 8): lane
+// 8 (i % 2) + h of the quarter holds the high 16-bit part of head h's query,
+// lane 16 + 8 (i % 2) + h its low part (f32 queries keep f32-grade products:
+// q = q_hi + q_lo in the cache's 16-bit type), so one Q K^T MMA of M = 128
+// gives both partial scores of every head of every row, in lanes l and
+// l ^ 16 of one warp, which add them with a shuffle; the M rows of unused
+// quarters are never read.  In O += P V the probabilities are stacked the
+// same way (p = p_hi + p_lo in the same two lanes) and the two O rows are
+// added at the end.
 //
-// Warp roles (16 warps, all of which stage the queries):
-//   warps 0, 4, 8, 12 (quarter 0) and 1, 5, 9, 13 (quarter 1)   softmax:
-//            warp 4 g + q takes key columns [16 g, +16) of every stage for
-//            the rows of quarter q (the high lane of a head columns 16 g ..
-//            + 7, the low lane 16 g + 8 .. + 15) and O columns [64 g, +64),
-//            then the epilogue; a stage's row max is exchanged between the
-//            quarter's four warps through shared memory
-//   warp 2   TMEM allocator; lane 0 issues every MMA; the warp zeroes the V
-//            rows of a ragged last stage
-//   warps 3, 7   TMA producers of K stages (64 keys x 256 dims, ring of 3)
-//                and of V stages (ring of 2)
-// Shared memory: Q (64 M rows x 256 dims, four 64-dim chunks of 8 KiB with
-// 128-byte swizzle; the descriptors of the last chunk reach on into the
-// bytes after it, which land only in unused M rows), the K and V rings.
+// Warp roles (16 warps for 4-row units, 19 for 8; all stage the queries):
+//   warps 4 g + q, q a quarter in use   softmax: key columns [16 g, +16)
+//            of every stage for the rows of quarter q (the high lane of a
+//            head columns 16 g .. + 7, the low lane 16 g + 8 .. + 15) and O
+//            columns [64 g, +64), then the epilogue; a stage's row max is
+//            exchanged between the quarter's four warps through shared memory
+//   warp 2 (16 for 8-row units)   TMEM allocator; lane 0 issues every MMA;
+//            the warp zeroes the V rows of a ragged last stage
+//   warps 3, 7 (17, 18)   TMA producers of K stages (64 keys x 256 dims, a
+//            ring of 3, of 2 for 8-row units) and of V stages (ring of 2)
+// Shared memory: Q (32 M rows per quarter in use x 256 dims, four 64-dim
+// chunks with 128-byte swizzle; for 4-row units the descriptors of the last
+// chunk reach on into the bytes after it, which land only in unused M rows),
+// the K and V rings.
 // Tensor memory (512 columns): S of stage j at [64 (j & 1), +64), P of stage
 // j at [128 + 32 (j & 1), +32) (16-bit pairs), O at [256, 512).
 // Per stage j the MMA thread issues Q K^T of stage j, then P V of stage
@@ -61,45 +63,57 @@
 namespace kca {
 namespace {
 
-constexpr int kRThreads = 512;
 constexpr int kRQuarterThreads = 128;                // the softmax warps of one TMEM lane quarter
 constexpr int kRKeys = 64;                           // keys per stage
 constexpr int kRBox = 64 * 64 * 2;                   // 64 rows x 64 dims (16-bit): 8 KiB
 constexpr int kRSlot = 4 * kRBox;                    // K or V of one stage: 32 KiB
-constexpr int kRKRing = 3, kRVRing = 2;
-constexpr int kRQRows = 8 * kMultiRows;              // 32 query rows x heads, twice (high, low)
-constexpr int kRQChunk = 2 * kRQRows * 128;          // 64 M rows x 64 dims: 8 KiB
-constexpr int kROffQ = 0;
-constexpr int kROffK = 4 * kRQChunk;                 // 32 KiB
-constexpr int kROffV = kROffK + kRKRing * kRSlot;    // 128 KiB
-constexpr int kROffBar = kROffV + kRVRing * kRSlot;  // 192 KiB
-constexpr int kRBarBytes = 4096;
-constexpr int kRSmemBytes = kROffBar + kRBarBytes + 1024;   // + alignment slack
-static_assert(kRSmemBytes <= 232448, "shared memory over the per-CTA limit");
-// A descriptor of 128 M rows starting at the last Q chunk reads 8 KiB past
-// the Q area, into the first K slot: those bytes only reach M rows 64-127
-// of S, which nothing reads (an MMA's D row depends on its A row alone).
-static_assert(kROffQ + 3 * kRQChunk + 16 * 1024 <= kROffV, "Q descriptors stay inside shared memory");
 constexpr uint32_t kRColS = 0, kRColP = 128, kRColO = 256, kRTmemCols = 512;
 constexpr float kRRescaleLog2 = 8.f;   // rescale O once a score passes the reference by 2^8
 // Merge tickets: one per unit, after the workspace's 256-byte status word.
 constexpr int kRTickets = (KCA_WORKSPACE_HEADER - 256) / 4;
 static_assert(KCA_MAX_BATCH * ((KCA_MAX_BATCH_ROWS + kMultiRows - 1) / kMultiRows) <= kRTickets, "tickets");
 
+// Layout of a unit of UR rows (4 or 8): UR / 2 TMEM lane quarters, four
+// softmax warps per quarter, then the MMA and producer warps; a wide unit's
+// Q takes all 128 M rows, so its K ring is one stage shorter.
+template <int UR>
+struct RowsTc {
+  static constexpr int NQ = UR / 2;                       // lane quarters in use
+  static constexpr int kWarps = UR == 4 ? 16 : 19;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kMmaWarp = UR == 4 ? 2 : 16, kKWarp = UR == 4 ? 3 : 17, kVWarp = UR == 4 ? 7 : 18;
+  static constexpr int kKRing = UR == 4 ? 3 : 2, kVRing = 2;
+  static constexpr int kQChunk = 32 * NQ * 128;           // 32 NQ M rows x 64 dims
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = 4 * kQChunk;
+  static constexpr int kOffV = kOffK + kKRing * kRSlot;
+  static constexpr int kOffBar = kOffV + kVRing * kRSlot;
+  static constexpr int kBarBytes = 8192;
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory over the per-CTA limit");
+  // A descriptor of 128 M rows starting at the last Q chunk reads past the Q
+  // area when UR = 4, into the first K slot: those bytes only reach M rows
+  // 64-127 of S, which nothing reads (an MMA's D row depends on its A row).
+  static_assert(kOffQ + 3 * kQChunk + 16 * 1024 <= kOffV, "Q descriptors stay inside shared memory");
+};
+
+template <int UR>
 struct RBars {
-  uint64_t kfull[kRKRing], kempty[kRKRing];
-  uint64_t vfull[kRVRing], vempty[kRVRing];
+  static constexpr int NQ = UR / 2;
+  uint64_t kfull[RowsTc<UR>::kKRing], kempty[RowsTc<UR>::kKRing];
+  uint64_t vfull[RowsTc<UR>::kVRing], vempty[RowsTc<UR>::kVRing];
   uint64_t s_full[2];   // Q K^T of stage j complete in S buffer j & 1 (MMA commit)
-  uint64_t p_full[2];   // P of stage j written and O corrected (the eight softmax warps)
+  uint64_t p_full[2];   // P of stage j written and O corrected (the softmax warps)
   uint64_t o_done[2];   // P V of stage j complete (MMA commit)
   uint64_t drain;       // every MMA complete (single use)
   uint32_t tmem_base;
   int abort;
   int last;             // this CTA drew the unit's last ticket: it merges the splits
-  float red[2][2][4][32];  // [stage parity][quarter][column group][lane]: partial row maxima
-  float red_l[2][4][32];   // [quarter][column group][lane]: partial row sums at the end
+  float red[2][NQ][4][32];  // [stage parity][quarter][column group][lane]: partial row maxima
+  float red_l[NQ][4][32];   // [quarter][column group][lane]: partial row sums at the end
 };
-static_assert(sizeof(RBars) <= kRBarBytes, "barrier block too large");
+static_assert(sizeof(RBars<8>) <= RowsTc<8>::kBarBytes && sizeof(RBars<4>) <= RowsTc<4>::kBarBytes,
+              "barrier block too large");
 
 template <int KT>
 __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
@@ -123,16 +137,20 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-template <int QT, int KT>
-__global__ void __launch_bounds__(kRThreads, 1)
+template <int QT, int KT, int UR>
+__global__ void __launch_bounds__(RowsTc<UR>::kThreads, 1)
     rows_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const RowsArgs a) {
+  using T = RowsTc<UR>;
+  constexpr int kRThreads = T::kThreads;
+  constexpr int kRKRing = T::kKRing, kRVRing = T::kVRing, kRQChunk = T::kQChunk;
+  constexpr int kROffQ = T::kOffQ, kROffK = T::kOffK, kROffV = T::kOffV;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
   unsigned char* smem = smem_raw + pad;
   const uint32_t sbase = raw_addr + pad;
-  RBars* bars = reinterpret_cast<RBars*>(smem + kROffBar);
+  RBars<UR>* bars = reinterpret_cast<RBars<UR>*>(smem + T::kOffBar);
   volatile int* abort_flag = &bars->abort;
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(a.status);
 
@@ -171,19 +189,19 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 2 * kRQuarterThreads / 32);
+      mbar_init(&bars->p_full[s], T::NQ * kRQuarterThreads / 32);
       mbar_init(&bars->o_done[s], 1);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
-  if (warp == 2) {
+  if (warp == T::kMmaWarp) {
     ptx::tmem_alloc(smem_u32(&bars->tmem_base), kRTmemCols);
     ptx::tmem_relinquish();
   }
-  if (threadIdx.x == 3 * 32) ptx::prefetch_tmap(&tmk);
-  if (threadIdx.x == 7 * 32) ptx::prefetch_tmap(&tmv);
+  if (threadIdx.x == T::kKWarp * 32) ptx::prefetch_tmap(&tmk);
+  if (threadIdx.x == T::kVWarp * 32) ptx::prefetch_tmap(&tmv);
   ptx::fence_before_sync();
   __syncthreads();
   ptx::fence_after_sync();
@@ -195,7 +213,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   // Stage the queries: M row m = 32 q + 16 part + 8 (i % 2) + h for query
   // row i = 2 q + ..., head h, part 0 (high) or 1 (low); absent rows zero.
   // 16-byte group u of the 256 dims: chunk u / 8, 128-byte swizzle within it.
-  for (int it = threadIdx.x; it < 64 * 32; it += kRThreads) {
+  for (int it = threadIdx.x; it < 32 * T::NQ * 32; it += kRThreads) {
     const int m = it >> 5, u = it & 31;
     const int part = (m >> 4) & 1, i = 2 * (m >> 5) + ((m >> 3) & 1), h = m & 7;
     float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -216,10 +234,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
   fence_proxy_async_smem();   // generic stores -> visible to the tensor core
   __syncthreads();
 
-  if (warp == 3 || warp == 7) {
+  if (warp == T::kKWarp || warp == T::kVWarp) {
     // ------------------------------------------------------------ producers
     if (lane == 0) {
-      const bool is_k = warp == 3;
+      const bool is_k = warp == T::kKWarp;
       const int ring = is_k ? kRKRing : kRVRing;
       uint64_t* full = is_k ? bars->kfull : bars->vfull;
       uint64_t* empty = is_k ? bars->kempty : bars->vempty;
@@ -245,7 +263,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 2) {
+  } else if (warp == T::kMmaWarp) {
     // ----------------------------------------------------------------- MMA
     constexpr uint32_t ab = KT == KCA_BF16 ? 1u : 0u;
     constexpr uint32_t id_qk = ptx::idesc_f16(ab, 128, kRKeys, 0);
@@ -317,7 +335,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (lane == 0) ptx::mma_commit(smem_u32(&bars->drain));
     __syncwarp();
     mbar_wait(&bars->drain, 0, nullptr, status, kSiteTcDrain);
-  } else if ((warp & 3) <= 1) {
+  } else if (warp < 16 && (warp & 3) < T::NQ) {
     // ------------------------------------------------------------- softmax
     // Warp 4 g + q: quarter q (query rows 2 q, 2 q + 1), key columns
     // [16 g, +16) of every stage, O columns [64 g, +64).  Lane l: query row
@@ -491,7 +509,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   // No warp leaves while MMAs may still read shared memory or write TMEM.
   ptx::fence_before_sync();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == T::kMmaWarp) {
     ptx::fence_after_sync();
     ptx::tmem_dealloc(tmem, kRTmemCols);
   }
@@ -545,14 +563,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-template <int QT, int KT>
+template <int QT, int KT, int UR>
 cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsArgs& a, cudaStream_t stream) {
-  auto kern = rows_tc_kernel<QT, KT>;
+  using T = RowsTc<UR>;
+  auto kern = rows_tc_kernel<QT, KT, UR>;
   static std::atomic<bool> attr_set[64];   // per device; zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmemBytes);
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -561,8 +580,8 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsA
   at.val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.max_splits, a.n_units, 1);
-  cfg.blockDim = dim3(kRThreads, 1, 1);
-  cfg.dynamicSmemBytes = kRSmemBytes;
+  cfg.blockDim = dim3(T::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = T::kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = &at;
   cfg.numAttrs = 1;
@@ -575,8 +594,10 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const RowsA
 
 cudaError_t launch_rows_tc(int q_dtype, int kv_dtype, const CUtensorMap& tmk, const CUtensorMap& tmv,
                            const RowsArgs& a, cudaStream_t stream) {
-#define KCA_RTC_CASE(QD, KD) \
-  if (q_dtype == QD && kv_dtype == KD) return launch_t<QD, KD>(tmk, tmv, a, stream);
+#define KCA_RTC_CASE(QD, KD)                                                                \
+  if (q_dtype == QD && kv_dtype == KD)                                                      \
+    return a.unit_rows == kMultiRowsWide ? launch_t<QD, KD, kMultiRowsWide>(tmk, tmv, a, stream) \
+                                         : launch_t<QD, KD, kMultiRows>(tmk, tmv, a, stream);
   KCA_RTC_CASE(KCA_F32, KCA_F16)
   KCA_RTC_CASE(KCA_F32, KCA_BF16)
   KCA_RTC_CASE(KCA_F16, KCA_F16)
