@@ -189,10 +189,12 @@ int attn_decode(const void *q, int32_t q_dtype,
  * sequence b has `rows` query rows, at positions ctx_len[b] - rows ..
  * ctx_len[b] - 1 (speculative or multi-row decode steps), every row seeing
  * its sequence's keys as in attn_prefill.  With a 16-bit cache and rows > 1,
- * one launch of the multi-row tensor-core kernel (units of up to 4
- * consecutive rows of a sequence, so each K/V row crosses to the SM once per
- * unit; the union of the unit's keys cut into splits across the GPU) plus a
- * merge launch; otherwise the rows path of decode (one unit per row).  As in
+ * one launch of the multi-row tcgen05 kernel (units of up to 4 consecutive
+ * rows of a sequence, 8 when rows > 4, so each K/V row crosses to the SM
+ * once per unit; the union of the unit's keys cut into splits across the
+ * GPU, merged in the same kernel, or by a second launch when a unit has
+ * more than 16 splits); otherwise the rows path of decode (one unit per
+ * row).  As in
  * tensor-core prefill, V must be finite on the rows of a unit's key union:
  * a masked key's zero probability multiplies its V row.
  * Passage: Karume v0.12.0 release notes, "Docs", ADR 0067 plan-size geometry
