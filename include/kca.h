@@ -58,11 +58,14 @@
  * q_dtype == kv_dtype in {F16, BF16} and chunk_rows >= 16 runs on the
  * tcgen05 tensor-core path (16-row tiles, f32 accumulation).  Chunks of 3-15
  * such rows take that path too when their first row sees at least 12,288
- * keys (one pass over the keys beats one pass per row there), else the rows
- * path, which also serves every other prefill combination: one unit per
- * query row, mma.sync with split-precision operands for 16-bit caches,
- * CUDA-core f32 for f32 caches.  attn_force_path pins either choice, so that
- * tests can compare the paths on the same inputs.
+ * keys (one pass over the keys beats one pass per row there).  Other chunks
+ * of 2-15 rows on a 16-bit cache (mixed dtypes, or 2 rows) whose first row
+ * sees at least 12,288 keys take multi-row units (the kernel of
+ * attn_prefill_batch for one sequence).  The rows path serves every other
+ * prefill combination: one unit per query row, mma.sync with
+ * split-precision operands for 16-bit caches, CUDA-core f32 for f32 caches.
+ * attn_force_path pins any of the three, so that tests can compare the
+ * paths on the same inputs.
  *
  * QUERIES: the workspace-size and plan queries come one per operation
  * (attn_prefill_workspace_bytes, attn_decode_workspace_bytes,
@@ -476,9 +479,16 @@ int attn_device_status(void *workspace, void *stream, uint32_t *detail);
  *     clusters-per-sequence + split / cluster size), or -1 when the unit is
  *     one cluster and merges in shared memory.  *cluster, if not NULL,
  *     receives the cluster size (1 on the CUDA-core kernel).
- * *path receives 0 for the rows path, 1 for the tensor-core path; it is set
- * once the arguments are valid, before any device query, so it also answers
- * a call that then fails for want of a device.
+ *   multi-row units (short chunks on 16-bit caches, see DTYPES): one item
+ *     per split of a unit of consecutive rows (4, or 8 when the chunk has
+ *     more than 4 rows), unit = the unit's index, [key_begin, key_end)
+ *     within the union of its rows' visible keys, slot = the split's index,
+ *     or -1 when the unit has one split; the plan of the rows kernels for
+ *     num_sms SMs (host only).
+ * *path receives 0 for the rows path, 1 for the tensor-core path, 2 for
+ * multi-row units; it is set once the arguments are valid, before any
+ * device query, so it also answers a call that then fails for want of a
+ * device.
  * Returns KCA_OK, or KCA_ERR_RANGE when more than max_items items exist
  * (*n_items still receives the count) or a capacity is negative.
  */
@@ -506,7 +516,8 @@ int attn_decode_cluster_capacity(int32_t *capacity);
  * attn_force_path -- pins the kernel family that later calls take,
  * process-wide, so that two paths can be compared on the same inputs (tests,
  * diagnosis).  op 0 (prefill): path 0 = the rows path, 1 = the tensor-core
- * path where eligible (q and cache both F16 or both BF16).  op 1 (the rows
+ * path where eligible (q and cache both F16 or both BF16), 2 = multi-row
+ * units where eligible (16-bit cache, 2-15 rows).  op 1 (the rows
  * path: decode, and prefill chunks on the rows path): path 0 = the CUDA-core
  * kernel, 1 = the tensor-core (mma.sync) kernel where eligible (16-bit
  * cache).  op 2 (attn_prefill_batch with 2 or more rows per sequence on a

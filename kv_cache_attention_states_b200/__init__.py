@@ -545,11 +545,12 @@ OP_PREFILL, OP_ROWS, OP_BATCH = 0, 1, 2           # attn_force_path operations
 PATH_AUTO, PATH_ROWS, PATH_TENSOR_CORE = -1, 0, 1
 PATH_CUDA_CORE = 0                               # OP_ROWS: the CUDA-core kernel
 PATH_MMA_SYNC, PATH_TCGEN05 = 0, 1               # OP_BATCH: the multi-row kernels
+PATH_MULTI_ROW = 2                               # OP_PREFILL: multi-row units (short chunks, 16-bit cache)
 
 
 def attn_force_path(op: int, path: int) -> None:
     """Pin the kernel family of later calls, process-wide (see include/kca.h):
-    op OP_PREFILL with PATH_ROWS / PATH_TENSOR_CORE, op OP_ROWS with
+    op OP_PREFILL with PATH_ROWS / PATH_TENSOR_CORE / PATH_MULTI_ROW, op OP_ROWS with
     PATH_CUDA_CORE / PATH_TENSOR_CORE, op OP_BATCH with PATH_MMA_SYNC /
     PATH_TCGEN05; PATH_AUTO restores the automatic choice."""
     _check(lib().attn_force_path(int(op), int(path)), "attn_force_path")
@@ -585,7 +586,8 @@ def _num_sms(num_sms):
 
 def attn_prefill_path(q_dtype: int, kv_dtype: int, chunk_start: int, chunk_rows: int,
                       window: int = 0) -> int:
-    """The path a prefill call takes: 1 tensor-core, 0 rows (host only; no device needed)."""
+    """The path a prefill call takes: 1 tensor-core, 2 multi-row units, 0 rows
+    (host only; no device needed)."""
     n = ctypes.c_int32(0)
     path = ctypes.c_int32(-1)
     # the path does not depend on the SM count; any positive count serves

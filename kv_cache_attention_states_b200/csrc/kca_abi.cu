@@ -64,14 +64,14 @@ std::atomic<int> g_batch_path{-1};
 // paths (1-15 rows at 1K-64K keys) put the crossover at about 3 rows once
 // the rows see 12K keys or more; below 12K keys the rows path wins up to 15
 // rows.
+// Chunks of 2-15 rows on a 16-bit cache that the tensor-core path does not
+// take (mixed dtypes, or 2 rows) go to multi-row units once the first row
+// sees 12,288 keys: each K/V stage crosses to the SM once per 4 or 8 rows
+// (at 131,072 keys, 8 f32-query rows on a bf16 cache: 110 us on the rows
+// path, 40 us on multi-row units; 15 rows: 231 against 52 us).
+int prefill_route(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, int32_t rows, int32_t window);
 bool use_tc(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, int32_t rows, int32_t window) {
-  const bool eligible = q_dtype == kv_dtype && (q_dtype == KCA_F16 || q_dtype == KCA_BF16);
-  const int forced = g_prefill_path.load(std::memory_order_relaxed);
-  if (forced == 0) return false;
-  if (forced == 1) return eligible;
-  if (!eligible) return false;
-  if (rows >= kca::kRowTile) return true;
-  return rows >= 3 && kca::n_visible(chunk_start, window) >= 12288;
+  return prefill_route(q_dtype, kv_dtype, chunk_start, rows, window) == 1;
 }
 
 std::vector<int64_t> prefill_unit_keys(int64_t chunk_start, int32_t rows, int32_t window) {
@@ -281,6 +281,21 @@ bool use_multirow(int32_t kv_dtype, int32_t rows) { return rows > 1 && use_rows_
 // mma.sync one (op 2, path 0).
 bool use_batch_tc() { return g_batch_path.load(std::memory_order_relaxed) != 0; }
 
+// Route of a prefill chunk: 1 the tensor-core path, 2 multi-row units, 0 the
+// rows path.  A forced route (attn_force_path op 0) wins where eligible.
+int prefill_route(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, int32_t rows, int32_t window) {
+  const bool tc_ok = q_dtype == kv_dtype && (q_dtype == KCA_F16 || q_dtype == KCA_BF16);
+  const bool mr_ok = use_multirow(kv_dtype, rows) && rows <= KCA_MAX_BATCH_ROWS;
+  const int forced = g_prefill_path.load(std::memory_order_relaxed);
+  if (forced == 0) return 0;
+  if (forced == 1) return tc_ok ? 1 : 0;
+  if (forced == 2) return mr_ok ? 2 : 0;
+  const int64_t keys = kca::n_visible(chunk_start, window);
+  if (tc_ok && (rows >= kca::kRowTile || (rows >= 3 && keys >= 12288))) return 1;
+  if (mr_ok && keys >= 12288) return 2;
+  return 0;
+}
+
 // Plan of the tensor-core rows kernel.  Each cluster size c in {8, 4, 2}
 // (and c = 1 when every unit fits one split, so nothing is merged) gets the
 // plan that fills the clusters resident at once; the one with the lowest
@@ -427,6 +442,62 @@ int rows_plan_items(int32_t kv_dtype, int32_t n, const int64_t* pos, const int64
   return KCA_OK;
 }
 
+// Multi-row units (16-bit caches, 2-15 rows per sequence): units of ur
+// rows of one sequence, the union of their keys cut into splits over the
+// GPU; the tcgen05 kernel (units of 8 rows when a sequence has more than 4)
+// or, pinned, the mma.sync one.  Serves attn_prefill_batch and attn_prefill's
+// short chunks (one sequence at ctx_len = chunk_start + rows).
+int32_t multirow_unit_rows(int32_t rows) {
+  return use_batch_tc() && rows > kca::kMultiRows ? kca::kMultiRowsWide : kca::kMultiRows;
+}
+size_t multirow_route_ws_bytes(int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window, int sms) {
+  const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, multirow_unit_rows(rows));
+  return multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms));
+}
+int launch_multirow_route(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache, int32_t kv_dtype,
+                          int64_t capacity, int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window,
+                          float scale, float* out, void* workspace, size_t workspace_bytes, int sms, cudaStream_t s) {
+  const bool tc = use_batch_tc();
+  const int32_t ur = multirow_unit_rows(rows);
+  const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, ur);
+  const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms);
+  if (workspace_bytes < multirow_ws_bytes(batch, rows, mp)) return KCA_ERR_WORKSPACE;
+  kca::RowsArgs a{};
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.out = out;
+  a.status = workspace;
+  a.seq_rows = capacity;
+  a.mode = 2;
+  a.rows_per_seq = rows;
+  a.unit_rows = ur;
+  a.n_units = (int32_t)nku.size();
+  a.split_len = mp.split_len;
+  a.max_splits = mp.max_splits;
+  a.window = window;
+  a.scale = scale;
+  for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
+  a.cache_rows = (int64_t)batch * capacity;
+  a.part_slots = mp.max_splits > 1 ? (int64_t)batch * rows * mp.max_splits : 0;
+  if (mp.max_splits > 1) {
+    carve(workspace, (size_t)batch * rows * mp.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
+    // self-resetting per-unit merge tickets of the tcgen05 kernel, which
+    // then merges in-kernel; a unit with many splits is merged by a second
+    // kernel instead (one CTA would read all its partials: at 1 x 131,072
+    // keys, 147 splits, 141 us against 52 us with the merge kernel)
+    if (mp.max_splits <= kca::kRowsTcMergeSplits)
+      a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+  }
+  CUtensorMap tmk, tmv;
+  if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, (int64_t)batch * capacity, 64) ||
+      !encode_kv_map(&tmv, v_cache, kv_dtype, 0, (int64_t)batch * capacity, 64))
+    return KCA_ERR_CUDA;
+  const cudaError_t e = tc ? kca::launch_rows_tc(q_dtype, kv_dtype, tmk, tmv, a, s)
+                           : kca::launch_decode_multirow(q_dtype, kv_dtype, tmk, tmv, a, s);
+  return e == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -443,7 +514,7 @@ int attn_decode_cluster_capacity(int32_t* capacity) {
 }
 
 int attn_force_path(int32_t op, int32_t path) {
-  if (path < -1 || path > 1) return KCA_ERR_RANGE;
+  if (path < -1 || path > (op == 0 ? 2 : 1)) return KCA_ERR_RANGE;
   if (op == 0) g_prefill_path.store(path);
   else if (op == 1) g_rows_path.store(path);
   else if (op == 2) g_batch_path.store(path);
@@ -477,7 +548,28 @@ int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, in
   if (cluster_capacity != nullptr && (cluster_capacity[0] < 0 || cluster_capacity[1] < 0 || cluster_capacity[2] < 0))
     return KCA_ERR_RANGE;
   int32_t count = 0;
-  if (use_tc(q_dtype, kv_dtype, chunk_start, chunk_rows, window)) {
+  const int route = prefill_route(q_dtype, kv_dtype, chunk_start, chunk_rows, window);
+  if (route == 2) {
+    // multi-row units: one item per split of a unit of rows
+    *path = 2;
+    const int64_t ctx = chunk_start + chunk_rows;
+    const int32_t ur = multirow_unit_rows(chunk_rows);
+    const std::vector<int64_t> nku = multirow_unit_keys(1, chunk_rows, &ctx, window, ur);
+    const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), num_sms);
+    for (int32_t u = 0; u < (int32_t)nku.size(); ++u) {
+      const int64_t lo = kca::lo_of(chunk_start + (int64_t)u * ur, window);
+      const int32_t ns = kca::rows_n_splits(nku[u], mp.split_len);
+      for (int32_t sp = 0; sp < ns; ++sp, ++count) {
+        if (count >= max_items) continue;
+        int64_t kb = lo + (int64_t)sp * mp.split_len, ke = kb + mp.split_len;
+        if (ke > lo + nku[u]) ke = lo + nku[u];
+        items[4 * count + 0] = u;
+        items[4 * count + 1] = kb;
+        items[4 * count + 2] = ke;
+        items[4 * count + 3] = ns > 1 ? sp : -1;
+      }
+    }
+  } else if (route == 1) {
     *path = 1;
     const kca::TcPlan p = kca::make_tc_plan(chunk_start, chunk_rows, window, num_sms / 2);
     for (int32_t i = 0; i < p.n_items; ++i) {
@@ -533,8 +625,12 @@ size_t attn_prefill_workspace_bytes(int32_t q_dtype, int32_t kv_dtype, int64_t c
   if (prefill_args_status(KCA_MAX_POSITION, chunk_start, chunk_rows) != KCA_OK) return 0;
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return 0;
-  if (use_tc(q_dtype, kv_dtype, chunk_start, chunk_rows, window))
-    return tc_ws_bytes(kca::make_tc_plan(chunk_start, chunk_rows, window, sms / 2));
+  const int route = prefill_route(q_dtype, kv_dtype, chunk_start, chunk_rows, window);
+  if (route == 1) return tc_ws_bytes(kca::make_tc_plan(chunk_start, chunk_rows, window, sms / 2));
+  if (route == 2) {
+    const int64_t ctx = chunk_start + chunk_rows;
+    return multirow_route_ws_bytes(1, chunk_rows, &ctx, window, sms);
+  }
   const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
   return rows_ws_bytes_any(chunk_rows, nk.data(), sms);
 }
@@ -655,6 +751,11 @@ int attn_prefill(const void* q_chunk, int32_t q_dtype, const void* k_cache, cons
                : KCA_ERR_CUDA;
   }
 
+  if (prefill_route(q_dtype, kv_dtype, chunk_start, chunk_rows, window) == 2) {
+    // one sequence of chunk_rows rows ending at ctx_len, in multi-row units
+    return launch_multirow_route(q_chunk, q_dtype, k_cache, v_cache, kv_dtype, capacity, 1, chunk_rows, &ctx_len,
+                                 window, scale, out, workspace, workspace_bytes, sms, s);
+  }
   const std::vector<int64_t> nk = prefill_unit_keys(chunk_start, chunk_rows, window);
   int cluster = 1;
   size_t need = 0;
@@ -856,48 +957,9 @@ int attn_prefill_batch(const void* q, int32_t q_dtype, const void* k_cache, cons
   int sms = 0;
   if (current_sms(&sms) != KCA_OK) return KCA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (use_multirow(kv_dtype, rows)) {
-    // the tcgen05 kernel takes units of 8 rows when a sequence has more than 4
-    const bool tc = use_batch_tc();
-    const int32_t ur = tc && rows > kca::kMultiRows ? kca::kMultiRowsWide : kca::kMultiRows;
-    const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, ur);
-    const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms);
-    if (workspace_bytes < multirow_ws_bytes(batch, rows, mp)) return KCA_ERR_WORKSPACE;
-    kca::RowsArgs a{};
-    a.q = q;
-    a.k = k_cache;
-    a.v = v_cache;
-    a.out = out;
-    a.status = workspace;
-    a.seq_rows = capacity;
-    a.mode = 2;
-    a.rows_per_seq = rows;
-    a.unit_rows = ur;
-    a.n_units = (int32_t)nku.size();
-    a.split_len = mp.split_len;
-    a.max_splits = mp.max_splits;
-    a.window = window;
-    a.scale = scale;
-    for (int32_t b = 0; b < batch; ++b) a.ctx[b] = ctx_len[b];
-    a.cache_rows = (int64_t)batch * capacity;
-    a.part_slots = mp.max_splits > 1 ? (int64_t)batch * rows * mp.max_splits : 0;
-    if (mp.max_splits > 1) {
-      carve(workspace, (size_t)batch * rows * mp.max_splits * kHeads * 2 * 4, &a.part_ml, &a.part_acc);
-      // self-resetting per-unit merge tickets of the tcgen05 kernel, which
-      // then merges in-kernel; a unit with many splits is merged by a second
-      // kernel instead (one CTA would read all its partials: at 1 x 131,072
-      // keys, 147 splits, 141 us against 52 us with the merge kernel)
-      if (mp.max_splits <= kca::kRowsTcMergeSplits)
-        a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
-    }
-    CUtensorMap tmk, tmv;
-    if (!encode_kv_map(&tmk, k_cache, kv_dtype, 0, (int64_t)batch * capacity, 64) ||
-        !encode_kv_map(&tmv, v_cache, kv_dtype, 0, (int64_t)batch * capacity, 64))
-      return KCA_ERR_CUDA;
-    const cudaError_t e = tc ? kca::launch_rows_tc(q_dtype, kv_dtype, tmk, tmv, a, s)
-                             : kca::launch_decode_multirow(q_dtype, kv_dtype, tmk, tmv, a, s);
-    return e == cudaSuccess ? KCA_OK : KCA_ERR_CUDA;
-  }
+  if (use_multirow(kv_dtype, rows))
+    return launch_multirow_route(q, q_dtype, k_cache, v_cache, kv_dtype, capacity, batch, rows, ctx_len, window,
+                                 scale, out, workspace, workspace_bytes, sms, s);
   const int32_t n_units = batch * rows;
   const std::vector<int64_t> nk = batch_unit_keys(batch, rows, ctx_len, window);
   int cluster = 1;

@@ -51,7 +51,7 @@ def test_every_declared_call_cites_its_passage():
 
 def test_force_path_validates_and_restores():
     lib = kca.lib()
-    assert lib.attn_force_path(3, 0) == -4 and lib.attn_force_path(0, 2) == -4
+    assert lib.attn_force_path(3, 0) == -4 and lib.attn_force_path(0, 3) == -4 and lib.attn_force_path(1, 2) == -4
     assert lib.attn_force_path(2, 0) == 0 and lib.attn_force_path(2, -1) == 0   # op 2: the multi-row kernels
     assert lib.attn_force_path(-1, 0) == -4 and lib.attn_force_path(1, -2) == -4
     assert kca.attn_prefill_path(kca.BF16, kca.BF16, 0, 768) == 1
@@ -396,6 +396,37 @@ def test_few_row_chunks_on_long_contexts_take_the_tensor_core_path():
     assert kca.attn_prefill_path(kca.F16, kca.F16, 12287, 15) == 1
     assert kca.attn_prefill_path(kca.BF16, kca.BF16, 12287, 3) == 1
     assert kca.attn_prefill_path(kca.BF16, kca.BF16, 12286, 3) == 0
-    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 16382, 2) == 0
     assert kca.attn_prefill_path(kca.BF16, kca.BF16, 16381, 3, 4096) == 0   # window: 4096 keys
     assert kca.attn_prefill_path(kca.F32, kca.F32, 16381, 3) == 0
+    # the other 2-15-row chunks on a 16-bit cache from 12,288 keys: multi-row units
+    assert kca.attn_prefill_path(kca.BF16, kca.BF16, 16382, 2) == 2
+    assert kca.attn_prefill_path(kca.F32, kca.BF16, 16381, 3) == 2
+    assert kca.attn_prefill_path(kca.F32, kca.F16, 12287, 15) == 2
+    assert kca.attn_prefill_path(kca.F32, kca.F16, 12286, 15) == 0
+    assert kca.attn_prefill_path(kca.F32, kca.BF16, 16368, 16) == 0     # 16 rows: one unit per row
+    assert kca.attn_prefill_path(kca.F32, kca.BF16, 16381, 3, 4096) == 0
+    with kca.forced_path(kca.OP_PREFILL, kca.PATH_MULTI_ROW):
+        assert kca.attn_prefill_path(kca.F32, kca.BF16, 10, 3) == 2
+        assert kca.attn_prefill_path(kca.BF16, kca.BF16, 10, 1) == 0        # one row: not a unit of rows
+        assert kca.attn_prefill_path(kca.F32, kca.F32, 16381, 3) == 0       # f32 cache: no multi-row kernel
+    with kca.forced_path(kca.OP_ROWS, kca.PATH_CUDA_CORE):                  # multi-row units need the TC rows kernels
+        assert kca.attn_prefill_path(kca.F32, kca.BF16, 16381, 3) == 0
+
+
+@pytest.mark.parametrize("chunk_start,rows,window", [(20000, 15, 0), (20000, 3, 0), (130000, 8, 0), (50000, 6, 15000)])
+def test_multi_row_plan_tiles_each_units_key_union(chunk_start, rows, window):
+    # path 2 items: per unit of 4 or 8 consecutive rows, splits that tile the
+    # union of the unit's visible keys exactly (the rows' lo .. the last
+    # row's position), in order, one plan split length apart
+    path, items = kca.attn_prefill_plan(kca.F32, kca.BF16, chunk_start, rows, window, num_sms=148)
+    assert path == 2
+    ur = 8 if rows > 4 else 4
+    units = (rows + ur - 1) // ur
+    assert sorted(set(items[:, 0].tolist())) == list(range(units))
+    for u in range(units):
+        it = items[items[:, 0] == u]
+        first, last = chunk_start + u * ur, min(chunk_start + rows, chunk_start + (u + 1) * ur) - 1
+        lo = max(0, first - window + 1) if window > 0 else 0
+        assert it[0, 1] == lo and it[-1, 2] == last + 1
+        assert (it[1:, 1] == it[:-1, 2]).all() and (it[:, 2] > it[:, 1]).all()
+        assert it[:, 3].tolist() == (list(range(len(it))) if len(it) > 1 else [-1])

@@ -190,3 +190,28 @@ def test_nan_in_a_value_row_reaches_the_whole_multirow_unit(path):
     out32 = kca.attn_prefill_batch(dev(q, "f32"), dev(k.astype(np.float32), "f32"), dev(v.astype(np.float32), "f32"),
                                    ctx).cpu().numpy()
     assert np.isfinite(out32[0, :2]).all() and np.isnan(out32[0, 2:]).any(axis=(1, 2)).all()
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype,rows,cs,window", [("f32", "bf16", 8, 20000, 0), ("f32", "f16", 15, 30000, 0),
+                                                            ("bf16", "bf16", 2, 16000, 0),
+                                                            ("f32", "bf16", 5, 40000, 20000)])
+def test_short_prefill_chunks_on_multi_row_units(q_dtype, kv_dtype, rows, cs, window):
+    # attn_prefill routes 2-15-row chunks on a 16-bit cache that the
+    # tensor-core path does not take to multi-row units from 12,288 keys: every
+    # row against the oracle, and the rows path (pinned) within tolerance
+    from tests.helpers import oracle_prefill
+    code = {"f32": kca.F32, "f16": kca.F16, "bf16": kca.BF16}
+    assert kca.attn_prefill_path(code[q_dtype], code[kv_dtype], cs, rows, window) == kca.PATH_MULTI_ROW
+    cap = cs + rows
+    q = synth.draw(67, "q", (rows, 8, 256), q_dtype)
+    k = synth.draw(67, "k", (cap, 256), kv_dtype)
+    v = synth.draw(67, "v", (cap, 256), kv_dtype)
+    qd, kd, vd = dev(q, q_dtype), dev(k, kv_dtype), dev(v, kv_dtype)
+    ws = kca.new_workspace(kca.attn_prefill_workspace_bytes(kca.dtype_code(qd), kca.dtype_code(kd), cs, rows, window))
+    got = kca.attn_prefill(qd, kd, vd, cs, window, workspace=ws).cpu().numpy()
+    assert kca.attn_device_status(ws)[0] == 0
+    want = oracle_prefill(q, k, v, cs, np.arange(rows), window, q_dtype, kv_dtype)
+    assert max_err(got, want) <= tol(q_dtype, kv_dtype)
+    with kca.forced_path(kca.OP_PREFILL, kca.PATH_ROWS):
+        ref = kca.attn_prefill(qd, kd, vd, cs, window).cpu().numpy()
+    assert np.max(np.abs(got - ref)) <= tol(q_dtype, kv_dtype)
