@@ -452,7 +452,7 @@ int32_t multirow_unit_rows(int32_t rows) {
 }
 size_t multirow_route_ws_bytes(int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window, int sms) {
   const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, multirow_unit_rows(rows));
-  return multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms));
+  return multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms, kca::kMultiRowMinSplit));
 }
 int launch_multirow_route(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache, int32_t kv_dtype,
                           int64_t capacity, int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window,
@@ -460,7 +460,7 @@ int launch_multirow_route(const void* q, int32_t q_dtype, const void* k_cache, c
   const bool tc = use_batch_tc();
   const int32_t ur = multirow_unit_rows(rows);
   const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, ur);
-  const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms);
+  const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms, kca::kMultiRowMinSplit);
   if (workspace_bytes < multirow_ws_bytes(batch, rows, mp)) return KCA_ERR_WORKSPACE;
   kca::RowsArgs a{};
   a.q = q;
@@ -555,7 +555,7 @@ int attn_prefill_plan(int32_t q_dtype, int32_t kv_dtype, int64_t chunk_start, in
     const int64_t ctx = chunk_start + chunk_rows;
     const int32_t ur = multirow_unit_rows(chunk_rows);
     const std::vector<int64_t> nku = multirow_unit_keys(1, chunk_rows, &ctx, window, ur);
-    const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), num_sms);
+    const kca::RowsPlan mp = kca::make_rows_plan((int32_t)nku.size(), nku.data(), num_sms, kca::kMultiRowMinSplit);
     for (int32_t u = 0; u < (int32_t)nku.size(); ++u) {
       const int64_t lo = kca::lo_of(chunk_start + (int64_t)u * ur, window);
       const int32_t ns = kca::rows_n_splits(nku[u], mp.split_len);
@@ -653,7 +653,7 @@ size_t attn_prefill_batch_workspace_bytes(int32_t batch, int32_t rows, const int
   if (rows > 1) {   // the multi-row kernels' partials, whichever path and unit size a call takes
     for (const int32_t ur : {kca::kMultiRows, kca::kMultiRowsWide}) {
       const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, ur);
-      const size_t mr = multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms));
+      const size_t mr = multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms, kca::kMultiRowMinSplit));
       if (mr > need) need = mr;
     }
   }

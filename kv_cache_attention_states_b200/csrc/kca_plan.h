@@ -70,9 +70,13 @@ constexpr int kRowsMinSplit = 64;
 constexpr int kRowsSplitQuantum = 16;
 
 // nkeys[u]: visible keys of unit u.  split_len is the smallest multiple of
-// the quantum (>= kRowsMinSplit) whose split count fits one wave; when even
-// one split per unit does not fit, every unit gets a single split.
-inline RowsPlan make_rows_plan(int32_t n_units, const int64_t* nkeys, int32_t num_sms) {
+// the quantum (>= min_split) whose split count fits one wave; when even one
+// split per unit does not fit, every unit gets a single split.  Multi-row
+// units, whose CTAs cost more to start (a unit's queries, tensor memory, a
+// merge of more rows), take longer splits at least.
+constexpr int kMultiRowMinSplit = 256;
+inline RowsPlan make_rows_plan(int32_t n_units, const int64_t* nkeys, int32_t num_sms,
+                               int32_t min_split = kRowsMinSplit) {
   RowsPlan p;
   p.n_units = n_units;
   int64_t max_keys = 0;
@@ -83,8 +87,8 @@ inline RowsPlan make_rows_plan(int32_t n_units, const int64_t* nkeys, int32_t nu
     for (int32_t u = 0; u < n_units; ++u) c += rows_n_splits(nkeys[u], (int32_t)len);
     return c;
   };
-  int64_t hi = cdiv(max_keys > kRowsMinSplit ? max_keys : kRowsMinSplit, kRowsSplitQuantum);
-  int64_t lo = cdiv(kRowsMinSplit, kRowsSplitQuantum);
+  int64_t hi = cdiv(max_keys > min_split ? max_keys : min_split, kRowsSplitQuantum);
+  int64_t lo = cdiv(min_split, kRowsSplitQuantum);
   if (count(lo * kRowsSplitQuantum) <= target) {
     hi = lo;
   } else {
