@@ -68,7 +68,7 @@ TRAFFIC = {
     "window_decode": (595456.0, "decode_mma_kernel<bf16, bf16>, one call, window 512 (cold caches)"),
     "long_chunk": (138080256.0 + 4125184.0, "prefill_tc_kernel, the 768-row chunk at 130304"),
     "decode_q8_ragged": (350935296.0 + 3392512.0, "decode_mma_kernel<f32, int8 K, f16 V>, one call of the 8 sequences"),
-    "prefill_batch": (301815040.0 + 470016.0, "rows_tc_kernel, one call of 32 sequences x 4 rows "
+    "prefill_batch": (301807360.0 + 525824.0, "rows_tc_kernel, one call of 32 sequences x 4 rows "
                                               "(its splits merged in-kernel)"),
 }
 E2E_GROUP = 4            # prefill chunks per host copy in the end-to-end leg
