@@ -40,9 +40,9 @@ def _rank(rank, world, port, values, out):
 def test_two_gloo_ranks_take_the_maximum_over_ranks():
     world = 2
     values = [[3.0, 10.0, 0.5], [7.0, 2.0, 0.5]]
-    with mp.Manager() as manager:
+    ctx = mp.get_context("spawn")          # the manager's server process too: no fork of a threaded process
+    with ctx.Manager() as manager:
         out = manager.dict()
-        ctx = mp.get_context("spawn")
         port = _free_port()
         procs = [ctx.Process(target=_rank, args=(r, world, port, values, out)) for r in range(world)]
         for p in procs:
@@ -94,9 +94,9 @@ def test_context_split_exchange_gathers_records_in_rank_order():
     from oracle import partial
     from kv_cache_attention_states_b200 import synth
     world = 2
-    with mp.Manager() as manager:
+    ctx_ = mp.get_context("spawn")
+    with ctx_.Manager() as manager:
         out = manager.dict()
-        ctx_ = mp.get_context("spawn")
         port = _free_port()
         procs = [ctx_.Process(target=_exchange_rank, args=(r, world, port, out)) for r in range(world)]
         for p in procs:
