@@ -71,7 +71,8 @@ TRAFFIC = {
     "prefill_batch": (301807360.0 + 525824.0, "rows_tc_kernel, one call of 32 sequences x 4 rows "
                                               "(its splits merged in-kernel)"),
 }
-E2E_GROUP = 4            # prefill chunks per host copy in the end-to-end leg
+E2E_FIRST = 2            # prefill chunks of the end-to-end leg's first host copy
+E2E_GROUP = 4            # prefill chunks per host copy after it
 METRIC = "prefill q-rows/s & decode tok/s at 16K ctx (1 B200); % of TC/HBM roofline"
 
 
@@ -716,7 +717,20 @@ def run_cuda(args, rank, world, local_rank):
     return res
 
 
-def run_e2e(w, args, stream):
+def e2e_groups(chunks, first=None, size=None):
+    """The end-to-end leg's copy groups: the first `first` chunks, then
+    groups of `size`.  The outputs (f32, 1.6x the inputs' bytes) decide the
+    time on the link, and the device-to-host copies start only when the
+    first group has crossed and computed, so the first group is kept small."""
+    first = E2E_FIRST if first is None else first
+    size = E2E_GROUP if size is None else size
+    groups = [list(chunks[:first])] if first > 0 else []
+    rest = list(chunks[first:])
+    groups += [rest[i:i + size] for i in range(0, len(rest), size)]
+    return [g for g in groups if g]
+
+
+def run_e2e(w, args, stream, groups=None):
     """Same metric through the public API with host buffers: each step copies
     its inputs (Q rows and the new K/V rows of every chunk, the decode query
     and its appended K/V row) from pinned host memory, runs the calls, and
@@ -752,16 +766,18 @@ def run_e2e(w, args, stream):
         h2d += hstage[t].numel()
         d2h += hdout[t].numel() * 4
 
-    # Prefill streams its chunks in groups of E2E_GROUP: the inputs of group
-    # g+1 cross PCIe (copy stream) while group g computes, and each group's
-    # outputs go back (a second copy stream) as soon as its chunks are done.
-    # Copies of a few chunks at once keep both directions near the link rate
-    # (one copy per chunk and direction ran ~25 % slower on B200: 3.7 against
-    # 3.2 ms per prompt).  The timed region spans the first copy to the last
-    # one on the compute stream.
+    # Prefill streams its chunks in copy groups (e2e_groups: E2E_FIRST chunks,
+    # then E2E_GROUP at a time): the inputs of group g+1 cross PCIe (copy
+    # stream) while group g computes, and each group's outputs go back (a
+    # second copy stream) as soon as its chunks are done.  Copies of a few
+    # chunks at once keep both directions near the link rate: on one B200,
+    # ms per prompt for (first, size) = (2, 4) 3.02, (1, 4) 3.06, (4, 4) 3.08,
+    # (1, 3) 3.09, (1, 6) 3.09, and one copy per chunk and direction 3.70.
+    # The timed region spans the first copy to the last one on the compute
+    # stream.
     h2d_s = torch.cuda.Stream()
     d2h_s = torch.cuda.Stream()
-    groups = [w.chunks[i:i + E2E_GROUP] for i in range(0, len(w.chunks), E2E_GROUP)]
+    groups = e2e_groups(w.chunks) if groups is None else groups
 
     def step(timed):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
