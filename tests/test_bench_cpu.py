@@ -34,3 +34,18 @@ def test_reference_arm_prints_one_json_line():
 
 def test_reference_arm_is_silent_on_other_ranks():
     assert _run({"WORLD_SIZE": "2", "RANK": "1"}) == []
+
+
+def test_e2e_copy_groups_cover_the_prompt_in_order():
+    """The end-to-end leg's copy groups: E2E_FIRST chunks, then E2E_GROUP at
+    a time, every chunk exactly once and in prompt order."""
+    sys.path.insert(0, ROOT)
+    import bench
+    chunks = [(768 * i, 768) for i in range(21)] + [(16128, 256)]
+    groups = bench.e2e_groups(chunks)
+    assert [c for g in groups for c in g] == chunks
+    assert len(groups[0]) == bench.E2E_FIRST
+    assert all(len(g) == bench.E2E_GROUP for g in groups[1:-1]) and 0 < len(groups[-1]) <= bench.E2E_GROUP
+    for first, size in ((0, 4), (1, 1), (4, 4), (30, 4), (2, 50)):
+        got = bench.e2e_groups(chunks, first, size)
+        assert [c for g in got for c in g] == chunks and all(got)
