@@ -452,7 +452,8 @@ int32_t multirow_unit_rows(int32_t rows) {
 }
 size_t multirow_route_ws_bytes(int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window, int sms) {
   const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, multirow_unit_rows(rows));
-  return multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms, kca::kMultiRowMinSplit));
+  return multirow_ws_bytes(batch, rows,
+                           kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms, kca::kMultiRowMinSplit));
 }
 int launch_multirow_route(const void* q, int32_t q_dtype, const void* k_cache, const void* v_cache, int32_t kv_dtype,
                           int64_t capacity, int32_t batch, int32_t rows, const int64_t* ctx_len, int32_t window,
@@ -653,7 +654,8 @@ size_t attn_prefill_batch_workspace_bytes(int32_t batch, int32_t rows, const int
   if (rows > 1) {   // the multi-row kernels' partials, whichever path and unit size a call takes
     for (const int32_t ur : {kca::kMultiRows, kca::kMultiRowsWide}) {
       const std::vector<int64_t> nku = multirow_unit_keys(batch, rows, ctx_len, window, ur);
-      const size_t mr = multirow_ws_bytes(batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms, kca::kMultiRowMinSplit));
+      const size_t mr = multirow_ws_bytes(
+          batch, rows, kca::make_rows_plan((int32_t)nku.size(), nku.data(), sms, kca::kMultiRowMinSplit));
       if (mr > need) need = mr;
     }
   }

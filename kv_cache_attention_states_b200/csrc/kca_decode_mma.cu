@@ -455,7 +455,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
       // t / 32), then every warp takes its A fragments with ldmatrix.
       const int h = threadIdx.x >> 5, d0 = 8 * (threadIdx.x & 31);
       float x[8];
-      load8<QT>(static_cast<const char*>(a.q) + ((int64_t)unit * kHeads * kDim + h * kDim + d0) * ElemBytes<QT>::value, x);
+      load8<QT>(static_cast<const char*>(a.q) +
+                    ((int64_t)unit * kHeads * kDim + h * kDim + d0) * ElemBytes<QT>::value,
+                x);
       if constexpr (kQ8) {
         // the head's scale amax * f32(1/127) over its 256 dims (warp h holds head h)
         float am = fabsf(x[0]);
@@ -644,8 +646,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
   // CTA rank r owns heads r, r+C, ... (C divides 8) and receives the C
   // partials of each by st.async into its own shared memory; once their
   // bytes have completed on its barrier rx, no CTA touches another's shared
-  // memory again, so no cluster barrier is needed before any CTA leaves.  Thread d owns dim d.  With one cluster per unit the
-  // merge of the C partials is the result.  Otherwise each CTA publishes its
+  // memory again, so no cluster barrier is needed before any CTA leaves.
+  // Thread d owns dim d.  With one cluster per unit the merge of the C
+  // partials is the result.  Otherwise each CTA publishes its
   // heads' cluster partials and takes a ticket of (unit, rank); the CTA that
   // draws the last one merges every cluster's partials of those heads.
   // Nothing waits on another CTA, so the order in which clusters run does not
@@ -917,7 +920,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
           lo[j] = pack16<KT>(x[2 * j] - f.x, x[2 * j + 1] - f.y);
         }
         *reinterpret_cast<uint4*>(qs + r * 16 * kDQRow + h * kDQRow + d0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(qs + r * 16 * kDQRow + (h + 8) * kDQRow + d0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(qs + r * 16 * kDQRow + (h + 8) * kDQRow + d0 * 2) =
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(kDWarps * 32) : "memory");
     }

@@ -660,7 +660,8 @@ cudaError_t launch_t(const CUtensorMap& tmk, const CUtensorMap& tmv, const CUten
   cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<DT>, tmk, tmv, tmq, tmo, tmpart, tmpart_rag, a);
   if (e != cudaSuccess || a.plan.n_slots == 0) return e;
   int ns_max = 0;
-  for (int32_t t = 0; t < a.plan.n_tiles && t < kTcMaxTiles; ++t) ns_max = a.tile_items[t] > ns_max ? a.tile_items[t] : ns_max;
+  for (int32_t t = 0; t < a.plan.n_tiles && t < kTcMaxTiles; ++t)
+    ns_max = a.tile_items[t] > ns_max ? a.tile_items[t] : ns_max;
   const int wpr = ns_max <= 8 ? 1 : ns_max <= 16 ? 2 : ns_max <= 32 ? 4 : 8;
   cfg.gridDim = dim3(a.plan.n_tiles, 16 * wpr);
   cfg.blockDim = dim3(256);

@@ -519,9 +519,10 @@ __global__ void __launch_bounds__(RowsTc<UR>::kThreads, 1)
     // multirow_merge_kernel), so no second kernel and no CTA waits on
     // another.  The host gives tickets only while a unit has few splits;
     // with many, multirow_merge_kernel merges across the whole GPU after
-    // this kernel instead of one CTA reading every partial.  Release: the block's partial stores, ordered by the barrier
-    // above before one thread's acq_rel atomic; acquire: the same atomic in
-    // the last CTA, then the barrier below.
+    // this kernel instead of one CTA reading every partial.  Release: the
+    // block's partial stores, ordered by the barrier above before one
+    // thread's acq_rel atomic; acquire: the same atomic in the last CTA,
+    // then the barrier below.
     if (threadIdx.x == 0) {
       int prev;
       asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(prev) : "l"(a.tickets + unit) : "memory");

@@ -14,9 +14,10 @@
 // address is looked up once per device (cudaGetSymbolAddress) on the first
 // call made with that device current -- and again if the device's context
 // was created anew since (cudaDeviceReset reloads the module, possibly at
-// another address); make that first call before any stream capture.  All calls on a device share the array, so calls whose execution
-// can overlap on the GPU (different streams, or graphs replayed
-// concurrently) race on it and must be serialised by the caller.  The array
+// another address); make that first call before any stream capture.  All
+// calls on a device share the array, so calls whose execution can overlap
+// on the GPU (different streams, or graphs replayed concurrently) race on
+// it and must be serialised by the caller.  The array
 // keeps the last call's contents.  Its first KCA_WORKSPACE_HEADER bytes must
 // be zero when a call starts: the status word, and the counters by which the
 // tensor-core decode kernel elects the CTA that merges a row (a call leaves
