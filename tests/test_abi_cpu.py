@@ -355,9 +355,15 @@ def test_decode_plan_fills_one_wave():
                                             (1000, 17, 0), (7, 16, 5), (100, 200, 64),
                                             (2000, 768, 1)])
 def test_prefill_tc_plan_covers_every_visible_key(cs, rows, window):
-    path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, rows, window, num_sms=148)
+    _check_tc_plan(cs, rows, window, 148)
+
+
+def _check_tc_plan(cs, rows, window, sms):
+    path, items = kca.attn_prefill_plan(kca.BF16, kca.BF16, cs, rows, window, num_sms=sms)
     assert path == 1
-    assert len(items) <= 148
+    assert len(items) <= 2 * 80                  # the launch's item table: 80 CTA pairs
+    if (rows + 31) // 32 <= sms // 2:
+        assert len(items) <= 2 * (sms // 2)      # one wave of CTA pairs whenever the row tiles fit one
     kv_lo = oracle.visible_range(cs, window)[0]
     ctx = cs + rows
     n_tiles = (rows + 15) // 16
@@ -430,3 +436,34 @@ def test_multi_row_plan_tiles_each_units_key_union(chunk_start, rows, window):
         assert it[0, 1] == lo and it[-1, 2] == last + 1
         assert (it[1:, 1] == it[:-1, 2]).all() and (it[:, 2] > it[:, 1]).all()
         assert it[:, 3].tolist() == (list(range(len(it))) if len(it) > 1 else [-1])
+
+
+# Randomised checks of the same integer bookkeeping: any chunk, window and SM
+# count gives plans that cover exactly what the definition J(pos) says.
+from hypothesis import HealthCheck, given, settings, strategies as st
+
+
+@settings(max_examples=400, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(rows=st.integers(16, 768), data=st.data(),
+       window=st.one_of(st.just(0), st.integers(1, 40000)), sms=st.sampled_from([148, 132, 96, 20]))
+def test_random_tensor_core_plans_cover_every_visible_key(rows, data, window, sms):
+    cs = data.draw(st.integers(0, 131072 - rows))
+    _check_tc_plan(cs, rows, window, sms)
+
+
+@settings(max_examples=400, deadline=None)
+@given(rows=st.integers(1, 15), data=st.data(), window=st.one_of(st.just(0), st.integers(1, 40000)),
+       sms=st.integers(1, 148))
+def test_random_rows_plans_cover_every_visible_key(rows, data, window, sms):
+    cs = data.draw(st.integers(0, 131072 - rows))
+    path, items = kca.attn_prefill_plan(kca.F32, kca.F32, cs, rows, window, num_sms=sms)
+    assert path == 0
+    _check_rows_plan(items, rows, lambda u: cs + u, window)
+
+
+@settings(max_examples=400, deadline=None)
+@given(ctx=st.lists(st.integers(0, 131072), min_size=1, max_size=16),
+       window=st.one_of(st.just(0), st.integers(1, 40000)), sms=st.integers(1, 148))
+def test_random_decode_plans_cover_every_visible_key(ctx, window, sms):
+    items = kca.attn_decode_plan(ctx, window, num_sms=sms)
+    _check_rows_plan(items, len(ctx), lambda u: ctx[u] - 1, window)
