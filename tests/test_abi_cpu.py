@@ -467,3 +467,22 @@ def test_random_rows_plans_cover_every_visible_key(rows, data, window, sms):
 def test_random_decode_plans_cover_every_visible_key(ctx, window, sms):
     items = kca.attn_decode_plan(ctx, window, num_sms=sms)
     _check_rows_plan(items, len(ctx), lambda u: ctx[u] - 1, window)
+
+
+@settings(max_examples=300, deadline=None)
+@given(rows=st.integers(2, 15), data=st.data(), window=st.one_of(st.just(0), st.integers(12288, 40000)),
+       sms=st.sampled_from([148, 132, 64]))
+def test_random_multi_row_plans_tile_each_units_key_union(rows, data, window, sms):
+    chunk_start = data.draw(st.integers(12288, 131072 - rows))
+    path, items = kca.attn_prefill_plan(kca.F32, kca.BF16, chunk_start, rows, window, num_sms=sms)
+    assert path == 2
+    ur = 8 if rows > 4 else 4
+    units = (rows + ur - 1) // ur
+    assert sorted(set(items[:, 0].tolist())) == list(range(units))
+    for u in range(units):
+        it = items[items[:, 0] == u]
+        first, last = chunk_start + u * ur, min(chunk_start + rows, chunk_start + (u + 1) * ur) - 1
+        lo = oracle.visible_range(first, window)[0]
+        assert it[0, 1] == lo and it[-1, 2] == last + 1
+        assert (it[1:, 1] == it[:-1, 2]).all() and (it[:, 2] > it[:, 1]).all()
+        assert it[:, 3].tolist() == (list(range(len(it))) if len(it) > 1 else [-1])
