@@ -124,3 +124,23 @@ def test_planner_without_larger_clusters_and_negative_capacity():
     assert cluster == 2
     with pytest.raises(kca.KcaError):
         kca.attn_decode_plan([100], 0, num_sms=SMS, kv_dtype=kca.F16, cluster_capacity=(74, -1, 15))
+
+
+# The same comparison on random batches, windows, SM counts and capacities.
+from hypothesis import given, settings, strategies as st
+
+
+@settings(max_examples=300, deadline=None)
+@given(ctx=st.lists(st.integers(0, 131072), min_size=1, max_size=12),
+       window=st.one_of(st.just(0), st.integers(1, 40000)),
+       sms=st.sampled_from([148, 132, 120, 64]),
+       cap=st.tuples(st.integers(1, 74), st.integers(1, 37), st.integers(1, 18)))
+def test_random_planner_choices_match_the_documented_cost_model(ctx, window, sms, cap):
+    nks = [max(0, oracle.visible_range(c - 1, window)[1] - oracle.visible_range(c - 1, window)[0] + 1)
+           for c in ctx]
+    c, length, mc = _choose(nks, sms, {2: cap[0], 4: cap[1], 8: cap[2]})
+    items, cluster = kca.attn_decode_plan(ctx, window, num_sms=sms, kv_dtype=kca.F16, cluster_capacity=cap,
+                                          with_cluster=True)
+    assert cluster == c
+    want = _items([x - 1 for x in ctx], window, c, length, mc)
+    assert items.shape == want.shape and np.array_equal(items, want)
