@@ -268,3 +268,21 @@ def test_visible_range_definition():
     assert oracle.visible_range(10, 4) == (7, 10)
     assert oracle.visible_range(2, 512) == (0, 2)
     assert oracle.visible_range(4159, 512) == (3648, 4159)
+
+
+# Random tiny problems against the decimal brute force: shapes, head groups,
+# positions, windows and scales drawn at random.
+from hypothesis import given, settings, strategies as st
+
+
+@settings(max_examples=60, deadline=None)
+@given(d=st.integers(1, 12), heads=st.sampled_from([(1, 1), (2, 1), (8, 1), (4, 2), (8, 4)]),
+       n_keys=st.integers(1, 7), data=st.data(), window=st.integers(0, 9),
+       scale=st.floats(0.01, 2.0), seed=st.integers(0, 2**31 - 1))
+def test_random_tiny_problems_match_decimal_brute_force(d, heads, n_keys, data, window, scale, seed):
+    hq, hkv = heads
+    pos = np.array(data.draw(st.lists(st.integers(0, n_keys - 1), min_size=1, max_size=4)), dtype=np.int64)
+    q, k, v = _tiny_case(seed, n_keys, d, hq, hkv, n_query=len(pos), std=1.5)
+    got = oracle.attention(q, k, v, pos, window=window, scale=scale, n_kv_heads=hkv)
+    ref = brute.to_float64(brute.attention(q, k, v, pos, window=window, scale=scale, n_kv_heads=hkv))
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
