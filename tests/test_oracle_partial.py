@@ -126,3 +126,23 @@ def test_nan_score_poisons_its_row():
     m, l, acc = _shards(q, k, v, [20], [0, 10, 20], 0, qd, kd)
     out = partial.merge_partials(m, l, acc)
     assert np.all(np.isnan(out))
+
+
+# Random cuts, contexts and windows: the merge of the shards' states is the
+# whole-context attention.
+from hypothesis import given, settings, strategies as st
+
+
+@settings(max_examples=40, deadline=None)
+@given(data=st.data(), dtype=st.sampled_from(["f32", "f16", "bf16"]),
+       window=st.one_of(st.just(0), st.integers(1, 120)), seed=st.integers(0, 10**6))
+def test_random_shard_cuts_merge_to_the_whole_context(data, dtype, window, seed):
+    rows = 96
+    q, k, v, qd, kd = _case(seed, 2, rows, dtype)
+    ctx = data.draw(st.lists(st.integers(0, rows), min_size=2, max_size=2))
+    inner = data.draw(st.lists(st.integers(1, rows - 1), max_size=5, unique=True))
+    cuts = [0] + sorted(inner) + [rows]
+    want = _full(q, k, v, ctx, window, qd, kd)
+    m, l, acc = _shards(q, k, v, ctx, cuts, window, qd, kd)
+    got = partial.merge_partials(m, l, acc)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
