@@ -138,3 +138,22 @@ def test_attention_nan_rows_and_empty_rows():
     assert np.isnan(out[2, 4]).all() and np.isfinite(np.delete(out[2], 4, axis=0)).all()
     out = quant.attention_q8(q[:1], "f32", kc, ks, v, "f32", [-1], scale=synth.SCALE)
     assert (out == 0).all()
+
+
+# Random rows of random magnitude (subnormal to large) against the same
+# brute force, with a few values planted at the row's extremes.
+from hypothesis import given, settings, strategies as st
+
+
+@settings(max_examples=25, deadline=None)
+@given(seed=st.integers(0, 10**6), log_std=st.floats(-40.0, 30.0), n_equal=st.integers(0, 4))
+def test_random_rows_quantise_as_the_decimal_brute_force(seed, log_std, n_equal):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((1, 256)) * (10.0 ** log_std)).astype(np.float32)
+    top = np.abs(x).max()
+    for i in range(n_equal):                         # ties at +-amax
+        x[0, 7 * i] = top if i % 2 == 0 else -top
+    codes, scales = quant.quantize_rows(x)
+    want_codes, want_scale = _brute_row(x[0])
+    assert scales[0] == want_scale or (np.isnan(scales[0]) and np.isnan(want_scale))
+    assert np.array_equal(codes[0].astype(np.int64), want_codes)
