@@ -80,3 +80,31 @@ def test_workspace_queries_return_a_size_or_zero_for_any_arguments(ctx, batch, r
         assert got == 0 or got >= kca.WORKSPACE_HEADER
     got = lib.attn_prefill_workspace_bytes(qd, kd, cs, rows, window)
     assert got == 0 or got >= kca.WORKSPACE_HEADER
+
+
+@settings(max_examples=300, deadline=None)
+@given(q=PTR, qd=DT, k=PTR, v=PTR, kd=DT, hq=I32, hkv=I32, d=I32, cap=I64, ctx=CTX, batch=I32, window=I32,
+       scale=SCALE, out=PTR, ws=PTR, wsb=WSB, bound=I64, key_begin=I64, ctx_dev=PTR)
+def test_device_context_static_and_partial_decode_return_a_status(q, qd, k, v, kd, hq, hkv, d, cap, ctx, batch,
+                                                                   window, scale, out, ws, wsb, bound, key_begin,
+                                                                   ctx_dev):
+    arr, ptr = _arr(ctx)
+    n = min(batch, len(arr)) if batch > 0 else batch
+    lib = kca.lib()
+    assert lib.attn_decode_dev(vp(q), qd, vp(k), vp(v), kd, hq, hkv, d, cap, batch, vp(ctx_dev), bound, window,
+                               scale, vp(out), vp(ws), wsb, None) in CODES
+    assert lib.attn_decode_static(vp(q), qd, vp(k), vp(v), kd, hq, hkv, d, cap, n, ptr, window, scale, vp(out),
+                                  None) in CODES
+    assert lib.attn_decode_partial(vp(q), qd, vp(k), vp(v), kd, hq, hkv, d, cap, n, ptr, key_begin, window, scale,
+                                   vp(out), vp(ws), wsb, None) in CODES
+
+
+@settings(max_examples=300, deadline=None)
+@given(kn=PTR, vn=PTR, ind=DT, n_rows=I32, cos=PTR, sin=PTR, kc=PTR, vc=PTR, kd=DT, cache_rows=I64, dst=PTR,
+       dst0=I64, ws=PTR, n_parts=I32, batch=I32, parts=PTR, stride=I64, out=PTR)
+def test_append_and_merge_return_a_status(kn, vn, ind, n_rows, cos, sin, kc, vc, kd, cache_rows, dst, dst0, ws,
+                                          n_parts, batch, parts, stride, out):
+    lib = kca.lib()
+    assert lib.attn_append_kv(vp(kn), vp(vn), ind, n_rows, vp(cos), vp(sin), vp(kc), vp(vc), kd, cache_rows,
+                              vp(dst), dst0, vp(ws), None) in CODES
+    assert lib.attn_merge_partials(n_parts, batch, vp(parts), stride, vp(out), None) in CODES
