@@ -102,3 +102,39 @@ def test_append_writes_only_the_destination_rows(in_dtype, kv_dtype):
     z = (src[:, :128] + 1j * src[:, 128:]) * np.exp(1j * ang)
     want_k = np.concatenate([z.real, z.imag], 1)
     assert np.max(np.abs(k32 - want_k)) <= rel * (1 + np.max(np.abs(want_k)))
+
+
+# Random rows and angles: the rotation equals the complex product of each
+# (i, i + 128) pair with e^(j theta), and dot products of rotated rows depend
+# only on the difference of their positions.
+from hypothesis import given, settings, strategies as st
+
+
+@settings(max_examples=60, deadline=None)
+@given(seed=st.integers(0, 10**6), scale=st.floats(1e-3, 1e3), lim=st.floats(0.0, 50.0))
+def test_random_rotations_are_complex_products(seed, scale, lim):
+    x = _rand(seed, (2, 256), scale)
+    ang = np.random.default_rng(seed + 1).uniform(-lim, lim, (2, 128))
+    cos = np.concatenate([np.cos(ang)] * 2, 1).astype(np.float32)
+    sin = np.concatenate([np.sin(ang)] * 2, 1).astype(np.float32)
+    got = rope.rope_rotate(x, cos, sin).astype(np.float64)
+    z = (x[:, :128].astype(np.float64) + 1j * x[:, 128:].astype(np.float64)) * \
+        (cos[:, :128].astype(np.float64) + 1j * sin[:, :128].astype(np.float64))
+    bound = 4e-7 * (np.abs(x[:, :128]).astype(np.float64) + np.abs(x[:, 128:]).astype(np.float64))
+    assert np.all(np.abs(got[:, :128] - z.real) <= bound + 1e-30)
+    assert np.all(np.abs(got[:, 128:] - z.imag) <= bound + 1e-30)
+
+
+@settings(max_examples=40, deadline=None)
+@given(seed=st.integers(0, 10**6), p=st.integers(0, 60000), q=st.integers(0, 60000), shift=st.integers(0, 60000))
+def test_random_dot_products_depend_on_relative_position(seed, p, q, shift):
+    a = _rand(seed, (1, 256)).astype(np.float64)
+    b = _rand(seed + 7, (1, 256)).astype(np.float64)
+    c1, s1 = rope.rope_tables([p, q])
+    c2, s2 = rope.rope_tables([p + shift, q + shift])
+    ra = rope.rope_rotate(np.concatenate([a, b]), c1, s1).astype(np.float64)
+    rb = rope.rope_rotate(np.concatenate([a, b]), c2, s2).astype(np.float64)
+    d1, d2 = float(ra[0] @ ra[1]), float(rb[0] @ rb[1])
+    # the tables' cos / sin are float64 values rounded once to float32, and
+    # the rotation rounds each product: a few float32 ulps of |a| |b|
+    assert abs(d1 - d2) <= 1e-5 * (np.linalg.norm(a) * np.linalg.norm(b))
