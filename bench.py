@@ -1052,7 +1052,8 @@ def main():
         return
     cpu = parts_cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows_s, tok_s, cores, desc = oracle_sample(768, 4)
+        # about 10 s of the oracle on a 16-core host: 2304 prefill rows, 12 decode steps
+        rows_s, tok_s, cores, desc = oracle_sample(2304, 12)
         cpu = {"value": rows_s, "unit": "q-rows/s", "cores": cores, "kind": "oracle", "sample": desc,
                "decode_tok_s": tok_s}
         samples, cores = oracle_part_samples()
