@@ -40,7 +40,7 @@ def _arr(ctx):
 vp = ctypes.c_void_p
 
 
-@settings(max_examples=400, deadline=None)
+@settings(max_examples=400, deadline=None, derandomize=True)
 @given(q=PTR, qd=DT, k=PTR, v=PTR, kd=DT, hq=I32, hkv=I32, d=I32, cap=I64, cs=I64, rows=I32, ctx=I64,
        window=I32, scale=SCALE, out=PTR, ws=PTR, wsb=WSB)
 def test_prefill_returns_a_status_for_any_arguments(q, qd, k, v, kd, hq, hkv, d, cap, cs, rows, ctx, window, scale,
@@ -50,7 +50,7 @@ def test_prefill_returns_a_status_for_any_arguments(q, qd, k, v, kd, hq, hkv, d,
     assert st_ in CODES
 
 
-@settings(max_examples=400, deadline=None)
+@settings(max_examples=400, deadline=None, derandomize=True)
 @given(q=PTR, qd=DT, k=PTR, v=PTR, kd=DT, hq=I32, hkv=I32, d=I32, cap=I64, ctx=CTX, batch=I32, window=I32,
        scale=SCALE, out=PTR, ws=PTR, wsb=WSB, rows=I32)
 def test_decode_and_batch_return_a_status_for_any_arguments(q, qd, k, v, kd, hq, hkv, d, cap, ctx, batch, window,
@@ -66,7 +66,7 @@ def test_decode_and_batch_return_a_status_for_any_arguments(q, qd, k, v, kd, hq,
                               wsb, None) in CODES
 
 
-@settings(max_examples=400, deadline=None)
+@settings(max_examples=400, deadline=None, derandomize=True)
 @given(ctx=CTX, batch=I32, rows=I32, window=I32, qd=DT, kd=DT, cs=I64, key_begin=I64, cap=I64)
 def test_workspace_queries_return_a_size_or_zero_for_any_arguments(ctx, batch, rows, window, qd, kd, cs, key_begin,
                                                                    cap):
@@ -82,7 +82,7 @@ def test_workspace_queries_return_a_size_or_zero_for_any_arguments(ctx, batch, r
     assert got == 0 or got >= kca.WORKSPACE_HEADER
 
 
-@settings(max_examples=300, deadline=None)
+@settings(max_examples=300, deadline=None, derandomize=True)
 @given(q=PTR, qd=DT, k=PTR, v=PTR, kd=DT, hq=I32, hkv=I32, d=I32, cap=I64, ctx=CTX, batch=I32, window=I32,
        scale=SCALE, out=PTR, ws=PTR, wsb=WSB, bound=I64, key_begin=I64, ctx_dev=PTR)
 def test_device_context_static_and_partial_decode_return_a_status(q, qd, k, v, kd, hq, hkv, d, cap, ctx, batch,
@@ -99,7 +99,7 @@ def test_device_context_static_and_partial_decode_return_a_status(q, qd, k, v, k
                                    vp(out), vp(ws), wsb, None) in CODES
 
 
-@settings(max_examples=300, deadline=None)
+@settings(max_examples=300, deadline=None, derandomize=True)
 @given(kn=PTR, vn=PTR, ind=DT, n_rows=I32, cos=PTR, sin=PTR, kc=PTR, vc=PTR, kd=DT, cache_rows=I64, dst=PTR,
        dst0=I64, ws=PTR, n_parts=I32, batch=I32, parts=PTR, stride=I64, out=PTR)
 def test_append_and_merge_return_a_status(kn, vn, ind, n_rows, cos, sin, kc, vc, kd, cache_rows, dst, dst0, ws,

@@ -275,7 +275,7 @@ def test_visible_range_definition():
 from hypothesis import given, settings, strategies as st
 
 
-@settings(max_examples=60, deadline=None)
+@settings(max_examples=60, deadline=None, derandomize=True)
 @given(d=st.integers(1, 12), heads=st.sampled_from([(1, 1), (2, 1), (8, 1), (4, 2), (8, 4)]),
        n_keys=st.integers(1, 7), data=st.data(), window=st.integers(0, 9),
        scale=st.floats(0.01, 2.0), seed=st.integers(0, 2**31 - 1))

@@ -145,7 +145,7 @@ def test_attention_nan_rows_and_empty_rows():
 from hypothesis import given, settings, strategies as st
 
 
-@settings(max_examples=25, deadline=None)
+@settings(max_examples=25, deadline=None, derandomize=True)
 @given(seed=st.integers(0, 10**6), log_std=st.floats(-40.0, 30.0), n_equal=st.integers(0, 4))
 def test_random_rows_quantise_as_the_decimal_brute_force(seed, log_std, n_equal):
     rng = np.random.default_rng(seed)

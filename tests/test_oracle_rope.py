@@ -110,7 +110,7 @@ def test_append_writes_only_the_destination_rows(in_dtype, kv_dtype):
 from hypothesis import given, settings, strategies as st
 
 
-@settings(max_examples=60, deadline=None)
+@settings(max_examples=60, deadline=None, derandomize=True)
 @given(seed=st.integers(0, 10**6), scale=st.floats(1e-3, 1e3), lim=st.floats(0.0, 50.0))
 def test_random_rotations_are_complex_products(seed, scale, lim):
     x = _rand(seed, (2, 256), scale)
@@ -125,7 +125,7 @@ def test_random_rotations_are_complex_products(seed, scale, lim):
     assert np.all(np.abs(got[:, 128:] - z.imag) <= bound + 1e-30)
 
 
-@settings(max_examples=40, deadline=None)
+@settings(max_examples=40, deadline=None, derandomize=True)
 @given(seed=st.integers(0, 10**6), p=st.integers(0, 60000), q=st.integers(0, 60000), shift=st.integers(0, 60000))
 def test_random_dot_products_depend_on_relative_position(seed, p, q, shift):
     a = _rand(seed, (1, 256)).astype(np.float64)

@@ -130,7 +130,7 @@ def test_planner_without_larger_clusters_and_negative_capacity():
 from hypothesis import given, settings, strategies as st
 
 
-@settings(max_examples=300, deadline=None)
+@settings(max_examples=300, deadline=None, derandomize=True)
 @given(ctx=st.lists(st.integers(0, 131072), min_size=1, max_size=12),
        window=st.one_of(st.just(0), st.integers(1, 40000)),
        sms=st.sampled_from([148, 132, 120, 64]),
